@@ -1,0 +1,63 @@
+"""Paged decode attention, the plain definition, in float64 (oracle only).
+
+For sequence b and query head h (kv-head g = h // (Hq // Hkv)), with
+n = context_lens[b] tokens:
+
+  K_j = k_cache[block_tables[b][j // bs], g, j % bs, :]     (V_j likewise)
+  s_j = scale * sum_d q[b,h,d] * K_j[d]
+  out[b,h,:] = sum_j softmax(s)_j * V_j
+
+"PagedAttention 与 vLLM 推理加速" §2.3: the block table maps each logical
+page to a physical block, the kernel reads every K of the sequence's blocks
+through it and Q x K gives the attention scores; §1: decode step t attends
+over the K/V of every token so far, itself included.  The softmax is the
+standard one, computed max-subtracted so exp never overflows.  A sequence
+with no tokens yields zeros.  Block-table entries past the sequence's last
+page, and the unused slots of its last block, are never read.
+"""
+import numpy as np
+
+from .storage import widen
+
+
+def _gather(cache: np.ndarray, pages: np.ndarray, g: int, n: int, bs: int) -> np.ndarray:
+    """Rows 0..n-1 of kv-head g in logical order: page j//bs, offset j%bs."""
+    tiles = cache[pages, g]  # [n_pages, bs, D]
+    return tiles.reshape(-1, tiles.shape[-1])[:n]
+
+
+def decode_head(q_row: np.ndarray, keys: np.ndarray, values: np.ndarray, scale: float) -> np.ndarray:
+    """Single-query softmax attention over float64 rows ``keys``/``values``."""
+    if keys.shape[0] == 0:
+        return np.zeros(values.shape[-1], dtype=np.float64)
+    s = scale * (keys @ q_row)
+    s = s - s.max()
+    p = np.exp(s)
+    p = p / p.sum()
+    return p @ values
+
+
+def paged_decode(q, k_cache, v_cache, block_tables, context_lens, scale, dtype,
+                 block_size=16, seqs=None):
+    """float64 output [B, Hq, D] (rows not in ``seqs`` are left NaN).
+
+    q: [B,Hq,D]; k_cache/v_cache: [num_blocks,Hkv,block_size,D] in the
+    storage format ``dtype`` ('f32', 'f16', or 'bf16' as uint16 bits);
+    block_tables: int [B, max_blocks]; context_lens: int [B].
+    ``seqs`` restricts the work to those sequence indices (sampled checks).
+    """
+    B, Hq, D = q.shape
+    Hkv = k_cache.shape[1]
+    G = Hq // Hkv
+    out = np.full((B, Hq, D), np.nan, dtype=np.float64)
+    for b in (range(B) if seqs is None else seqs):
+        n = int(context_lens[b])
+        n_pages = -(-n // block_size)
+        pages = np.asarray(block_tables[b][:n_pages], dtype=np.int64)
+        qb = widen(q[b], dtype)
+        for g in range(Hkv):
+            keys = widen(_gather(k_cache, pages, g, n, block_size), dtype)
+            values = widen(_gather(v_cache, pages, g, n, block_size), dtype)
+            for h in range(g * G, (g + 1) * G):
+                out[b, h] = decode_head(qb[h], keys, values, scale)
+    return out

@@ -1,0 +1,83 @@
+"""Test-side helpers shared by the oracle pins and the GPU parity tests."""
+import numpy as np
+
+
+def logical_token_ids(wl):
+    """For each step sequence, the ids of its tokens in logical order.
+
+    An id is an index into the prefill arrays (k_tokens/v_tokens) or
+    ('new', b) for the step's token of batch entry b.  Worked out from the
+    op log alone -- no allocator, slot or block table is involved.
+    """
+    seqs = {}
+    cursor = 0
+    for op in wl.ops:
+        if op[0] == "add":
+            seqs[op[1]] = []
+        elif op[0] == "append":
+            seqs[op[1]] = seqs[op[1]] + list(range(cursor, cursor + op[2]))
+            cursor += op[2]
+        elif op[0] == "fork":
+            seqs[op[2]] = list(seqs[op[1]])
+        elif op[0] == "free":
+            del seqs[op[1]]
+    out = []
+    for b, sid in enumerate(wl.step_seqs):
+        ids = list(seqs[int(sid)])
+        if wl.step_append_mask[b]:
+            ids.append(("new", b))
+        out.append(ids)
+    return out
+
+
+def logical_rows(wl, values, b, kv_head, widen):
+    """(keys, values) float64 rows of step sequence b, kv-head ``kv_head``."""
+    ids = logical_token_ids(wl)[b]
+    ks, vs = [], []
+    for t in ids:
+        if isinstance(t, tuple):
+            ks.append(values["k_new"][t[1], kv_head])
+            vs.append(values["v_new"][t[1], kv_head])
+        else:
+            ks.append(values["k_tokens"][t, kv_head])
+            vs.append(values["v_tokens"][t, kv_head])
+    if not ks:
+        return np.zeros((0, wl.D)), np.zeros((0, wl.D))
+    return widen(np.stack(ks), wl.dtype), widen(np.stack(vs), wl.dtype)
+
+
+def relabel_blocks(cache_k, cache_v, tables, context_lens, perm, block_size=16):
+    """Move every physical block i to perm[i]; rewrite the tables to match."""
+    k2 = np.empty_like(cache_k)
+    v2 = np.empty_like(cache_v)
+    k2[perm] = cache_k
+    v2[perm] = cache_v
+    t2 = tables.copy()
+    for b, n in enumerate(context_lens):
+        pages = -(-int(n) // block_size)
+        t2[b, :pages] = perm[tables[b, :pages]]
+    return k2, v2, t2
+
+
+def privatise(cache_k, cache_v, tables, context_lens, block_size=16):
+    """Give every sequence its own copy of every block its table names.
+
+    Returns a larger pool where no block is shared, and the new tables.
+    """
+    pages = [-(-int(n) // block_size) for n in context_lens]
+    nb0 = cache_k.shape[0]
+    total = nb0 + sum(pages)
+    k2 = np.empty((total,) + cache_k.shape[1:], dtype=cache_k.dtype)
+    v2 = np.empty_like(k2)
+    k2[:nb0] = cache_k
+    v2[:nb0] = cache_v
+    t2 = tables.copy()
+    nxt = nb0
+    for b, p in enumerate(pages):
+        for j in range(p):
+            src = tables[b, j]
+            k2[nxt] = cache_k[src]
+            v2[nxt] = cache_v[src]
+            t2[b, j] = nxt
+            nxt += 1
+    return k2, v2, t2
