@@ -1,0 +1,489 @@
+"""Benchmark of the paged decode step: KV-cache GB/s (% of HBM peak),
+sequence-steps/s and us per step.
+
+One step = the whole device path for one batch: the copy-on-write block
+copies (when the step has any), the slot-mapped append of the new tokens'
+K/V, and paged decode attention (partition kernel, plus the merge kernel
+when a sequence spans several partitions).  The host allocator's step is
+planned before the timed region (host microseconds, not device work); the
+same planned step is replayed every iteration (its copies and appends are
+idempotent).
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+  python bench.py --impl reference ...   (the fp64 CPU oracle, bounded sample)
+
+N > 1: one process per GPU (torchrun), each rank decoding its own replica
+batch (different seed), no collective on the data path; value = all ranks'
+KV bytes / the slowest rank's time.  Prints one JSON line on rank 0.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import re
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import workloads  # noqa: E402
+
+METRIC = "paged decode attention: KV-cache HBM GB/s (% of peak), seq-steps/s"
+UNIT = "GB/s"
+FALLBACK_HBM_GBS = 6650.0
+STORAGE = {"f32": 4, "f16": 2, "bf16": 2}
+DTYPE_NAME = {"f32": "fp32", "f16": "fp16", "bf16": "bf16"}
+DECODE_SOURCES = ["paged_kv_cache_365_b200/csrc/decode.cuh", "paged_kv_cache_365_b200/csrc/common.cuh",
+                  "paged_kv_cache_365_b200/csrc/pkv_api.cu"]
+
+
+# ---------------------------------------------------------------------------
+# workload accounting (algorithmic bytes)
+# ---------------------------------------------------------------------------
+def kv_bytes(wl, unique: bool) -> int:
+    """K+V bytes the decode must read: each token once per kv-head.
+
+    With ``unique`` a block shared by several sequences counts once (the
+    shared prefix of the prefix workload); otherwise per sequence.
+    """
+    per_tok = wl.kv_bytes_per_token
+    logical = int(np.sum(wl.context_lens.astype(np.int64))) * per_tok
+    if not unique or wl.name != "prefix13b":
+        return logical
+    prefix = 1024
+    return logical - (wl.B - 1) * prefix * per_tok
+
+
+def decode_algorithmic_bytes(wl, unique: bool = True) -> int:
+    """Bytes one decode launch must move: K/V + q in + out + tables + lengths."""
+    es = STORAGE[wl.dtype]
+    pages = int(np.sum((wl.context_lens.astype(np.int64) + 15) // 16))
+    return kv_bytes(wl, unique) + 2 * wl.B * wl.Hq * wl.D * es + 4 * pages + 4 * wl.B
+
+
+def source_digest() -> str:
+    h = hashlib.sha256()
+    for f in DECODE_SOURCES:
+        with open(os.path.join(ROOT, f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def measured_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def recorded_traffic(workload: str):
+    """DRAM bytes per decode launch from the committed ncu summary, if it
+    was taken on the current decode source (else None)."""
+    path = os.path.join(ROOT, "profiles", f"paged_decode_{workload}.md")
+    if not os.path.exists(path):
+        return None
+    text = open(path).read()
+    m = re.search(r"traffic_bytes_per_launch:\s*([0-9]+)", text)
+    s = re.search(r"decode_source_digest:\s*([0-9a-f]+)", text)
+    if not m or not s or s.group(1) != source_digest():
+        return None
+    return int(m.group(1))
+
+
+# ---------------------------------------------------------------------------
+# clocks during the timed region (NVML, read-only)
+# ---------------------------------------------------------------------------
+class ClockSampler:
+    REASONS = {
+        0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap", 0x8: "hw_slowdown",
+        0x10: "sync_boost", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
+        0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting",
+    }
+
+    def __init__(self, device_index: int, period_s: float = 0.01):
+        self.samples, self.reasons, self.ok = [], 0, False
+        self.period = period_s
+        self._stop = threading.Event()
+        try:
+            import pynvml
+            import torch
+            pynvml.nvmlInit()
+            uuid = str(torch.cuda.get_device_properties(device_index).uuid)
+            uuid = uuid if uuid.startswith("GPU-") else "GPU-" + uuid
+            self.h = pynvml.nvmlDeviceGetHandleByUUID(uuid.encode())
+            self.nv = pynvml
+            self.max_mhz = int(pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM))
+            self.ok = True
+        except Exception as e:  # pragma: no cover - reported in the JSON
+            self.err = repr(e)
+
+    def _run(self):
+        nv = self.nv
+        while not self._stop.is_set():
+            try:
+                self.samples.append(int(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM)))
+                self.reasons |= int(nv.nvmlDeviceGetCurrentClocksEventReasons(self.h))
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.ok:
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+        return self
+
+    def __exit__(self, *exc):
+        if self.ok:
+            self._stop.set()
+            self.t.join()
+
+    def summary(self):
+        if not self.ok:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "error": getattr(self, "err", "")}
+        names = [n for bit, n in self.REASONS.items() if self.reasons & bit and n != "gpu_idle"]
+        return {"sm_mhz": statistics.median(self.samples) if self.samples else None,
+                "sm_max_mhz": self.max_mhz, "reasons": names, "samples": len(self.samples)}
+
+
+# ---------------------------------------------------------------------------
+# the CUDA path
+# ---------------------------------------------------------------------------
+def device_values(wl, seed, device):
+    """Seeded synthetic N(0,1) values drawn on the device (fast at full size)."""
+    import torch
+    g = torch.Generator(device=device)
+    g.manual_seed(int(seed) * 7919 + 17)
+    dt = {"f32": torch.float32, "f16": torch.float16, "bf16": torch.bfloat16}[wl.dtype]
+    shapes = {"q": (wl.B, wl.Hq, wl.D), "k_new": (wl.B, wl.Hkv, wl.D), "v_new": (wl.B, wl.Hkv, wl.D),
+              "k_tokens": (wl.n_prefill_tokens, wl.Hkv, wl.D), "v_tokens": (wl.n_prefill_tokens, wl.Hkv, wl.D)}
+    out = {}
+    for k, shp in shapes.items():
+        t = torch.empty(shp, dtype=dt, device=device)
+        n = t.numel()
+        flat = t.view(-1)
+        chunk = 1 << 26
+        for s in range(0, n, chunk):
+            e = min(n, s + chunk)
+            flat[s:e] = torch.randn(e - s, generator=g, device=device, dtype=torch.float32).to(dt)
+        out[k] = t
+    return out
+
+
+def run_cuda(args, rank, world, local_rank):
+    import torch
+    from paged_kv_cache_365_b200.replay import build_step
+    import paged_kv_cache_365_b200 as pkv
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    wl = workloads.named(args.workload, args.seed + rank)
+    vals = device_values(wl, args.seed + rank, dev)
+    st = build_step(wl, {}, dev, device_values=vals)
+    del vals
+    cache = st["cache"]
+    stream = torch.cuda.current_stream(dev)
+    B, Hq, D = wl.B, wl.Hq, wl.D
+    max_ctx = st["max_context_len"]
+    n_pairs = int(st["cow_pairs"].shape[0])
+    ws = cache.workspace(pkv.decode_workspace_bytes(B, Hq, D, max_ctx, args.partition))
+    out = torch.empty_like(st["q"])
+    P = max(1, math.ceil(max_ctx / (args.partition or pkv.DEFAULT_PARTITION)))
+    launches_per_step = 1 + 1 + (1 if n_pairs else 0) + (1 if P > 1 else 0)
+    scale = 1.0 / math.sqrt(D)
+
+    def pre_decode():
+        if n_pairs:
+            pkv.copy_blocks(cache.k, cache.v, st["cow_pairs"], stream)
+        pkv.kv_append(st["k_new"], st["v_new"], cache.k, cache.v, st["slot_mapping"], stream)
+
+    def decode():
+        pkv.paged_attention_decode(st["q"], cache.k, cache.v, st["block_tables"], st["context_lens"], max_ctx,
+                                   scale, out=out, workspace=ws, partition=args.partition, stream=stream)
+
+    def barrier():
+        if world > 1:
+            torch.distributed.barrier()
+
+    for _ in range(args.warmup):
+        pre_decode()
+        decode()
+    torch.cuda.synchronize()
+    if pkv.get_error() != 0:
+        raise RuntimeError("device error flags raised during warm-up")
+    barrier()
+    torch.cuda.synchronize()
+
+    K = args.steps
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
+    with ClockSampler(local_rank) as clocks:
+        for i in range(K):
+            ev[i][0].record(stream)
+            pre_decode()
+            ev[i][1].record(stream)
+            decode()
+            ev[i][2].record(stream)
+        torch.cuda.synchronize()
+    barrier()
+    torch.cuda.synchronize()
+    total_ms = ev[0][0].elapsed_time(ev[K - 1][2])
+    dec_ms = [ev[i][1].elapsed_time(ev[i][2]) for i in range(K)]
+    dec_avg_ms = sum(dec_ms) / K
+
+    # e2e: the same step with its inputs in pinned host memory, copied in
+    # every step, and the output read back every step
+    host = {k: st[k].cpu().pin_memory() for k in ("q", "k_new", "v_new", "slot_mapping", "cow_pairs",
+                                                    "block_tables", "context_lens")}
+    out_host = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
+    h2d = sum(t.numel() * t.element_size() for t in host.values())
+    d2h = out_host.numel() * out_host.element_size()
+
+    def e2e_step():
+        cache.run_step(host["slot_mapping"], host["cow_pairs"], host["block_tables"], host["context_lens"],
+                       max_ctx, host["q"], host["k_new"], host["v_new"], out=out_host, scale=scale,
+                       partition=args.partition, stream=stream)
+
+    for _ in range(args.warmup):
+        e2e_step()
+    torch.cuda.synchronize()
+    barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(K):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    e2e_ms = e0.elapsed_time(e1)
+    if pkv.get_error() != 0:
+        raise RuntimeError("device error flags raised during timing")
+
+    times = torch.tensor([total_ms, e2e_ms, dec_avg_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        torch.distributed.all_reduce(times, op=torch.distributed.ReduceOp.MAX)
+    total_ms, e2e_ms, dec_avg_ms = [float(x) for x in times.tolist()]
+
+    res = dict(wl=wl, K=K, total_ms=total_ms, e2e_ms=e2e_ms, dec_avg_ms=dec_avg_ms,
+               launches=launches_per_step * K, h2d=h2d, d2h=d2h, clocks=clocks.summary(), P=P,
+               n_pairs=n_pairs, cache=cache, st=st)
+    return res
+
+
+# ---------------------------------------------------------------------------
+# the oracle on the host cores
+# ---------------------------------------------------------------------------
+def oracle_units_timed(wl, ref, vals, units):
+    """Time the oracle on a list of (sequence, kv-head) units; return
+    (seconds, KV bytes the units read)."""
+    import oracle
+    G = wl.Hq // wl.Hkv
+    t0 = time.perf_counter()
+    nbytes = 0
+    for b, g in units:
+        n = int(ref["context_lens"][b])
+        pages = -(-n // 16)
+        tbl = ref["block_tables"][b, :pages].astype(np.int64)
+        keys = oracle.widen(ref["cache"].k[tbl, g].reshape(-1, wl.D)[:n], wl.dtype)
+        values = oracle.widen(ref["cache"].v[tbl, g].reshape(-1, wl.D)[:n], wl.dtype)
+        qb = oracle.widen(vals["q"][b], wl.dtype)
+        for h in range(g * G, (g + 1) * G):
+            oracle.decode_head(qb[h], keys, values, wl.scale)
+        nbytes += 2 * n * wl.D * STORAGE[wl.dtype]
+    return time.perf_counter() - t0, nbytes
+
+
+def oracle_setup(wl):
+    import oracle
+    vals = workloads.draw_values(wl)
+    ref = oracle.replay(wl, vals)
+    return vals, ref
+
+
+def pick_units(wl, rng, budget_s, per_byte_s):
+    """Random (sequence, kv-head) units whose estimated oracle time fills
+    ``budget_s`` (the whole workload, repeated, when it is smaller)."""
+    units, est = [], 0.0
+    cand = [(b, g) for b in range(wl.B) for g in range(wl.Hkv) if wl.context_lens[b] > 0]
+    while est < budget_s:
+        added = False
+        for i in rng.permutation(len(cand)):
+            b, g = cand[i]
+            cost = 2 * int(wl.context_lens[b]) * wl.D * STORAGE[wl.dtype] * per_byte_s
+            if units and est + cost > budget_s:
+                continue
+            units.append((b, g))
+            est += cost
+            added = True
+            if est >= budget_s:
+                break
+        if not added:
+            break
+    return units
+
+
+def calibrate(wl, ref, vals):
+    b = int(np.argmax(wl.context_lens))
+    s, nb = oracle_units_timed(wl, ref, vals, [(b, 0)])
+    return s / max(nb, 1)
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_limits
+        return threadpool_limits
+    except Exception:  # pragma: no cover
+        return None
+
+
+def cpu_baseline(wl, budget_s=12.0, seed=0):
+    """The oracle as it stands, one host thread, on a bounded sample."""
+    limits = blas_threads()
+    ctx = limits(limits=1) if limits else None
+    if ctx:
+        ctx.__enter__()
+    try:
+        vals, ref = oracle_setup(wl)
+        per_byte = calibrate(wl, ref, vals)
+        units = pick_units(wl, np.random.default_rng(seed), budget_s, per_byte)
+        secs, nbytes = oracle_units_timed(wl, ref, vals, units)
+    finally:
+        if ctx:
+            ctx.__exit__(None, None, None)
+    return {"value": nbytes / secs / 1e9, "unit": UNIT, "cores": 1, "kind": "oracle",
+            "sample": f"{len(units)} (sequence, kv-head) units of workload {wl.name} seed {wl.seed}, "
+                      f"{nbytes / 1e6:.1f} MB of K/V, fp64 numpy, BLAS limited to 1 thread, {secs:.1f} s"}
+
+
+def config_of(wl, args, P):
+    return {"workload": wl.name, "global_batch": wl.B, "num_q_heads": wl.Hq, "num_kv_heads": wl.Hkv,
+            "head_dim": wl.D, "block_size": 16, "num_blocks": wl.num_blocks,
+            "context_lens": {"min": int(wl.context_lens.min()), "max": int(wl.context_lens.max()),
+                             "sum": int(wl.context_lens.astype(np.int64).sum())},
+            "partition_tokens": args.partition or 512, "partitions_max": P, "seed": args.seed,
+            "parallelism": f"replicas{args.gpus}" if args.gpus > 1 else "single-gpu",
+            "l2": "inputs larger than L2 (no flush)" if kv_bytes(wl, True) > 126e6 else "inputs fit in L2"}
+
+
+def run_reference(args, rank, world):
+    """The oracle timed on the host cores, every step a bounded sample."""
+    if rank != 0:
+        return
+    wl = workloads.named(args.workload, args.seed)
+    limits = blas_threads()
+    ctx = limits(limits=1) if limits else None
+    if ctx:
+        ctx.__enter__()
+    try:
+        vals, ref = oracle_setup(wl)
+        per_byte = calibrate(wl, ref, vals)
+        per_step = min(1.0, 150.0 / max(1, args.steps + args.warmup))
+        rng = np.random.default_rng(args.seed)
+        for _ in range(args.warmup):
+            oracle_units_timed(wl, ref, vals, pick_units(wl, rng, per_step, per_byte))
+        tot_s, tot_b, n_units = 0.0, 0, 0
+        for _ in range(args.steps):
+            units = pick_units(wl, rng, per_step, per_byte)
+            s, nb = oracle_units_timed(wl, ref, vals, units)
+            tot_s += s
+            tot_b += nb
+            n_units += len(units)
+    finally:
+        if ctx:
+            ctx.__exit__(None, None, None)
+    value = tot_b / tot_s / 1e9
+    sample = (f"each step: ~{n_units / max(1, args.steps):.1f} random (sequence, kv-head) units of workload "
+              f"{wl.name} ({tot_b / max(1, args.steps) / 1e6:.1f} MB of K/V), fp64 numpy, one thread")
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * tot_s / max(1, args.steps),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": config_of(wl, args, 0),
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="llama7b", choices=sorted(workloads.NAMED))
+    ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--partition", type=int, default=0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+        return 0
+
+    import torch
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local_rank)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=torch.device("cuda", local_rank))
+    try:
+        r = run_cuda(args, rank, world, local_rank)
+    finally:
+        pass
+    if world > 1:
+        torch.distributed.destroy_process_group()
+    if rank != 0:
+        return 0
+
+    wl = r["wl"]
+    peak, peak_kind = measured_peak()
+    K = r["K"]
+    step_s = r["total_ms"] / 1e3 / K
+    kv_unique = kv_bytes(wl, True)
+    kv_logical = kv_bytes(wl, False)
+    value = world * kv_logical / step_s / 1e9
+    dec_bytes = decode_algorithmic_bytes(wl, unique=True)
+    achieved = dec_bytes / (r["dec_avg_ms"] / 1e3) / 1e9
+    e2e_step_s = r["e2e_ms"] / 1e3 / K
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": args.warmup,
+        "ms_per_step": r["total_ms"] / K, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": wl.dtype, "data": "synthetic (seeded N(0,1) q/K/V on the device, seeded lengths and placement)",
+        "config": config_of(wl, args, r["P"]),
+        "us_per_step": 1e3 * r["total_ms"] / K,
+        "seq_steps_per_s": world * wl.B / step_s,
+        "pct_hbm_peak": 100.0 * (world * kv_unique / step_s / 1e9) / (peak * world),
+        "kv_bytes_per_step": {"logical": kv_logical, "unique": kv_unique},
+        "clocks": r["clocks"],
+        "e2e": {"value": world * kv_logical / e2e_step_s / 1e9, "unit": UNIT,
+                "h2d_bytes_per_step": r["h2d"], "d2h_bytes_per_step": r["d2h"],
+                "us_per_step": 1e6 * e2e_step_s},
+        "gpu_launches": r["launches"],
+        "roofline": {"kernel": "paged_decode (partition + merge kernels)", "bound": "hbm",
+                     "achieved": achieved, "peak": peak, "peak_kind": f"{peak_kind} (MEASURED_PEAKS hbm_gbs)"
+                     if peak_kind == "measured" else "fallback", "unit": "GB/s", "frac": achieved / peak,
+                     "traffic": recorded_traffic(wl.name), "algorithmic_bytes_per_launch": dec_bytes,
+                     "avg_launch_us": 1e3 * r["dec_avg_ms"]},
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(wl, seed=args.seed)
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,243 @@
+/*
+ * pkv.h -- C ABI of the paged KV-cache decode library (libpkv.so).
+ *
+ * The KV cache of every sequence is kept in fixed 16-token blocks drawn from
+ * one shared pool and reached through a per-sequence block table (logical
+ * page n -> physical block), so a sequence never needs contiguous memory and
+ * grows one block at a time ("PagedAttention 与 vLLM 推理加速" §2.2-§2.3;
+ * "vLLM + PagedAttention：打造高并发LLM推理引擎", "它是怎么工作的").
+ *
+ * Device entry points take plain device pointers to memory the caller owns
+ * (the library never allocates device memory) and enqueue work on the given
+ * stream (a cudaStream_t passed as void*; NULL = the legacy default stream).
+ * They return after the launch, not after the work.  Every argument the host
+ * can check is checked before anything is launched; a bad one returns
+ * PKV_EINVAL and launches nothing.  Values that live on the device (block
+ * ids in tables, slots, context lengths, copy pairs) are range-checked inside
+ * the kernels: an out-of-range value is never dereferenced, the work that
+ * needed it is skipped, and a bit is set in the device error word that
+ * pkv_get_error() reads back.
+ *
+ * Layouts (all row-major, contiguous):
+ *   q, out            [num_seqs, num_q_heads, head_dim]            dtype
+ *   k_new, v_new      [num_tokens, num_kv_heads, head_dim]         dtype
+ *   k_cache, v_cache  [num_blocks, num_kv_heads, 16, head_dim]     dtype
+ *   block_tables      [num_seqs, max_blocks_per_seq]               int32
+ *   context_lens      [num_seqs]                                   int32
+ *   slot_mapping      [num_tokens]                                 int64
+ *   copy pairs        [num_pairs, 2] = (src, dst)                  int32
+ * A slot names one token position of the pool: slot = block * 16 + offset.
+ * Query head h reads kv-head h / (num_q_heads / num_kv_heads).
+ *
+ * Supported: head_dim 64 or 128; dtype fp32, fp16, bf16 (K, V, q and out
+ * share it); num_q_heads / num_kv_heads in {1, 2, 4, 8}.  Device pointers
+ * must be 16-byte aligned.
+ */
+#ifndef PKV_H
+#define PKV_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define PKV_BLOCK_SIZE 16
+#define PKV_DEFAULT_PARTITION 512
+
+typedef enum { PKV_F32 = 0, PKV_F16 = 1, PKV_BF16 = 2 } pkv_dtype;
+
+typedef enum {
+  PKV_OK = 0,
+  PKV_EINVAL = 1, /* a bad argument; nothing launched, no state changed */
+  PKV_ENOMEM = 2, /* allocator: the pool cannot serve the call; no state changed */
+  PKV_ECUDA = 3   /* a CUDA runtime call or launch failed */
+} pkv_status;
+
+/* Bits of the device error word (pkv_get_error). */
+#define PKV_ERR_BLOCK_RANGE 0x1u   /* a block-table entry inside a sequence's pages is outside [0, num_blocks) */
+#define PKV_ERR_CONTEXT_RANGE 0x2u /* a context length < 0, > max_context_len or > 16 * max_blocks_per_seq (clamped) */
+#define PKV_ERR_SLOT_RANGE 0x4u    /* an append slot names a block outside the pool (the write is skipped) */
+#define PKV_ERR_COPY_RANGE 0x8u    /* a copy pair names a block outside the pool (the copy is skipped) */
+#define PKV_ERR_TIMEOUT 0x10u      /* a staging wait gave up after its time limit */
+
+/* Static description of a status code. */
+const char* pkv_status_string(pkv_status status);
+
+/* ABI version of this header (increases when a signature changes). */
+int pkv_abi_version(void);
+
+/* ------------------------------------------------------------------------
+ * pkv_kv_append -- slot-mapped write of new tokens' K/V into the pool.
+ *
+ * "vLLM + PagedAttention：打造高并发LLM推理引擎", "它是怎么工作的" (items 2
+ * and 3): each request's page table records which block its n-th token is
+ * in; a growing sequence writes its new token into that slot and never
+ * moves old data.
+ *
+ * For every token i with slot_mapping[i] >= 0:
+ *   k_cache[slot / 16, h, slot % 16, :] = k_new[i, h, :]   (all h; V alike)
+ * A negative slot is padding and writes nothing.  Slots must be distinct
+ * within one call (two tokens writing one slot race).  Bit copy: the stored
+ * bytes equal the input bytes.  A slot whose block is >= num_blocks is
+ * skipped and sets PKV_ERR_SLOT_RANGE.
+ * -------------------------------------------------------------------- */
+pkv_status pkv_kv_append(const void* k_new, const void* v_new, void* k_cache, void* v_cache,
+                         const int64_t* slot_mapping, int num_tokens, int num_kv_heads,
+                         int head_dim, int num_blocks, pkv_dtype dtype, void* stream);
+
+/* ------------------------------------------------------------------------
+ * pkv_copy_blocks -- copy-on-write block copy.
+ *
+ * "PagedAttention 与 vLLM 推理加速" §3.2(3) and "LLM Systems 24: Efficient
+ * LLM Inference with PagedAttention and vLLM" §3: a block shared by several
+ * sequences is never copied while it is only read; before a sequence writes
+ * into it, the block is copied to a fresh block that the writer then owns.
+ *
+ * For each pair (src, dst) in pairs[num_pairs][2] (device memory):
+ *   k_cache[dst] = k_cache[src];  v_cache[dst] = v_cache[src]
+ * (all num_kv_heads * 16 * head_dim elements; bit copy).  The dst values must
+ * be distinct and no dst may also be a src of the same call (otherwise the
+ * result depends on the order of the copies); pkv_copy_blocks_check verifies
+ * this on a host copy of the pairs.  A pair naming a block outside
+ * [0, num_blocks) is skipped and sets PKV_ERR_COPY_RANGE.
+ * -------------------------------------------------------------------- */
+pkv_status pkv_copy_blocks(void* k_cache, void* v_cache, const int32_t* pairs, int num_pairs,
+                           int num_kv_heads, int head_dim, int num_blocks, pkv_dtype dtype,
+                           void* stream);
+
+/* Host-side check of copy pairs (host memory): every id in range, dst ids
+ * distinct, no dst equal to any src.  PKV_OK or PKV_EINVAL. */
+pkv_status pkv_copy_blocks_check(const int32_t* pairs_host, int num_pairs, int num_blocks);
+
+/* ------------------------------------------------------------------------
+ * pkv_decode_workspace_bytes -- device workspace pkv_paged_attention_decode
+ * needs for these sizes (0 when no sequence can span two partitions).
+ * partition_tokens: 0 = PKV_DEFAULT_PARTITION, else a multiple of 16 in
+ * [16, 2048].  Returns 0 for arguments pkv_paged_attention_decode rejects.
+ *
+ * Workspace layout (fp32): partial outputs [num_seqs][num_q_heads][P][head_dim]
+ * followed by (running max, running sum) pairs [num_seqs][num_q_heads][P][2],
+ * P = ceil(max_context_len / partition_tokens).
+ * -------------------------------------------------------------------- */
+size_t pkv_decode_workspace_bytes(int num_seqs, int num_q_heads, int head_dim,
+                                  int max_context_len, int partition_tokens);
+
+/* ------------------------------------------------------------------------
+ * pkv_paged_attention_decode -- single-query attention of every sequence
+ * over its paged K/V.
+ *
+ * "PagedAttention 与 vLLM 推理加速" §2.3: the kernel walks the sequence's
+ * blocks through its block table and takes Q (the current token) x K over
+ * every key in them to get the attention scores; §1: each decode step
+ * attends over the K/V of every token so far, the current one included
+ * (context_lens count the token just appended).  With n = context_lens[b]
+ * and g = h / (num_q_heads / num_kv_heads):
+ *   K_j = k_cache[block_tables[b][j / 16], g, j % 16, :]   (V_j alike)
+ *   s_j = scale * <q[b,h,:], K_j>,   j < n
+ *   out[b,h,:] = sum_j softmax(s)_j V_j     (zeros when n == 0)
+ * computed in fp32 and rounded once to dtype.  Entries of block_tables past
+ * page ceil(n/16) - 1 and the unused slots of the last block are never read.
+ *
+ * Work is split into partitions of partition_tokens tokens (0 = 512; else a
+ * multiple of 16 in [16, 2048]); each (sequence, kv-head, partition) keeps
+ * the running max and sum of its exponentials and a partial output, and a
+ * second kernel merges the partitions of sequences longer than one
+ * partition by rescaling each to the overall max (log-sum-exp merge).  The
+ * summation order depends only on logical token positions, so the output
+ * is bit-identical under any relabelling of physical blocks.
+ *
+ * max_context_len: a host-side bound on context_lens (sizes the grid and the
+ *   workspace); max_context_len <= 16 * max_blocks_per_seq.
+ * workspace: device scratch of at least pkv_decode_workspace_bytes(...)
+ *   bytes, 16-byte aligned (may be NULL when that is 0).  Its contents need
+ *   no initialisation and are garbage afterwards.  Two calls that overlap
+ *   on the GPU must not share a workspace.
+ * -------------------------------------------------------------------- */
+pkv_status pkv_paged_attention_decode(void* out, const void* q, const void* k_cache,
+                                      const void* v_cache, const int32_t* block_tables,
+                                      int max_blocks_per_seq, const int32_t* context_lens,
+                                      int max_context_len, int num_seqs, int num_q_heads,
+                                      int num_kv_heads, int head_dim, int num_blocks,
+                                      float scale, int partition_tokens, pkv_dtype dtype,
+                                      void* workspace, size_t workspace_bytes, void* stream);
+
+/* Read and clear the current device's error word (PKV_ERR_* bits) after the
+ * work queued on `stream` so far has finished.  Blocks the host. */
+pkv_status pkv_get_error(uint32_t* flags, void* stream);
+
+/* ------------------------------------------------------------------------
+ * Host block allocator.
+ *
+ * "vLLM + PagedAttention：打造高并发LLM推理引擎", "它是怎么工作的": blocks are
+ * taken on demand as a request grows and go back to the pool when it ends.
+ * "PagedAttention 与 vLLM 推理加速" §3.2(3) and "LLM Systems 24 ..." §3:
+ * requests share blocks (common prefixes, parallel samples) through
+ * reference counts, and a shared block is copied only when one of them
+ * writes into it.
+ *
+ * Policy (the pages leave it open; this is the plain deterministic one):
+ *   - the free list is FIFO, initialised from initial_free_order (NULL =
+ *     0..num_blocks-1); allocation pops the front; a block whose count drops
+ *     to 0 is pushed to the back; free_seq releases a table in table order;
+ *   - fork: the child gets a copy of the parent's table and length, and every
+ *     block in it gains one reference;
+ *   - appending at position p: when p % 16 == 0 a fresh block is appended to
+ *     the table; otherwise, when the last block is shared (count > 1), a
+ *     fresh block replaces it, the old block loses one reference and the
+ *     pair (old, new) is reported for pkv_copy_blocks; otherwise the token
+ *     goes into the last block.  A full shared block is never copied;
+ *   - slot = table[p / 16] * 16 + p % 16.
+ * Every call either succeeds or returns an error and changes nothing.
+ * The handle is not thread-safe; one thread at a time.
+ * -------------------------------------------------------------------- */
+typedef struct pkv_alloc pkv_alloc;
+
+/* Create an allocator over num_blocks blocks (> 0).  initial_free_order,
+ * when not NULL, must be a permutation of 0..num_blocks-1 (host memory). */
+pkv_status pkv_alloc_create(int num_blocks, const int32_t* initial_free_order, pkv_alloc** out);
+void pkv_alloc_destroy(pkv_alloc* a);
+
+/* Add an empty sequence (EINVAL if the id exists). */
+pkv_status pkv_alloc_add_seq(pkv_alloc* a, int64_t seq_id);
+/* Child shares the parent's blocks (EINVAL: no parent, or child exists). */
+pkv_status pkv_alloc_fork(pkv_alloc* a, int64_t parent, int64_t child);
+/* Drop a sequence and its references (EINVAL: unknown id). */
+pkv_status pkv_alloc_free_seq(pkv_alloc* a, int64_t seq_id);
+
+/* Append one token.  *slot receives its slot; *cow_src / *cow_dst receive the
+ * copy pair, or -1 / -1 when no copy is needed. */
+pkv_status pkv_alloc_append_slot(pkv_alloc* a, int64_t seq_id, int64_t* slot, int32_t* cow_src,
+                                 int32_t* cow_dst);
+/* Append n >= 0 tokens to one sequence: slots[n]; cow_pairs[2] receives the
+ * single possible copy pair and *n_cow 0 or 1.  All or nothing. */
+pkv_status pkv_alloc_append_tokens(pkv_alloc* a, int64_t seq_id, int n, int64_t* slots,
+                                   int32_t* cow_pairs, int* n_cow);
+/* One decode step: append one token to each of seq_ids[n] (distinct, known)
+ * in order.  slots[n]; cow_pairs[2 * n] receives *n_cow pairs in order.
+ * All or nothing (PKV_ENOMEM if the pool cannot serve the whole step). */
+pkv_status pkv_alloc_step(pkv_alloc* a, const int64_t* seq_ids, int n, int64_t* slots,
+                          int32_t* cow_pairs, int* n_cow);
+
+/* One sequence's table (up to cap entries), its block count and length. */
+pkv_status pkv_alloc_block_table(const pkv_alloc* a, int64_t seq_id, int32_t* out, int cap,
+                                 int* n_blocks, int64_t* context_len);
+/* Dense tables for a batch: tables[n][width] (entries past a sequence's
+ * last block set to pad) and context_lens[n].  EINVAL if a table is wider
+ * than width or a length exceeds INT32_MAX. */
+pkv_status pkv_alloc_block_tables(const pkv_alloc* a, const int64_t* seq_ids, int n,
+                                  int32_t* tables, int width, int32_t pad, int32_t* context_lens);
+/* Free list in order (free_list[num_blocks] may be NULL) and the count of
+ * every block (refcounts[num_blocks] may be NULL). */
+pkv_status pkv_alloc_state(const pkv_alloc* a, int32_t* free_list, int* n_free,
+                           int32_t* refcounts);
+int pkv_alloc_num_free(const pkv_alloc* a);
+int pkv_alloc_num_blocks(const pkv_alloc* a);
+int pkv_alloc_num_seqs(const pkv_alloc* a);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PKV_H */

@@ -1,0 +1,349 @@
+"""Python binding of libpkv: torch tensors in, C-ABI calls out.
+
+Argument marshalling only -- shape/dtype/device checks, raw pointers, the
+current CUDA stream.  Every step of the path runs in the library's CUDA
+kernels (device ops) or its C++ allocator (host bookkeeping).  PyTorch
+provides device memory and streams.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+from typing import Iterable, List, Optional, Sequence, Tuple
+
+import numpy as np
+import torch
+
+from . import _lib
+from ._lib import check, lib
+
+BLOCK_SIZE = 16
+DEFAULT_PARTITION = 512
+_DT = {torch.float32: 0, torch.float16: 1, torch.bfloat16: 2}
+
+
+def kv_cache_bytes(num_layers: int, num_heads: int, head_dim: int, seq_len: int, dtype_bytes: int) -> int:
+    """Bytes of K plus V for one sequence: 2 * L * H * D * S * dtype_size
+    ("PagedAttention 与 vLLM 推理加速" §1)."""
+    return 2 * num_layers * num_heads * head_dim * seq_len * dtype_bytes
+
+
+def _stream(stream, device) -> int:
+    if stream is None:
+        stream = torch.cuda.current_stream(device)
+    return int(stream.cuda_stream) if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def _dev(t: torch.Tensor, name: str, dtype=None) -> int:
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    return t.data_ptr()
+
+
+def _cache_dims(k_cache: torch.Tensor, v_cache: torch.Tensor):
+    if k_cache.dim() != 4 or k_cache.shape != v_cache.shape or k_cache.dtype != v_cache.dtype:
+        raise ValueError("k_cache/v_cache must both be [num_blocks, Hkv, 16, D] of one dtype")
+    nb, hkv, bs, d = k_cache.shape
+    if bs != BLOCK_SIZE:
+        raise ValueError(f"block size must be {BLOCK_SIZE}")
+    if k_cache.dtype not in _DT:
+        raise ValueError(f"unsupported dtype {k_cache.dtype}")
+    return nb, hkv, d
+
+
+def kv_append(k_new: torch.Tensor, v_new: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
+              slot_mapping: torch.Tensor, stream=None) -> None:
+    """Write each new token's K/V into its slot (slot < 0: skipped).
+
+    k_new/v_new [N, Hkv, D]; slot_mapping int64 [N] on the device.
+    """
+    nb, hkv, d = _cache_dims(k_cache, v_cache)
+    if k_new.shape != v_new.shape or k_new.dim() != 3 or tuple(k_new.shape[1:]) != (hkv, d):
+        raise ValueError("k_new/v_new must be [N, Hkv, D] matching the cache")
+    n = k_new.shape[0]
+    if slot_mapping.shape != (n,):
+        raise ValueError("slot_mapping must be [N]")
+    check(lib.pkv_kv_append(_dev(k_new, "k_new", k_cache.dtype), _dev(v_new, "v_new", k_cache.dtype),
+                            _dev(k_cache, "k_cache"), _dev(v_cache, "v_cache"),
+                            _dev(slot_mapping, "slot_mapping", torch.int64), n, hkv, d, nb,
+                            _DT[k_cache.dtype], _stream(stream, k_cache.device)), "pkv_kv_append")
+
+
+def copy_blocks_check(pairs_host: np.ndarray, num_blocks: int) -> None:
+    """Host check of copy pairs (ids in range, distinct dst, no dst is a src)."""
+    p = np.ascontiguousarray(pairs_host, dtype=np.int32).reshape(-1, 2)
+    check(lib.pkv_copy_blocks_check(p.ctypes.data_as(ctypes.POINTER(ctypes.c_int32)), p.shape[0], num_blocks),
+          "pkv_copy_blocks_check")
+
+
+def copy_blocks(k_cache: torch.Tensor, v_cache: torch.Tensor, pairs: torch.Tensor, stream=None) -> None:
+    """cache[dst] = cache[src] for each (src, dst) row of int32 ``pairs`` [n, 2] (device)."""
+    nb, hkv, d = _cache_dims(k_cache, v_cache)
+    if pairs.dim() != 2 or pairs.shape[1] != 2:
+        raise ValueError("pairs must be [n, 2]")
+    n = pairs.shape[0]
+    if n == 0:
+        return
+    check(lib.pkv_copy_blocks(_dev(k_cache, "k_cache"), _dev(v_cache, "v_cache"),
+                              _dev(pairs, "pairs", torch.int32), n, hkv, d, nb, _DT[k_cache.dtype],
+                              _stream(stream, k_cache.device)), "pkv_copy_blocks")
+
+
+def decode_workspace_bytes(num_seqs: int, num_q_heads: int, head_dim: int, max_context_len: int,
+                           partition: int = 0) -> int:
+    return int(lib.pkv_decode_workspace_bytes(num_seqs, num_q_heads, head_dim, max_context_len, partition))
+
+
+def paged_attention_decode(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
+                           block_tables: torch.Tensor, context_lens: torch.Tensor, max_context_len: int,
+                           scale: float, out: Optional[torch.Tensor] = None,
+                           workspace: Optional[torch.Tensor] = None, partition: int = 0,
+                           stream=None) -> torch.Tensor:
+    """Single-query attention of each sequence over its paged K/V.
+
+    q [B, Hq, D]; block_tables int32 [B, max_blocks]; context_lens int32 [B]
+    (lengths after this step's append); max_context_len: host bound on
+    context_lens.  Returns ``out`` [B, Hq, D] in q's dtype.  ``workspace``
+    (uint8, >= decode_workspace_bytes) is allocated here when not given.
+    """
+    nb, hkv, d = _cache_dims(k_cache, v_cache)
+    if q.dim() != 3 or q.shape[2] != d or q.dtype != k_cache.dtype:
+        raise ValueError("q must be [B, Hq, D] in the cache dtype")
+    B, hq, _ = q.shape
+    if block_tables.dim() != 2 or block_tables.shape[0] != B or context_lens.shape != (B,):
+        raise ValueError("block_tables must be [B, max_blocks] and context_lens [B]")
+    if out is None:
+        out = torch.empty_like(q)
+    need = decode_workspace_bytes(B, hq, d, max_context_len, partition)
+    if need and workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    ws_ptr = _dev(workspace, "workspace") if need else None
+    ws_len = workspace.numel() * workspace.element_size() if need else 0
+    check(lib.pkv_paged_attention_decode(
+        _dev(out, "out", q.dtype), _dev(q, "q"), _dev(k_cache, "k_cache"), _dev(v_cache, "v_cache"),
+        _dev(block_tables, "block_tables", torch.int32), block_tables.shape[1],
+        _dev(context_lens, "context_lens", torch.int32), int(max_context_len), B, hq, hkv, d, nb,
+        float(scale), int(partition), _DT[k_cache.dtype], ws_ptr, ws_len,
+        _stream(stream, q.device)), "pkv_paged_attention_decode")
+    return out
+
+
+def get_error(stream=None, device=None) -> int:
+    """Read and clear the device error word (PKV_ERR_* bits); synchronises."""
+    v = ctypes.c_uint32(0)
+    check(lib.pkv_get_error(ctypes.byref(v), _stream(stream, device)), "pkv_get_error")
+    return int(v.value)
+
+
+# ---------------------------------------------------------------------------
+# host allocator
+# ---------------------------------------------------------------------------
+def _i32p(a: np.ndarray):
+    return a.ctypes.data_as(ctypes.POINTER(ctypes.c_int32))
+
+
+def _i64p(a: np.ndarray):
+    return a.ctypes.data_as(ctypes.POINTER(ctypes.c_int64))
+
+
+class BlockAllocator:
+    """The library's host block allocator (FIFO free list, refcounts, CoW)."""
+
+    def __init__(self, num_blocks: int, free_order: Optional[Sequence[int]] = None):
+        h = ctypes.c_void_p()
+        order = None if free_order is None else np.ascontiguousarray(free_order, dtype=np.int32)
+        check(lib.pkv_alloc_create(int(num_blocks), None if order is None else _i32p(order), ctypes.byref(h)),
+              "pkv_alloc_create")
+        self._h = h
+        self.num_blocks = int(num_blocks)
+
+    def close(self) -> None:
+        if self._h:
+            lib.pkv_alloc_destroy(self._h)
+            self._h = ctypes.c_void_p()
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    def add_seq(self, sid: int) -> None:
+        check(lib.pkv_alloc_add_seq(self._h, int(sid)), "pkv_alloc_add_seq")
+
+    def fork(self, parent: int, child: int) -> None:
+        check(lib.pkv_alloc_fork(self._h, int(parent), int(child)), "pkv_alloc_fork")
+
+    def free_seq(self, sid: int) -> None:
+        check(lib.pkv_alloc_free_seq(self._h, int(sid)), "pkv_alloc_free_seq")
+
+    def append_slot(self, sid: int) -> Tuple[int, Optional[Tuple[int, int]]]:
+        slot, s, d = ctypes.c_int64(), ctypes.c_int32(), ctypes.c_int32()
+        check(lib.pkv_alloc_append_slot(self._h, int(sid), ctypes.byref(slot), ctypes.byref(s), ctypes.byref(d)),
+              "pkv_alloc_append_slot")
+        return slot.value, (None if s.value < 0 else (s.value, d.value))
+
+    def append_tokens(self, sid: int, n: int) -> Tuple[np.ndarray, np.ndarray]:
+        slots = np.empty(max(n, 1), dtype=np.int64)
+        pairs = np.empty(2, dtype=np.int32)
+        nc = ctypes.c_int()
+        check(lib.pkv_alloc_append_tokens(self._h, int(sid), int(n), _i64p(slots), _i32p(pairs), ctypes.byref(nc)),
+              "pkv_alloc_append_tokens")
+        return slots[:n], pairs[:2 * nc.value].reshape(-1, 2)
+
+    def step(self, sids: Iterable[int]) -> Tuple[np.ndarray, np.ndarray]:
+        ids = np.ascontiguousarray(list(sids), dtype=np.int64)
+        n = ids.shape[0]
+        slots = np.empty(max(n, 1), dtype=np.int64)
+        pairs = np.empty(max(2 * n, 2), dtype=np.int32)
+        nc = ctypes.c_int()
+        check(lib.pkv_alloc_step(self._h, _i64p(ids), n, _i64p(slots), _i32p(pairs), ctypes.byref(nc)),
+              "pkv_alloc_step")
+        return slots[:n], pairs[:2 * nc.value].reshape(-1, 2)
+
+    def block_table(self, sid: int) -> Tuple[List[int], int]:
+        nb, ln = ctypes.c_int(), ctypes.c_int64()
+        check(lib.pkv_alloc_block_table(self._h, int(sid), None, 0, ctypes.byref(nb), ctypes.byref(ln)),
+              "pkv_alloc_block_table")
+        out = np.empty(max(nb.value, 1), dtype=np.int32)
+        check(lib.pkv_alloc_block_table(self._h, int(sid), _i32p(out), nb.value, ctypes.byref(nb),
+                                        ctypes.byref(ln)), "pkv_alloc_block_table")
+        return [int(x) for x in out[:nb.value]], int(ln.value)
+
+    def block_tables(self, sids: Sequence[int], width: int, pad: int) -> Tuple[np.ndarray, np.ndarray]:
+        ids = np.ascontiguousarray(list(sids), dtype=np.int64)
+        n = ids.shape[0]
+        tables = np.empty((max(n, 1), max(width, 1)), dtype=np.int32)
+        lens = np.empty(max(n, 1), dtype=np.int32)
+        check(lib.pkv_alloc_block_tables(self._h, _i64p(ids), n, _i32p(tables), int(width), int(pad), _i32p(lens)),
+              "pkv_alloc_block_tables")
+        return tables[:n, :width], lens[:n]
+
+    def state(self) -> Tuple[List[int], List[int]]:
+        free = np.empty(self.num_blocks, dtype=np.int32)
+        rc = np.empty(self.num_blocks, dtype=np.int32)
+        nf = ctypes.c_int()
+        check(lib.pkv_alloc_state(self._h, _i32p(free), ctypes.byref(nf), _i32p(rc)), "pkv_alloc_state")
+        return [int(x) for x in free[:nf.value]], [int(x) for x in rc]
+
+    @property
+    def num_free(self) -> int:
+        return int(lib.pkv_alloc_num_free(self._h))
+
+    @property
+    def num_seqs(self) -> int:
+        return int(lib.pkv_alloc_num_seqs(self._h))
+
+
+# ---------------------------------------------------------------------------
+# a paged KV cache: the pool (torch device memory) plus the allocator
+# ---------------------------------------------------------------------------
+class PagedKVCache:
+    """One layer's paged K/V pool on a device, with its block allocator.
+
+    ``step(seq_ids, q, k_new, v_new)`` is one decode step of the hot path:
+    the allocator hands out each sequence's slot (and copy-on-write pairs),
+    the shared blocks are copied, the new K/V are appended and every
+    sequence's query attends over its whole context.  Inputs may live on
+    the host (they are copied in) or on the device; the result is returned
+    on the inputs' device.
+    """
+
+    def __init__(self, num_blocks: int, num_kv_heads: int, head_dim: int, dtype: torch.dtype,
+                 device="cuda", free_order: Optional[Sequence[int]] = None, fill=float("nan")):
+        self.device = torch.device(device)
+        self.dtype = dtype
+        self.num_blocks, self.Hkv, self.D = int(num_blocks), int(num_kv_heads), int(head_dim)
+        shape = (self.num_blocks, self.Hkv, BLOCK_SIZE, self.D)
+        self.k = torch.full(shape, fill, dtype=dtype, device=self.device)
+        self.v = torch.full(shape, fill, dtype=dtype, device=self.device)
+        self.alloc = BlockAllocator(num_blocks, free_order)
+        self._ws = torch.empty(0, dtype=torch.uint8, device=self.device)
+
+    def workspace(self, nbytes: int) -> torch.Tensor:
+        if self._ws.numel() < nbytes:
+            self._ws = torch.empty(nbytes, dtype=torch.uint8, device=self.device)
+        return self._ws
+
+    # bookkeeping passthroughs
+    def add_seq(self, sid):
+        self.alloc.add_seq(sid)
+
+    def fork(self, parent, child):
+        self.alloc.fork(parent, child)
+
+    def free_seq(self, sid):
+        self.alloc.free_seq(sid)
+
+    def prefill(self, sid: int, k: torch.Tensor, v: torch.Tensor, stream=None) -> np.ndarray:
+        """Append n tokens' K/V ([n, Hkv, D]) to one sequence."""
+        slots, pairs = self.alloc.append_tokens(sid, k.shape[0])
+        if len(pairs):
+            copy_blocks(self.k, self.v, torch.from_numpy(pairs).to(self.device), stream)
+        kv_append(k.to(self.device), v.to(self.device), self.k, self.v,
+                  torch.from_numpy(slots).to(self.device), stream)
+        return slots
+
+    def plan_step(self, seq_ids: Sequence[int], width: Optional[int] = None):
+        """Host part of a decode step: slots, CoW pairs, tables, lengths."""
+        slots, pairs = self.alloc.step(seq_ids)
+        copy_blocks_check(pairs, self.num_blocks)
+        if width is None:
+            width = max(1, max(len(self.alloc.block_table(s)[0]) for s in seq_ids)) if len(seq_ids) else 1
+        tables, lens = self.alloc.block_tables(seq_ids, width, self.num_blocks)
+        return slots, pairs, tables, lens
+
+    def run_step(self, slot_mapping: torch.Tensor, cow_pairs: torch.Tensor, block_tables: torch.Tensor,
+                 context_lens: torch.Tensor, max_context_len: int, q: torch.Tensor, k_new: torch.Tensor,
+                 v_new: torch.Tensor, out: Optional[torch.Tensor] = None, scale: Optional[float] = None,
+                 partition: int = 0, stream=None) -> torch.Tensor:
+        """Device part of a decode step: copy-on-write copies, append, decode.
+
+        Inputs may be host tensors (pinned for asynchronous copies) or
+        device tensors.  When ``out`` is a host tensor the result is copied
+        into it asynchronously on the stream; synchronise before reading.
+        Returns the device output.
+        """
+        dev = self.device
+        st = torch.cuda.current_stream(dev) if stream is None else stream
+
+        def d(t):
+            return t if t.device == dev else t.to(dev, non_blocking=True)
+
+        with torch.cuda.stream(st):
+            if cow_pairs.shape[0]:
+                copy_blocks(self.k, self.v, d(cow_pairs), st)
+            kv_append(d(k_new), d(v_new), self.k, self.v, d(slot_mapping), st)
+            B, hq = q.shape[0], q.shape[1]
+            ws = self.workspace(decode_workspace_bytes(B, hq, self.D, max_context_len, partition))
+            if out is not None and out.device == dev:
+                res = out
+            else:
+                res = self._out_buffer(q.shape)
+            paged_attention_decode(d(q), self.k, self.v, d(block_tables), d(context_lens), max_context_len,
+                                   (1.0 / math.sqrt(self.D)) if scale is None else scale, out=res,
+                                   workspace=ws, partition=partition, stream=st)
+            if out is not None and out.device != dev:
+                out.copy_(res, non_blocking=True)
+        return res
+
+    def _out_buffer(self, shape) -> torch.Tensor:
+        buf = getattr(self, "_out", None)
+        if buf is None or tuple(buf.shape) != tuple(shape):
+            buf = torch.empty(tuple(shape), dtype=self.dtype, device=self.device)
+            self._out = buf
+        return buf
+
+    def step(self, seq_ids: Sequence[int], q: torch.Tensor, k_new: torch.Tensor, v_new: torch.Tensor,
+             scale: Optional[float] = None, partition: int = 0, stream=None) -> torch.Tensor:
+        """Host plan (allocator) + device step; returns the output on q's device."""
+        slots, pairs, tables, lens = self.plan_step(seq_ids)
+        max_ctx = int(lens.max()) if len(lens) else 0
+        out = self.run_step(torch.from_numpy(slots), torch.from_numpy(np.ascontiguousarray(pairs)),
+                            torch.from_numpy(np.ascontiguousarray(tables)), torch.from_numpy(lens), max_ctx,
+                            q, k_new, v_new, scale=scale, partition=partition, stream=stream)
+        return out.clone() if q.device == self.device else out.to(q.device)

@@ -1,0 +1,79 @@
+// Slot-mapped append of new tokens' K/V and copy-on-write block copy.
+//
+// Both are bit copies of 16-byte chunks: one thread moves one chunk, so a
+// warp moves 512 contiguous bytes of a row (append) or of a block (copy),
+// fully coalesced on both sides.
+#pragma once
+
+#include "common.cuh"
+
+namespace pkv {
+
+// "vLLM + PagedAttention：打造高并发LLM推理引擎", "它是怎么工作的": token t
+// lands in slot s = block * 16 + offset of its sequence's page table; old
+// tokens never move.  Chunks [0, total) are K, [total, 2 total) are V, where
+// total = num_tokens * Hkv * row_chunks.
+__global__ void __launch_bounds__(256)
+    kv_append_kernel(const uint4* __restrict__ k_new, const uint4* __restrict__ v_new,
+                     uint4* __restrict__ k_cache, uint4* __restrict__ v_cache,
+                     const int64_t* __restrict__ slots, long long total, int Hkv, int row_chunks,
+                     int num_blocks) {
+  const long long stride = static_cast<long long>(gridDim.x) * blockDim.x;
+  for (long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; i < 2 * total;
+       i += stride) {
+    const bool is_v = i >= total;
+    const long long j = is_v ? i - total : i;
+    const int c = static_cast<int>(j % row_chunks);
+    const long long th = j / row_chunks;
+    const int h = static_cast<int>(th % Hkv);
+    const long long t = th / Hkv;
+    const int64_t s = slots[t];
+    if (s < 0) continue;  // padding
+    const int64_t blk = s / kBlockSize;
+    const int off = static_cast<int>(s % kBlockSize);
+    if (blk >= num_blocks) {
+      raise_error(PKV_ERR_SLOT_RANGE);
+      continue;
+    }
+    const long long dst = ((blk * Hkv + h) * kBlockSize + off) * row_chunks + c;
+    if (is_v)
+      v_cache[dst] = v_new[j];
+    else
+      k_cache[dst] = k_new[j];
+  }
+}
+
+// "PagedAttention 与 vLLM 推理加速" §3.2(3): copy a shared block before a
+// writer appends into it.  grid = (chunk groups, pair, K|V).
+__global__ void __launch_bounds__(256)
+    copy_blocks_kernel(uint4* __restrict__ k_cache, uint4* __restrict__ v_cache,
+                       const int32_t* __restrict__ pairs, long long block_chunks, int num_blocks) {
+  constexpr int kUnroll = 4;
+  const int p = blockIdx.y;
+  const int src = pairs[2 * p];
+  const int dst = pairs[2 * p + 1];
+  if (src < 0 || src >= num_blocks || dst < 0 || dst >= num_blocks) {
+    if (threadIdx.x == 0 && blockIdx.x == 0) raise_error(PKV_ERR_COPY_RANGE);
+    return;
+  }
+  uint4* cache = blockIdx.z ? v_cache : k_cache;
+  const uint4* from = cache + static_cast<size_t>(src) * block_chunks;
+  uint4* to = cache + static_cast<size_t>(dst) * block_chunks;
+  const long long step = static_cast<long long>(gridDim.x) * blockDim.x * kUnroll;
+  for (long long base = static_cast<long long>(blockIdx.x) * blockDim.x * kUnroll + threadIdx.x;
+       base < block_chunks; base += step) {
+    uint4 v[kUnroll];
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u) {
+      const long long i = base + static_cast<long long>(u) * blockDim.x;
+      if (i < block_chunks) v[u] = from[i];
+    }
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u) {
+      const long long i = base + static_cast<long long>(u) * blockDim.x;
+      if (i < block_chunks) to[i] = v[u];
+    }
+  }
+}
+
+}  // namespace pkv

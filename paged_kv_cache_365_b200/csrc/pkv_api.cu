@@ -1,0 +1,235 @@
+// C ABI of libpkv: argument checks, dispatch to the kernel instantiations,
+// launches.  Every host-checkable argument is checked before any CUDA call,
+// so a rejected call has no side effect (and works without a GPU).
+#include <cmath>
+#include <cstdint>
+#include <unordered_set>
+
+#include "cache_ops.cuh"
+#include "decode.cuh"
+#include "pkv.h"
+
+namespace pkv {
+__device__ unsigned int g_error_snapshot = 0u;
+
+__global__ void take_error_snapshot_kernel() { g_error_snapshot = atomicExch(&g_error_word, 0u); }
+}  // namespace pkv
+
+namespace {
+
+constexpr int kWarps = 4;
+constexpr int kMaxPartition = kWarps * 32 * PKV_BLOCK_SIZE;  // one table entry per lane
+constexpr float kLog2e = 1.4426950408889634f;
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int dtype_bytes(pkv_dtype dt) {
+  switch (dt) {
+    case PKV_F32: return 4;
+    case PKV_F16: return 2;
+    case PKV_BF16: return 2;
+  }
+  return 0;
+}
+
+int resolve_partition(int p) {
+  if (p == 0) return PKV_DEFAULT_PARTITION;
+  if (p < PKV_BLOCK_SIZE || p > kMaxPartition || p % PKV_BLOCK_SIZE != 0) return -1;
+  return p;
+}
+
+bool head_dim_ok(int d) { return d == 64 || d == 128; }
+bool group_ok(int g) { return g == 1 || g == 2 || g == 4 || g == 8; }
+
+// Stages per warp: keep roughly 24 KB of K+V in flight per warp.
+constexpr int stages_for(int stage_bytes) {
+  return stage_bytes >= 16384 ? 2 : (24576 / stage_bytes > 8 ? 8 : 24576 / stage_bytes);
+}
+
+pkv_status launched() { return cudaGetLastError() == cudaSuccess ? PKV_OK : PKV_ECUDA; }
+
+template <typename T, int D, int G>
+pkv_status launch_decode(const pkv::DecodeArgs& a, cudaStream_t st) {
+  constexpr int kStages = stages_for(2 * PKV_BLOCK_SIZE * D * static_cast<int>(sizeof(T)));
+  using S = pkv::DecodeShape<T, D, G, kWarps, kStages>;
+  auto kfn = pkv::paged_decode_partition_kernel<T, D, G, kWarps, kStages>;
+  if (cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(S::kSmem)) !=
+      cudaSuccess)
+    return PKV_ECUDA;
+  const dim3 grid(a.num_kv_heads, a.num_seqs, a.num_parts);
+  kfn<<<grid, kWarps * 32, S::kSmem, st>>>(a);
+  if (launched() != PKV_OK) return PKV_ECUDA;
+  if (a.num_parts > 1) {
+    const dim3 g2((a.num_q_heads + 3) / 4, a.num_seqs);
+    pkv::paged_decode_reduce_kernel<T, D><<<g2, 128, 0, st>>>(a);
+    if (launched() != PKV_OK) return PKV_ECUDA;
+  }
+  return PKV_OK;
+}
+
+template <typename T, int D>
+pkv_status dispatch_group(const pkv::DecodeArgs& a, int G, cudaStream_t st) {
+  switch (G) {
+    case 1: return launch_decode<T, D, 1>(a, st);
+    case 2: return launch_decode<T, D, 2>(a, st);
+    case 4: return launch_decode<T, D, 4>(a, st);
+    case 8: return launch_decode<T, D, 8>(a, st);
+  }
+  return PKV_EINVAL;
+}
+
+template <typename T>
+pkv_status dispatch_dim(const pkv::DecodeArgs& a, int D, int G, cudaStream_t st) {
+  if (D == 64) return dispatch_group<T, 64>(a, G, st);
+  if (D == 128) return dispatch_group<T, 128>(a, G, st);
+  return PKV_EINVAL;
+}
+
+size_t workspace_bytes(long long B, long long Hq, long long D, long long P) {
+  if (P <= 1) return 0;
+  return static_cast<size_t>(B * Hq * P * (D + 2) * 4);
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* pkv_status_string(pkv_status s) {
+  switch (s) {
+    case PKV_OK: return "ok";
+    case PKV_EINVAL: return "invalid argument";
+    case PKV_ENOMEM: return "block pool exhausted";
+    case PKV_ECUDA: return "CUDA error";
+  }
+  return "unknown status";
+}
+
+int pkv_abi_version(void) { return 1; }
+
+pkv_status pkv_kv_append(const void* k_new, const void* v_new, void* k_cache, void* v_cache,
+                         const int64_t* slot_mapping, int num_tokens, int num_kv_heads, int head_dim,
+                         int num_blocks, pkv_dtype dtype, void* stream) {
+  const int es = dtype_bytes(dtype);
+  if (es == 0 || num_tokens < 0 || num_kv_heads <= 0 || !head_dim_ok(head_dim) || num_blocks <= 0)
+    return PKV_EINVAL;
+  if (num_tokens == 0) return PKV_OK;
+  if (!k_new || !v_new || !k_cache || !v_cache || !slot_mapping) return PKV_EINVAL;
+  if (!aligned16(k_new) || !aligned16(v_new) || !aligned16(k_cache) || !aligned16(v_cache)) return PKV_EINVAL;
+  const int row_chunks = head_dim * es / 16;
+  const long long total = static_cast<long long>(num_tokens) * num_kv_heads * row_chunks;
+  const long long want = (2 * total + 255) / 256;
+  const int blocks = static_cast<int>(want < 148 * 32 ? want : 148 * 32);
+  pkv::kv_append_kernel<<<blocks, 256, 0, static_cast<cudaStream_t>(stream)>>>(
+      static_cast<const uint4*>(k_new), static_cast<const uint4*>(v_new), static_cast<uint4*>(k_cache),
+      static_cast<uint4*>(v_cache), slot_mapping, total, num_kv_heads, row_chunks, num_blocks);
+  return launched();
+}
+
+pkv_status pkv_copy_blocks(void* k_cache, void* v_cache, const int32_t* pairs, int num_pairs, int num_kv_heads,
+                           int head_dim, int num_blocks, pkv_dtype dtype, void* stream) {
+  const int es = dtype_bytes(dtype);
+  if (es == 0 || num_pairs < 0 || num_pairs > 65535 || num_kv_heads <= 0 || !head_dim_ok(head_dim) ||
+      num_blocks <= 0)
+    return PKV_EINVAL;
+  if (num_pairs == 0) return PKV_OK;
+  if (!k_cache || !v_cache || !pairs || !aligned16(k_cache) || !aligned16(v_cache)) return PKV_EINVAL;
+  const long long block_chunks = static_cast<long long>(num_kv_heads) * PKV_BLOCK_SIZE * head_dim * es / 16;
+  const long long per_cta = 256 * 4;
+  const int gx = static_cast<int>((block_chunks + per_cta - 1) / per_cta);
+  const dim3 grid(gx, num_pairs, 2);
+  pkv::copy_blocks_kernel<<<grid, 256, 0, static_cast<cudaStream_t>(stream)>>>(
+      static_cast<uint4*>(k_cache), static_cast<uint4*>(v_cache), pairs, block_chunks, num_blocks);
+  return launched();
+}
+
+pkv_status pkv_copy_blocks_check(const int32_t* pairs_host, int num_pairs, int num_blocks) {
+  if (num_pairs < 0 || num_blocks <= 0 || (num_pairs > 0 && pairs_host == nullptr)) return PKV_EINVAL;
+  std::unordered_set<int32_t> dsts, srcs;
+  for (int i = 0; i < num_pairs; ++i) {
+    const int32_t s = pairs_host[2 * i], d = pairs_host[2 * i + 1];
+    if (s < 0 || s >= num_blocks || d < 0 || d >= num_blocks) return PKV_EINVAL;
+    if (!dsts.insert(d).second) return PKV_EINVAL;
+    srcs.insert(s);
+  }
+  for (int32_t d : dsts)
+    if (srcs.count(d)) return PKV_EINVAL;
+  return PKV_OK;
+}
+
+size_t pkv_decode_workspace_bytes(int num_seqs, int num_q_heads, int head_dim, int max_context_len,
+                                  int partition_tokens) {
+  const int part = resolve_partition(partition_tokens);
+  if (part < 0 || num_seqs < 0 || num_q_heads <= 0 || !head_dim_ok(head_dim) || max_context_len < 0) return 0;
+  const long long P = (static_cast<long long>(max_context_len) + part - 1) / part;
+  return workspace_bytes(num_seqs, num_q_heads, head_dim, P);
+}
+
+pkv_status pkv_paged_attention_decode(void* out, const void* q, const void* k_cache, const void* v_cache,
+                                      const int32_t* block_tables, int max_blocks_per_seq,
+                                      const int32_t* context_lens, int max_context_len, int num_seqs,
+                                      int num_q_heads, int num_kv_heads, int head_dim, int num_blocks, float scale,
+                                      int partition_tokens, pkv_dtype dtype, void* workspace,
+                                      size_t workspace_bytes_given, void* stream) {
+  const int part = resolve_partition(partition_tokens);
+  if (dtype_bytes(dtype) == 0 || part < 0 || num_seqs < 0 || num_seqs > 65535 || num_kv_heads <= 0 ||
+      num_kv_heads > 65535 || num_q_heads <= 0 || num_q_heads % num_kv_heads != 0 ||
+      !group_ok(num_q_heads / num_kv_heads) || !head_dim_ok(head_dim) || num_blocks <= 0 ||
+      max_context_len < 0 || max_blocks_per_seq <= 0 ||
+      static_cast<long long>(max_context_len) > static_cast<long long>(max_blocks_per_seq) * PKV_BLOCK_SIZE ||
+      !std::isfinite(scale))
+    return PKV_EINVAL;
+  if (num_seqs == 0) return PKV_OK;
+  if (!out || !q || !k_cache || !v_cache || !block_tables || !context_lens) return PKV_EINVAL;
+  if (!aligned16(out) || !aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache)) return PKV_EINVAL;
+  const long long P = (static_cast<long long>(max_context_len) + part - 1) / part;
+  if (P > 65535) return PKV_EINVAL;
+  const size_t need = workspace_bytes(num_seqs, num_q_heads, head_dim, P);
+  if (need > 0 && (workspace == nullptr || workspace_bytes_given < need || !aligned16(workspace)))
+    return PKV_EINVAL;
+
+  pkv::DecodeArgs a;
+  a.out = out;
+  a.q = q;
+  a.k_cache = static_cast<const unsigned char*>(k_cache);
+  a.v_cache = static_cast<const unsigned char*>(v_cache);
+  a.block_tables = block_tables;
+  a.context_lens = context_lens;
+  a.ws_o = static_cast<float*>(need ? workspace : nullptr);
+  a.ws_ml = need ? reinterpret_cast<float2*>(static_cast<float*>(workspace) +
+                                              static_cast<size_t>(num_seqs) * num_q_heads * P * head_dim)
+                 : nullptr;
+  a.bt_stride = max_blocks_per_seq;
+  a.max_ctx = max_context_len;
+  a.num_seqs = num_seqs;
+  a.num_q_heads = num_q_heads;
+  a.num_kv_heads = num_kv_heads;
+  a.num_blocks = num_blocks;
+  a.partition = part;
+  a.num_parts = P > 1 ? static_cast<int>(P) : 1;
+  a.qk_scale = scale * kLog2e;
+
+  const int G = num_q_heads / num_kv_heads;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  switch (dtype) {
+    case PKV_F32: return dispatch_dim<float>(a, head_dim, G, st);
+    case PKV_F16: return dispatch_dim<__half>(a, head_dim, G, st);
+    case PKV_BF16: return dispatch_dim<__nv_bfloat16>(a, head_dim, G, st);
+  }
+  return PKV_EINVAL;
+}
+
+pkv_status pkv_get_error(uint32_t* flags, void* stream) {
+  if (flags == nullptr) return PKV_EINVAL;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  pkv::take_error_snapshot_kernel<<<1, 1, 0, st>>>();
+  if (cudaGetLastError() != cudaSuccess) return PKV_ECUDA;
+  unsigned int v = 0;
+  if (cudaMemcpyFromSymbolAsync(&v, pkv::g_error_snapshot, sizeof(v), 0, cudaMemcpyDeviceToHost, st) !=
+      cudaSuccess)
+    return PKV_ECUDA;
+  if (cudaStreamSynchronize(st) != cudaSuccess) return PKV_ECUDA;
+  *flags = v;
+  return PKV_OK;
+}
+
+}  // extern "C"

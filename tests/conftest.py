@@ -24,3 +24,15 @@ def pytest_collection_modifyitems(config, items):
     for item in items:
         if "gpu" in item.keywords:
             item.add_marker(skip)
+
+
+def pytest_sessionstart(session):
+    # the CPU suite loads libpkv.so (allocator, ABI checks): build it when it
+    # is missing or older than its sources (nvcc cross-compiles without a GPU)
+    import importlib.util
+    path = os.path.join(ROOT, "paged_kv_cache_365_b200", "_build.py")
+    spec = importlib.util.spec_from_file_location("_pkv_build", path)
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)  # loads the build script without importing the package
+    if not mod.up_to_date():
+        mod.build()

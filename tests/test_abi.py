@@ -1,0 +1,128 @@
+"""The C-ABI library loads, exports every entry point include/pkv.h
+declares, and rejects bad arguments before touching the GPU (no compute
+calls here: these run without a GPU)."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "pkv.h")
+
+
+def header_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(pkv_[a-z0-9_]+)\s*\(", text)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from paged_kv_cache_365_b200 import _lib
+    return _lib.lib
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = header_functions()
+    assert len(names) >= 20
+    raw = ctypes.CDLL(os.path.join(ROOT, "paged_kv_cache_365_b200", "libpkv.so"))
+    for n in names:
+        assert hasattr(raw, n), n
+
+
+def test_binding_prototypes_cover_the_header():
+    from paged_kv_cache_365_b200 import _lib
+    assert sorted(_lib.PROTOTYPES) == header_functions()
+
+
+def test_status_strings(lib):
+    assert lib.pkv_status_string(0) == b"ok"
+    assert lib.pkv_status_string(2) == b"block pool exhausted"
+    assert lib.pkv_abi_version() == 1
+
+
+FAKE = ctypes.c_void_p(1 << 20)  # 16-byte aligned; never dereferenced (rejected first)
+ODD = ctypes.c_void_p((1 << 20) + 8)
+
+
+def decode(lib, **kw):
+    args = dict(out=FAKE, q=FAKE, k=FAKE, v=FAKE, bt=FAKE, mb=8, cl=FAKE, maxctx=100, B=2, Hq=8, Hkv=2,
+                D=128, NB=64, scale=0.1, part=0, dt=1, ws=FAKE, wsb=1 << 30, stream=None)
+    args.update(kw)
+    return lib.pkv_paged_attention_decode(args["out"], args["q"], args["k"], args["v"], args["bt"], args["mb"],
+                                          args["cl"], args["maxctx"], args["B"], args["Hq"], args["Hkv"],
+                                          args["D"], args["NB"], args["scale"], args["part"], args["dt"],
+                                          args["ws"], args["wsb"], args["stream"])
+
+
+@pytest.mark.parametrize("bad", [
+    dict(D=96), dict(D=256), dict(Hq=6, Hkv=2), dict(Hq=7, Hkv=2), dict(Hq=32, Hkv=2), dict(part=17),
+    dict(part=4096), dict(part=8), dict(dt=3), dict(NB=0), dict(mb=0), dict(maxctx=8 * 16 + 1),
+    dict(maxctx=-1), dict(B=-1), dict(B=70000), dict(out=ODD), dict(k=ODD), dict(q=None),
+    dict(scale=float("nan")), dict(maxctx=1000, mb=100, ws=None), dict(maxctx=1000, mb=100, wsb=100),
+])
+def test_decode_rejects_bad_arguments(lib, bad):
+    assert decode(lib, **bad) == 1
+
+
+def test_decode_workspace_bytes(lib):
+    # one partition: nothing needed
+    assert lib.pkv_decode_workspace_bytes(4, 8, 128, 512, 0) == 0
+    # 3 partitions of 512: B*Hq*P*(D+2)*4
+    assert lib.pkv_decode_workspace_bytes(4, 8, 128, 1025, 0) == 4 * 8 * 3 * 130 * 4
+    assert lib.pkv_decode_workspace_bytes(4, 8, 64, 100, 16) == 4 * 8 * 7 * 66 * 4
+    assert lib.pkv_decode_workspace_bytes(4, 8, 96, 1000, 0) == 0  # unsupported -> 0
+    assert lib.pkv_decode_workspace_bytes(4, 8, 128, 1000, 17) == 0
+
+
+def test_zero_sized_calls_are_no_ops(lib):
+    assert decode(lib, B=0, out=None, q=None) == 0
+    assert lib.pkv_kv_append(None, None, None, None, None, 0, 2, 64, 16, 0, None) == 0
+    assert lib.pkv_copy_blocks(None, None, None, 0, 2, 64, 16, 0, None) == 0
+
+
+@pytest.mark.parametrize("args", [
+    (FAKE, FAKE, FAKE, FAKE, FAKE, 4, 2, 80, 16, 1, None),     # head_dim
+    (FAKE, FAKE, FAKE, FAKE, FAKE, 4, 0, 64, 16, 1, None),     # Hkv
+    (FAKE, FAKE, FAKE, FAKE, FAKE, -1, 2, 64, 16, 1, None),    # num_tokens
+    (FAKE, FAKE, ODD, FAKE, FAKE, 4, 2, 64, 16, 1, None),      # alignment
+    (FAKE, FAKE, FAKE, FAKE, None, 4, 2, 64, 16, 1, None),     # slots
+    (FAKE, FAKE, FAKE, FAKE, FAKE, 4, 2, 64, 16, 7, None),     # dtype
+])
+def test_append_rejects_bad_arguments(lib, args):
+    assert lib.pkv_kv_append(*args) == 1
+
+
+def test_copy_rejects_bad_arguments(lib):
+    assert lib.pkv_copy_blocks(FAKE, FAKE, FAKE, 70000, 2, 64, 16, 1, None) == 1
+    assert lib.pkv_copy_blocks(FAKE, FAKE, None, 3, 2, 64, 16, 1, None) == 1
+    assert lib.pkv_copy_blocks(ODD, FAKE, FAKE, 3, 2, 64, 16, 1, None) == 1
+
+
+@pytest.mark.parametrize("pairs,ok", [
+    ([[0, 1], [2, 3]], True),
+    ([], True),
+    ([[0, 1], [2, 1]], False),   # duplicate dst
+    ([[0, 1], [1, 2]], False),   # dst 1 is also a src
+    ([[0, 16]], False),          # out of range
+    ([[-1, 3]], False),
+])
+def test_copy_pairs_host_check(pairs, ok):
+    from paged_kv_cache_365_b200 import PkvError, copy_blocks_check
+    p = np.array(pairs, dtype=np.int32).reshape(-1, 2)
+    if ok:
+        copy_blocks_check(p, 16)
+    else:
+        with pytest.raises(PkvError):
+            copy_blocks_check(p, 16)
+
+
+def test_kv_cache_bytes_matches_page_example():
+    import json
+    from paged_kv_cache_365_b200 import kv_cache_bytes
+    g = json.load(open(os.path.join(ROOT, "tests", "golden", "kv_size_example.json")))
+    n = kv_cache_bytes(g["layers"], g["heads"], g["head_dim"], g["seq_len"], g["dtype_bytes"])
+    assert n == g["expected_bytes"]
+    assert abs(n / 1e9 - g["page_figure_gb"]) / g["page_figure_gb"] < g["page_figure_rel_tol"]

@@ -178,6 +178,16 @@ def llama7b(seed: int = 0) -> Workload:
     return _independent("llama7b", 64, 32, 32, 128, "f16", ctx, 16384, seed, rng)
 
 
+def llama7b_compact(seed: int = 0) -> Workload:
+    """llama7b's lengths, heads and dtype in a pool of 1.1x the blocks used
+    (about 1.3 GB instead of 4.3 GB): the small case for full profiler
+    captures of the same kernel."""
+    rng = np.random.default_rng(seed)
+    ctx = rng.integers(128, 2048, size=64, endpoint=True)
+    need = sum(_blocks_for(c) for c in ctx)
+    return _independent("llama7b_compact", 64, 32, 32, 128, "f16", ctx, math.ceil(1.1 * need), seed, rng)
+
+
 def gqa8b(seed: int = 0, sigma: float = 1.0) -> Workload:
     rng = np.random.default_rng(seed)
     raw = rng.lognormal(mean=math.log(1024.0), sigma=sigma, size=256)
@@ -248,6 +258,7 @@ def custom(ctx: Sequence[int], Hq: int, Hkv: int, D: int, dtype: str,
 NAMED = {
     "tiny": tiny,
     "llama7b": llama7b,
+    "llama7b_compact": llama7b_compact,
     "gqa8b": gqa8b,
     "prefix13b": prefix13b,
     "long": long,
