@@ -163,6 +163,44 @@ pkv_status pkv_paged_attention_decode(void* out, const void* q, const void* k_ca
                                       float scale, int partition_tokens, pkv_dtype dtype,
                                       void* workspace, size_t workspace_bytes, void* stream);
 
+/* ------------------------------------------------------------------------
+ * pkv_paged_attention_decode_static_ws -- pkv_paged_attention_decode for
+ * callers that cannot allocate device memory.
+ *
+ * The pages have no counterpart to this call; it exists for library users.
+ * Some callers must not call cudaMalloc: code running under a framework's
+ * caching allocator that has already reserved the GPU's memory (a raw
+ * cudaMalloc can fail there, or fragment the pool), and code on a
+ * latency-critical path, where cudaMalloc/cudaFree may synchronise the
+ * device.  Such a caller has no way to provide the split-K workspace that
+ * pkv_paged_attention_decode needs for contexts longer than one partition.
+ *
+ * This variant takes the same arguments minus the workspace and uses a
+ * fixed scratch area of PKV_STATIC_WORKSPACE_BYTES that the library itself
+ * holds in device memory: every GPU that loads libpkv.so keeps that much
+ * memory until the process exits.  It allocates nothing.
+ *   - If pkv_decode_workspace_bytes(...) for the call exceeds
+ *     PKV_STATIC_WORKSPACE_BYTES, it returns PKV_EINVAL and launches nothing
+ *     (use pkv_paged_attention_decode with a caller-owned workspace then).
+ *   - The first call on a device looks up that device's address of the
+ *     scratch area (a runtime query, no allocation), with the caller's
+ *     current device; make that first call before any stream capture.
+ *   - All calls on a device share the one scratch area, and it keeps what
+ *     the previous call left in it.  The decode writes every scratch value
+ *     before it reads it, so nothing needs clearing between calls, but two
+ *     calls whose work overlaps on the GPU (different streams without
+ *     ordering between them) race on the scratch area.
+ * Other arguments, results and errors are those of pkv_paged_attention_decode.
+ * -------------------------------------------------------------------- */
+#define PKV_STATIC_WORKSPACE_BYTES (16u << 20)
+pkv_status pkv_paged_attention_decode_static_ws(void* out, const void* q, const void* k_cache,
+                                                const void* v_cache, const int32_t* block_tables,
+                                                int max_blocks_per_seq, const int32_t* context_lens,
+                                                int max_context_len, int num_seqs, int num_q_heads,
+                                                int num_kv_heads, int head_dim, int num_blocks,
+                                                float scale, int partition_tokens, pkv_dtype dtype,
+                                                void* stream);
+
 /* Read and clear the current device's error word (PKV_ERR_* bits) after the
  * work queued on `stream` so far has finished.  Blocks the host. */
 pkv_status pkv_get_error(uint32_t* flags, void* stream);

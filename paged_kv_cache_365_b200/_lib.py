@@ -22,6 +22,8 @@ ERR_SLOT_RANGE = 0x4
 ERR_COPY_RANGE = 0x8
 ERR_TIMEOUT = 0x10
 
+STATIC_WORKSPACE_BYTES = 16 << 20  # PKV_STATIC_WORKSPACE_BYTES
+
 # name -> (restype, argtypes); the same list as include/pkv.h
 PROTOTYPES = {
     "pkv_status_string": (ctypes.c_char_p, [c_int]),
@@ -35,6 +37,9 @@ PROTOTYPES = {
     "pkv_paged_attention_decode": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_int,
                                            c_void_p, c_int, c_int, c_int, c_int, c_int, c_int,
                                            c_float, c_int, c_int, c_void_p, c_size_t, c_void_p]),
+    "pkv_paged_attention_decode_static_ws": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_int,
+                                                     c_void_p, c_int, c_int, c_int, c_int, c_int, c_int,
+                                                     c_float, c_int, c_int, c_void_p]),
     "pkv_get_error": (c_int, [P(c_uint32), c_void_p]),
     "pkv_alloc_create": (c_int, [c_int, P(c_int32), P(c_void_p)]),
     "pkv_alloc_destroy": (None, [c_void_p]),

@@ -347,3 +347,30 @@ class PagedKVCache:
                             torch.from_numpy(np.ascontiguousarray(tables)), torch.from_numpy(lens), max_ctx,
                             q, k_new, v_new, scale=scale, partition=partition, stream=stream)
         return out.clone() if q.device == self.device else out.to(q.device)
+
+
+def paged_attention_decode_static_ws(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
+                                     block_tables: torch.Tensor, context_lens: torch.Tensor,
+                                     max_context_len: int, scale: float, out: Optional[torch.Tensor] = None,
+                                     partition: int = 0, stream=None) -> torch.Tensor:
+    """``paged_attention_decode`` for callers that must not allocate device
+    memory: the split-K scratch is a fixed area the library holds on each
+    device (``_lib.STATIC_WORKSPACE_BYTES``), shared by all calls on that
+    device.  Raises PkvError (invalid argument) when the call needs more
+    scratch than that.  Pass ``out`` to avoid the one allocation this
+    wrapper would otherwise make."""
+    nb, hkv, d = _cache_dims(k_cache, v_cache)
+    if q.dim() != 3 or q.shape[2] != d or q.dtype != k_cache.dtype:
+        raise ValueError("q must be [B, Hq, D] in the cache dtype")
+    B, hq, _ = q.shape
+    if block_tables.dim() != 2 or block_tables.shape[0] != B or context_lens.shape != (B,):
+        raise ValueError("block_tables must be [B, max_blocks] and context_lens [B]")
+    if out is None:
+        out = torch.empty_like(q)
+    check(lib.pkv_paged_attention_decode_static_ws(
+        _dev(out, "out", q.dtype), _dev(q, "q"), _dev(k_cache, "k_cache"), _dev(v_cache, "v_cache"),
+        _dev(block_tables, "block_tables", torch.int32), block_tables.shape[1],
+        _dev(context_lens, "context_lens", torch.int32), int(max_context_len), B, hq, hkv, d, nb,
+        float(scale), int(partition), _DT[k_cache.dtype], _stream(stream, q.device)),
+        "pkv_paged_attention_decode_static_ws")
+    return out

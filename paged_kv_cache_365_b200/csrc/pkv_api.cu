@@ -3,6 +3,7 @@
 // so a rejected call has no side effect (and works without a GPU).
 #include <cmath>
 #include <cstdint>
+#include <mutex>
 #include <unordered_set>
 
 #include "cache_ops.cuh"
@@ -216,6 +217,58 @@ pkv_status pkv_paged_attention_decode(void* out, const void* q, const void* k_ca
     case PKV_BF16: return dispatch_dim<__nv_bfloat16>(a, head_dim, G, st);
   }
   return PKV_EINVAL;
+}
+
+}  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Decode without caller-provided scratch: the split-K workspace lives in a
+// fixed device array owned by the library (see pkv.h for who needs this).
+// ---------------------------------------------------------------------------
+namespace {
+
+static __device__ __align__(256) unsigned char g_static_workspace[PKV_STATIC_WORKSPACE_BYTES];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_static_ws_mutex;
+void* g_static_ws_addr[kMaxDevices] = {};
+
+// Device address of g_static_workspace on the current device.  In host code
+// the array's name only stands in for it, so the address is looked up once
+// per device (with that device current) and kept.
+pkv_status static_workspace_address(void** addr) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return PKV_ECUDA;
+  std::lock_guard<std::mutex> lock(g_static_ws_mutex);
+  if (g_static_ws_addr[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_static_workspace) != cudaSuccess || p == nullptr) return PKV_ECUDA;
+    g_static_ws_addr[dev] = p;
+  }
+  *addr = g_static_ws_addr[dev];
+  return PKV_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+pkv_status pkv_paged_attention_decode_static_ws(void* out, const void* q, const void* k_cache,
+                                                const void* v_cache, const int32_t* block_tables,
+                                                int max_blocks_per_seq, const int32_t* context_lens,
+                                                int max_context_len, int num_seqs, int num_q_heads,
+                                                int num_kv_heads, int head_dim, int num_blocks, float scale,
+                                                int partition_tokens, pkv_dtype dtype, void* stream) {
+  // the size this call needs; larger than the fixed area -> rejected up front
+  const size_t need =
+      pkv_decode_workspace_bytes(num_seqs, num_q_heads, head_dim, max_context_len, partition_tokens);
+  if (need > static_cast<size_t>(PKV_STATIC_WORKSPACE_BYTES)) return PKV_EINVAL;
+  void* ws = nullptr;
+  const pkv_status st = static_workspace_address(&ws);
+  if (st != PKV_OK) return st;
+  return pkv_paged_attention_decode(out, q, k_cache, v_cache, block_tables, max_blocks_per_seq, context_lens,
+                                    max_context_len, num_seqs, num_q_heads, num_kv_heads, head_dim, num_blocks,
+                                    scale, partition_tokens, dtype, ws, PKV_STATIC_WORKSPACE_BYTES, stream);
 }
 
 pkv_status pkv_get_error(uint32_t* flags, void* stream) {
