@@ -6,8 +6,11 @@
 #include <mutex>
 #include <unordered_set>
 
+#include <cudaTypedefs.h>
+
 #include "cache_ops.cuh"
 #include "decode.cuh"
+#include "decode_mma.cuh"
 #include "pkv.h"
 
 namespace pkv {
@@ -66,6 +69,75 @@ pkv_status launch_decode(const pkv::DecodeArgs& a, cudaStream_t st) {
     if (launched() != PKV_OK) return PKV_ECUDA;
   }
   return PKV_OK;
+}
+
+// ---- tensor-core path (fp16 / bf16): tensor-map TMA + mma.sync ----------
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = []() -> PFN_cuTensorMapEncodeTiled_v12000 {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return nullptr;
+    return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }();
+  return fn;
+}
+
+// The pool viewed as a 2-D tensor [num_blocks * Hkv * 16 rows, D columns],
+// loaded in 16 x 64 boxes with the 128-byte swizzle.
+bool encode_cache_map(CUtensorMap* map, const void* base, CUtensorMapDataType dt, int D, long long rows) {
+  PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
+  if (enc == nullptr) return false;
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(rows)};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(D) * 2};
+  const cuuint32_t box[2] = {64, 16};
+  const cuuint32_t elem_strides[2] = {1, 1};
+  return enc(map, dt, 2, const_cast<void*>(base), dims, strides, box, elem_strides, CU_TENSOR_MAP_INTERLEAVE_NONE,
+             CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <typename T, int D, int G>
+pkv_status launch_decode_mma(const pkv::DecodeArgs& a, cudaStream_t st) {
+  constexpr int kStages = 3;
+  using S = pkv::MmaShape<T, D, G, kWarps, kStages>;
+  CUtensorMap mk, mv;
+  const long long rows = static_cast<long long>(a.num_blocks) * a.num_kv_heads * PKV_BLOCK_SIZE;
+  if (!encode_cache_map(&mk, a.k_cache, pkv::Mma<T>::kTmaType, D, rows) ||
+      !encode_cache_map(&mv, a.v_cache, pkv::Mma<T>::kTmaType, D, rows))
+    return PKV_ECUDA;
+  auto kfn = pkv::paged_decode_mma_kernel<T, D, G, kWarps, kStages>;
+  if (cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(S::kSmem)) !=
+      cudaSuccess)
+    return PKV_ECUDA;
+  const dim3 grid(a.num_kv_heads, a.num_seqs, a.num_parts);
+  kfn<<<grid, kWarps * 32, S::kSmem, st>>>(a, mk, mv);
+  if (launched() != PKV_OK) return PKV_ECUDA;
+  if (a.num_parts > 1) {
+    const dim3 g2((a.num_q_heads + 3) / 4, a.num_seqs);
+    pkv::paged_decode_reduce_kernel<T, D><<<g2, 128, 0, st>>>(a);
+    if (launched() != PKV_OK) return PKV_ECUDA;
+  }
+  return PKV_OK;
+}
+
+template <typename T, int D>
+pkv_status dispatch_group_mma(const pkv::DecodeArgs& a, int G, cudaStream_t st) {
+  switch (G) {
+    case 1: return launch_decode_mma<T, D, 1>(a, st);
+    case 2: return launch_decode_mma<T, D, 2>(a, st);
+    case 4: return launch_decode_mma<T, D, 4>(a, st);
+    case 8: return launch_decode_mma<T, D, 8>(a, st);
+  }
+  return PKV_EINVAL;
+}
+
+template <typename T>
+pkv_status dispatch_dim_mma(const pkv::DecodeArgs& a, int D, int G, cudaStream_t st) {
+  if (D == 64) return dispatch_group_mma<T, 64>(a, G, st);
+  if (D == 128) return dispatch_group_mma<T, 128>(a, G, st);
+  return PKV_EINVAL;
 }
 
 template <typename T, int D>
@@ -184,6 +256,8 @@ pkv_status pkv_paged_attention_decode(void* out, const void* q, const void* k_ca
   if (!aligned16(out) || !aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache)) return PKV_EINVAL;
   const long long P = (static_cast<long long>(max_context_len) + part - 1) / part;
   if (P > 65535) return PKV_EINVAL;
+  // tile row coordinates of the 2-D cache view are 32-bit
+  if (static_cast<long long>(num_blocks) * num_kv_heads * PKV_BLOCK_SIZE > 0x7fffffffLL) return PKV_EINVAL;
   const size_t need = workspace_bytes(num_seqs, num_q_heads, head_dim, P);
   if (need > 0 && (workspace == nullptr || workspace_bytes_given < need || !aligned16(workspace)))
     return PKV_EINVAL;
@@ -213,8 +287,8 @@ pkv_status pkv_paged_attention_decode(void* out, const void* q, const void* k_ca
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   switch (dtype) {
     case PKV_F32: return dispatch_dim<float>(a, head_dim, G, st);
-    case PKV_F16: return dispatch_dim<__half>(a, head_dim, G, st);
-    case PKV_BF16: return dispatch_dim<__nv_bfloat16>(a, head_dim, G, st);
+    case PKV_F16: return dispatch_dim_mma<__half>(a, head_dim, G, st);
+    case PKV_BF16: return dispatch_dim_mma<__nv_bfloat16>(a, head_dim, G, st);
   }
   return PKV_EINVAL;
 }
