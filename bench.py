@@ -41,8 +41,8 @@ UNIT = "GB/s"
 FALLBACK_HBM_GBS = 6650.0
 STORAGE = {"f32": 4, "f16": 2, "bf16": 2}
 DTYPE_NAME = {"f32": "fp32", "f16": "fp16", "bf16": "bf16"}
-DECODE_SOURCES = ["paged_kv_cache_365_b200/csrc/decode.cuh", "paged_kv_cache_365_b200/csrc/common.cuh",
-                  "paged_kv_cache_365_b200/csrc/pkv_api.cu"]
+DECODE_SOURCES = ["paged_kv_cache_365_b200/csrc/decode.cuh", "paged_kv_cache_365_b200/csrc/decode_mma.cuh",
+                  "paged_kv_cache_365_b200/csrc/common.cuh", "paged_kv_cache_365_b200/csrc/pkv_api.cu"]
 
 
 # ---------------------------------------------------------------------------
