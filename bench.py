@@ -222,8 +222,18 @@ def run_cuda(args, rank, world, local_rank):
     ws = cache.workspace(pkv.decode_workspace_bytes(B, Hq, D, max_ctx, args.partition))
     out = torch.empty_like(st["q"])
     P = max(1, math.ceil(max_ctx / (args.partition or pkv.DEFAULT_PARTITION)))
-    launches_per_step = 1 + 1 + (1 if n_pairs else 0) + (1 if P > 1 else 0)
     scale = 1.0 / math.sqrt(D)
+    # a batch that shares leading blocks is decoded with the cascade (the
+    # shared prefix is read once per kv-head)
+    pp = pkv.common_prefix_pages(st["host"]["block_tables"], st["host"]["context_lens"])
+    use_cascade = (wl.dtype != "f32" and pp >= pkv.api.CASCADE_MIN_PAGES and B >= pkv.api.CASCADE_MIN_SEQS
+                   and not args.no_cascade)
+    prefix = torch.from_numpy(np.ascontiguousarray(st["host"]["block_tables"][0, :pp])).to(dev) if use_cascade else None
+    if use_cascade:
+        ws = cache.workspace(pkv.decode_prefix_workspace_bytes(B, Hq, D, max_ctx, pp, args.partition))
+        launches_per_step = 1 + (1 if n_pairs else 0) + 3
+    else:
+        launches_per_step = 1 + 1 + (1 if n_pairs else 0) + (1 if P > 1 else 0)
 
     def pre_decode():
         if n_pairs:
@@ -231,8 +241,13 @@ def run_cuda(args, rank, world, local_rank):
         pkv.kv_append(st["k_new"], st["v_new"], cache.k, cache.v, st["slot_mapping"], stream)
 
     def decode():
-        pkv.paged_attention_decode(st["q"], cache.k, cache.v, st["block_tables"], st["context_lens"], max_ctx,
-                                   scale, out=out, workspace=ws, partition=args.partition, stream=stream)
+        if use_cascade:
+            pkv.paged_attention_decode_prefix(st["q"], cache.k, cache.v, st["block_tables"], st["context_lens"],
+                                              max_ctx, prefix, scale, out=out, workspace=ws,
+                                              partition=args.partition, stream=stream)
+        else:
+            pkv.paged_attention_decode(st["q"], cache.k, cache.v, st["block_tables"], st["context_lens"], max_ctx,
+                                       scale, out=out, workspace=ws, partition=args.partition, stream=stream)
 
     def barrier():
         if world > 1:
@@ -267,6 +282,8 @@ def run_cuda(args, rank, world, local_rank):
     # every step, and the output read back every step
     host = {k: st[k].cpu().pin_memory() for k in ("q", "k_new", "v_new", "slot_mapping", "cow_pairs",
                                                     "block_tables", "context_lens")}
+    if use_cascade:
+        host["prefix_blocks"] = prefix.cpu().pin_memory()
     out_host = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
     h2d = sum(t.numel() * t.element_size() for t in host.values())
     d2h = out_host.numel() * out_host.element_size()
@@ -274,7 +291,7 @@ def run_cuda(args, rank, world, local_rank):
     def e2e_step():
         cache.run_step(host["slot_mapping"], host["cow_pairs"], host["block_tables"], host["context_lens"],
                        max_ctx, host["q"], host["k_new"], host["v_new"], out=out_host, scale=scale,
-                       partition=args.partition, stream=stream)
+                       partition=args.partition, stream=stream, prefix_blocks=host.get("prefix_blocks"))
 
     for _ in range(args.warmup):
         e2e_step()
@@ -295,7 +312,7 @@ def run_cuda(args, rank, world, local_rank):
 
     res = dict(wl=wl, K=K, total_ms=total_ms, e2e_ms=e2e_ms, dec_avg_ms=dec_avg_ms,
                launches=launches_per_step * K, h2d=h2d, d2h=d2h, clocks=clocks.summary(), P=P,
-               n_pairs=n_pairs, cache=cache, st=st)
+               n_pairs=n_pairs, cache=cache, st=st, cascade_pages=pp if use_cascade else 0)
     return res
 
 
@@ -442,6 +459,8 @@ def main(argv=None):
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--partition", type=int, default=0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-cascade", action="store_true",
+                    help="decode a shared-prefix batch with the plain paged kernel")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
@@ -492,7 +511,9 @@ def main(argv=None):
                 "h2d_bytes_per_step": r["h2d"], "d2h_bytes_per_step": r["d2h"],
                 "us_per_step": 1e6 * e2e_step_s},
         "gpu_launches": r["launches"],
-        "roofline": {"kernel": "paged_decode (partition + merge kernels)", "bound": "hbm",
+        "cascade_prefix_pages": r["cascade_pages"],
+        "roofline": {"kernel": ("paged_decode cascade (suffix + prefix + merge kernels)" if r["cascade_pages"]
+                                else "paged_decode (partition + merge kernels)"), "bound": "hbm",
                      "achieved": achieved, "peak": peak, "peak_kind": f"{peak_kind} (MEASURED_PEAKS hbm_gbs)"
                      if peak_kind == "measured" else "fallback", "unit": "GB/s", "frac": achieved / peak,
                      "traffic": recorded_traffic(wl.name), "algorithmic_bytes_per_launch": dec_bytes,

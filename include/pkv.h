@@ -164,6 +164,42 @@ pkv_status pkv_paged_attention_decode(void* out, const void* q, const void* k_ca
                                       void* workspace, size_t workspace_bytes, void* stream);
 
 /* ------------------------------------------------------------------------
+ * pkv_paged_attention_decode_prefix -- pkv_paged_attention_decode for a
+ * batch whose sequences share a common prefix of blocks (cascade decode).
+ *
+ * "PagedAttention 与 vLLM 推理加速" §3.2(3): requests with the same system
+ * prompt map the same physical blocks, stored once.  Here those blocks are
+ * also READ once per kv-head: a prefix pass attends the queries of every
+ * sequence to each shared (block, kv-head) tile on the tensor cores, the
+ * paged pass covers each sequence's own suffix, and a merge kernel combines
+ * the two partial results by the log-sum-exp rule.  The output is the same
+ * attention as pkv_paged_attention_decode (up to fp32 rounding order).
+ *
+ * prefix_blocks (device, int32 [prefix_pages]): the shared blocks, in
+ *   logical order.  Sequence b "conforms" when its first prefix_pages table
+ *   entries equal them and context_lens[b] >= 16 * prefix_pages (all prefix
+ *   pages full).  This is checked on the device; a sequence that does not
+ *   conform is decoded over its whole context instead (still correct).
+ * dtype: PKV_F16 or PKV_BF16 (tensor-core path); 1 <= prefix_pages <=
+ *   max_blocks_per_seq; the other arguments are those of
+ *   pkv_paged_attention_decode.
+ * workspace: at least pkv_decode_prefix_workspace_bytes(...) bytes, 16-byte
+ *   aligned, always required; no initialisation needed.
+ * An out-of-range id in prefix_blocks sets PKV_ERR_BLOCK_RANGE and that
+ * page is skipped.
+ * -------------------------------------------------------------------- */
+size_t pkv_decode_prefix_workspace_bytes(int num_seqs, int num_q_heads, int head_dim, int max_context_len,
+                                         int prefix_pages, int partition_tokens);
+pkv_status pkv_paged_attention_decode_prefix(void* out, const void* q, const void* k_cache,
+                                             const void* v_cache, const int32_t* block_tables,
+                                             int max_blocks_per_seq, const int32_t* context_lens,
+                                             int max_context_len, const int32_t* prefix_blocks,
+                                             int prefix_pages, int num_seqs, int num_q_heads,
+                                             int num_kv_heads, int head_dim, int num_blocks, float scale,
+                                             int partition_tokens, pkv_dtype dtype, void* workspace,
+                                             size_t workspace_bytes, void* stream);
+
+/* ------------------------------------------------------------------------
  * pkv_paged_attention_decode_static_ws -- pkv_paged_attention_decode for
  * callers that cannot allocate device memory.
  *

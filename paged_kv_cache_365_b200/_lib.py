@@ -37,6 +37,10 @@ PROTOTYPES = {
     "pkv_paged_attention_decode": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_int,
                                            c_void_p, c_int, c_int, c_int, c_int, c_int, c_int,
                                            c_float, c_int, c_int, c_void_p, c_size_t, c_void_p]),
+    "pkv_decode_prefix_workspace_bytes": (c_size_t, [c_int, c_int, c_int, c_int, c_int, c_int]),
+    "pkv_paged_attention_decode_prefix": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_int,
+                                                  c_void_p, c_int, c_void_p, c_int, c_int, c_int, c_int, c_int,
+                                                  c_int, c_float, c_int, c_int, c_void_p, c_size_t, c_void_p]),
     "pkv_paged_attention_decode_static_ws": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_int,
                                                      c_void_p, c_int, c_int, c_int, c_int, c_int, c_int,
                                                      c_float, c_int, c_int, c_void_p]),

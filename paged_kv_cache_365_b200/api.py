@@ -19,6 +19,10 @@ from ._lib import check, lib
 
 BLOCK_SIZE = 16
 DEFAULT_PARTITION = 512
+# a batch whose sequences share at least this many leading pages (and has at
+# least this many sequences) is decoded with the cascade (prefix read once)
+CASCADE_MIN_PAGES = 8
+CASCADE_MIN_SEQS = 4
 _DT = {torch.float32: 0, torch.float16: 1, torch.bfloat16: 2}
 
 
@@ -129,6 +133,58 @@ def paged_attention_decode(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torc
         _dev(context_lens, "context_lens", torch.int32), int(max_context_len), B, hq, hkv, d, nb,
         float(scale), int(partition), _DT[k_cache.dtype], ws_ptr, ws_len,
         _stream(stream, q.device)), "pkv_paged_attention_decode")
+    return out
+
+
+def decode_prefix_workspace_bytes(num_seqs: int, num_q_heads: int, head_dim: int, max_context_len: int,
+                                  prefix_pages: int, partition: int = 0) -> int:
+    return int(lib.pkv_decode_prefix_workspace_bytes(num_seqs, num_q_heads, head_dim, max_context_len,
+                                                     prefix_pages, partition))
+
+
+def common_prefix_pages(block_tables: np.ndarray, context_lens: np.ndarray) -> int:
+    """Number of leading pages that every sequence of the batch shares (same
+    physical blocks) and fills completely: the prefix the cascade decode
+    can read once.  Host arrays: tables [B, W], lengths [B]."""
+    bt = np.asarray(block_tables)
+    lens = np.asarray(context_lens)
+    if bt.shape[0] < 2:
+        return 0
+    full = int(lens.min()) // BLOCK_SIZE
+    full = min(full, bt.shape[1])
+    if full == 0:
+        return 0
+    same = np.all(bt[:, :full] == bt[0:1, :full], axis=0)
+    return int(full if same.all() else np.argmin(same))
+
+
+def paged_attention_decode_prefix(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
+                                  block_tables: torch.Tensor, context_lens: torch.Tensor, max_context_len: int,
+                                  prefix_blocks: torch.Tensor, scale: float, out: Optional[torch.Tensor] = None,
+                                  workspace: Optional[torch.Tensor] = None, partition: int = 0,
+                                  stream=None) -> torch.Tensor:
+    """Cascade decode for a batch sharing the blocks ``prefix_blocks``
+    (int32 [prefix_pages], device) at the start of every table: the shared
+    pages are read once per kv-head.  Same result as paged_attention_decode."""
+    nb, hkv, d = _cache_dims(k_cache, v_cache)
+    if q.dim() != 3 or q.shape[2] != d or q.dtype != k_cache.dtype:
+        raise ValueError("q must be [B, Hq, D] in the cache dtype")
+    B, hq, _ = q.shape
+    if block_tables.dim() != 2 or block_tables.shape[0] != B or context_lens.shape != (B,):
+        raise ValueError("block_tables must be [B, max_blocks] and context_lens [B]")
+    pp = int(prefix_blocks.numel())
+    if out is None:
+        out = torch.empty_like(q)
+    need = decode_prefix_workspace_bytes(B, hq, d, max_context_len, pp, partition)
+    if workspace is None or workspace.numel() * workspace.element_size() < need:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
+    check(lib.pkv_paged_attention_decode_prefix(
+        _dev(out, "out", q.dtype), _dev(q, "q"), _dev(k_cache, "k_cache"), _dev(v_cache, "v_cache"),
+        _dev(block_tables, "block_tables", torch.int32), block_tables.shape[1],
+        _dev(context_lens, "context_lens", torch.int32), int(max_context_len),
+        _dev(prefix_blocks, "prefix_blocks", torch.int32), pp, B, hq, hkv, d, nb, float(scale), int(partition),
+        _DT[k_cache.dtype], _dev(workspace, "workspace"), workspace.numel() * workspace.element_size(),
+        _stream(stream, q.device)), "pkv_paged_attention_decode_prefix")
     return out
 
 
@@ -300,12 +356,14 @@ class PagedKVCache:
     def run_step(self, slot_mapping: torch.Tensor, cow_pairs: torch.Tensor, block_tables: torch.Tensor,
                  context_lens: torch.Tensor, max_context_len: int, q: torch.Tensor, k_new: torch.Tensor,
                  v_new: torch.Tensor, out: Optional[torch.Tensor] = None, scale: Optional[float] = None,
-                 partition: int = 0, stream=None) -> torch.Tensor:
+                 partition: int = 0, stream=None, prefix_blocks: Optional[torch.Tensor] = None) -> torch.Tensor:
         """Device part of a decode step: copy-on-write copies, append, decode.
 
         Inputs may be host tensors (pinned for asynchronous copies) or
         device tensors.  When ``out`` is a host tensor the result is copied
         into it asynchronously on the stream; synchronise before reading.
+        With ``prefix_blocks`` (int32, the blocks every sequence's table
+        starts with) the cascade decode reads that shared prefix once.
         Returns the device output.
         """
         dev = self.device
@@ -319,14 +377,21 @@ class PagedKVCache:
                 copy_blocks(self.k, self.v, d(cow_pairs), st)
             kv_append(d(k_new), d(v_new), self.k, self.v, d(slot_mapping), st)
             B, hq = q.shape[0], q.shape[1]
-            ws = self.workspace(decode_workspace_bytes(B, hq, self.D, max_context_len, partition))
             if out is not None and out.device == dev:
                 res = out
             else:
                 res = self._out_buffer(q.shape)
-            paged_attention_decode(d(q), self.k, self.v, d(block_tables), d(context_lens), max_context_len,
-                                   (1.0 / math.sqrt(self.D)) if scale is None else scale, out=res,
-                                   workspace=ws, partition=partition, stream=st)
+            sc = (1.0 / math.sqrt(self.D)) if scale is None else scale
+            if prefix_blocks is not None and prefix_blocks.numel() > 0:
+                ws = self.workspace(decode_prefix_workspace_bytes(B, hq, self.D, max_context_len,
+                                                                  prefix_blocks.numel(), partition))
+                paged_attention_decode_prefix(d(q), self.k, self.v, d(block_tables), d(context_lens),
+                                              max_context_len, d(prefix_blocks), sc, out=res, workspace=ws,
+                                              partition=partition, stream=st)
+            else:
+                ws = self.workspace(decode_workspace_bytes(B, hq, self.D, max_context_len, partition))
+                paged_attention_decode(d(q), self.k, self.v, d(block_tables), d(context_lens), max_context_len,
+                                       sc, out=res, workspace=ws, partition=partition, stream=st)
             if out is not None and out.device != dev:
                 out.copy_(res, non_blocking=True)
         return res
@@ -343,9 +408,13 @@ class PagedKVCache:
         """Host plan (allocator) + device step; returns the output on q's device."""
         slots, pairs, tables, lens = self.plan_step(seq_ids)
         max_ctx = int(lens.max()) if len(lens) else 0
+        pp = common_prefix_pages(tables, lens) if self.dtype != torch.float32 else 0
+        prefix = (torch.from_numpy(np.ascontiguousarray(tables[0, :pp]))
+                  if pp >= CASCADE_MIN_PAGES and len(lens) >= CASCADE_MIN_SEQS else None)
         out = self.run_step(torch.from_numpy(slots), torch.from_numpy(np.ascontiguousarray(pairs)),
                             torch.from_numpy(np.ascontiguousarray(tables)), torch.from_numpy(lens), max_ctx,
-                            q, k_new, v_new, scale=scale, partition=partition, stream=stream)
+                            q, k_new, v_new, scale=scale, partition=partition, stream=stream,
+                            prefix_blocks=prefix)
         return out.clone() if q.device == self.device else out.to(q.device)
 
 

@@ -57,6 +57,14 @@ struct DecodeArgs {
   int partition;      // tokens per partition, multiple of 16
   int num_parts;      // P = ceil(max_context_len / partition), >= 1
   float qk_scale;     // scale * log2(e)
+  // shared-prefix (cascade) mode; prefix_blocks == nullptr otherwise
+  const int32_t* prefix_blocks;  // [prefix_pages] blocks every sequence is expected to start with
+  int prefix_pages;
+  int chunk_pages;     // prefix pages per prefix-pass CTA
+  int num_chunks;      // ceil(prefix_pages / chunk_pages)
+  float* wp_o;         // [B][Hq][num_chunks][D] prefix partial outputs
+  float2* wp_ml;       // [B][Hq][num_chunks] (max, sum)
+  int* conform;        // [B]: 1 when sequence b starts with the prefix
 };
 
 constexpr unsigned kFull = 0xffffffffu;

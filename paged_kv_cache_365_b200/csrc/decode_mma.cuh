@@ -157,17 +157,32 @@ __global__ void __launch_bounds__(NWARPS * 32)
     if (threadIdx.x == 0 && kvh == 0 && part == 0) raise_error(PKV_ERR_CONTEXT_RANGE);
     ctx = ctx < 0 ? 0 : a.max_ctx;
   }
-  const int nparts = (ctx + a.partition - 1) / a.partition;
+  // shared-prefix mode: a sequence that starts with the prefix blocks only
+  // covers its suffix here (the prefix pass covered the rest); one that
+  // does not covers its whole context
+  const bool cascade = a.prefix_blocks != nullptr;
+  int tok_begin = 0;
+  if (cascade) {
+    int same = 1;
+    for (int j = threadIdx.x; j < a.prefix_pages; j += NWARPS * 32)
+      if (a.block_tables[static_cast<long long>(b) * a.bt_stride + j] != a.prefix_blocks[j]) same = 0;
+    const bool conforming = __syncthreads_and(same) && ctx >= a.prefix_pages * kBlockSize;
+    if (conforming) tok_begin = a.prefix_pages * kBlockSize;
+    if (threadIdx.x == 0 && kvh == 0 && part == 0) a.conform[b] = conforming ? 1 : 0;
+  }
+  const int span = ctx - tok_begin;
+  const int nparts = (span + a.partition - 1) / a.partition;
   if (part >= (nparts > 0 ? nparts : 1)) return;
 
   const int h0 = kvh * G;
   T* out = reinterpret_cast<T*>(a.out) + (static_cast<size_t>(b) * a.num_q_heads + h0) * D;
-  if (ctx == 0) {
-    for (int i = threadIdx.x; i < G * D; i += NWARPS * 32) out[i] = Fmt<T>::from_f32(0.f);
+  if (span == 0) {
+    if (tok_begin == 0)  // nothing to attend to at all
+      for (int i = threadIdx.x; i < G * D; i += NWARPS * 32) out[i] = Fmt<T>::from_f32(0.f);
     return;
   }
 
-  const int tok0 = part * a.partition;
+  const int tok0 = tok_begin + part * a.partition;
   const int tok1 = min(ctx, tok0 + a.partition);
   const int pg0 = tok0 / kBlockSize;
   const int nblk = (tok1 - tok0 + kBlockSize - 1) / kBlockSize;
@@ -389,7 +404,7 @@ __global__ void __launch_bounds__(NWARPS * 32)
       num = fmaf(sc, r[g * D + d], num);
       den = fmaf(sc, r[G * D + G + g], den);
     }
-    if (nparts == 1) {
+    if (nparts == 1 && !cascade) {
       out[idx] = Fmt<T>::from_f32(num / den);
     } else {
       const size_t row = (static_cast<size_t>(b) * a.num_q_heads + h0 + g) * a.num_parts + part;

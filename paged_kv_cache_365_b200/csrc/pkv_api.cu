@@ -11,6 +11,7 @@
 #include "cache_ops.cuh"
 #include "decode.cuh"
 #include "decode_mma.cuh"
+#include "decode_prefix.cuh"
 #include "pkv.h"
 
 namespace pkv {
@@ -140,6 +141,123 @@ pkv_status dispatch_dim_mma(const pkv::DecodeArgs& a, int D, int G, cudaStream_t
   return PKV_EINVAL;
 }
 
+// ---- shared-prefix (cascade) path ------------------------------------------
+constexpr int kPrefixChunkPages = 16;  // prefix pages per prefix-pass CTA
+constexpr int kPrefixWarps = 8;        // 16 queries per warp
+constexpr int kPrefixStages = 4;
+
+struct PrefixLayout {
+  long long parts, chunks;
+  size_t off_so, off_sml, off_po, off_pml, off_conform, total;
+};
+
+// Workspace of the cascade: suffix partials [B][Hq][P][D] + (max, sum)
+// [B][Hq][P], prefix partials [B][Hq][C][D] + [B][Hq][C], flags [B].
+PrefixLayout prefix_layout(long long B, long long Hq, long long D, long long max_ctx, long long prefix_pages,
+                           long long part) {
+  auto up16 = [](size_t x) { return (x + 15) / 16 * 16; };
+  PrefixLayout L;
+  L.parts = (max_ctx + part - 1) / part;
+  if (L.parts < 1) L.parts = 1;
+  L.chunks = (prefix_pages + kPrefixChunkPages - 1) / kPrefixChunkPages;
+  L.off_so = 0;
+  L.off_sml = up16(L.off_so + static_cast<size_t>(B * Hq * L.parts * D * 4));
+  L.off_po = up16(L.off_sml + static_cast<size_t>(B * Hq * L.parts * 8));
+  L.off_pml = up16(L.off_po + static_cast<size_t>(B * Hq * L.chunks * D * 4));
+  L.off_conform = up16(L.off_pml + static_cast<size_t>(B * Hq * L.chunks * 8));
+  L.total = up16(L.off_conform + static_cast<size_t>(B * 4));
+  return L;
+}
+
+template <typename T, int D, int G>
+pkv_status launch_decode_prefix(const pkv::DecodeArgs& a, cudaStream_t st) {
+  constexpr int kStages = 3;
+  using S = pkv::MmaShape<T, D, G, kWarps, kStages>;
+  using SP = pkv::PrefixShape<T, D, kPrefixWarps, kPrefixStages>;
+  CUtensorMap mk, mv;
+  const long long rows = static_cast<long long>(a.num_blocks) * a.num_kv_heads * PKV_BLOCK_SIZE;
+  if (!encode_cache_map(&mk, a.k_cache, pkv::Mma<T>::kTmaType, D, rows) ||
+      !encode_cache_map(&mv, a.v_cache, pkv::Mma<T>::kTmaType, D, rows))
+    return PKV_ECUDA;
+  // (1) each sequence's suffix (whole context when it does not share the prefix)
+  auto kfn = pkv::paged_decode_mma_kernel<T, D, G, kWarps, kStages>;
+  if (cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(S::kSmem)) !=
+      cudaSuccess)
+    return PKV_ECUDA;
+  kfn<<<dim3(a.num_kv_heads, a.num_seqs, a.num_parts), kWarps * 32, S::kSmem, st>>>(a, mk, mv);
+  if (launched() != PKV_OK) return PKV_ECUDA;
+  // (2) the shared prefix, once per kv-head, for every sequence's queries
+  auto pfn = pkv::paged_decode_prefix_kernel<T, D, G, kPrefixWarps, kPrefixStages>;
+  if (cudaFuncSetAttribute(pfn, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(SP::kSmem)) !=
+      cudaSuccess)
+    return PKV_ECUDA;
+  const int qgroups = (a.num_seqs * G + kPrefixWarps * 16 - 1) / (kPrefixWarps * 16);
+  pfn<<<dim3(a.num_kv_heads, a.num_chunks, qgroups), kPrefixWarps * 32, SP::kSmem, st>>>(a, mk, mv);
+  if (launched() != PKV_OK) return PKV_ECUDA;
+  // (3) merge prefix chunks and suffix partitions
+  pkv::paged_decode_prefix_merge_kernel<T, D><<<dim3((a.num_q_heads + 3) / 4, a.num_seqs), 128, 0, st>>>(a);
+  return launched();
+}
+
+template <typename T, int D>
+pkv_status dispatch_group_prefix(const pkv::DecodeArgs& a, int G, cudaStream_t st) {
+  switch (G) {
+    case 1: return launch_decode_prefix<T, D, 1>(a, st);
+    case 2: return launch_decode_prefix<T, D, 2>(a, st);
+    case 4: return launch_decode_prefix<T, D, 4>(a, st);
+    case 8: return launch_decode_prefix<T, D, 8>(a, st);
+  }
+  return PKV_EINVAL;
+}
+
+template <typename T>
+pkv_status dispatch_dim_prefix(const pkv::DecodeArgs& a, int D, int G, cudaStream_t st) {
+  if (D == 64) return dispatch_group_prefix<T, 64>(a, G, st);
+  if (D == 128) return dispatch_group_prefix<T, 128>(a, G, st);
+  return PKV_EINVAL;
+}
+
+// Checks shared by the decode entry points; fills `a` (everything but the
+// workspace) and the partition count.  No CUDA call.
+pkv_status prepare_decode(void* out, const void* q, const void* k_cache, const void* v_cache,
+                          const int32_t* block_tables, int max_blocks_per_seq, const int32_t* context_lens,
+                          int max_context_len, int num_seqs, int num_q_heads, int num_kv_heads, int head_dim,
+                          int num_blocks, float scale, int partition_tokens, pkv_dtype dtype, pkv::DecodeArgs* a,
+                          long long* P_out) {
+  const int part = resolve_partition(partition_tokens);
+  if (dtype_bytes(dtype) == 0 || part < 0 || num_seqs < 0 || num_seqs > 65535 || num_kv_heads <= 0 ||
+      num_kv_heads > 65535 || num_q_heads <= 0 || num_q_heads % num_kv_heads != 0 ||
+      !group_ok(num_q_heads / num_kv_heads) || !head_dim_ok(head_dim) || num_blocks <= 0 ||
+      max_context_len < 0 || max_blocks_per_seq <= 0 ||
+      static_cast<long long>(max_context_len) > static_cast<long long>(max_blocks_per_seq) * PKV_BLOCK_SIZE ||
+      !std::isfinite(scale))
+    return PKV_EINVAL;
+  if (num_seqs == 0) return PKV_OK;
+  if (!out || !q || !k_cache || !v_cache || !block_tables || !context_lens) return PKV_EINVAL;
+  if (!aligned16(out) || !aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache)) return PKV_EINVAL;
+  const long long P = (static_cast<long long>(max_context_len) + part - 1) / part;
+  if (P > 65535) return PKV_EINVAL;
+  // tile row coordinates of the 2-D cache view are 32-bit
+  if (static_cast<long long>(num_blocks) * num_kv_heads * PKV_BLOCK_SIZE > 0x7fffffffLL) return PKV_EINVAL;
+  a->out = out;
+  a->q = q;
+  a->k_cache = static_cast<const unsigned char*>(k_cache);
+  a->v_cache = static_cast<const unsigned char*>(v_cache);
+  a->block_tables = block_tables;
+  a->context_lens = context_lens;
+  a->bt_stride = max_blocks_per_seq;
+  a->max_ctx = max_context_len;
+  a->num_seqs = num_seqs;
+  a->num_q_heads = num_q_heads;
+  a->num_kv_heads = num_kv_heads;
+  a->num_blocks = num_blocks;
+  a->partition = part;
+  a->num_parts = P > 1 ? static_cast<int>(P) : 1;
+  a->qk_scale = scale * kLog2e;
+  *P_out = P;
+  return PKV_OK;
+}
+
 template <typename T, int D>
 pkv_status dispatch_group(const pkv::DecodeArgs& a, int G, cudaStream_t st) {
   switch (G) {
@@ -243,45 +361,19 @@ pkv_status pkv_paged_attention_decode(void* out, const void* q, const void* k_ca
                                       int num_q_heads, int num_kv_heads, int head_dim, int num_blocks, float scale,
                                       int partition_tokens, pkv_dtype dtype, void* workspace,
                                       size_t workspace_bytes_given, void* stream) {
-  const int part = resolve_partition(partition_tokens);
-  if (dtype_bytes(dtype) == 0 || part < 0 || num_seqs < 0 || num_seqs > 65535 || num_kv_heads <= 0 ||
-      num_kv_heads > 65535 || num_q_heads <= 0 || num_q_heads % num_kv_heads != 0 ||
-      !group_ok(num_q_heads / num_kv_heads) || !head_dim_ok(head_dim) || num_blocks <= 0 ||
-      max_context_len < 0 || max_blocks_per_seq <= 0 ||
-      static_cast<long long>(max_context_len) > static_cast<long long>(max_blocks_per_seq) * PKV_BLOCK_SIZE ||
-      !std::isfinite(scale))
-    return PKV_EINVAL;
-  if (num_seqs == 0) return PKV_OK;
-  if (!out || !q || !k_cache || !v_cache || !block_tables || !context_lens) return PKV_EINVAL;
-  if (!aligned16(out) || !aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache)) return PKV_EINVAL;
-  const long long P = (static_cast<long long>(max_context_len) + part - 1) / part;
-  if (P > 65535) return PKV_EINVAL;
-  // tile row coordinates of the 2-D cache view are 32-bit
-  if (static_cast<long long>(num_blocks) * num_kv_heads * PKV_BLOCK_SIZE > 0x7fffffffLL) return PKV_EINVAL;
+  pkv::DecodeArgs a{};
+  long long P = 0;
+  const pkv_status st0 = prepare_decode(out, q, k_cache, v_cache, block_tables, max_blocks_per_seq, context_lens,
+                                        max_context_len, num_seqs, num_q_heads, num_kv_heads, head_dim, num_blocks,
+                                        scale, partition_tokens, dtype, &a, &P);
+  if (st0 != PKV_OK || num_seqs == 0) return st0;
   const size_t need = workspace_bytes(num_seqs, num_q_heads, head_dim, P);
   if (need > 0 && (workspace == nullptr || workspace_bytes_given < need || !aligned16(workspace)))
     return PKV_EINVAL;
-
-  pkv::DecodeArgs a;
-  a.out = out;
-  a.q = q;
-  a.k_cache = static_cast<const unsigned char*>(k_cache);
-  a.v_cache = static_cast<const unsigned char*>(v_cache);
-  a.block_tables = block_tables;
-  a.context_lens = context_lens;
   a.ws_o = static_cast<float*>(need ? workspace : nullptr);
   a.ws_ml = need ? reinterpret_cast<float2*>(static_cast<float*>(workspace) +
                                               static_cast<size_t>(num_seqs) * num_q_heads * P * head_dim)
                  : nullptr;
-  a.bt_stride = max_blocks_per_seq;
-  a.max_ctx = max_context_len;
-  a.num_seqs = num_seqs;
-  a.num_q_heads = num_q_heads;
-  a.num_kv_heads = num_kv_heads;
-  a.num_blocks = num_blocks;
-  a.partition = part;
-  a.num_parts = P > 1 ? static_cast<int>(P) : 1;
-  a.qk_scale = scale * kLog2e;
 
   const int G = num_q_heads / num_kv_heads;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
@@ -291,6 +383,51 @@ pkv_status pkv_paged_attention_decode(void* out, const void* q, const void* k_ca
     case PKV_BF16: return dispatch_dim_mma<__nv_bfloat16>(a, head_dim, G, st);
   }
   return PKV_EINVAL;
+}
+
+size_t pkv_decode_prefix_workspace_bytes(int num_seqs, int num_q_heads, int head_dim, int max_context_len,
+                                         int prefix_pages, int partition_tokens) {
+  const int part = resolve_partition(partition_tokens);
+  if (part < 0 || num_seqs < 0 || num_q_heads <= 0 || !head_dim_ok(head_dim) || max_context_len < 0 ||
+      prefix_pages <= 0)
+    return 0;
+  return prefix_layout(num_seqs, num_q_heads, head_dim, max_context_len, prefix_pages, part).total;
+}
+
+pkv_status pkv_paged_attention_decode_prefix(void* out, const void* q, const void* k_cache, const void* v_cache,
+                                             const int32_t* block_tables, int max_blocks_per_seq,
+                                             const int32_t* context_lens, int max_context_len,
+                                             const int32_t* prefix_blocks, int prefix_pages, int num_seqs,
+                                             int num_q_heads, int num_kv_heads, int head_dim, int num_blocks,
+                                             float scale, int partition_tokens, pkv_dtype dtype, void* workspace,
+                                             size_t workspace_bytes_given, void* stream) {
+  if (dtype != PKV_F16 && dtype != PKV_BF16) return PKV_EINVAL;  // tensor-core path only
+  if (prefix_pages <= 0 || prefix_pages > max_blocks_per_seq) return PKV_EINVAL;
+  pkv::DecodeArgs a{};
+  long long P = 0;
+  const pkv_status st0 = prepare_decode(out, q, k_cache, v_cache, block_tables, max_blocks_per_seq, context_lens,
+                                        max_context_len, num_seqs, num_q_heads, num_kv_heads, head_dim, num_blocks,
+                                        scale, partition_tokens, dtype, &a, &P);
+  if (st0 != PKV_OK || num_seqs == 0) return st0;
+  if (prefix_blocks == nullptr) return PKV_EINVAL;
+  const PrefixLayout L = prefix_layout(num_seqs, num_q_heads, head_dim, max_context_len, prefix_pages, a.partition);
+  if (workspace == nullptr || workspace_bytes_given < L.total || !aligned16(workspace)) return PKV_EINVAL;
+  unsigned char* ws = static_cast<unsigned char*>(workspace);
+  a.num_parts = static_cast<int>(L.parts);
+  a.ws_o = reinterpret_cast<float*>(ws + L.off_so);
+  a.ws_ml = reinterpret_cast<float2*>(ws + L.off_sml);
+  a.wp_o = reinterpret_cast<float*>(ws + L.off_po);
+  a.wp_ml = reinterpret_cast<float2*>(ws + L.off_pml);
+  a.conform = reinterpret_cast<int*>(ws + L.off_conform);
+  a.prefix_blocks = prefix_blocks;
+  a.prefix_pages = prefix_pages;
+  a.chunk_pages = kPrefixChunkPages;
+  a.num_chunks = static_cast<int>(L.chunks);
+
+  const int G = num_q_heads / num_kv_heads;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (dtype == PKV_F16) return dispatch_dim_prefix<__half>(a, head_dim, G, st);
+  return dispatch_dim_prefix<__nv_bfloat16>(a, head_dim, G, st);
 }
 
 }  // extern "C"

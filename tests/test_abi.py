@@ -126,3 +126,18 @@ def test_kv_cache_bytes_matches_page_example():
     n = kv_cache_bytes(g["layers"], g["heads"], g["head_dim"], g["seq_len"], g["dtype_bytes"])
     assert n == g["expected_bytes"]
     assert abs(n / 1e9 - g["page_figure_gb"]) / g["page_figure_gb"] < g["page_figure_rel_tol"]
+
+
+def test_prefix_workspace_and_rejections(lib):
+    up = lambda x: (x + 15) // 16 * 16
+    B, Hq, D, ctx, pp = 4, 8, 128, 1100, 20
+    P, C = 3, 2  # ceil(1100/512), ceil(20/16)
+    want = up(up(up(up(up(B * Hq * P * D * 4) + B * Hq * P * 8) + B * Hq * C * D * 4) + B * Hq * C * 8) + B * 4)
+    assert lib.pkv_decode_prefix_workspace_bytes(B, Hq, D, ctx, pp, 0) == want
+    assert lib.pkv_decode_prefix_workspace_bytes(B, Hq, D, ctx, 0, 0) == 0
+    args = [FAKE, FAKE, FAKE, FAKE, FAKE, 100, FAKE, 1100, FAKE, 20, 4, 8, 2, 128, 64, ctypes.c_float(0.1), 0,
+            1, FAKE, 1 << 30, None]
+    for idx, bad in ((17, 0), (9, 0), (9, 101), (8, None), (18, None), (19, 16)):
+        a = list(args)
+        a[idx] = bad
+        assert lib.pkv_paged_attention_decode_prefix(*a) == 1, (idx, bad)

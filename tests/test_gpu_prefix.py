@@ -1,0 +1,133 @@
+"""GPU parity of the shared-prefix (cascade) decode against the fp64 oracle.
+
+The cascade reads the shared prefix once per kv-head for all sequences, then
+each sequence's suffix, and merges; the oracle is the plain definition over
+each sequence's whole context.  Sequences that do not start with the given
+prefix (a relabelled block, a context shorter than the prefix) must still
+come out right: the kernel checks each table on the device and decodes such
+a sequence over its whole context.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads
+
+pytestmark = pytest.mark.gpu
+
+TOL = {"f16": 2e-3, "bf16": 1e-2}
+
+
+def prepared(wl):
+    import paged_kv_cache_365_b200 as pkv
+    from paged_kv_cache_365_b200.replay import build_step
+    vals = workloads.draw_values(wl)
+    st = build_step(wl, vals, "cuda")
+    c = st["cache"]
+    pkv.copy_blocks(c.k, c.v, st["cow_pairs"])
+    pkv.kv_append(st["k_new"], st["v_new"], c.k, c.v, st["slot_mapping"])
+    ref = oracle.replay(wl, vals)
+    return vals, st, ref
+
+
+def cascade(st, wl, bt=None, cl=None, prefix_pages=None):
+    import paged_kv_cache_365_b200 as pkv
+    c = st["cache"]
+    tables = st["host"]["block_tables"]
+    lens = st["host"]["context_lens"]
+    pp = pkv.common_prefix_pages(tables, lens) if prefix_pages is None else prefix_pages
+    assert pp > 0
+    prefix = torch.from_numpy(np.ascontiguousarray(tables[0, :pp])).cuda()
+    out = pkv.paged_attention_decode_prefix(st["q"], c.k, c.v, st["block_tables"] if bt is None else bt,
+                                            st["context_lens"] if cl is None else cl, st["max_context_len"],
+                                            prefix, wl.scale)
+    torch.cuda.synchronize()
+    assert pkv.get_error() == 0
+    return out.float().cpu().numpy().astype(np.float64), pp
+
+
+CASES = [
+    workloads.prefix13b(seed=31, B=12, prefix_tokens=256, suffix_range=(1, 100), Hq=8, Hkv=8, D=128,
+                        dtype="f16", name="pfx_f16_mha"),
+    workloads.prefix13b(seed=32, B=20, prefix_tokens=512, suffix_range=(0, 700), Hq=16, Hkv=2, D=128,
+                        dtype="bf16", name="pfx_bf16_gqa8"),
+    workloads.prefix13b(seed=33, B=9, prefix_tokens=160, suffix_range=(3, 40), Hq=8, Hkv=2, D=64,
+                        dtype="bf16", name="pfx_bf16_d64"),
+    workloads.prefix13b(seed=34, B=140, prefix_tokens=64, suffix_range=(1, 30), Hq=2, Hkv=2, D=128,
+                        dtype="f16", name="pfx_f16_many_seqs"),
+]
+
+
+@pytest.mark.parametrize("wl", CASES, ids=lambda w: w.name)
+def test_cascade_matches_oracle(wl):
+    vals, st, ref = prepared(wl)
+    got, pp = cascade(st, wl)
+    assert pp * 16 == {"pfx_f16_mha": 256, "pfx_bf16_gqa8": 512, "pfx_bf16_d64": 160,
+                       "pfx_f16_many_seqs": 64}[wl.name]
+    want = oracle.paged_decode(vals["q"], ref["cache"].k, ref["cache"].v, ref["block_tables"],
+                               ref["context_lens"], wl.scale, wl.dtype)
+    assert np.isfinite(got).all()
+    assert np.abs(got - want).max() <= TOL[wl.dtype]
+
+
+def test_cascade_full_size_prefix_workload():
+    wl = workloads.named("prefix13b", 0)
+    vals, st, ref = prepared(wl)
+    got, pp = cascade(st, wl)
+    assert pp == 64
+    seqs = list(range(0, wl.B, 9)) + [wl.B - 1]
+    want = oracle.paged_decode(vals["q"], ref["cache"].k, ref["cache"].v, ref["block_tables"],
+                               ref["context_lens"], wl.scale, wl.dtype, seqs=seqs)
+    assert np.abs(got[seqs] - want[seqs]).max() <= TOL[wl.dtype]
+
+
+def test_non_conforming_sequences_fall_back_to_their_whole_context():
+    import paged_kv_cache_365_b200 as pkv
+    wl = CASES[0]
+    vals, st, ref = prepared(wl)
+    c = st["cache"]
+    tables = st["host"]["block_tables"].copy()
+    lens = st["host"]["context_lens"].copy()
+    pp = pkv.common_prefix_pages(tables, lens)
+    # sequence 3: its third prefix page moved to a private copy (same data)
+    free = sorted(set(range(wl.num_blocks)) - set(int(x) for x in tables[:, :].ravel() if x < wl.num_blocks))
+    src, dst = int(tables[3, 2]), int(free[0])
+    pkv.copy_blocks(c.k, c.v, torch.tensor([[src, dst]], dtype=torch.int32, device="cuda"))
+    tables[3, 2] = dst
+    # sequence 5: a context shorter than the prefix
+    lens[5] = 37
+    bt = torch.from_numpy(tables).cuda()
+    cl = torch.from_numpy(lens).cuda()
+    got, _ = cascade(st, wl, bt=bt, cl=cl, prefix_pages=pp)
+    ref_tables = ref["block_tables"].copy()
+    ref_tables[3, 2] = dst
+    ref["cache"].copy_blocks([(src, dst)])
+    want = oracle.paged_decode(vals["q"], ref["cache"].k, ref["cache"].v, ref_tables, lens, wl.scale, wl.dtype)
+    assert np.abs(got - want).max() <= TOL[wl.dtype]
+
+
+def test_sequence_with_empty_suffix():
+    """A sequence whose context is exactly the prefix: all of it comes from
+    the prefix pass."""
+    wl = CASES[0]
+    vals, st, ref = prepared(wl)
+    lens = st["host"]["context_lens"].copy()
+    import paged_kv_cache_365_b200 as pkv
+    pp = pkv.common_prefix_pages(st["host"]["block_tables"], lens)
+    lens[0] = pp * 16
+    got, _ = cascade(st, wl, cl=torch.from_numpy(lens).cuda(), prefix_pages=pp)
+    want = oracle.paged_decode(vals["q"], ref["cache"].k, ref["cache"].v, ref["block_tables"], lens, wl.scale,
+                               wl.dtype)
+    assert np.abs(got - want).max() <= TOL[wl.dtype]
+
+
+def test_cascade_agrees_with_plain_decode():
+    import paged_kv_cache_365_b200 as pkv
+    wl = CASES[1]
+    vals, st, ref = prepared(wl)
+    got, _ = cascade(st, wl)
+    c = st["cache"]
+    plain = pkv.paged_attention_decode(st["q"], c.k, c.v, st["block_tables"], st["context_lens"],
+                                       st["max_context_len"], wl.scale).float().cpu().numpy()
+    assert np.abs(got - plain).max() <= TOL[wl.dtype]
