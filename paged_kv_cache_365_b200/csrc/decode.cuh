@@ -62,6 +62,8 @@ struct DecodeArgs {
   int prefix_pages;
   int chunk_pages;     // prefix pages per prefix-pass CTA
   int num_chunks;      // ceil(prefix_pages / chunk_pages)
+  int num_qgroups;     // prefix-role CTAs per (kv-head, chunk): ceil(B * G / 8)
+  int suffix_z;        // partitions in flight per sequence (suffix-role CTAs per sequence)
   float* wp_o;         // [B][Hq][num_chunks][D] prefix partial outputs
   float2* wp_ml;       // [B][Hq][num_chunks] (max, sum)
   int* conform;        // [B]: 1 when sequence b starts with the prefix
@@ -412,52 +414,77 @@ __global__ void __launch_bounds__(NWARPS * 32)
   }
 }
 
-// Merge the partitions of every (sequence, query head) whose context spans
-// more than one partition: out = sum_p 2^(m_p - M) o_p / sum_p 2^(m_p - M) l_p
-// with M = max_p m_p, partitions taken in order.  One warp per head.
-template <typename T, int D>
-__global__ void __launch_bounds__(128) paged_decode_reduce_kernel(const DecodeArgs a) {
+// Merge n partial results (running max m_p in log2 units, running sum l_p,
+// unnormalised output o_p) of one (sequence, query head):
+//   out = sum_p 2^(m_p - M) o_p / sum_p 2^(m_p - M) l_p,   M = max_p m_p.
+// One CTA of kMergeWarps warps: warp w accumulates partials w, w + 8, ... in
+// order (independent loads, unrolled), then the warps' sums are added in a
+// fixed order.  `ml(p)` / `op(p)` give partial p's (m, l) and output row.
+constexpr int kMergeWarps = 8;
+
+template <typename T, int D, typename ML, typename OP>
+__device__ __forceinline__ void merge_partials(int n, ML ml, OP op, T* out) {
   constexpr int kEpl = D / 32;
+  __shared__ float red_o[kMergeWarps][D];
+  __shared__ float red_den[kMergeWarps];
+  __shared__ float red_max[kMergeWarps];
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int h = blockIdx.x * 4 + warp;
-  const int b = blockIdx.y;
-  if (h >= a.num_q_heads) return;
-  int ctx = a.context_lens[b];
-  ctx = ctx < 0 ? 0 : (ctx > a.max_ctx ? a.max_ctx : ctx);
-  const int nparts = (ctx + a.partition - 1) / a.partition;
-  if (nparts <= 1) return;
-
-  const size_t row0 = (static_cast<size_t>(b) * a.num_q_heads + h) * a.num_parts;
+  if (n <= 0) {
+    for (int d = threadIdx.x; d < D; d += kMergeWarps * 32) out[d] = Fmt<T>::from_f32(0.f);
+    return;
+  }
   float M = -INFINITY;
-  for (int p = lane; p < nparts; p += 32) M = fmaxf(M, a.ws_ml[row0 + p].x);
+  for (int p = threadIdx.x; p < n; p += kMergeWarps * 32) M = fmaxf(M, ml(p).x);
   M = warp_max(M);
+  if (lane == 0) red_max[warp] = M;
+  __syncthreads();
+  M = red_max[0];
+#pragma unroll
+  for (int w = 1; w < kMergeWarps; ++w) M = fmaxf(M, red_max[w]);
 
   float acc[kEpl];
 #pragma unroll
   for (int e = 0; e < kEpl; ++e) acc[e] = 0.f;
   float den = 0.f;
 #pragma unroll 4
-  for (int p = 0; p < nparts; ++p) {
-    const float2 ml = a.ws_ml[row0 + p];
-    const float w = exp2f(ml.x - M);
-    den = fmaf(w, ml.y, den);
-    const float* op = a.ws_o + (row0 + p) * D + lane * kEpl;
-    if constexpr (kEpl == 4) {
-      const float4 t = *reinterpret_cast<const float4*>(op);
-      acc[0] = fmaf(w, t.x, acc[0]);
-      acc[1] = fmaf(w, t.y, acc[1]);
-      acc[2] = fmaf(w, t.z, acc[2]);
-      acc[3] = fmaf(w, t.w, acc[3]);
-    } else {
-      const float2 t = *reinterpret_cast<const float2*>(op);
-      acc[0] = fmaf(w, t.x, acc[0]);
-      acc[1] = fmaf(w, t.y, acc[1]);
-    }
-  }
-  T* out = reinterpret_cast<T*>(a.out) + (static_cast<size_t>(b) * a.num_q_heads + h) * D + lane * kEpl;
+  for (int p = warp; p < n; p += kMergeWarps) {
+    const float2 v = ml(p);
+    const float w = exp2f(v.x - M);
+    den = fmaf(w, v.y, den);
+    const float* o = op(p) + lane * kEpl;
 #pragma unroll
-  for (int e = 0; e < kEpl; ++e) out[e] = Fmt<T>::from_f32(acc[e] / den);
+    for (int e = 0; e < kEpl; ++e) acc[e] = fmaf(w, o[e], acc[e]);
+  }
+#pragma unroll
+  for (int e = 0; e < kEpl; ++e) red_o[warp][lane * kEpl + e] = acc[e];
+  if (lane == 0) red_den[warp] = den;
+  __syncthreads();
+  for (int d = threadIdx.x; d < D; d += kMergeWarps * 32) {
+    float num = 0.f, dd = 0.f;
+#pragma unroll
+    for (int w = 0; w < kMergeWarps; ++w) {
+      num += red_o[w][d];
+      dd += red_den[w];
+    }
+    out[d] = Fmt<T>::from_f32(num / dd);
+  }
+}
+
+// Split-K merge: per (query head h = blockIdx.x, sequence b = blockIdx.y)
+// whose context spans more than one partition, the partitions in order.
+template <typename T, int D>
+__global__ void __launch_bounds__(kMergeWarps * 32) paged_decode_reduce_kernel(const DecodeArgs a) {
+  const int h = blockIdx.x;
+  const int b = blockIdx.y;
+  int ctx = a.context_lens[b];
+  ctx = ctx < 0 ? 0 : (ctx > a.max_ctx ? a.max_ctx : ctx);
+  const int nparts = (ctx + a.partition - 1) / a.partition;
+  if (nparts <= 1) return;  // written by the partition kernel
+  const size_t row0 = (static_cast<size_t>(b) * a.num_q_heads + h) * a.num_parts;
+  T* out = reinterpret_cast<T*>(a.out) + (static_cast<size_t>(b) * a.num_q_heads + h) * D;
+  merge_partials<T, D>(
+      nparts, [&](int p) { return a.ws_ml[row0 + p]; }, [&](int p) { return a.ws_o + (row0 + p) * D; }, out);
 }
 
 }  // namespace pkv

@@ -131,100 +131,57 @@ struct MmaShape {
   static constexpr size_t kSmemStages = size_t(NWARPS) * kWarpStageBytes;
   static constexpr size_t kSmemBars = size_t(NWARPS) * NSTAGE * 8;
   static constexpr size_t kSmem = 1024 /* alignment slack */ + kSmemStages + kSmemBars;
+  // warp record: o[8][D], m[8], l[8] (8 query columns, the MMA's N)
+  static constexpr int kRecM = 8 * D, kRecL = 8 * D + 8;
+  // block-table entries a lane holds: a warp's pages of a 2048-token partition
+  static constexpr int kTab = (128 + 32 * NWARPS - 1) / (32 * NWARPS);
   static_assert(D % 64 == 0, "a tile row is a whole number of 128-byte boxes");
   static_assert(G >= 1 && G <= 8, "the group is the MMA's N = 8 dimension");
-  static_assert(size_t(G) * (D + 2) * sizeof(float) <= size_t(kWarpStageBytes),
+  static_assert(size_t(8) * (D + 2) * sizeof(float) <= size_t(kWarpStageBytes),
                 "a warp's merge record must fit in its own stages");
   static_assert(kStage % 1024 == 0, "swizzled boxes need 1024-byte alignment");
 };
 
-template <typename T, int D, int G, int NWARPS, int NSTAGE>
-__global__ void __launch_bounds__(NWARPS * 32)
-    paged_decode_mma_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tmap_k,
-                            const __grid_constant__ CUtensorMap tmap_v) {
-  using S = MmaShape<T, D, G, NWARPS, NSTAGE>;
+// Prefix role, one warp: 16 queries of kv-head kvh (query i = sequence i / G,
+// head i % G) over pages [pg0, pg0 + nblk) of the shared prefix, queries as
+// the MMA's M dimension:
+//   S[16 q x 16 tok] = Q[16 x D] . K^T     (A = Q in registers, B = K via ldmatrix)
+//   O[16 q x D]     += P[16 x 16] . V      (A = P straight from the S fragments,
+//                                           B = V via ldmatrix.trans; hi + lo P)
+// Every warp of the CTA walks all pages with its own stages (the tiles come
+// from L2 after the first warp's read) and writes its queries' partial
+// results directly: warps have disjoint queries, nothing to merge.
+template <typename T, int D, int G, int NSTAGE>
+__device__ __forceinline__ bool prefix_warp(const DecodeArgs& a, const CUtensorMap* tmap_k,
+                                            const CUtensorMap* tmap_v, int kvh, int q0, int chunk, int pg0,
+                                            int nblk, uint32_t stage0, uint32_t bar0, uint32_t& phase_bits,
+                                            int lane) {
   using M = Mma<T>;
-  const int kvh = blockIdx.x;
-  const int b = blockIdx.y;
-  const int part = blockIdx.z;
-  const int warp = threadIdx.x >> 5;
-  const int lane = threadIdx.x & 31;
-  const int g8 = lane >> 2;  // fragment row group
-  const int t4 = lane & 3;   // thread in group
-
-  int ctx = a.context_lens[b];
-  if (ctx < 0 || ctx > a.max_ctx) {
-    if (threadIdx.x == 0 && kvh == 0 && part == 0) raise_error(PKV_ERR_CONTEXT_RANGE);
-    ctx = ctx < 0 ? 0 : a.max_ctx;
-  }
-  // shared-prefix mode: a sequence that starts with the prefix blocks only
-  // covers its suffix here (the prefix pass covered the rest); one that
-  // does not covers its whole context
-  const bool cascade = a.prefix_blocks != nullptr;
-  int tok_begin = 0;
-  if (cascade) {
-    int same = 1;
-    for (int j = threadIdx.x; j < a.prefix_pages; j += NWARPS * 32)
-      if (a.block_tables[static_cast<long long>(b) * a.bt_stride + j] != a.prefix_blocks[j]) same = 0;
-    const bool conforming = __syncthreads_and(same) && ctx >= a.prefix_pages * kBlockSize;
-    if (conforming) tok_begin = a.prefix_pages * kBlockSize;
-    if (threadIdx.x == 0 && kvh == 0 && part == 0) a.conform[b] = conforming ? 1 : 0;
-  }
-  const int span = ctx - tok_begin;
-  const int nparts = (span + a.partition - 1) / a.partition;
-  if (part >= (nparts > 0 ? nparts : 1)) return;
-
-  const int h0 = kvh * G;
-  T* out = reinterpret_cast<T*>(a.out) + (static_cast<size_t>(b) * a.num_q_heads + h0) * D;
-  if (span == 0) {
-    if (tok_begin == 0)  // nothing to attend to at all
-      for (int i = threadIdx.x; i < G * D; i += NWARPS * 32) out[i] = Fmt<T>::from_f32(0.f);
-    return;
-  }
-
-  const int tok0 = tok_begin + part * a.partition;
-  const int tok1 = min(ctx, tok0 + a.partition);
-  const int pg0 = tok0 / kBlockSize;
-  const int nblk = (tok1 - tok0 + kBlockSize - 1) / kBlockSize;
-  const int my_n = warp < nblk ? (nblk - warp + NWARPS - 1) / NWARPS : 0;
-
-  extern __shared__ unsigned char smem_raw[];
-  // swizzled boxes want 1024-byte aligned destinations
-  const uint32_t raw_addr = smem_addr(smem_raw);
-  const uint32_t pad = ((raw_addr + 1023u) & ~1023u) - raw_addr;
-  unsigned char* smem = smem_raw + pad;
-  unsigned char* my_stages = smem + static_cast<size_t>(warp) * S::kWarpStageBytes;
-  const uint32_t stage0 = smem_addr(my_stages);
-  const uint32_t bar0 = smem_addr(smem + S::kSmemStages) + warp * NSTAGE * 8;
-
-  // lane j: physical block of this warp's j-th page (page warp + j*NWARPS)
+  constexpr int kTile = kBlockSize * D * 2, kStage = 2 * kTile, kKSteps = D / 16, kNTiles = D / 8;
+  const int g8 = lane >> 2, t4 = lane & 3, lm = lane >> 3, lr = lane & 7;
+  const int nq = a.num_seqs * G;
+  // lane j: block of page pg0 + j (nblk <= 32)
   int my_phys = -1;
-  if (lane < my_n) {
-    const int e = a.block_tables[static_cast<long long>(b) * a.bt_stride + pg0 + warp + lane * NWARPS];
+  if (lane < nblk) {
+    const int e = a.prefix_blocks[pg0 + lane];
     if (e >= 0 && e < a.num_blocks)
       my_phys = e;
     else
       raise_error(PKV_ERR_BLOCK_RANGE);
   }
-  if (lane == 0) {
-    for (int s = 0; s < NSTAGE; ++s) mbar_init(bar0 + 8 * s, 1);
-    fence_barrier_init();
-  }
-  __syncwarp();
-
   auto issue = [&](int i) {
     const int phys = __shfl_sync(kFull, my_phys, i & 31);
-    if (lane == 0 && i < my_n) {
+    if (lane == 0 && i < nblk) {
       const uint32_t bar = bar0 + 8 * (i % NSTAGE);
       if (phys >= 0) {
-        const uint32_t dst = stage0 + (i % NSTAGE) * S::kStage;
+        const uint32_t dst = stage0 + (i % NSTAGE) * kStage;
         const int y = (phys * a.num_kv_heads + kvh) * kBlockSize;
         fence_proxy_async_smem();
-        mbar_arrive_expect_tx(bar, S::kStage);
+        mbar_arrive_expect_tx(bar, kStage);
 #pragma unroll
-        for (int bx = 0; bx < S::kBoxes; ++bx) {
-          tma_load_2d(dst + bx * 2048, &tmap_k, bx * 64, y, bar);
-          tma_load_2d(dst + S::kTile + bx * 2048, &tmap_v, bx * 64, y, bar);
+        for (int bx = 0; bx < D / 64; ++bx) {
+          tma_load_2d(dst + bx * 2048, tmap_k, bx * 64, y, bar);
+          tma_load_2d(dst + kTile + bx * 2048, tmap_v, bx * 64, y, bar);
         }
       } else {
         mbar_arrive(bar);
@@ -234,33 +191,36 @@ __global__ void __launch_bounds__(NWARPS * 32)
 #pragma unroll
   for (int i = 0; i < NSTAGE; ++i) issue(i);
 
-  // B fragments of Q^T (k = d, n = head): head g8 of the group, zero past G
-  uint32_t qb[S::kKSteps][2];
+  // A fragments of the 16 queries (rows past the batch are zero)
+  uint32_t qa[kKSteps][4];
   {
-    const T* qp = reinterpret_cast<const T*>(a.q) + (static_cast<size_t>(b) * a.num_q_heads + h0 + g8) * D;
+    const int ra = q0 + g8, rb = q0 + g8 + 8;
+    const T* pa = ra < nq ? reinterpret_cast<const T*>(a.q) +
+                                (static_cast<size_t>(ra / G) * a.num_q_heads + kvh * G + ra % G) * D
+                          : nullptr;
+    const T* pb = rb < nq ? reinterpret_cast<const T*>(a.q) +
+                                (static_cast<size_t>(rb / G) * a.num_q_heads + kvh * G + rb % G) * D
+                          : nullptr;
 #pragma unroll
-    for (int ks = 0; ks < S::kKSteps; ++ks) {
-      qb[ks][0] = g8 < G ? *reinterpret_cast<const uint32_t*>(qp + ks * 16 + 2 * t4) : 0u;
-      qb[ks][1] = g8 < G ? *reinterpret_cast<const uint32_t*>(qp + ks * 16 + 8 + 2 * t4) : 0u;
+    for (int ks = 0; ks < kKSteps; ++ks) {
+      const int d = ks * 16 + 2 * t4;
+      qa[ks][0] = pa ? *reinterpret_cast<const uint32_t*>(pa + d) : 0u;
+      qa[ks][1] = pb ? *reinterpret_cast<const uint32_t*>(pb + d) : 0u;
+      qa[ks][2] = pa ? *reinterpret_cast<const uint32_t*>(pa + d + 8) : 0u;
+      qa[ks][3] = pb ? *reinterpret_cast<const uint32_t*>(pb + d + 8) : 0u;
     }
   }
-
-  // O^T accumulator fragments: o[i] = rows d = 16 i + g8 (+8), heads 2 t4 (+1)
-  float o[S::kKSteps][4];
+  float o[kNTiles][4];
 #pragma unroll
-  for (int i = 0; i < S::kKSteps; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
-  float m0 = -INFINITY, m1 = -INFINITY;  // running max of heads 2 t4, 2 t4 + 1 (log2 units)
-  float l0 = 0.f, l1 = 0.f;              // this lane's share of their running sums
-  uint32_t phase_bits = 0;
+  for (int j = 0; j < kNTiles; ++j) o[j][0] = o[j][1] = o[j][2] = o[j][3] = 0.f;
+  float mA = -INFINITY, mB = -INFINITY;  // rows g8, g8 + 8
+  float lA = 0.f, lB = 0.f;
+
   int consumed = 0;
-
-  // per-lane ldmatrix row/chunk selectors
-  const int lm = lane >> 3;   // which 8x8 matrix this lane addresses
-  const int lr = lane & 7;    // row within it
-
-  for (int i = 0; i < my_n; ++i) {
+  bool ok = true;
+  for (int i = 0; i < nblk; ++i) {
     const int s = i % NSTAGE;
-    bool ok = mbar_wait_bounded(bar0 + 8 * s, (phase_bits >> s) & 1u);
+    ok = mbar_wait_bounded(bar0 + 8 * s, (phase_bits >> s) & 1u);
     phase_bits ^= 1u << s;
     ok = __all_sync(kFull, ok);
     if (!ok) {
@@ -268,149 +228,461 @@ __global__ void __launch_bounds__(NWARPS * 32)
       break;
     }
     consumed = i + 1;
-    const int phys = __shfl_sync(kFull, my_phys, i);
-    if (phys >= 0) {
-      const int page_tok = tok0 + (warp + i * NWARPS) * kBlockSize;
-      const int nvalid = min(kBlockSize, tok1 - page_tok);
-      const uint32_t kt = stage0 + s * S::kStage;
-      const uint32_t vt = kt + S::kTile;
-
-      // (1) S^T = K . Q^T
-      float sc[4] = {0.f, 0.f, 0.f, 0.f};
+    if (__shfl_sync(kFull, my_phys, i) >= 0) {
+      const uint32_t kt = stage0 + s * kStage;
+      const uint32_t vt = kt + kTile;
+      float sc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
       {
-        const int row = lr + ((lm & 1) << 3);
+        const int row = lr + ((lm >> 1) << 3);  // token
 #pragma unroll
-        for (int ks = 0; ks < S::kKSteps; ++ks) {
-          uint32_t a0, a1, a2, a3;
-          ldsm_x4(kt + swz(row, 2 * ks + (lm >> 1)), a0, a1, a2, a3);
-          M::run(sc, a0, a1, a2, a3, qb[ks][0], qb[ks][1]);
+        for (int ks = 0; ks < kKSteps; ++ks) {
+          uint32_t b0, b1, b2, b3;
+          ldsm_x4(kt + swz(row, 2 * ks + (lm & 1)), b0, b1, b2, b3);
+          M::run(sc[0], qa[ks][0], qa[ks][1], qa[ks][2], qa[ks][3], b0, b1);
+          M::run(sc[1], qa[ks][0], qa[ks][1], qa[ks][2], qa[ks][3], b2, b3);
         }
       }
-      // (2) scale, mask the tail, online softmax per head
-      const bool v_lo = g8 < nvalid, v_hi = g8 + 8 < nvalid;
-      const float x0 = v_lo ? sc[0] * a.qk_scale : -INFINITY;  // token g8,   head 2 t4
-      const float x1 = v_lo ? sc[1] * a.qk_scale : -INFINITY;  // token g8,   head 2 t4 + 1
-      const float x2 = v_hi ? sc[2] * a.qk_scale : -INFINITY;  // token g8+8, head 2 t4
-      const float x3 = v_hi ? sc[3] * a.qk_scale : -INFINITY;  // token g8+8, head 2 t4 + 1
-      float mx0 = fmaxf(x0, x2), mx1 = fmaxf(x1, x3);
+      float x[2][4];
 #pragma unroll
-      for (int msk = 4; msk <= 16; msk <<= 1) {
-        mx0 = fmaxf(mx0, __shfl_xor_sync(kFull, mx0, msk));
-        mx1 = fmaxf(mx1, __shfl_xor_sync(kFull, mx1, msk));
-      }
-      const float n0 = fmaxf(m0, mx0), n1 = fmaxf(m1, mx1);
-      const float al0 = exp2f(m0 - n0), al1 = exp2f(m1 - n1);
-      m0 = n0;
-      m1 = n1;
-      const float p0 = exp2f(x0 - n0), p1 = exp2f(x1 - n1), p2 = exp2f(x2 - n0), p3 = exp2f(x3 - n1);
-      l0 = fmaf(l0, al0, p0 + p2);
-      l1 = fmaf(l1, al1, p1 + p3);
+      for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
-      for (int mt = 0; mt < S::kKSteps; ++mt) {
-        o[mt][0] *= al0;
-        o[mt][1] *= al1;
-        o[mt][2] *= al0;
-        o[mt][3] *= al1;
+        for (int e = 0; e < 4; ++e) x[nt][e] = sc[nt][e] * a.qk_scale;
+      float mxA = fmaxf(fmaxf(x[0][0], x[0][1]), fmaxf(x[1][0], x[1][1]));
+      float mxB = fmaxf(fmaxf(x[0][2], x[0][3]), fmaxf(x[1][2], x[1][3]));
+#pragma unroll
+      for (int msk = 1; msk <= 2; msk <<= 1) {
+        mxA = fmaxf(mxA, __shfl_xor_sync(kFull, mxA, msk));
+        mxB = fmaxf(mxB, __shfl_xor_sync(kFull, mxB, msk));
       }
-      // (3) P^T as B fragments, split into hi + lo 16-bit parts
-      const uint32_t top_hi = M::pack(p0, p1), bot_hi = M::pack(p2, p3);
-      const float2 th = M::unpack(top_hi), bh = M::unpack(bot_hi);
-      const uint32_t top_lo = M::pack(p0 - th.x, p1 - th.y), bot_lo = M::pack(p2 - bh.x, p3 - bh.y);
-      const uint32_t pb0 = movm_t(top_hi), pb1 = movm_t(bot_hi);
-      const uint32_t pl0 = movm_t(top_lo), pl1 = movm_t(bot_lo);
-      // V^T fragment halves of tokens past the context are zeroed
-      uint32_t keep_lo = 0xffffffffu, keep_hi = 0xffffffffu;
-      if (nvalid < kBlockSize) {
-        keep_lo = (2 * t4 < nvalid ? 0x0000ffffu : 0u) | (2 * t4 + 1 < nvalid ? 0xffff0000u : 0u);
-        keep_hi = (2 * t4 + 8 < nvalid ? 0x0000ffffu : 0u) | (2 * t4 + 9 < nvalid ? 0xffff0000u : 0u);
+      const float nA = fmaxf(mA, mxA), nB = fmaxf(mB, mxB);
+      const float alA = exp2f(mA - nA), alB = exp2f(mB - nB);
+      mA = nA;
+      mB = nB;
+      float p[2][4];
+#pragma unroll
+      for (int nt = 0; nt < 2; ++nt) {
+        p[nt][0] = exp2f(x[nt][0] - nA);
+        p[nt][1] = exp2f(x[nt][1] - nA);
+        p[nt][2] = exp2f(x[nt][2] - nB);
+        p[nt][3] = exp2f(x[nt][3] - nB);
       }
-      // (4) O^T += V^T . P^T
+      lA = fmaf(lA, alA, p[0][0] + p[0][1] + p[1][0] + p[1][1]);
+      lB = fmaf(lB, alB, p[0][2] + p[0][3] + p[1][2] + p[1][3]);
+      if (__any_sync(kFull, alA != 1.f || alB != 1.f)) {
+#pragma unroll
+        for (int j = 0; j < kNTiles; ++j) {
+          o[j][0] *= alA;
+          o[j][1] *= alA;
+          o[j][2] *= alB;
+          o[j][3] *= alB;
+        }
+      }
+      uint32_t ph[4], pl[4];
       {
-        const int row = lr + ((lm >> 1) << 3);
+        const float v[4][2] = {{p[0][0], p[0][1]}, {p[0][2], p[0][3]}, {p[1][0], p[1][1]}, {p[1][2], p[1][3]}};
 #pragma unroll
-        for (int mt = 0; mt < S::kKSteps; ++mt) {
-          uint32_t a0, a1, a2, a3;
-          ldsm_x4_t(vt + swz(row, 2 * mt + (lm & 1)), a0, a1, a2, a3);
-          a0 &= keep_lo;
-          a1 &= keep_lo;
-          a2 &= keep_hi;
-          a3 &= keep_hi;
-          M::run(o[mt], a0, a1, a2, a3, pb0, pb1);
-          M::run(o[mt], a0, a1, a2, a3, pl0, pl1);
+        for (int r = 0; r < 4; ++r) {
+          ph[r] = M::pack(v[r][0], v[r][1]);
+          const float2 hv = M::unpack(ph[r]);
+          pl[r] = M::pack(v[r][0] - hv.x, v[r][1] - hv.y);
+        }
+      }
+      {
+        const int row = lr + ((lm & 1) << 3);  // token
+#pragma unroll
+        for (int j = 0; j < kNTiles; j += 2) {
+          uint32_t b0, b1, b2, b3;
+          ldsm_x4_t(vt + swz(row, j + (lm >> 1)), b0, b1, b2, b3);
+          M::run(o[j], ph[0], ph[1], ph[2], ph[3], b0, b1);
+          M::run(o[j], pl[0], pl[1], pl[2], pl[3], b0, b1);
+          M::run(o[j + 1], ph[0], ph[1], ph[2], ph[3], b2, b3);
+          M::run(o[j + 1], pl[0], pl[1], pl[2], pl[3], b2, b3);
         }
       }
     }
     __syncwarp();
     issue(i + NSTAGE);
   }
-
-  // after a give-up, wait (bounded) for the copies still in flight
-  if (consumed < my_n) {
-    const int last = min(my_n, consumed + NSTAGE);
+  if (consumed < nblk) {  // after a give-up: wait (bounded) for copies in flight
+    const int last = min(nblk, consumed + NSTAGE);
     for (int i = consumed + 1; i < last; ++i) {
       const int s = i % NSTAGE;
       mbar_wait_bounded(bar0 + 8 * s, (phase_bits >> s) & 1u);
       phase_bits ^= 1u << s;
     }
+    return false;
   }
+#pragma unroll
+  for (int msk = 1; msk <= 2; msk <<= 1) {
+    lA += __shfl_xor_sync(kFull, lA, msk);
+    lB += __shfl_xor_sync(kFull, lB, msk);
+  }
+  const int rows[2] = {q0 + g8, q0 + g8 + 8};
+  const float ms[2] = {mA, mB}, ls[2] = {lA, lB};
+#pragma unroll
+  for (int r = 0; r < 2; ++r) {
+    const int qi = rows[r];
+    if (qi >= nq) continue;
+    const size_t slot = (static_cast<size_t>(qi / G) * a.num_q_heads + kvh * G + qi % G) * a.num_chunks + chunk;
+    float* dst = a.wp_o + slot * D;
+#pragma unroll
+    for (int j = 0; j < kNTiles; ++j)
+      *reinterpret_cast<float2*>(dst + 8 * j + 2 * t4) = make_float2(o[j][2 * r], o[j][2 * r + 1]);
+    if (t4 == 0) a.wp_ml[slot] = make_float2(ms[r], ls[r]);
+  }
+  return true;
+}
 
-  // running sums over the lanes of each head (same t4)
-#pragma unroll
-  for (int msk = 4; msk <= 16; msk <<= 1) {
-    l0 += __shfl_xor_sync(kFull, l0, msk);
-    l1 += __shfl_xor_sync(kFull, l1, msk);
-  }
+// One CTA of 4 warps does one of two jobs:
+//  * sequence role: the G query heads of (sequence b, kv-head) over the
+//    partitions part, part + Z, ... of the sequence's context (in a cascade
+//    launch: of its suffix, when its table starts with the shared prefix);
+//  * prefix role (cascade launch only): 16 queries per warp, 64 per CTA, of
+//    one kv-head, taken from consecutive sequences (query i = sequence
+//    i / G, head i % G), over one chunk of the shared prefix pages
+//    (prefix_warp).  The prefix tiles are read from L2 by every query
+//    group; HBM sees them once.
+// Grid: plain (Hkv, B, Z); cascade (Hkv, QG * NC + B * Z) with the prefix
+// CTAs first, so they start early and overlap the suffix streaming.
+template <typename T, int D, int G, int NWARPS, int NSTAGE, bool kCascade>
+__global__ void __launch_bounds__(NWARPS * 32)
+    paged_decode_mma_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tmap_k,
+                            const __grid_constant__ CUtensorMap tmap_v) {
+  using S = MmaShape<T, D, G, NWARPS, NSTAGE>;
+  using M = Mma<T>;
+  const int kvh = blockIdx.x;
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int g8 = lane >> 2;  // fragment row group (also: this lane's query column)
+  const int t4 = lane & 3;   // thread in group
+  constexpr bool cascade = kCascade;  // launched by the shared-prefix entry point
 
-  // warp record [o: G x D][m: G][l: G] in the warp's own (drained) stages
-  float* rec = reinterpret_cast<float*>(my_stages);
-  const int ha = 2 * t4, hb = 2 * t4 + 1;
-#pragma unroll
-  for (int mt = 0; mt < S::kKSteps; ++mt) {
-    const int d0 = 16 * mt + g8;
-    if (ha < G) {
-      rec[ha * D + d0] = o[mt][0];
-      rec[ha * D + d0 + 8] = o[mt][2];
-    }
-    if (hb < G) {
-      rec[hb * D + d0] = o[mt][1];
-      rec[hb * D + d0 + 8] = o[mt][3];
-    }
-  }
-  if (g8 == 0) {
-    if (ha < G) {
-      rec[G * D + ha] = m0;
-      rec[G * D + G + ha] = l0;
-    }
-    if (hb < G) {
-      rec[G * D + hb] = m1;
-      rec[G * D + G + hb] = l1;
-    }
-  }
-  __syncthreads();
-
-  // merge the warps in a fixed order
-  for (int idx = threadIdx.x; idx < G * D; idx += NWARPS * 32) {
-    const int g = idx / D;
-    const int d = idx % D;
-    float Mx = -INFINITY;
-#pragma unroll
-    for (int w = 0; w < NWARPS; ++w)
-      Mx = fmaxf(Mx, reinterpret_cast<const float*>(smem + w * S::kWarpStageBytes)[G * D + g]);
-    float num = 0.f, den = 0.f;
-#pragma unroll
-    for (int w = 0; w < NWARPS; ++w) {
-      const float* r = reinterpret_cast<const float*>(smem + w * S::kWarpStageBytes);
-      const float sc = exp2f(r[G * D + g] - Mx);
-      num = fmaf(sc, r[g * D + d], num);
-      den = fmaf(sc, r[G * D + G + g], den);
-    }
-    if (nparts == 1 && !cascade) {
-      out[idx] = Fmt<T>::from_f32(num / den);
+  // ---- role, work range, query columns ------------------------------------
+  bool prefix_role = false;
+  int b = 0, part = 0, stride = gridDim.z, chunk = 0, qg = 0;
+  if (cascade) {
+    const int npre = a.num_qgroups * a.num_chunks;
+    if (static_cast<int>(blockIdx.y) < npre) {
+      prefix_role = true;
+      qg = blockIdx.y / a.num_chunks;
+      chunk = blockIdx.y % a.num_chunks;
     } else {
-      const size_t row = (static_cast<size_t>(b) * a.num_q_heads + h0 + g) * a.num_parts + part;
-      a.ws_o[row * D + d] = num;
-      if (d == 0) a.ws_ml[row] = make_float2(Mx, den);
+      const int y = blockIdx.y - npre;
+      b = y % a.num_seqs;
+      part = y / a.num_seqs;
     }
+    stride = a.suffix_z;
+  } else {
+    b = blockIdx.y;
+    part = blockIdx.z;
+  }
+
+  int ctx = 0, tok_begin = 0, nparts = 0, span = 0;
+  if (!prefix_role) {
+    // A sequence whose table starts with the prefix blocks covers only its
+    // suffix (the prefix role covers the rest); one that does not covers
+    // its whole context.  The check's loads go out with the length's.
+    int same = 1;
+    if (cascade)
+      for (int j = threadIdx.x; j < a.prefix_pages; j += NWARPS * 32)
+        if (a.block_tables[static_cast<long long>(b) * a.bt_stride + j] != a.prefix_blocks[j]) same = 0;
+    ctx = a.context_lens[b];
+    if (ctx < 0 || ctx > a.max_ctx) {
+      if (threadIdx.x == 0 && kvh == 0 && part == 0) raise_error(PKV_ERR_CONTEXT_RANGE);
+      ctx = ctx < 0 ? 0 : a.max_ctx;
+    }
+    if (cascade) {
+      const bool conforming = __syncthreads_and(same) && ctx >= a.prefix_pages * kBlockSize;
+      if (conforming) tok_begin = a.prefix_pages * kBlockSize;
+      if (threadIdx.x == 0 && kvh == 0 && part == 0) a.conform[b] = conforming ? 1 : 0;
+    }
+    span = ctx - tok_begin;
+    nparts = (span + a.partition - 1) / a.partition;
+    if (part >= (nparts > 0 ? nparts : 1)) return;
+    if (span == 0) {
+      if (tok_begin == 0) {  // nothing to attend to at all
+        T* out = reinterpret_cast<T*>(a.out) + (static_cast<size_t>(b) * a.num_q_heads + kvh * G) * D;
+        for (int i = threadIdx.x; i < G * D; i += NWARPS * 32) out[i] = Fmt<T>::from_f32(0.f);
+      }
+      return;
+    }
+  } else {
+    nparts = 1;
+  }
+  // query columns of this CTA: the G heads of sequence b
+  const int ncol = G;
+  auto col_valid = [&](int n) { return n < ncol; };
+  auto col_row = [&](int n) -> size_t {  // row of q / out for query column n
+    return static_cast<size_t>(b) * a.num_q_heads + kvh * G + n;
+  };
+
+  extern __shared__ unsigned char smem_raw[];
+  // swizzled boxes want 1024-byte aligned destinations
+  const uint32_t raw_addr = smem_addr(smem_raw);
+  const uint32_t pad = ((raw_addr + 1023u) & ~1023u) - raw_addr;
+  unsigned char* smem = smem_raw + pad;
+  unsigned char* my_stages = smem + static_cast<size_t>(warp) * S::kWarpStageBytes;
+  const uint32_t stage0 = smem_addr(my_stages);
+  const uint32_t bar0 = smem_addr(smem + S::kSmemStages) + warp * NSTAGE * 8;
+  if (lane == 0) {
+    for (int s = 0; s < NSTAGE; ++s) mbar_init(bar0 + 8 * s, 1);
+    fence_barrier_init();
+  }
+  __syncwarp();
+
+  uint32_t phase_bits = 0;  // barrier phase parity per stage (carries across partitions)
+  if (cascade && prefix_role) {
+    // warp w: queries (qg * NWARPS + w) * 16 .. + 15 over the chunk's pages
+    const int pg0 = chunk * a.chunk_pages;
+    const int nblk = min(a.prefix_pages - pg0, a.chunk_pages);
+    prefix_warp<T, D, G, NSTAGE>(a, &tmap_k, &tmap_v, kvh, (qg * NWARPS + warp) * 16, chunk, pg0, nblk, stage0,
+                                 bar0, phase_bits, lane);
+    return;
+  }
+
+  // B fragments of Q^T (k = d, n = query column g8), zero past the columns
+  uint32_t qb[S::kKSteps][2];
+  {
+    const bool ok = col_valid(g8);
+    const T* qp = reinterpret_cast<const T*>(a.q) + (ok ? col_row(g8) : 0) * D;
+#pragma unroll
+    for (int ks = 0; ks < S::kKSteps; ++ks) {
+      qb[ks][0] = ok ? *reinterpret_cast<const uint32_t*>(qp + ks * 16 + 2 * t4) : 0u;
+      qb[ks][1] = ok ? *reinterpret_cast<const uint32_t*>(qp + ks * 16 + 8 + 2 * t4) : 0u;
+    }
+  }
+  // per-lane ldmatrix row/chunk selectors
+  const int lm = lane >> 3;  // which 8x8 matrix this lane addresses
+  const int lr = lane & 7;   // row within it
+  bool timed_out = false;
+
+  for (int pidx = part; pidx < nparts; pidx += stride) {
+    // pages of this work item: a partition of the sequence, or a prefix chunk
+    const int tok0 = tok_begin + pidx * a.partition;
+    const int tok1 = min(ctx, tok0 + a.partition);
+    const int pg0 = tok0 / kBlockSize;
+    const int nblk = (tok1 - tok0 + kBlockSize - 1) / kBlockSize;
+    const int my_n = warp < nblk ? (nblk - warp + NWARPS - 1) / NWARPS : 0;  // <= 32 * S::kTab
+
+    // lane j: physical blocks of this warp's pages j, j + 32, ... (page
+    // warp + j*NWARPS of the partition, and so on)
+    int my_phys[S::kTab];
+#pragma unroll
+    for (int h = 0; h < S::kTab; ++h) {
+      my_phys[h] = -1;
+      const int j = lane + 32 * h;
+      if (j < my_n) {
+        const int pg = pg0 + warp + j * NWARPS;
+        const int e = a.block_tables[static_cast<long long>(b) * a.bt_stride + pg];
+        if (e >= 0 && e < a.num_blocks)
+          my_phys[h] = e;
+        else
+          raise_error(PKV_ERR_BLOCK_RANGE);
+      }
+    }
+    auto phys_of = [&](int i) {  // block of this warp's page i (all lanes)
+      int r = -1;
+#pragma unroll
+      for (int h = 0; h < S::kTab; ++h) {
+        const int v = __shfl_sync(kFull, my_phys[h], i & 31);
+        if ((i >> 5) == h) r = v;
+      }
+      return r;
+    };
+
+    auto issue = [&](int i) {
+      const int phys = phys_of(i);
+      if (lane == 0 && i < my_n) {
+        const uint32_t bar = bar0 + 8 * (i % NSTAGE);
+        if (phys >= 0) {
+          const uint32_t dst = stage0 + (i % NSTAGE) * S::kStage;
+          const int y = (phys * a.num_kv_heads + kvh) * kBlockSize;
+          fence_proxy_async_smem();
+          mbar_arrive_expect_tx(bar, S::kStage);
+#pragma unroll
+          for (int bx = 0; bx < S::kBoxes; ++bx) {
+            tma_load_2d(dst + bx * 2048, &tmap_k, bx * 64, y, bar);
+            tma_load_2d(dst + S::kTile + bx * 2048, &tmap_v, bx * 64, y, bar);
+          }
+        } else {
+          mbar_arrive(bar);
+        }
+      }
+    };
+#pragma unroll
+    for (int i = 0; i < NSTAGE; ++i) issue(i);
+
+    // O^T accumulator fragments: o[i] = rows d = 16 i + g8 (+8), columns 2 t4 (+1)
+    float o[S::kKSteps][4];
+#pragma unroll
+    for (int i = 0; i < S::kKSteps; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
+    float m0 = -INFINITY, m1 = -INFINITY;  // running max of columns 2 t4, 2 t4 + 1 (log2 units)
+    float l0 = 0.f, l1 = 0.f;              // this lane's share of their running sums
+    int consumed = 0;
+
+    for (int i = 0; i < my_n; ++i) {
+      const int s = i % NSTAGE;
+      bool ok = mbar_wait_bounded(bar0 + 8 * s, (phase_bits >> s) & 1u);
+      phase_bits ^= 1u << s;
+      ok = __all_sync(kFull, ok);
+      if (!ok) {
+        if (lane == 0) raise_error(PKV_ERR_TIMEOUT);
+        timed_out = true;
+        break;
+      }
+      consumed = i + 1;
+      const int phys = phys_of(i);
+      if (phys >= 0) {
+        const int page_tok = tok0 + (warp + i * NWARPS) * kBlockSize;
+        const int nvalid = min(kBlockSize, tok1 - page_tok);
+        const uint32_t kt = stage0 + s * S::kStage;
+        const uint32_t vt = kt + S::kTile;
+
+        // (1) S^T = K . Q^T
+        float sc[4] = {0.f, 0.f, 0.f, 0.f};
+        {
+          const int row = lr + ((lm & 1) << 3);
+#pragma unroll
+          for (int ks = 0; ks < S::kKSteps; ++ks) {
+            uint32_t a0, a1, a2, a3;
+            ldsm_x4(kt + swz(row, 2 * ks + (lm >> 1)), a0, a1, a2, a3);
+            M::run(sc, a0, a1, a2, a3, qb[ks][0], qb[ks][1]);
+          }
+        }
+        // (2) scale, mask the tail, online softmax per query column
+        const bool v_lo = g8 < nvalid, v_hi = g8 + 8 < nvalid;
+        const float x0 = v_lo ? sc[0] * a.qk_scale : -INFINITY;  // token g8,   column 2 t4
+        const float x1 = v_lo ? sc[1] * a.qk_scale : -INFINITY;  // token g8,   column 2 t4 + 1
+        const float x2 = v_hi ? sc[2] * a.qk_scale : -INFINITY;  // token g8+8, column 2 t4
+        const float x3 = v_hi ? sc[3] * a.qk_scale : -INFINITY;  // token g8+8, column 2 t4 + 1
+        float mx0 = fmaxf(x0, x2), mx1 = fmaxf(x1, x3);
+#pragma unroll
+        for (int msk = 4; msk <= 16; msk <<= 1) {
+          mx0 = fmaxf(mx0, __shfl_xor_sync(kFull, mx0, msk));
+          mx1 = fmaxf(mx1, __shfl_xor_sync(kFull, mx1, msk));
+        }
+        const float n0 = fmaxf(m0, mx0), n1 = fmaxf(m1, mx1);
+        const float al0 = exp2f(m0 - n0), al1 = exp2f(m1 - n1);
+        m0 = n0;
+        m1 = n1;
+        const float p0 = exp2f(x0 - n0), p1 = exp2f(x1 - n1), p2 = exp2f(x2 - n0), p3 = exp2f(x3 - n1);
+        l0 = fmaf(l0, al0, p0 + p2);
+        l1 = fmaf(l1, al1, p1 + p3);
+        if (__any_sync(kFull, al0 != 1.f || al1 != 1.f)) {  // a running max moved
+#pragma unroll
+          for (int mt = 0; mt < S::kKSteps; ++mt) {
+            o[mt][0] *= al0;
+            o[mt][1] *= al1;
+            o[mt][2] *= al0;
+            o[mt][3] *= al1;
+          }
+        }
+        // (3) P^T as B fragments, split into hi + lo 16-bit parts
+        const uint32_t top_hi = M::pack(p0, p1), bot_hi = M::pack(p2, p3);
+        const float2 th = M::unpack(top_hi), bh = M::unpack(bot_hi);
+        const uint32_t top_lo = M::pack(p0 - th.x, p1 - th.y), bot_lo = M::pack(p2 - bh.x, p3 - bh.y);
+        const uint32_t pb0 = movm_t(top_hi), pb1 = movm_t(bot_hi);
+        const uint32_t pl0 = movm_t(top_lo), pl1 = movm_t(bot_lo);
+        // V^T fragment halves of tokens past the context are zeroed
+        uint32_t keep_lo = 0xffffffffu, keep_hi = 0xffffffffu;
+        if (nvalid < kBlockSize) {
+          keep_lo = (2 * t4 < nvalid ? 0x0000ffffu : 0u) | (2 * t4 + 1 < nvalid ? 0xffff0000u : 0u);
+          keep_hi = (2 * t4 + 8 < nvalid ? 0x0000ffffu : 0u) | (2 * t4 + 9 < nvalid ? 0xffff0000u : 0u);
+        }
+        // (4) O^T += V^T . P^T
+        {
+          const int row = lr + ((lm >> 1) << 3);
+#pragma unroll
+          for (int mt = 0; mt < S::kKSteps; ++mt) {
+            uint32_t a0, a1, a2, a3;
+            ldsm_x4_t(vt + swz(row, 2 * mt + (lm & 1)), a0, a1, a2, a3);
+            a0 &= keep_lo;
+            a1 &= keep_lo;
+            a2 &= keep_hi;
+            a3 &= keep_hi;
+            M::run(o[mt], a0, a1, a2, a3, pb0, pb1);
+            M::run(o[mt], a0, a1, a2, a3, pl0, pl1);
+          }
+        }
+      }
+      __syncwarp();
+      issue(i + NSTAGE);
+    }
+
+    // after a give-up, wait (bounded) for the copies still in flight
+    if (consumed < my_n) {
+      const int last = min(my_n, consumed + NSTAGE);
+      for (int i = consumed + 1; i < last; ++i) {
+        const int s = i % NSTAGE;
+        mbar_wait_bounded(bar0 + 8 * s, (phase_bits >> s) & 1u);
+        phase_bits ^= 1u << s;
+      }
+    }
+
+    // running sums over the lanes of each column (same t4)
+#pragma unroll
+    for (int msk = 4; msk <= 16; msk <<= 1) {
+      l0 += __shfl_xor_sync(kFull, l0, msk);
+      l1 += __shfl_xor_sync(kFull, l1, msk);
+    }
+
+    // warp record [o: 8 x D][m: 8][l: 8] in the warp's own (drained) stages
+    float* rec = reinterpret_cast<float*>(my_stages);
+    const int ha = 2 * t4, hb = 2 * t4 + 1;
+    const bool va = ha < ncol, vb = hb < ncol;
+#pragma unroll
+    for (int mt = 0; mt < S::kKSteps; ++mt) {
+      const int d0 = 16 * mt + g8;
+      if (va) {
+        rec[ha * D + d0] = o[mt][0];
+        rec[ha * D + d0 + 8] = o[mt][2];
+      }
+      if (vb) {
+        rec[hb * D + d0] = o[mt][1];
+        rec[hb * D + d0 + 8] = o[mt][3];
+      }
+    }
+    if (g8 == 0) {
+      if (va) {
+        rec[S::kRecM + ha] = m0;
+        rec[S::kRecL + ha] = l0;
+      }
+      if (vb) {
+        rec[S::kRecM + hb] = m1;
+        rec[S::kRecL + hb] = l1;
+      }
+    }
+    __syncthreads();
+
+    // merge the warps in a fixed order
+    for (int idx = threadIdx.x; idx < ncol * D; idx += NWARPS * 32) {
+      const int g = idx / D;
+      const int d = idx % D;
+      if (!col_valid(g)) continue;
+      float Mx = -INFINITY;
+#pragma unroll
+      for (int w = 0; w < NWARPS; ++w)
+        Mx = fmaxf(Mx, reinterpret_cast<const float*>(smem + w * S::kWarpStageBytes)[S::kRecM + g]);
+      float num = 0.f, den = 0.f;
+#pragma unroll
+      for (int w = 0; w < NWARPS; ++w) {
+        const float* r = reinterpret_cast<const float*>(smem + w * S::kWarpStageBytes);
+        const float sc = exp2f(r[S::kRecM + g] - Mx);
+        num = fmaf(sc, r[g * D + d], num);
+        den = fmaf(sc, r[S::kRecL + g], den);
+      }
+      const size_t row = col_row(g);
+      if (nparts == 1 && !cascade) {
+        reinterpret_cast<T*>(a.out)[row * D + d] = Fmt<T>::from_f32(num / den);
+      } else {
+        const size_t wrow = row * a.num_parts + pidx;
+        a.ws_o[wrow * D + d] = num;
+        if (d == 0) a.ws_ml[wrow] = make_float2(Mx, den);
+      }
+    }
+    // the records must be read before the next partition's copies land
+    __syncthreads();
+    if (__syncthreads_or(timed_out)) break;
   }
 }
 

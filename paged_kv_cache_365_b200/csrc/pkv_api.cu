@@ -22,8 +22,21 @@ __global__ void take_error_snapshot_kernel() { g_error_snapshot = atomicExch(&g_
 
 namespace {
 
-constexpr int kWarps = 4;
-constexpr int kMaxPartition = kWarps * 32 * PKV_BLOCK_SIZE;  // one table entry per lane
+constexpr int kWarps = 4;  // CUDA-core (fp32) kernel
+// tensor-core kernel: warps per CTA and staged pages per warp
+#ifndef PKV_MMA_WARPS
+#define PKV_MMA_WARPS 2
+#endif
+#ifndef PKV_MMA_STAGES
+#define PKV_MMA_STAGES 2
+#endif
+constexpr int kMmaWarps = PKV_MMA_WARPS;
+constexpr int kMmaStages = PKV_MMA_STAGES;
+// tokens per work unit: the fp32 kernel's warps hold one table entry per
+// lane, the tensor-core kernel's warps as many as a partition needs
+constexpr int kMaxPartition = 2048;
+static_assert(kMaxPartition <= kWarps * 32 * PKV_BLOCK_SIZE, "fp32 kernel: one table entry per lane");
+static_assert(kMaxPartition <= 128 * PKV_BLOCK_SIZE, "tensor-core kernel: its warps hold a partition's table entries");
 constexpr float kLog2e = 1.4426950408889634f;
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -65,8 +78,7 @@ pkv_status launch_decode(const pkv::DecodeArgs& a, cudaStream_t st) {
   kfn<<<grid, kWarps * 32, S::kSmem, st>>>(a);
   if (launched() != PKV_OK) return PKV_ECUDA;
   if (a.num_parts > 1) {
-    const dim3 g2((a.num_q_heads + 3) / 4, a.num_seqs);
-    pkv::paged_decode_reduce_kernel<T, D><<<g2, 128, 0, st>>>(a);
+    pkv::paged_decode_reduce_kernel<T, D><<<dim3(a.num_q_heads, a.num_seqs), pkv::kMergeWarps * 32, 0, st>>>(a);
     if (launched() != PKV_OK) return PKV_ECUDA;
   }
   return PKV_OK;
@@ -101,23 +113,22 @@ bool encode_cache_map(CUtensorMap* map, const void* base, CUtensorMapDataType dt
 
 template <typename T, int D, int G>
 pkv_status launch_decode_mma(const pkv::DecodeArgs& a, cudaStream_t st) {
-  constexpr int kStages = 3;
-  using S = pkv::MmaShape<T, D, G, kWarps, kStages>;
+  constexpr int kStages = kMmaStages;
+  using S = pkv::MmaShape<T, D, G, kMmaWarps, kStages>;
   CUtensorMap mk, mv;
   const long long rows = static_cast<long long>(a.num_blocks) * a.num_kv_heads * PKV_BLOCK_SIZE;
   if (!encode_cache_map(&mk, a.k_cache, pkv::Mma<T>::kTmaType, D, rows) ||
       !encode_cache_map(&mv, a.v_cache, pkv::Mma<T>::kTmaType, D, rows))
     return PKV_ECUDA;
-  auto kfn = pkv::paged_decode_mma_kernel<T, D, G, kWarps, kStages>;
+  auto kfn = pkv::paged_decode_mma_kernel<T, D, G, kMmaWarps, kStages, false>;
   if (cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(S::kSmem)) !=
       cudaSuccess)
     return PKV_ECUDA;
   const dim3 grid(a.num_kv_heads, a.num_seqs, a.num_parts);
-  kfn<<<grid, kWarps * 32, S::kSmem, st>>>(a, mk, mv);
+  kfn<<<grid, kMmaWarps * 32, S::kSmem, st>>>(a, mk, mv);
   if (launched() != PKV_OK) return PKV_ECUDA;
   if (a.num_parts > 1) {
-    const dim3 g2((a.num_q_heads + 3) / 4, a.num_seqs);
-    pkv::paged_decode_reduce_kernel<T, D><<<g2, 128, 0, st>>>(a);
+    pkv::paged_decode_reduce_kernel<T, D><<<dim3(a.num_q_heads, a.num_seqs), pkv::kMergeWarps * 32, 0, st>>>(a);
     if (launched() != PKV_OK) return PKV_ECUDA;
   }
   return PKV_OK;
@@ -142,9 +153,19 @@ pkv_status dispatch_dim_mma(const pkv::DecodeArgs& a, int D, int G, cudaStream_t
 }
 
 // ---- shared-prefix (cascade) path ------------------------------------------
-constexpr int kPrefixChunkPages = 16;  // prefix pages per prefix-pass CTA
-constexpr int kPrefixWarps = 8;        // 16 queries per warp
-constexpr int kPrefixStages = 4;
+constexpr int kPrefixChunkPages = 32;  // prefix pages per prefix-role CTA (one table entry per lane)
+
+// Partition of the cascade's suffix pass.  Auto (0): the longest suffix
+// (context past the prefix) rounded up to whole pages, kept in [512, 2048],
+// so that a batch of short suffixes needs one partition per sequence.
+int resolve_prefix_partition(int partition_tokens, int max_context_len, int prefix_pages) {
+  if (partition_tokens != 0) return resolve_partition(partition_tokens);
+  const long long span = static_cast<long long>(max_context_len) - static_cast<long long>(prefix_pages) * 16;
+  long long p = (span + 15) / 16 * 16;
+  if (p < PKV_DEFAULT_PARTITION) p = PKV_DEFAULT_PARTITION;
+  if (p > kMaxPartition) p = kMaxPartition;
+  return static_cast<int>(p);
+}
 
 struct PrefixLayout {
   long long parts, chunks;
@@ -171,31 +192,27 @@ PrefixLayout prefix_layout(long long B, long long Hq, long long D, long long max
 
 template <typename T, int D, int G>
 pkv_status launch_decode_prefix(const pkv::DecodeArgs& a, cudaStream_t st) {
-  constexpr int kStages = 3;
-  using S = pkv::MmaShape<T, D, G, kWarps, kStages>;
-  using SP = pkv::PrefixShape<T, D, kPrefixWarps, kPrefixStages>;
+  constexpr int kStages = kMmaStages;
+  using S = pkv::MmaShape<T, D, G, kMmaWarps, kStages>;
   CUtensorMap mk, mv;
   const long long rows = static_cast<long long>(a.num_blocks) * a.num_kv_heads * PKV_BLOCK_SIZE;
   if (!encode_cache_map(&mk, a.k_cache, pkv::Mma<T>::kTmaType, D, rows) ||
       !encode_cache_map(&mv, a.v_cache, pkv::Mma<T>::kTmaType, D, rows))
     return PKV_ECUDA;
-  // (1) each sequence's suffix (whole context when it does not share the prefix)
-  auto kfn = pkv::paged_decode_mma_kernel<T, D, G, kWarps, kStages>;
+  // one launch: prefix-role CTAs first (the shared pages, from L2), then one
+  // CTA per (kv-head, sequence, suffix partition in flight)
+  auto kfn = pkv::paged_decode_mma_kernel<T, D, G, kMmaWarps, kStages, true>;
   if (cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(S::kSmem)) !=
       cudaSuccess)
     return PKV_ECUDA;
-  kfn<<<dim3(a.num_kv_heads, a.num_seqs, a.num_parts), kWarps * 32, S::kSmem, st>>>(a, mk, mv);
-  if (launched() != PKV_OK) return PKV_ECUDA;
-  // (2) the shared prefix, once per kv-head, for every sequence's queries
-  auto pfn = pkv::paged_decode_prefix_kernel<T, D, G, kPrefixWarps, kPrefixStages>;
-  if (cudaFuncSetAttribute(pfn, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(SP::kSmem)) !=
-      cudaSuccess)
-    return PKV_ECUDA;
-  const int qgroups = (a.num_seqs * G + kPrefixWarps * 16 - 1) / (kPrefixWarps * 16);
-  pfn<<<dim3(a.num_kv_heads, a.num_chunks, qgroups), kPrefixWarps * 32, SP::kSmem, st>>>(a, mk, mv);
+  const long long ygrid = static_cast<long long>(a.num_qgroups) * a.num_chunks +
+                          static_cast<long long>(a.num_seqs) * a.suffix_z;
+  if (ygrid > 65535) return PKV_EINVAL;
+  kfn<<<dim3(a.num_kv_heads, static_cast<unsigned>(ygrid), 1), kMmaWarps * 32, S::kSmem, st>>>(a, mk, mv);
   if (launched() != PKV_OK) return PKV_ECUDA;
   // (3) merge prefix chunks and suffix partitions
-  pkv::paged_decode_prefix_merge_kernel<T, D><<<dim3((a.num_q_heads + 3) / 4, a.num_seqs), 128, 0, st>>>(a);
+  pkv::paged_decode_prefix_merge_kernel<T, D>
+      <<<dim3(a.num_q_heads, a.num_seqs), pkv::kMergeWarps * 32, 0, st>>>(a);
   return launched();
 }
 
@@ -387,7 +404,7 @@ pkv_status pkv_paged_attention_decode(void* out, const void* q, const void* k_ca
 
 size_t pkv_decode_prefix_workspace_bytes(int num_seqs, int num_q_heads, int head_dim, int max_context_len,
                                          int prefix_pages, int partition_tokens) {
-  const int part = resolve_partition(partition_tokens);
+  const int part = resolve_prefix_partition(partition_tokens, max_context_len, prefix_pages);
   if (part < 0 || num_seqs < 0 || num_q_heads <= 0 || !head_dim_ok(head_dim) || max_context_len < 0 ||
       prefix_pages <= 0)
     return 0;
@@ -405,9 +422,11 @@ pkv_status pkv_paged_attention_decode_prefix(void* out, const void* q, const voi
   if (prefix_pages <= 0 || prefix_pages > max_blocks_per_seq) return PKV_EINVAL;
   pkv::DecodeArgs a{};
   long long P = 0;
+  const int part = resolve_prefix_partition(partition_tokens, max_context_len, prefix_pages);
+  if (part < 0) return PKV_EINVAL;
   const pkv_status st0 = prepare_decode(out, q, k_cache, v_cache, block_tables, max_blocks_per_seq, context_lens,
                                         max_context_len, num_seqs, num_q_heads, num_kv_heads, head_dim, num_blocks,
-                                        scale, partition_tokens, dtype, &a, &P);
+                                        scale, part, dtype, &a, &P);
   if (st0 != PKV_OK || num_seqs == 0) return st0;
   if (prefix_blocks == nullptr) return PKV_EINVAL;
   const PrefixLayout L = prefix_layout(num_seqs, num_q_heads, head_dim, max_context_len, prefix_pages, a.partition);
@@ -423,6 +442,14 @@ pkv_status pkv_paged_attention_decode_prefix(void* out, const void* q, const voi
   a.prefix_pages = prefix_pages;
   a.chunk_pages = kPrefixChunkPages;
   a.num_chunks = static_cast<int>(L.chunks);
+  a.num_qgroups = (num_seqs * (num_q_heads / num_kv_heads) + kMmaWarps * 16 - 1) / (kMmaWarps * 16);  // 16 queries per prefix warp
+  // suffix partitions in flight per sequence: enough for the longest suffix
+  // of a sequence that shares the prefix; a sequence that does not share it
+  // loops over its extra partitions
+  const long long span_max = static_cast<long long>(max_context_len) - static_cast<long long>(prefix_pages) * PKV_BLOCK_SIZE;
+  a.suffix_z = span_max > 0 ? static_cast<int>((span_max + a.partition - 1) / a.partition) : 1;
+  if (static_cast<long long>(a.num_qgroups) * a.num_chunks + static_cast<long long>(num_seqs) * a.suffix_z > 65535)
+    return PKV_EINVAL;
 
   const int G = num_q_heads / num_kv_heads;
   cudaStream_t st = static_cast<cudaStream_t>(stream);

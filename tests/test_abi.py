@@ -131,10 +131,14 @@ def test_kv_cache_bytes_matches_page_example():
 def test_prefix_workspace_and_rejections(lib):
     up = lambda x: (x + 15) // 16 * 16
     B, Hq, D, ctx, pp = 4, 8, 128, 1100, 20
-    P, C = 3, 2  # ceil(1100/512), ceil(20/16)
+    # auto partition: the longest suffix 1100 - 320 = 780 rounded up to 784
+    P, C = 2, 1  # ceil(1100/784), ceil(20/64)
     want = up(up(up(up(up(B * Hq * P * D * 4) + B * Hq * P * 8) + B * Hq * C * D * 4) + B * Hq * C * 8) + B * 4)
     assert lib.pkv_decode_prefix_workspace_bytes(B, Hq, D, ctx, pp, 0) == want
     assert lib.pkv_decode_prefix_workspace_bytes(B, Hq, D, ctx, 0, 0) == 0
+    # explicit partition 512: P = 3
+    want512 = up(up(up(up(up(B * Hq * 3 * D * 4) + B * Hq * 3 * 8) + B * Hq * C * D * 4) + B * Hq * C * 8) + B * 4)
+    assert lib.pkv_decode_prefix_workspace_bytes(B, Hq, D, ctx, pp, 512) == want512
     args = [FAKE, FAKE, FAKE, FAKE, FAKE, 100, FAKE, 1100, FAKE, 20, 4, 8, 2, 128, 64, ctypes.c_float(0.1), 0,
             1, FAKE, 1 << 30, None]
     for idx, bad in ((17, 0), (9, 0), (9, 101), (8, None), (18, None), (19, 16)):
