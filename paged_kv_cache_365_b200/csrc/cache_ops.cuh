@@ -18,6 +18,7 @@ __global__ void __launch_bounds__(256)
                      uint4* __restrict__ k_cache, uint4* __restrict__ v_cache,
                      const int64_t* __restrict__ slots, long long total, int Hkv, int row_chunks,
                      int num_blocks) {
+  pdl_enter();
   const long long stride = static_cast<long long>(gridDim.x) * blockDim.x;
   for (long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; i < 2 * total;
        i += stride) {
@@ -48,6 +49,7 @@ __global__ void __launch_bounds__(256)
 __global__ void __launch_bounds__(256)
     copy_blocks_kernel(uint4* __restrict__ k_cache, uint4* __restrict__ v_cache,
                        const int32_t* __restrict__ pairs, long long block_chunks, int num_blocks) {
+  pdl_enter();
   constexpr int kUnroll = 4;
   const int p = blockIdx.y;
   const int src = pairs[2 * p];

@@ -21,6 +21,19 @@ __device__ unsigned int g_error_word = 0u;
 
 __device__ __forceinline__ void raise_error(unsigned int bits) { atomicOr(&g_error_word, bits); }
 
+// Programmatic dependent launch.  Every library kernel is launched with
+// programmatic stream serialization, so it may be scheduled while the
+// previous kernel in the stream is still draining.  Each kernel calls
+// pdl_wait() before its first global-memory access (that makes the previous
+// kernel's writes visible, whatever that kernel was), then pdl_trigger() so
+// that the next kernel can be scheduled once every CTA of this one started.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+__device__ __forceinline__ void pdl_enter() {
+  pdl_wait();
+  pdl_trigger();
+}
+
 // ---------------------------------------------------------------------------
 // storage formats: a 16-byte chunk holds kVec elements
 // ---------------------------------------------------------------------------

@@ -153,6 +153,7 @@ __device__ __forceinline__ void load_probs(const float* p, float (&out)[G]) {
 template <typename T, int D, int G, int NWARPS, int NSTAGE>
 __global__ void __launch_bounds__(NWARPS * 32)
     paged_decode_partition_kernel(const DecodeArgs a) {
+  pdl_enter();
   using S = DecodeShape<T, D, G, NWARPS, NSTAGE>;
   const int kvh = blockIdx.x;
   const int b = blockIdx.y;
@@ -475,6 +476,7 @@ __device__ __forceinline__ void merge_partials(int n, ML ml, OP op, T* out) {
 // whose context spans more than one partition, the partitions in order.
 template <typename T, int D>
 __global__ void __launch_bounds__(kMergeWarps * 32) paged_decode_reduce_kernel(const DecodeArgs a) {
+  pdl_enter();
   const int h = blockIdx.x;
   const int b = blockIdx.y;
   int ctx = a.context_lens[b];

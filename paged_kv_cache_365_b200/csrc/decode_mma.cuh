@@ -348,6 +348,7 @@ template <typename T, int D, int G, int NWARPS, int NSTAGE, bool kCascade>
 __global__ void __launch_bounds__(NWARPS * 32)
     paged_decode_mma_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tmap_k,
                             const __grid_constant__ CUtensorMap tmap_v) {
+  pdl_enter();
   using S = MmaShape<T, D, G, NWARPS, NSTAGE>;
   using M = Mma<T>;
   const int kvh = blockIdx.x;

@@ -21,6 +21,7 @@ namespace pkv {
 // prefix) then the suffix partitions, in order, rescaled to their common max.
 template <typename T, int D>
 __global__ void __launch_bounds__(kMergeWarps * 32) paged_decode_prefix_merge_kernel(const DecodeArgs a) {
+  pdl_enter();
   const int h = blockIdx.x;
   const int b = blockIdx.y;
   int ctx = a.context_lens[b];

@@ -64,7 +64,22 @@ constexpr int stages_for(int stage_bytes) {
   return stage_bytes >= 16384 ? 2 : (24576 / stage_bytes > 8 ? 8 : 24576 / stage_bytes);
 }
 
-pkv_status launched() { return cudaGetLastError() == cudaSuccess ? PKV_OK : PKV_ECUDA; }
+
+// Launch with programmatic stream serialization (see pdl_wait in common.cuh).
+template <typename... KArgs, typename... Args>
+pkv_status launch(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, args...) == cudaSuccess ? PKV_OK : PKV_ECUDA;
+}
 
 template <typename T, int D, int G>
 pkv_status launch_decode(const pkv::DecodeArgs& a, cudaStream_t st) {
@@ -75,11 +90,11 @@ pkv_status launch_decode(const pkv::DecodeArgs& a, cudaStream_t st) {
       cudaSuccess)
     return PKV_ECUDA;
   const dim3 grid(a.num_kv_heads, a.num_seqs, a.num_parts);
-  kfn<<<grid, kWarps * 32, S::kSmem, st>>>(a);
-  if (launched() != PKV_OK) return PKV_ECUDA;
+  if (launch(kfn, grid, dim3(kWarps * 32), S::kSmem, st, a) != PKV_OK) return PKV_ECUDA;
   if (a.num_parts > 1) {
-    pkv::paged_decode_reduce_kernel<T, D><<<dim3(a.num_q_heads, a.num_seqs), pkv::kMergeWarps * 32, 0, st>>>(a);
-    if (launched() != PKV_OK) return PKV_ECUDA;
+    if (launch(pkv::paged_decode_reduce_kernel<T, D>, dim3(a.num_q_heads, a.num_seqs), dim3(pkv::kMergeWarps * 32), 0,
+               st, a) != PKV_OK)
+      return PKV_ECUDA;
   }
   return PKV_OK;
 }
@@ -125,11 +140,11 @@ pkv_status launch_decode_mma(const pkv::DecodeArgs& a, cudaStream_t st) {
       cudaSuccess)
     return PKV_ECUDA;
   const dim3 grid(a.num_kv_heads, a.num_seqs, a.num_parts);
-  kfn<<<grid, kMmaWarps * 32, S::kSmem, st>>>(a, mk, mv);
-  if (launched() != PKV_OK) return PKV_ECUDA;
+  if (launch(kfn, dim3(grid), dim3(kMmaWarps * 32), S::kSmem, st, a, mk, mv) != PKV_OK) return PKV_ECUDA;
   if (a.num_parts > 1) {
-    pkv::paged_decode_reduce_kernel<T, D><<<dim3(a.num_q_heads, a.num_seqs), pkv::kMergeWarps * 32, 0, st>>>(a);
-    if (launched() != PKV_OK) return PKV_ECUDA;
+    if (launch(pkv::paged_decode_reduce_kernel<T, D>, dim3(a.num_q_heads, a.num_seqs), dim3(pkv::kMergeWarps * 32), 0,
+               st, a) != PKV_OK)
+      return PKV_ECUDA;
   }
   return PKV_OK;
 }
@@ -208,12 +223,12 @@ pkv_status launch_decode_prefix(const pkv::DecodeArgs& a, cudaStream_t st) {
   const long long ygrid = static_cast<long long>(a.num_qgroups) * a.num_chunks +
                           static_cast<long long>(a.num_seqs) * a.suffix_z;
   if (ygrid > 65535) return PKV_EINVAL;
-  kfn<<<dim3(a.num_kv_heads, static_cast<unsigned>(ygrid), 1), kMmaWarps * 32, S::kSmem, st>>>(a, mk, mv);
-  if (launched() != PKV_OK) return PKV_ECUDA;
+  if (launch(kfn, dim3(a.num_kv_heads, static_cast<unsigned>(ygrid), 1), dim3(kMmaWarps * 32), S::kSmem, st, a, mk,
+             mv) != PKV_OK)
+    return PKV_ECUDA;
   // (3) merge prefix chunks and suffix partitions
-  pkv::paged_decode_prefix_merge_kernel<T, D>
-      <<<dim3(a.num_q_heads, a.num_seqs), pkv::kMergeWarps * 32, 0, st>>>(a);
-  return launched();
+  return launch(pkv::paged_decode_prefix_merge_kernel<T, D>, dim3(a.num_q_heads, a.num_seqs),
+                dim3(pkv::kMergeWarps * 32), 0, st, a);
 }
 
 template <typename T, int D>
@@ -327,10 +342,9 @@ pkv_status pkv_kv_append(const void* k_new, const void* v_new, void* k_cache, vo
   const long long total = static_cast<long long>(num_tokens) * num_kv_heads * row_chunks;
   const long long want = (2 * total + 255) / 256;
   const int blocks = static_cast<int>(want < 148 * 32 ? want : 148 * 32);
-  pkv::kv_append_kernel<<<blocks, 256, 0, static_cast<cudaStream_t>(stream)>>>(
-      static_cast<const uint4*>(k_new), static_cast<const uint4*>(v_new), static_cast<uint4*>(k_cache),
-      static_cast<uint4*>(v_cache), slot_mapping, total, num_kv_heads, row_chunks, num_blocks);
-  return launched();
+  return launch(pkv::kv_append_kernel, dim3(blocks), dim3(256), 0, static_cast<cudaStream_t>(stream),
+                static_cast<const uint4*>(k_new), static_cast<const uint4*>(v_new), static_cast<uint4*>(k_cache),
+                static_cast<uint4*>(v_cache), slot_mapping, total, num_kv_heads, row_chunks, num_blocks);
 }
 
 pkv_status pkv_copy_blocks(void* k_cache, void* v_cache, const int32_t* pairs, int num_pairs, int num_kv_heads,
@@ -345,9 +359,8 @@ pkv_status pkv_copy_blocks(void* k_cache, void* v_cache, const int32_t* pairs, i
   const long long per_cta = 256 * 4;
   const int gx = static_cast<int>((block_chunks + per_cta - 1) / per_cta);
   const dim3 grid(gx, num_pairs, 2);
-  pkv::copy_blocks_kernel<<<grid, 256, 0, static_cast<cudaStream_t>(stream)>>>(
-      static_cast<uint4*>(k_cache), static_cast<uint4*>(v_cache), pairs, block_chunks, num_blocks);
-  return launched();
+  return launch(pkv::copy_blocks_kernel, grid, dim3(256), 0, static_cast<cudaStream_t>(stream),
+                static_cast<uint4*>(k_cache), static_cast<uint4*>(v_cache), pairs, block_chunks, num_blocks);
 }
 
 pkv_status pkv_copy_blocks_check(const int32_t* pairs_host, int num_pairs, int num_blocks) {
