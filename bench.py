@@ -235,27 +235,44 @@ def run_cuda(args, rank, world, local_rank):
     else:
         launches_per_step = 1 + 1 + (1 if n_pairs else 0) + (1 if P > 1 else 0)
 
+    # every call goes to the current stream at call time (so that a CUDA
+    # graph capture records it)
     def pre_decode():
         if n_pairs:
-            pkv.copy_blocks(cache.k, cache.v, st["cow_pairs"], stream)
-        pkv.kv_append(st["k_new"], st["v_new"], cache.k, cache.v, st["slot_mapping"], stream)
+            pkv.copy_blocks(cache.k, cache.v, st["cow_pairs"])
+        pkv.kv_append(st["k_new"], st["v_new"], cache.k, cache.v, st["slot_mapping"])
 
     def decode():
         if use_cascade:
             pkv.paged_attention_decode_prefix(st["q"], cache.k, cache.v, st["block_tables"], st["context_lens"],
                                               max_ctx, prefix, scale, out=out, workspace=ws,
-                                              partition=args.partition, stream=stream)
+                                              partition=args.partition)
         else:
             pkv.paged_attention_decode(st["q"], cache.k, cache.v, st["block_tables"], st["context_lens"], max_ctx,
-                                       scale, out=out, workspace=ws, partition=args.partition, stream=stream)
+                                       scale, out=out, workspace=ws, partition=args.partition)
+
+    def eager_step():
+        pre_decode()
+        decode()
+
+    run_step = eager_step
+    if args.graph:
+        # one whole step captured once, replayed every iteration
+        for _ in range(3):
+            eager_step()
+        torch.cuda.synchronize()
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            eager_step()
+        torch.cuda.synchronize()
+        run_step = graph.replay
 
     def barrier():
         if world > 1:
             torch.distributed.barrier()
 
     for _ in range(args.warmup):
-        pre_decode()
-        decode()
+        run_step()
     torch.cuda.synchronize()
     if pkv.get_error() != 0:
         raise RuntimeError("device error flags raised during warm-up")
@@ -269,8 +286,7 @@ def run_cuda(args, rank, world, local_rank):
     with ClockSampler(local_rank) as clocks:
         t0.record(stream)
         for i in range(K):
-            pre_decode()
-            decode()
+            run_step()
         t1.record(stream)
         torch.cuda.synchronize()
     barrier()
@@ -416,6 +432,7 @@ def config_of(wl, args, P):
             "context_lens": {"min": int(wl.context_lens.min()), "max": int(wl.context_lens.max()),
                              "sum": int(wl.context_lens.astype(np.int64).sum())},
             "partition_tokens": args.partition or 512, "partitions_max": P, "seed": args.seed,
+            "cuda_graph": bool(getattr(args, "graph", False)),
             "parallelism": f"replicas{args.gpus}" if args.gpus > 1 else "single-gpu",
             "l2": "inputs larger than L2 (no flush)" if kv_bytes(wl, True) > 126e6 else "inputs fit in L2"}
 
@@ -468,6 +485,8 @@ def main(argv=None):
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--partition", type=int, default=0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--graph", action="store_true",
+                    help="capture one step in a CUDA graph and replay it (launch-bound batches)")
     ap.add_argument("--no-cascade", action="store_true",
                     help="decode a shared-prefix batch with the plain paged kernel")
     args = ap.parse_args(argv)
