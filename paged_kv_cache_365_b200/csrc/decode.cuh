@@ -418,38 +418,40 @@ __global__ void __launch_bounds__(NWARPS * 32)
 // Merge n partial results (running max m_p in log2 units, running sum l_p,
 // unnormalised output o_p) of one (sequence, query head):
 //   out = sum_p 2^(m_p - M) o_p / sum_p 2^(m_p - M) l_p,   M = max_p m_p.
-// One CTA of kMergeWarps warps: warp w accumulates partials w, w + 8, ... in
-// order (independent loads, unrolled), then the warps' sums are added in a
+// A CTA of kMergeWarps warps serves HPC heads with WPH = kMergeWarps / HPC
+// warps each (many warps per head when a head has many partials, one when
+// it has few).  Warp w of a head accumulates partials w, w + WPH, ... in
+// order (independent loads, unrolled); the warps' sums are then added in a
 // fixed order.  `ml(p)` / `op(p)` give partial p's (m, l) and output row.
 constexpr int kMergeWarps = 8;
 
-template <typename T, int D, typename ML, typename OP>
-__device__ __forceinline__ void merge_partials(int n, ML ml, OP op, T* out) {
+template <typename T, int D, int HPC, typename ML, typename OP>
+__device__ __forceinline__ void merge_partials(int n, ML ml, OP op, T* out, int hs /* head slot in the CTA */) {
   constexpr int kEpl = D / 32;
+  constexpr int WPH = kMergeWarps / HPC;
+  static_assert(kMergeWarps % HPC == 0, "heads per CTA must divide the warps");
   __shared__ float red_o[kMergeWarps][D];
   __shared__ float red_den[kMergeWarps];
   __shared__ float red_max[kMergeWarps];
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  if (n <= 0) {
-    for (int d = threadIdx.x; d < D; d += kMergeWarps * 32) out[d] = Fmt<T>::from_f32(0.f);
-    return;
-  }
+  const int wi = warp % WPH;  // warp within the head
+  const int w0 = hs * WPH;    // first warp of the head
   float M = -INFINITY;
-  for (int p = threadIdx.x; p < n; p += kMergeWarps * 32) M = fmaxf(M, ml(p).x);
+  for (int p = wi * 32 + lane; p < n; p += WPH * 32) M = fmaxf(M, ml(p).x);
   M = warp_max(M);
   if (lane == 0) red_max[warp] = M;
   __syncthreads();
-  M = red_max[0];
+  M = red_max[w0];
 #pragma unroll
-  for (int w = 1; w < kMergeWarps; ++w) M = fmaxf(M, red_max[w]);
+  for (int w = 1; w < WPH; ++w) M = fmaxf(M, red_max[w0 + w]);
 
   float acc[kEpl];
 #pragma unroll
   for (int e = 0; e < kEpl; ++e) acc[e] = 0.f;
   float den = 0.f;
 #pragma unroll 4
-  for (int p = warp; p < n; p += kMergeWarps) {
+  for (int p = wi; p < n; p += WPH) {
     const float2 v = ml(p);
     const float w = exp2f(v.x - M);
     den = fmaf(w, v.y, den);
@@ -457,36 +459,54 @@ __device__ __forceinline__ void merge_partials(int n, ML ml, OP op, T* out) {
 #pragma unroll
     for (int e = 0; e < kEpl; ++e) acc[e] = fmaf(w, o[e], acc[e]);
   }
+  if constexpr (WPH == 1) {
+    if (n > 0) {
 #pragma unroll
-  for (int e = 0; e < kEpl; ++e) red_o[warp][lane * kEpl + e] = acc[e];
-  if (lane == 0) red_den[warp] = den;
-  __syncthreads();
-  for (int d = threadIdx.x; d < D; d += kMergeWarps * 32) {
-    float num = 0.f, dd = 0.f;
+      for (int e = 0; e < kEpl; ++e) out[lane * kEpl + e] = Fmt<T>::from_f32(acc[e] / den);
+    } else {
 #pragma unroll
-    for (int w = 0; w < kMergeWarps; ++w) {
-      num += red_o[w][d];
-      dd += red_den[w];
+      for (int e = 0; e < kEpl; ++e) out[lane * kEpl + e] = Fmt<T>::from_f32(0.f);
     }
-    out[d] = Fmt<T>::from_f32(num / dd);
+  } else {
+#pragma unroll
+    for (int e = 0; e < kEpl; ++e) red_o[warp][lane * kEpl + e] = acc[e];
+    if (lane == 0) red_den[warp] = den;
+    __syncthreads();
+    for (int d = wi * 32 + lane; d < D; d += WPH * 32) {
+      float num = 0.f, dd = 0.f;
+#pragma unroll
+      for (int w = 0; w < WPH; ++w) {
+        num += red_o[w0 + w][d];
+        dd += red_den[w0 + w];
+      }
+      out[d] = Fmt<T>::from_f32(n > 0 ? num / dd : 0.f);
+    }
   }
 }
 
-// Split-K merge: per (query head h = blockIdx.x, sequence b = blockIdx.y)
-// whose context spans more than one partition, the partitions in order.
-template <typename T, int D>
+// Split-K merge: per (query head, sequence b = blockIdx.y) whose context
+// spans more than one partition, the partitions in order.  Head of this
+// warp: blockIdx.x * HPC + warp / (kMergeWarps / HPC).
+template <typename T, int D, int HPC>
 __global__ void __launch_bounds__(kMergeWarps * 32) paged_decode_reduce_kernel(const DecodeArgs a) {
   pdl_enter();
-  const int h = blockIdx.x;
+  const int hs = (threadIdx.x >> 5) / (kMergeWarps / HPC);
+  const int h = blockIdx.x * HPC + hs;
   const int b = blockIdx.y;
   int ctx = a.context_lens[b];
   ctx = ctx < 0 ? 0 : (ctx > a.max_ctx ? a.max_ctx : ctx);
   const int nparts = (ctx + a.partition - 1) / a.partition;
-  if (nparts <= 1) return;  // written by the partition kernel
-  const size_t row0 = (static_cast<size_t>(b) * a.num_q_heads + h) * a.num_parts;
-  T* out = reinterpret_cast<T*>(a.out) + (static_cast<size_t>(b) * a.num_q_heads + h) * D;
-  merge_partials<T, D>(
-      nparts, [&](int p) { return a.ws_ml[row0 + p]; }, [&](int p) { return a.ws_o + (row0 + p) * D; }, out);
+  // one partition: written by the partition kernel; a head past Hq: nothing
+  // (the CTA-wide barriers below still need every warp, so no early exit)
+  const bool skip = nparts <= 1 || h >= a.num_q_heads;
+  const int hh = h < a.num_q_heads ? h : 0;
+  const size_t row0 = (static_cast<size_t>(b) * a.num_q_heads + hh) * a.num_parts;
+  if (__syncthreads_and(skip)) return;
+  T* out = reinterpret_cast<T*>(a.out) + (static_cast<size_t>(b) * a.num_q_heads + hh) * D;
+  __shared__ T sink[D];  // output of a skipped head slot (discarded)
+  merge_partials<T, D, HPC>(
+      skip ? 0 : nparts, [&](int p) { return a.ws_ml[row0 + p]; }, [&](int p) { return a.ws_o + (row0 + p) * D; },
+      skip ? sink : out, hs);
 }
 
 }  // namespace pkv

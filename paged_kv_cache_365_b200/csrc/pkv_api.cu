@@ -81,6 +81,26 @@ pkv_status launch(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, 
   return cudaLaunchKernelEx(&cfg, kernel, args...) == cudaSuccess ? PKV_OK : PKV_ECUDA;
 }
 
+// Merge launches: heads per CTA from the number of partials per head
+// (8 warps on one head when there are many, one warp per head when few).
+template <typename T, int D, template <typename, int, int> class K>
+pkv_status launch_merge(const pkv::DecodeArgs& a, int partials_per_head, cudaStream_t st) {
+  const dim3 block(pkv::kMergeWarps * 32);
+  if (partials_per_head >= 32)
+    return launch(K<T, D, 1>::fn, dim3(a.num_q_heads, a.num_seqs), block, 0, st, a);
+  if (partials_per_head >= 8)
+    return launch(K<T, D, 4>::fn, dim3((a.num_q_heads + 3) / 4, a.num_seqs), block, 0, st, a);
+  return launch(K<T, D, 8>::fn, dim3((a.num_q_heads + 7) / 8, a.num_seqs), block, 0, st, a);
+}
+template <typename T, int D, int HPC>
+struct ReduceK {
+  static constexpr auto fn = pkv::paged_decode_reduce_kernel<T, D, HPC>;
+};
+template <typename T, int D, int HPC>
+struct PrefixMergeK {
+  static constexpr auto fn = pkv::paged_decode_prefix_merge_kernel<T, D, HPC>;
+};
+
 template <typename T, int D, int G>
 pkv_status launch_decode(const pkv::DecodeArgs& a, cudaStream_t st) {
   constexpr int kStages = stages_for(2 * PKV_BLOCK_SIZE * D * static_cast<int>(sizeof(T)));
@@ -92,9 +112,7 @@ pkv_status launch_decode(const pkv::DecodeArgs& a, cudaStream_t st) {
   const dim3 grid(a.num_kv_heads, a.num_seqs, a.num_parts);
   if (launch(kfn, grid, dim3(kWarps * 32), S::kSmem, st, a) != PKV_OK) return PKV_ECUDA;
   if (a.num_parts > 1) {
-    if (launch(pkv::paged_decode_reduce_kernel<T, D>, dim3(a.num_q_heads, a.num_seqs), dim3(pkv::kMergeWarps * 32), 0,
-               st, a) != PKV_OK)
-      return PKV_ECUDA;
+    if (launch_merge<T, D, ReduceK>(a, a.num_parts, st) != PKV_OK) return PKV_ECUDA;
   }
   return PKV_OK;
 }
@@ -142,9 +160,7 @@ pkv_status launch_decode_mma(const pkv::DecodeArgs& a, cudaStream_t st) {
   const dim3 grid(a.num_kv_heads, a.num_seqs, a.num_parts);
   if (launch(kfn, dim3(grid), dim3(kMmaWarps * 32), S::kSmem, st, a, mk, mv) != PKV_OK) return PKV_ECUDA;
   if (a.num_parts > 1) {
-    if (launch(pkv::paged_decode_reduce_kernel<T, D>, dim3(a.num_q_heads, a.num_seqs), dim3(pkv::kMergeWarps * 32), 0,
-               st, a) != PKV_OK)
-      return PKV_ECUDA;
+    if (launch_merge<T, D, ReduceK>(a, a.num_parts, st) != PKV_OK) return PKV_ECUDA;
   }
   return PKV_OK;
 }
@@ -227,8 +243,7 @@ pkv_status launch_decode_prefix(const pkv::DecodeArgs& a, cudaStream_t st) {
              mv) != PKV_OK)
     return PKV_ECUDA;
   // (3) merge prefix chunks and suffix partitions
-  return launch(pkv::paged_decode_prefix_merge_kernel<T, D>, dim3(a.num_q_heads, a.num_seqs),
-                dim3(pkv::kMergeWarps * 32), 0, st, a);
+  return launch_merge<T, D, PrefixMergeK>(a, a.num_chunks + a.num_parts, st);
 }
 
 template <typename T, int D>
@@ -374,6 +389,76 @@ pkv_status pkv_copy_blocks_check(const int32_t* pairs_host, int num_pairs, int n
   }
   for (int32_t d : dsts)
     if (srcs.count(d)) return PKV_EINVAL;
+  return PKV_OK;
+}
+
+// Device address of caller memory the kernels may touch: device memory of
+// the current device, managed memory, or page-locked host memory mapped
+// into the device's address space.  Pageable host memory, another device's
+// memory and unknown pointers are rejected.
+bool device_view(const void* p, void** out) {
+  cudaPointerAttributes at;
+  if (cudaPointerGetAttributes(&at, p) != cudaSuccess) {
+    cudaGetLastError();
+    return false;
+  }
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) return false;
+  switch (at.type) {
+    case cudaMemoryTypeDevice:
+      if (at.device != dev) return false;
+      *out = const_cast<void*>(p);
+      return true;
+    case cudaMemoryTypeManaged:
+      *out = const_cast<void*>(p);
+      return true;
+    case cudaMemoryTypeHost:
+      if (at.devicePointer == nullptr) return false;
+      *out = at.devicePointer;
+      return true;
+    default:
+      return false;
+  }
+}
+
+pkv_status pkv_swap_blocks(void* dst_k, void* dst_v, int dst_blocks, const void* src_k, const void* src_v,
+                           int src_blocks, const int32_t* pairs, int num_pairs, int num_kv_heads, int head_dim,
+                           pkv_dtype dtype, void* stream) {
+  const int es = dtype_bytes(dtype);
+  if (es == 0 || num_pairs < 0 || num_kv_heads <= 0 || !head_dim_ok(head_dim) || dst_blocks <= 0 ||
+      src_blocks <= 0)
+    return PKV_EINVAL;
+  if (num_pairs == 0) return PKV_OK;
+  if (!dst_k || !dst_v || !src_k || !src_v || !pairs || !aligned16(dst_k) || !aligned16(dst_v) ||
+      !aligned16(src_k) || !aligned16(src_v))
+    return PKV_EINVAL;
+  void *dk, *dv, *sk, *sv, *pp;
+  if (!device_view(dst_k, &dk) || !device_view(dst_v, &dv) || !device_view(src_k, &sk) ||
+      !device_view(src_v, &sv) || !device_view(pairs, &pp))
+    return PKV_EINVAL;
+  const long long block_chunks = static_cast<long long>(num_kv_heads) * PKV_BLOCK_SIZE * head_dim * es / 16;
+  const long long total = block_chunks * num_pairs;
+  int sms = 148;
+  int dev = 0;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const long long per_cta = 256LL * 4;
+  long long blocks = (2 * total + per_cta - 1) / per_cta;
+  if (blocks > static_cast<long long>(sms) * 8) blocks = static_cast<long long>(sms) * 8;
+  return launch(pkv::swap_blocks_kernel, dim3(static_cast<unsigned>(blocks)), dim3(256), 0,
+                static_cast<cudaStream_t>(stream), static_cast<uint4*>(dk), static_cast<uint4*>(dv),
+                static_cast<const uint4*>(sk), static_cast<const uint4*>(sv), static_cast<const int32_t*>(pp),
+                block_chunks, total, src_blocks, dst_blocks);
+}
+
+pkv_status pkv_swap_blocks_check(const int32_t* pairs_host, int num_pairs, int src_blocks, int dst_blocks) {
+  if (num_pairs < 0 || src_blocks <= 0 || dst_blocks <= 0 || (num_pairs > 0 && pairs_host == nullptr))
+    return PKV_EINVAL;
+  std::unordered_set<int32_t> dsts;
+  for (int i = 0; i < num_pairs; ++i) {
+    const int32_t s = pairs_host[2 * i], d = pairs_host[2 * i + 1];
+    if (s < 0 || s >= src_blocks || d < 0 || d >= dst_blocks) return PKV_EINVAL;
+    if (!dsts.insert(d).second) return PKV_EINVAL;
+  }
   return PKV_OK;
 }
 
