@@ -112,6 +112,39 @@ pkv_status pkv_copy_blocks(void* k_cache, void* v_cache, const int32_t* pairs, i
 pkv_status pkv_copy_blocks_check(const int32_t* pairs_host, int num_pairs, int num_blocks);
 
 /* ------------------------------------------------------------------------
+ * pkv_swap_blocks -- block copy between two pools (preemption by swapping).
+ *
+ * "LLM Systems 24: Efficient LLM Inference with PagedAttention and vLLM" §3
+ * (conclusion): when the pool runs out of KV blocks a request is preempted;
+ * its blocks are swapped out to host memory and later swapped back in.
+ *
+ * For each pair (src, dst) in pairs[num_pairs][2]:
+ *   dst_k[dst] = src_k[src];  dst_v[dst] = src_v[src]
+ * (all num_kv_heads * 16 * head_dim elements; bit copy).  Both pools have
+ * the layout [blocks, num_kv_heads, 16, head_dim] of one dtype; the source
+ * has src_blocks blocks, the destination dst_blocks.  Each of the four
+ * cache pointers and `pairs` may be device memory of the current device
+ * or page-locked host memory mapped into the device's address space
+ * (cudaHostAlloc / cudaMallocHost, or cudaHostRegister'ed memory); pageable
+ * host memory, another device's memory or an unknown pointer returns
+ * PKV_EINVAL.  The pairs pkv_alloc_swap_out / pkv_alloc_swap_in report are
+ * (device, host) and (host, device) pairs for this call.  dst values must
+ * be distinct (pkv_swap_blocks_check) and the two pools must not overlap.
+ * A pair outside [0, src_blocks) x [0, dst_blocks) is skipped and sets
+ * PKV_ERR_COPY_RANGE.  Host memory is read or written by the kernel while
+ * it runs: keep it allocated and untouched by the host until the stream
+ * has passed the call.
+ * -------------------------------------------------------------------- */
+pkv_status pkv_swap_blocks(void* dst_k, void* dst_v, int dst_blocks, const void* src_k, const void* src_v,
+                           int src_blocks, const int32_t* pairs, int num_pairs, int num_kv_heads,
+                           int head_dim, pkv_dtype dtype, void* stream);
+
+/* Host-side check of swap pairs (host memory): src in [0, src_blocks), dst
+ * in [0, dst_blocks), dst ids distinct.  PKV_OK or PKV_EINVAL. */
+pkv_status pkv_swap_blocks_check(const int32_t* pairs_host, int num_pairs, int src_blocks, int dst_blocks);
+
+
+/* ------------------------------------------------------------------------
  * pkv_decode_workspace_bytes -- device workspace pkv_paged_attention_decode
  * needs for these sizes (0 when no sequence can span two partitions).
  * partition_tokens: 0 = PKV_DEFAULT_PARTITION, else a multiple of 16 in
@@ -308,7 +341,44 @@ pkv_status pkv_alloc_state(const pkv_alloc* a, int32_t* free_list, int* n_free,
                            int32_t* refcounts);
 int pkv_alloc_num_free(const pkv_alloc* a);
 int pkv_alloc_num_blocks(const pkv_alloc* a);
+/* Resident sequences (swapped ones not counted). */
 int pkv_alloc_num_seqs(const pkv_alloc* a);
+
+/* Preemption by swapping ("LLM Systems 24 ..." §3, conclusion).  The pages
+ * give no policy; this one is:
+ *   - a host-side pool of num_host_blocks blocks with its own FIFO free list
+ *     (0..num_host_blocks-1) and reference counts, set (or re-set) by
+ *     pkv_alloc_set_host_pool while no sequence is swapped out (else
+ *     EINVAL);
+ *   - swap_out(seq_ids[n]) (distinct, resident): every distinct device block
+ *     of the listed tables, in id order then table order, gets the next
+ *     free host block, and the pair (device, host) is written to
+ *     pairs[cap][2] (*n_pairs pairs).  A block shared by several listed
+ *     sequences maps to one host block that they share; each holder drops
+ *     one device reference (a block reaching 0 goes to the back of the
+ *     device free list; blocks shared with sequences not listed stay with
+ *     them) and the listed sequences become swapped;
+ *   - swap_in(seq_ids[n]) (distinct, swapped): the same with the roles of
+ *     the pools exchanged; pairs are (host, device);
+ *   - all or nothing: PKV_ENOMEM when the destination pool has too few free
+ *     blocks, PKV_EINVAL when cap is smaller than the number of pairs;
+ *   - a swapped sequence may only be freed (its host references are
+ *     dropped) or swapped in; append, step, fork and block_table reject it.
+ * The caller copies the pairs with pkv_swap_blocks: a swap-out's copy must
+ * be enqueued before anything that writes the released device blocks, a
+ * swap-in's before the sequence is next read. */
+pkv_status pkv_alloc_set_host_pool(pkv_alloc* a, int num_host_blocks);
+pkv_status pkv_alloc_swap_out(pkv_alloc* a, const int64_t* seq_ids, int n, int32_t* pairs, int cap,
+                              int* n_pairs);
+pkv_status pkv_alloc_swap_in(pkv_alloc* a, const int64_t* seq_ids, int n, int32_t* pairs, int cap,
+                             int* n_pairs);
+/* Host free list in order (free_list[num_host_blocks] may be NULL) and the
+ * count of every host block (refcounts[num_host_blocks] may be NULL). */
+pkv_status pkv_alloc_host_state(const pkv_alloc* a, int32_t* free_list, int* n_free, int32_t* refcounts);
+/* A swapped sequence's host table (up to cap entries), block count, length. */
+pkv_status pkv_alloc_swapped_table(const pkv_alloc* a, int64_t seq_id, int32_t* out, int cap, int* n_blocks,
+                                   int64_t* context_len);
+int pkv_alloc_num_swapped(const pkv_alloc* a);
 
 #ifdef __cplusplus
 }

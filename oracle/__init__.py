@@ -19,6 +19,10 @@ What each function follows (page titles as printed on the pages):
   "PagedAttention 与 vLLM 推理加速" §3.2(3) (shared blocks are only copied
   when a writer appends) and "LLM Systems 24 ..." §3 (reference counts and
   copy-on-write share KV blocks across samples).
+* ``RefAllocator.swap_out`` / ``swap_in`` and ``cache.swap_blocks`` --
+  "LLM Systems 24 ..." §3, conclusion (a request preempted for lack of KV
+  blocks is swapped out and later swapped back in); the policy details are
+  readings stated in ``allocator``.
 * ``brute.contiguous_decode`` -- the contiguous-cache baseline the pages
   contrast paging with ("PagedAttention 与 vLLM 推理加速" §2.2), in pure
   Python, used only to pin ``paged_decode`` on tiny inputs.
@@ -30,7 +34,7 @@ versus private-copy layouts, closed forms, and the pages' worked examples.
 
 from .storage import widen, nan_fill  # noqa: F401
 from .attention import paged_decode, decode_head  # noqa: F401
-from .cache import RefCache  # noqa: F401
+from .cache import RefCache, swap_blocks  # noqa: F401
 from .allocator import RefAllocator, RefAllocError  # noqa: F401
 from .brute import contiguous_decode  # noqa: F401
 from .replay import replay  # noqa: F401

@@ -27,6 +27,27 @@ What the pages leave open, read the plainest deterministic way:
 * slot = physical block * block_size + offset;
 * a call that fails (unknown or duplicate id, pool exhausted) raises and
   leaves every piece of state as it was.
+
+Preemption by swapping ("LLM Systems 24 ..." §3, conclusion: when the pool
+runs out of KV blocks a request is preempted and later swapped back in or
+recomputed).  The pages give no policy; the readings taken here:
+* a second, host-side pool of ``num_host_blocks`` blocks with its own FIFO
+  free list (0..n-1) and reference counts;
+* ``swap_out(ids)`` moves the listed resident sequences to the host pool:
+  every distinct device block their tables hold (in id order, then table
+  order) gets one host block, and the pair (device, host) is returned for
+  the caller to copy; a block that several listed sequences share maps to
+  one host block that they share; each holder drops one device reference
+  and a device block whose count reaches zero goes to the back of the
+  device free list (blocks shared with sequences not listed stay where
+  they are, still held by those);
+* ``swap_in(ids)`` is the mirror image: every distinct host block of the
+  listed swapped sequences gets a fresh device block (pair (host, device)),
+  host references are dropped the same way;
+* both are all or nothing; a swapped sequence can only be freed or swapped
+  in (no append, fork or step);
+* the copies of a swap-out must run before anything writes the device
+  blocks it released; those of a swap-in before the sequence is read.
 """
 from collections import deque
 
@@ -38,7 +59,7 @@ class RefAllocError(Exception):
 
 
 class RefAllocator:
-    def __init__(self, num_blocks: int, free_order=None, block_size: int = 16):
+    def __init__(self, num_blocks: int, free_order=None, block_size: int = 16, num_host_blocks: int = 0):
         if free_order is None:
             free_order = range(num_blocks)
         free_order = [int(x) for x in free_order]
@@ -50,16 +71,20 @@ class RefAllocator:
         self.refcount = [0] * num_blocks
         self.tables = {}  # seq id -> list of physical blocks
         self.lengths = {}  # seq id -> number of tokens
+        self.num_host_blocks = num_host_blocks
+        self.host_free = deque(range(num_host_blocks))
+        self.host_refcount = [0] * num_host_blocks
+        self.swapped = {}  # seq id -> (list of host blocks, number of tokens)
 
     # -- sequences ---------------------------------------------------------
     def add_seq(self, sid: int) -> None:
-        if sid in self.tables:
+        if sid in self.tables or sid in self.swapped:
             raise RefAllocError("inval", f"sequence {sid} exists")
         self.tables[sid] = []
         self.lengths[sid] = 0
 
     def fork(self, parent: int, child: int) -> None:
-        if parent not in self.tables or child in self.tables:
+        if parent not in self.tables or child in self.tables or child in self.swapped:
             raise RefAllocError("inval", f"fork {parent}->{child}")
         self.tables[child] = list(self.tables[parent])
         self.lengths[child] = self.lengths[parent]
@@ -67,6 +92,12 @@ class RefAllocator:
             self.refcount[blk] += 1
 
     def free_seq(self, sid: int) -> None:
+        if sid in self.swapped:
+            for blk in self.swapped.pop(sid)[0]:
+                self.host_refcount[blk] -= 1
+                if self.host_refcount[blk] == 0:
+                    self.host_free.append(blk)
+            return
         if sid not in self.tables:
             raise RefAllocError("inval", f"unknown sequence {sid}")
         for blk in self.tables.pop(sid):
@@ -158,6 +189,69 @@ class RefAllocator:
             if c is not None:
                 cows.append(c)
         return slots, cows
+
+    # -- preemption by swapping ------------------------------------------------
+    @staticmethod
+    def _move(sids, table_of, src_ref, src_free, dst_ref, dst_free):
+        """Give every distinct block of the listed tables a block popped from
+        dst_free; drop the holders' references on the source side.  Returns
+        (pairs, new tables).  The caller has checked that dst_free suffices."""
+        mapping, pairs, tables = {}, [], []
+        for s in sids:
+            new = []
+            for blk in table_of(s):
+                if blk not in mapping:
+                    mapping[blk] = dst_free.popleft()
+                    pairs.append((blk, mapping[blk]))
+                new.append(mapping[blk])
+            tables.append(new)
+        for s, new in zip(sids, tables):
+            for blk, nb in zip(table_of(s), new):
+                dst_ref[nb] += 1
+                src_ref[blk] -= 1
+                if src_ref[blk] == 0:
+                    src_free.append(blk)
+        return pairs, tables
+
+    def swap_out(self, sids):
+        """Move resident sequences to the host pool; return the (device block,
+        host block) pairs to copy.  All or nothing."""
+        sids = list(sids)
+        if len(set(sids)) != len(sids) or any(s not in self.tables for s in sids):
+            raise RefAllocError("inval", "swap_out ids must be distinct, resident sequences")
+        need = len({b for s in sids for b in self.tables[s]})
+        if need > len(self.host_free):
+            raise RefAllocError("nomem", "host pool exhausted")
+        pairs, tables = self._move(sids, lambda s: self.tables[s], self.refcount, self.free, self.host_refcount,
+                                   self.host_free)
+        for s, t in zip(sids, tables):
+            self.swapped[s] = (t, self.lengths.pop(s))
+            del self.tables[s]
+        return pairs
+
+    def swap_in(self, sids):
+        """Bring swapped sequences back to the device pool; return the (host
+        block, device block) pairs to copy.  All or nothing."""
+        sids = list(sids)
+        if len(set(sids)) != len(sids) or any(s not in self.swapped for s in sids):
+            raise RefAllocError("inval", "swap_in ids must be distinct, swapped sequences")
+        need = len({b for s in sids for b in self.swapped[s][0]})
+        if need > len(self.free):
+            raise RefAllocError("nomem", "pool exhausted")
+        pairs, tables = self._move(sids, lambda s: self.swapped[s][0], self.host_refcount, self.host_free,
+                                   self.refcount, self.free)
+        for s, t in zip(sids, tables):
+            self.tables[s] = t
+            self.lengths[s] = self.swapped.pop(s)[1]
+        return pairs
+
+    def host_state(self):
+        """(host free list in order, host refcount of every host block)."""
+        return list(self.host_free), list(self.host_refcount)
+
+    def swapped_table(self, sid: int):
+        t, n = self.swapped[sid]
+        return list(t), n
 
     # -- views ---------------------------------------------------------------
     def block_table(self, sid: int):

@@ -12,6 +12,9 @@ writes nothing.
   never copied).
 * copy_blocks -- "PagedAttention 与 vLLM 推理加速" §3.2(3): a shared block is
   copied only when a writer is about to append into it (copy-on-write).
+* swap_blocks -- "LLM Systems 24 ..." §3, conclusion: a preempted request's
+  blocks are swapped out of the device pool and back in later; a block of
+  one pool is copied whole into a block of another pool of the same shape.
 """
 import numpy as np
 
@@ -55,3 +58,10 @@ class RefCache:
         for src, dst in pairs:
             self.k[int(dst)] = self.k[int(src)]
             self.v[int(dst)] = self.v[int(src)]
+
+
+def swap_blocks(dst: "RefCache", src: "RefCache", pairs) -> None:
+    """dst[d] = src[s] for each (s, d), K and V (pools of the same shape)."""
+    for s, d in pairs:
+        dst.k[int(d)] = src.k[int(s)]
+        dst.v[int(d)] = src.v[int(s)]

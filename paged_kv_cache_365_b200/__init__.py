@@ -1,6 +1,7 @@
 """B200-native paged KV-cache decode: slot-mapped append, copy-on-write block
-copy, paged single-query attention with split-K partitions, and a host block
-allocator -- behind the C ABI of libpkv.so (include/pkv.h).
+copy, paged single-query attention with split-K partitions, block swapping
+to a host pool, and a host block allocator -- behind the C ABI of libpkv.so
+(include/pkv.h).
 
 Importing the package loads libpkv.so; it raises ImportError when the library
 has not been built.  There is no CPU or Python fallback.
@@ -10,4 +11,4 @@ from ._lib import (ERR_BLOCK_RANGE, ERR_CONTEXT_RANGE, ERR_COPY_RANGE, ERR_SLOT_
 from .api import (BLOCK_SIZE, DEFAULT_PARTITION, BlockAllocator, PagedKVCache, copy_blocks,  # noqa: F401
                   copy_blocks_check, decode_workspace_bytes, get_error, kv_append, kv_cache_bytes,
                   paged_attention_decode, paged_attention_decode_static_ws, paged_attention_decode_prefix,
-                  decode_prefix_workspace_bytes, common_prefix_pages)
+                  decode_prefix_workspace_bytes, common_prefix_pages, swap_blocks, swap_blocks_check)

@@ -33,6 +33,9 @@ PROTOTYPES = {
     "pkv_copy_blocks": (c_int, [c_void_p, c_void_p, c_void_p, c_int, c_int, c_int, c_int, c_int,
                                 c_void_p]),
     "pkv_copy_blocks_check": (c_int, [P(c_int32), c_int, c_int]),
+    "pkv_swap_blocks": (c_int, [c_void_p, c_void_p, c_int, c_void_p, c_void_p, c_int, c_void_p, c_int, c_int,
+                                c_int, c_int, c_void_p]),
+    "pkv_swap_blocks_check": (c_int, [P(c_int32), c_int, c_int, c_int]),
     "pkv_decode_workspace_bytes": (c_size_t, [c_int, c_int, c_int, c_int, c_int]),
     "pkv_paged_attention_decode": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_int,
                                            c_void_p, c_int, c_int, c_int, c_int, c_int, c_int,
@@ -60,6 +63,12 @@ PROTOTYPES = {
     "pkv_alloc_num_free": (c_int, [c_void_p]),
     "pkv_alloc_num_blocks": (c_int, [c_void_p]),
     "pkv_alloc_num_seqs": (c_int, [c_void_p]),
+    "pkv_alloc_set_host_pool": (c_int, [c_void_p, c_int]),
+    "pkv_alloc_swap_out": (c_int, [c_void_p, P(c_int64), c_int, P(c_int32), c_int, P(c_int)]),
+    "pkv_alloc_swap_in": (c_int, [c_void_p, P(c_int64), c_int, P(c_int32), c_int, P(c_int)]),
+    "pkv_alloc_host_state": (c_int, [c_void_p, P(c_int32), P(c_int), P(c_int32)]),
+    "pkv_alloc_swapped_table": (c_int, [c_void_p, c_int64, P(c_int32), c_int, P(c_int), P(c_int64)]),
+    "pkv_alloc_num_swapped": (c_int, [c_void_p]),
 }
 
 

@@ -97,6 +97,48 @@ def copy_blocks(k_cache: torch.Tensor, v_cache: torch.Tensor, pairs: torch.Tenso
                               _stream(stream, k_cache.device)), "pkv_copy_blocks")
 
 
+def _any(t: torch.Tensor, name: str, dtype=None) -> int:
+    """Device tensor, or page-locked host tensor (the library maps it)."""
+    if not isinstance(t, torch.Tensor) or not (t.is_cuda or t.is_pinned()):
+        raise ValueError(f"{name} must be a CUDA tensor or a pinned host tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    return t.data_ptr()
+
+
+def swap_blocks_check(pairs_host: np.ndarray, src_blocks: int, dst_blocks: int) -> None:
+    """Host check of swap pairs (ids in range, distinct dst)."""
+    p = np.ascontiguousarray(pairs_host, dtype=np.int32).reshape(-1, 2)
+    check(lib.pkv_swap_blocks_check(p.ctypes.data_as(ctypes.POINTER(ctypes.c_int32)), p.shape[0], src_blocks,
+                                    dst_blocks), "pkv_swap_blocks_check")
+
+
+def swap_blocks(dst_k: torch.Tensor, dst_v: torch.Tensor, src_k: torch.Tensor, src_v: torch.Tensor,
+                pairs: torch.Tensor, stream=None, device=None) -> None:
+    """dst[d] = src[s] for each (s, d) row of int32 ``pairs`` [n, 2], K and V.
+
+    Each pool is [blocks, Hkv, 16, D] on the device or in pinned host memory
+    (preemption by swapping); ``pairs`` on the device or pinned.  Runs on the
+    current stream of ``device`` (default: the device of a CUDA operand)."""
+    dnb, hkv, d = _cache_dims(dst_k, dst_v)
+    snb, shkv, sd = _cache_dims(src_k, src_v)
+    if (shkv, sd) != (hkv, d) or src_k.dtype != dst_k.dtype:
+        raise ValueError("source and destination pools must share Hkv, D and dtype")
+    if pairs.dim() != 2 or pairs.shape[1] != 2:
+        raise ValueError("pairs must be [n, 2]")
+    n = pairs.shape[0]
+    if n == 0:
+        return
+    if device is None:
+        cuda = [t for t in (dst_k, src_k, pairs) if t.is_cuda]
+        device = cuda[0].device if cuda else torch.device("cuda", torch.cuda.current_device())
+    check(lib.pkv_swap_blocks(_any(dst_k, "dst_k"), _any(dst_v, "dst_v"), dnb, _any(src_k, "src_k"),
+                              _any(src_v, "src_v"), snb, _any(pairs, "pairs", torch.int32), n, hkv, d,
+                              _DT[dst_k.dtype], _stream(stream, device)), "pkv_swap_blocks")
+
+
 def decode_workspace_bytes(num_seqs: int, num_q_heads: int, head_dim: int, max_context_len: int,
                            partition: int = 0) -> int:
     return int(lib.pkv_decode_workspace_bytes(num_seqs, num_q_heads, head_dim, max_context_len, partition))
@@ -292,7 +334,50 @@ class BlockAllocator:
 
     @property
     def num_seqs(self) -> int:
+        """Resident sequences (swapped ones not counted)."""
         return int(lib.pkv_alloc_num_seqs(self._h))
+
+    # -- preemption by swapping --------------------------------------------
+    def set_host_pool(self, num_host_blocks: int) -> None:
+        check(lib.pkv_alloc_set_host_pool(self._h, int(num_host_blocks)), "pkv_alloc_set_host_pool")
+        self.num_host_blocks = int(num_host_blocks)
+
+    def _swap(self, fn, name, sids) -> np.ndarray:
+        ids = np.ascontiguousarray(list(sids), dtype=np.int64)
+        cap = max(self.num_blocks, getattr(self, "num_host_blocks", 0), 1)
+        pairs = np.empty((cap, 2), dtype=np.int32)
+        n = ctypes.c_int()
+        check(fn(self._h, _i64p(ids), ids.shape[0], _i32p(pairs), cap, ctypes.byref(n)), name)
+        return pairs[:n.value]
+
+    def swap_out(self, sids: Iterable[int]) -> np.ndarray:
+        """Move resident sequences to the host pool; (device, host) pairs [n, 2]."""
+        return self._swap(lib.pkv_alloc_swap_out, "pkv_alloc_swap_out", sids)
+
+    def swap_in(self, sids: Iterable[int]) -> np.ndarray:
+        """Bring swapped sequences back; (host, device) pairs [n, 2]."""
+        return self._swap(lib.pkv_alloc_swap_in, "pkv_alloc_swap_in", sids)
+
+    def host_state(self) -> Tuple[List[int], List[int]]:
+        nh = getattr(self, "num_host_blocks", 0)
+        free = np.empty(max(nh, 1), dtype=np.int32)
+        rc = np.empty(max(nh, 1), dtype=np.int32)
+        nf = ctypes.c_int()
+        check(lib.pkv_alloc_host_state(self._h, _i32p(free), ctypes.byref(nf), _i32p(rc)), "pkv_alloc_host_state")
+        return [int(x) for x in free[:nf.value]], [int(x) for x in rc[:nh]]
+
+    def swapped_table(self, sid: int) -> Tuple[List[int], int]:
+        nb, ln = ctypes.c_int(), ctypes.c_int64()
+        check(lib.pkv_alloc_swapped_table(self._h, int(sid), None, 0, ctypes.byref(nb), ctypes.byref(ln)),
+              "pkv_alloc_swapped_table")
+        out = np.empty(max(nb.value, 1), dtype=np.int32)
+        check(lib.pkv_alloc_swapped_table(self._h, int(sid), _i32p(out), nb.value, ctypes.byref(nb),
+                                          ctypes.byref(ln)), "pkv_alloc_swapped_table")
+        return [int(x) for x in out[:nb.value]], int(ln.value)
+
+    @property
+    def num_swapped(self) -> int:
+        return int(lib.pkv_alloc_num_swapped(self._h))
 
 
 # ---------------------------------------------------------------------------
@@ -334,6 +419,31 @@ class PagedKVCache:
 
     def free_seq(self, sid):
         self.alloc.free_seq(sid)
+
+    # preemption by swapping
+    def enable_swap(self, num_host_blocks: int) -> None:
+        """Give the cache a pinned host pool of ``num_host_blocks`` blocks."""
+        shape = (int(num_host_blocks), self.Hkv, BLOCK_SIZE, self.D)
+        self.host_k = torch.empty(shape, dtype=self.dtype, pin_memory=True)
+        self.host_v = torch.empty(shape, dtype=self.dtype, pin_memory=True)
+        self.alloc.set_host_pool(num_host_blocks)
+
+    def swap_out(self, seq_ids: Sequence[int], stream=None) -> np.ndarray:
+        """Preempt sequences: their blocks go to the host pool (copied on the
+        stream before anything later on it can reuse the released blocks)."""
+        pairs = self.alloc.swap_out(seq_ids)
+        if len(pairs):
+            swap_blocks(self.host_k, self.host_v, self.k, self.v,
+                        torch.from_numpy(np.ascontiguousarray(pairs)).to(self.device), stream, self.device)
+        return pairs
+
+    def swap_in(self, seq_ids: Sequence[int], stream=None) -> np.ndarray:
+        """Bring preempted sequences back into the device pool."""
+        pairs = self.alloc.swap_in(seq_ids)
+        if len(pairs):
+            swap_blocks(self.k, self.v, self.host_k, self.host_v,
+                        torch.from_numpy(np.ascontiguousarray(pairs)).to(self.device), stream, self.device)
+        return pairs
 
     def prefill(self, sid: int, k: torch.Tensor, v: torch.Tensor, stream=None) -> np.ndarray:
         """Append n tokens' K/V ([n, Hkv, D]) to one sequence."""

@@ -8,6 +8,11 @@
 // Inference with PagedAttention and vLLM" §3).  The policy for the parts the
 // pages leave open is stated in pkv.h.  Every call validates first and
 // mutates only once it cannot fail, so a failed call changes nothing.
+//
+// Preemption by swapping ("LLM Systems 24 ..." §3, conclusion): a second,
+// host-side pool with its own FIFO free list and counts; swap-out moves the
+// listed sequences' blocks there, swap-in brings them back, both returning
+// the block pairs for the caller to copy.
 
 #include <climits>
 #include <cstdint>
@@ -58,8 +63,15 @@ struct pkv_alloc {
   FreeRing free_list;
   std::vector<int32_t> refcount;
   std::unordered_map<int64_t, Seq> seqs;
+  // host-side swap pool
+  int num_host_blocks = 0;
+  FreeRing host_free{0};
+  std::vector<int32_t> host_refcount;
+  std::unordered_map<int64_t, Seq> swapped;  // tables hold host block ids
 
   explicit pkv_alloc(int nb) : num_blocks(nb), free_list(nb), refcount(static_cast<size_t>(nb), 0) {}
+
+  bool known(int64_t id) const { return seqs.count(id) != 0 || swapped.count(id) != 0; }
 
   // Does appending to s take a block?  `count` gives the (possibly
   // adjusted) reference count of a block.
@@ -118,7 +130,7 @@ pkv_status pkv_alloc_create(int num_blocks, const int32_t* initial_free_order, p
 void pkv_alloc_destroy(pkv_alloc* a) { delete a; }
 
 pkv_status pkv_alloc_add_seq(pkv_alloc* a, int64_t seq_id) {
-  if (a == nullptr || a->seqs.count(seq_id)) return PKV_EINVAL;
+  if (a == nullptr || a->known(seq_id)) return PKV_EINVAL;
   a->seqs.emplace(seq_id, Seq{});
   return PKV_OK;
 }
@@ -126,7 +138,7 @@ pkv_status pkv_alloc_add_seq(pkv_alloc* a, int64_t seq_id) {
 pkv_status pkv_alloc_fork(pkv_alloc* a, int64_t parent, int64_t child) {
   if (a == nullptr) return PKV_EINVAL;
   auto it = a->seqs.find(parent);
-  if (it == a->seqs.end() || a->seqs.count(child)) return PKV_EINVAL;
+  if (it == a->seqs.end() || a->known(child)) return PKV_EINVAL;
   Seq copy = it->second;
   for (int32_t blk : copy.table) a->refcount[blk] += 1;
   a->seqs.emplace(child, std::move(copy));
@@ -135,6 +147,14 @@ pkv_status pkv_alloc_fork(pkv_alloc* a, int64_t parent, int64_t child) {
 
 pkv_status pkv_alloc_free_seq(pkv_alloc* a, int64_t seq_id) {
   if (a == nullptr) return PKV_EINVAL;
+  auto sw = a->swapped.find(seq_id);
+  if (sw != a->swapped.end()) {
+    for (int32_t blk : sw->second.table) {
+      if (--a->host_refcount[blk] == 0) a->host_free.push_back(blk);
+    }
+    a->swapped.erase(sw);
+    return PKV_OK;
+  }
   auto it = a->seqs.find(seq_id);
   if (it == a->seqs.end()) return PKV_EINVAL;
   for (int32_t blk : it->second.table) {
@@ -280,5 +300,120 @@ pkv_status pkv_alloc_state(const pkv_alloc* a, int32_t* free_list, int* n_free, 
 int pkv_alloc_num_free(const pkv_alloc* a) { return a ? a->free_list.size() : -1; }
 int pkv_alloc_num_blocks(const pkv_alloc* a) { return a ? a->num_blocks : -1; }
 int pkv_alloc_num_seqs(const pkv_alloc* a) { return a ? static_cast<int>(a->seqs.size()) : -1; }
+
+// ---- preemption by swapping -------------------------------------------------
+
+pkv_status pkv_alloc_set_host_pool(pkv_alloc* a, int num_host_blocks) {
+  if (a == nullptr || num_host_blocks < 0 || !a->swapped.empty()) return PKV_EINVAL;
+  FreeRing ring(num_host_blocks);
+  for (int i = 0; i < num_host_blocks; ++i) ring.push_back(i);
+  a->host_free = std::move(ring);
+  a->host_refcount.assign(static_cast<size_t>(num_host_blocks), 0);
+  a->num_host_blocks = num_host_blocks;
+  return PKV_OK;
+}
+
+namespace {
+
+// Move the listed sequences from `from` (tables over the source pool) to
+// `to` (tables over the destination pool): every distinct source block, in
+// id order then table order, gets one block popped from `dst_free`; every
+// holder drops one source reference (a block reaching zero goes to the back
+// of `src_free`) and adds one destination reference.  Validates first: ids
+// distinct and in `from`, the destination pool and `cap` large enough.
+pkv_status move_seqs(std::unordered_map<int64_t, Seq>& from, std::unordered_map<int64_t, Seq>& to,
+                     std::vector<int32_t>& src_ref, FreeRing& src_free, std::vector<int32_t>& dst_ref,
+                     FreeRing& dst_free, const int64_t* seq_ids, int n, int32_t* pairs, int cap, int* n_pairs) {
+  if (n < 0 || n_pairs == nullptr || cap < 0 || (n > 0 && seq_ids == nullptr) || (cap > 0 && pairs == nullptr))
+    return PKV_EINVAL;
+  std::vector<Seq*> list(static_cast<size_t>(n));
+  std::unordered_set<int64_t> seen;
+  std::unordered_set<int32_t> distinct;
+  for (int i = 0; i < n; ++i) {
+    auto it = from.find(seq_ids[i]);
+    if (it == from.end() || !seen.insert(seq_ids[i]).second) return PKV_EINVAL;
+    list[i] = &it->second;
+    for (int32_t b : it->second.table) distinct.insert(b);
+  }
+  const int64_t need = static_cast<int64_t>(distinct.size());
+  if (need > cap) return PKV_EINVAL;
+  if (need > dst_free.size()) return PKV_ENOMEM;
+  std::unordered_map<int32_t, int32_t> map;
+  map.reserve(distinct.size() * 2);
+  int np = 0;
+  std::vector<Seq> moved(static_cast<size_t>(n));
+  for (int i = 0; i < n; ++i) {
+    moved[i].len = list[i]->len;
+    moved[i].table.reserve(list[i]->table.size());
+    for (int32_t b : list[i]->table) {
+      auto m = map.find(b);
+      int32_t nb;
+      if (m == map.end()) {
+        nb = dst_free.pop_front();
+        map.emplace(b, nb);
+        pairs[2 * np] = b;
+        pairs[2 * np + 1] = nb;
+        ++np;
+      } else {
+        nb = m->second;
+      }
+      moved[i].table.push_back(nb);
+    }
+  }
+  for (int i = 0; i < n; ++i) {
+    for (size_t j = 0; j < list[i]->table.size(); ++j) {
+      dst_ref[moved[i].table[j]] += 1;
+      const int32_t b = list[i]->table[j];
+      if (--src_ref[b] == 0) src_free.push_back(b);
+    }
+  }
+  for (int i = 0; i < n; ++i) {
+    from.erase(seq_ids[i]);
+    to.emplace(seq_ids[i], std::move(moved[i]));
+  }
+  *n_pairs = np;
+  return PKV_OK;
+}
+
+}  // namespace
+
+pkv_status pkv_alloc_swap_out(pkv_alloc* a, const int64_t* seq_ids, int n, int32_t* pairs, int cap, int* n_pairs) {
+  if (a == nullptr) return PKV_EINVAL;
+  return move_seqs(a->seqs, a->swapped, a->refcount, a->free_list, a->host_refcount, a->host_free, seq_ids, n,
+                   pairs, cap, n_pairs);
+}
+
+pkv_status pkv_alloc_swap_in(pkv_alloc* a, const int64_t* seq_ids, int n, int32_t* pairs, int cap, int* n_pairs) {
+  if (a == nullptr) return PKV_EINVAL;
+  return move_seqs(a->swapped, a->seqs, a->host_refcount, a->host_free, a->refcount, a->free_list, seq_ids, n,
+                   pairs, cap, n_pairs);
+}
+
+pkv_status pkv_alloc_host_state(const pkv_alloc* a, int32_t* free_list, int* n_free, int32_t* refcounts) {
+  if (a == nullptr) return PKV_EINVAL;
+  const int nf = a->host_free.size();
+  if (n_free) *n_free = nf;
+  if (free_list)
+    for (int i = 0; i < nf; ++i) free_list[i] = a->host_free.at(i);
+  if (refcounts && !a->host_refcount.empty())
+    std::memcpy(refcounts, a->host_refcount.data(), sizeof(int32_t) * a->host_refcount.size());
+  return PKV_OK;
+}
+
+pkv_status pkv_alloc_swapped_table(const pkv_alloc* a, int64_t seq_id, int32_t* out, int cap, int* n_blocks,
+                                   int64_t* context_len) {
+  if (a == nullptr || cap < 0 || (cap > 0 && out == nullptr)) return PKV_EINVAL;
+  auto it = a->swapped.find(seq_id);
+  if (it == a->swapped.end()) return PKV_EINVAL;
+  const Seq& s = it->second;
+  const int nb = static_cast<int>(s.table.size());
+  if (n_blocks) *n_blocks = nb;
+  if (context_len) *context_len = s.len;
+  const int m = nb < cap ? nb : cap;
+  if (m > 0) std::memcpy(out, s.table.data(), sizeof(int32_t) * static_cast<size_t>(m));
+  return PKV_OK;
+}
+
+int pkv_alloc_num_swapped(const pkv_alloc* a) { return a ? static_cast<int>(a->swapped.size()) : -1; }
 
 }  // extern "C"

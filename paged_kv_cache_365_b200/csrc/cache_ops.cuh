@@ -1,6 +1,7 @@
-// Slot-mapped append of new tokens' K/V and copy-on-write block copy.
+// Slot-mapped append of new tokens' K/V, copy-on-write block copy, and the
+// block copy between the device pool and a host pool (swap).
 //
-// Both are bit copies of 16-byte chunks: one thread moves one chunk, so a
+// All are bit copies of 16-byte chunks: one thread moves one chunk, so a
 // warp moves 512 contiguous bytes of a row (append) or of a block (copy),
 // fully coalesced on both sides.
 #pragma once
@@ -74,6 +75,51 @@ __global__ void __launch_bounds__(256)
     for (int u = 0; u < kUnroll; ++u) {
       const long long i = base + static_cast<long long>(u) * blockDim.x;
       if (i < block_chunks) to[i] = v[u];
+    }
+  }
+}
+
+// "LLM Systems 24: Efficient LLM Inference with PagedAttention and vLLM" §3
+// (conclusion): a request preempted for lack of KV blocks is swapped out
+// and later swapped back in.  dst[d] = src[s] for each pair (s, d), K and V;
+// either pool may be page-locked host memory mapped into the device's
+// address space (the kernel then reads or writes it over the host link).
+// The (pair, K|V, chunk) space is walked by a grid-stride loop with kUnroll
+// independent loads in flight per thread before the stores, so a slow link
+// still sees enough outstanding requests.
+__global__ void __launch_bounds__(256)
+    swap_blocks_kernel(uint4* __restrict__ dst_k, uint4* __restrict__ dst_v, const uint4* __restrict__ src_k,
+                       const uint4* __restrict__ src_v, const int32_t* __restrict__ pairs, long long block_chunks,
+                       long long total /* num_pairs * block_chunks */, int src_blocks, int dst_blocks) {
+  pdl_enter();
+  constexpr int kUnroll = 4;
+  const long long stride = static_cast<long long>(gridDim.x) * blockDim.x;
+  for (long long base = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; base < 2 * total;
+       base += stride * kUnroll) {
+    uint4 v[kUnroll];
+    long long to[kUnroll];  // destination chunk; -1: nothing to store
+    bool is_v[kUnroll];
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u) {
+      const long long i = base + u * stride;
+      to[u] = -1;
+      is_v[u] = i >= total;
+      if (i >= 2 * total) continue;
+      const long long j = is_v[u] ? i - total : i;
+      const long long p = j / block_chunks;
+      const long long c = j - p * block_chunks;
+      const int s = pairs[2 * p];
+      const int d = pairs[2 * p + 1];
+      if (s < 0 || s >= src_blocks || d < 0 || d >= dst_blocks) {
+        if (c == 0) raise_error(PKV_ERR_COPY_RANGE);
+        continue;
+      }
+      v[u] = (is_v[u] ? src_v : src_k)[static_cast<long long>(s) * block_chunks + c];
+      to[u] = static_cast<long long>(d) * block_chunks + c;
+    }
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u) {
+      if (to[u] >= 0) (is_v[u] ? dst_v : dst_k)[to[u]] = v[u];
     }
   }
 }
