@@ -12,6 +12,10 @@ What each function follows (page titles as printed on the pages):
   table, Q x K gives the attention scores) and §1 (each new token attends
   over every earlier token's K/V, itself included); the softmax and the
   weighted sum of V are the standard scaled-dot-product attention.
+* ``attention.paged_multi`` -- several query tokens per sequence (the
+  verification pass of speculative decoding, "PagedAttention 与 vLLM 推理
+  加速" §6; prefill chunks in mixed batches, "LLM Systems 24 ..."
+  §2.2.1.3), each attending causally over its sequence's tokens.
 * ``cache.RefCache.append`` -- "vLLM + PagedAttention：打造高并发LLM推理引擎",
   "它是怎么工作的": the page table records which block token n lives in;
   a new token is written into its slot, old tokens are never moved.
@@ -33,7 +37,7 @@ versus private-copy layouts, closed forms, and the pages' worked examples.
 """
 
 from .storage import widen, nan_fill  # noqa: F401
-from .attention import paged_decode, decode_head  # noqa: F401
+from .attention import paged_decode, paged_multi, decode_head  # noqa: F401
 from .cache import RefCache, swap_blocks  # noqa: F401
 from .allocator import RefAllocator, RefAllocError  # noqa: F401
 from .brute import contiguous_decode  # noqa: F401

@@ -14,6 +14,14 @@ over the K/V of every token so far, itself included.  The softmax is the
 standard one, computed max-subtracted so exp never overflows.  A sequence
 with no tokens yields zeros.  Block-table entries past the sequence's last
 page, and the unused slots of its last block, are never read.
+
+Several query tokens per sequence (``paged_multi``): "PagedAttention 与 vLLM
+推理加速" §6 (the large model verifies the small model's guessed tokens --
+several new tokens of one sequence scored in one pass) and "LLM Systems 24
+..." §2.2.1.3 (batches that mix prefill chunks and decode steps).  Query
+token i of a sequence with n new tokens sits at position ctx - n + i and,
+by §1's rule (a token attends over every token so far, itself included),
+attends over positions 0..ctx - n + i and no later ones.
 """
 import numpy as np
 
@@ -60,4 +68,39 @@ def paged_decode(q, k_cache, v_cache, block_tables, context_lens, scale, dtype,
             values = widen(_gather(v_cache, pages, g, n, block_size), dtype)
             for h in range(g * G, (g + 1) * G):
                 out[b, h] = decode_head(qb[h], keys, values, scale)
+    return out
+
+
+def paged_multi(q, k_cache, v_cache, block_tables, context_lens, query_start, scale, dtype,
+                block_size=16, seqs=None):
+    """float64 output [T, Hq, D] for T = query_start[-1] query tokens.
+
+    Rows query_start[b] .. query_start[b+1]-1 of q [T, Hq, D] are sequence
+    b's n_b new tokens, the last n_b of its context_lens[b] tokens; row
+    query_start[b] + i attends over the sequence's tokens 0 .. ctx - n_b + i.
+    A row whose position would be negative (n_b > ctx) yields zeros.
+    ``seqs`` restricts the work to those sequences (other rows stay NaN).
+    """
+    T, Hq, D = q.shape
+    Hkv = k_cache.shape[1]
+    G = Hq // Hkv
+    out = np.full((T, Hq, D), np.nan, dtype=np.float64)
+    B = len(context_lens)
+    for b in (range(B) if seqs is None else seqs):
+        n = int(context_lens[b])
+        r0, r1 = int(query_start[b]), int(query_start[b + 1])
+        nq = r1 - r0
+        n_pages = -(-n // block_size)
+        pages = np.asarray(block_tables[b][:n_pages], dtype=np.int64)
+        for g in range(Hkv):
+            keys = widen(_gather(k_cache, pages, g, n, block_size), dtype)
+            values = widen(_gather(v_cache, pages, g, n, block_size), dtype)
+            for i in range(nq):
+                pos = n - nq + i
+                qi = widen(q[r0 + i], dtype)
+                for h in range(g * G, (g + 1) * G):
+                    if pos < 0:
+                        out[r0 + i, h] = 0.0
+                    else:
+                        out[r0 + i, h] = decode_head(qi[h], keys[:pos + 1], values[:pos + 1], scale)
     return out

@@ -1,6 +1,8 @@
 """Test-side helpers shared by the oracle pins and the GPU parity tests."""
 import numpy as np
 
+import oracle
+
 
 def logical_token_ids(wl):
     """For each step sequence, the ids of its tokens in logical order.
@@ -81,3 +83,38 @@ def privatise(cache_k, cache_v, tables, context_lens, block_size=16):
             t2[b, j] = nxt
             nxt += 1
     return k2, v2, t2
+
+
+def make_multi_case(ctx, nq, Hq, Hkv, D, dtype, seed):
+    """Pool, tables and values for sequences of lengths ``ctx`` (the last
+    ``nq[b]`` tokens being the new ones); blocks placed by a permutation."""
+    rng = np.random.default_rng(seed)
+    pages = [-(-c // 16) for c in ctx]
+    nb = sum(pages) + 5
+    perm = rng.permutation(nb)
+    store = {"f32": np.float32, "f16": np.float16, "bf16": np.float32}[dtype]
+    k = oracle.nan_fill((nb, Hkv, 16, D), dtype)
+    v = oracle.nan_fill((nb, Hkv, 16, D), dtype)
+    W = max(pages) + 2
+    tables = np.full((len(ctx), W), nb + 100, dtype=np.int32)
+    rows_k, rows_v = [], []
+    used = 0
+    for b, c in enumerate(ctx):
+        tables[b, :pages[b]] = perm[used:used + pages[b]]
+        used += pages[b]
+        kk = rng.standard_normal((c, Hkv, D)).astype(store)
+        vv = rng.standard_normal((c, Hkv, D)).astype(store)
+        if dtype == "bf16":  # keep the upper half: exact bf16 values
+            kk = (kk.view(np.uint32) >> 16).astype(np.uint16)
+            vv = (vv.view(np.uint32) >> 16).astype(np.uint16)
+        for j in range(c):
+            k[tables[b, j // 16], :, j % 16] = kk[j]
+            v[tables[b, j // 16], :, j % 16] = vv[j]
+        rows_k.append(kk)
+        rows_v.append(vv)
+    qs = np.concatenate([[0], np.cumsum(nq)]).astype(np.int32)
+    q = rng.standard_normal((int(qs[-1]), Hq, D)).astype(store)
+    if dtype == "bf16":
+        q = (q.view(np.uint32) >> 16).astype(np.uint16)
+    return dict(q=q, k=k, v=v, tables=tables, ctx=np.array(ctx, dtype=np.int32), qs=qs, rows_k=rows_k,
+                rows_v=rows_v, dtype=dtype, G=Hq // Hkv)
