@@ -11,6 +11,9 @@ idempotent).
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
   python bench.py --impl reference ...   (the fp64 CPU oracle, bounded sample)
+  python bench.py --row swap ...         (preemption by swapping: one step =
+      swap a quarter of the batch out to pinned host memory and back in;
+      GB/s over the host link against cudaMemcpyAsync of the same bytes)
 
 N > 1: one process per GPU (torchrun), each rank decoding its own replica
 batch (different seed), no collective on the data path; value = all ranks'
@@ -37,6 +40,7 @@ sys.path.insert(0, ROOT)
 import workloads  # noqa: E402
 
 METRIC = "paged decode attention: KV-cache HBM GB/s (% of peak), seq-steps/s"
+SWAP_METRIC = "block swap device<->pinned host (preempt + resume): GB/s over the host link"
 UNIT = "GB/s"
 FALLBACK_HBM_GBS = 6650.0
 STORAGE = {"f32": 4, "f16": 2, "bf16": 2}
@@ -342,6 +346,148 @@ def run_cuda(args, rank, world, local_rank):
 
 
 # ---------------------------------------------------------------------------
+# preemption by swapping: a quarter of the batch out to pinned host memory
+# and back in
+# ---------------------------------------------------------------------------
+def swap_plan(wl):
+    """Sequences a swap step preempts: the first quarter of the step batch."""
+    ids = [int(s) for s in wl.step_seqs]
+    return ids[:max(1, len(ids) // 4)]
+
+
+def run_swap(args, rank, world, local_rank):
+    import torch
+    from paged_kv_cache_365_b200.replay import build_step
+    import paged_kv_cache_365_b200 as pkv
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    wl = workloads.named(args.workload, replica_seed(args.seed, rank))
+    vals = device_values(wl, replica_seed(args.seed, rank), dev)
+    st = build_step(wl, {}, dev, device_values=vals)
+    del vals
+    cache = st["cache"]
+    stream = torch.cuda.current_stream(dev)
+    ids = swap_plan(wl)
+    n_host = sum(len(cache.alloc.block_table(s)[0]) for s in ids)
+    cache.enable_swap(n_host)
+    # one preempt/resume cycle planned on the host; its copies replayed
+    out_pairs = cache.alloc.swap_out(ids)
+    in_pairs = cache.alloc.swap_in(ids)
+    d_out = torch.from_numpy(np.ascontiguousarray(out_pairs)).to(dev)
+    d_in = torch.from_numpy(np.ascontiguousarray(in_pairs)).to(dev)
+    es = STORAGE[wl.dtype]
+    block_bytes = 2 * wl.Hkv * 16 * wl.D * es  # K and V
+    out_bytes, in_bytes = len(out_pairs) * block_bytes, len(in_pairs) * block_bytes
+
+    def swap_out():
+        pkv.swap_blocks(cache.host_k, cache.host_v, cache.k, cache.v, d_out, stream, dev)
+
+    def swap_in():
+        pkv.swap_blocks(cache.k, cache.v, cache.host_k, cache.host_v, d_in, stream, dev)
+
+    # the copy engine over the same link and bytes: cudaMemcpyAsync of one
+    # contiguous pinned buffer each way (the roofline's denominator)
+    dbuf = torch.empty(out_bytes, dtype=torch.uint8, device=dev)
+    hbuf = torch.empty(out_bytes, dtype=torch.uint8, pin_memory=True)
+
+    def timed(fn, K):
+        for _ in range(args.warmup):
+            fn()
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(K):
+            fn()
+        b.record(stream)
+        torch.cuda.synchronize()
+        return a.elapsed_time(b)
+
+    K = args.steps
+    with ClockSampler(local_rank) as clocks:
+        total_ms = timed(lambda: (swap_out(), swap_in()), K)
+    out_ms = timed(swap_out, K)
+    in_ms = timed(swap_in, K)
+    ce_d2h_ms = timed(lambda: hbuf.copy_(dbuf, non_blocking=True), K)
+    ce_h2d_ms = timed(lambda: dbuf.copy_(hbuf, non_blocking=True), K)
+    if pkv.get_error() != 0:
+        raise RuntimeError("device error flags raised during the swap timing")
+    # end to end through the public API: allocator plan + pairs upload +
+    # copies, every step (alternating device blocks, all valid)
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    for _ in range(args.warmup):
+        cache.swap_out(ids, stream)
+        cache.swap_in(ids, stream)
+    torch.cuda.synchronize()
+    t0.record(stream)
+    for _ in range(K):
+        cache.swap_out(ids, stream)
+        cache.swap_in(ids, stream)
+    t1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = t0.elapsed_time(t1)
+    total_ms, out_ms, in_ms, ce_d2h_ms, ce_h2d_ms, e2e_ms = max_over_ranks(
+        [total_ms, out_ms, in_ms, ce_d2h_ms, ce_h2d_ms, e2e_ms], world, dev)
+    return dict(wl=wl, K=K, ids=ids, out_bytes=out_bytes, in_bytes=in_bytes, total_ms=total_ms, out_ms=out_ms,
+                in_ms=in_ms, ce_d2h_ms=ce_d2h_ms, ce_h2d_ms=ce_h2d_ms, e2e_ms=e2e_ms, clocks=clocks.summary(),
+                n_pairs=(len(out_pairs), len(in_pairs)), block_bytes=block_bytes)
+
+
+def swap_cpu_baseline(wl, budget_s=3.0):
+    """The oracle's swap_blocks (numpy block copies) on a bounded sample."""
+    import oracle
+    n = 64
+    dev = oracle.RefCache(n, wl.Hkv, wl.D, wl.dtype)
+    host = oracle.RefCache(n, wl.Hkv, wl.D, wl.dtype)
+    pairs = [(i, (i * 7) % n) for i in range(n)]
+    block_bytes = 2 * wl.Hkv * 16 * wl.D * STORAGE[wl.dtype]
+    reps, t0 = 0, time.perf_counter()
+    while time.perf_counter() - t0 < budget_s:
+        oracle.swap_blocks(host, dev, pairs)
+        reps += 1
+    secs = time.perf_counter() - t0
+    return {"value": reps * n * block_bytes / secs / 1e9, "unit": UNIT, "cores": 1, "kind": "oracle",
+            "sample": f"{reps} x {n} blocks of workload {wl.name}'s shape copied between two numpy pools, "
+                      f"one thread, {secs:.1f} s"}
+
+
+def swap_line(args, r, world):
+    wl = r["wl"]
+    K = r["K"]
+    step_bytes = r["out_bytes"] + r["in_bytes"]
+    gbs = lambda b, ms: b * K / (ms / 1e3) / 1e9  # noqa: E731
+    # the memcpy buffers hold out_bytes; scale the inbound copy to in_bytes
+    ce_ms = r["ce_d2h_ms"] + r["ce_h2d_ms"] * r["in_bytes"] / max(1, r["out_bytes"])
+    achieved = gbs(step_bytes, r["out_ms"] + r["in_ms"])
+    peak = gbs(step_bytes, ce_ms)
+    line = {
+        "metric": SWAP_METRIC, "value": world * gbs(step_bytes, r["total_ms"]), "unit": UNIT, "n_gpus": world,
+        "steps": K, "warmup": args.warmup, "ms_per_step": r["total_ms"] / K, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": wl.dtype,
+        "data": "synthetic (seeded N(0,1) K/V on the device, seeded lengths and placement)",
+        "config": {"workload": f"{wl.name} preempt+resume", "swapped_seqs": len(r["ids"]),
+                   "blocks_out": r["n_pairs"][0], "blocks_in": r["n_pairs"][1], "block_bytes_kv": r["block_bytes"],
+                   "bytes_per_step": step_bytes, "num_kv_heads": wl.Hkv, "head_dim": wl.D, "seed": args.seed,
+                   "parallelism": f"replicas{args.gpus}" if args.gpus > 1 else "single-gpu",
+                   "l2": "device side larger than L2 (no flush)" if r["out_bytes"] > 126e6 else "fits in L2"},
+        "swap_out_gbs": gbs(r["out_bytes"], r["out_ms"]), "swap_in_gbs": gbs(r["in_bytes"], r["in_ms"]),
+        "memcpy_d2h_gbs": gbs(r["out_bytes"], r["ce_d2h_ms"]), "memcpy_h2d_gbs": gbs(r["out_bytes"], r["ce_h2d_ms"]),
+        "clocks": r["clocks"],
+        "e2e": {"value": world * gbs(step_bytes, r["e2e_ms"]), "unit": UNIT,
+                "h2d_bytes_per_step": r["in_bytes"] + 8 * sum(r["n_pairs"]),
+                "d2h_bytes_per_step": r["out_bytes"], "us_per_step": 1e3 * r["e2e_ms"] / K},
+        "gpu_launches": 2 * K,
+        "roofline": {"kernel": "swap_blocks_kernel (out + in)", "bound": "host link", "achieved": achieved,
+                     "peak": peak, "peak_kind": "cudaMemcpyAsync of the same bytes each way, this run",
+                     "unit": "GB/s", "frac": achieved / peak, "traffic": None,
+                     "algorithmic_bytes_per_launch": step_bytes / 2, "avg_launch_us": 1e3 * (r["out_ms"] + r["in_ms"]) / (2 * K)},
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = swap_cpu_baseline(wl)
+    return line
+
+
+# ---------------------------------------------------------------------------
 # the oracle on the host cores
 # ---------------------------------------------------------------------------
 def oracle_units_timed(wl, ref, vals, units):
@@ -442,6 +588,16 @@ def run_reference(args, rank, world):
     if rank != 0:
         return
     wl = workloads.named(args.workload, args.seed)
+    if getattr(args, "row", "step") == "swap":
+        b = swap_cpu_baseline(wl, budget_s=min(60.0, 0.5 * (args.steps + args.warmup)))
+        print(json.dumps({"impl": "reference", "metric": SWAP_METRIC, "value": b["value"], "unit": UNIT,
+                          "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup, "ms_per_step": None,
+                          "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": wl.dtype,
+                          "data": "synthetic", "config": {"workload": f"{wl.name} preempt+resume"},
+                          "cpu_baseline": b,
+                          "e2e": {"value": b["value"], "unit": UNIT, "h2d_bytes_per_step": 0,
+                                  "d2h_bytes_per_step": 0}}), flush=True)
+        return
     limits = blas_threads()
     ctx = limits(limits=1) if limits else None
     if ctx:
@@ -478,7 +634,7 @@ def run_reference(args, rank, world):
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--steps", type=int, default=None, help="timed steps (default 2000; 20 with --row swap)")
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="llama7b", choices=sorted(workloads.NAMED))
@@ -489,7 +645,11 @@ def main(argv=None):
                     help="capture one step in a CUDA graph and replay it (launch-bound batches)")
     ap.add_argument("--no-cascade", action="store_true",
                     help="decode a shared-prefix batch with the plain paged kernel")
+    ap.add_argument("--row", choices=["step", "swap"], default="step",
+                    help="step: the decode step (default); swap: preemption by swapping")
     args = ap.parse_args(argv)
+    if args.steps is None:
+        args.steps = 20 if args.row == "swap" else 2000
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
 
@@ -506,10 +666,14 @@ def main(argv=None):
         torch.cuda.set_device(local_rank)
         torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                              device_id=torch.device("cuda", local_rank))
-    try:
-        r = run_cuda(args, rank, world, local_rank)
-    finally:
-        pass
+    if args.row == "swap":
+        r = run_swap(args, rank, world, local_rank)
+        if world > 1:
+            torch.distributed.destroy_process_group()
+        if rank == 0:
+            print(json.dumps(swap_line(args, r, world)), flush=True)
+        return 0
+    r = run_cuda(args, rank, world, local_rank)
     if world > 1:
         torch.distributed.destroy_process_group()
     if rank != 0:

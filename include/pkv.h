@@ -275,6 +275,42 @@ pkv_status pkv_paged_attention_decode_static_ws(void* out, const void* q, const 
 pkv_status pkv_get_error(uint32_t* flags, void* stream);
 
 /* ------------------------------------------------------------------------
+ * pkv_paged_attention_multi -- paged attention for several query tokens
+ * per sequence (speculative-decoding verification, prefill chunks).
+ *
+ * "PagedAttention 与 vLLM 推理加速" §6 (the large model verifies several
+ * tokens the small model guessed, in one pass) and "LLM Systems 24 ..."
+ * §2.2.1.3 (batches mixing prefill chunks and decode steps); §1 of the
+ * former: a token attends over every token so far, itself included.
+ *
+ * Sequence b brings n_b = query_start[b+1] - query_start[b] new tokens,
+ * rows query_start[b] .. query_start[b+1]-1 of q / out, whose K/V are
+ * already appended (context_lens[b] counts them).  New token i sits at
+ * position p = context_lens[b] - n_b + i; for every query head h:
+ *   out[row, h, :] = softmax_j(scale * q[row, h, :] . K_j) V_j,  j = 0 .. p
+ * with K_j / V_j read through block_tables as in pkv_paged_attention_decode.
+ * A row with p < 0 (n_b > context_lens[b]) is zeros and sets
+ * PKV_ERR_CONTEXT_RANGE.  One query token per sequence is decode.
+ *
+ * q, out [total_query_tokens, num_q_heads, head_dim]; query_start int32
+ * [num_seqs + 1] (device), non-decreasing, query_start[num_seqs] <=
+ * total_query_tokens, every n_b <= max_query_len (a sequence that breaks
+ * this is skipped, its rows left unwritten, and PKV_ERR_CONTEXT_RANGE set).
+ * fp16 / bf16 only (tensor cores).  num_seqs * ceil(max_query_len * G / 16)
+ * <= 65535.  workspace: pkv_multi_workspace_bytes(...) bytes (0 when
+ * max_context_len <= partition), 16-byte aligned.
+ * -------------------------------------------------------------------- */
+size_t pkv_multi_workspace_bytes(int total_query_tokens, int num_q_heads, int head_dim, int max_context_len,
+                                 int partition_tokens);
+pkv_status pkv_paged_attention_multi(void* out, const void* q, const void* k_cache, const void* v_cache,
+                                     const int32_t* block_tables, int max_blocks_per_seq,
+                                     const int32_t* context_lens, int max_context_len,
+                                     const int32_t* query_start, int max_query_len, int total_query_tokens,
+                                     int num_seqs, int num_q_heads, int num_kv_heads, int head_dim,
+                                     int num_blocks, float scale, int partition_tokens, pkv_dtype dtype,
+                                     void* workspace, size_t workspace_bytes, void* stream);
+
+/* ------------------------------------------------------------------------
  * Host block allocator.
  *
  * "vLLM + PagedAttention：打造高并发LLM推理引擎", "它是怎么工作的": blocks are

@@ -11,4 +11,5 @@ from ._lib import (ERR_BLOCK_RANGE, ERR_CONTEXT_RANGE, ERR_COPY_RANGE, ERR_SLOT_
 from .api import (BLOCK_SIZE, DEFAULT_PARTITION, BlockAllocator, PagedKVCache, copy_blocks,  # noqa: F401
                   copy_blocks_check, decode_workspace_bytes, get_error, kv_append, kv_cache_bytes,
                   paged_attention_decode, paged_attention_decode_static_ws, paged_attention_decode_prefix,
-                  decode_prefix_workspace_bytes, common_prefix_pages, swap_blocks, swap_blocks_check)
+                  decode_prefix_workspace_bytes, common_prefix_pages, swap_blocks, swap_blocks_check,
+                  paged_attention_multi, multi_workspace_bytes)

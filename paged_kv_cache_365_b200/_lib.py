@@ -47,6 +47,10 @@ PROTOTYPES = {
     "pkv_paged_attention_decode_static_ws": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_int,
                                                      c_void_p, c_int, c_int, c_int, c_int, c_int, c_int,
                                                      c_float, c_int, c_int, c_void_p]),
+    "pkv_multi_workspace_bytes": (c_size_t, [c_int, c_int, c_int, c_int, c_int]),
+    "pkv_paged_attention_multi": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_int, c_void_p, c_int,
+                                          c_void_p, c_int, c_int, c_int, c_int, c_int, c_int, c_int, c_float, c_int,
+                                          c_int, c_void_p, c_size_t, c_void_p]),
     "pkv_get_error": (c_int, [P(c_uint32), c_void_p]),
     "pkv_alloc_create": (c_int, [c_int, P(c_int32), P(c_void_p)]),
     "pkv_alloc_destroy": (None, [c_void_p]),

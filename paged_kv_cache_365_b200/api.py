@@ -230,6 +230,48 @@ def paged_attention_decode_prefix(q: torch.Tensor, k_cache: torch.Tensor, v_cach
     return out
 
 
+def multi_workspace_bytes(total_query_tokens: int, num_q_heads: int, head_dim: int, max_context_len: int,
+                          partition: int = 0) -> int:
+    return int(lib.pkv_multi_workspace_bytes(total_query_tokens, num_q_heads, head_dim, max_context_len, partition))
+
+
+def paged_attention_multi(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
+                          block_tables: torch.Tensor, context_lens: torch.Tensor, query_start: torch.Tensor,
+                          max_context_len: int, max_query_len: int, scale: float,
+                          out: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
+                          partition: int = 0, stream=None) -> torch.Tensor:
+    """Several query tokens per sequence, each attending causally over its
+    sequence's paged K/V up to its own position.
+
+    q [T, Hq, D] (fp16/bf16); query_start int32 [B + 1] (sequence b's rows
+    are query_start[b] .. query_start[b+1]-1, its last n_b tokens, already
+    appended); block_tables int32 [B, W]; context_lens int32 [B].
+    max_context_len / max_query_len: host bounds.  Returns out [T, Hq, D].
+    """
+    nb, hkv, d = _cache_dims(k_cache, v_cache)
+    if q.dim() != 3 or q.shape[2] != d or q.dtype != k_cache.dtype:
+        raise ValueError("q must be [T, Hq, D] in the cache dtype")
+    T, hq, _ = q.shape
+    B = block_tables.shape[0]
+    if block_tables.dim() != 2 or context_lens.shape != (B,) or query_start.shape != (B + 1,):
+        raise ValueError("block_tables [B, W], context_lens [B] and query_start [B + 1] required")
+    if out is None:
+        out = torch.empty_like(q)
+    need = multi_workspace_bytes(T, hq, d, max_context_len, partition)
+    if need and (workspace is None or workspace.numel() * workspace.element_size() < need):
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    ws_ptr = _dev(workspace, "workspace") if need else None
+    ws_len = workspace.numel() * workspace.element_size() if need else 0
+    check(lib.pkv_paged_attention_multi(
+        _dev(out, "out", q.dtype), _dev(q, "q"), _dev(k_cache, "k_cache"), _dev(v_cache, "v_cache"),
+        _dev(block_tables, "block_tables", torch.int32), block_tables.shape[1],
+        _dev(context_lens, "context_lens", torch.int32), int(max_context_len),
+        _dev(query_start, "query_start", torch.int32), int(max_query_len), T, B, hq, hkv, d, nb, float(scale),
+        int(partition), _DT[k_cache.dtype], ws_ptr, ws_len, _stream(stream, q.device)),
+        "pkv_paged_attention_multi")
+    return out
+
+
 def get_error(stream=None, device=None) -> int:
     """Read and clear the device error word (PKV_ERR_* bits); synchronises."""
     v = ctypes.c_uint32(0)

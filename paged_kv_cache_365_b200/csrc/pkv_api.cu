@@ -12,6 +12,7 @@
 #include "decode.cuh"
 #include "decode_mma.cuh"
 #include "decode_prefix.cuh"
+#include "multi_mma.cuh"
 #include "pkv.h"
 
 namespace pkv {
@@ -181,6 +182,60 @@ pkv_status dispatch_dim_mma(const pkv::DecodeArgs& a, int D, int G, cudaStream_t
   if (D == 64) return dispatch_group_mma<T, 64>(a, G, st);
   if (D == 128) return dispatch_group_mma<T, 128>(a, G, st);
   return PKV_EINVAL;
+}
+
+// ---- several query tokens per sequence (tensor cores) -----------------------
+template <typename T, int D, int HPC>
+struct MultiMergeK {
+  static constexpr auto fn = pkv::paged_multi_merge_kernel<T, D, HPC>;
+};
+
+template <typename T, int D, int G>
+pkv_status launch_multi(const pkv::MultiArgs& a, const void* k_cache, const void* v_cache, int num_blocks,
+                        cudaStream_t st) {
+  constexpr int kStages = kMmaStages;
+  using S = pkv::MmaShape<T, D, G, kMmaWarps, kStages>;
+  CUtensorMap mk, mv;
+  const long long rows = static_cast<long long>(num_blocks) * a.num_kv_heads * PKV_BLOCK_SIZE;
+  if (!encode_cache_map(&mk, k_cache, pkv::Mma<T>::kTmaType, D, rows) ||
+      !encode_cache_map(&mv, v_cache, pkv::Mma<T>::kTmaType, D, rows))
+    return PKV_ECUDA;
+  auto kfn = pkv::paged_multi_mma_kernel<T, D, G, kMmaWarps, kStages>;
+  if (cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(S::kSmem)) !=
+      cudaSuccess)
+    return PKV_ECUDA;
+  const dim3 grid(a.num_kv_heads, a.num_seqs * a.tiles, a.num_parts);
+  if (launch(kfn, grid, dim3(kMmaWarps * 32), S::kSmem, st, a, mk, mv) != PKV_OK) return PKV_ECUDA;
+  if (a.num_parts > 1) {
+    const dim3 block(pkv::kMergeWarps * 32);
+    // one CTA per query token; heads per CTA from the partitions a row may span
+    if (a.num_parts >= 32)
+      return launch(MultiMergeK<T, D, 1>::fn, dim3(a.total_q, a.num_q_heads), block, 0, st, a);
+    if (a.num_parts >= 8)
+      return launch(MultiMergeK<T, D, 4>::fn, dim3(a.total_q, (a.num_q_heads + 3) / 4), block, 0, st, a);
+    return launch(MultiMergeK<T, D, 8>::fn, dim3(a.total_q, (a.num_q_heads + 7) / 8), block, 0, st, a);
+  }
+  return PKV_OK;
+}
+
+template <typename T, int D>
+pkv_status dispatch_group_multi(const pkv::MultiArgs& a, int G, const void* k, const void* v, int nb,
+                                cudaStream_t st) {
+  switch (G) {
+    case 1: return launch_multi<T, D, 1>(a, k, v, nb, st);
+    case 2: return launch_multi<T, D, 2>(a, k, v, nb, st);
+    case 4: return launch_multi<T, D, 4>(a, k, v, nb, st);
+    case 8: return launch_multi<T, D, 8>(a, k, v, nb, st);
+  }
+  return PKV_EINVAL;
+}
+
+// Workspace of the multi-token path: partials [T][Hq][P][D] then (max, sum)
+// [T][Hq][P]; nothing when every key fits one partition.
+size_t multi_workspace_bytes(long long total_q, long long Hq, long long D, long long P) {
+  if (P <= 1) return 0;
+  const size_t o = static_cast<size_t>(total_q * Hq * P * D * 4);
+  return (o + 15) / 16 * 16 + static_cast<size_t>(total_q * Hq * P * 8);
 }
 
 // ---- shared-prefix (cascade) path ------------------------------------------
@@ -619,6 +674,75 @@ pkv_status pkv_get_error(uint32_t* flags, void* stream) {
   if (cudaStreamSynchronize(st) != cudaSuccess) return PKV_ECUDA;
   *flags = v;
   return PKV_OK;
+}
+
+size_t pkv_multi_workspace_bytes(int total_query_tokens, int num_q_heads, int head_dim, int max_context_len,
+                                 int partition_tokens) {
+  const int part = resolve_partition(partition_tokens);
+  if (part < 0 || total_query_tokens < 0 || num_q_heads <= 0 || !head_dim_ok(head_dim) || max_context_len < 0)
+    return 0;
+  const long long P = (static_cast<long long>(max_context_len) + part - 1) / part;
+  return multi_workspace_bytes(total_query_tokens, num_q_heads, head_dim, P);
+}
+
+pkv_status pkv_paged_attention_multi(void* out, const void* q, const void* k_cache, const void* v_cache,
+                                     const int32_t* block_tables, int max_blocks_per_seq,
+                                     const int32_t* context_lens, int max_context_len,
+                                     const int32_t* query_start, int max_query_len, int total_query_tokens,
+                                     int num_seqs, int num_q_heads, int num_kv_heads, int head_dim, int num_blocks,
+                                     float scale, int partition_tokens, pkv_dtype dtype, void* workspace,
+                                     size_t workspace_bytes_given, void* stream) {
+  if (dtype != PKV_F16 && dtype != PKV_BF16) return PKV_EINVAL;  // tensor-core path only
+  const int part = resolve_partition(partition_tokens);
+  if (part < 0 || num_seqs < 0 || num_kv_heads <= 0 || num_kv_heads > 65535 || num_q_heads <= 0 ||
+      num_q_heads % num_kv_heads != 0 || !group_ok(num_q_heads / num_kv_heads) || !head_dim_ok(head_dim) ||
+      num_blocks <= 0 || max_context_len < 0 || max_blocks_per_seq <= 0 || max_query_len < 0 ||
+      total_query_tokens < 0 || num_q_heads > 65535 ||
+      static_cast<long long>(max_context_len) > static_cast<long long>(max_blocks_per_seq) * PKV_BLOCK_SIZE ||
+      !std::isfinite(scale))
+    return PKV_EINVAL;
+  if (num_seqs == 0 || total_query_tokens == 0 || max_query_len == 0) return PKV_OK;
+  if (!out || !q || !k_cache || !v_cache || !block_tables || !context_lens || !query_start) return PKV_EINVAL;
+  if (!aligned16(out) || !aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache)) return PKV_EINVAL;
+  if (static_cast<long long>(num_blocks) * num_kv_heads * PKV_BLOCK_SIZE > 0x7fffffffLL) return PKV_EINVAL;
+  const int G = num_q_heads / num_kv_heads;
+  const long long tiles = (static_cast<long long>(max_query_len) * G + 15) / 16;
+  const long long P = (static_cast<long long>(max_context_len) + part - 1) / part;
+  if (tiles * num_seqs > 65535 || P > 65535) return PKV_EINVAL;
+  const size_t need = multi_workspace_bytes(total_query_tokens, num_q_heads, head_dim, P);
+  if (need > 0 && (workspace == nullptr || workspace_bytes_given < need || !aligned16(workspace)))
+    return PKV_EINVAL;
+  pkv::MultiArgs a{};
+  a.out = out;
+  a.q = q;
+  a.block_tables = block_tables;
+  a.context_lens = context_lens;
+  a.query_start = query_start;
+  if (need) {
+    a.ws_o = static_cast<float*>(workspace);
+    const size_t o = static_cast<size_t>(total_query_tokens) * num_q_heads * P * head_dim * 4;
+    a.ws_ml = reinterpret_cast<float2*>(static_cast<unsigned char*>(workspace) + (o + 15) / 16 * 16);
+  }
+  a.bt_stride = max_blocks_per_seq;
+  a.max_ctx = max_context_len;
+  a.num_seqs = num_seqs;
+  a.num_q_heads = num_q_heads;
+  a.num_kv_heads = num_kv_heads;
+  a.num_blocks = num_blocks;
+  a.partition = part;
+  a.num_parts = P > 1 ? static_cast<int>(P) : 1;
+  a.tiles = static_cast<int>(tiles);
+  a.max_q = max_query_len;
+  a.total_q = total_query_tokens;
+  a.qk_scale = scale * kLog2e;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  auto run = [&](auto tag) -> pkv_status {
+    using T = decltype(tag);
+    if (head_dim == 64) return dispatch_group_multi<T, 64>(a, G, k_cache, v_cache, num_blocks, st);
+    return dispatch_group_multi<T, 128>(a, G, k_cache, v_cache, num_blocks, st);
+  };
+  if (dtype == PKV_F16) return run(__half{});
+  return run(__nv_bfloat16{});
 }
 
 }  // extern "C"

@@ -1,0 +1,120 @@
+"""GPU parity of multi-token paged attention (several query tokens per
+sequence, causal over the paged context) against the fp64 oracle on the
+same seeded inputs: max-abs error within 2e-3 (fp16) / 1e-2 (bf16).
+Unwritten slots hold NaN and tables are padded with out-of-range ids, so a
+read outside a row's visible tokens shows up."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from helpers import make_multi_case
+
+pytestmark = pytest.mark.gpu
+
+TOL = {"f16": 2e-3, "bf16": 1e-2}
+TORCH = {"f16": torch.float16, "bf16": torch.bfloat16}
+
+
+def pkv():
+    import paged_kv_cache_365_b200 as m
+    return m
+
+
+def to_dev(a, dtype):
+    t = torch.from_numpy(np.ascontiguousarray(a))
+    if dtype == "bf16":
+        t = t.view(torch.int16).view(torch.bfloat16)
+    return t.cuda()
+
+
+def run_gpu(c, scale, partition=0, max_q=None):
+    m = pkv()
+    dt = c["dtype"]
+    q, k, v = to_dev(c["q"], dt), to_dev(c["k"], dt), to_dev(c["v"], dt)
+    nq = np.diff(c["qs"])
+    out = m.paged_attention_multi(q, k, v, torch.from_numpy(c["tables"]).cuda(), torch.from_numpy(c["ctx"]).cuda(),
+                                  torch.from_numpy(c["qs"]).cuda(), int(c["ctx"].max()),
+                                  int(nq.max()) if max_q is None else max_q, scale, partition=partition)
+    torch.cuda.synchronize()
+    return out.float().cpu().numpy(), m.get_error()
+
+
+CASES = [
+    # ctx, nq, Hq, Hkv, D, dtype
+    ([5, 16, 17, 40, 1], [1, 4, 17, 8, 1], 4, 4, 128, "f16"),
+    ([33, 20, 3, 64], [5, 20, 3, 16], 8, 2, 64, "bf16"),
+    ([48, 7, 300], [16, 2, 9], 8, 1, 128, "f16"),
+    ([100, 130, 520, 1100], [2, 3, 4, 5], 16, 4, 128, "bf16"),
+    ([1030, 600], [40, 33], 2, 2, 64, "f16"),
+]
+
+
+@pytest.mark.parametrize("case", CASES, ids=lambda c: f"{c[5]}_G{c[2] // c[3]}_D{c[4]}")
+@pytest.mark.parametrize("partition", [0, 16, 64])
+def test_multi_matches_oracle(case, partition):
+    ctx, nq, Hq, Hkv, D, dt = case
+    c = make_multi_case(ctx, nq, Hq, Hkv, D, dt, seed=sum(ctx) + partition)
+    scale = D ** -0.5
+    want = oracle.paged_multi(c["q"], c["k"], c["v"], c["tables"], c["ctx"], c["qs"], scale, dt)
+    got, err = run_gpu(c, scale, partition)
+    assert err == 0
+    assert np.isfinite(got).all()
+    assert np.abs(got - want).max() <= TOL[dt]
+
+
+def test_one_token_per_sequence_agrees_with_decode():
+    m = pkv()
+    c = make_multi_case([9, 16, 50, 700, 2100], [1] * 5, 8, 2, 128, "bf16", seed=3)
+    scale = 128 ** -0.5
+    got, err = run_gpu(c, scale)
+    dec = m.paged_attention_decode(to_dev(c["q"], "bf16"), to_dev(c["k"], "bf16"), to_dev(c["v"], "bf16"),
+                                   torch.from_numpy(c["tables"]).cuda(), torch.from_numpy(c["ctx"]).cuda(),
+                                   int(c["ctx"].max()), scale)
+    assert err == 0
+    assert np.abs(got - dec.float().cpu().numpy()).max() <= TOL["bf16"]
+
+
+def test_speculative_verify_shape_sampled():
+    """64 sequences of a 7B shape (32 heads, D 128, fp16), contexts up to
+    2048, 4 draft tokens + 1 verified each; every 8th sequence checked."""
+    rng = np.random.default_rng(21)
+    ctx = [int(x) for x in rng.integers(128, 2049, 64)]
+    c = make_multi_case(ctx, [5] * 64, 32, 32, 128, "f16", seed=22)
+    scale = 128 ** -0.5
+    got, err = run_gpu(c, scale)
+    assert err == 0
+    seqs = list(range(0, 64, 8))
+    want = oracle.paged_multi(c["q"], c["k"], c["v"], c["tables"], c["ctx"], c["qs"], scale, "f16", seqs=seqs)
+    rows = np.concatenate([np.arange(c["qs"][b], c["qs"][b + 1]) for b in seqs])
+    assert np.abs(got[rows] - want[rows]).max() <= TOL["f16"]
+
+
+def test_prefill_chunk_sampled():
+    """A 512-token prefill chunk at the end of a 2000-token context (GQA 4,
+    bf16): every row against the oracle."""
+    c = make_multi_case([2000, 700], [512, 300], 8, 2, 128, "bf16", seed=31)
+    scale = 128 ** -0.5
+    got, err = run_gpu(c, scale)
+    want = oracle.paged_multi(c["q"], c["k"], c["v"], c["tables"], c["ctx"], c["qs"], scale, "bf16")
+    assert err == 0
+    assert np.abs(got - want).max() <= TOL["bf16"]
+
+
+def test_edge_rows_and_flags():
+    m = pkv()
+    # more new tokens than context: the first rows are zeros, flagged
+    c = make_multi_case([3, 20], [5, 4], 4, 2, 64, "f16", seed=5)
+    want = oracle.paged_multi(c["q"], c["k"], c["v"], c["tables"], c["ctx"], c["qs"], 0.125, "f16")
+    got, err = run_gpu(c, 0.125)
+    assert err == m.ERR_CONTEXT_RANGE
+    assert np.abs(got - want).max() <= TOL["f16"]
+    # a sequence with no new token, and max_query_len smaller than a
+    # sequence's tokens: that sequence is skipped and flagged
+    c = make_multi_case([40, 30, 50], [3, 0, 6], 4, 4, 64, "f16", seed=6)
+    want = oracle.paged_multi(c["q"], c["k"], c["v"], c["tables"], c["ctx"], c["qs"], 0.125, "f16")
+    got, err = run_gpu(c, 0.125)
+    assert err == 0 and np.abs(got - want).max() <= TOL["f16"]
+    got, err = run_gpu(c, 0.125, max_q=4)
+    assert err == m.ERR_CONTEXT_RANGE
+    assert np.abs(got[:3] - want[:3]).max() <= TOL["f16"]
