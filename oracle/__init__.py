@@ -27,6 +27,10 @@ What each function follows (page titles as printed on the pages):
   "LLM Systems 24 ..." §3, conclusion (a request preempted for lack of KV
   blocks is swapped out and later swapped back in); the policy details are
   readings stated in ``allocator``.
+* ``fp8`` and ``RefCache.append_fp8`` -- an FP8 E4M3 KV cache with one
+  scale for K and one for V (the pages name FP8 only for TensorRT-LLM's
+  low-precision operators; the format and the scaling are readings stated
+  in ``fp8``).
 * ``brute.contiguous_decode`` -- the contiguous-cache baseline the pages
   contrast paging with ("PagedAttention 与 vLLM 推理加速" §2.2), in pure
   Python, used only to pin ``paged_decode`` on tiny inputs.
@@ -42,3 +46,4 @@ from .cache import RefCache, swap_blocks  # noqa: F401
 from .allocator import RefAllocator, RefAllocError  # noqa: F401
 from .brute import contiguous_decode  # noqa: F401
 from .replay import replay  # noqa: F401
+from . import fp8  # noqa: F401

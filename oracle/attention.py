@@ -46,14 +46,17 @@ def decode_head(q_row: np.ndarray, keys: np.ndarray, values: np.ndarray, scale: 
 
 
 def paged_decode(q, k_cache, v_cache, block_tables, context_lens, scale, dtype,
-                 block_size=16, seqs=None):
+                 block_size=16, seqs=None, kv_dtype=None, k_scale=1.0, v_scale=1.0):
     """float64 output [B, Hq, D] (rows not in ``seqs`` are left NaN).
 
     q: [B,Hq,D]; k_cache/v_cache: [num_blocks,Hkv,block_size,D] in the
     storage format ``dtype`` ('f32', 'f16', or 'bf16' as uint16 bits);
     block_tables: int [B, max_blocks]; context_lens: int [B].
     ``seqs`` restricts the work to those sequence indices (sampled checks).
+    An FP8 cache: ``kv_dtype='e4m3'`` (q stays in ``dtype``); a stored K
+    value is its code's value times ``k_scale`` (V alike).
     """
+    kvd = dtype if kv_dtype is None else kv_dtype
     B, Hq, D = q.shape
     Hkv = k_cache.shape[1]
     G = Hq // Hkv
@@ -64,8 +67,8 @@ def paged_decode(q, k_cache, v_cache, block_tables, context_lens, scale, dtype,
         pages = np.asarray(block_tables[b][:n_pages], dtype=np.int64)
         qb = widen(q[b], dtype)
         for g in range(Hkv):
-            keys = widen(_gather(k_cache, pages, g, n, block_size), dtype)
-            values = widen(_gather(v_cache, pages, g, n, block_size), dtype)
+            keys = widen(_gather(k_cache, pages, g, n, block_size), kvd) * k_scale
+            values = widen(_gather(v_cache, pages, g, n, block_size), kvd) * v_scale
             for h in range(g * G, (g + 1) * G):
                 out[b, h] = decode_head(qb[h], keys, values, scale)
     return out

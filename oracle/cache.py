@@ -53,6 +53,18 @@ class RefCache:
         self.k[blk, :, off, :] = k_new[keep]
         self.v[blk, :, off, :] = v_new[keep]
 
+    def append_fp8(self, k_new: np.ndarray, v_new: np.ndarray, slots: np.ndarray, src_dtype: str,
+                   k_scale: float, v_scale: float) -> None:
+        """An FP8 cache's append: each new K (V) element x (storage format
+        ``src_dtype``) is stored as the E4M3 code of x / k_scale (v_scale),
+        the division in float32 (``oracle.fp8.quantize``)."""
+        from .fp8 import quantize
+        from .storage import widen
+        assert self.dtype == "e4m3"
+        kq = quantize(widen(k_new, src_dtype).astype(np.float32), k_scale)
+        vq = quantize(widen(v_new, src_dtype).astype(np.float32), v_scale)
+        self.append(kq, vq, slots)
+
     def copy_blocks(self, pairs) -> None:
         """cache[dst] = cache[src] for each (src, dst), K and V."""
         for src, dst in pairs:

@@ -1,5 +1,7 @@
 """Exact widening of the stored K/V/q formats to float64 (oracle only).
 
+FP8 E4M3 codes (uint8) widen through the code table of ``oracle.fp8``.
+
 fp32 and fp16 widen exactly through numpy.  bf16 values arrive as their
 uint16 bit patterns: a bf16 number is the upper half of a float32, so
 shifting the pattern 16 bits up and reinterpreting it as float32 gives the
@@ -7,8 +9,9 @@ value exactly, and float32 -> float64 is exact too.
 """
 import numpy as np
 
-NAN_PATTERN = {"f32": np.float32(np.nan), "f16": np.float16(np.nan), "bf16": np.uint16(0x7FC0)}
-STORAGE_NP = {"f32": np.float32, "f16": np.float16, "bf16": np.uint16}
+NAN_PATTERN = {"f32": np.float32(np.nan), "f16": np.float16(np.nan), "bf16": np.uint16(0x7FC0),
+               "e4m3": np.uint8(0x7F)}
+STORAGE_NP = {"f32": np.float32, "f16": np.float16, "bf16": np.uint16, "e4m3": np.uint8}
 
 
 def widen(x: np.ndarray, dtype: str) -> np.ndarray:
@@ -22,6 +25,10 @@ def widen(x: np.ndarray, dtype: str) -> np.ndarray:
     if dtype == "bf16":
         assert x.dtype == np.uint16
         return (x.astype(np.uint32) << np.uint32(16)).view(np.float32).astype(np.float64)
+    if dtype == "e4m3":  # FP8 codes (oracle.fp8); the cache's scale is applied by the caller
+        from .fp8 import e4m3_decode
+        assert x.dtype == np.uint8
+        return e4m3_decode(x)
     raise ValueError(dtype)
 
 
