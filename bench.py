@@ -14,6 +14,9 @@ idempotent).
   python bench.py --row swap ...         (preemption by swapping: one step =
       swap a quarter of the batch out to pinned host memory and back in;
       GB/s over the host link against cudaMemcpyAsync of the same bytes)
+  python bench.py --row multi [--new-tokens N] ...  (one step = append N new
+      tokens per sequence + causal attention of all of them over the paged
+      context: a speculative-verification pass, N = drafted + 1)
 
 N > 1: one process per GPU (torchrun), each rank decoding its own replica
 batch (different seed), no collective on the data path; value = all ranks'
@@ -41,12 +44,17 @@ import workloads  # noqa: E402
 
 METRIC = "paged decode attention: KV-cache HBM GB/s (% of peak), seq-steps/s"
 SWAP_METRIC = "block swap device<->pinned host (preempt + resume): GB/s over the host link"
+MULTI_METRIC = ("paged multi-token attention (several new tokens per sequence, causal): KV-cache HBM GB/s "
+                "(% of peak), query-tokens/s")
 UNIT = "GB/s"
 FALLBACK_HBM_GBS = 6650.0
 STORAGE = {"f32": 4, "f16": 2, "bf16": 2}
 DTYPE_NAME = {"f32": "fp32", "f16": "fp16", "bf16": "bf16"}
+# the decode kernels and their launch configuration: a committed ncu traffic
+# figure counts only while these are unchanged
 DECODE_SOURCES = ["paged_kv_cache_365_b200/csrc/decode.cuh", "paged_kv_cache_365_b200/csrc/decode_mma.cuh",
-                  "paged_kv_cache_365_b200/csrc/common.cuh", "paged_kv_cache_365_b200/csrc/pkv_api.cu"]
+                  "paged_kv_cache_365_b200/csrc/decode_prefix.cuh", "paged_kv_cache_365_b200/csrc/common.cuh",
+                  "paged_kv_cache_365_b200/csrc/decode_launch.cuh"]
 
 
 # ---------------------------------------------------------------------------
@@ -346,6 +354,171 @@ def run_cuda(args, rank, world, local_rank):
 
 
 # ---------------------------------------------------------------------------
+# several new tokens per sequence (speculative verification)
+# ---------------------------------------------------------------------------
+def run_multi(args, rank, world, local_rank):
+    import torch
+    from paged_kv_cache_365_b200.replay import build_multi_step
+    import paged_kv_cache_365_b200 as pkv
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    wl = workloads.named(args.workload, replica_seed(args.seed, rank))
+    if wl.dtype == "f32":
+        raise SystemExit("--row multi needs an fp16 / bf16 workload")
+    vals = device_values(wl, replica_seed(args.seed, rank), dev)
+    st = build_multi_step(wl, args.new_tokens, dev, device_values=vals, seed=replica_seed(args.seed, rank))
+    del vals
+    cache = st["cache"]
+    stream = torch.cuda.current_stream(dev)
+    lens = st["host"]["context_lens"]
+    T = int(st["q"].shape[0])
+    max_ctx, max_q = st["max_context_len"], st["max_query_len"]
+    ws = cache.workspace(pkv.multi_workspace_bytes(T, wl.Hq, wl.D, max_ctx, args.partition))
+    out = torch.empty_like(st["q"])
+    scale = 1.0 / math.sqrt(wl.D)
+    n_pairs = int(st["cow_pairs"].shape[0])
+    P = max(1, math.ceil(max_ctx / (args.partition or pkv.DEFAULT_PARTITION)))
+
+    def pre():
+        if n_pairs:
+            pkv.copy_blocks(cache.k, cache.v, st["cow_pairs"])
+        pkv.kv_append(st["k_new"], st["v_new"], cache.k, cache.v, st["slot_mapping"])
+
+    def attend():
+        pkv.paged_attention_multi(st["q"], cache.k, cache.v, st["block_tables"], st["context_lens"],
+                                  st["query_start"], max_ctx, max_q, scale, out=out, workspace=ws,
+                                  partition=args.partition)
+
+    def step():
+        pre()
+        attend()
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if pkv.get_error() != 0:
+        raise RuntimeError("device error flags raised during warm-up")
+    K = args.steps
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local_rank) as clocks:
+        t0.record(stream)
+        for _ in range(K):
+            step()
+        t1.record(stream)
+        torch.cuda.synchronize()
+    total_ms = t0.elapsed_time(t1)
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(K)]
+    for i in range(K):
+        ev[i][0].record(stream)
+        attend()
+        ev[i][1].record(stream)
+    torch.cuda.synchronize()
+    att_ms = sum(ev[i][0].elapsed_time(ev[i][1]) for i in range(K)) / K
+    # e2e: inputs from pinned host memory every step, output read back
+    host = {k: st[k].cpu().pin_memory() for k in ("q", "k_new", "v_new", "slot_mapping", "cow_pairs",
+                                                    "block_tables", "context_lens", "query_start")}
+    out_host = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
+    h2d = sum(t.numel() * t.element_size() for t in host.values())
+    d2h = out_host.numel() * out_host.element_size()
+
+    def e2e_step():
+        cache.run_multi_step(host["slot_mapping"], host["cow_pairs"], host["block_tables"], host["context_lens"],
+                             max_ctx, host["query_start"], max_q, host["q"], host["k_new"], host["v_new"],
+                             out=out_host, scale=scale, partition=args.partition, stream=stream)
+
+    for _ in range(args.warmup):
+        e2e_step()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(K):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1)
+    if pkv.get_error() != 0:
+        raise RuntimeError("device error flags raised during timing")
+    total_ms, att_ms, e2e_ms = max_over_ranks([total_ms, att_ms, e2e_ms], world, dev)
+    es = STORAGE[wl.dtype]
+    kv = int(np.asarray(lens, dtype=np.int64).sum()) * wl.Hkv * wl.D * 2 * es
+    att_bytes = kv + 2 * T * wl.Hq * wl.D * es + int(sum(-(-int(n) // 16) for n in lens)) * 4 + 8 * wl.B + 4
+    launches = (1 + (1 if n_pairs else 0) + 1 + (1 if P > 1 else 0)) * K
+    return dict(wl=wl, K=K, T=T, kv=kv, att_bytes=att_bytes, total_ms=total_ms, att_ms=att_ms, e2e_ms=e2e_ms,
+                h2d=h2d, d2h=d2h, clocks=clocks.summary(), P=P, launches=launches, lens=lens)
+
+
+def multi_cpu_baseline(wl, n_new, budget_s=10.0, seed=0):
+    """The oracle's multi-token attention, one thread, on sampled sequences
+    of the same workload (n_new new tokens each, the last of the context)."""
+    import oracle
+    limits = blas_threads()
+    ctx = limits(limits=1) if limits else None
+    if ctx:
+        ctx.__enter__()
+    try:
+        vals, ref = oracle_setup(wl)
+        rng = np.random.default_rng(seed)
+        order = rng.permutation(wl.B)
+        es = STORAGE[wl.dtype]
+        secs, nbytes, done = 0.0, 0, 0
+        for b in order:
+            qs = np.array([0, n_new], dtype=np.int32)
+            qrows = workloads._to_storage(rng.standard_normal((n_new, wl.Hq, wl.D)).astype(np.float32), wl.dtype)
+            t0 = time.perf_counter()
+            oracle.paged_multi(qrows, ref["cache"].k, ref["cache"].v, ref["block_tables"][b:b + 1],
+                               ref["context_lens"][b:b + 1], qs, wl.scale, wl.dtype)
+            secs += time.perf_counter() - t0
+            nbytes += int(ref["context_lens"][b]) * wl.Hkv * wl.D * 2 * es
+            done += 1
+            if secs >= budget_s:
+                break
+    finally:
+        if ctx:
+            ctx.__exit__(None, None, None)
+    return {"value": nbytes / secs / 1e9, "unit": UNIT, "cores": 1, "kind": "oracle",
+            "sample": f"{done} sequences of workload {wl.name} seed {wl.seed}, {n_new} new tokens each, "
+                      f"{nbytes / 1e6:.1f} MB of K/V, fp64 numpy, BLAS limited to 1 thread, {secs:.1f} s"}
+
+
+def multi_line(args, r, world):
+    wl = r["wl"]
+    K = r["K"]
+    peak, peak_kind = measured_peak()
+    step_s = r["total_ms"] / 1e3 / K
+    achieved = r["att_bytes"] / (r["att_ms"] / 1e3) / 1e9
+    line = {
+        "metric": MULTI_METRIC, "value": job_throughput(r["kv"], world, K, r["total_ms"] / 1e3), "unit": UNIT,
+        "n_gpus": world, "steps": K, "warmup": args.warmup, "ms_per_step": r["total_ms"] / K,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": wl.dtype,
+        "data": "synthetic (seeded N(0,1) q/K/V on the device, seeded lengths and placement)",
+        "config": {"workload": f"{wl.name} + {args.new_tokens} new tokens per sequence", "global_batch": wl.B,
+                   "new_tokens": args.new_tokens, "query_tokens": r["T"], "num_q_heads": wl.Hq,
+                   "num_kv_heads": wl.Hkv, "head_dim": wl.D, "block_size": 16,
+                   "context_lens": {"min": int(np.min(r["lens"])), "max": int(np.max(r["lens"])),
+                                    "sum": int(np.sum(r["lens"]))},
+                   "partition_tokens": args.partition or 512, "partitions_max": r["P"], "seed": args.seed,
+                   "parallelism": f"replicas{args.gpus}" if args.gpus > 1 else "single-gpu",
+                   "l2": "inputs larger than L2 (no flush)" if r["kv"] > 126e6 else "inputs fit in L2"},
+        "us_per_step": 1e3 * r["total_ms"] / K,
+        "query_tokens_per_s": world * r["T"] / step_s,
+        "pct_hbm_peak": 100.0 * (r["kv"] / step_s / 1e9) / peak,
+        "clocks": r["clocks"],
+        "e2e": {"value": job_throughput(r["kv"], world, K, r["e2e_ms"] / 1e3), "unit": UNIT,
+                "h2d_bytes_per_step": r["h2d"], "d2h_bytes_per_step": r["d2h"],
+                "us_per_step": 1e3 * r["e2e_ms"] / K},
+        "gpu_launches": r["launches"],
+        "roofline": {"kernel": "paged_multi (partition + merge kernels)", "bound": "hbm", "achieved": achieved,
+                     "peak": peak, "peak_kind": f"{peak_kind} (MEASURED_PEAKS hbm_gbs)" if peak_kind == "measured"
+                     else "fallback", "unit": "GB/s", "frac": achieved / peak, "traffic": None,
+                     "algorithmic_bytes_per_launch": r["att_bytes"], "avg_launch_us": 1e3 * r["att_ms"]},
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = multi_cpu_baseline(wl, args.new_tokens, seed=args.seed)
+    return line
+
+
+# ---------------------------------------------------------------------------
 # preemption by swapping: a quarter of the batch out to pinned host memory
 # and back in
 # ---------------------------------------------------------------------------
@@ -588,6 +761,18 @@ def run_reference(args, rank, world):
     if rank != 0:
         return
     wl = workloads.named(args.workload, args.seed)
+    if getattr(args, "row", "step") == "multi":
+        b = multi_cpu_baseline(wl, args.new_tokens, budget_s=min(60.0, 0.5 * (args.steps + args.warmup)),
+                               seed=args.seed)
+        print(json.dumps({"impl": "reference", "metric": MULTI_METRIC, "value": b["value"], "unit": UNIT,
+                          "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup, "ms_per_step": None,
+                          "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+                          "data": "synthetic",
+                          "config": {"workload": f"{wl.name} + {args.new_tokens} new tokens per sequence"},
+                          "cpu_baseline": b,
+                          "e2e": {"value": b["value"], "unit": UNIT, "h2d_bytes_per_step": 0,
+                                  "d2h_bytes_per_step": 0}}), flush=True)
+        return
     if getattr(args, "row", "step") == "swap":
         b = swap_cpu_baseline(wl, budget_s=min(60.0, 0.5 * (args.steps + args.warmup)))
         print(json.dumps({"impl": "reference", "metric": SWAP_METRIC, "value": b["value"], "unit": UNIT,
@@ -645,8 +830,11 @@ def main(argv=None):
                     help="capture one step in a CUDA graph and replay it (launch-bound batches)")
     ap.add_argument("--no-cascade", action="store_true",
                     help="decode a shared-prefix batch with the plain paged kernel")
-    ap.add_argument("--row", choices=["step", "swap"], default="step",
-                    help="step: the decode step (default); swap: preemption by swapping")
+    ap.add_argument("--row", choices=["step", "swap", "multi"], default="step",
+                    help="step: the decode step (default); swap: preemption by swapping; "
+                         "multi: several new tokens per sequence")
+    ap.add_argument("--new-tokens", type=int, default=5,
+                    help="--row multi: new tokens per sequence (drafted + 1)")
     args = ap.parse_args(argv)
     if args.steps is None:
         args.steps = 20 if args.row == "swap" else 2000
@@ -666,6 +854,13 @@ def main(argv=None):
         torch.cuda.set_device(local_rank)
         torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                              device_id=torch.device("cuda", local_rank))
+    if args.row == "multi":
+        r = run_multi(args, rank, world, local_rank)
+        if world > 1:
+            torch.distributed.destroy_process_group()
+        if rank == 0:
+            print(json.dumps(multi_line(args, r, world)), flush=True)
+        return 0
     if args.row == "swap":
         r = run_swap(args, rank, world, local_rank)
         if world > 1:

@@ -548,6 +548,56 @@ class PagedKVCache:
                 out.copy_(res, non_blocking=True)
         return res
 
+    def plan_multi_step(self, seq_ids: Sequence[int], n_new: Sequence[int], width: Optional[int] = None):
+        """Host part of a multi-token step: append n_new[i] tokens to each
+        sequence (in order); returns slots [sum n], CoW pairs [k, 2],
+        query_start [B + 1], tables and lengths.  Each sequence's append is
+        all or nothing; a failure leaves earlier sequences' appends done."""
+        slots, pairs = [], []
+        for sid, n in zip(seq_ids, n_new):
+            s_, p_ = self.alloc.append_tokens(sid, int(n))
+            slots.append(s_)
+            if len(p_):
+                pairs.append(p_)
+        slots = np.concatenate(slots) if slots else np.zeros(0, dtype=np.int64)
+        pairs = np.concatenate(pairs).astype(np.int32) if pairs else np.zeros((0, 2), dtype=np.int32)
+        copy_blocks_check(pairs, self.num_blocks)
+        qs = np.concatenate([[0], np.cumsum(np.asarray(n_new, dtype=np.int64))]).astype(np.int32)
+        if width is None:
+            width = max(1, max(len(self.alloc.block_table(s)[0]) for s in seq_ids)) if len(seq_ids) else 1
+        tables, lens = self.alloc.block_tables(seq_ids, width, self.num_blocks)
+        return slots, pairs, qs, tables, lens
+
+    def run_multi_step(self, slot_mapping: torch.Tensor, cow_pairs: torch.Tensor, block_tables: torch.Tensor,
+                       context_lens: torch.Tensor, max_context_len: int, query_start: torch.Tensor,
+                       max_query_len: int, q: torch.Tensor, k_new: torch.Tensor, v_new: torch.Tensor,
+                       out: Optional[torch.Tensor] = None, scale: Optional[float] = None, partition: int = 0,
+                       stream=None) -> torch.Tensor:
+        """Device part of a multi-token step (speculative verification or a
+        prefill chunk): copy-on-write copies, append of every new token,
+        causal attention of each new token over its sequence.  Host inputs
+        are copied in (pinned: asynchronously); a host ``out`` receives the
+        result asynchronously.  Returns the device output [T, Hq, D]."""
+        dev = self.device
+        st = torch.cuda.current_stream(dev) if stream is None else stream
+
+        def d(t):
+            return t if t.device == dev else t.to(dev, non_blocking=True)
+
+        with torch.cuda.stream(st):
+            if cow_pairs.shape[0]:
+                copy_blocks(self.k, self.v, d(cow_pairs), st)
+            kv_append(d(k_new), d(v_new), self.k, self.v, d(slot_mapping), st)
+            res = out if (out is not None and out.device == dev) else self._out_buffer(q.shape)
+            sc = (1.0 / math.sqrt(self.D)) if scale is None else scale
+            ws = self.workspace(multi_workspace_bytes(q.shape[0], q.shape[1], self.D, max_context_len, partition))
+            paged_attention_multi(d(q), self.k, self.v, d(block_tables), d(context_lens), d(query_start),
+                                  max_context_len, max_query_len, sc, out=res, workspace=ws, partition=partition,
+                                  stream=st)
+            if out is not None and out.device != dev:
+                out.copy_(res, non_blocking=True)
+        return res
+
     def _out_buffer(self, shape) -> torch.Tensor:
         buf = getattr(self, "_out", None)
         if buf is None or tuple(buf.shape) != tuple(shape):

@@ -301,9 +301,11 @@ int pkv_alloc_num_free(const pkv_alloc* a) { return a ? a->free_list.size() : -1
 int pkv_alloc_num_blocks(const pkv_alloc* a) { return a ? a->num_blocks : -1; }
 int pkv_alloc_num_seqs(const pkv_alloc* a) { return a ? static_cast<int>(a->seqs.size()) : -1; }
 
+}  // extern "C"
+
 // ---- preemption by swapping -------------------------------------------------
 
-pkv_status pkv_alloc_set_host_pool(pkv_alloc* a, int num_host_blocks) {
+extern "C" pkv_status pkv_alloc_set_host_pool(pkv_alloc* a, int num_host_blocks) {
   if (a == nullptr || num_host_blocks < 0 || !a->swapped.empty()) return PKV_EINVAL;
   FreeRing ring(num_host_blocks);
   for (int i = 0; i < num_host_blocks; ++i) ring.push_back(i);
@@ -376,6 +378,8 @@ pkv_status move_seqs(std::unordered_map<int64_t, Seq>& from, std::unordered_map<
 }
 
 }  // namespace
+
+extern "C" {
 
 pkv_status pkv_alloc_swap_out(pkv_alloc* a, const int64_t* seq_ids, int n, int32_t* pairs, int cap, int* n_pairs) {
   if (a == nullptr) return PKV_EINVAL;

@@ -103,3 +103,37 @@ def build_step(wl, values: Dict[str, np.ndarray], device="cuda", fill=float("nan
         "host": {"step_slots": step_slots, "cow_pairs": pairs, "block_tables": tables,
                  "context_lens": lens, "prefill_slots": prefill_slots},
     }
+
+
+def build_multi_step(wl, n_new: int, device="cuda", fill=float("nan"),
+                     device_values: Optional[Dict[str, torch.Tensor]] = None, stream=None, seed: int = 0):
+    """Rebuild ``wl``'s cache on the device (its op log, without the decode
+    step) and plan a multi-token step: ``n_new`` new tokens for each of the
+    step's sequences.  New q / K / V are seeded N(0,1) draws on the device.
+    The step's copy / append / attention are NOT run."""
+    dt = _TORCH[wl.dtype]
+    cache = PagedKVCache(wl.num_blocks, wl.Hkv, wl.D, dt, device, wl.free_order, fill=fill)
+    dv = device_values or {}
+    replay_ops(cache, wl.ops, dv["k_tokens"], dv["v_tokens"], stream)
+    ids = [int(s) for s in wl.step_seqs]
+    slots, pairs, qs, tables, lens = cache.plan_multi_step(ids, [n_new] * len(ids), None)
+    dev = cache.device
+    T = int(qs[-1])
+    g = torch.Generator(device=dev)
+    g.manual_seed(int(seed) * 104729 + 3)
+    draw = lambda *shape: torch.randn(*shape, generator=g, device=dev, dtype=torch.float32).to(dt)  # noqa: E731
+    return {
+        "cache": cache,
+        "q": draw(T, wl.Hq, wl.D),
+        "k_new": draw(T, wl.Hkv, wl.D),
+        "v_new": draw(T, wl.Hkv, wl.D),
+        "slot_mapping": torch.from_numpy(slots).to(dev),
+        "cow_pairs": torch.from_numpy(np.ascontiguousarray(pairs)).to(dev),
+        "block_tables": torch.from_numpy(np.ascontiguousarray(tables)).to(dev),
+        "context_lens": torch.from_numpy(np.ascontiguousarray(lens)).to(dev),
+        "query_start": torch.from_numpy(qs).to(dev),
+        "max_context_len": int(lens.max()) if len(lens) else 0,
+        "max_query_len": int(n_new),
+        "host": {"slots": slots, "cow_pairs": pairs, "block_tables": tables, "context_lens": lens,
+                 "query_start": qs},
+    }

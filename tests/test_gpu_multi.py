@@ -118,3 +118,57 @@ def test_edge_rows_and_flags():
     got, err = run_gpu(c, 0.125, max_q=4)
     assert err == m.ERR_CONTEXT_RANGE
     assert np.abs(got[:3] - want[:3]).max() <= TOL["f16"]
+
+
+def test_multi_step_through_the_cache_api():
+    """PagedKVCache.plan_multi_step + run_multi_step (host inputs, one of
+    them forcing a copy-on-write) against the oracle allocator, cache and
+    attention: slots, pairs and the pool bit-exact, output within 2e-3."""
+    m = pkv()
+    rng = np.random.default_rng(41)
+    Hq, Hkv, D, nb = 8, 4, 128, 48
+    order = rng.permutation(nb).astype(np.int32)
+    cache = m.PagedKVCache(nb, Hkv, D, torch.float16, free_order=order)
+    ref = oracle.RefAllocator(nb, order)
+    dev = oracle.RefCache(nb, Hkv, D, "f16")
+
+    def write(sid, n):
+        vals = rng.standard_normal((2, n, Hkv, D)).astype(np.float16)
+        slots, cows = ref.append_tokens(sid, n)
+        dev.copy_blocks(cows)
+        dev.append(vals[0], vals[1], np.array(slots))
+        cache.prefill(sid, torch.from_numpy(vals[0]), torch.from_numpy(vals[1]))
+
+    for sid, n in ((0, 70), (1, 16), (2, 200)):
+        ref.add_seq(sid)
+        cache.add_seq(sid)
+        write(sid, n)
+    ref.fork(0, 3)
+    cache.fork(0, 3)  # shares a partial last block: the step copies it
+    ids, n_new = [0, 1, 2, 3], [5, 3, 8, 4]
+    slots, pairs, qs, tables, lens = cache.plan_multi_step(ids, n_new)
+    r_slots, r_pairs = [], []
+    for sid, n in zip(ids, n_new):
+        s_, p_ = ref.append_tokens(sid, n)
+        r_slots += s_
+        r_pairs += p_
+    assert list(slots) == r_slots and [tuple(p) for p in pairs] == r_pairs
+    T = int(qs[-1])
+    q = rng.standard_normal((T, Hq, D)).astype(np.float16)
+    kn = rng.standard_normal((T, Hkv, D)).astype(np.float16)
+    vn = rng.standard_normal((T, Hkv, D)).astype(np.float16)
+    dev.copy_blocks(r_pairs)
+    dev.append(kn, vn, np.array(r_slots))
+    out = torch.empty((T, Hq, D), dtype=torch.float16, pin_memory=True)
+    cache.run_multi_step(torch.from_numpy(slots).pin_memory(), torch.from_numpy(pairs).pin_memory(),
+                         torch.from_numpy(tables).pin_memory(), torch.from_numpy(lens).pin_memory(),
+                         int(lens.max()), torch.from_numpy(qs).pin_memory(), max(n_new),
+                         torch.from_numpy(q).pin_memory(), torch.from_numpy(kn).pin_memory(),
+                         torch.from_numpy(vn).pin_memory(), out=out)
+    torch.cuda.synchronize()
+    assert m.get_error() == 0
+    held = sorted({b for t in ref.tables.values() for b in t})
+    assert np.array_equal(cache.k.cpu().view(torch.int16).numpy()[held], dev.k.view(np.int16)[held])
+    assert np.array_equal(cache.v.cpu().view(torch.int16).numpy()[held], dev.v.view(np.int16)[held])
+    want = oracle.paged_multi(q, dev.k, dev.v, tables, lens, qs, D ** -0.5, "f16")
+    assert np.abs(out.float().numpy() - want).max() <= TOL["f16"]
