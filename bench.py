@@ -43,6 +43,7 @@ sys.path.insert(0, ROOT)
 import workloads  # noqa: E402
 
 METRIC = "paged decode attention: KV-cache HBM GB/s (% of peak), seq-steps/s"
+FP8_SCALE = 6.0 / 448.0  # --kv-fp8: one scale for K and V (448 = E4M3's largest value)
 SWAP_METRIC = "block swap device<->pinned host (preempt + resume): GB/s over the host link"
 MULTI_METRIC = ("paged multi-token attention (several new tokens per sequence, causal): KV-cache HBM GB/s "
                 "(% of peak), query-tokens/s")
@@ -60,13 +61,14 @@ DECODE_SOURCES = ["paged_kv_cache_365_b200/csrc/decode.cuh", "paged_kv_cache_365
 # ---------------------------------------------------------------------------
 # workload accounting (algorithmic bytes)
 # ---------------------------------------------------------------------------
-def kv_bytes(wl, unique: bool) -> int:
+def kv_bytes(wl, unique: bool, fp8: bool = False) -> int:
     """K+V bytes the decode must read: each token once per kv-head.
 
     With ``unique`` a block shared by several sequences counts once (the
-    shared prefix of the prefix workload); otherwise per sequence.
+    shared prefix of the prefix workload); otherwise per sequence.  ``fp8``:
+    the cache holds one-byte E4M3 codes instead of the workload's dtype.
     """
-    per_tok = wl.kv_bytes_per_token
+    per_tok = wl.kv_bytes_per_token // (STORAGE[wl.dtype] if fp8 else 1)
     logical = int(np.sum(wl.context_lens.astype(np.int64))) * per_tok
     if not unique or wl.name != "prefix13b":
         return logical
@@ -74,11 +76,11 @@ def kv_bytes(wl, unique: bool) -> int:
     return logical - (wl.B - 1) * prefix * per_tok
 
 
-def decode_algorithmic_bytes(wl, unique: bool = True) -> int:
+def decode_algorithmic_bytes(wl, unique: bool = True, fp8: bool = False) -> int:
     """Bytes one decode launch must move: K/V + q in + out + tables + lengths."""
     es = STORAGE[wl.dtype]
     pages = int(np.sum((wl.context_lens.astype(np.int64) + 15) // 16))
-    return kv_bytes(wl, unique) + 2 * wl.B * wl.Hq * wl.D * es + 4 * pages + 4 * wl.B
+    return kv_bytes(wl, unique, fp8) + 2 * wl.B * wl.Hq * wl.D * es + 4 * pages + 4 * wl.B
 
 
 def source_digest() -> str:
@@ -239,7 +241,23 @@ def run_cuda(args, rank, world, local_rank):
     # shared prefix is read once per kv-head)
     pp = pkv.common_prefix_pages(st["host"]["block_tables"], st["host"]["context_lens"])
     use_cascade = (wl.dtype != "f32" and pp >= pkv.api.CASCADE_MIN_PAGES and B >= pkv.api.CASCADE_MIN_SEQS
-                   and not args.no_cascade)
+                   and not args.no_cascade and not args.kv_fp8)
+    fp8 = bool(args.kv_fp8)
+    if fp8:
+        if wl.dtype == "f32":
+            raise SystemExit("--kv-fp8 needs an fp16 / bf16 workload")
+        # the same pool quantised once to E4M3 codes (one scale for K, one
+        # for V, covering ~6 standard deviations of the N(0,1) values)
+        NB, Hkv = cache.k.shape[0], cache.k.shape[1]
+        k8 = torch.empty(cache.k.shape, dtype=torch.uint8, device=dev)
+        v8 = torch.empty(cache.v.shape, dtype=torch.uint8, device=dev)
+        all_slots = torch.arange(NB * 16, dtype=torch.int64, device=dev)
+        for src, dst in ((cache.k, k8), (cache.v, v8)):
+            rows = src.permute(0, 2, 1, 3).reshape(NB * 16, Hkv, D).contiguous()
+            pkv.kv_append_fp8(rows, rows, dst, dst, all_slots, FP8_SCALE, FP8_SCALE)
+            del rows
+        cache.k, cache.v = k8, v8  # the 16-bit pool is released
+        torch.cuda.synchronize()
     prefix = torch.from_numpy(np.ascontiguousarray(st["host"]["block_tables"][0, :pp])).to(dev) if use_cascade else None
     if use_cascade:
         ws = cache.workspace(pkv.decode_prefix_workspace_bytes(B, Hq, D, max_ctx, pp, args.partition))
@@ -252,10 +270,17 @@ def run_cuda(args, rank, world, local_rank):
     def pre_decode():
         if n_pairs:
             pkv.copy_blocks(cache.k, cache.v, st["cow_pairs"])
-        pkv.kv_append(st["k_new"], st["v_new"], cache.k, cache.v, st["slot_mapping"])
+        if fp8:
+            pkv.kv_append_fp8(st["k_new"], st["v_new"], cache.k, cache.v, st["slot_mapping"], FP8_SCALE, FP8_SCALE)
+        else:
+            pkv.kv_append(st["k_new"], st["v_new"], cache.k, cache.v, st["slot_mapping"])
 
     def decode():
-        if use_cascade:
+        if fp8:
+            pkv.paged_attention_decode_fp8(st["q"], cache.k, cache.v, st["block_tables"], st["context_lens"],
+                                           max_ctx, scale, FP8_SCALE, FP8_SCALE, out=out, workspace=ws,
+                                           partition=args.partition)
+        elif use_cascade:
             pkv.paged_attention_decode_prefix(st["q"], cache.k, cache.v, st["block_tables"], st["context_lens"],
                                               max_ctx, prefix, scale, out=out, workspace=ws,
                                               partition=args.partition)
@@ -326,6 +351,18 @@ def run_cuda(args, rank, world, local_rank):
     d2h = out_host.numel() * out_host.element_size()
 
     def e2e_step():
+        if fp8:
+            # the same calls a user makes, inputs from pinned host memory
+            dv = {k: t.to(dev, non_blocking=True) for k, t in host.items()}
+            if n_pairs:
+                pkv.copy_blocks(cache.k, cache.v, dv["cow_pairs"])
+            pkv.kv_append_fp8(dv["k_new"], dv["v_new"], cache.k, cache.v, dv["slot_mapping"], FP8_SCALE,
+                              FP8_SCALE)
+            pkv.paged_attention_decode_fp8(dv["q"], cache.k, cache.v, dv["block_tables"], dv["context_lens"],
+                                           max_ctx, scale, FP8_SCALE, FP8_SCALE, out=out, workspace=ws,
+                                           partition=args.partition)
+            out_host.copy_(out, non_blocking=True)
+            return
         cache.run_step(host["slot_mapping"], host["cow_pairs"], host["block_tables"], host["context_lens"],
                        max_ctx, host["q"], host["k_new"], host["v_new"], out=out_host, scale=scale,
                        partition=args.partition, stream=stream, prefix_blocks=host.get("prefix_blocks"))
@@ -830,6 +867,8 @@ def main(argv=None):
                     help="capture one step in a CUDA graph and replay it (launch-bound batches)")
     ap.add_argument("--no-cascade", action="store_true",
                     help="decode a shared-prefix batch with the plain paged kernel")
+    ap.add_argument("--kv-fp8", action="store_true",
+                    help="the step over an FP8 (E4M3) cache: quantising append + FP8 decode")
     ap.add_argument("--row", choices=["step", "swap", "multi"], default="step",
                     help="step: the decode step (default); swap: preemption by swapping; "
                          "multi: several new tokens per sequence")
@@ -878,10 +917,11 @@ def main(argv=None):
     peak, peak_kind = measured_peak()
     K = r["K"]
     step_s = r["total_ms"] / 1e3 / K
-    kv_unique = kv_bytes(wl, True)
-    kv_logical = kv_bytes(wl, False)
+    fp8 = bool(args.kv_fp8)
+    kv_unique = kv_bytes(wl, True, fp8)
+    kv_logical = kv_bytes(wl, False, fp8)
     value = job_throughput(kv_logical, world, K, r["total_ms"] / 1e3)
-    dec_bytes = decode_algorithmic_bytes(wl, unique=True)
+    dec_bytes = decode_algorithmic_bytes(wl, unique=True, fp8=fp8)
     achieved = dec_bytes / (r["dec_avg_ms"] / 1e3) / 1e9
     e2e_step_s = r["e2e_ms"] / 1e3 / K
     line = {
@@ -899,14 +939,16 @@ def main(argv=None):
                 "us_per_step": 1e6 * e2e_step_s},
         "gpu_launches": r["launches"],
         "cascade_prefix_pages": r["cascade_pages"],
+        "kv_cache": "e4m3 (FP8) codes, scale %.6g for K and V" % FP8_SCALE if fp8 else wl.dtype,
         "roofline": {"kernel": ("paged_decode cascade (prefix/suffix kernel + merge kernel)" if r["cascade_pages"]
+                                else "paged_decode_fp8 (partition + merge kernels)" if fp8
                                 else "paged_decode (partition + merge kernels)"), "bound": "hbm",
                      "achieved": achieved, "peak": peak, "peak_kind": f"{peak_kind} (MEASURED_PEAKS hbm_gbs)"
                      if peak_kind == "measured" else "fallback", "unit": "GB/s", "frac": achieved / peak,
-                     "traffic": recorded_traffic(wl.name), "algorithmic_bytes_per_launch": dec_bytes,
+                     "traffic": None if fp8 else recorded_traffic(wl.name), "algorithmic_bytes_per_launch": dec_bytes,
                      "avg_launch_us": 1e3 * r["dec_avg_ms"]},
     }
-    if world == 1 and not args.no_cpu_baseline:
+    if world == 1 and not args.no_cpu_baseline and not fp8:
         line["cpu_baseline"] = cpu_baseline(wl, seed=args.seed)
     print(json.dumps(line), flush=True)
     return 0

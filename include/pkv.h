@@ -46,7 +46,11 @@ extern "C" {
 #define PKV_BLOCK_SIZE 16
 #define PKV_DEFAULT_PARTITION 512
 
-typedef enum { PKV_F32 = 0, PKV_F16 = 1, PKV_BF16 = 2 } pkv_dtype;
+/* PKV_E4M3: FP8 E4M3 codes (one byte) of an FP8 cache; see
+ * pkv_kv_append_fp8.  Byte copies (pkv_kv_append of codes, pkv_copy_blocks,
+ * pkv_swap_blocks) take it like the others; attention over an FP8 cache is
+ * pkv_paged_attention_decode_fp8. */
+typedef enum { PKV_F32 = 0, PKV_F16 = 1, PKV_BF16 = 2, PKV_E4M3 = 3 } pkv_dtype;
 
 typedef enum {
   PKV_OK = 0,
@@ -273,6 +277,42 @@ pkv_status pkv_paged_attention_decode_static_ws(void* out, const void* q, const 
 /* Read and clear the current device's error word (PKV_ERR_* bits) after the
  * work queued on `stream` so far has finished.  Blocks the host. */
 pkv_status pkv_get_error(uint32_t* flags, void* stream);
+
+/* ------------------------------------------------------------------------
+ * FP8 KV cache: half the bytes of a 16-bit cache per token.
+ *
+ * The pages name FP8 only as a low-precision format of TensorRT-LLM's
+ * operators ("vLLM 推理加速：PagedAttention、FlashAttention 与动态批处理",
+ * "TensorRT-LLM"); the format and the scaling are this library's choice:
+ * OCP FP8 E4M3 (bias 7, subnormals, max 448, no infinities) with one float
+ * scale for all of K and one for all of V.  The pool layout is that of a
+ * 16-bit cache with one-byte elements: [num_blocks, num_kv_heads, 16,
+ * head_dim] uint8 codes; a stored value is code's value * scale.
+ *
+ * pkv_kv_append_fp8: for every token i with slot_mapping[i] >= 0,
+ *   k_cache[slot / 16, h, slot % 16, d] = E4M3(k_new[i, h, d] / k_scale)
+ * (V alike with v_scale): k_new / v_new in src_dtype (fp16 or bf16), the
+ * division in float32 (IEEE, round to nearest), then round to the nearest
+ * E4M3 value, ties to even, magnitudes past 448 saturating to +-448.  Codes
+ * are bit-exact.  Slot rules and errors as pkv_kv_append.  Scales must be
+ * finite and > 0.
+ *
+ * pkv_paged_attention_decode_fp8: pkv_paged_attention_decode over an FP8
+ * cache; q and out in q_dtype (fp16 or bf16);
+ *   s_j = scale * k_scale * q . code(K_j),  out = v_scale * sum_j softmax(s)_j code(V_j)
+ * Same arguments, layouts, workspace (pkv_decode_workspace_bytes) and errors
+ * as pkv_paged_attention_decode.
+ * -------------------------------------------------------------------- */
+pkv_status pkv_kv_append_fp8(const void* k_new, const void* v_new, void* k_cache, void* v_cache,
+                             const int64_t* slot_mapping, int num_tokens, int num_kv_heads, int head_dim,
+                             int num_blocks, pkv_dtype src_dtype, float k_scale, float v_scale, void* stream);
+pkv_status pkv_paged_attention_decode_fp8(void* out, const void* q, const void* k_cache, const void* v_cache,
+                                          const int32_t* block_tables, int max_blocks_per_seq,
+                                          const int32_t* context_lens, int max_context_len, int num_seqs,
+                                          int num_q_heads, int num_kv_heads, int head_dim, int num_blocks,
+                                          float scale, float k_scale, float v_scale, int partition_tokens,
+                                          pkv_dtype q_dtype, void* workspace, size_t workspace_bytes,
+                                          void* stream);
 
 /* ------------------------------------------------------------------------
  * pkv_paged_attention_multi -- paged attention for several query tokens

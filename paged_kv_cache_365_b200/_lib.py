@@ -47,6 +47,11 @@ PROTOTYPES = {
     "pkv_paged_attention_decode_static_ws": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_int,
                                                      c_void_p, c_int, c_int, c_int, c_int, c_int, c_int,
                                                      c_float, c_int, c_int, c_void_p]),
+    "pkv_kv_append_fp8": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_int, c_int, c_int, c_int,
+                                  c_int, c_float, c_float, c_void_p]),
+    "pkv_paged_attention_decode_fp8": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_int, c_void_p,
+                                               c_int, c_int, c_int, c_int, c_int, c_int, c_float, c_float, c_float,
+                                               c_int, c_int, c_void_p, c_size_t, c_void_p]),
     "pkv_multi_workspace_bytes": (c_size_t, [c_int, c_int, c_int, c_int, c_int]),
     "pkv_paged_attention_multi": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_int, c_void_p, c_int,
                                           c_void_p, c_int, c_int, c_int, c_int, c_int, c_int, c_int, c_float, c_int,

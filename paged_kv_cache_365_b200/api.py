@@ -23,7 +23,9 @@ DEFAULT_PARTITION = 512
 # least this many sequences) is decoded with the cascade (prefix read once)
 CASCADE_MIN_PAGES = 8
 CASCADE_MIN_SEQS = 4
-_DT = {torch.float32: 0, torch.float16: 1, torch.bfloat16: 2}
+# an FP8 cache holds E4M3 codes: torch.float8_e4m3fn, or uint8 bytes
+_DT = {torch.float32: 0, torch.float16: 1, torch.bfloat16: 2, torch.float8_e4m3fn: 3, torch.uint8: 3}
+_FP8 = (torch.float8_e4m3fn, torch.uint8)
 
 
 def kv_cache_bytes(num_layers: int, num_heads: int, head_dim: int, seq_len: int, dtype_bytes: int) -> int:
@@ -137,6 +139,57 @@ def swap_blocks(dst_k: torch.Tensor, dst_v: torch.Tensor, src_k: torch.Tensor, s
     check(lib.pkv_swap_blocks(_any(dst_k, "dst_k"), _any(dst_v, "dst_v"), dnb, _any(src_k, "src_k"),
                               _any(src_v, "src_v"), snb, _any(pairs, "pairs", torch.int32), n, hkv, d,
                               _DT[dst_k.dtype], _stream(stream, device)), "pkv_swap_blocks")
+
+
+def kv_append_fp8(k_new: torch.Tensor, v_new: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
+                  slot_mapping: torch.Tensor, k_scale: float, v_scale: float, stream=None) -> None:
+    """Quantise each new token's K/V (fp16/bf16 [N, Hkv, D]) into its slot of
+    an FP8 cache: code = E4M3(x / scale), one scale for K and one for V."""
+    nb, hkv, d = _cache_dims(k_cache, v_cache)
+    if k_cache.dtype not in _FP8:
+        raise ValueError("kv_append_fp8 writes an FP8 cache (float8_e4m3fn or uint8)")
+    if k_new.shape != v_new.shape or k_new.dim() != 3 or tuple(k_new.shape[1:]) != (hkv, d):
+        raise ValueError("k_new/v_new must be [N, Hkv, D] matching the cache")
+    if k_new.dtype not in (torch.float16, torch.bfloat16) or v_new.dtype != k_new.dtype:
+        raise ValueError("k_new/v_new must be fp16 or bf16")
+    n = k_new.shape[0]
+    if slot_mapping.shape != (n,):
+        raise ValueError("slot_mapping must be [N]")
+    check(lib.pkv_kv_append_fp8(_dev(k_new, "k_new"), _dev(v_new, "v_new"), _dev(k_cache, "k_cache"),
+                                _dev(v_cache, "v_cache"), _dev(slot_mapping, "slot_mapping", torch.int64), n, hkv, d,
+                                nb, _DT[k_new.dtype], float(k_scale), float(v_scale),
+                                _stream(stream, k_cache.device)), "pkv_kv_append_fp8")
+
+
+def paged_attention_decode_fp8(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
+                               block_tables: torch.Tensor, context_lens: torch.Tensor, max_context_len: int,
+                               scale: float, k_scale: float, v_scale: float, out: Optional[torch.Tensor] = None,
+                               workspace: Optional[torch.Tensor] = None, partition: int = 0,
+                               stream=None) -> torch.Tensor:
+    """paged_attention_decode over an FP8 cache (E4M3 codes, one scale for K
+    and one for V); q and the output in fp16 or bf16."""
+    nb, hkv, d = _cache_dims(k_cache, v_cache)
+    if k_cache.dtype not in _FP8:
+        raise ValueError("an FP8 cache (float8_e4m3fn or uint8) is required")
+    if q.dim() != 3 or q.shape[2] != d or q.dtype not in (torch.float16, torch.bfloat16):
+        raise ValueError("q must be [B, Hq, D] in fp16 or bf16")
+    B, hq, _ = q.shape
+    if block_tables.dim() != 2 or block_tables.shape[0] != B or context_lens.shape != (B,):
+        raise ValueError("block_tables must be [B, max_blocks] and context_lens [B]")
+    if out is None:
+        out = torch.empty_like(q)
+    need = decode_workspace_bytes(B, hq, d, max_context_len, partition)
+    if need and (workspace is None or workspace.numel() * workspace.element_size() < need):
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    ws_ptr = _dev(workspace, "workspace") if need else None
+    ws_len = workspace.numel() * workspace.element_size() if need else 0
+    check(lib.pkv_paged_attention_decode_fp8(
+        _dev(out, "out", q.dtype), _dev(q, "q"), _dev(k_cache, "k_cache"), _dev(v_cache, "v_cache"),
+        _dev(block_tables, "block_tables", torch.int32), block_tables.shape[1],
+        _dev(context_lens, "context_lens", torch.int32), int(max_context_len), B, hq, hkv, d, nb, float(scale),
+        float(k_scale), float(v_scale), int(partition), _DT[q.dtype], ws_ptr, ws_len, _stream(stream, q.device)),
+        "pkv_paged_attention_decode_fp8")
+    return out
 
 
 def decode_workspace_bytes(num_seqs: int, num_q_heads: int, head_dim: int, max_context_len: int,

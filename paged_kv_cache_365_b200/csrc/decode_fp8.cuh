@@ -1,0 +1,411 @@
+// Paged decode over an FP8 (E4M3) KV cache, queries in fp16 or bf16.
+//
+// The cache stores code = E4M3(x / scale) with one scale for K and one for
+// V (see pkv.h); a K/V tile is half the bytes of a 16-bit one, so a decode
+// step streams half the HBM bytes.  Work split, staging and merging are
+// those of paged_decode_mma_kernel (decode_mma.cuh): one CTA per (kv-head,
+// sequence, partition), warp w walks pages w, w + NWARPS, ... with its own
+// ring of TMA-staged tiles (16 rows x D bytes, swizzled), per-warp online
+// softmax, fixed-order merge.  What changes is how a page is consumed:
+//
+//  * Q.K on the 16-bit tensor cores, S^T[16 tokens x 8] = K . Q^T: ldmatrix
+//    reads the FP8 tile as 16-bit pairs, so lane (g, t) receives the 4
+//    bytes d = 16c + 4t .. 16c + 4t + 3 of chunk c; each E4M3 pair is
+//    converted exactly to two 16-bit values.  The MMA's k index 2t, 2t+1,
+//    2t+8, 2t+9 then stands for d = 16c + 4t .. + 3, and the queries (the
+//    B operand, in registers) are loaded in that same order of d, so the
+//    dot product runs over the same pairs.
+//  * P.V with P as the A operand (queries as M) and V as the B operand,
+//    O[8 queries x D]: lane (g, t) needs V[token][d] for tokens 2t, 2t+1,
+//    2t+8, 2t+9 and column g of every n-tile; with d = (D/8) n + j for
+//    n-tile j and column n, those are D/8 consecutive bytes of four rows:
+//    four shared loads, byte permutes and exact E4M3 -> 16-bit conversions.
+//    Rows 0-7 of A carry the high 16-bit part of P, rows 8-15 the low part,
+//    so one MMA per n-tile accumulates both (their sum is the result).
+//  * The K scale is folded into the logit scale, the V scale into the
+//    output.
+#pragma once
+
+#include "decode_mma.cuh"
+
+namespace pkv {
+
+// E4M3 pair (low byte -> low half) to two 16-bit floats of type T (exact:
+// every E4M3 value is an fp16 and a bf16 value).
+template <typename T>
+__device__ __forceinline__ uint32_t e4m3x2_to(uint32_t pair16);
+
+template <>
+__device__ __forceinline__ uint32_t e4m3x2_to<__half>(uint32_t pair16) {
+  uint32_t d;
+  const unsigned short a = static_cast<unsigned short>(pair16);
+  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(d) : "h"(a));
+  return d;
+}
+
+template <>
+__device__ __forceinline__ uint32_t e4m3x2_to<__nv_bfloat16>(uint32_t pair16) {
+  const uint32_t h = e4m3x2_to<__half>(pair16);
+  const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&h));
+  const __nv_bfloat162 b = __floats2bfloat162_rn(f.x, f.y);  // exact
+  return *reinterpret_cast<const uint32_t*>(&b);
+}
+
+// Byte offset of 16-byte chunk `chunk` of row `row` in an FP8 tile of 16
+// rows x D bytes stored with the TMA swizzle matching its row length
+// (128-byte rows: chunk ^ (row & 7); 64-byte rows: chunk ^ ((row >> 1) & 3)).
+template <int D>
+__device__ __forceinline__ uint32_t swz8(int row, int chunk) {
+  if constexpr (D == 128)
+    return static_cast<uint32_t>(row * 128 + ((chunk ^ (row & 7)) << 4));
+  else
+    return static_cast<uint32_t>(row * 64 + ((chunk ^ ((row >> 1) & 3)) << 4));
+}
+
+template <int D, int NWARPS, int NSTAGE>
+struct Fp8Shape {
+  static constexpr int kTile = kBlockSize * D;  // bytes of a (block, kv-head) tile
+  static constexpr int kStage = 2 * kTile;      // K + V
+  static constexpr int kChunks = D / 16;        // 16-byte chunks per row
+  static constexpr int kWarpStageBytes = NSTAGE * kStage;
+  static constexpr size_t kSmemStages = size_t(NWARPS) * kWarpStageBytes;
+  static constexpr size_t kSmem = 1024 + kSmemStages + size_t(NWARPS) * NSTAGE * 8;
+  static constexpr int kRecM = 8 * D, kRecL = 8 * D + 8;
+  static constexpr int kTab = (128 + 32 * NWARPS - 1) / (32 * NWARPS);
+  static_assert(D == 64 || D == 128, "a tile row is one swizzle span");
+  static_assert(size_t(8) * (D + 2) * sizeof(float) <= size_t(kWarpStageBytes),
+                "a warp's merge record must fit in its own stages");
+  static_assert(kTile % 512 == 0, "swizzled tiles want 512/1024-byte alignment");
+};
+
+template <typename T, int D, int G, int NWARPS, int NSTAGE>
+__global__ void __launch_bounds__(NWARPS * 32)
+    paged_decode_fp8_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tmap_k,
+                            const __grid_constant__ CUtensorMap tmap_v, float v_scale) {
+  pdl_enter();
+  using S = Fp8Shape<D, NWARPS, NSTAGE>;
+  using M = Mma<T>;
+  constexpr int kNT = D / 8;  // PV n-tiles; also the d values a column spans
+  const int kvh = blockIdx.x;
+  const int b = blockIdx.y;
+  const int part = blockIdx.z;
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int g8 = lane >> 2, t4 = lane & 3, lm = lane >> 3, lr = lane & 7;
+
+  int ctx = a.context_lens[b];
+  if (ctx < 0 || ctx > a.max_ctx) {
+    if (threadIdx.x == 0 && kvh == 0 && part == 0) raise_error(PKV_ERR_CONTEXT_RANGE);
+    ctx = ctx < 0 ? 0 : a.max_ctx;
+  }
+  const int nparts = (ctx + a.partition - 1) / a.partition;
+  if (part >= (nparts > 0 ? nparts : 1)) return;
+  if (ctx == 0) {
+    T* out = reinterpret_cast<T*>(a.out) + (static_cast<size_t>(b) * a.num_q_heads + kvh * G) * D;
+    for (int i = threadIdx.x; i < G * D; i += NWARPS * 32) out[i] = Fmt<T>::from_f32(0.f);
+    return;
+  }
+  auto col_row = [&](int n) -> size_t { return static_cast<size_t>(b) * a.num_q_heads + kvh * G + n; };
+
+  extern __shared__ unsigned char smem_raw[];
+  const uint32_t raw_addr = smem_addr(smem_raw);
+  const uint32_t pad = ((raw_addr + 1023u) & ~1023u) - raw_addr;
+  unsigned char* smem = smem_raw + pad;
+  unsigned char* my_stages = smem + static_cast<size_t>(warp) * S::kWarpStageBytes;
+  const uint32_t stage0 = smem_addr(my_stages);
+  const uint32_t bar0 = smem_addr(smem + S::kSmemStages) + warp * NSTAGE * 8;
+  if (lane == 0) {
+    for (int s = 0; s < NSTAGE; ++s) mbar_init(bar0 + 8 * s, 1);
+    fence_barrier_init();
+  }
+  __syncwarp();
+
+  // Q^T as B fragments in the d order the converted K fragments use:
+  // chunk c: b0 = q[16c + 4t .. +1], b1 = q[16c + 4t + 2 .. +3]
+  uint32_t qb[S::kChunks][2];
+  {
+    const bool ok = g8 < G;
+    const T* qp = reinterpret_cast<const T*>(a.q) + (ok ? col_row(g8) : 0) * D;
+#pragma unroll
+    for (int c = 0; c < S::kChunks; ++c) {
+      qb[c][0] = ok ? *reinterpret_cast<const uint32_t*>(qp + 16 * c + 4 * t4) : 0u;
+      qb[c][1] = ok ? *reinterpret_cast<const uint32_t*>(qp + 16 * c + 4 * t4 + 2) : 0u;
+    }
+  }
+
+  const int tok0 = part * a.partition;
+  const int tok1 = min(ctx, tok0 + a.partition);
+  const int pg0 = tok0 / kBlockSize;
+  const int nblk = (tok1 - tok0 + kBlockSize - 1) / kBlockSize;
+  const int my_n = warp < nblk ? (nblk - warp + NWARPS - 1) / NWARPS : 0;
+  int my_phys[S::kTab];
+#pragma unroll
+  for (int h = 0; h < S::kTab; ++h) {
+    my_phys[h] = -1;
+    const int j = lane + 32 * h;
+    if (j < my_n) {
+      const int e = a.block_tables[static_cast<long long>(b) * a.bt_stride + pg0 + warp + j * NWARPS];
+      if (e >= 0 && e < a.num_blocks)
+        my_phys[h] = e;
+      else
+        raise_error(PKV_ERR_BLOCK_RANGE);
+    }
+  }
+  auto phys_of = [&](int i) {
+    int r = -1;
+#pragma unroll
+    for (int h = 0; h < S::kTab; ++h) {
+      const int v = __shfl_sync(kFull, my_phys[h], i & 31);
+      if ((i >> 5) == h) r = v;
+    }
+    return r;
+  };
+  uint32_t phase_bits = 0;
+  auto issue = [&](int i) {
+    const int phys = phys_of(i);
+    if (lane == 0 && i < my_n) {
+      const uint32_t bar = bar0 + 8 * (i % NSTAGE);
+      if (phys >= 0) {
+        const uint32_t dst = stage0 + (i % NSTAGE) * S::kStage;
+        const int y = (phys * a.num_kv_heads + kvh) * kBlockSize;
+        fence_proxy_async_smem();
+        mbar_arrive_expect_tx(bar, S::kStage);
+        tma_load_2d(dst, &tmap_k, 0, y, bar);
+        tma_load_2d(dst + S::kTile, &tmap_v, 0, y, bar);
+      } else {
+        mbar_arrive(bar);
+      }
+    }
+  };
+#pragma unroll
+  for (int i = 0; i < NSTAGE; ++i) issue(i);
+
+  // O[query g8][d]: n-tile j, columns 2 t4, 2 t4 + 1 -> d = kNT (2 t4) + j,
+  // kNT (2 t4 + 1) + j; [0..1] from P's high part, [2..3] from its low part
+  float o[kNT][4];
+#pragma unroll
+  for (int j = 0; j < kNT; ++j) o[j][0] = o[j][1] = o[j][2] = o[j][3] = 0.f;
+  float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;  // query columns 2 t4, 2 t4 + 1
+  int consumed = 0;
+  bool timed_out = false;
+
+  for (int i = 0; i < my_n; ++i) {
+    const int s = i % NSTAGE;
+    bool ok = mbar_wait_bounded(bar0 + 8 * s, (phase_bits >> s) & 1u);
+    phase_bits ^= 1u << s;
+    ok = __all_sync(kFull, ok);
+    if (!ok) {
+      if (lane == 0) raise_error(PKV_ERR_TIMEOUT);
+      timed_out = true;
+      break;
+    }
+    consumed = i + 1;
+    if (phys_of(i) >= 0) {
+      const int page_tok = tok0 + (warp + i * NWARPS) * kBlockSize;
+      const int nvalid = min(kBlockSize, tok1 - page_tok);
+      const uint32_t kt = stage0 + s * S::kStage;
+      const uint32_t vt = kt + S::kTile;
+      // (1) S^T = K . Q^T, two chunks of d per ldmatrix
+      float sc[4] = {0.f, 0.f, 0.f, 0.f};
+      {
+        const int row = lr + ((lm & 1) << 3);
+#pragma unroll
+        for (int c = 0; c < S::kChunks; c += 2) {
+          uint32_t r0, r1, r2, r3;
+          ldsm_x4(kt + swz8<D>(row, c + (lm >> 1)), r0, r1, r2, r3);
+          M::run(sc, e4m3x2_to<T>(r0 & 0xffffu), e4m3x2_to<T>(r1 & 0xffffu), e4m3x2_to<T>(r0 >> 16),
+                 e4m3x2_to<T>(r1 >> 16), qb[c][0], qb[c][1]);
+          M::run(sc, e4m3x2_to<T>(r2 & 0xffffu), e4m3x2_to<T>(r3 & 0xffffu), e4m3x2_to<T>(r2 >> 16),
+                 e4m3x2_to<T>(r3 >> 16), qb[c + 1][0], qb[c + 1][1]);
+        }
+      }
+      // (2) scale (K scale folded in), mask the tail, online softmax
+      const bool v_lo = g8 < nvalid, v_hi = g8 + 8 < nvalid;
+      const float x0 = v_lo ? sc[0] * a.qk_scale : -INFINITY;
+      const float x1 = v_lo ? sc[1] * a.qk_scale : -INFINITY;
+      const float x2 = v_hi ? sc[2] * a.qk_scale : -INFINITY;
+      const float x3 = v_hi ? sc[3] * a.qk_scale : -INFINITY;
+      float mx0 = fmaxf(x0, x2), mx1 = fmaxf(x1, x3);
+#pragma unroll
+      for (int msk = 4; msk <= 16; msk <<= 1) {
+        mx0 = fmaxf(mx0, __shfl_xor_sync(kFull, mx0, msk));
+        mx1 = fmaxf(mx1, __shfl_xor_sync(kFull, mx1, msk));
+      }
+      const float n0 = fmaxf(m0, mx0), n1 = fmaxf(m1, mx1);
+      const float al0 = exp2f(m0 - n0), al1 = exp2f(m1 - n1);
+      m0 = n0;
+      m1 = n1;
+      const float p0 = exp2f(x0 - n0), p1 = exp2f(x1 - n1), p2 = exp2f(x2 - n0), p3 = exp2f(x3 - n1);
+      l0 = fmaf(l0, al0, p0 + p2);
+      l1 = fmaf(l1, al1, p1 + p3);
+      // this lane's O rows belong to query g8: its factor comes from the
+      // lane holding query column g8 (t4 = g8 / 2)
+      const float ae = __shfl_sync(kFull, al0, g8 >> 1), ao = __shfl_sync(kFull, al1, g8 >> 1);
+      const float alpha = (g8 & 1) ? ao : ae;
+      if (__any_sync(kFull, alpha != 1.f)) {
+#pragma unroll
+        for (int j = 0; j < kNT; ++j) {
+          o[j][0] *= alpha;
+          o[j][1] *= alpha;
+          o[j][2] *= alpha;
+          o[j][3] *= alpha;
+        }
+      }
+      // (3) P as A fragments: rows g8 = P high part, rows g8 + 8 = low part
+      const uint32_t top_hi = M::pack(p0, p1), bot_hi = M::pack(p2, p3);
+      const float2 th = M::unpack(top_hi), bh = M::unpack(bot_hi);
+      const uint32_t top_lo = M::pack(p0 - th.x, p1 - th.y), bot_lo = M::pack(p2 - bh.x, p3 - bh.y);
+      const uint32_t pa0 = movm_t(top_hi), pa1 = movm_t(top_lo), pa2 = movm_t(bot_hi), pa3 = movm_t(bot_lo);
+      // (4) bytes d = kNT g8 .. kNT g8 + kNT - 1 (in 16-byte chunk vch, from
+      // byte vb0) of rows 2 t4, 2 t4 + 1, 2 t4 + 8, 2 t4 + 9; rows past the
+      // context are zeroed (an unused slot may hold a NaN code)
+      constexpr int kW = kNT / 4;  // 32-bit words per row segment (4 or 2)
+      const int vch = (kNT * g8) >> 4, vb0 = (kNT * g8) & 15;
+      uint32_t w0[kW], w1[kW], w8[kW], w9[kW];
+      {
+        const unsigned char* vbase = my_stages + s * S::kStage + S::kTile;
+        auto load = [&](int row, uint32_t (&w)[kW]) {
+          const unsigned char* p = vbase + swz8<D>(row, vch) + vb0;
+          if constexpr (kW == 4) {
+            const uint4 v = row < nvalid ? *reinterpret_cast<const uint4*>(p) : make_uint4(0u, 0u, 0u, 0u);
+            w[0] = v.x;
+            w[1] = v.y;
+            w[2] = v.z;
+            w[3] = v.w;
+          } else {
+            const uint2 v = row < nvalid ? *reinterpret_cast<const uint2*>(p) : make_uint2(0u, 0u);
+            w[0] = v.x;
+            w[1] = v.y;
+          }
+        };
+        load(2 * t4, w0);
+        load(2 * t4 + 1, w1);
+        load(2 * t4 + 8, w8);
+        load(2 * t4 + 9, w9);
+      }
+      // n-tile j uses byte j of each row segment; two n-tiles per permute
+#pragma unroll
+      for (int j = 0; j < kNT; j += 2) {
+        const int w = j >> 2, bsel = j & 3;
+        // (row a byte j, row b byte j, row a byte j+1, row b byte j+1)
+        const uint32_t sel = bsel | ((4 + bsel) << 4) | ((bsel + 1) << 8) | ((5 + bsel) << 12);
+        const uint32_t lo01 = __byte_perm(w0[w], w1[w], sel);
+        const uint32_t lo89 = __byte_perm(w8[w], w9[w], sel);
+        const uint32_t b0j = e4m3x2_to<T>(lo01 & 0xffffu), b0k = e4m3x2_to<T>(lo01 >> 16);
+        const uint32_t b1j = e4m3x2_to<T>(lo89 & 0xffffu), b1k = e4m3x2_to<T>(lo89 >> 16);
+        M::run(o[j], pa0, pa1, pa2, pa3, b0j, b1j);
+        M::run(o[j + 1], pa0, pa1, pa2, pa3, b0k, b1k);
+      }
+    }
+    __syncwarp();
+    issue(i + NSTAGE);
+  }
+  if (consumed < my_n) {
+    const int last = min(my_n, consumed + NSTAGE);
+    for (int i = consumed + 1; i < last; ++i) {
+      const int s = i % NSTAGE;
+      mbar_wait_bounded(bar0 + 8 * s, (phase_bits >> s) & 1u);
+      phase_bits ^= 1u << s;
+    }
+  }
+#pragma unroll
+  for (int msk = 4; msk <= 16; msk <<= 1) {
+    l0 += __shfl_xor_sync(kFull, l0, msk);
+    l1 += __shfl_xor_sync(kFull, l1, msk);
+  }
+
+  // warp record [o: 8 x D][m: 8][l: 8]
+  float* rec = reinterpret_cast<float*>(my_stages);
+  if (g8 < G) {
+#pragma unroll
+    for (int j = 0; j < kNT; ++j) {
+      rec[g8 * D + kNT * (2 * t4) + j] = o[j][0] + o[j][2];
+      rec[g8 * D + kNT * (2 * t4 + 1) + j] = o[j][1] + o[j][3];
+    }
+  }
+  if (g8 == 0) {
+    if (2 * t4 < G) {
+      rec[S::kRecM + 2 * t4] = m0;
+      rec[S::kRecL + 2 * t4] = l0;
+    }
+    if (2 * t4 + 1 < G) {
+      rec[S::kRecM + 2 * t4 + 1] = m1;
+      rec[S::kRecL + 2 * t4 + 1] = l1;
+    }
+  }
+  if (__syncthreads_or(timed_out)) return;
+
+  for (int idx = threadIdx.x; idx < G * D; idx += NWARPS * 32) {
+    const int g = idx / D, d = idx % D;
+    float Mx = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < NWARPS; ++w)
+      Mx = fmaxf(Mx, reinterpret_cast<const float*>(smem + w * S::kWarpStageBytes)[S::kRecM + g]);
+    float num = 0.f, den = 0.f;
+#pragma unroll
+    for (int w = 0; w < NWARPS; ++w) {
+      const float* r = reinterpret_cast<const float*>(smem + w * S::kWarpStageBytes);
+      const float sc = exp2f(r[S::kRecM + g] - Mx);
+      num = fmaf(sc, r[g * D + d], num);
+      den = fmaf(sc, r[S::kRecL + g], den);
+    }
+    num *= v_scale;
+    const size_t row = col_row(g);
+    if (nparts == 1) {
+      reinterpret_cast<T*>(a.out)[row * D + d] = Fmt<T>::from_f32(num / den);
+    } else {
+      const size_t wrow = row * a.num_parts + part;
+      a.ws_o[wrow * D + d] = num;
+      if (d == 0) a.ws_ml[wrow] = make_float2(Mx, den);
+    }
+  }
+}
+
+// Slot-mapped append into an FP8 cache: code = E4M3(x / scale) (x fp16 or
+// bf16, the division in float32, round to nearest even, saturating at
+// +-448).  One thread converts 8 elements (16 bytes in, 8 bytes out).
+// Chunks [0, total) are K, [total, 2 total) V; total = tokens * Hkv * D / 8.
+template <typename T>
+__global__ void __launch_bounds__(256)
+    kv_append_fp8_kernel(const uint4* __restrict__ k_new, const uint4* __restrict__ v_new,
+                         uint2* __restrict__ k_cache, uint2* __restrict__ v_cache, const int64_t* __restrict__ slots,
+                         long long total, int Hkv, int row_chunks, int num_blocks, float k_scale, float v_scale) {
+  pdl_enter();
+  const long long stride = static_cast<long long>(gridDim.x) * blockDim.x;
+  for (long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; i < 2 * total; i += stride) {
+    const bool is_v = i >= total;
+    const long long j = is_v ? i - total : i;
+    const int c = static_cast<int>(j % row_chunks);
+    const long long th = j / row_chunks;
+    const int h = static_cast<int>(th % Hkv);
+    const long long t = th / Hkv;
+    const int64_t s = slots[t];
+    if (s < 0) continue;
+    const int64_t blk = s / kBlockSize;
+    const int off = static_cast<int>(s % kBlockSize);
+    if (blk >= num_blocks) {
+      raise_error(PKV_ERR_SLOT_RANGE);
+      continue;
+    }
+    const uint4 in = (is_v ? v_new : k_new)[j];
+    const float sc = is_v ? v_scale : k_scale;
+    const uint32_t w[4] = {in.x, in.y, in.z, in.w};
+    uint32_t packed[2];
+#pragma unroll
+    for (int p = 0; p < 2; ++p) {
+      unsigned short q2[2];
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh) {
+        const float2 f = Mma<T>::unpack(w[2 * p + hh]);
+        const float x0 = __fdiv_rn(f.x, sc), x1 = __fdiv_rn(f.y, sc);
+        // first operand -> upper byte, second -> lower byte
+        asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(q2[hh]) : "f"(x1), "f"(x0));
+      }
+      packed[p] = static_cast<uint32_t>(q2[0]) | (static_cast<uint32_t>(q2[1]) << 16);
+    }
+    const long long dst = ((blk * Hkv + h) * kBlockSize + off) * row_chunks + c;
+    (is_v ? v_cache : k_cache)[dst] = make_uint2(packed[0], packed[1]);
+  }
+}
+
+}  // namespace pkv

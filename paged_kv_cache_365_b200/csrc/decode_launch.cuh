@@ -40,6 +40,7 @@ int dtype_bytes(pkv_dtype dt) {
     case PKV_F32: return 4;
     case PKV_F16: return 2;
     case PKV_BF16: return 2;
+    case PKV_E4M3: return 1;
   }
   return 0;
 }

@@ -8,20 +8,20 @@
 // new token i sits at position ctx - n_b + i and attends over positions
 // 0 .. ctx - n_b + i (§1: every token so far, itself included).
 //
-// Work split: one CTA per (kv-head, sequence, tile of 16 query rows,
+// Work split: one CTA per (kv-head, sequence, tile of 8 NT query rows,
 // partition of keys).  A tile's rows are (token, head) pairs of one
-// kv-head: row r is token r / G, head r % G of the group, so one tile
-// covers 16 / G tokens and every K/V tile of the sequence is read once per
-// kv-head and row tile.  Within the CTA, warp w walks pages w, w + NWARPS,
-// ... of the partition with its own ring of TMA-staged tiles (as in the
-// decode kernel) and keeps all 16 rows' state; the warps' states are merged
-// in a fixed order at the end.  Per page:
-//   S[16 rows x 16 tokens] = Q[16 x D] . K^T   (A = Q in registers,
-//                                               B = K via ldmatrix)
-//   causal mask: token j of row r counts when j <= pos(r)
-//   O[16 x D] += P . V                           (A = P from the S
-//                                               fragments, hi + lo parts,
-//                                               B = V via ldmatrix.trans)
+// kv-head: row r is token r / G, head r % G of the group; they are the
+// MMA's N dimension in NT n-tiles of 8, exactly as the GQA group is in the
+// decode kernel, so one page's K and V fragments are loaded once and serve
+// every row of the tile (NT is chosen per launch from the rows a sequence
+// brings: a speculative-verification pass of a few tokens is one tile).
+// Within the CTA, warp w walks pages w, w + NWARPS, ... of the partition
+// with its own ring of TMA-staged tiles and keeps every row's state; the
+// warps' states are merged in a fixed order at the end.  Per page:
+//   S^T[16 tokens x 8 NT] = K . Q^T   (A = K via ldmatrix, B = queries)
+//   causal mask: token j counts for row r when j <= pos(r)
+//   O^T[D x 8 NT] += V^T . P^T         (A = V via ldmatrix.trans,
+//                                       B = P^T by movmatrix, hi + lo parts)
 // A key partition past a tile's last position is skipped.  Sequences whose
 // whole context fits one partition write normalised rows; the others write
 // per-partition partials that paged_multi_merge_kernel combines.
@@ -72,16 +72,16 @@ __device__ __forceinline__ bool multi_seq(const MultiArgs& a, int b, int& ctx, i
   return true;
 }
 
-template <typename T, int D, int G, int NWARPS, int NSTAGE>
+template <typename T, int D, int G, int NT, int NWARPS, int NSTAGE>
 __global__ void __launch_bounds__(NWARPS * 32)
     paged_multi_mma_kernel(const MultiArgs a, const __grid_constant__ CUtensorMap tmap_k,
                            const __grid_constant__ CUtensorMap tmap_v) {
   pdl_enter();
   using S = MmaShape<T, D, G, NWARPS, NSTAGE>;
   using M = Mma<T>;
-  constexpr int kNTiles = D / 8;  // PV n-tiles (8 columns of d each)
-  constexpr int kRec = 16 * D;    // warp record: o[16][D], m[16], l[16]
-  static_assert(size_t(kRec + 32) * sizeof(float) <= size_t(S::kWarpStageBytes),
+  constexpr int kCols = 8 * NT;                 // query rows of a tile (the MMA's N)
+  constexpr int kRecM = kCols * D, kRecL = kCols * D + kCols;  // warp record: o[kCols][D], m, l
+  static_assert(size_t(kRecL + kCols) * sizeof(float) <= size_t(S::kWarpStageBytes),
                 "a warp's record must fit in its own stages");
   const int kvh = blockIdx.x;
   const int b = blockIdx.y / a.tiles;
@@ -93,11 +93,11 @@ __global__ void __launch_bounds__(NWARPS * 32)
 
   int ctx, q0, nq;
   if (!multi_seq(a, b, ctx, q0, nq, threadIdx.x == 0 && kvh == 0 && tile == 0 && z == 0)) return;
-  const int R = nq * G;      // rows of this kv-head
-  const int r0 = tile * 16;  // first row of the tile
+  const int R = nq * G;          // rows of this kv-head: row r = token r / G, head r % G
+  const int r0 = tile * kCols;   // first row of the tile
   if (r0 >= R) return;
-  const int base = ctx - nq;  // position of new token 0
-  const int p_hi = base + (min(R, r0 + 16) - 1) / G;
+  const int base = ctx - nq;     // position of new token 0
+  const int p_hi = base + (min(R, r0 + kCols) - 1) / G;
   const bool direct = ctx <= a.partition;  // one partition holds every key of the sequence
   const int tok0 = z * a.partition;
   const int tok1 = min(min(ctx, tok0 + a.partition), p_hi + 1);
@@ -108,7 +108,7 @@ __global__ void __launch_bounds__(NWARPS * 32)
     // no key of this partition is visible to the tile; with one partition
     // (z = 0) every row sits before position 0: zeros
     if (direct && z == 0)
-      for (int idx = threadIdx.x; idx < 16 * D; idx += NWARPS * 32) {
+      for (int idx = threadIdx.x; idx < kCols * D; idx += NWARPS * 32) {
         const int tr = r0 + idx / D;
         if (tr < R) reinterpret_cast<T*>(a.out)[out_row(tr) * D + idx % D] = Fmt<T>::from_f32(0.f);
       }
@@ -176,28 +176,36 @@ __global__ void __launch_bounds__(NWARPS * 32)
 #pragma unroll
   for (int i = 0; i < NSTAGE; ++i) issue(i);
 
-  // A fragments of the tile's rows g8 and g8 + 8 (zero past the rows), and
-  // their positions (-1: sees no key)
-  const int ra = r0 + g8, rb = r0 + g8 + 8;
-  const int posA = ra < R ? base + ra / G : -1;
-  const int posB = rb < R ? base + rb / G : -1;
-  uint32_t qa[S::kKSteps][4];
-  {
-    const T* pa = ra < R ? reinterpret_cast<const T*>(a.q) + out_row(ra) * D : nullptr;
-    const T* pb = rb < R ? reinterpret_cast<const T*>(a.q) + out_row(rb) * D : nullptr;
+  // Q^T B fragments of column g8 of every n-tile (zero past the rows), and
+  // the positions of this lane's columns 2 t4, 2 t4 + 1 (-1: sees no key)
+  uint32_t qb[NT][S::kKSteps][2];
+  int pos[NT][2];
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt) {
+    const int tr = r0 + 8 * nt + g8;
+    const bool ok = tr < R;
+    const T* qp = reinterpret_cast<const T*>(a.q) + (ok ? out_row(tr) : 0) * D;
 #pragma unroll
     for (int ks = 0; ks < S::kKSteps; ++ks) {
-      const int d = ks * 16 + 2 * t4;
-      qa[ks][0] = pa ? *reinterpret_cast<const uint32_t*>(pa + d) : 0u;
-      qa[ks][1] = pb ? *reinterpret_cast<const uint32_t*>(pb + d) : 0u;
-      qa[ks][2] = pa ? *reinterpret_cast<const uint32_t*>(pa + d + 8) : 0u;
-      qa[ks][3] = pb ? *reinterpret_cast<const uint32_t*>(pb + d + 8) : 0u;
+      qb[nt][ks][0] = ok ? *reinterpret_cast<const uint32_t*>(qp + ks * 16 + 2 * t4) : 0u;
+      qb[nt][ks][1] = ok ? *reinterpret_cast<const uint32_t*>(qp + ks * 16 + 8 + 2 * t4) : 0u;
+    }
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+      const int c = r0 + 8 * nt + 2 * t4 + e;
+      pos[nt][e] = c < R ? base + c / G : -1;
     }
   }
-  float o[kNTiles][4];
+
+  // O^T accumulators: o[nt][mt] = rows d = 16 mt + g8 (+8), columns 2 t4 (+1)
+  float o[NT][S::kKSteps][4];
 #pragma unroll
-  for (int j = 0; j < kNTiles; ++j) o[j][0] = o[j][1] = o[j][2] = o[j][3] = 0.f;
-  float mA = -INFINITY, mB = -INFINITY, lA = 0.f, lB = 0.f;
+  for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+    for (int mt = 0; mt < S::kKSteps; ++mt) o[nt][mt][0] = o[nt][mt][1] = o[nt][mt][2] = o[nt][mt][3] = 0.f;
+  float mr[NT][2], lr_[NT][2];
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt) mr[nt][0] = mr[nt][1] = -INFINITY, lr_[nt][0] = lr_[nt][1] = 0.f;
   int consumed = 0;
   bool timed_out = false;
 
@@ -217,92 +225,89 @@ __global__ void __launch_bounds__(NWARPS * 32)
       const int nvalid = min(kBlockSize, tok1 - page_tok);
       const uint32_t kt = stage0 + s * S::kStage;
       const uint32_t vt = kt + S::kTile;
-      // (1) S = Q . K^T
-      float sc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+      // (1) S^T = K . Q^T for every n-tile, K fragments loaded once
+      float sc[NT][4];
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) sc[nt][0] = sc[nt][1] = sc[nt][2] = sc[nt][3] = 0.f;
       {
-        const int row = lr + ((lm >> 1) << 3);  // token
+        const int row = lr + ((lm & 1) << 3);
 #pragma unroll
         for (int ks = 0; ks < S::kKSteps; ++ks) {
-          uint32_t b0, b1, b2, b3;
-          ldsm_x4(kt + swz(row, 2 * ks + (lm & 1)), b0, b1, b2, b3);
-          M::run(sc[0], qa[ks][0], qa[ks][1], qa[ks][2], qa[ks][3], b0, b1);
-          M::run(sc[1], qa[ks][0], qa[ks][1], qa[ks][2], qa[ks][3], b2, b3);
+          uint32_t a0, a1, a2, a3;
+          ldsm_x4(kt + swz(row, 2 * ks + (lm >> 1)), a0, a1, a2, a3);
+#pragma unroll
+          for (int nt = 0; nt < NT; ++nt) M::run(sc[nt], a0, a1, a2, a3, qb[nt][ks][0], qb[nt][ks][1]);
         }
       }
-      // (2) scale, causal mask, online softmax per row
-      float x[2][4];
+      // (2) causal mask per column, online softmax per column
+      const int jA = page_tok + g8, jB = page_tok + g8 + 8;  // this lane's tokens
+      uint32_t pb[NT][4];  // P^T B fragments: hi top, hi bottom, lo top, lo bottom
+      bool moved = false;
+      float al[NT][2];
 #pragma unroll
-      for (int nt = 0; nt < 2; ++nt)
+      for (int nt = 0; nt < NT; ++nt) {
+        const float x0 = jA <= pos[nt][0] ? sc[nt][0] * a.qk_scale : -INFINITY;
+        const float x1 = jA <= pos[nt][1] ? sc[nt][1] * a.qk_scale : -INFINITY;
+        const float x2 = jB <= pos[nt][0] ? sc[nt][2] * a.qk_scale : -INFINITY;
+        const float x3 = jB <= pos[nt][1] ? sc[nt][3] * a.qk_scale : -INFINITY;
+        float mx0 = fmaxf(x0, x2), mx1 = fmaxf(x1, x3);
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const int j = page_tok + nt * 8 + 2 * t4 + (e & 1);
-          x[nt][e] = j <= (e < 2 ? posA : posB) ? sc[nt][e] * a.qk_scale : -INFINITY;
+        for (int msk = 4; msk <= 16; msk <<= 1) {
+          mx0 = fmaxf(mx0, __shfl_xor_sync(kFull, mx0, msk));
+          mx1 = fmaxf(mx1, __shfl_xor_sync(kFull, mx1, msk));
         }
-      float mxA = fmaxf(fmaxf(x[0][0], x[0][1]), fmaxf(x[1][0], x[1][1]));
-      float mxB = fmaxf(fmaxf(x[0][2], x[0][3]), fmaxf(x[1][2], x[1][3]));
-#pragma unroll
-      for (int msk = 1; msk <= 2; msk <<= 1) {
-        mxA = fmaxf(mxA, __shfl_xor_sync(kFull, mxA, msk));
-        mxB = fmaxf(mxB, __shfl_xor_sync(kFull, mxB, msk));
+        const float n0 = fmaxf(mr[nt][0], mx0), n1 = fmaxf(mr[nt][1], mx1);
+        // a column that has seen no key yet keeps max -inf: subtract 0 instead
+        const float u0 = n0 == -INFINITY ? 0.f : n0, u1 = n1 == -INFINITY ? 0.f : n1;
+        al[nt][0] = exp2f(mr[nt][0] - u0);
+        al[nt][1] = exp2f(mr[nt][1] - u1);
+        mr[nt][0] = n0;
+        mr[nt][1] = n1;
+        const float p0 = exp2f(x0 - u0), p1 = exp2f(x1 - u1), p2 = exp2f(x2 - u0), p3 = exp2f(x3 - u1);
+        lr_[nt][0] = fmaf(lr_[nt][0], al[nt][0], p0 + p2);
+        lr_[nt][1] = fmaf(lr_[nt][1], al[nt][1], p1 + p3);
+        moved |= al[nt][0] != 1.f || al[nt][1] != 1.f;
+        const uint32_t top_hi = M::pack(p0, p1), bot_hi = M::pack(p2, p3);
+        const float2 th = M::unpack(top_hi), bh = M::unpack(bot_hi);
+        pb[nt][0] = movm_t(top_hi);
+        pb[nt][1] = movm_t(bot_hi);
+        pb[nt][2] = movm_t(M::pack(p0 - th.x, p1 - th.y));
+        pb[nt][3] = movm_t(M::pack(p2 - bh.x, p3 - bh.y));
       }
-      const float nA = fmaxf(mA, mxA), nB = fmaxf(mB, mxB);
-      // a row that has seen no key yet keeps max -inf: subtract 0 instead
-      const float uA = nA == -INFINITY ? 0.f : nA, uB = nB == -INFINITY ? 0.f : nB;
-      const float alA = exp2f(mA - uA), alB = exp2f(mB - uB);
-      mA = nA;
-      mB = nB;
-      float p[2][4];
+      if (__any_sync(kFull, moved)) {
 #pragma unroll
-      for (int nt = 0; nt < 2; ++nt) {
-        p[nt][0] = exp2f(x[nt][0] - uA);
-        p[nt][1] = exp2f(x[nt][1] - uA);
-        p[nt][2] = exp2f(x[nt][2] - uB);
-        p[nt][3] = exp2f(x[nt][3] - uB);
-      }
-      lA = fmaf(lA, alA, p[0][0] + p[0][1] + p[1][0] + p[1][1]);
-      lB = fmaf(lB, alB, p[0][2] + p[0][3] + p[1][2] + p[1][3]);
-      if (__any_sync(kFull, alA != 1.f || alB != 1.f)) {
+        for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
-        for (int j = 0; j < kNTiles; ++j) {
-          o[j][0] *= alA;
-          o[j][1] *= alA;
-          o[j][2] *= alB;
-          o[j][3] *= alB;
-        }
+          for (int mt = 0; mt < S::kKSteps; ++mt) {
+            o[nt][mt][0] *= al[nt][0];
+            o[nt][mt][1] *= al[nt][1];
+            o[nt][mt][2] *= al[nt][0];
+            o[nt][mt][3] *= al[nt][1];
+          }
       }
-      // (3) P as A fragments, hi + lo 16-bit parts
-      uint32_t ph[4], pl[4];
-      {
-        const float v[4][2] = {{p[0][0], p[0][1]}, {p[0][2], p[0][3]}, {p[1][0], p[1][1]}, {p[1][2], p[1][3]}};
-#pragma unroll
-        for (int r = 0; r < 4; ++r) {
-          ph[r] = M::pack(v[r][0], v[r][1]);
-          const float2 hv = M::unpack(ph[r]);
-          pl[r] = M::pack(v[r][0] - hv.x, v[r][1] - hv.y);
-        }
-      }
-      // V fragment halves of tokens past the visible range are zeroed (an
+      // V^T fragment halves of tokens past the visible range are zeroed (an
       // unwritten slot may hold NaN, and 0 * NaN is NaN)
       uint32_t keep_lo = 0xffffffffu, keep_hi = 0xffffffffu;
       if (nvalid < kBlockSize) {
         keep_lo = (2 * t4 < nvalid ? 0x0000ffffu : 0u) | (2 * t4 + 1 < nvalid ? 0xffff0000u : 0u);
         keep_hi = (2 * t4 + 8 < nvalid ? 0x0000ffffu : 0u) | (2 * t4 + 9 < nvalid ? 0xffff0000u : 0u);
       }
-      // (4) O += P . V
+      // (3) O^T += V^T . P^T, V fragments loaded once for every n-tile
       {
-        const int row = lr + ((lm & 1) << 3);  // token
+        const int row = lr + ((lm >> 1) << 3);
 #pragma unroll
-        for (int j = 0; j < kNTiles; j += 2) {
-          uint32_t b0, b1, b2, b3;
-          ldsm_x4_t(vt + swz(row, j + (lm >> 1)), b0, b1, b2, b3);
-          b0 &= keep_lo;
-          b1 &= keep_hi;
-          b2 &= keep_lo;
-          b3 &= keep_hi;
-          M::run(o[j], ph[0], ph[1], ph[2], ph[3], b0, b1);
-          M::run(o[j], pl[0], pl[1], pl[2], pl[3], b0, b1);
-          M::run(o[j + 1], ph[0], ph[1], ph[2], ph[3], b2, b3);
-          M::run(o[j + 1], pl[0], pl[1], pl[2], pl[3], b2, b3);
+        for (int mt = 0; mt < S::kKSteps; ++mt) {
+          uint32_t a0, a1, a2, a3;
+          ldsm_x4_t(vt + swz(row, 2 * mt + (lm & 1)), a0, a1, a2, a3);
+          a0 &= keep_lo;
+          a1 &= keep_lo;
+          a2 &= keep_hi;
+          a3 &= keep_hi;
+#pragma unroll
+          for (int nt = 0; nt < NT; ++nt) {
+            M::run(o[nt][mt], a0, a1, a2, a3, pb[nt][0], pb[nt][1]);
+            M::run(o[nt][mt], a0, a1, a2, a3, pb[nt][2], pb[nt][3]);
+          }
         }
       }
     }
@@ -317,51 +322,60 @@ __global__ void __launch_bounds__(NWARPS * 32)
       phase_bits ^= 1u << s;
     }
   }
+  // running sums over the lanes of each column (same t4)
 #pragma unroll
-  for (int msk = 1; msk <= 2; msk <<= 1) {
-    lA += __shfl_xor_sync(kFull, lA, msk);
-    lB += __shfl_xor_sync(kFull, lB, msk);
-  }
+  for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+    for (int msk = 4; msk <= 16; msk <<= 1) {
+      lr_[nt][0] += __shfl_xor_sync(kFull, lr_[nt][0], msk);
+      lr_[nt][1] += __shfl_xor_sync(kFull, lr_[nt][1], msk);
+    }
 
-  // warp record [o: 16 x D][m: 16][l: 16] in the warp's own (drained) stages
+  // warp record [o: kCols x D][m: kCols][l: kCols] in the warp's own stages
   float* rec = reinterpret_cast<float*>(my_stages);
 #pragma unroll
-  for (int j = 0; j < kNTiles; ++j) {
-    const int d = 8 * j + 2 * t4;
-    *reinterpret_cast<float2*>(rec + g8 * D + d) = make_float2(o[j][0], o[j][1]);
-    *reinterpret_cast<float2*>(rec + (g8 + 8) * D + d) = make_float2(o[j][2], o[j][3]);
-  }
-  if (t4 == 0) {
-    rec[kRec + g8] = mA;
-    rec[kRec + g8 + 8] = mB;
-    rec[kRec + 16 + g8] = lA;
-    rec[kRec + 16 + g8 + 8] = lB;
+  for (int nt = 0; nt < NT; ++nt) {
+    const int ca = 8 * nt + 2 * t4, cb = ca + 1;
+#pragma unroll
+    for (int mt = 0; mt < S::kKSteps; ++mt) {
+      const int d0 = 16 * mt + g8;
+      rec[ca * D + d0] = o[nt][mt][0];
+      rec[ca * D + d0 + 8] = o[nt][mt][2];
+      rec[cb * D + d0] = o[nt][mt][1];
+      rec[cb * D + d0 + 8] = o[nt][mt][3];
+    }
+    if (g8 == 0) {
+      rec[kRecM + ca] = mr[nt][0];
+      rec[kRecL + ca] = lr_[nt][0];
+      rec[kRecM + cb] = mr[nt][1];
+      rec[kRecL + cb] = lr_[nt][1];
+    }
   }
   if (__syncthreads_or(timed_out)) return;
 
   // merge the warps in a fixed order; rows with no key in this partition
   // are left to the other partitions (the merge never reads them)
-  for (int idx = threadIdx.x; idx < 16 * D; idx += NWARPS * 32) {
-    const int r = idx / D, d = idx % D;
-    const int tr = r0 + r;
+  for (int idx = threadIdx.x; idx < kCols * D; idx += NWARPS * 32) {
+    const int c = idx / D, d = idx % D;
+    const int tr = r0 + c;
     if (tr >= R) continue;
-    const int pos = base + tr / G;
+    const int p = base + tr / G;
     const size_t row = out_row(tr);
-    if (pos < tok0) {
+    if (p < tok0) {
       if (direct) reinterpret_cast<T*>(a.out)[row * D + d] = Fmt<T>::from_f32(0.f);
       continue;
     }
     float Mx = -INFINITY;
 #pragma unroll
     for (int w = 0; w < NWARPS; ++w)
-      Mx = fmaxf(Mx, reinterpret_cast<const float*>(smem + w * S::kWarpStageBytes)[kRec + r]);
+      Mx = fmaxf(Mx, reinterpret_cast<const float*>(smem + w * S::kWarpStageBytes)[kRecM + c]);
     float num = 0.f, den = 0.f;
 #pragma unroll
     for (int w = 0; w < NWARPS; ++w) {
       const float* rw = reinterpret_cast<const float*>(smem + w * S::kWarpStageBytes);
-      const float sc = exp2f(rw[kRec + r] - Mx);
-      num = fmaf(sc, rw[r * D + d], num);
-      den = fmaf(sc, rw[kRec + 16 + r], den);
+      const float sc = exp2f(rw[kRecM + c] - Mx);
+      num = fmaf(sc, rw[c * D + d], num);
+      den = fmaf(sc, rw[kRecL + c], den);
     }
     if (direct) {
       reinterpret_cast<T*>(a.out)[row * D + d] = Fmt<T>::from_f32(num / den);

@@ -9,6 +9,7 @@
 #include <cudaTypedefs.h>
 
 #include "cache_ops.cuh"
+#include "decode_fp8.cuh"
 #include "decode_launch.cuh"
 #include "multi_mma.cuh"
 #include "pkv.h"
@@ -27,7 +28,7 @@ struct MultiMergeK {
   static constexpr auto fn = pkv::paged_multi_merge_kernel<T, D, HPC>;
 };
 
-template <typename T, int D, int G>
+template <typename T, int D, int G, int NT>
 pkv_status launch_multi(const pkv::MultiArgs& a, const void* k_cache, const void* v_cache, int num_blocks,
                         cudaStream_t st) {
   constexpr int kStages = kMmaStages;
@@ -37,7 +38,7 @@ pkv_status launch_multi(const pkv::MultiArgs& a, const void* k_cache, const void
   if (!encode_cache_map(&mk, k_cache, pkv::Mma<T>::kTmaType, D, rows) ||
       !encode_cache_map(&mv, v_cache, pkv::Mma<T>::kTmaType, D, rows))
     return PKV_ECUDA;
-  auto kfn = pkv::paged_multi_mma_kernel<T, D, G, kMmaWarps, kStages>;
+  auto kfn = pkv::paged_multi_mma_kernel<T, D, G, NT, kMmaWarps, kStages>;
   if (cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(S::kSmem)) !=
       cudaSuccess)
     return PKV_ECUDA;
@@ -55,14 +56,75 @@ pkv_status launch_multi(const pkv::MultiArgs& a, const void* k_cache, const void
   return PKV_OK;
 }
 
+// Rows per tile (8 NT) for the rows a sequence brings (max_query_len * G):
+// one tile up to 24 rows, else tiles of 24.
+int multi_ntiles(long long rows) { return rows <= 8 ? 1 : rows <= 16 ? 2 : 3; }
+
+template <typename T, int D, int G>
+pkv_status dispatch_nt_multi(const pkv::MultiArgs& a, int NT, const void* k, const void* v, int nb,
+                             cudaStream_t st) {
+  switch (NT) {
+    case 1: return launch_multi<T, D, G, 1>(a, k, v, nb, st);
+    case 2: return launch_multi<T, D, G, 2>(a, k, v, nb, st);
+    case 3: return launch_multi<T, D, G, 3>(a, k, v, nb, st);
+  }
+  return PKV_EINVAL;
+}
+
 template <typename T, int D>
-pkv_status dispatch_group_multi(const pkv::MultiArgs& a, int G, const void* k, const void* v, int nb,
+pkv_status dispatch_group_multi(const pkv::MultiArgs& a, int G, int NT, const void* k, const void* v, int nb,
                                 cudaStream_t st) {
   switch (G) {
-    case 1: return launch_multi<T, D, 1>(a, k, v, nb, st);
-    case 2: return launch_multi<T, D, 2>(a, k, v, nb, st);
-    case 4: return launch_multi<T, D, 4>(a, k, v, nb, st);
-    case 8: return launch_multi<T, D, 8>(a, k, v, nb, st);
+    case 1: return dispatch_nt_multi<T, D, 1>(a, NT, k, v, nb, st);
+    case 2: return dispatch_nt_multi<T, D, 2>(a, NT, k, v, nb, st);
+    case 4: return dispatch_nt_multi<T, D, 4>(a, NT, k, v, nb, st);
+    case 8: return dispatch_nt_multi<T, D, 8>(a, NT, k, v, nb, st);
+  }
+  return PKV_EINVAL;
+}
+
+// ---- FP8 (E4M3) cache ---------------------------------------------------------
+// The pool viewed as [num_blocks * Hkv * 16 rows, D bytes], one box per tile
+// row span with the swizzle of that span (128 or 64 bytes).
+bool encode_fp8_map(CUtensorMap* map, const void* base, int D, long long rows) {
+  PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
+  if (enc == nullptr) return false;
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(rows)};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(D)};
+  const cuuint32_t box[2] = {static_cast<cuuint32_t>(D), 16};
+  const cuuint32_t elem_strides[2] = {1, 1};
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, elem_strides,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, D == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+constexpr int kFp8Stages = 4;  // pages in flight per warp (4 KB each at D = 128)
+
+template <typename T, int D, int G>
+pkv_status launch_decode_fp8(const pkv::DecodeArgs& a, float v_scale, cudaStream_t st) {
+  using S = pkv::Fp8Shape<D, kMmaWarps, kFp8Stages>;
+  CUtensorMap mk, mv;
+  const long long rows = static_cast<long long>(a.num_blocks) * a.num_kv_heads * PKV_BLOCK_SIZE;
+  if (!encode_fp8_map(&mk, a.k_cache, D, rows) || !encode_fp8_map(&mv, a.v_cache, D, rows)) return PKV_ECUDA;
+  auto kfn = pkv::paged_decode_fp8_kernel<T, D, G, kMmaWarps, kFp8Stages>;
+  if (cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(S::kSmem)) !=
+      cudaSuccess)
+    return PKV_ECUDA;
+  const dim3 grid(a.num_kv_heads, a.num_seqs, a.num_parts);
+  if (launch(kfn, grid, dim3(kMmaWarps * 32), S::kSmem, st, a, mk, mv, v_scale) != PKV_OK) return PKV_ECUDA;
+  if (a.num_parts > 1) {
+    if (launch_merge<T, D, ReduceK>(a, a.num_parts, st) != PKV_OK) return PKV_ECUDA;
+  }
+  return PKV_OK;
+}
+
+template <typename T, int D>
+pkv_status dispatch_group_fp8(const pkv::DecodeArgs& a, int G, float v_scale, cudaStream_t st) {
+  switch (G) {
+    case 1: return launch_decode_fp8<T, D, 1>(a, v_scale, st);
+    case 2: return launch_decode_fp8<T, D, 2>(a, v_scale, st);
+    case 4: return launch_decode_fp8<T, D, 4>(a, v_scale, st);
+    case 8: return launch_decode_fp8<T, D, 8>(a, v_scale, st);
   }
   return PKV_EINVAL;
 }
@@ -398,7 +460,8 @@ pkv_status pkv_paged_attention_multi(void* out, const void* q, const void* k_cac
   if (!aligned16(out) || !aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache)) return PKV_EINVAL;
   if (static_cast<long long>(num_blocks) * num_kv_heads * PKV_BLOCK_SIZE > 0x7fffffffLL) return PKV_EINVAL;
   const int G = num_q_heads / num_kv_heads;
-  const long long tiles = (static_cast<long long>(max_query_len) * G + 15) / 16;
+  const int NT = multi_ntiles(static_cast<long long>(max_query_len) * G);
+  const long long tiles = (static_cast<long long>(max_query_len) * G + 8 * NT - 1) / (8 * NT);
   const long long P = (static_cast<long long>(max_context_len) + part - 1) / part;
   if (tiles * num_seqs > 65535 || P > 65535) return PKV_EINVAL;
   const size_t need = multi_workspace_bytes(total_query_tokens, num_q_heads, head_dim, P);
@@ -430,10 +493,70 @@ pkv_status pkv_paged_attention_multi(void* out, const void* q, const void* k_cac
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   auto run = [&](auto tag) -> pkv_status {
     using T = decltype(tag);
-    if (head_dim == 64) return dispatch_group_multi<T, 64>(a, G, k_cache, v_cache, num_blocks, st);
-    return dispatch_group_multi<T, 128>(a, G, k_cache, v_cache, num_blocks, st);
+    if (head_dim == 64) return dispatch_group_multi<T, 64>(a, G, NT, k_cache, v_cache, num_blocks, st);
+    return dispatch_group_multi<T, 128>(a, G, NT, k_cache, v_cache, num_blocks, st);
   };
   if (dtype == PKV_F16) return run(__half{});
+  return run(__nv_bfloat16{});
+}
+
+pkv_status pkv_kv_append_fp8(const void* k_new, const void* v_new, void* k_cache, void* v_cache,
+                             const int64_t* slot_mapping, int num_tokens, int num_kv_heads, int head_dim,
+                             int num_blocks, pkv_dtype src_dtype, float k_scale, float v_scale, void* stream) {
+  if ((src_dtype != PKV_F16 && src_dtype != PKV_BF16) || num_tokens < 0 || num_kv_heads <= 0 ||
+      !head_dim_ok(head_dim) || num_blocks <= 0 || !std::isfinite(k_scale) || !std::isfinite(v_scale) ||
+      !(k_scale > 0.f) || !(v_scale > 0.f))
+    return PKV_EINVAL;
+  if (num_tokens == 0) return PKV_OK;
+  if (!k_new || !v_new || !k_cache || !v_cache || !slot_mapping || !aligned16(k_new) || !aligned16(v_new) ||
+      !aligned16(k_cache) || !aligned16(v_cache))
+    return PKV_EINVAL;
+  const int row_chunks = head_dim / 8;  // 8 elements: 16 bytes in, 8 bytes out
+  const long long total = static_cast<long long>(num_tokens) * num_kv_heads * row_chunks;
+  long long blocks = (2 * total + 255) / 256;
+  if (blocks > 148LL * 16) blocks = 148LL * 16;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  auto run = [&](auto kernel) {
+    return launch(kernel, dim3(static_cast<unsigned>(blocks)), dim3(256), 0, st, static_cast<const uint4*>(k_new),
+                  static_cast<const uint4*>(v_new), static_cast<uint2*>(k_cache), static_cast<uint2*>(v_cache),
+                  slot_mapping, total, num_kv_heads, row_chunks, num_blocks, k_scale, v_scale);
+  };
+  if (src_dtype == PKV_F16) return run(pkv::kv_append_fp8_kernel<__half>);
+  return run(pkv::kv_append_fp8_kernel<__nv_bfloat16>);
+}
+
+pkv_status pkv_paged_attention_decode_fp8(void* out, const void* q, const void* k_cache, const void* v_cache,
+                                          const int32_t* block_tables, int max_blocks_per_seq,
+                                          const int32_t* context_lens, int max_context_len, int num_seqs,
+                                          int num_q_heads, int num_kv_heads, int head_dim, int num_blocks,
+                                          float scale, float k_scale, float v_scale, int partition_tokens,
+                                          pkv_dtype q_dtype, void* workspace, size_t workspace_bytes_given,
+                                          void* stream) {
+  if (q_dtype != PKV_F16 && q_dtype != PKV_BF16) return PKV_EINVAL;
+  if (!std::isfinite(k_scale) || !std::isfinite(v_scale) || !(k_scale > 0.f) || !(v_scale > 0.f))
+    return PKV_EINVAL;
+  pkv::DecodeArgs a{};
+  long long P = 0;
+  const pkv_status st0 = prepare_decode(out, q, k_cache, v_cache, block_tables, max_blocks_per_seq, context_lens,
+                                        max_context_len, num_seqs, num_q_heads, num_kv_heads, head_dim, num_blocks,
+                                        scale, partition_tokens, q_dtype, &a, &P);
+  if (st0 != PKV_OK || num_seqs == 0) return st0;
+  const size_t need = workspace_bytes(num_seqs, num_q_heads, head_dim, P);
+  if (need > 0 && (workspace == nullptr || workspace_bytes_given < need || !aligned16(workspace)))
+    return PKV_EINVAL;
+  a.ws_o = static_cast<float*>(need ? workspace : nullptr);
+  a.ws_ml = need ? reinterpret_cast<float2*>(static_cast<float*>(workspace) +
+                                              static_cast<size_t>(num_seqs) * num_q_heads * P * head_dim)
+                 : nullptr;
+  a.qk_scale *= k_scale;
+  const int G = num_q_heads / num_kv_heads;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  auto run = [&](auto tag) -> pkv_status {
+    using T = decltype(tag);
+    if (head_dim == 64) return dispatch_group_fp8<T, 64>(a, G, v_scale, st);
+    return dispatch_group_fp8<T, 128>(a, G, v_scale, st);
+  };
+  if (q_dtype == PKV_F16) return run(__half{});
   return run(__nv_bfloat16{});
 }
 

@@ -168,3 +168,22 @@ def test_multi_workspace_and_rejections(lib):
     a = list(args)
     a[10] = 0
     assert lib.pkv_paged_attention_multi(*a) == 0
+
+
+def test_fp8_rejections(lib):
+    f = ctypes.c_float
+    ok = [FAKE, FAKE, FAKE, FAKE, FAKE, 4, 2, 64, 16, 1, f(0.1), f(0.1), None]
+    for idx, bad in ((9, 0), (9, 3), (7, 96), (10, f(0.0)), (11, f(-1.0)), (10, f(float("nan"))), (4, None),
+                     (2, ODD)):
+        a = list(ok)
+        a[idx] = bad
+        assert lib.pkv_kv_append_fp8(*a) == 1, (idx, bad)
+    a = list(ok)
+    a[5] = 0
+    assert lib.pkv_kv_append_fp8(*a) == 0
+    dec = [FAKE, FAKE, FAKE, FAKE, FAKE, 8, FAKE, 100, 2, 8, 2, 128, 64, f(0.1), f(0.1), f(0.1), 0, 1, FAKE,
+           1 << 30, None]
+    for idx, bad in ((17, 0), (17, 3), (14, f(0.0)), (15, f(float("inf"))), (11, 96), (9, 6)):
+        a = list(dec)
+        a[idx] = bad
+        assert lib.pkv_paged_attention_decode_fp8(*a) == 1, (idx, bad)
