@@ -54,8 +54,8 @@ def build(ctx, Hkv, D, dt, ks, vs, seed):
         slots += [int(tables[b, j // 16]) * 16 + j % 16 for j in range(c)]
     slots = np.array(slots, dtype=np.int64)
     n = len(slots)
-    kx = storage(rng.standard_normal((n, Hkv, D)).astype(np.float32) * 2, dt)
-    vx = storage(rng.standard_normal((n, Hkv, D)).astype(np.float32) * 2, dt)
+    kx = storage(rng.standard_normal((n, Hkv, D)).astype(np.float32), dt)
+    vx = storage(rng.standard_normal((n, Hkv, D)).astype(np.float32), dt)
     ref = oracle.RefCache(nb, Hkv, D, "e4m3")
     ref.append_fp8(kx, vx, slots, dt, ks, vs)
     kc = torch.full((nb, Hkv, 16, D), 0x7F, dtype=torch.uint8, device="cuda")
