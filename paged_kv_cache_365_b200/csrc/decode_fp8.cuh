@@ -24,14 +24,20 @@
 //    so one MMA per n-tile accumulates both (their sum is the result).
 //  * The K scale is folded into the logit scale, the V scale into the
 //    output.
+//  * The MMAs run in fp16 whatever the query dtype: E4M3 -> fp16 is one
+//    instruction per pair.  bf16 queries are brought into fp16 exactly by
+//    a power-of-two factor per query row (its largest magnitude lands in
+//    [2^14, 2^15)), undone on that row's logits.
 #pragma once
+
+#include <type_traits>
 
 #include "decode_mma.cuh"
 
 namespace pkv {
 
-// E4M3 pair (low byte -> low half) to two 16-bit floats of type T (exact:
-// every E4M3 value is an fp16 and a bf16 value).
+// E4M3 pair (low byte -> low half) to two fp16 values (exact: every E4M3
+// value is an fp16 value).
 template <typename T>
 __device__ __forceinline__ uint32_t e4m3x2_to(uint32_t pair16);
 
@@ -43,13 +49,6 @@ __device__ __forceinline__ uint32_t e4m3x2_to<__half>(uint32_t pair16) {
   return d;
 }
 
-template <>
-__device__ __forceinline__ uint32_t e4m3x2_to<__nv_bfloat16>(uint32_t pair16) {
-  const uint32_t h = e4m3x2_to<__half>(pair16);
-  const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&h));
-  const __nv_bfloat162 b = __floats2bfloat162_rn(f.x, f.y);  // exact
-  return *reinterpret_cast<const uint32_t*>(&b);
-}
 
 // Byte offset of 16-byte chunk `chunk` of row `row` in an FP8 tile of 16
 // rows x D bytes stored with the TMA swizzle matching its row length
@@ -84,7 +83,7 @@ __global__ void __launch_bounds__(NWARPS * 32)
                             const __grid_constant__ CUtensorMap tmap_v, float v_scale) {
   pdl_enter();
   using S = Fp8Shape<D, NWARPS, NSTAGE>;
-  using M = Mma<T>;
+  using M = Mma<__half>;      // the MMAs run in fp16 (see above)
   constexpr int kNT = D / 8;  // PV n-tiles; also the d values a column spans
   const int kvh = blockIdx.x;
   const int b = blockIdx.y;
@@ -120,18 +119,50 @@ __global__ void __launch_bounds__(NWARPS * 32)
   }
   __syncwarp();
 
-  // Q^T as B fragments in the d order the converted K fragments use:
-  // chunk c: b0 = q[16c + 4t .. +1], b1 = q[16c + 4t + 2 .. +3]
+  // Q^T as fp16 B fragments in the d order the converted K fragments use:
+  // chunk c: b0 = q[16c + 4t .. +1], b1 = q[16c + 4t + 2 .. +3].  A bf16
+  // row is first scaled by 2^kq (exact) so that it fits fp16.
   uint32_t qb[S::kChunks][2];
+  int kq = 0;  // this lane's row (query g8): q was multiplied by 2^kq
   {
     const bool ok = g8 < G;
     const T* qp = reinterpret_cast<const T*>(a.q) + (ok ? col_row(g8) : 0) * D;
+    float qf[S::kChunks][4];
 #pragma unroll
     for (int c = 0; c < S::kChunks; ++c) {
-      qb[c][0] = ok ? *reinterpret_cast<const uint32_t*>(qp + 16 * c + 4 * t4) : 0u;
-      qb[c][1] = ok ? *reinterpret_cast<const uint32_t*>(qp + 16 * c + 4 * t4 + 2) : 0u;
+      const float2 lo = ok ? Mma<T>::unpack(*reinterpret_cast<const uint32_t*>(qp + 16 * c + 4 * t4))
+                           : make_float2(0.f, 0.f);
+      const float2 hi = ok ? Mma<T>::unpack(*reinterpret_cast<const uint32_t*>(qp + 16 * c + 4 * t4 + 2))
+                           : make_float2(0.f, 0.f);
+      qf[c][0] = lo.x;
+      qf[c][1] = lo.y;
+      qf[c][2] = hi.x;
+      qf[c][3] = hi.y;
+    }
+    float sc = 1.f;
+    if constexpr (!std::is_same<T, __half>::value) {
+      float mx = 0.f;
+#pragma unroll
+      for (int c = 0; c < S::kChunks; ++c)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) mx = fmaxf(mx, fabsf(qf[c][e]));
+      mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 1));
+      mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 2));
+      const int ex = static_cast<int>((__float_as_uint(mx) >> 23) & 0xffu) - 127;  // floor(log2 mx) (normal mx)
+      kq = mx > 0.f ? min(max(14 - ex, -126), 126) : 0;
+      sc = __uint_as_float(static_cast<uint32_t>(kq + 127) << 23);  // 2^kq
+    }
+#pragma unroll
+    for (int c = 0; c < S::kChunks; ++c) {
+      qb[c][0] = M::pack(qf[c][0] * sc, qf[c][1] * sc);
+      qb[c][1] = M::pack(qf[c][2] * sc, qf[c][3] * sc);
     }
   }
+  // logit scale of this lane's S^T columns 2 t4, 2 t4 + 1 (query rows
+  // 2 t4, 2 t4 + 1 held their factor 2^kq in lanes 8 t4, 8 t4 + 4)
+  const int kq0 = __shfl_sync(kFull, kq, 8 * t4), kq1 = __shfl_sync(kFull, kq, 8 * t4 + 4);
+  const float xs0 = a.qk_scale * __uint_as_float(static_cast<uint32_t>(127 - kq0) << 23);
+  const float xs1 = a.qk_scale * __uint_as_float(static_cast<uint32_t>(127 - kq1) << 23);
 
   const int tok0 = part * a.partition;
   const int tok1 = min(ctx, tok0 + a.partition);
@@ -213,18 +244,18 @@ __global__ void __launch_bounds__(NWARPS * 32)
         for (int c = 0; c < S::kChunks; c += 2) {
           uint32_t r0, r1, r2, r3;
           ldsm_x4(kt + swz8<D>(row, c + (lm >> 1)), r0, r1, r2, r3);
-          M::run(sc, e4m3x2_to<T>(r0 & 0xffffu), e4m3x2_to<T>(r1 & 0xffffu), e4m3x2_to<T>(r0 >> 16),
-                 e4m3x2_to<T>(r1 >> 16), qb[c][0], qb[c][1]);
-          M::run(sc, e4m3x2_to<T>(r2 & 0xffffu), e4m3x2_to<T>(r3 & 0xffffu), e4m3x2_to<T>(r2 >> 16),
-                 e4m3x2_to<T>(r3 >> 16), qb[c + 1][0], qb[c + 1][1]);
+          M::run(sc, e4m3x2_to<__half>(r0 & 0xffffu), e4m3x2_to<__half>(r1 & 0xffffu),
+                 e4m3x2_to<__half>(r0 >> 16), e4m3x2_to<__half>(r1 >> 16), qb[c][0], qb[c][1]);
+          M::run(sc, e4m3x2_to<__half>(r2 & 0xffffu), e4m3x2_to<__half>(r3 & 0xffffu),
+                 e4m3x2_to<__half>(r2 >> 16), e4m3x2_to<__half>(r3 >> 16), qb[c + 1][0], qb[c + 1][1]);
         }
       }
       // (2) scale (K scale folded in), mask the tail, online softmax
       const bool v_lo = g8 < nvalid, v_hi = g8 + 8 < nvalid;
-      const float x0 = v_lo ? sc[0] * a.qk_scale : -INFINITY;
-      const float x1 = v_lo ? sc[1] * a.qk_scale : -INFINITY;
-      const float x2 = v_hi ? sc[2] * a.qk_scale : -INFINITY;
-      const float x3 = v_hi ? sc[3] * a.qk_scale : -INFINITY;
+      const float x0 = v_lo ? sc[0] * xs0 : -INFINITY;
+      const float x1 = v_lo ? sc[1] * xs1 : -INFINITY;
+      const float x2 = v_hi ? sc[2] * xs0 : -INFINITY;
+      const float x3 = v_hi ? sc[3] * xs1 : -INFINITY;
       float mx0 = fmaxf(x0, x2), mx1 = fmaxf(x1, x3);
 #pragma unroll
       for (int msk = 4; msk <= 16; msk <<= 1) {
@@ -291,8 +322,8 @@ __global__ void __launch_bounds__(NWARPS * 32)
         const uint32_t sel = bsel | ((4 + bsel) << 4) | ((bsel + 1) << 8) | ((5 + bsel) << 12);
         const uint32_t lo01 = __byte_perm(w0[w], w1[w], sel);
         const uint32_t lo89 = __byte_perm(w8[w], w9[w], sel);
-        const uint32_t b0j = e4m3x2_to<T>(lo01 & 0xffffu), b0k = e4m3x2_to<T>(lo01 >> 16);
-        const uint32_t b1j = e4m3x2_to<T>(lo89 & 0xffffu), b1k = e4m3x2_to<T>(lo89 >> 16);
+        const uint32_t b0j = e4m3x2_to<__half>(lo01 & 0xffffu), b0k = e4m3x2_to<__half>(lo01 >> 16);
+        const uint32_t b1j = e4m3x2_to<__half>(lo89 & 0xffffu), b1k = e4m3x2_to<__half>(lo89 >> 16);
         M::run(o[j], pa0, pa1, pa2, pa3, b0j, b1j);
         M::run(o[j + 1], pa0, pa1, pa2, pa3, b0k, b1k);
       }
