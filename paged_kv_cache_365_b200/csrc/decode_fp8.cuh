@@ -77,8 +77,13 @@ struct Fp8Shape {
   static_assert(kTile % 512 == 0, "swizzled tiles want 512/1024-byte alignment");
 };
 
+// CTAs per SM the FP8 kernel's register budget is sized for
+#ifndef PKV_FP8_MIN_CTAS
+#define PKV_FP8_MIN_CTAS 1
+#endif
+
 template <typename T, int D, int G, int NWARPS, int NSTAGE>
-__global__ void __launch_bounds__(NWARPS * 32)
+__global__ void __launch_bounds__(NWARPS * 32, PKV_FP8_MIN_CTAS)
     paged_decode_fp8_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tmap_k,
                             const __grid_constant__ CUtensorMap tmap_v, float v_scale) {
   pdl_enter();

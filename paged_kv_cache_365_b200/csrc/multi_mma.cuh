@@ -387,6 +387,282 @@ __global__ void __launch_bounds__(NWARPS * 32)
   }
 }
 
+// Many rows per sequence (more than two n-tiles' worth): the warps of a CTA
+// split the rows instead of the pages.  Warp w owns the 8 rows r0 + 8 w ..
+// r0 + 8 w + 7 (one n-tile, so registers stay as in decode) and every warp
+// consumes every page of the partition from one CTA-wide ring of NSTAGE
+// staged tiles: thread 0 issues the TMA copies, all warps wait on a stage's
+// mbarrier, and a CTA barrier after each page frees its stage for the page
+// NSTAGE ahead.  A page is read once per CTA for all its 8 NW rows; the
+// warps' rows are disjoint, so each writes its own outputs.
+template <int D, int NW, int NSTAGE>
+struct RowsShape {
+  static constexpr int kTile = kBlockSize * D * 2;
+  static constexpr int kStage = 2 * kTile;
+  static constexpr int kKSteps = D / 16;
+  static constexpr int kBoxes = D / 64;
+  static constexpr size_t kSmem = 1024 + size_t(NSTAGE) * kStage + size_t(NSTAGE) * 8;
+  static constexpr int kTab = 4;  // table entries a lane holds: 128 pages of a 2048-token partition
+  static_assert(kStage % 1024 == 0, "swizzled boxes need 1024-byte alignment");
+};
+
+template <typename T, int D, int G, int NW, int NSTAGE>
+__global__ void __launch_bounds__(NW * 32)
+    paged_multi_rows_kernel(const MultiArgs a, const __grid_constant__ CUtensorMap tmap_k,
+                            const __grid_constant__ CUtensorMap tmap_v) {
+  pdl_enter();
+  using S = RowsShape<D, NW, NSTAGE>;
+  using M = Mma<T>;
+  constexpr int kCols = 8 * NW;
+  const int kvh = blockIdx.x;
+  const int b = blockIdx.y / a.tiles;
+  const int tile = blockIdx.y % a.tiles;
+  const int z = blockIdx.z;
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int g8 = lane >> 2, t4 = lane & 3, lm = lane >> 3, lr = lane & 7;
+
+  int ctx, q0, nq;
+  if (!multi_seq(a, b, ctx, q0, nq, threadIdx.x == 0 && kvh == 0 && tile == 0 && z == 0)) return;
+  const int R = nq * G;
+  const int r0 = tile * kCols;
+  if (r0 >= R) return;
+  const int base = ctx - nq;
+  const int p_hi = base + (min(R, r0 + kCols) - 1) / G;
+  const bool direct = ctx <= a.partition;
+  const int tok0 = z * a.partition;
+  const int tok1 = min(min(ctx, tok0 + a.partition), p_hi + 1);
+  auto out_row = [&](int tr) -> size_t {
+    return static_cast<size_t>(q0 + tr / G) * a.num_q_heads + kvh * G + tr % G;
+  };
+  if (tok1 <= tok0) {
+    if (direct && z == 0)
+      for (int idx = threadIdx.x; idx < kCols * D; idx += NW * 32) {
+        const int tr = r0 + idx / D;
+        if (tr < R) reinterpret_cast<T*>(a.out)[out_row(tr) * D + idx % D] = Fmt<T>::from_f32(0.f);
+      }
+    return;
+  }
+
+  extern __shared__ unsigned char smem_raw[];
+  const uint32_t raw_addr = smem_addr(smem_raw);
+  const uint32_t pad = ((raw_addr + 1023u) & ~1023u) - raw_addr;
+  unsigned char* smem = smem_raw + pad;
+  const uint32_t stage0 = smem_addr(smem);
+  const uint32_t bar0 = smem_addr(smem + size_t(NSTAGE) * S::kStage);
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < NSTAGE; ++s) mbar_init(bar0 + 8 * s, 1);
+    fence_barrier_init();
+  }
+  __syncthreads();
+
+  const int pg0 = tok0 / kBlockSize;
+  const int nblk = (tok1 - tok0 + kBlockSize - 1) / kBlockSize;  // <= 128 = 32 * S::kTab
+  int my_phys[S::kTab];
+#pragma unroll
+  for (int h = 0; h < S::kTab; ++h) {
+    my_phys[h] = -1;
+    const int j = lane + 32 * h;
+    if (j < nblk) {
+      const int e = a.block_tables[static_cast<long long>(b) * a.bt_stride + pg0 + j];
+      if (e >= 0 && e < a.num_blocks)
+        my_phys[h] = e;
+      else if (warp == 0)
+        raise_error(PKV_ERR_BLOCK_RANGE);
+    }
+  }
+  auto phys_of = [&](int i) {
+    int r = -1;
+#pragma unroll
+    for (int h = 0; h < S::kTab; ++h) {
+      const int v = __shfl_sync(kFull, my_phys[h], i & 31);
+      if ((i >> 5) == h) r = v;
+    }
+    return r;
+  };
+  auto issue = [&](int i) {  // warp 0 only (its lanes take part in the shuffle)
+    const int phys = phys_of(i);
+    if (lane == 0 && i < nblk) {
+      const uint32_t bar = bar0 + 8 * (i % NSTAGE);
+      if (phys >= 0) {
+        const uint32_t dst = stage0 + (i % NSTAGE) * S::kStage;
+        const int y = (phys * a.num_kv_heads + kvh) * kBlockSize;
+        fence_proxy_async_smem();
+        mbar_arrive_expect_tx(bar, S::kStage);
+#pragma unroll
+        for (int bx = 0; bx < S::kBoxes; ++bx) {
+          tma_load_2d(dst + bx * 2048, &tmap_k, bx * 64, y, bar);
+          tma_load_2d(dst + S::kTile + bx * 2048, &tmap_v, bx * 64, y, bar);
+        }
+      } else {
+        mbar_arrive(bar);
+      }
+    }
+  };
+  if (warp == 0) {
+#pragma unroll
+    for (int i = 0; i < NSTAGE; ++i) issue(i);
+  }
+
+  // this warp's column g8 (row r0 + 8 warp + g8) and its lane's columns 2 t4, 2 t4 + 1
+  uint32_t qb[S::kKSteps][2];
+  int pos0, pos1;
+  {
+    const int tr = r0 + 8 * warp + g8;
+    const bool ok = tr < R;
+    const T* qp = reinterpret_cast<const T*>(a.q) + (ok ? out_row(tr) : 0) * D;
+#pragma unroll
+    for (int ks = 0; ks < S::kKSteps; ++ks) {
+      qb[ks][0] = ok ? *reinterpret_cast<const uint32_t*>(qp + ks * 16 + 2 * t4) : 0u;
+      qb[ks][1] = ok ? *reinterpret_cast<const uint32_t*>(qp + ks * 16 + 8 + 2 * t4) : 0u;
+    }
+    const int c0 = r0 + 8 * warp + 2 * t4;
+    pos0 = c0 < R ? base + c0 / G : -1;
+    pos1 = c0 + 1 < R ? base + (c0 + 1) / G : -1;
+  }
+  float o[S::kKSteps][4];
+#pragma unroll
+  for (int mt = 0; mt < S::kKSteps; ++mt) o[mt][0] = o[mt][1] = o[mt][2] = o[mt][3] = 0.f;
+  float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
+  uint32_t phase_bits = 0;
+  int consumed = 0;
+  bool bad = false;
+
+  for (int i = 0; i < nblk; ++i) {
+    const int s = i % NSTAGE;
+    const bool ok = __all_sync(kFull, mbar_wait_bounded(bar0 + 8 * s, (phase_bits >> s) & 1u));
+    phase_bits ^= 1u << s;
+    if (!ok) {
+      if (lane == 0) raise_error(PKV_ERR_TIMEOUT);
+      bad = true;
+    }
+    if (!bad && phys_of(i) >= 0) {
+      const int page_tok = tok0 + i * kBlockSize;
+      const int nvalid = min(kBlockSize, tok1 - page_tok);
+      const uint32_t kt = stage0 + s * S::kStage;
+      const uint32_t vt = kt + S::kTile;
+      float sc[4] = {0.f, 0.f, 0.f, 0.f};
+      {
+        const int row = lr + ((lm & 1) << 3);
+#pragma unroll
+        for (int ks = 0; ks < S::kKSteps; ++ks) {
+          uint32_t a0, a1, a2, a3;
+          ldsm_x4(kt + swz(row, 2 * ks + (lm >> 1)), a0, a1, a2, a3);
+          M::run(sc, a0, a1, a2, a3, qb[ks][0], qb[ks][1]);
+        }
+      }
+      const int jA = page_tok + g8, jB = page_tok + g8 + 8;
+      const float x0 = jA <= pos0 ? sc[0] * a.qk_scale : -INFINITY;
+      const float x1 = jA <= pos1 ? sc[1] * a.qk_scale : -INFINITY;
+      const float x2 = jB <= pos0 ? sc[2] * a.qk_scale : -INFINITY;
+      const float x3 = jB <= pos1 ? sc[3] * a.qk_scale : -INFINITY;
+      float mx0 = fmaxf(x0, x2), mx1 = fmaxf(x1, x3);
+#pragma unroll
+      for (int msk = 4; msk <= 16; msk <<= 1) {
+        mx0 = fmaxf(mx0, __shfl_xor_sync(kFull, mx0, msk));
+        mx1 = fmaxf(mx1, __shfl_xor_sync(kFull, mx1, msk));
+      }
+      const float n0 = fmaxf(m0, mx0), n1 = fmaxf(m1, mx1);
+      const float u0 = n0 == -INFINITY ? 0.f : n0, u1 = n1 == -INFINITY ? 0.f : n1;
+      const float al0 = exp2f(m0 - u0), al1 = exp2f(m1 - u1);
+      m0 = n0;
+      m1 = n1;
+      const float p0 = exp2f(x0 - u0), p1 = exp2f(x1 - u1), p2 = exp2f(x2 - u0), p3 = exp2f(x3 - u1);
+      l0 = fmaf(l0, al0, p0 + p2);
+      l1 = fmaf(l1, al1, p1 + p3);
+      if (__any_sync(kFull, al0 != 1.f || al1 != 1.f)) {
+#pragma unroll
+        for (int mt = 0; mt < S::kKSteps; ++mt) {
+          o[mt][0] *= al0;
+          o[mt][1] *= al1;
+          o[mt][2] *= al0;
+          o[mt][3] *= al1;
+        }
+      }
+      const uint32_t top_hi = M::pack(p0, p1), bot_hi = M::pack(p2, p3);
+      const float2 th = M::unpack(top_hi), bh = M::unpack(bot_hi);
+      const uint32_t pb0 = movm_t(top_hi), pb1 = movm_t(bot_hi);
+      const uint32_t pl0 = movm_t(M::pack(p0 - th.x, p1 - th.y)), pl1 = movm_t(M::pack(p2 - bh.x, p3 - bh.y));
+      uint32_t keep_lo = 0xffffffffu, keep_hi = 0xffffffffu;
+      if (nvalid < kBlockSize) {
+        keep_lo = (2 * t4 < nvalid ? 0x0000ffffu : 0u) | (2 * t4 + 1 < nvalid ? 0xffff0000u : 0u);
+        keep_hi = (2 * t4 + 8 < nvalid ? 0x0000ffffu : 0u) | (2 * t4 + 9 < nvalid ? 0xffff0000u : 0u);
+      }
+      {
+        const int row = lr + ((lm >> 1) << 3);
+#pragma unroll
+        for (int mt = 0; mt < S::kKSteps; ++mt) {
+          uint32_t a0, a1, a2, a3;
+          ldsm_x4_t(vt + swz(row, 2 * mt + (lm & 1)), a0, a1, a2, a3);
+          a0 &= keep_lo;
+          a1 &= keep_lo;
+          a2 &= keep_hi;
+          a3 &= keep_hi;
+          M::run(o[mt], a0, a1, a2, a3, pb0, pb1);
+          M::run(o[mt], a0, a1, a2, a3, pl0, pl1);
+        }
+      }
+    }
+    // every warp is done with stage s: it may take the page NSTAGE ahead
+    if (__syncthreads_or(bad)) {
+      bad = true;
+      break;
+    }
+    consumed = i + 1;
+    if (warp == 0) issue(i + NSTAGE);
+  }
+  if (bad) {  // after a give-up: thread 0 waits (bounded) for the copies in flight
+    if (threadIdx.x == 0) {
+      const int last = min(nblk, consumed + NSTAGE);
+      for (int i = consumed + 1; i < last; ++i) {
+        const int s = i % NSTAGE;
+        mbar_wait_bounded(bar0 + 8 * s, (phase_bits >> s) & 1u);
+        phase_bits ^= 1u << s;
+      }
+    }
+    return;
+  }
+#pragma unroll
+  for (int msk = 4; msk <= 16; msk <<= 1) {
+    l0 += __shfl_xor_sync(kFull, l0, msk);
+    l1 += __shfl_xor_sync(kFull, l1, msk);
+  }
+  // columns 2 t4, 2 t4 + 1 of this warp: rows d = 16 mt + g8 (+8)
+#pragma unroll
+  for (int e = 0; e < 2; ++e) {
+    const int tr = r0 + 8 * warp + 2 * t4 + e;
+    if (tr >= R) continue;
+    const int p = base + tr / G;
+    const size_t row = out_row(tr);
+    const float mm = e ? m1 : m0, ll = e ? l1 : l0;
+    if (p < tok0) {  // no key of this partition (or before position 0)
+      if (direct)
+#pragma unroll
+        for (int mt = 0; mt < S::kKSteps; ++mt) {
+          reinterpret_cast<T*>(a.out)[row * D + 16 * mt + g8] = Fmt<T>::from_f32(0.f);
+          reinterpret_cast<T*>(a.out)[row * D + 16 * mt + g8 + 8] = Fmt<T>::from_f32(0.f);
+        }
+      continue;
+    }
+    if (direct) {
+      const float inv = 1.f / ll;
+#pragma unroll
+      for (int mt = 0; mt < S::kKSteps; ++mt) {
+        reinterpret_cast<T*>(a.out)[row * D + 16 * mt + g8] = Fmt<T>::from_f32(o[mt][e] * inv);
+        reinterpret_cast<T*>(a.out)[row * D + 16 * mt + g8 + 8] = Fmt<T>::from_f32(o[mt][2 + e] * inv);
+      }
+    } else {
+      const size_t wrow = row * a.num_parts + z;
+#pragma unroll
+      for (int mt = 0; mt < S::kKSteps; ++mt) {
+        a.ws_o[wrow * D + 16 * mt + g8] = o[mt][e];
+        a.ws_o[wrow * D + 16 * mt + g8 + 8] = o[mt][2 + e];
+      }
+      if (g8 == 0) a.ws_ml[wrow] = make_float2(mm, ll);
+    }
+  }
+}
+
 // Merge of the key partitions of each query row (token t = blockIdx.x, HPC
 // heads per CTA from head blockIdx.y * HPC): the row at position pos uses
 // partitions 0 .. pos / partition.

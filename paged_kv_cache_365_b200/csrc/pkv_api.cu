@@ -56,17 +56,49 @@ pkv_status launch_multi(const pkv::MultiArgs& a, const void* k_cache, const void
   return PKV_OK;
 }
 
-// Rows per tile (8 NT) for the rows a sequence brings (max_query_len * G):
-// one tile up to 24 rows, else tiles of 24.
-int multi_ntiles(long long rows) { return rows <= 8 ? 1 : rows <= 16 ? 2 : 3; }
+// Up to 16 rows per sequence (max_query_len * G): one tile of 8 NT rows,
+// the warps splitting the pages.  More: tiles of 8 NW rows, one warp per
+// 8 rows, the warps sharing the pages (paged_multi_rows_kernel).
+int multi_ntiles(long long rows) { return rows <= 8 ? 1 : 2; }
+int multi_rows_warps(long long rows) { return rows <= 16 ? 0 : rows <= 24 ? 3 : 4; }
+constexpr int kRowsStages = 3;
+
+template <typename T, int D, int G, int NW>
+pkv_status launch_multi_rows(const pkv::MultiArgs& a, const void* k_cache, const void* v_cache, int num_blocks,
+                             cudaStream_t st) {
+  using S = pkv::RowsShape<D, NW, kRowsStages>;
+  CUtensorMap mk, mv;
+  const long long rows = static_cast<long long>(num_blocks) * a.num_kv_heads * PKV_BLOCK_SIZE;
+  if (!encode_cache_map(&mk, k_cache, pkv::Mma<T>::kTmaType, D, rows) ||
+      !encode_cache_map(&mv, v_cache, pkv::Mma<T>::kTmaType, D, rows))
+    return PKV_ECUDA;
+  auto kfn = pkv::paged_multi_rows_kernel<T, D, G, NW, kRowsStages>;
+  if (cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(S::kSmem)) !=
+      cudaSuccess)
+    return PKV_ECUDA;
+  const dim3 grid(a.num_kv_heads, a.num_seqs * a.tiles, a.num_parts);
+  if (launch(kfn, grid, dim3(NW * 32), S::kSmem, st, a, mk, mv) != PKV_OK) return PKV_ECUDA;
+  if (a.num_parts > 1) {
+    const dim3 block(pkv::kMergeWarps * 32);
+    if (a.num_parts >= 32)
+      return launch(MultiMergeK<T, D, 1>::fn, dim3(a.total_q, a.num_q_heads), block, 0, st, a);
+    if (a.num_parts >= 8)
+      return launch(MultiMergeK<T, D, 4>::fn, dim3(a.total_q, (a.num_q_heads + 3) / 4), block, 0, st, a);
+    return launch(MultiMergeK<T, D, 8>::fn, dim3(a.total_q, (a.num_q_heads + 7) / 8), block, 0, st, a);
+  }
+  return PKV_OK;
+}
 
 template <typename T, int D, int G>
 pkv_status dispatch_nt_multi(const pkv::MultiArgs& a, int NT, const void* k, const void* v, int nb,
                              cudaStream_t st) {
+  // NT > 0: n-tiles per CTA (pages split over the warps); NT < 0: -NT warps
+  // splitting the rows
   switch (NT) {
     case 1: return launch_multi<T, D, G, 1>(a, k, v, nb, st);
     case 2: return launch_multi<T, D, G, 2>(a, k, v, nb, st);
-    case 3: return launch_multi<T, D, G, 3>(a, k, v, nb, st);
+    case -3: return launch_multi_rows<T, D, G, 3>(a, k, v, nb, st);
+    case -4: return launch_multi_rows<T, D, G, 4>(a, k, v, nb, st);
   }
   return PKV_EINVAL;
 }
@@ -98,7 +130,10 @@ bool encode_fp8_map(CUtensorMap* map, const void* base, int D, long long rows) {
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-constexpr int kFp8Stages = 4;  // pages in flight per warp (4 KB each at D = 128)
+#ifndef PKV_FP8_STAGES
+#define PKV_FP8_STAGES 4
+#endif
+constexpr int kFp8Stages = PKV_FP8_STAGES;  // pages in flight per warp (4 KB each at D = 128)
 
 template <typename T, int D, int G>
 pkv_status launch_decode_fp8(const pkv::DecodeArgs& a, float v_scale, cudaStream_t st) {
@@ -305,6 +340,7 @@ pkv_status pkv_paged_attention_decode(void* out, const void* q, const void* k_ca
     case PKV_F32: return dispatch_dim<float>(a, head_dim, G, st);
     case PKV_F16: return dispatch_dim_mma<__half>(a, head_dim, G, st);
     case PKV_BF16: return dispatch_dim_mma<__nv_bfloat16>(a, head_dim, G, st);
+    case PKV_E4M3: break;  // an FP8 cache decodes through pkv_paged_attention_decode_fp8
   }
   return PKV_EINVAL;
 }
@@ -460,8 +496,11 @@ pkv_status pkv_paged_attention_multi(void* out, const void* q, const void* k_cac
   if (!aligned16(out) || !aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache)) return PKV_EINVAL;
   if (static_cast<long long>(num_blocks) * num_kv_heads * PKV_BLOCK_SIZE > 0x7fffffffLL) return PKV_EINVAL;
   const int G = num_q_heads / num_kv_heads;
-  const int NT = multi_ntiles(static_cast<long long>(max_query_len) * G);
-  const long long tiles = (static_cast<long long>(max_query_len) * G + 8 * NT - 1) / (8 * NT);
+  const long long rows_max = static_cast<long long>(max_query_len) * G;
+  const int NW = multi_rows_warps(rows_max);
+  const int NT = NW ? -NW : multi_ntiles(rows_max);
+  const int tile_rows = 8 * (NW ? NW : NT);
+  const long long tiles = (rows_max + tile_rows - 1) / tile_rows;
   const long long P = (static_cast<long long>(max_context_len) + part - 1) / part;
   if (tiles * num_seqs > 65535 || P > 65535) return PKV_EINVAL;
   const size_t need = multi_workspace_bytes(total_query_tokens, num_q_heads, head_dim, P);
