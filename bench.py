@@ -235,7 +235,7 @@ def run_cuda(args, rank, world, local_rank):
     n_pairs = int(st["cow_pairs"].shape[0])
     ws = cache.workspace(pkv.decode_workspace_bytes(B, Hq, D, max_ctx, args.partition))
     out = torch.empty_like(st["q"])
-    P = max(1, math.ceil(max_ctx / (args.partition or pkv.DEFAULT_PARTITION)))
+    P = max(1, math.ceil(max_ctx / (args.partition or pkv.api.auto_partition(max_ctx))))
     scale = 1.0 / math.sqrt(D)
     # a batch that shares leading blocks is decoded with the cascade (the
     # shared prefix is read once per kv-head)
@@ -415,7 +415,7 @@ def run_multi(args, rank, world, local_rank):
     out = torch.empty_like(st["q"])
     scale = 1.0 / math.sqrt(wl.D)
     n_pairs = int(st["cow_pairs"].shape[0])
-    P = max(1, math.ceil(max_ctx / (args.partition or pkv.DEFAULT_PARTITION)))
+    P = max(1, math.ceil(max_ctx / (args.partition or pkv.api.auto_partition(max_ctx))))
 
     def pre():
         if n_pairs:
@@ -534,7 +534,8 @@ def multi_line(args, r, world):
                    "num_kv_heads": wl.Hkv, "head_dim": wl.D, "block_size": 16,
                    "context_lens": {"min": int(np.min(r["lens"])), "max": int(np.max(r["lens"])),
                                     "sum": int(np.sum(r["lens"]))},
-                   "partition_tokens": args.partition or 512, "partitions_max": r["P"], "seed": args.seed,
+                   "partition_tokens": args.partition or ("auto (%d)" % (1024 if int(np.max(r["lens"])) > 4096 else 512)),
+                   "partitions_max": r["P"], "seed": args.seed,
                    "parallelism": f"replicas{args.gpus}" if args.gpus > 1 else "single-gpu",
                    "l2": "inputs larger than L2 (no flush)" if r["kv"] > 126e6 else "inputs fit in L2"},
         "us_per_step": 1e3 * r["total_ms"] / K,
@@ -787,7 +788,8 @@ def config_of(wl, args, P):
             "head_dim": wl.D, "block_size": 16, "num_blocks": wl.num_blocks,
             "context_lens": {"min": int(wl.context_lens.min()), "max": int(wl.context_lens.max()),
                              "sum": int(wl.context_lens.astype(np.int64).sum())},
-            "partition_tokens": args.partition or 512, "partitions_max": P, "seed": args.seed,
+            "partition_tokens": args.partition or ("auto (%d)" % (1024 if int(wl.context_lens.max()) > 4096 else 512)),
+            "partitions_max": P, "seed": args.seed,
             "cuda_graph": bool(getattr(args, "graph", False)),
             "parallelism": f"replicas{args.gpus}" if args.gpus > 1 else "single-gpu",
             "l2": "inputs larger than L2 (no flush)" if kv_bytes(wl, True) > 126e6 else "inputs fit in L2"}

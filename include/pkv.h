@@ -151,8 +151,9 @@ pkv_status pkv_swap_blocks_check(const int32_t* pairs_host, int num_pairs, int s
 /* ------------------------------------------------------------------------
  * pkv_decode_workspace_bytes -- device workspace pkv_paged_attention_decode
  * needs for these sizes (0 when no sequence can span two partitions).
- * partition_tokens: 0 = PKV_DEFAULT_PARTITION, else a multiple of 16 in
- * [16, 2048].  Returns 0 for arguments pkv_paged_attention_decode rejects.
+ * partition_tokens: 0 = auto (PKV_DEFAULT_PARTITION = 512 tokens, or 1024
+ * when max_context_len > 4096), else a multiple of 16 in [16, 2048].
+ * Returns 0 for arguments pkv_paged_attention_decode rejects.
  *
  * Workspace layout (fp32): partial outputs [num_seqs][num_q_heads][P][head_dim]
  * followed by (running max, running sum) pairs [num_seqs][num_q_heads][P][2],
@@ -177,8 +178,8 @@ size_t pkv_decode_workspace_bytes(int num_seqs, int num_q_heads, int head_dim,
  * computed in fp32 and rounded once to dtype.  Entries of block_tables past
  * page ceil(n/16) - 1 and the unused slots of the last block are never read.
  *
- * Work is split into partitions of partition_tokens tokens (0 = 512; else a
- * multiple of 16 in [16, 2048]); each (sequence, kv-head, partition) keeps
+ * Work is split into partitions of partition_tokens tokens (0 = auto: 512,
+ * or 1024 when max_context_len > 4096; else a multiple of 16 in [16, 2048]); each (sequence, kv-head, partition) keeps
  * the running max and sum of its exponentials and a partial output, and a
  * second kernel merges the partitions of sequences longer than one
  * partition by rescaling each to the overall max (log-sum-exp merge).  The

@@ -19,6 +19,11 @@ from ._lib import check, lib
 
 BLOCK_SIZE = 16
 DEFAULT_PARTITION = 512
+
+
+def auto_partition(max_context_len: int) -> int:
+    """The library's partition for partition=0: 512 tokens, 1024 past 4096."""
+    return 2 * DEFAULT_PARTITION if max_context_len > 4096 else DEFAULT_PARTITION
 # a batch whose sequences share at least this many leading pages (and has at
 # least this many sequences) is decoded with the cascade (prefix read once)
 CASCADE_MIN_PAGES = 8

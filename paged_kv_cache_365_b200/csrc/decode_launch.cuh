@@ -45,8 +45,11 @@ int dtype_bytes(pkv_dtype dt) {
   return 0;
 }
 
-int resolve_partition(int p) {
-  if (p == 0) return PKV_DEFAULT_PARTITION;
+// Tokens per split-K partition.  Auto (0): 512, or 1024 when the longest
+// context exceeds 4096 tokens (long contexts: half the partials to merge and
+// half the per-CTA fixed cost, still thousands of CTAs).
+int resolve_partition(int p, long long max_ctx) {
+  if (p == 0) return max_ctx > 4096 ? 2 * PKV_DEFAULT_PARTITION : PKV_DEFAULT_PARTITION;
   if (p < PKV_BLOCK_SIZE || p > kMaxPartition || p % PKV_BLOCK_SIZE != 0) return -1;
   return p;
 }
@@ -185,7 +188,7 @@ constexpr int kPrefixChunkPages = 32;  // prefix pages per prefix-role CTA (one 
 // (context past the prefix) rounded up to whole pages, kept in [512, 2048],
 // so that a batch of short suffixes needs one partition per sequence.
 int resolve_prefix_partition(int partition_tokens, int max_context_len, int prefix_pages) {
-  if (partition_tokens != 0) return resolve_partition(partition_tokens);
+  if (partition_tokens != 0) return resolve_partition(partition_tokens, max_context_len);
   const long long span = static_cast<long long>(max_context_len) - static_cast<long long>(prefix_pages) * 16;
   long long p = (span + 15) / 16 * 16;
   if (p < PKV_DEFAULT_PARTITION) p = PKV_DEFAULT_PARTITION;
@@ -266,7 +269,7 @@ pkv_status prepare_decode(void* out, const void* q, const void* k_cache, const v
                           int max_context_len, int num_seqs, int num_q_heads, int num_kv_heads, int head_dim,
                           int num_blocks, float scale, int partition_tokens, pkv_dtype dtype, pkv::DecodeArgs* a,
                           long long* P_out) {
-  const int part = resolve_partition(partition_tokens);
+  const int part = resolve_partition(partition_tokens, max_context_len);
   if (dtype_bytes(dtype) == 0 || part < 0 || num_seqs < 0 || num_seqs > 65535 || num_kv_heads <= 0 ||
       num_kv_heads > 65535 || num_q_heads <= 0 || num_q_heads % num_kv_heads != 0 ||
       !group_ok(num_q_heads / num_kv_heads) || !head_dim_ok(head_dim) || num_blocks <= 0 ||

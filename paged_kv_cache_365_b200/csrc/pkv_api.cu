@@ -308,7 +308,7 @@ pkv_status pkv_swap_blocks_check(const int32_t* pairs_host, int num_pairs, int s
 
 size_t pkv_decode_workspace_bytes(int num_seqs, int num_q_heads, int head_dim, int max_context_len,
                                   int partition_tokens) {
-  const int part = resolve_partition(partition_tokens);
+  const int part = resolve_partition(partition_tokens, max_context_len);
   if (part < 0 || num_seqs < 0 || num_q_heads <= 0 || !head_dim_ok(head_dim) || max_context_len < 0) return 0;
   const long long P = (static_cast<long long>(max_context_len) + part - 1) / part;
   return workspace_bytes(num_seqs, num_q_heads, head_dim, P);
@@ -468,7 +468,7 @@ pkv_status pkv_get_error(uint32_t* flags, void* stream) {
 
 size_t pkv_multi_workspace_bytes(int total_query_tokens, int num_q_heads, int head_dim, int max_context_len,
                                  int partition_tokens) {
-  const int part = resolve_partition(partition_tokens);
+  const int part = resolve_partition(partition_tokens, max_context_len);
   if (part < 0 || total_query_tokens < 0 || num_q_heads <= 0 || !head_dim_ok(head_dim) || max_context_len < 0)
     return 0;
   const long long P = (static_cast<long long>(max_context_len) + part - 1) / part;
@@ -483,7 +483,7 @@ pkv_status pkv_paged_attention_multi(void* out, const void* q, const void* k_cac
                                      float scale, int partition_tokens, pkv_dtype dtype, void* workspace,
                                      size_t workspace_bytes_given, void* stream) {
   if (dtype != PKV_F16 && dtype != PKV_BF16) return PKV_EINVAL;  // tensor-core path only
-  const int part = resolve_partition(partition_tokens);
+  const int part = resolve_partition(partition_tokens, max_context_len);
   if (part < 0 || num_seqs < 0 || num_kv_heads <= 0 || num_kv_heads > 65535 || num_q_heads <= 0 ||
       num_q_heads % num_kv_heads != 0 || !group_ok(num_q_heads / num_kv_heads) || !head_dim_ok(head_dim) ||
       num_blocks <= 0 || max_context_len < 0 || max_blocks_per_seq <= 0 || max_query_len < 0 ||

@@ -74,6 +74,10 @@ def test_decode_workspace_bytes(lib):
     assert lib.pkv_decode_workspace_bytes(4, 8, 128, 1025, 0) == 4 * 8 * 3 * 130 * 4
     assert lib.pkv_decode_workspace_bytes(4, 8, 64, 100, 16) == 4 * 8 * 7 * 66 * 4
     assert lib.pkv_decode_workspace_bytes(4, 8, 96, 1000, 0) == 0  # unsupported -> 0
+    # auto past 4096 tokens: 1024-token partitions
+    assert lib.pkv_decode_workspace_bytes(2, 8, 128, 8192, 0) == 2 * 8 * 8 * 130 * 4
+    assert lib.pkv_decode_workspace_bytes(2, 8, 128, 4096, 0) == 2 * 8 * 8 * 130 * 4
+    assert lib.pkv_decode_workspace_bytes(2, 8, 128, 4097, 0) == 2 * 8 * 5 * 130 * 4
     assert lib.pkv_decode_workspace_bytes(4, 8, 128, 1000, 17) == 0
 
 
