@@ -242,6 +242,7 @@ def run_cuda(args, rank, world, local_rank):
     pp = pkv.common_prefix_pages(st["host"]["block_tables"], st["host"]["context_lens"])
     use_cascade = (wl.dtype != "f32" and pp >= pkv.api.CASCADE_MIN_PAGES and B >= pkv.api.CASCADE_MIN_SEQS
                    and not args.no_cascade and not args.kv_fp8)
+    args._cascade = use_cascade
     fp8 = bool(args.kv_fp8)
     if fp8:
         if wl.dtype == "f32":
@@ -261,7 +262,8 @@ def run_cuda(args, rank, world, local_rank):
     prefix = torch.from_numpy(np.ascontiguousarray(st["host"]["block_tables"][0, :pp])).to(dev) if use_cascade else None
     if use_cascade:
         ws = cache.workspace(pkv.decode_prefix_workspace_bytes(B, Hq, D, max_ctx, pp, args.partition))
-        launches_per_step = 1 + (1 if n_pairs else 0) + 2  # append, copies, fused decode, merge
+        # append, copies, cascade (one launch, or prefix + suffix passes), merge
+        launches_per_step = 1 + (1 if n_pairs else 0) + (3 if args.cascade_overlap else 2)
     else:
         launches_per_step = 1 + 1 + (1 if n_pairs else 0) + (1 if P > 1 else 0)
 
@@ -275,7 +277,34 @@ def run_cuda(args, rank, world, local_rank):
         else:
             pkv.kv_append(st["k_new"], st["v_new"], cache.k, cache.v, st["slot_mapping"])
 
+    side = torch.cuda.Stream(dev) if use_cascade else None
+    fork, join = torch.cuda.Event(), torch.cuda.Event()
+    overlap = use_cascade and args.cascade_overlap
+
+    def cascade(phase, s):
+        pkv.paged_attention_decode_prefix(st["q"], cache.k, cache.v, st["block_tables"], st["context_lens"],
+                                          max_ctx, prefix, scale, out=out, workspace=ws, partition=args.partition,
+                                          stream=s, phase=phase)
+
+    def overlapped(pre):
+        # the prefix pass (q and the shared, full prefix blocks only) on a
+        # second stream beside the step's copies and append
+        cur = torch.cuda.current_stream(dev)
+        fork.record(cur)
+        side.wait_event(fork)
+        with torch.cuda.stream(side):
+            cascade(0, side)
+            join.record(side)
+        if pre:
+            pre_decode()
+        cascade(1, cur)
+        cur.wait_event(join)
+        cascade(2, cur)
+
     def decode():
+        if overlap:
+            overlapped(False)
+            return
         if fp8:
             pkv.paged_attention_decode_fp8(st["q"], cache.k, cache.v, st["block_tables"], st["context_lens"],
                                            max_ctx, scale, FP8_SCALE, FP8_SCALE, out=out, workspace=ws,
@@ -289,6 +318,9 @@ def run_cuda(args, rank, world, local_rank):
                                        scale, out=out, workspace=ws, partition=args.partition)
 
     def eager_step():
+        if overlap:
+            overlapped(True)
+            return
         pre_decode()
         decode()
 
@@ -791,6 +823,8 @@ def config_of(wl, args, P):
             "partition_tokens": args.partition or ("auto (%d)" % (1024 if int(wl.context_lens.max()) > 4096 else 512)),
             "partitions_max": P, "seed": args.seed,
             "cuda_graph": bool(getattr(args, "graph", False)),
+            "cascade": None if not getattr(args, "_cascade", False) else
+            ("prefix pass on a second stream beside copies + append" if args.cascade_overlap else "one launch"),
             "parallelism": f"replicas{args.gpus}" if args.gpus > 1 else "single-gpu",
             "l2": "inputs larger than L2 (no flush)" if kv_bytes(wl, True) > 126e6 else "inputs fit in L2"}
 
@@ -869,6 +903,9 @@ def main(argv=None):
                     help="capture one step in a CUDA graph and replay it (launch-bound batches)")
     ap.add_argument("--no-cascade", action="store_true",
                     help="decode a shared-prefix batch with the plain paged kernel")
+    ap.add_argument("--cascade-overlap", action="store_true",
+                    help="run the cascade's prefix pass on a second stream beside the copies and append "
+                         "(three launches instead of one; no faster on B200 so far)")
     ap.add_argument("--kv-fp8", action="store_true",
                     help="the step over an FP8 (E4M3) cache: quantising append + FP8 decode")
     ap.add_argument("--row", choices=["step", "swap", "multi"], default="step",

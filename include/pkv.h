@@ -237,6 +237,28 @@ pkv_status pkv_paged_attention_decode_prefix(void* out, const void* q, const voi
                                              int partition_tokens, pkv_dtype dtype, void* workspace,
                                              size_t workspace_bytes, void* stream);
 
+/* The same cascade launched in phases, so that the prefix pass can run on
+ * another stream beside the step's copy-on-write copies and append (which
+ * never write a full, shared prefix block):
+ *   phase 0: the prefix pass (reads q and the prefix blocks; writes the
+ *            prefix partials of the workspace);
+ *   phase 1: the suffix pass (reads the tables, lengths and suffix blocks
+ *            after this step's append; writes the suffix partials and the
+ *            per-sequence conformity flags);
+ *   phase 2: the merge (needs phases 0 and 1 complete; writes out).
+ * All three take the arguments of pkv_paged_attention_decode_prefix and the
+ * same workspace; ordering between streams is the caller's (an event from
+ * the phase-0 stream before phase 2).  The result is bit-identical to
+ * pkv_paged_attention_decode_prefix.  PKV_EINVAL for another phase. */
+pkv_status pkv_paged_attention_decode_prefix_phase(void* out, const void* q, const void* k_cache,
+                                                   const void* v_cache, const int32_t* block_tables,
+                                                   int max_blocks_per_seq, const int32_t* context_lens,
+                                                   int max_context_len, const int32_t* prefix_blocks,
+                                                   int prefix_pages, int num_seqs, int num_q_heads,
+                                                   int num_kv_heads, int head_dim, int num_blocks, float scale,
+                                                   int partition_tokens, pkv_dtype dtype, void* workspace,
+                                                   size_t workspace_bytes, int phase, void* stream);
+
 /* ------------------------------------------------------------------------
  * pkv_paged_attention_decode_static_ws -- pkv_paged_attention_decode for
  * callers that cannot allocate device memory.

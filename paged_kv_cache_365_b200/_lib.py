@@ -44,6 +44,10 @@ PROTOTYPES = {
     "pkv_paged_attention_decode_prefix": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_int,
                                                   c_void_p, c_int, c_void_p, c_int, c_int, c_int, c_int, c_int,
                                                   c_int, c_float, c_int, c_int, c_void_p, c_size_t, c_void_p]),
+    "pkv_paged_attention_decode_prefix_phase": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_int,
+                                                        c_void_p, c_int, c_void_p, c_int, c_int, c_int, c_int,
+                                                        c_int, c_int, c_float, c_int, c_int, c_void_p, c_size_t,
+                                                        c_int, c_void_p]),
     "pkv_paged_attention_decode_static_ws": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_int,
                                                      c_void_p, c_int, c_int, c_int, c_int, c_int, c_int,
                                                      c_float, c_int, c_int, c_void_p]),

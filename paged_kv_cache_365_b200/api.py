@@ -262,10 +262,14 @@ def paged_attention_decode_prefix(q: torch.Tensor, k_cache: torch.Tensor, v_cach
                                   block_tables: torch.Tensor, context_lens: torch.Tensor, max_context_len: int,
                                   prefix_blocks: torch.Tensor, scale: float, out: Optional[torch.Tensor] = None,
                                   workspace: Optional[torch.Tensor] = None, partition: int = 0,
-                                  stream=None) -> torch.Tensor:
+                                  stream=None, phase: int = -1) -> torch.Tensor:
     """Cascade decode for a batch sharing the blocks ``prefix_blocks``
     (int32 [prefix_pages], device) at the start of every table: the shared
-    pages are read once per kv-head.  Same result as paged_attention_decode."""
+    pages are read once per kv-head.  Same result as paged_attention_decode.
+
+    ``phase`` -1 runs the whole cascade; 0 / 1 / 2 run its prefix pass,
+    suffix pass and merge alone (same arguments and workspace for all three;
+    the caller orders them across streams)."""
     nb, hkv, d = _cache_dims(k_cache, v_cache)
     if q.dim() != 3 or q.shape[2] != d or q.dtype != k_cache.dtype:
         raise ValueError("q must be [B, Hq, D] in the cache dtype")
@@ -277,14 +281,20 @@ def paged_attention_decode_prefix(q: torch.Tensor, k_cache: torch.Tensor, v_cach
         out = torch.empty_like(q)
     need = decode_prefix_workspace_bytes(B, hq, d, max_context_len, pp, partition)
     if workspace is None or workspace.numel() * workspace.element_size() < need:
+        if phase != -1:
+            raise ValueError("the phases of one cascade must share a workspace the caller provides")
         workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
-    check(lib.pkv_paged_attention_decode_prefix(
-        _dev(out, "out", q.dtype), _dev(q, "q"), _dev(k_cache, "k_cache"), _dev(v_cache, "v_cache"),
-        _dev(block_tables, "block_tables", torch.int32), block_tables.shape[1],
-        _dev(context_lens, "context_lens", torch.int32), int(max_context_len),
-        _dev(prefix_blocks, "prefix_blocks", torch.int32), pp, B, hq, hkv, d, nb, float(scale), int(partition),
-        _DT[k_cache.dtype], _dev(workspace, "workspace"), workspace.numel() * workspace.element_size(),
-        _stream(stream, q.device)), "pkv_paged_attention_decode_prefix")
+    args = (_dev(out, "out", q.dtype), _dev(q, "q"), _dev(k_cache, "k_cache"), _dev(v_cache, "v_cache"),
+            _dev(block_tables, "block_tables", torch.int32), block_tables.shape[1],
+            _dev(context_lens, "context_lens", torch.int32), int(max_context_len),
+            _dev(prefix_blocks, "prefix_blocks", torch.int32), pp, B, hq, hkv, d, nb, float(scale), int(partition),
+            _DT[k_cache.dtype], _dev(workspace, "workspace"), workspace.numel() * workspace.element_size())
+    if phase == -1:
+        check(lib.pkv_paged_attention_decode_prefix(*args, _stream(stream, q.device)),
+              "pkv_paged_attention_decode_prefix")
+    else:
+        check(lib.pkv_paged_attention_decode_prefix_phase(*args, int(phase), _stream(stream, q.device)),
+              "pkv_paged_attention_decode_prefix_phase")
     return out
 
 
@@ -583,9 +593,6 @@ class PagedKVCache:
             return t if t.device == dev else t.to(dev, non_blocking=True)
 
         with torch.cuda.stream(st):
-            if cow_pairs.shape[0]:
-                copy_blocks(self.k, self.v, d(cow_pairs), st)
-            kv_append(d(k_new), d(v_new), self.k, self.v, d(slot_mapping), st)
             B, hq = q.shape[0], q.shape[1]
             if out is not None and out.device == dev:
                 res = out
@@ -593,12 +600,18 @@ class PagedKVCache:
                 res = self._out_buffer(q.shape)
             sc = (1.0 / math.sqrt(self.D)) if scale is None else scale
             if prefix_blocks is not None and prefix_blocks.numel() > 0:
+                if cow_pairs.shape[0]:
+                    copy_blocks(self.k, self.v, d(cow_pairs), st)
+                kv_append(d(k_new), d(v_new), self.k, self.v, d(slot_mapping), st)
                 ws = self.workspace(decode_prefix_workspace_bytes(B, hq, self.D, max_context_len,
                                                                   prefix_blocks.numel(), partition))
                 paged_attention_decode_prefix(d(q), self.k, self.v, d(block_tables), d(context_lens),
                                               max_context_len, d(prefix_blocks), sc, out=res, workspace=ws,
                                               partition=partition, stream=st)
             else:
+                if cow_pairs.shape[0]:
+                    copy_blocks(self.k, self.v, d(cow_pairs), st)
+                kv_append(d(k_new), d(v_new), self.k, self.v, d(slot_mapping), st)
                 ws = self.workspace(decode_workspace_bytes(B, hq, self.D, max_context_len, partition))
                 paged_attention_decode(d(q), self.k, self.v, d(block_tables), d(context_lens), max_context_len,
                                        sc, out=res, workspace=ws, partition=partition, stream=st)

@@ -67,6 +67,7 @@ struct DecodeArgs {
   float* wp_o;         // [B][Hq][num_chunks][D] prefix partial outputs
   float2* wp_ml;       // [B][Hq][num_chunks] (max, sum)
   int* conform;        // [B]: 1 when sequence b starts with the prefix
+  int y_offset;        // cascade launched in parts: blockIdx.y + y_offset is the role index
 };
 
 constexpr unsigned kFull = 0xffffffffu;

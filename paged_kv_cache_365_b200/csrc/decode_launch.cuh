@@ -219,46 +219,55 @@ PrefixLayout prefix_layout(long long B, long long Hq, long long D, long long max
   return L;
 }
 
+// Cascade launch.  phase -1: the whole cascade (one launch of both roles,
+// prefix-role CTAs first, then the merge); 0: the prefix-role CTAs only; 1:
+// the suffix-role CTAs only; 2: the merge only.  Split into phases, the
+// prefix pass (which reads only q and the shared, full prefix blocks) can
+// run beside the step's copies and append on another stream.
 template <typename T, int D, int G>
-pkv_status launch_decode_prefix(const pkv::DecodeArgs& a, cudaStream_t st) {
+pkv_status launch_decode_prefix(const pkv::DecodeArgs& a0, int phase, cudaStream_t st) {
   constexpr int kStages = kMmaStages;
   using S = pkv::MmaShape<T, D, G, kMmaWarps, kStages>;
-  CUtensorMap mk, mv;
-  const long long rows = static_cast<long long>(a.num_blocks) * a.num_kv_heads * PKV_BLOCK_SIZE;
-  if (!encode_cache_map(&mk, a.k_cache, pkv::Mma<T>::kTmaType, D, rows) ||
-      !encode_cache_map(&mv, a.v_cache, pkv::Mma<T>::kTmaType, D, rows))
-    return PKV_ECUDA;
-  // one launch: prefix-role CTAs first (the shared pages, from L2), then one
-  // CTA per (kv-head, sequence, suffix partition in flight)
-  auto kfn = pkv::paged_decode_mma_kernel<T, D, G, kMmaWarps, kStages, true>;
-  if (cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(S::kSmem)) !=
-      cudaSuccess)
-    return PKV_ECUDA;
-  const long long ygrid = static_cast<long long>(a.num_qgroups) * a.num_chunks +
-                          static_cast<long long>(a.num_seqs) * a.suffix_z;
-  if (ygrid > 65535) return PKV_EINVAL;
-  if (launch(kfn, dim3(a.num_kv_heads, static_cast<unsigned>(ygrid), 1), dim3(kMmaWarps * 32), S::kSmem, st, a, mk,
-             mv) != PKV_OK)
-    return PKV_ECUDA;
-  // (3) merge prefix chunks and suffix partitions
+  pkv::DecodeArgs a = a0;
+  const long long npre = static_cast<long long>(a.num_qgroups) * a.num_chunks;
+  const long long nsuf = static_cast<long long>(a.num_seqs) * a.suffix_z;
+  if (npre + nsuf > 65535) return PKV_EINVAL;
+  if (phase != 2) {
+    CUtensorMap mk, mv;
+    const long long rows = static_cast<long long>(a.num_blocks) * a.num_kv_heads * PKV_BLOCK_SIZE;
+    if (!encode_cache_map(&mk, a.k_cache, pkv::Mma<T>::kTmaType, D, rows) ||
+        !encode_cache_map(&mv, a.v_cache, pkv::Mma<T>::kTmaType, D, rows))
+      return PKV_ECUDA;
+    auto kfn = pkv::paged_decode_mma_kernel<T, D, G, kMmaWarps, kStages, true>;
+    if (cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(S::kSmem)) !=
+        cudaSuccess)
+      return PKV_ECUDA;
+    const long long ygrid = phase == 0 ? npre : phase == 1 ? nsuf : npre + nsuf;
+    a.y_offset = phase == 1 ? static_cast<int>(npre) : 0;
+    if (ygrid > 0 && launch(kfn, dim3(a.num_kv_heads, static_cast<unsigned>(ygrid), 1), dim3(kMmaWarps * 32),
+                            S::kSmem, st, a, mk, mv) != PKV_OK)
+      return PKV_ECUDA;
+    if (phase >= 0) return PKV_OK;
+  }
+  // merge prefix chunks and suffix partitions
   return launch_merge<T, D, PrefixMergeK>(a, a.num_chunks + a.num_parts, st);
 }
 
 template <typename T, int D>
-pkv_status dispatch_group_prefix(const pkv::DecodeArgs& a, int G, cudaStream_t st) {
+pkv_status dispatch_group_prefix(const pkv::DecodeArgs& a, int G, int phase, cudaStream_t st) {
   switch (G) {
-    case 1: return launch_decode_prefix<T, D, 1>(a, st);
-    case 2: return launch_decode_prefix<T, D, 2>(a, st);
-    case 4: return launch_decode_prefix<T, D, 4>(a, st);
-    case 8: return launch_decode_prefix<T, D, 8>(a, st);
+    case 1: return launch_decode_prefix<T, D, 1>(a, phase, st);
+    case 2: return launch_decode_prefix<T, D, 2>(a, phase, st);
+    case 4: return launch_decode_prefix<T, D, 4>(a, phase, st);
+    case 8: return launch_decode_prefix<T, D, 8>(a, phase, st);
   }
   return PKV_EINVAL;
 }
 
 template <typename T>
-pkv_status dispatch_dim_prefix(const pkv::DecodeArgs& a, int D, int G, cudaStream_t st) {
-  if (D == 64) return dispatch_group_prefix<T, 64>(a, G, st);
-  if (D == 128) return dispatch_group_prefix<T, 128>(a, G, st);
+pkv_status dispatch_dim_prefix(const pkv::DecodeArgs& a, int D, int G, int phase, cudaStream_t st) {
+  if (D == 64) return dispatch_group_prefix<T, 64>(a, G, phase, st);
+  if (D == 128) return dispatch_group_prefix<T, 128>(a, G, phase, st);
   return PKV_EINVAL;
 }
 

@@ -363,12 +363,13 @@ __global__ void __launch_bounds__(NWARPS * 32)
   int b = 0, part = 0, stride = gridDim.z, chunk = 0, qg = 0;
   if (cascade) {
     const int npre = a.num_qgroups * a.num_chunks;
-    if (static_cast<int>(blockIdx.y) < npre) {
+    const int yy = static_cast<int>(blockIdx.y) + a.y_offset;  // a split launch covers part of the roles
+    if (yy < npre) {
       prefix_role = true;
-      qg = blockIdx.y / a.num_chunks;
-      chunk = blockIdx.y % a.num_chunks;
+      qg = yy / a.num_chunks;
+      chunk = yy % a.num_chunks;
     } else {
-      const int y = blockIdx.y - npre;
+      const int y = yy - npre;
       b = y % a.num_seqs;
       part = y / a.num_seqs;
     }

@@ -354,13 +354,16 @@ size_t pkv_decode_prefix_workspace_bytes(int num_seqs, int num_q_heads, int head
   return prefix_layout(num_seqs, num_q_heads, head_dim, max_context_len, prefix_pages, part).total;
 }
 
-pkv_status pkv_paged_attention_decode_prefix(void* out, const void* q, const void* k_cache, const void* v_cache,
+}  // extern "C"
+
+namespace {
+pkv_status decode_prefix_impl(void* out, const void* q, const void* k_cache, const void* v_cache,
                                              const int32_t* block_tables, int max_blocks_per_seq,
                                              const int32_t* context_lens, int max_context_len,
                                              const int32_t* prefix_blocks, int prefix_pages, int num_seqs,
                                              int num_q_heads, int num_kv_heads, int head_dim, int num_blocks,
                                              float scale, int partition_tokens, pkv_dtype dtype, void* workspace,
-                                             size_t workspace_bytes_given, void* stream) {
+                                             size_t workspace_bytes_given, int phase, void* stream) {
   if (dtype != PKV_F16 && dtype != PKV_BF16) return PKV_EINVAL;  // tensor-core path only
   if (prefix_pages <= 0 || prefix_pages > max_blocks_per_seq) return PKV_EINVAL;
   pkv::DecodeArgs a{};
@@ -396,8 +399,39 @@ pkv_status pkv_paged_attention_decode_prefix(void* out, const void* q, const voi
 
   const int G = num_q_heads / num_kv_heads;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if (dtype == PKV_F16) return dispatch_dim_prefix<__half>(a, head_dim, G, st);
-  return dispatch_dim_prefix<__nv_bfloat16>(a, head_dim, G, st);
+  if (dtype == PKV_F16) return dispatch_dim_prefix<__half>(a, head_dim, G, phase, st);
+  return dispatch_dim_prefix<__nv_bfloat16>(a, head_dim, G, phase, st);
+}
+}  // namespace
+
+extern "C" {
+
+pkv_status pkv_paged_attention_decode_prefix(void* out, const void* q, const void* k_cache, const void* v_cache,
+                                             const int32_t* block_tables, int max_blocks_per_seq,
+                                             const int32_t* context_lens, int max_context_len,
+                                             const int32_t* prefix_blocks, int prefix_pages, int num_seqs,
+                                             int num_q_heads, int num_kv_heads, int head_dim, int num_blocks,
+                                             float scale, int partition_tokens, pkv_dtype dtype, void* workspace,
+                                             size_t workspace_bytes_given, void* stream) {
+  return decode_prefix_impl(out, q, k_cache, v_cache, block_tables, max_blocks_per_seq, context_lens,
+                            max_context_len, prefix_blocks, prefix_pages, num_seqs, num_q_heads, num_kv_heads,
+                            head_dim, num_blocks, scale, partition_tokens, dtype, workspace, workspace_bytes_given, -1,
+                            stream);
+}
+
+pkv_status pkv_paged_attention_decode_prefix_phase(void* out, const void* q, const void* k_cache,
+                                                   const void* v_cache, const int32_t* block_tables,
+                                                   int max_blocks_per_seq, const int32_t* context_lens,
+                                                   int max_context_len, const int32_t* prefix_blocks,
+                                                   int prefix_pages, int num_seqs, int num_q_heads,
+                                                   int num_kv_heads, int head_dim, int num_blocks, float scale,
+                                                   int partition_tokens, pkv_dtype dtype, void* workspace,
+                                                   size_t workspace_bytes_given, int phase, void* stream) {
+  if (phase < 0 || phase > 2) return PKV_EINVAL;
+  return decode_prefix_impl(out, q, k_cache, v_cache, block_tables, max_blocks_per_seq, context_lens,
+                            max_context_len, prefix_blocks, prefix_pages, num_seqs, num_q_heads, num_kv_heads,
+                            head_dim, num_blocks, scale, partition_tokens, dtype, workspace, workspace_bytes_given,
+                            phase, stream);
 }
 
 }  // extern "C"

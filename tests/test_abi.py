@@ -149,6 +149,8 @@ def test_prefix_workspace_and_rejections(lib):
         a = list(args)
         a[idx] = bad
         assert lib.pkv_paged_attention_decode_prefix(*a) == 1, (idx, bad)
+    for phase in (-1, 3):
+        assert lib.pkv_paged_attention_decode_prefix_phase(*args[:-1], phase, None) == 1
 
 
 def test_multi_workspace_and_rejections(lib):

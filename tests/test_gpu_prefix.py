@@ -131,3 +131,56 @@ def test_cascade_agrees_with_plain_decode():
     plain = pkv.paged_attention_decode(st["q"], c.k, c.v, st["block_tables"], st["context_lens"],
                                        st["max_context_len"], wl.scale).float().cpu().numpy()
     assert np.abs(got - plain).max() <= TOL[wl.dtype]
+
+
+@pytest.mark.parametrize("wl", CASES[:2], ids=lambda w: w.name)
+def test_phases_on_two_streams_are_bit_identical(wl):
+    """Prefix pass on a second stream, suffix pass and merge on the first:
+    the same bits as the one-launch cascade."""
+    import paged_kv_cache_365_b200 as pkv
+    vals, st, ref = prepared(wl)
+    want, pp = cascade(st, wl)
+    c = st["cache"]
+    tables = st["host"]["block_tables"]
+    prefix = torch.from_numpy(np.ascontiguousarray(tables[0, :pp])).cuda()
+    B, hq, d = st["q"].shape
+    ws = torch.empty(pkv.decode_prefix_workspace_bytes(B, hq, d, st["max_context_len"], pp), dtype=torch.uint8,
+                     device="cuda")
+    out = torch.full_like(st["q"], float("nan"))
+    main, side = torch.cuda.current_stream(), torch.cuda.Stream()
+    fork, join = torch.cuda.Event(), torch.cuda.Event()
+    args = (st["q"], c.k, c.v, st["block_tables"], st["context_lens"], st["max_context_len"], prefix, wl.scale)
+    fork.record(main)
+    side.wait_event(fork)
+    with torch.cuda.stream(side):
+        pkv.paged_attention_decode_prefix(*args, out=out, workspace=ws, stream=side, phase=0)
+        join.record(side)
+    pkv.paged_attention_decode_prefix(*args, out=out, workspace=ws, stream=main, phase=1)
+    main.wait_event(join)
+    pkv.paged_attention_decode_prefix(*args, out=out, workspace=ws, stream=main, phase=2)
+    torch.cuda.synchronize()
+    assert pkv.get_error() == 0
+    assert np.array_equal(out.float().cpu().numpy().astype(np.float64), want)
+    with pytest.raises(ValueError):  # the phases need the caller's workspace
+        pkv.paged_attention_decode_prefix(*args, phase=0)
+
+
+def test_cache_step_on_a_shared_prefix_batch():
+    """PagedKVCache.step on a shared-prefix batch (copy-on-write copies,
+    append, the cascade) against the oracle."""
+    import paged_kv_cache_365_b200 as pkv
+    from paged_kv_cache_365_b200.replay import replay_ops, to_torch
+    wl = workloads.prefix13b(seed=41, B=16, prefix_tokens=256, suffix_range=(1, 60), Hq=8, Hkv=4, D=128,
+                             dtype="f16", name="pfx_step")
+    vals = workloads.draw_values(wl)
+    cache = pkv.PagedKVCache(wl.num_blocks, wl.Hkv, wl.D, torch.float16, "cuda", wl.free_order)
+    replay_ops(cache, wl.ops, to_torch(vals["k_tokens"], "f16", "cuda"), to_torch(vals["v_tokens"], "f16", "cuda"))
+    ids = [int(s) for s in wl.step_seqs]
+    out = cache.step(ids, torch.from_numpy(vals["q"]), torch.from_numpy(vals["k_new"]),
+                     torch.from_numpy(vals["v_new"]), scale=wl.scale)
+    torch.cuda.synchronize()
+    assert pkv.get_error() == 0
+    ref = oracle.replay(wl, vals)
+    want = oracle.paged_decode(vals["q"], ref["cache"].k, ref["cache"].v, ref["block_tables"], ref["context_lens"],
+                               wl.scale, "f16")
+    assert np.abs(out.float().numpy() - want).max() <= TOL["f16"]
