@@ -405,8 +405,10 @@ def run_cuda(args, rank, world, local_rank):
     barrier()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
+    cache.staging_after(stream)   # the first upload starts after e0
     for _ in range(K):
         e2e_step()
+    cache.wait_downloads(stream)  # the last download ends before e1
     e1.record(stream)
     torch.cuda.synchronize()
     barrier()
@@ -501,8 +503,10 @@ def run_multi(args, rank, world, local_rank):
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
+    cache.staging_after(stream)   # the first upload starts after e0
     for _ in range(K):
         e2e_step()
+    cache.wait_downloads(stream)  # the last download ends before e1
     e1.record(stream)
     torch.cuda.synchronize()
     e2e_ms = e0.elapsed_time(e1)

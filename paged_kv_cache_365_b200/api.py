@@ -491,6 +491,82 @@ class BlockAllocator:
 
 
 # ---------------------------------------------------------------------------
+# host <-> device staging of a step's inputs and output
+# ---------------------------------------------------------------------------
+class _Staging:
+    """Double-buffered device copies of a step's host inputs and of its
+    output, on two side streams: the uploads of step i+1 and the download of
+    step i run while the compute stream runs step i / i+1.  Buffer set i % 2
+    is reused only after the compute that read it (inputs) and the download
+    that read it (output) have finished."""
+
+    def __init__(self, device):
+        self.device = device
+        self.h2d = torch.cuda.Stream(device)
+        self.d2h = torch.cuda.Stream(device)
+        self.slot = 0
+        self.bufs = [{}, {}]
+        self.computed = [None, None]    # compute that last read set s is done
+        self.downloaded = [None, None]  # download that last read set s's output is done
+
+    def _buf(self, key, shape, dtype, st):
+        b = self.bufs[self.slot].get(key)
+        if b is None or tuple(b.shape) != tuple(shape) or b.dtype != dtype:
+            b = torch.empty(tuple(shape), dtype=dtype, device=self.device)
+            b.record_stream(st)
+            b.record_stream(self.h2d)
+            b.record_stream(self.d2h)
+            self.bufs[self.slot][key] = b
+        return b
+
+    def upload(self, st, named):
+        """Device tensors for ``named``: device inputs as they are, host ones
+        copied on the upload stream; ``st`` waits for the copies."""
+        s = self.slot
+        out, host = {}, {}
+        for k, t in named.items():
+            if t is None or t.device == self.device:
+                out[k] = t
+            else:
+                host[k] = t
+        if host:
+            if self.computed[s] is not None:
+                self.h2d.wait_event(self.computed[s])
+            for k, t in host.items():
+                out[k] = self._buf(k, t.shape, t.dtype, st)
+            with torch.cuda.stream(self.h2d):
+                for k, t in host.items():
+                    out[k].copy_(t, non_blocking=True)
+                ready = torch.cuda.Event()
+                ready.record(self.h2d)
+            st.wait_event(ready)
+        return out
+
+    def output(self, st, shape, dtype):
+        """This step's device output buffer (free of any pending download)."""
+        s = self.slot
+        if self.downloaded[s] is not None:
+            st.wait_event(self.downloaded[s])
+        return self._buf("_out", shape, dtype, st)
+
+    def finish(self, st, res, out):
+        """After the step's kernels on ``st``: download into a host ``out`` on
+        the download stream; flip to the other buffer set."""
+        s = self.slot
+        done = torch.cuda.Event()
+        done.record(st)
+        self.computed[s] = done
+        if out is not None and out.device != self.device:
+            self.d2h.wait_event(done)
+            with torch.cuda.stream(self.d2h):
+                out.copy_(res, non_blocking=True)
+                ev = torch.cuda.Event()
+                ev.record(self.d2h)
+            self.downloaded[s] = ev
+        self.slot ^= 1
+
+
+# ---------------------------------------------------------------------------
 # a paged KV cache: the pool (torch device memory) plus the allocator
 # ---------------------------------------------------------------------------
 class PagedKVCache:
@@ -580,44 +656,62 @@ class PagedKVCache:
         """Device part of a decode step: copy-on-write copies, append, decode.
 
         Inputs may be host tensors (pinned for asynchronous copies) or
-        device tensors.  When ``out`` is a host tensor the result is copied
-        into it asynchronously on the stream; synchronise before reading.
-        With ``prefix_blocks`` (int32, the blocks every sequence's table
-        starts with) the cascade decode reads that shared prefix once.
-        Returns the device output.
+        device tensors.  Host inputs are uploaded, and a host ``out`` is
+        filled, on two side streams with double-buffered device copies, so a
+        step's transfers overlap the previous / next step's kernels; call
+        ``wait_downloads`` (or synchronise the device) before reading a host
+        ``out``.  With ``prefix_blocks`` (int32, the blocks every sequence's
+        table starts with) the cascade decode reads that shared prefix once.
+        Returns the device output (valid until the call after next reuses
+        its buffer, unless ``out`` is a device tensor).
         """
         dev = self.device
         st = torch.cuda.current_stream(dev) if stream is None else stream
-
-        def d(t):
-            return t if t.device == dev else t.to(dev, non_blocking=True)
-
+        stg = self._staging()
+        x = stg.upload(st, {"slots": slot_mapping, "pairs": cow_pairs, "tables": block_tables,
+                            "lens": context_lens, "q": q, "k": k_new, "v": v_new, "prefix": prefix_blocks})
         with torch.cuda.stream(st):
             B, hq = q.shape[0], q.shape[1]
-            if out is not None and out.device == dev:
-                res = out
-            else:
-                res = self._out_buffer(q.shape)
+            res = out if (out is not None and out.device == dev) else stg.output(st, q.shape, self.dtype)
             sc = (1.0 / math.sqrt(self.D)) if scale is None else scale
+            if cow_pairs.shape[0]:
+                copy_blocks(self.k, self.v, x["pairs"], st)
+            kv_append(x["k"], x["v"], self.k, self.v, x["slots"], st)
             if prefix_blocks is not None and prefix_blocks.numel() > 0:
-                if cow_pairs.shape[0]:
-                    copy_blocks(self.k, self.v, d(cow_pairs), st)
-                kv_append(d(k_new), d(v_new), self.k, self.v, d(slot_mapping), st)
                 ws = self.workspace(decode_prefix_workspace_bytes(B, hq, self.D, max_context_len,
                                                                   prefix_blocks.numel(), partition))
-                paged_attention_decode_prefix(d(q), self.k, self.v, d(block_tables), d(context_lens),
-                                              max_context_len, d(prefix_blocks), sc, out=res, workspace=ws,
-                                              partition=partition, stream=st)
+                paged_attention_decode_prefix(x["q"], self.k, self.v, x["tables"], x["lens"], max_context_len,
+                                              x["prefix"], sc, out=res, workspace=ws, partition=partition,
+                                              stream=st)
             else:
-                if cow_pairs.shape[0]:
-                    copy_blocks(self.k, self.v, d(cow_pairs), st)
-                kv_append(d(k_new), d(v_new), self.k, self.v, d(slot_mapping), st)
                 ws = self.workspace(decode_workspace_bytes(B, hq, self.D, max_context_len, partition))
-                paged_attention_decode(d(q), self.k, self.v, d(block_tables), d(context_lens), max_context_len,
-                                       sc, out=res, workspace=ws, partition=partition, stream=st)
-            if out is not None and out.device != dev:
-                out.copy_(res, non_blocking=True)
+                paged_attention_decode(x["q"], self.k, self.v, x["tables"], x["lens"], max_context_len, sc,
+                                       out=res, workspace=ws, partition=partition, stream=st)
+        stg.finish(st, res, out)
         return res
+
+    def _staging(self) -> "_Staging":
+        stg = getattr(self, "_stg", None)
+        if stg is None:
+            stg = _Staging(self.device)
+            self._stg = stg
+        return stg
+
+    def staging_after(self, stream=None) -> None:
+        """Order the staging streams' next copies after the work already on
+        ``stream`` (default: current), e.g. after a timing event."""
+        st = torch.cuda.current_stream(self.device) if stream is None else stream
+        stg = self._staging()
+        stg.h2d.wait_stream(st)
+        stg.d2h.wait_stream(st)
+
+    def wait_downloads(self, stream=None) -> None:
+        """Make ``stream`` (default: current) wait for the outputs that
+        run_step / run_multi_step are still copying to host tensors."""
+        stg = getattr(self, "_stg", None)
+        if stg is not None:
+            st = torch.cuda.current_stream(self.device) if stream is None else stream
+            st.wait_stream(stg.d2h)
 
     def plan_multi_step(self, seq_ids: Sequence[int], n_new: Sequence[int], width: Optional[int] = None):
         """Host part of a multi-token step: append n_new[i] tokens to each
@@ -651,30 +745,20 @@ class PagedKVCache:
         result asynchronously.  Returns the device output [T, Hq, D]."""
         dev = self.device
         st = torch.cuda.current_stream(dev) if stream is None else stream
-
-        def d(t):
-            return t if t.device == dev else t.to(dev, non_blocking=True)
-
+        stg = self._staging()
+        x = stg.upload(st, {"slots": slot_mapping, "pairs": cow_pairs, "tables": block_tables, "lens": context_lens,
+                            "qs": query_start, "q": q, "k": k_new, "v": v_new})
         with torch.cuda.stream(st):
             if cow_pairs.shape[0]:
-                copy_blocks(self.k, self.v, d(cow_pairs), st)
-            kv_append(d(k_new), d(v_new), self.k, self.v, d(slot_mapping), st)
-            res = out if (out is not None and out.device == dev) else self._out_buffer(q.shape)
+                copy_blocks(self.k, self.v, x["pairs"], st)
+            kv_append(x["k"], x["v"], self.k, self.v, x["slots"], st)
+            res = out if (out is not None and out.device == dev) else stg.output(st, q.shape, self.dtype)
             sc = (1.0 / math.sqrt(self.D)) if scale is None else scale
             ws = self.workspace(multi_workspace_bytes(q.shape[0], q.shape[1], self.D, max_context_len, partition))
-            paged_attention_multi(d(q), self.k, self.v, d(block_tables), d(context_lens), d(query_start),
-                                  max_context_len, max_query_len, sc, out=res, workspace=ws, partition=partition,
-                                  stream=st)
-            if out is not None and out.device != dev:
-                out.copy_(res, non_blocking=True)
+            paged_attention_multi(x["q"], self.k, self.v, x["tables"], x["lens"], x["qs"], max_context_len,
+                                  max_query_len, sc, out=res, workspace=ws, partition=partition, stream=st)
+        stg.finish(st, res, out)
         return res
-
-    def _out_buffer(self, shape) -> torch.Tensor:
-        buf = getattr(self, "_out", None)
-        if buf is None or tuple(buf.shape) != tuple(shape):
-            buf = torch.empty(tuple(shape), dtype=self.dtype, device=self.device)
-            self._out = buf
-        return buf
 
     def step(self, seq_ids: Sequence[int], q: torch.Tensor, k_new: torch.Tensor, v_new: torch.Tensor,
              scale: Optional[float] = None, partition: int = 0, stream=None) -> torch.Tensor:
