@@ -271,3 +271,50 @@ def test_device_range_checks_raise_flags_without_faulting():
     m.copy_blocks(c.k, c.v, torch.tensor([[0, wl.num_blocks]], dtype=torch.int32, device="cuda"))
     assert m.get_error() & m.ERR_COPY_RANGE
     assert m.get_error() == 0
+
+
+def test_workspace_contents_and_graph_replays_do_not_matter():
+    """A split-K decode with a workspace full of garbage, or one reused by a
+    replayed CUDA graph, gives the same bits as with a fresh zeroed one, with
+    no error flag."""
+    m = pkv()
+    wl = workloads.custom([3000, 1700, 40, 2049], Hq=8, Hkv=2, D=128, dtype="f16", seed=77, name="fold")
+    vals = workloads.draw_values(wl)
+    from paged_kv_cache_365_b200.replay import build_step
+    st = build_step(wl, vals, "cuda")
+    c = st["cache"]
+    m.copy_blocks(c.k, c.v, st["cow_pairs"])
+    m.kv_append(st["k_new"], st["v_new"], c.k, c.v, st["slot_mapping"])
+    args = (st["q"], c.k, c.v, st["block_tables"], st["context_lens"], st["max_context_len"], wl.scale)
+    need = m.decode_workspace_bytes(wl.B, wl.Hq, wl.D, st["max_context_len"])
+    assert need > 0
+    clean = m.paged_attention_decode(*args, workspace=torch.zeros(need, dtype=torch.uint8, device="cuda"))
+    garbage = torch.randint(0, 256, (need,), dtype=torch.uint8, device="cuda")
+    dirty = m.paged_attention_decode(*args, workspace=garbage)
+    again = m.paged_attention_decode(*args, workspace=garbage)
+    torch.cuda.synchronize()
+    assert m.get_error() == 0
+    assert torch.equal(clean.view(torch.int16), dirty.view(torch.int16))
+    assert torch.equal(clean.view(torch.int16), again.view(torch.int16))
+    # a captured call replayed: the same epoch every replay
+    ws = torch.zeros(need, dtype=torch.uint8, device="cuda")
+    out = torch.empty_like(st["q"])
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        m.paged_attention_decode(*args, out=out, workspace=ws)  # warm-up outside the capture
+    torch.cuda.current_stream().wait_stream(s)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        m.paged_attention_decode(*args, out=out, workspace=ws)
+    for _ in range(3):
+        out.zero_()
+        g.replay()
+        torch.cuda.synchronize()
+        assert torch.equal(clean.view(torch.int16), out.view(torch.int16))
+    assert m.get_error() == 0
+    ref = oracle.replay(wl, vals)
+    want = oracle.paged_decode(vals["q"], ref["cache"].k, ref["cache"].v, ref["block_tables"], ref["context_lens"],
+                               wl.scale, wl.dtype)
+    assert np.abs(clean.float().cpu().numpy() - want).max() <= TOL["f16"]
