@@ -49,24 +49,22 @@ def e4m3_decode(codes: np.ndarray) -> np.ndarray:
 
 def e4m3_encode(x: np.ndarray) -> np.ndarray:
     """uint8 codes of the float values ``x``: nearest E4M3 value, ties to the
-    even code, saturating at +-448; NaN -> 0x7F (sign kept)."""
+    even code, saturating at +-448; NaN -> 0x7F (sign kept).
+
+    The non-negative codes are increasing in value, so the nearest one to
+    |x| is one of the two table entries around it (found by bisection)."""
     x = np.asarray(x, dtype=np.float64)
     a = np.abs(x).ravel()
-    out = np.empty(a.shape, dtype=np.uint8)
-    chunk = 1 << 16
-    for s in range(0, a.size, chunk):
-        v = a[s:s + chunk, None]
-        d = np.abs(v - _POS[None, :])          # distance to every candidate
-        best = d.min(axis=1, keepdims=True)
-        tie = d == best                         # nearest candidates (one or two)
-        # among the nearest, prefer the even code (lowest set of bit 0)
-        even = tie & ((np.arange(0x7F) & 1) == 0)[None, :]
-        pick = np.where(even.any(axis=1), even.argmax(axis=1), tie.argmax(axis=1))
-        out[s:s + chunk] = pick.astype(np.uint8)
-    out = out.reshape(x.shape)
-    out[np.abs(x) > 448.0] = 0x7E               # saturate (the table search already does up to 448)
+    hi = np.searchsorted(_POS, a, side="left")          # first entry >= |x|
+    hi = np.clip(hi, 0, len(_POS) - 1)
+    lo = np.clip(hi - 1, 0, len(_POS) - 1)
+    d_lo, d_hi = np.abs(a - _POS[lo]), np.abs(_POS[hi] - a)
+    pick = np.where(d_lo < d_hi, lo, np.where(d_hi < d_lo, hi, np.where(lo % 2 == 0, lo, hi)))
+    pick = np.where(a > 448.0, 0x7E, pick)               # saturate
+    out = pick.astype(np.uint8).reshape(x.shape)
     out = out | np.where(np.signbit(x), 0x80, 0).astype(np.uint8)
-    out[np.isnan(x)] = NAN_CODE | (np.where(np.signbit(x[np.isnan(x)]), 0x80, 0).astype(np.uint8))
+    nan = np.isnan(x)
+    out[nan] = NAN_CODE | np.where(np.signbit(x[nan]), 0x80, 0).astype(np.uint8)
     return out
 
 
