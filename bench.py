@@ -258,6 +258,7 @@ def run_cuda(args, rank, world, local_rank):
             pkv.kv_append_fp8(rows, rows, dst, dst, all_slots, FP8_SCALE, FP8_SCALE)
             del rows
         cache.k, cache.v = k8, v8  # the 16-bit pool is released
+        cache.fp8 = (FP8_SCALE, FP8_SCALE)
         torch.cuda.synchronize()
     prefix = torch.from_numpy(np.ascontiguousarray(st["host"]["block_tables"][0, :pp])).to(dev) if use_cascade else None
     if use_cascade:
@@ -383,18 +384,6 @@ def run_cuda(args, rank, world, local_rank):
     d2h = out_host.numel() * out_host.element_size()
 
     def e2e_step():
-        if fp8:
-            # the same calls a user makes, inputs from pinned host memory
-            dv = {k: t.to(dev, non_blocking=True) for k, t in host.items()}
-            if n_pairs:
-                pkv.copy_blocks(cache.k, cache.v, dv["cow_pairs"])
-            pkv.kv_append_fp8(dv["k_new"], dv["v_new"], cache.k, cache.v, dv["slot_mapping"], FP8_SCALE,
-                              FP8_SCALE)
-            pkv.paged_attention_decode_fp8(dv["q"], cache.k, cache.v, dv["block_tables"], dv["context_lens"],
-                                           max_ctx, scale, FP8_SCALE, FP8_SCALE, out=out, workspace=ws,
-                                           partition=args.partition)
-            out_host.copy_(out, non_blocking=True)
-            return
         cache.run_step(host["slot_mapping"], host["cow_pairs"], host["block_tables"], host["context_lens"],
                        max_ctx, host["q"], host["k_new"], host["v_new"], out=out_host, scale=scale,
                        partition=args.partition, stream=stream, prefix_blocks=host.get("prefix_blocks"))

@@ -581,15 +581,31 @@ class PagedKVCache:
     """
 
     def __init__(self, num_blocks: int, num_kv_heads: int, head_dim: int, dtype: torch.dtype,
-                 device="cuda", free_order: Optional[Sequence[int]] = None, fill=float("nan")):
+                 device="cuda", free_order: Optional[Sequence[int]] = None, fill=float("nan"),
+                 fp8_scales: Optional[Tuple[float, float]] = None):
+        """``dtype``: the queries' (and, without ``fp8_scales``, the pool's)
+        dtype.  With ``fp8_scales`` = (k_scale, v_scale) the pool holds FP8
+        E4M3 codes (half the bytes) written by the quantising append; new
+        K/V still arrive in ``dtype``."""
         self.device = torch.device(device)
         self.dtype = dtype
         self.num_blocks, self.Hkv, self.D = int(num_blocks), int(num_kv_heads), int(head_dim)
         shape = (self.num_blocks, self.Hkv, BLOCK_SIZE, self.D)
-        self.k = torch.full(shape, fill, dtype=dtype, device=self.device)
-        self.v = torch.full(shape, fill, dtype=dtype, device=self.device)
+        self.fp8 = None if fp8_scales is None else (float(fp8_scales[0]), float(fp8_scales[1]))
+        if self.fp8 is None:
+            self.k = torch.full(shape, fill, dtype=dtype, device=self.device)
+            self.v = torch.full(shape, fill, dtype=dtype, device=self.device)
+        else:  # unwritten slots hold the NaN code
+            self.k = torch.full(shape, 0x7F, dtype=torch.uint8, device=self.device)
+            self.v = torch.full(shape, 0x7F, dtype=torch.uint8, device=self.device)
         self.alloc = BlockAllocator(num_blocks, free_order)
         self._ws = torch.empty(0, dtype=torch.uint8, device=self.device)
+
+    def _append(self, k: torch.Tensor, v: torch.Tensor, slots: torch.Tensor, stream) -> None:
+        if self.fp8 is None:
+            kv_append(k, v, self.k, self.v, slots, stream)
+        else:
+            kv_append_fp8(k, v, self.k, self.v, slots, self.fp8[0], self.fp8[1], stream)
 
     def workspace(self, nbytes: int) -> torch.Tensor:
         if self._ws.numel() < nbytes:
@@ -610,8 +626,8 @@ class PagedKVCache:
     def enable_swap(self, num_host_blocks: int) -> None:
         """Give the cache a pinned host pool of ``num_host_blocks`` blocks."""
         shape = (int(num_host_blocks), self.Hkv, BLOCK_SIZE, self.D)
-        self.host_k = torch.empty(shape, dtype=self.dtype, pin_memory=True)
-        self.host_v = torch.empty(shape, dtype=self.dtype, pin_memory=True)
+        self.host_k = torch.empty(shape, dtype=self.k.dtype, pin_memory=True)
+        self.host_v = torch.empty(shape, dtype=self.k.dtype, pin_memory=True)
         self.alloc.set_host_pool(num_host_blocks)
 
     def swap_out(self, seq_ids: Sequence[int], stream=None) -> np.ndarray:
@@ -636,8 +652,7 @@ class PagedKVCache:
         slots, pairs = self.alloc.append_tokens(sid, k.shape[0])
         if len(pairs):
             copy_blocks(self.k, self.v, torch.from_numpy(pairs).to(self.device), stream)
-        kv_append(k.to(self.device), v.to(self.device), self.k, self.v,
-                  torch.from_numpy(slots).to(self.device), stream)
+        self._append(k.to(self.device), v.to(self.device), torch.from_numpy(slots).to(self.device), stream)
         return slots
 
     def plan_step(self, seq_ids: Sequence[int], width: Optional[int] = None):
@@ -676,8 +691,13 @@ class PagedKVCache:
             sc = (1.0 / math.sqrt(self.D)) if scale is None else scale
             if cow_pairs.shape[0]:
                 copy_blocks(self.k, self.v, x["pairs"], st)
-            kv_append(x["k"], x["v"], self.k, self.v, x["slots"], st)
-            if prefix_blocks is not None and prefix_blocks.numel() > 0:
+            self._append(x["k"], x["v"], x["slots"], st)
+            if self.fp8 is not None:  # (the cascade reads 16-bit pools only)
+                ws = self.workspace(decode_workspace_bytes(B, hq, self.D, max_context_len, partition))
+                paged_attention_decode_fp8(x["q"], self.k, self.v, x["tables"], x["lens"], max_context_len, sc,
+                                           self.fp8[0], self.fp8[1], out=res, workspace=ws, partition=partition,
+                                           stream=st)
+            elif prefix_blocks is not None and prefix_blocks.numel() > 0:
                 ws = self.workspace(decode_prefix_workspace_bytes(B, hq, self.D, max_context_len,
                                                                   prefix_blocks.numel(), partition))
                 paged_attention_decode_prefix(x["q"], self.k, self.v, x["tables"], x["lens"], max_context_len,
@@ -743,6 +763,8 @@ class PagedKVCache:
         causal attention of each new token over its sequence.  Host inputs
         are copied in (pinned: asynchronously); a host ``out`` receives the
         result asynchronously.  Returns the device output [T, Hq, D]."""
+        if self.fp8 is not None:
+            raise ValueError("multi-token attention reads 16-bit pools only")
         dev = self.device
         st = torch.cuda.current_stream(dev) if stream is None else stream
         stg = self._staging()
@@ -765,7 +787,7 @@ class PagedKVCache:
         """Host plan (allocator) + device step; returns the output on q's device."""
         slots, pairs, tables, lens = self.plan_step(seq_ids)
         max_ctx = int(lens.max()) if len(lens) else 0
-        pp = common_prefix_pages(tables, lens) if self.dtype != torch.float32 else 0
+        pp = common_prefix_pages(tables, lens) if (self.dtype != torch.float32 and self.fp8 is None) else 0
         prefix = (torch.from_numpy(np.ascontiguousarray(tables[0, :pp]))
                   if pp >= CASCADE_MIN_PAGES and len(lens) >= CASCADE_MIN_SEQS else None)
         out = self.run_step(torch.from_numpy(slots), torch.from_numpy(np.ascontiguousarray(pairs)),

@@ -34,6 +34,15 @@ __device__ __forceinline__ void pdl_enter() {
   pdl_trigger();
 }
 
+// 2^x for the online softmax: the SFU's approximate base-2 exponential
+// (PTX ex2.approx.ftz.f32: a few ulp; results below 2^-126 flush to zero, a
+// weight no sum can notice next to the running max's 2^0; 2^-inf = 0).
+__device__ __forceinline__ float exp2_sfu(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 // ---------------------------------------------------------------------------
 // storage formats: a 16-byte chunk holds kVec elements
 // ---------------------------------------------------------------------------

@@ -268,10 +268,10 @@ __global__ void __launch_bounds__(NWARPS * 32, PKV_FP8_MIN_CTAS)
         mx1 = fmaxf(mx1, __shfl_xor_sync(kFull, mx1, msk));
       }
       const float n0 = fmaxf(m0, mx0), n1 = fmaxf(m1, mx1);
-      const float al0 = exp2f(m0 - n0), al1 = exp2f(m1 - n1);
+      const float al0 = exp2_sfu(m0 - n0), al1 = exp2_sfu(m1 - n1);
       m0 = n0;
       m1 = n1;
-      const float p0 = exp2f(x0 - n0), p1 = exp2f(x1 - n1), p2 = exp2f(x2 - n0), p3 = exp2f(x3 - n1);
+      const float p0 = exp2_sfu(x0 - n0), p1 = exp2_sfu(x1 - n1), p2 = exp2_sfu(x2 - n0), p3 = exp2_sfu(x3 - n1);
       l0 = fmaf(l0, al0, p0 + p2);
       l1 = fmaf(l1, al1, p1 + p3);
       // this lane's O rows belong to query g8: its factor comes from the

@@ -31,6 +31,8 @@
 #include <cuda.h>
 #include <math.h>
 
+#include <type_traits>
+
 #include "common.cuh"
 #include "decode.cuh"
 
@@ -255,16 +257,16 @@ __device__ __forceinline__ bool prefix_warp(const DecodeArgs& a, const CUtensorM
         mxB = fmaxf(mxB, __shfl_xor_sync(kFull, mxB, msk));
       }
       const float nA = fmaxf(mA, mxA), nB = fmaxf(mB, mxB);
-      const float alA = exp2f(mA - nA), alB = exp2f(mB - nB);
+      const float alA = exp2_sfu(mA - nA), alB = exp2_sfu(mB - nB);
       mA = nA;
       mB = nB;
       float p[2][4];
 #pragma unroll
       for (int nt = 0; nt < 2; ++nt) {
-        p[nt][0] = exp2f(x[nt][0] - nA);
-        p[nt][1] = exp2f(x[nt][1] - nA);
-        p[nt][2] = exp2f(x[nt][2] - nB);
-        p[nt][3] = exp2f(x[nt][3] - nB);
+        p[nt][0] = exp2_sfu(x[nt][0] - nA);
+        p[nt][1] = exp2_sfu(x[nt][1] - nA);
+        p[nt][2] = exp2_sfu(x[nt][2] - nB);
+        p[nt][3] = exp2_sfu(x[nt][3] - nB);
       }
       lA = fmaf(lA, alA, p[0][0] + p[0][1] + p[1][0] + p[1][1]);
       lB = fmaf(lB, alB, p[0][2] + p[0][3] + p[1][2] + p[1][3]);
@@ -564,10 +566,10 @@ __global__ void __launch_bounds__(NWARPS * 32)
           mx1 = fmaxf(mx1, __shfl_xor_sync(kFull, mx1, msk));
         }
         const float n0 = fmaxf(m0, mx0), n1 = fmaxf(m1, mx1);
-        const float al0 = exp2f(m0 - n0), al1 = exp2f(m1 - n1);
+        const float al0 = exp2_sfu(m0 - n0), al1 = exp2_sfu(m1 - n1);
         m0 = n0;
         m1 = n1;
-        const float p0 = exp2f(x0 - n0), p1 = exp2f(x1 - n1), p2 = exp2f(x2 - n0), p3 = exp2f(x3 - n1);
+        const float p0 = exp2_sfu(x0 - n0), p1 = exp2_sfu(x1 - n1), p2 = exp2_sfu(x2 - n0), p3 = exp2_sfu(x3 - n1);
         l0 = fmaf(l0, al0, p0 + p2);
         l1 = fmaf(l1, al1, p1 + p3);
         if (__any_sync(kFull, al0 != 1.f || al1 != 1.f)) {  // a running max moved
@@ -591,21 +593,27 @@ __global__ void __launch_bounds__(NWARPS * 32)
           keep_lo = (2 * t4 < nvalid ? 0x0000ffffu : 0u) | (2 * t4 + 1 < nvalid ? 0xffff0000u : 0u);
           keep_hi = (2 * t4 + 8 < nvalid ? 0x0000ffffu : 0u) | (2 * t4 + 9 < nvalid ? 0xffff0000u : 0u);
         }
-        // (4) O^T += V^T . P^T
-        {
+        // (4) O^T += V^T . P^T (the masks only on a partial last page)
+        auto pv = [&](auto masked) {
           const int row = lr + ((lm >> 1) << 3);
 #pragma unroll
           for (int mt = 0; mt < S::kKSteps; ++mt) {
             uint32_t a0, a1, a2, a3;
             ldsm_x4_t(vt + swz(row, 2 * mt + (lm & 1)), a0, a1, a2, a3);
-            a0 &= keep_lo;
-            a1 &= keep_lo;
-            a2 &= keep_hi;
-            a3 &= keep_hi;
+            if constexpr (decltype(masked)::value) {
+              a0 &= keep_lo;
+              a1 &= keep_lo;
+              a2 &= keep_hi;
+              a3 &= keep_hi;
+            }
             M::run(o[mt], a0, a1, a2, a3, pb0, pb1);
             M::run(o[mt], a0, a1, a2, a3, pl0, pl1);
           }
-        }
+        };
+        if (nvalid < kBlockSize)
+          pv(std::true_type{});
+        else
+          pv(std::false_type{});
       }
       __syncwarp();
       issue(i + NSTAGE);

@@ -259,11 +259,11 @@ __global__ void __launch_bounds__(NWARPS * 32)
         const float n0 = fmaxf(mr[nt][0], mx0), n1 = fmaxf(mr[nt][1], mx1);
         // a column that has seen no key yet keeps max -inf: subtract 0 instead
         const float u0 = n0 == -INFINITY ? 0.f : n0, u1 = n1 == -INFINITY ? 0.f : n1;
-        al[nt][0] = exp2f(mr[nt][0] - u0);
-        al[nt][1] = exp2f(mr[nt][1] - u1);
+        al[nt][0] = exp2_sfu(mr[nt][0] - u0);
+        al[nt][1] = exp2_sfu(mr[nt][1] - u1);
         mr[nt][0] = n0;
         mr[nt][1] = n1;
-        const float p0 = exp2f(x0 - u0), p1 = exp2f(x1 - u1), p2 = exp2f(x2 - u0), p3 = exp2f(x3 - u1);
+        const float p0 = exp2_sfu(x0 - u0), p1 = exp2_sfu(x1 - u1), p2 = exp2_sfu(x2 - u0), p3 = exp2_sfu(x3 - u1);
         lr_[nt][0] = fmaf(lr_[nt][0], al[nt][0], p0 + p2);
         lr_[nt][1] = fmaf(lr_[nt][1], al[nt][1], p1 + p3);
         moved |= al[nt][0] != 1.f || al[nt][1] != 1.f;
@@ -292,24 +292,31 @@ __global__ void __launch_bounds__(NWARPS * 32)
         keep_lo = (2 * t4 < nvalid ? 0x0000ffffu : 0u) | (2 * t4 + 1 < nvalid ? 0xffff0000u : 0u);
         keep_hi = (2 * t4 + 8 < nvalid ? 0x0000ffffu : 0u) | (2 * t4 + 9 < nvalid ? 0xffff0000u : 0u);
       }
-      // (3) O^T += V^T . P^T, V fragments loaded once for every n-tile
-      {
+      // (3) O^T += V^T . P^T, V fragments loaded once for every n-tile (the
+      // masks only on a partial last page)
+      auto pv = [&](auto masked) {
         const int row = lr + ((lm >> 1) << 3);
 #pragma unroll
         for (int mt = 0; mt < S::kKSteps; ++mt) {
           uint32_t a0, a1, a2, a3;
           ldsm_x4_t(vt + swz(row, 2 * mt + (lm & 1)), a0, a1, a2, a3);
-          a0 &= keep_lo;
-          a1 &= keep_lo;
-          a2 &= keep_hi;
-          a3 &= keep_hi;
+          if constexpr (decltype(masked)::value) {
+            a0 &= keep_lo;
+            a1 &= keep_lo;
+            a2 &= keep_hi;
+            a3 &= keep_hi;
+          }
 #pragma unroll
           for (int nt = 0; nt < NT; ++nt) {
             M::run(o[nt][mt], a0, a1, a2, a3, pb[nt][0], pb[nt][1]);
             M::run(o[nt][mt], a0, a1, a2, a3, pb[nt][2], pb[nt][3]);
           }
         }
-      }
+      };
+      if (nvalid < kBlockSize)
+        pv(std::true_type{});
+      else
+        pv(std::false_type{});
     }
     __syncwarp();
     issue(i + NSTAGE);
@@ -564,10 +571,10 @@ __global__ void __launch_bounds__(NW * 32)
       }
       const float n0 = fmaxf(m0, mx0), n1 = fmaxf(m1, mx1);
       const float u0 = n0 == -INFINITY ? 0.f : n0, u1 = n1 == -INFINITY ? 0.f : n1;
-      const float al0 = exp2f(m0 - u0), al1 = exp2f(m1 - u1);
+      const float al0 = exp2_sfu(m0 - u0), al1 = exp2_sfu(m1 - u1);
       m0 = n0;
       m1 = n1;
-      const float p0 = exp2f(x0 - u0), p1 = exp2f(x1 - u1), p2 = exp2f(x2 - u0), p3 = exp2f(x3 - u1);
+      const float p0 = exp2_sfu(x0 - u0), p1 = exp2_sfu(x1 - u1), p2 = exp2_sfu(x2 - u0), p3 = exp2_sfu(x3 - u1);
       l0 = fmaf(l0, al0, p0 + p2);
       l1 = fmaf(l1, al1, p1 + p3);
       if (__any_sync(kFull, al0 != 1.f || al1 != 1.f)) {
@@ -588,20 +595,26 @@ __global__ void __launch_bounds__(NW * 32)
         keep_lo = (2 * t4 < nvalid ? 0x0000ffffu : 0u) | (2 * t4 + 1 < nvalid ? 0xffff0000u : 0u);
         keep_hi = (2 * t4 + 8 < nvalid ? 0x0000ffffu : 0u) | (2 * t4 + 9 < nvalid ? 0xffff0000u : 0u);
       }
-      {
+      auto pv = [&](auto masked) {
         const int row = lr + ((lm >> 1) << 3);
 #pragma unroll
         for (int mt = 0; mt < S::kKSteps; ++mt) {
           uint32_t a0, a1, a2, a3;
           ldsm_x4_t(vt + swz(row, 2 * mt + (lm & 1)), a0, a1, a2, a3);
-          a0 &= keep_lo;
-          a1 &= keep_lo;
-          a2 &= keep_hi;
-          a3 &= keep_hi;
+          if constexpr (decltype(masked)::value) {
+            a0 &= keep_lo;
+            a1 &= keep_lo;
+            a2 &= keep_hi;
+            a3 &= keep_hi;
+          }
           M::run(o[mt], a0, a1, a2, a3, pb0, pb1);
           M::run(o[mt], a0, a1, a2, a3, pl0, pl1);
         }
-      }
+      };
+      if (nvalid < kBlockSize)
+        pv(std::true_type{});
+      else
+        pv(std::false_type{});
     }
     // every warp is done with stage s: it may take the page NSTAGE ahead
     if (__syncthreads_or(bad)) {

@@ -134,3 +134,50 @@ def test_decode_fp8_float8_dtype_and_zero_context():
     got = out.float().cpu().numpy()
     assert np.array_equal(got[1], np.zeros_like(got[1]))
     assert np.abs(got - want).max() <= TOL["f16"]
+
+
+def test_cache_with_fp8_pool_steps_like_the_oracle():
+    """PagedKVCache with an FP8 pool: prefill and two decode steps (one with
+    a copy-on-write) through the quantising append, host inputs staged; the
+    pool's codes and the outputs against the oracle."""
+    m = pkv()
+    rng = np.random.default_rng(2)
+    Hq, Hkv, D, nb, ks, vs = 8, 2, 128, 40, 0.013, 0.019
+    order = rng.permutation(nb).astype(np.int32)
+    cache = m.PagedKVCache(nb, Hkv, D, torch.bfloat16, free_order=order, fp8_scales=(ks, vs))
+    ref = oracle.RefAllocator(nb, order)
+    dev = oracle.RefCache(nb, Hkv, D, "e4m3")
+
+    def vals(n):
+        return (storage(rng.standard_normal((n, Hkv, D)).astype(np.float32), "bf16"),
+                storage(rng.standard_normal((n, Hkv, D)).astype(np.float32), "bf16"))
+
+    for sid, n in ((0, 50), (1, 7), (2, 130)):
+        ref.add_seq(sid)
+        cache.add_seq(sid)
+        k, v = vals(n)
+        slots, cows = ref.append_tokens(sid, n)
+        dev.copy_blocks(cows)
+        dev.append_fp8(k, v, np.array(slots), "bf16", ks, vs)
+        cache.prefill(sid, to_dev(k, "bf16"), to_dev(v, "bf16"))
+    ref.fork(0, 3)
+    cache.fork(0, 3)
+    ids = [0, 1, 2, 3]
+    for _ in range(2):
+        q = storage(rng.standard_normal((4, Hq, D)).astype(np.float32), "bf16")
+        k, v = vals(4)
+        slots, cows = ref.step(ids)
+        dev.copy_blocks(cows)
+        dev.append_fp8(k, v, np.array(slots), "bf16", ks, vs)
+        out = cache.step(ids, to_dev(q, "bf16").cpu(), to_dev(k, "bf16").cpu(), to_dev(v, "bf16").cpu())
+        torch.cuda.synchronize()
+        assert m.get_error() == 0
+        tables = np.array([ref.block_table(s)[0] + [nb + 3] * (20 - len(ref.block_table(s)[0])) for s in ids],
+                          dtype=np.int32)
+        lens = np.array([ref.block_table(s)[1] for s in ids], dtype=np.int32)
+        want = oracle.paged_decode(q, dev.k, dev.v, tables, lens, D ** -0.5, "bf16", kv_dtype="e4m3", k_scale=ks,
+                                   v_scale=vs)
+        assert np.abs(out.float().numpy() - want).max() <= TOL["bf16"]
+    held = sorted({b for t in ref.tables.values() for b in t})
+    assert np.array_equal(cache.k.cpu().numpy()[held], dev.k[held])
+    assert np.array_equal(cache.v.cpu().numpy()[held], dev.v[held])
