@@ -263,18 +263,25 @@ def run_cuda(args, rank, world, local_rank):
     prefix = torch.from_numpy(np.ascontiguousarray(st["host"]["block_tables"][0, :pp])).to(dev) if use_cascade else None
     if use_cascade:
         ws = cache.workspace(pkv.decode_prefix_workspace_bytes(B, Hq, D, max_ctx, pp, args.partition))
-        # append, copies, cascade (one launch, or prefix + suffix passes), merge
-        launches_per_step = 1 + (1 if n_pairs else 0) + (3 if args.cascade_overlap else 2)
+        # copies + append (one launch), cascade (one launch, or prefix + suffix passes), merge
+        launches_per_step = 1 + (1 if (n_pairs and fp8) else 0) + (3 if args.cascade_overlap else 2)
     else:
-        launches_per_step = 1 + 1 + (1 if n_pairs else 0) + (1 if P > 1 else 0)
+        launches_per_step = 1 + 1 + (1 if (n_pairs and fp8) else 0) + (1 if P > 1 else 0)
 
     # every call goes to the current stream at call time (so that a CUDA
     # graph capture records it)
+    # the step's copy-on-write copies cut to the rows that hold tokens, in
+    # one launch with the append (16-bit pools)
+    copies_host = pkv.cow_copy_rows(st["host"]["cow_pairs"], st["host"]["step_slots"])
+    copies = torch.from_numpy(copies_host).to(dev)
+
     def pre_decode():
-        if n_pairs:
-            pkv.copy_blocks(cache.k, cache.v, st["cow_pairs"])
         if fp8:
+            if n_pairs:
+                pkv.copy_blocks(cache.k, cache.v, st["cow_pairs"])
             pkv.kv_append_fp8(st["k_new"], st["v_new"], cache.k, cache.v, st["slot_mapping"], FP8_SCALE, FP8_SCALE)
+        elif n_pairs:
+            pkv.kv_append_copy(st["k_new"], st["v_new"], cache.k, cache.v, st["slot_mapping"], copies)
         else:
             pkv.kv_append(st["k_new"], st["v_new"], cache.k, cache.v, st["slot_mapping"])
 
@@ -377,6 +384,8 @@ def run_cuda(args, rank, world, local_rank):
     # every step, and the output read back every step
     host = {k: st[k].cpu().pin_memory() for k in ("q", "k_new", "v_new", "slot_mapping", "cow_pairs",
                                                     "block_tables", "context_lens")}
+    if n_pairs and not fp8:
+        host["cow_pairs"] = torch.from_numpy(copies_host).pin_memory()
     if use_cascade:
         host["prefix_blocks"] = prefix.cpu().pin_memory()
     out_host = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)

@@ -116,6 +116,28 @@ pkv_status pkv_copy_blocks(void* k_cache, void* v_cache, const int32_t* pairs, i
 pkv_status pkv_copy_blocks_check(const int32_t* pairs_host, int num_pairs, int num_blocks);
 
 /* ------------------------------------------------------------------------
+ * pkv_kv_append_copy -- a decode step's copy-on-write copies and append in
+ * one launch, each copy cut to the rows that hold tokens.
+ *
+ * "PagedAttention 与 vLLM 推理加速" §3.2(3): a shared, partially filled
+ * block is copied before a sharer appends into it.  Only its first rows
+ * hold tokens; the rows past them are never read.  For each copy
+ * (src, dst, rows) in copies[num_copies][3] (device):
+ *   k_cache[dst, :, r, :] = k_cache[src, :, r, :]  for r < rows   (V alike)
+ * and for every token i with slot_mapping[i] >= 0 the write of
+ * pkv_kv_append.  rows must not exceed the first row a token of this call
+ * writes into dst (then copies and appends touch disjoint rows; the result
+ * on every row below dst's first unwritten row equals pkv_copy_blocks
+ * followed by pkv_kv_append); rows of dst past the appended ones keep what
+ * they held.  Layouts, bit-exactness and the slot rules as pkv_kv_append;
+ * a copy naming a block outside [0, num_blocks), or rows > 16, is skipped
+ * and sets PKV_ERR_COPY_RANGE.
+ * -------------------------------------------------------------------- */
+pkv_status pkv_kv_append_copy(const void* k_new, const void* v_new, void* k_cache, void* v_cache,
+                              const int64_t* slot_mapping, int num_tokens, const int32_t* copies, int num_copies,
+                              int num_kv_heads, int head_dim, int num_blocks, pkv_dtype dtype, void* stream);
+
+/* ------------------------------------------------------------------------
  * pkv_swap_blocks -- block copy between two pools (preemption by swapping).
  *
  * "LLM Systems 24: Efficient LLM Inference with PagedAttention and vLLM" §3

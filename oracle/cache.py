@@ -65,6 +65,17 @@ class RefCache:
         vq = quantize(widen(v_new, src_dtype).astype(np.float32), v_scale)
         self.append(kq, vq, slots)
 
+    def copy_rows_then_append(self, copies, k_new, v_new, slots) -> None:
+        """The step's copy-on-write and append with the copies cut to the
+        rows that hold tokens: for each (src, dst, rows), rows 0..rows-1 of
+        dst receive src's, then the new tokens go to their slots.  Rows of
+        dst at or past ``rows`` that no token is written into keep what they
+        held (no token of the sequence lives there)."""
+        for src, dst, rows in copies:
+            self.k[int(dst), :, :int(rows)] = self.k[int(src), :, :int(rows)]
+            self.v[int(dst), :, :int(rows)] = self.v[int(src), :, :int(rows)]
+        self.append(k_new, v_new, slots)
+
     def copy_blocks(self, pairs) -> None:
         """cache[dst] = cache[src] for each (src, dst), K and V."""
         for src, dst in pairs:

@@ -33,6 +33,8 @@ PROTOTYPES = {
     "pkv_copy_blocks": (c_int, [c_void_p, c_void_p, c_void_p, c_int, c_int, c_int, c_int, c_int,
                                 c_void_p]),
     "pkv_copy_blocks_check": (c_int, [P(c_int32), c_int, c_int]),
+    "pkv_kv_append_copy": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_int, c_void_p, c_int, c_int,
+                                   c_int, c_int, c_int, c_void_p]),
     "pkv_swap_blocks": (c_int, [c_void_p, c_void_p, c_int, c_void_p, c_void_p, c_int, c_void_p, c_int, c_int,
                                 c_int, c_int, c_void_p]),
     "pkv_swap_blocks_check": (c_int, [P(c_int32), c_int, c_int, c_int]),

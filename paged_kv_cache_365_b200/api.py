@@ -197,6 +197,39 @@ def paged_attention_decode_fp8(q: torch.Tensor, k_cache: torch.Tensor, v_cache: 
     return out
 
 
+def cow_copy_rows(pairs: np.ndarray, slots: np.ndarray) -> np.ndarray:
+    """(src, dst, rows) for each copy-on-write pair of a step: rows = the
+    first row a slot of the step writes into dst (16 when none does), the
+    rows of dst that hold tokens and must be copied."""
+    p = np.asarray(pairs, dtype=np.int64).reshape(-1, 2)
+    s = np.asarray(slots, dtype=np.int64)
+    s = s[s >= 0]
+    out = np.empty((p.shape[0], 3), dtype=np.int32)
+    for i, (src, dst) in enumerate(p):
+        hit = s[s // BLOCK_SIZE == dst] % BLOCK_SIZE
+        out[i] = (src, dst, int(hit.min()) if hit.size else BLOCK_SIZE)
+    return out
+
+
+def kv_append_copy(k_new: torch.Tensor, v_new: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
+                   slot_mapping: torch.Tensor, copies: torch.Tensor, stream=None) -> None:
+    """The step's copy-on-write copies and append in one launch: int32
+    ``copies`` [n, 3] = (src, dst, rows) (``cow_copy_rows``): rows 0..rows-1
+    of dst from src, then every token into its slot."""
+    nb, hkv, d = _cache_dims(k_cache, v_cache)
+    if k_new.shape != v_new.shape or k_new.dim() != 3 or tuple(k_new.shape[1:]) != (hkv, d):
+        raise ValueError("k_new/v_new must be [N, Hkv, D] matching the cache")
+    n = k_new.shape[0]
+    if slot_mapping.shape != (n,) or copies.dim() != 2 or copies.shape[1] != 3:
+        raise ValueError("slot_mapping must be [N] and copies [n, 3]")
+    check(lib.pkv_kv_append_copy(_dev(k_new, "k_new", k_cache.dtype), _dev(v_new, "v_new", k_cache.dtype),
+                                 _dev(k_cache, "k_cache"), _dev(v_cache, "v_cache"),
+                                 _dev(slot_mapping, "slot_mapping", torch.int64), n,
+                                 _dev(copies, "copies", torch.int32) if copies.shape[0] else None, copies.shape[0],
+                                 hkv, d, nb, _DT[k_cache.dtype], _stream(stream, k_cache.device)),
+          "pkv_kv_append_copy")
+
+
 def decode_workspace_bytes(num_seqs: int, num_q_heads: int, head_dim: int, max_context_len: int,
                            partition: int = 0) -> int:
     return int(lib.pkv_decode_workspace_bytes(num_seqs, num_q_heads, head_dim, max_context_len, partition))
@@ -601,6 +634,18 @@ class PagedKVCache:
         self.alloc = BlockAllocator(num_blocks, free_order)
         self._ws = torch.empty(0, dtype=torch.uint8, device=self.device)
 
+    def _copy_append(self, pair_shape, x, st) -> None:
+        """The step's copy-on-write copies and append: (src, dst, rows)
+        copies with a 16-bit pool go in one launch with the append, cut to
+        the rows that hold tokens; (src, dst) pairs copy whole blocks."""
+        n = pair_shape[0]
+        if n and pair_shape[1] == 3 and self.fp8 is None:
+            kv_append_copy(x["k"], x["v"], self.k, self.v, x["slots"], x["pairs"], st)
+            return
+        if n:
+            copy_blocks(self.k, self.v, x["pairs"][:, :2].contiguous(), st)
+        self._append(x["k"], x["v"], x["slots"], st)
+
     def _append(self, k: torch.Tensor, v: torch.Tensor, slots: torch.Tensor, stream) -> None:
         if self.fp8 is None:
             kv_append(k, v, self.k, self.v, slots, stream)
@@ -670,6 +715,9 @@ class PagedKVCache:
                  partition: int = 0, stream=None, prefix_blocks: Optional[torch.Tensor] = None) -> torch.Tensor:
         """Device part of a decode step: copy-on-write copies, append, decode.
 
+        ``cow_pairs``: int32 [n, 2] (src, dst) whole-block copies, or [n, 3]
+        (src, dst, rows) from ``cow_copy_rows``: the copies cut to the rows
+        that hold tokens, in one launch with the append.
         Inputs may be host tensors (pinned for asynchronous copies) or
         device tensors.  Host inputs are uploaded, and a host ``out`` is
         filled, on two side streams with double-buffered device copies, so a
@@ -689,9 +737,7 @@ class PagedKVCache:
             B, hq = q.shape[0], q.shape[1]
             res = out if (out is not None and out.device == dev) else stg.output(st, q.shape, self.dtype)
             sc = (1.0 / math.sqrt(self.D)) if scale is None else scale
-            if cow_pairs.shape[0]:
-                copy_blocks(self.k, self.v, x["pairs"], st)
-            self._append(x["k"], x["v"], x["slots"], st)
+            self._copy_append(cow_pairs.shape, x, st)
             if self.fp8 is not None:  # (the cascade reads 16-bit pools only)
                 ws = self.workspace(decode_workspace_bytes(B, hq, self.D, max_context_len, partition))
                 paged_attention_decode_fp8(x["q"], self.k, self.v, x["tables"], x["lens"], max_context_len, sc,
@@ -771,9 +817,7 @@ class PagedKVCache:
         x = stg.upload(st, {"slots": slot_mapping, "pairs": cow_pairs, "tables": block_tables, "lens": context_lens,
                             "qs": query_start, "q": q, "k": k_new, "v": v_new})
         with torch.cuda.stream(st):
-            if cow_pairs.shape[0]:
-                copy_blocks(self.k, self.v, x["pairs"], st)
-            kv_append(x["k"], x["v"], self.k, self.v, x["slots"], st)
+            self._copy_append(cow_pairs.shape, x, st)
             res = out if (out is not None and out.device == dev) else stg.output(st, q.shape, self.dtype)
             sc = (1.0 / math.sqrt(self.D)) if scale is None else scale
             ws = self.workspace(multi_workspace_bytes(q.shape[0], q.shape[1], self.D, max_context_len, partition))
@@ -790,7 +834,8 @@ class PagedKVCache:
         pp = common_prefix_pages(tables, lens) if (self.dtype != torch.float32 and self.fp8 is None) else 0
         prefix = (torch.from_numpy(np.ascontiguousarray(tables[0, :pp]))
                   if pp >= CASCADE_MIN_PAGES and len(lens) >= CASCADE_MIN_SEQS else None)
-        out = self.run_step(torch.from_numpy(slots), torch.from_numpy(np.ascontiguousarray(pairs)),
+        copies = cow_copy_rows(pairs, slots)  # copy only the rows that hold tokens
+        out = self.run_step(torch.from_numpy(slots), torch.from_numpy(copies),
                             torch.from_numpy(np.ascontiguousarray(tables)), torch.from_numpy(lens), max_ctx,
                             q, k_new, v_new, scale=scale, partition=partition, stream=stream,
                             prefix_blocks=prefix)

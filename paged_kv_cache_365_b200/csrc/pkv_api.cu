@@ -251,6 +251,29 @@ pkv_status pkv_copy_blocks(void* k_cache, void* v_cache, const int32_t* pairs, i
                 static_cast<uint4*>(k_cache), static_cast<uint4*>(v_cache), pairs, block_chunks, num_blocks);
 }
 
+pkv_status pkv_kv_append_copy(const void* k_new, const void* v_new, void* k_cache, void* v_cache,
+                              const int64_t* slot_mapping, int num_tokens, const int32_t* copies, int num_copies,
+                              int num_kv_heads, int head_dim, int num_blocks, pkv_dtype dtype, void* stream) {
+  const int es = dtype_bytes(dtype);
+  if (es == 0 || num_tokens < 0 || num_copies < 0 || num_kv_heads <= 0 || !head_dim_ok(head_dim) ||
+      num_blocks <= 0)
+    return PKV_EINVAL;
+  if (num_tokens == 0 && num_copies == 0) return PKV_OK;
+  if (!k_cache || !v_cache || !aligned16(k_cache) || !aligned16(v_cache)) return PKV_EINVAL;
+  if (num_tokens > 0 && (!k_new || !v_new || !slot_mapping || !aligned16(k_new) || !aligned16(v_new)))
+    return PKV_EINVAL;
+  if (num_copies > 0 && !copies) return PKV_EINVAL;
+  const int row_chunks = head_dim * es / 16;
+  const long long ncopy = 2LL * num_copies * num_kv_heads * PKV_BLOCK_SIZE * row_chunks;
+  const long long nappend = 2LL * num_tokens * num_kv_heads * row_chunks;
+  long long blocks = (ncopy + nappend + 255) / 256;
+  if (blocks > 148LL * 16) blocks = 148LL * 16;
+  return launch(pkv::kv_append_copy_kernel, dim3(static_cast<unsigned>(blocks)), dim3(256), 0,
+                static_cast<cudaStream_t>(stream), static_cast<const uint4*>(k_new), static_cast<const uint4*>(v_new),
+                static_cast<uint4*>(k_cache), static_cast<uint4*>(v_cache), slot_mapping, copies, ncopy, nappend,
+                num_kv_heads, row_chunks, num_blocks);
+}
+
 pkv_status pkv_copy_blocks_check(const int32_t* pairs_host, int num_pairs, int num_blocks) {
   if (num_pairs < 0 || num_blocks <= 0 || (num_pairs > 0 && pairs_host == nullptr)) return PKV_EINVAL;
   std::unordered_set<int32_t> dsts, srcs;

@@ -193,3 +193,20 @@ def test_fp8_rejections(lib):
         a = list(dec)
         a[idx] = bad
         assert lib.pkv_paged_attention_decode_fp8(*a) == 1, (idx, bad)
+
+
+def test_append_copy_rejections(lib):
+    ok = [FAKE, FAKE, FAKE, FAKE, FAKE, 4, FAKE, 2, 2, 64, 16, 1, None]
+    for idx, bad in ((11, 7), (9, 80), (8, 0), (5, -1), (7, -1), (2, ODD), (4, None), (6, None)):
+        a = list(ok)
+        a[idx] = bad
+        assert lib.pkv_kv_append_copy(*a) == 1, (idx, bad)
+    a = list(ok)
+    a[5], a[7] = 0, 0
+    assert lib.pkv_kv_append_copy(*a) == 0
+
+
+def test_cow_copy_rows():
+    from paged_kv_cache_365_b200 import cow_copy_rows
+    rows = cow_copy_rows(np.array([[3, 7], [4, 9], [5, 11]]), np.array([7 * 16 + 5, 9 * 16 + 15, -1, 9 * 16 + 3]))
+    assert rows.tolist() == [[3, 7, 5], [4, 9, 3], [5, 11, 16]]

@@ -184,3 +184,33 @@ def test_cache_step_on_a_shared_prefix_batch():
     want = oracle.paged_decode(vals["q"], ref["cache"].k, ref["cache"].v, ref["block_tables"], ref["context_lens"],
                                wl.scale, "f16")
     assert np.abs(out.float().numpy() - want).max() <= TOL["f16"]
+
+
+def test_partial_copy_append_matches_oracle_on_every_token():
+    """The shared-prefix step with its copy-on-write copies cut to the rows
+    that hold tokens, fused with the append: every token row of every
+    sequence bit-exact against the oracle's full copy + append, the decode
+    within tolerance."""
+    import paged_kv_cache_365_b200 as pkv
+    from paged_kv_cache_365_b200.replay import build_step
+    wl = workloads.prefix13b(seed=51, B=24, prefix_tokens=128, suffix_range=(1, 90), Hq=8, Hkv=8, D=128,
+                             dtype="f16", name="pfx_rows_gpu")
+    vals = workloads.draw_values(wl)
+    st = build_step(wl, vals, "cuda")
+    c = st["cache"]
+    copies = pkv.cow_copy_rows(st["host"]["cow_pairs"], st["host"]["step_slots"])
+    assert len(copies) and (copies[:, 2] < 16).all()
+    pkv.kv_append_copy(st["k_new"], st["v_new"], c.k, c.v, st["slot_mapping"], torch.from_numpy(copies).cuda())
+    torch.cuda.synchronize()
+    assert pkv.get_error() == 0
+    ref = oracle.replay(wl, vals)
+    gk, gv = c.k.cpu().view(torch.int16).numpy(), c.v.cpu().view(torch.int16).numpy()
+    tables, lens = ref["block_tables"], ref["context_lens"]
+    for b in range(wl.B):
+        tok = np.arange(int(lens[b]))
+        blk, off = tables[b, tok // 16], tok % 16
+        assert np.array_equal(gk[blk, :, off], ref["cache"].k[blk, :, off].view(np.int16))
+        assert np.array_equal(gv[blk, :, off], ref["cache"].v[blk, :, off].view(np.int16))
+    got, _ = cascade(st, wl)
+    want = oracle.paged_decode(vals["q"], ref["cache"].k, ref["cache"].v, tables, lens, wl.scale, wl.dtype)
+    assert np.abs(got - want).max() <= TOL["f16"]

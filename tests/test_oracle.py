@@ -199,3 +199,49 @@ def test_unwritten_slots_stay_nan():
         written += int(n)
     finite_rows = np.isfinite(k[:, 0, :, 0]).sum()
     assert finite_rows == written
+
+
+def test_partial_copy_then_append_matches_full_copy_on_every_token():
+    """Cutting a copy-on-write copy to the rows below the first appended row
+    changes no token any sequence holds: for the shared-prefix workload's
+    step (a copy per sequence), every (sequence, token) row is identical to
+    the full-copy step's, and the decode output is bit-identical."""
+    wl = workloads.prefix13b(seed=3, B=10, prefix_tokens=48, suffix_range=(1, 40), Hq=4, Hkv=2, D=8, dtype="f16",
+                             name="pfx_rows")
+    vals = workloads.draw_values(wl)
+    full = oracle.replay(wl, vals)
+    alloc = oracle.RefAllocator(wl.num_blocks, wl.free_order)
+    cache = oracle.RefCache(wl.num_blocks, wl.Hkv, wl.D, wl.dtype)
+    cursor = 0
+    for op in wl.ops:
+        if op[0] == "add":
+            alloc.add_seq(op[1])
+        elif op[0] == "fork":
+            alloc.fork(op[1], op[2])
+        elif op[0] == "free":
+            alloc.free_seq(op[1])
+        else:
+            s_, c_ = alloc.append_tokens(op[1], op[2])
+            cache.copy_blocks(c_)
+            cache.append_many(vals["k_tokens"][cursor:cursor + op[2]], vals["v_tokens"][cursor:cursor + op[2]],
+                              np.array(s_))
+            cursor += op[2]
+    ids = [int(s) for s in wl.step_seqs]
+    slots, pairs = alloc.step(ids)
+    assert len(pairs) > 0
+    copies = []
+    for src, dst in pairs:
+        rows = min(int(s) % 16 for s in slots if int(s) // 16 == dst)
+        copies.append((src, dst, rows))
+    assert any(r < 16 for _, _, r in copies)
+    cache.copy_rows_then_append(copies, vals["k_new"], vals["v_new"], np.array(slots))
+    for b, sid in enumerate(ids):
+        table, n = alloc.block_table(sid)
+        for j in range(n):
+            blk, off = table[j // 16], j % 16
+            assert np.array_equal(cache.k[blk, :, off].view(np.int16), full["cache"].k[blk, :, off].view(np.int16))
+            assert np.array_equal(cache.v[blk, :, off].view(np.int16), full["cache"].v[blk, :, off].view(np.int16))
+    a = oracle.paged_decode(vals["q"], cache.k, cache.v, full["block_tables"], full["context_lens"], wl.scale, wl.dtype)
+    b = oracle.paged_decode(vals["q"], full["cache"].k, full["cache"].v, full["block_tables"], full["context_lens"],
+                            wl.scale, wl.dtype)
+    assert np.array_equal(a, b)
