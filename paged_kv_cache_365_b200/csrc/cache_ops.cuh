@@ -81,60 +81,57 @@ __global__ void __launch_bounds__(256)
 
 // A decode step's copy-on-write and append in one launch, the copies cut to
 // the rows that hold tokens: for each copy (src, dst, rows), rows 0..rows-1
-// of dst receive src's (all kv-heads, K and V); every token with a slot gets
-// its K/V row.  The caller gives each copy the first row a token of this
-// call writes into dst, so copies and appends touch disjoint rows and need
-// no ordering.  Items [0, ncopy) are copy chunks (copy, K|V, head, row,
-// chunk), the rest append chunks (K|V, token, head, chunk).
+// of dst receive src's (all kv-heads); every token with a slot gets its row.
+// The caller gives each copy the first row a token of this call writes into
+// dst, so copies and appends touch disjoint rows and need no ordering.
+// Grid (x, n_copies + A, 2): z = K | V; y < n_copies: copy y, its
+// Hkv * rows * row_chunks chunks over the x CTAs; the other A rows of y
+// share the appends.
 __global__ void __launch_bounds__(256)
     kv_append_copy_kernel(const uint4* __restrict__ k_new, const uint4* __restrict__ v_new,
                           uint4* __restrict__ k_cache, uint4* __restrict__ v_cache,
-                          const int64_t* __restrict__ slots, const int32_t* __restrict__ copies,
-                          long long ncopy /* n_copies * 2 * Hkv * 16 * row_chunks */,
-                          long long nappend /* 2 * tokens * Hkv * row_chunks */, int Hkv, int row_chunks,
-                          int num_blocks) {
+                          const int64_t* __restrict__ slots, const int32_t* __restrict__ copies, int n_copies,
+                          int n_tok, int Hkv, int row_chunks, int num_blocks) {
   pdl_enter();
-  const long long stride = static_cast<long long>(gridDim.x) * blockDim.x;
-  const long long per_block = static_cast<long long>(Hkv) * kBlockSize * row_chunks;  // chunks of K (or V) of a block
-  for (long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; i < ncopy + nappend;
-       i += stride) {
-    if (i < ncopy) {
-      const long long p = i / (2 * per_block);
-      const long long w = i - p * 2 * per_block;
-      const bool is_v = w >= per_block;
-      const long long j = is_v ? w - per_block : w;  // (head, row, chunk) within the block
-      const int row = static_cast<int>((j / row_chunks) % kBlockSize);
-      const int src = copies[3 * p], dst = copies[3 * p + 1], rows = copies[3 * p + 2];
-      if (row >= rows) continue;
-      if (src < 0 || src >= num_blocks || dst < 0 || dst >= num_blocks || rows > kBlockSize) {
-        if (j == 0 && !is_v) raise_error(PKV_ERR_COPY_RANGE);
-        continue;
-      }
-      uint4* cache = is_v ? v_cache : k_cache;
-      cache[static_cast<long long>(dst) * per_block + j] = cache[static_cast<long long>(src) * per_block + j];
-    } else {
-      const long long a = i - ncopy;
-      const long long half = nappend / 2;
-      const bool is_v = a >= half;
-      const long long j = is_v ? a - half : a;
-      const int c = static_cast<int>(j % row_chunks);
-      const long long th = j / row_chunks;
-      const int h = static_cast<int>(th % Hkv);
-      const long long t = th / Hkv;
-      const int64_t s = slots[t];
-      if (s < 0) continue;
-      const int64_t blk = s / kBlockSize;
-      const int off = static_cast<int>(s % kBlockSize);
-      if (blk >= num_blocks) {
-        raise_error(PKV_ERR_SLOT_RANGE);
-        continue;
-      }
-      const long long dsti = ((blk * Hkv + h) * kBlockSize + off) * row_chunks + c;
-      if (is_v)
-        v_cache[dsti] = v_new[j];
-      else
-        k_cache[dsti] = k_new[j];
+  const bool is_v = blockIdx.z != 0;
+  uint4* cache = is_v ? v_cache : k_cache;
+  const long long per_block = static_cast<long long>(Hkv) * kBlockSize * row_chunks;
+  if (static_cast<int>(blockIdx.y) < n_copies) {
+    const int p = blockIdx.y;
+    const int src = copies[3 * p], dst = copies[3 * p + 1], rows = copies[3 * p + 2];
+    if (src < 0 || src >= num_blocks || dst < 0 || dst >= num_blocks || rows < 0 || rows > kBlockSize) {
+      if (threadIdx.x == 0 && blockIdx.x == 0 && !is_v) raise_error(PKV_ERR_COPY_RANGE);
+      return;
     }
+    const int per_head = rows * row_chunks;  // chunks of one head's first `rows` rows
+    const int items = Hkv * per_head;
+    const uint4* from = cache + static_cast<long long>(src) * per_block;
+    uint4* to = cache + static_cast<long long>(dst) * per_block;
+    for (int t = blockIdx.x * blockDim.x + threadIdx.x; t < items; t += gridDim.x * blockDim.x) {
+      const int h = t / per_head;
+      const int off = h * kBlockSize * row_chunks + (t - h * per_head);
+      to[off] = from[off];
+    }
+    return;
+  }
+  const long long items = static_cast<long long>(n_tok) * Hkv * row_chunks;
+  const long long stride = static_cast<long long>(gridDim.y - n_copies) * gridDim.x * blockDim.x;
+  for (long long j = (static_cast<long long>(blockIdx.y - n_copies) * gridDim.x + blockIdx.x) * blockDim.x +
+                     threadIdx.x;
+       j < items; j += stride) {
+    const int c = static_cast<int>(j % row_chunks);
+    const long long th = j / row_chunks;
+    const int h = static_cast<int>(th % Hkv);
+    const long long t = th / Hkv;
+    const int64_t s = slots[t];
+    if (s < 0) continue;
+    const int64_t blk = s / kBlockSize;
+    const int off = static_cast<int>(s % kBlockSize);
+    if (blk >= num_blocks) {
+      raise_error(PKV_ERR_SLOT_RANGE);
+      continue;
+    }
+    cache[((blk * Hkv + h) * kBlockSize + off) * row_chunks + c] = (is_v ? v_new : k_new)[j];
   }
 }
 

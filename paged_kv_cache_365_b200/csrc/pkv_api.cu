@@ -264,14 +264,19 @@ pkv_status pkv_kv_append_copy(const void* k_new, const void* v_new, void* k_cach
     return PKV_EINVAL;
   if (num_copies > 0 && !copies) return PKV_EINVAL;
   const int row_chunks = head_dim * es / 16;
-  const long long ncopy = 2LL * num_copies * num_kv_heads * PKV_BLOCK_SIZE * row_chunks;
-  const long long nappend = 2LL * num_tokens * num_kv_heads * row_chunks;
-  long long blocks = (ncopy + nappend + 255) / 256;
-  if (blocks > 148LL * 16) blocks = 148LL * 16;
-  return launch(pkv::kv_append_copy_kernel, dim3(static_cast<unsigned>(blocks)), dim3(256), 0,
-                static_cast<cudaStream_t>(stream), static_cast<const uint4*>(k_new), static_cast<const uint4*>(v_new),
-                static_cast<uint4*>(k_cache), static_cast<uint4*>(v_cache), slot_mapping, copies, ncopy, nappend,
-                num_kv_heads, row_chunks, num_blocks);
+  if (num_copies > 65535 - 1024) return PKV_EINVAL;  // copies are grid rows
+  // x: enough CTAs for one whole block's chunks; the appends take A more rows
+  const long long per_block = static_cast<long long>(num_kv_heads) * PKV_BLOCK_SIZE * row_chunks;
+  const int gx = static_cast<int>((per_block + 255) / 256);
+  const long long append_items = static_cast<long long>(num_tokens) * num_kv_heads * row_chunks;
+  long long A = (append_items + static_cast<long long>(gx) * 256 - 1) / (static_cast<long long>(gx) * 256);
+  if (A < 1) A = 1;
+  if (A > 1024) A = 1024;
+  const dim3 grid(gx, static_cast<unsigned>(num_copies + A), 2);
+  return launch(pkv::kv_append_copy_kernel, grid, dim3(256), 0, static_cast<cudaStream_t>(stream),
+                static_cast<const uint4*>(k_new), static_cast<const uint4*>(v_new), static_cast<uint4*>(k_cache),
+                static_cast<uint4*>(v_cache), slot_mapping, copies, num_copies, num_tokens, num_kv_heads, row_chunks,
+                num_blocks);
 }
 
 pkv_status pkv_copy_blocks_check(const int32_t* pairs_host, int num_pairs, int num_blocks) {
