@@ -49,7 +49,7 @@ pkv_status launch_multi(const pkv::MultiArgs& a, const void* k_cache, const void
     // one CTA per query token; heads per CTA from the partitions a row may span
     if (a.num_parts >= 32)
       return launch(MultiMergeK<T, D, 1>::fn, dim3(a.total_q, a.num_q_heads), block, 0, st, a);
-    if (a.num_parts >= 8)
+    if (a.num_parts >= 16)  // (a row's own partitions are usually far fewer than the batch's most)
       return launch(MultiMergeK<T, D, 4>::fn, dim3(a.total_q, (a.num_q_heads + 3) / 4), block, 0, st, a);
     return launch(MultiMergeK<T, D, 8>::fn, dim3(a.total_q, (a.num_q_heads + 7) / 8), block, 0, st, a);
   }
@@ -82,7 +82,7 @@ pkv_status launch_multi_rows(const pkv::MultiArgs& a, const void* k_cache, const
     const dim3 block(pkv::kMergeWarps * 32);
     if (a.num_parts >= 32)
       return launch(MultiMergeK<T, D, 1>::fn, dim3(a.total_q, a.num_q_heads), block, 0, st, a);
-    if (a.num_parts >= 8)
+    if (a.num_parts >= 16)  // (a row's own partitions are usually far fewer than the batch's most)
       return launch(MultiMergeK<T, D, 4>::fn, dim3(a.total_q, (a.num_q_heads + 3) / 4), block, 0, st, a);
     return launch(MultiMergeK<T, D, 8>::fn, dim3(a.total_q, (a.num_q_heads + 7) / 8), block, 0, st, a);
   }
