@@ -107,10 +107,25 @@ __global__ void __launch_bounds__(256)
     const int items = Hkv * per_head;
     const uint4* from = cache + static_cast<long long>(src) * per_block;
     uint4* to = cache + static_cast<long long>(dst) * per_block;
-    for (int t = blockIdx.x * blockDim.x + threadIdx.x; t < items; t += gridDim.x * blockDim.x) {
-      const int h = t / per_head;
-      const int off = h * kBlockSize * row_chunks + (t - h * per_head);
-      to[off] = from[off];
+    // each thread moves several chunks, kUnroll loads in flight
+    constexpr int kUnroll = 4;
+    const int step = gridDim.x * blockDim.x;
+    for (int t0 = blockIdx.x * blockDim.x + threadIdx.x; t0 < items; t0 += step * kUnroll) {
+      uint4 v[kUnroll];
+      int off[kUnroll];
+#pragma unroll
+      for (int u = 0; u < kUnroll; ++u) {
+        const int t = t0 + u * step;
+        off[u] = -1;
+        if (t < items) {
+          const int h = t / per_head;
+          off[u] = h * kBlockSize * row_chunks + (t - h * per_head);
+          v[u] = from[off[u]];
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < kUnroll; ++u)
+        if (off[u] >= 0) to[off[u]] = v[u];
     }
     return;
   }

@@ -265,9 +265,10 @@ pkv_status pkv_kv_append_copy(const void* k_new, const void* v_new, void* k_cach
   if (num_copies > 0 && !copies) return PKV_EINVAL;
   const int row_chunks = head_dim * es / 16;
   if (num_copies > 65535 - 1024) return PKV_EINVAL;  // copies are grid rows
-  // x: enough CTAs for one whole block's chunks; the appends take A more rows
+  // x: CTAs per copy, each thread moving up to 8 chunks of a whole block;
+  // the appends take A more rows of the grid
   const long long per_block = static_cast<long long>(num_kv_heads) * PKV_BLOCK_SIZE * row_chunks;
-  const int gx = static_cast<int>((per_block + 255) / 256);
+  const int gx = static_cast<int>((per_block + 256 * 8 - 1) / (256 * 8));
   const long long append_items = static_cast<long long>(num_tokens) * num_kv_heads * row_chunks;
   long long A = (append_items + static_cast<long long>(gx) * 256 - 1) / (static_cast<long long>(gx) * 256);
   if (A < 1) A = 1;
