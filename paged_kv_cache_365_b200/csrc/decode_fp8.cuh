@@ -241,8 +241,9 @@ __global__ void __launch_bounds__(NWARPS * 32, PKV_FP8_MIN_CTAS)
       const int nvalid = min(kBlockSize, tok1 - page_tok);
       const uint32_t kt = stage0 + s * S::kStage;
       const uint32_t vt = kt + S::kTile;
-      // (1) S^T = K . Q^T, two chunks of d per ldmatrix
-      float sc[4] = {0.f, 0.f, 0.f, 0.f};
+      // (1) S^T = K . Q^T, two chunks of d per ldmatrix, into two
+      // independent accumulation chains (even and odd chunks)
+      float sc[4] = {0.f, 0.f, 0.f, 0.f}, sd[4] = {0.f, 0.f, 0.f, 0.f};
       {
         const int row = lr + ((lm & 1) << 3);
 #pragma unroll
@@ -251,16 +252,16 @@ __global__ void __launch_bounds__(NWARPS * 32, PKV_FP8_MIN_CTAS)
           ldsm_x4(kt + swz8<D>(row, c + (lm >> 1)), r0, r1, r2, r3);
           M::run(sc, e4m3x2_to<__half>(r0 & 0xffffu), e4m3x2_to<__half>(r1 & 0xffffu),
                  e4m3x2_to<__half>(r0 >> 16), e4m3x2_to<__half>(r1 >> 16), qb[c][0], qb[c][1]);
-          M::run(sc, e4m3x2_to<__half>(r2 & 0xffffu), e4m3x2_to<__half>(r3 & 0xffffu),
+          M::run(sd, e4m3x2_to<__half>(r2 & 0xffffu), e4m3x2_to<__half>(r3 & 0xffffu),
                  e4m3x2_to<__half>(r2 >> 16), e4m3x2_to<__half>(r3 >> 16), qb[c + 1][0], qb[c + 1][1]);
         }
       }
       // (2) scale (K scale folded in), mask the tail, online softmax
       const bool v_lo = g8 < nvalid, v_hi = g8 + 8 < nvalid;
-      const float x0 = v_lo ? sc[0] * xs0 : -INFINITY;
-      const float x1 = v_lo ? sc[1] * xs1 : -INFINITY;
-      const float x2 = v_hi ? sc[2] * xs0 : -INFINITY;
-      const float x3 = v_hi ? sc[3] * xs1 : -INFINITY;
+      const float x0 = v_lo ? (sc[0] + sd[0]) * xs0 : -INFINITY;
+      const float x1 = v_lo ? (sc[1] + sd[1]) * xs1 : -INFINITY;
+      const float x2 = v_hi ? (sc[2] + sd[2]) * xs0 : -INFINITY;
+      const float x3 = v_hi ? (sc[3] + sd[3]) * xs1 : -INFINITY;
       float mx0 = fmaxf(x0, x2), mx1 = fmaxf(x1, x3);
 #pragma unroll
       for (int msk = 4; msk <= 16; msk <<= 1) {
@@ -303,16 +304,19 @@ __global__ void __launch_bounds__(NWARPS * 32, PKV_FP8_MIN_CTAS)
         auto load = [&](int row, uint32_t (&w)[kW]) {
           const unsigned char* p = vbase + swz8<D>(row, vch) + vb0;
           if constexpr (kW == 4) {
-            const uint4 v = row < nvalid ? *reinterpret_cast<const uint4*>(p) : make_uint4(0u, 0u, 0u, 0u);
+            const uint4 v = *reinterpret_cast<const uint4*>(p);
             w[0] = v.x;
             w[1] = v.y;
             w[2] = v.z;
             w[3] = v.w;
           } else {
-            const uint2 v = row < nvalid ? *reinterpret_cast<const uint2*>(p) : make_uint2(0u, 0u);
+            const uint2 v = *reinterpret_cast<const uint2*>(p);
             w[0] = v.x;
             w[1] = v.y;
           }
+          if (nvalid < kBlockSize && row >= nvalid)
+#pragma unroll
+            for (int e = 0; e < kW; ++e) w[e] = 0u;
         };
         load(2 * t4, w0);
         load(2 * t4 + 1, w1);

@@ -398,23 +398,35 @@ __global__ void __launch_bounds__(NWARPS * 32)
 // split the rows instead of the pages.  Warp w owns the 8 rows r0 + 8 w ..
 // r0 + 8 w + 7 (one n-tile, so registers stay as in decode) and every warp
 // consumes every page of the partition from one CTA-wide ring of NSTAGE
-// staged tiles: thread 0 issues the TMA copies, all warps wait on a stage's
-// mbarrier, and a CTA barrier after each page frees its stage for the page
-// NSTAGE ahead.  A page is read once per CTA for all its 8 NW rows; the
-// warps' rows are disjoint, so each writes its own outputs.
+// staged tiles.  All warps wait on a stage's mbarrier; after its last read
+// of a stage a warp counts itself out on that stage's counter, and the warp
+// that completes the count refills the stage with the page NSTAGE ahead, so
+// the warps drift up to NSTAGE pages apart instead of meeting at a CTA
+// barrier per page.  The partition's page table sits in shared memory.  A
+// page is read once per CTA for all its 8 NW rows; the warps' rows are
+// disjoint, so each writes its own outputs.
 template <int D, int NW, int NSTAGE>
 struct RowsShape {
   static constexpr int kTile = kBlockSize * D * 2;
   static constexpr int kStage = 2 * kTile;
   static constexpr int kKSteps = D / 16;
   static constexpr int kBoxes = D / 64;
-  static constexpr size_t kSmem = 1024 + size_t(NSTAGE) * kStage + size_t(NSTAGE) * 8;
-  static constexpr int kTab = 4;  // table entries a lane holds: 128 pages of a 2048-token partition
+  static constexpr int kMaxPages = 128;  // pages of the longest partition (2048 tokens)
+  // stages | full barriers | release counters | page table
+  static constexpr size_t kBarOff = size_t(NSTAGE) * kStage;
+  static constexpr size_t kCntOff = kBarOff + size_t(NSTAGE) * 8;
+  static constexpr size_t kTabOff = kCntOff + size_t(NSTAGE) * 4;
+  static constexpr size_t kSmem = 1024 + kTabOff + size_t(kMaxPages) * 4;
   static_assert(kStage % 1024 == 0, "swizzled boxes need 1024-byte alignment");
 };
 
+// Resident warps per SM the register budget is sized for (6 CTAs of 3
+// warps): capping registers for 8 such CTAs measured slower.
+#ifndef PKV_ROWS_WARPS_PER_SM
+#define PKV_ROWS_WARPS_PER_SM 18
+#endif
 template <typename T, int D, int G, int NW, int NSTAGE>
-__global__ void __launch_bounds__(NW * 32)
+__global__ void __launch_bounds__(NW * 32, PKV_ROWS_WARPS_PER_SM / NW)
     paged_multi_rows_kernel(const MultiArgs a, const __grid_constant__ CUtensorMap tmap_k,
                             const __grid_constant__ CUtensorMap tmap_v) {
   pdl_enter();
@@ -456,60 +468,49 @@ __global__ void __launch_bounds__(NW * 32)
   const uint32_t pad = ((raw_addr + 1023u) & ~1023u) - raw_addr;
   unsigned char* smem = smem_raw + pad;
   const uint32_t stage0 = smem_addr(smem);
-  const uint32_t bar0 = smem_addr(smem + size_t(NSTAGE) * S::kStage);
+  const uint32_t bar0 = smem_addr(smem + S::kBarOff);
+  unsigned int* released = reinterpret_cast<unsigned int*>(smem + S::kCntOff);  // warps done, per stage
+  int* table = reinterpret_cast<int*>(smem + S::kTabOff);                       // physical page i, or -1
+
+  const int pg0 = tok0 / kBlockSize;
+  const int nblk = (tok1 - tok0 + kBlockSize - 1) / kBlockSize;  // <= S::kMaxPages
+  for (int j = threadIdx.x; j < nblk; j += NW * 32) {
+    const int e = a.block_tables[static_cast<long long>(b) * a.bt_stride + pg0 + j];
+    const bool in = e >= 0 && e < a.num_blocks;
+    if (!in) raise_error(PKV_ERR_BLOCK_RANGE);
+    table[j] = in ? e : -1;
+  }
   if (threadIdx.x == 0) {
-    for (int s = 0; s < NSTAGE; ++s) mbar_init(bar0 + 8 * s, 1);
+    for (int s = 0; s < NSTAGE; ++s) {
+      mbar_init(bar0 + 8 * s, 1);
+      released[s] = 0u;
+    }
     fence_barrier_init();
   }
   __syncthreads();
 
-  const int pg0 = tok0 / kBlockSize;
-  const int nblk = (tok1 - tok0 + kBlockSize - 1) / kBlockSize;  // <= 128 = 32 * S::kTab
-  int my_phys[S::kTab];
+  // page i into stage i % NSTAGE (one lane; a page outside the pool only
+  // completes its stage's phase)
+  auto issue = [&](int i) {
+    if (i >= nblk) return;
+    const uint32_t bar = bar0 + 8 * (i % NSTAGE);
+    const int phys = table[i];
+    if (phys >= 0) {
+      const uint32_t dst = stage0 + (i % NSTAGE) * S::kStage;
+      const int y = (phys * a.num_kv_heads + kvh) * kBlockSize;
+      fence_proxy_async_smem();
+      mbar_arrive_expect_tx(bar, S::kStage);
 #pragma unroll
-  for (int h = 0; h < S::kTab; ++h) {
-    my_phys[h] = -1;
-    const int j = lane + 32 * h;
-    if (j < nblk) {
-      const int e = a.block_tables[static_cast<long long>(b) * a.bt_stride + pg0 + j];
-      if (e >= 0 && e < a.num_blocks)
-        my_phys[h] = e;
-      else if (warp == 0)
-        raise_error(PKV_ERR_BLOCK_RANGE);
-    }
-  }
-  auto phys_of = [&](int i) {
-    int r = -1;
-#pragma unroll
-    for (int h = 0; h < S::kTab; ++h) {
-      const int v = __shfl_sync(kFull, my_phys[h], i & 31);
-      if ((i >> 5) == h) r = v;
-    }
-    return r;
-  };
-  auto issue = [&](int i) {  // warp 0 only (its lanes take part in the shuffle)
-    const int phys = phys_of(i);
-    if (lane == 0 && i < nblk) {
-      const uint32_t bar = bar0 + 8 * (i % NSTAGE);
-      if (phys >= 0) {
-        const uint32_t dst = stage0 + (i % NSTAGE) * S::kStage;
-        const int y = (phys * a.num_kv_heads + kvh) * kBlockSize;
-        fence_proxy_async_smem();
-        mbar_arrive_expect_tx(bar, S::kStage);
-#pragma unroll
-        for (int bx = 0; bx < S::kBoxes; ++bx) {
-          tma_load_2d(dst + bx * 2048, &tmap_k, bx * 64, y, bar);
-          tma_load_2d(dst + S::kTile + bx * 2048, &tmap_v, bx * 64, y, bar);
-        }
-      } else {
-        mbar_arrive(bar);
+      for (int bx = 0; bx < S::kBoxes; ++bx) {
+        tma_load_2d(dst + bx * 2048, &tmap_k, bx * 64, y, bar);
+        tma_load_2d(dst + S::kTile + bx * 2048, &tmap_v, bx * 64, y, bar);
       }
+    } else {
+      mbar_arrive(bar);
     }
   };
-  if (warp == 0) {
-#pragma unroll
+  if (threadIdx.x == 0)
     for (int i = 0; i < NSTAGE; ++i) issue(i);
-  }
 
   // this warp's column g8 (row r0 + 8 warp + g8) and its lane's columns 2 t4, 2 t4 + 1
   uint32_t qb[S::kKSteps][2];
@@ -532,37 +533,40 @@ __global__ void __launch_bounds__(NW * 32)
   for (int mt = 0; mt < S::kKSteps; ++mt) o[mt][0] = o[mt][1] = o[mt][2] = o[mt][3] = 0.f;
   float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
   uint32_t phase_bits = 0;
-  int consumed = 0;
   bool bad = false;
 
   for (int i = 0; i < nblk; ++i) {
     const int s = i % NSTAGE;
     const bool ok = __all_sync(kFull, mbar_wait_bounded(bar0 + 8 * s, (phase_bits >> s) & 1u));
     phase_bits ^= 1u << s;
-    if (!ok) {
+    if (!ok) {  // this warp gives up; the others time out on the pages it never releases
       if (lane == 0) raise_error(PKV_ERR_TIMEOUT);
       bad = true;
+      break;
     }
-    if (!bad && phys_of(i) >= 0) {
+    if (table[i] >= 0) {
       const int page_tok = tok0 + i * kBlockSize;
       const int nvalid = min(kBlockSize, tok1 - page_tok);
       const uint32_t kt = stage0 + s * S::kStage;
       const uint32_t vt = kt + S::kTile;
-      float sc[4] = {0.f, 0.f, 0.f, 0.f};
+      // two independent accumulation chains over the k-steps
+      float sc[4] = {0.f, 0.f, 0.f, 0.f}, sd[4] = {0.f, 0.f, 0.f, 0.f};
       {
         const int row = lr + ((lm & 1) << 3);
 #pragma unroll
-        for (int ks = 0; ks < S::kKSteps; ++ks) {
-          uint32_t a0, a1, a2, a3;
+        for (int ks = 0; ks < S::kKSteps; ks += 2) {
+          uint32_t a0, a1, a2, a3, b0, b1, b2, b3;
           ldsm_x4(kt + swz(row, 2 * ks + (lm >> 1)), a0, a1, a2, a3);
+          ldsm_x4(kt + swz(row, 2 * ks + 2 + (lm >> 1)), b0, b1, b2, b3);
           M::run(sc, a0, a1, a2, a3, qb[ks][0], qb[ks][1]);
+          M::run(sd, b0, b1, b2, b3, qb[ks + 1][0], qb[ks + 1][1]);
         }
       }
       const int jA = page_tok + g8, jB = page_tok + g8 + 8;
-      const float x0 = jA <= pos0 ? sc[0] * a.qk_scale : -INFINITY;
-      const float x1 = jA <= pos1 ? sc[1] * a.qk_scale : -INFINITY;
-      const float x2 = jB <= pos0 ? sc[2] * a.qk_scale : -INFINITY;
-      const float x3 = jB <= pos1 ? sc[3] * a.qk_scale : -INFINITY;
+      const float x0 = jA <= pos0 ? (sc[0] + sd[0]) * a.qk_scale : -INFINITY;
+      const float x1 = jA <= pos1 ? (sc[1] + sd[1]) * a.qk_scale : -INFINITY;
+      const float x2 = jB <= pos0 ? (sc[2] + sd[2]) * a.qk_scale : -INFINITY;
+      const float x3 = jB <= pos1 ? (sc[3] + sd[3]) * a.qk_scale : -INFINITY;
       float mx0 = fmaxf(x0, x2), mx1 = fmaxf(x1, x3);
 #pragma unroll
       for (int msk = 4; msk <= 16; msk <<= 1) {
@@ -616,22 +620,28 @@ __global__ void __launch_bounds__(NW * 32)
       else
         pv(std::false_type{});
     }
-    // every warp is done with stage s: it may take the page NSTAGE ahead
-    if (__syncthreads_or(bad)) {
-      bad = true;
-      break;
-    }
-    consumed = i + 1;
-    if (warp == 0) issue(i + NSTAGE);
-  }
-  if (bad) {  // after a give-up: thread 0 waits (bounded) for the copies in flight
-    if (threadIdx.x == 0) {
-      const int last = min(nblk, consumed + NSTAGE);
-      for (int i = consumed + 1; i < last; ++i) {
-        const int s = i % NSTAGE;
-        mbar_wait_bounded(bar0 + 8 * s, (phase_bits >> s) & 1u);
-        phase_bits ^= 1u << s;
+    // this warp is done with stage s; the last of the NW warps to say so
+    // refills it with the page NSTAGE ahead (the fences order every warp's
+    // reads of the stage before the copy that overwrites it)
+    __syncwarp();
+    if (lane == 0) {
+      __threadfence_block();
+      const unsigned int before = atomicAdd(&released[s], 1u);
+      if (before % NW == NW - 1) {
+        __threadfence_block();
+        issue(i + NSTAGE);
       }
+    }
+  }
+  // every copy this CTA issued lands before the CTA exits: after a give-up,
+  // thread 0 waits (bounded) for the last page issued into each stage
+  if (__syncthreads_or(bad)) {
+    if (threadIdx.x == 0) {
+      unsigned int issued = 0;  // pages issued: NSTAGE + the refills (one per NW releases)
+      for (int st = 0; st < NSTAGE; ++st) issued += released[st] / NW;
+      issued = min(static_cast<unsigned int>(nblk), issued + NSTAGE);
+      for (int i = max(0, static_cast<int>(issued) - NSTAGE); i < static_cast<int>(issued); ++i)
+        mbar_wait_bounded(bar0 + 8 * (i % NSTAGE), (i / NSTAGE) & 1u);
     }
     return;
   }

@@ -67,6 +67,7 @@ template <typename T, int D, int G, int NW>
 pkv_status launch_multi_rows(const pkv::MultiArgs& a, const void* k_cache, const void* v_cache, int num_blocks,
                              cudaStream_t st) {
   using S = pkv::RowsShape<D, NW, kRowsStages>;
+  static_assert(kMaxPartition / PKV_BLOCK_SIZE <= S::kMaxPages, "the page table of a partition fits shared memory");
   CUtensorMap mk, mv;
   const long long rows = static_cast<long long>(num_blocks) * a.num_kv_heads * PKV_BLOCK_SIZE;
   if (!encode_cache_map(&mk, k_cache, pkv::Mma<T>::kTmaType, D, rows) ||
