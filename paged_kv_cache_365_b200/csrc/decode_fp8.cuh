@@ -49,6 +49,13 @@ __device__ __forceinline__ uint32_t e4m3x2_to<__half>(uint32_t pair16) {
   return d;
 }
 
+// Four E4M3 codes (bytes 0..3 of w) to fp16 pairs: lo = bytes 0, 1 and
+// hi = bytes 2, 3.
+__device__ __forceinline__ void e4m3x4_to_f16(uint32_t w, uint32_t& lo, uint32_t& hi) {
+  lo = e4m3x2_to<__half>(w & 0xffffu);
+  hi = e4m3x2_to<__half>(w >> 16);
+}
+
 
 // Byte offset of 16-byte chunk `chunk` of row `row` in an FP8 tile of 16
 // rows x D bytes stored with the TMA swizzle matching its row length
@@ -250,10 +257,13 @@ __global__ void __launch_bounds__(NWARPS * 32, PKV_FP8_MIN_CTAS)
         for (int c = 0; c < S::kChunks; c += 2) {
           uint32_t r0, r1, r2, r3;
           ldsm_x4(kt + swz8<D>(row, c + (lm >> 1)), r0, r1, r2, r3);
-          M::run(sc, e4m3x2_to<__half>(r0 & 0xffffu), e4m3x2_to<__half>(r1 & 0xffffu),
-                 e4m3x2_to<__half>(r0 >> 16), e4m3x2_to<__half>(r1 >> 16), qb[c][0], qb[c][1]);
-          M::run(sd, e4m3x2_to<__half>(r2 & 0xffffu), e4m3x2_to<__half>(r3 & 0xffffu),
-                 e4m3x2_to<__half>(r2 >> 16), e4m3x2_to<__half>(r3 >> 16), qb[c + 1][0], qb[c + 1][1]);
+          uint32_t f0, f1, f2, f3, f4, f5, f6, f7;
+          e4m3x4_to_f16(r0, f0, f2);
+          e4m3x4_to_f16(r1, f1, f3);
+          e4m3x4_to_f16(r2, f4, f6);
+          e4m3x4_to_f16(r3, f5, f7);
+          M::run(sc, f0, f1, f2, f3, qb[c][0], qb[c][1]);
+          M::run(sd, f4, f5, f6, f7, qb[c + 1][0], qb[c + 1][1]);
         }
       }
       // (2) scale (K scale folded in), mask the tail, online softmax
@@ -331,8 +341,9 @@ __global__ void __launch_bounds__(NWARPS * 32, PKV_FP8_MIN_CTAS)
         const uint32_t sel = bsel | ((4 + bsel) << 4) | ((bsel + 1) << 8) | ((5 + bsel) << 12);
         const uint32_t lo01 = __byte_perm(w0[w], w1[w], sel);
         const uint32_t lo89 = __byte_perm(w8[w], w9[w], sel);
-        const uint32_t b0j = e4m3x2_to<__half>(lo01 & 0xffffu), b0k = e4m3x2_to<__half>(lo01 >> 16);
-        const uint32_t b1j = e4m3x2_to<__half>(lo89 & 0xffffu), b1k = e4m3x2_to<__half>(lo89 >> 16);
+        uint32_t b0j, b0k, b1j, b1k;
+        e4m3x4_to_f16(lo01, b0j, b0k);
+        e4m3x4_to_f16(lo89, b1j, b1k);
         M::run(o[j], pa0, pa1, pa2, pa3, b0j, b1j);
         M::run(o[j + 1], pa0, pa1, pa2, pa3, b0k, b1k);
       }

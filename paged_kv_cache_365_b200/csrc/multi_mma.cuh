@@ -398,17 +398,21 @@ __global__ void __launch_bounds__(NWARPS * 32)
 // split the rows instead of the pages.  Warp w owns the 8 rows r0 + 8 w ..
 // r0 + 8 w + 7 (one n-tile, so registers stay as in decode) and every warp
 // consumes every page of the partition from one CTA-wide ring of NSTAGE
-// staged tiles.  All warps wait on a stage's mbarrier; after its last read
-// of a stage a warp counts itself out on that stage's counter, and the warp
-// that completes the count refills the stage with the page NSTAGE ahead, so
-// the warps drift up to NSTAGE pages apart instead of meeting at a CTA
-// barrier per page.  The partition's page table sits in shared memory.  A
-// page is read once per CTA for all its 8 NW rows; the warps' rows are
-// disjoint, so each writes its own outputs.
-template <int D, int NW, int NSTAGE>
+// stages of KP pages each.  A warp takes a stage's KP pages in one step: their
+// score MMAs form independent chains, one max / rescale serves all of them,
+// and their P.V products interleave, so a step has KP times the independent
+// work of a page at the same per-step softmax cost.  All warps wait on a
+// stage's mbarrier; after its last read of a stage a warp counts itself out
+// on that stage's counter, and the warp that completes the count refills the
+// stage with the pages NSTAGE steps ahead, so the warps drift up to NSTAGE
+// steps apart instead of meeting at a CTA barrier.  The partition's page
+// table sits in shared memory.  A page is read once per CTA for all its
+// 8 NW rows; the warps' rows are disjoint, so each writes its own outputs.
+template <int D, int NW, int NSTAGE, int KP>
 struct RowsShape {
   static constexpr int kTile = kBlockSize * D * 2;
-  static constexpr int kStage = 2 * kTile;
+  static constexpr int kPage = 2 * kTile;      // K tile, then V tile
+  static constexpr int kStage = KP * kPage;
   static constexpr int kKSteps = D / 16;
   static constexpr int kBoxes = D / 64;
   static constexpr int kMaxPages = 128;  // pages of the longest partition (2048 tokens)
@@ -417,20 +421,21 @@ struct RowsShape {
   static constexpr size_t kCntOff = kBarOff + size_t(NSTAGE) * 8;
   static constexpr size_t kTabOff = kCntOff + size_t(NSTAGE) * 4;
   static constexpr size_t kSmem = 1024 + kTabOff + size_t(kMaxPages) * 4;
-  static_assert(kStage % 1024 == 0, "swizzled boxes need 1024-byte alignment");
+  static_assert(kPage % 1024 == 0, "swizzled boxes need 1024-byte alignment");
 };
 
-// Resident warps per SM the register budget is sized for (6 CTAs of 3
-// warps): capping registers for 8 such CTAs measured slower.
+// Resident warps per SM the register budget is sized for: 5 CTAs of 3
+// warps (up to 128 registers a thread, no spills) measured faster than 6
+// CTAs (96 registers) or 8 (80).
 #ifndef PKV_ROWS_WARPS_PER_SM
-#define PKV_ROWS_WARPS_PER_SM 18
+#define PKV_ROWS_WARPS_PER_SM 15
 #endif
-template <typename T, int D, int G, int NW, int NSTAGE>
+template <typename T, int D, int G, int NW, int NSTAGE, int KP>
 __global__ void __launch_bounds__(NW * 32, PKV_ROWS_WARPS_PER_SM / NW)
     paged_multi_rows_kernel(const MultiArgs a, const __grid_constant__ CUtensorMap tmap_k,
                             const __grid_constant__ CUtensorMap tmap_v) {
   pdl_enter();
-  using S = RowsShape<D, NW, NSTAGE>;
+  using S = RowsShape<D, NW, NSTAGE, KP>;
   using M = Mma<T>;
   constexpr int kCols = 8 * NW;
   const int kvh = blockIdx.x;
@@ -474,6 +479,7 @@ __global__ void __launch_bounds__(NW * 32, PKV_ROWS_WARPS_PER_SM / NW)
 
   const int pg0 = tok0 / kBlockSize;
   const int nblk = (tok1 - tok0 + kBlockSize - 1) / kBlockSize;  // <= S::kMaxPages
+  const int nstep = (nblk + KP - 1) / KP;
   for (int j = threadIdx.x; j < nblk; j += NW * 32) {
     const int e = a.block_tables[static_cast<long long>(b) * a.bt_stride + pg0 + j];
     const bool in = e >= 0 && e < a.num_blocks;
@@ -489,28 +495,39 @@ __global__ void __launch_bounds__(NW * 32, PKV_ROWS_WARPS_PER_SM / NW)
   }
   __syncthreads();
 
-  // page i into stage i % NSTAGE (one lane; a page outside the pool only
-  // completes its stage's phase)
-  auto issue = [&](int i) {
-    if (i >= nblk) return;
-    const uint32_t bar = bar0 + 8 * (i % NSTAGE);
-    const int phys = table[i];
-    if (phys >= 0) {
-      const uint32_t dst = stage0 + (i % NSTAGE) * S::kStage;
-      const int y = (phys * a.num_kv_heads + kvh) * kBlockSize;
-      fence_proxy_async_smem();
-      mbar_arrive_expect_tx(bar, S::kStage);
+  // pages KP c .. KP c + KP - 1 into stage c % NSTAGE (one lane); pages past
+  // the partition or outside the pool are not copied
+  auto issue = [&](int c) {
+    if (c >= nstep) return;
+    const uint32_t bar = bar0 + 8 * (c % NSTAGE);
+    uint32_t bytes = 0;
 #pragma unroll
-      for (int bx = 0; bx < S::kBoxes; ++bx) {
-        tma_load_2d(dst + bx * 2048, &tmap_k, bx * 64, y, bar);
-        tma_load_2d(dst + S::kTile + bx * 2048, &tmap_v, bx * 64, y, bar);
-      }
-    } else {
+    for (int p = 0; p < KP; ++p) {
+      const int i = c * KP + p;
+      if (i < nblk && table[i] >= 0) bytes += S::kPage;
+    }
+    if (bytes == 0) {
       mbar_arrive(bar);
+      return;
+    }
+    fence_proxy_async_smem();
+    mbar_arrive_expect_tx(bar, bytes);
+#pragma unroll
+    for (int p = 0; p < KP; ++p) {
+      const int i = c * KP + p;
+      if (i < nblk && table[i] >= 0) {
+        const uint32_t dst = stage0 + (c % NSTAGE) * S::kStage + p * S::kPage;
+        const int y = (table[i] * a.num_kv_heads + kvh) * kBlockSize;
+#pragma unroll
+        for (int bx = 0; bx < S::kBoxes; ++bx) {
+          tma_load_2d(dst + bx * 2048, &tmap_k, bx * 64, y, bar);
+          tma_load_2d(dst + S::kTile + bx * 2048, &tmap_v, bx * 64, y, bar);
+        }
+      }
     }
   };
   if (threadIdx.x == 0)
-    for (int i = 0; i < NSTAGE; ++i) issue(i);
+    for (int c = 0; c < NSTAGE; ++c) issue(c);
 
   // this warp's column g8 (row r0 + 8 warp + g8) and its lane's columns 2 t4, 2 t4 + 1
   uint32_t qb[S::kKSteps][2];
@@ -535,23 +552,34 @@ __global__ void __launch_bounds__(NW * 32, PKV_ROWS_WARPS_PER_SM / NW)
   uint32_t phase_bits = 0;
   bool bad = false;
 
-  for (int i = 0; i < nblk; ++i) {
-    const int s = i % NSTAGE;
+  for (int c = 0; c < nstep; ++c) {
+    const int s = c % NSTAGE;
     const bool ok = __all_sync(kFull, mbar_wait_bounded(bar0 + 8 * s, (phase_bits >> s) & 1u));
     phase_bits ^= 1u << s;
-    if (!ok) {  // this warp gives up; the others time out on the pages it never releases
+    if (!ok) {  // this warp gives up; the others time out on the stages it never releases
       if (lane == 0) raise_error(PKV_ERR_TIMEOUT);
       bad = true;
       break;
     }
-    if (table[i] >= 0) {
-      const int page_tok = tok0 + i * kBlockSize;
-      const int nvalid = min(kBlockSize, tok1 - page_tok);
-      const uint32_t kt = stage0 + s * S::kStage;
-      const uint32_t vt = kt + S::kTile;
-      // two independent accumulation chains over the k-steps
+    // the step's pages: held (copied) or not, and tokens in each
+    bool held[KP];
+    int nvalid[KP];
+    bool full = true;
+#pragma unroll
+    for (int p = 0; p < KP; ++p) {
+      const int i = c * KP + p;
+      held[p] = i < nblk && table[i] >= 0;
+      nvalid[p] = held[p] ? min(kBlockSize, tok1 - tok0 - i * kBlockSize) : 0;
+      full = full && nvalid[p] == kBlockSize;
+    }
+    const uint32_t st = stage0 + s * S::kStage;
+    // S^T per page in two independent accumulation chains
+    float x[KP][4];
+#pragma unroll
+    for (int p = 0; p < KP; ++p) {
       float sc[4] = {0.f, 0.f, 0.f, 0.f}, sd[4] = {0.f, 0.f, 0.f, 0.f};
-      {
+      if (held[p]) {
+        const uint32_t kt = st + p * S::kPage;
         const int row = lr + ((lm & 1) << 3);
 #pragma unroll
         for (int ks = 0; ks < S::kKSteps; ks += 2) {
@@ -562,86 +590,115 @@ __global__ void __launch_bounds__(NW * 32, PKV_ROWS_WARPS_PER_SM / NW)
           M::run(sd, b0, b1, b2, b3, qb[ks + 1][0], qb[ks + 1][1]);
         }
       }
-      const int jA = page_tok + g8, jB = page_tok + g8 + 8;
-      const float x0 = jA <= pos0 ? (sc[0] + sd[0]) * a.qk_scale : -INFINITY;
-      const float x1 = jA <= pos1 ? (sc[1] + sd[1]) * a.qk_scale : -INFINITY;
-      const float x2 = jB <= pos0 ? (sc[2] + sd[2]) * a.qk_scale : -INFINITY;
-      const float x3 = jB <= pos1 ? (sc[3] + sd[3]) * a.qk_scale : -INFINITY;
-      float mx0 = fmaxf(x0, x2), mx1 = fmaxf(x1, x3);
-#pragma unroll
-      for (int msk = 4; msk <= 16; msk <<= 1) {
-        mx0 = fmaxf(mx0, __shfl_xor_sync(kFull, mx0, msk));
-        mx1 = fmaxf(mx1, __shfl_xor_sync(kFull, mx1, msk));
-      }
-      const float n0 = fmaxf(m0, mx0), n1 = fmaxf(m1, mx1);
-      const float u0 = n0 == -INFINITY ? 0.f : n0, u1 = n1 == -INFINITY ? 0.f : n1;
-      const float al0 = exp2_sfu(m0 - u0), al1 = exp2_sfu(m1 - u1);
-      m0 = n0;
-      m1 = n1;
-      const float p0 = exp2_sfu(x0 - u0), p1 = exp2_sfu(x1 - u1), p2 = exp2_sfu(x2 - u0), p3 = exp2_sfu(x3 - u1);
-      l0 = fmaf(l0, al0, p0 + p2);
-      l1 = fmaf(l1, al1, p1 + p3);
-      if (__any_sync(kFull, al0 != 1.f || al1 != 1.f)) {
-#pragma unroll
-        for (int mt = 0; mt < S::kKSteps; ++mt) {
-          o[mt][0] *= al0;
-          o[mt][1] *= al1;
-          o[mt][2] *= al0;
-          o[mt][3] *= al1;
-        }
-      }
-      const uint32_t top_hi = M::pack(p0, p1), bot_hi = M::pack(p2, p3);
-      const float2 th = M::unpack(top_hi), bh = M::unpack(bot_hi);
-      const uint32_t pb0 = movm_t(top_hi), pb1 = movm_t(bot_hi);
-      const uint32_t pl0 = movm_t(M::pack(p0 - th.x, p1 - th.y)), pl1 = movm_t(M::pack(p2 - bh.x, p3 - bh.y));
-      uint32_t keep_lo = 0xffffffffu, keep_hi = 0xffffffffu;
-      if (nvalid < kBlockSize) {
-        keep_lo = (2 * t4 < nvalid ? 0x0000ffffu : 0u) | (2 * t4 + 1 < nvalid ? 0xffff0000u : 0u);
-        keep_hi = (2 * t4 + 8 < nvalid ? 0x0000ffffu : 0u) | (2 * t4 + 9 < nvalid ? 0xffff0000u : 0u);
-      }
-      auto pv = [&](auto masked) {
-        const int row = lr + ((lm >> 1) << 3);
-#pragma unroll
-        for (int mt = 0; mt < S::kKSteps; ++mt) {
-          uint32_t a0, a1, a2, a3;
-          ldsm_x4_t(vt + swz(row, 2 * mt + (lm & 1)), a0, a1, a2, a3);
-          if constexpr (decltype(masked)::value) {
-            a0 &= keep_lo;
-            a1 &= keep_lo;
-            a2 &= keep_hi;
-            a3 &= keep_hi;
-          }
-          M::run(o[mt], a0, a1, a2, a3, pb0, pb1);
-          M::run(o[mt], a0, a1, a2, a3, pl0, pl1);
-        }
-      };
-      if (nvalid < kBlockSize)
-        pv(std::true_type{});
-      else
-        pv(std::false_type{});
+      // causal mask (it also cuts the partition's end and a missing page:
+      // every column's position is below tok1)
+      const int jA = tok0 + (c * KP + p) * kBlockSize + g8, jB = jA + 8;
+      const bool h = held[p];
+      x[p][0] = h && jA <= pos0 ? (sc[0] + sd[0]) * a.qk_scale : -INFINITY;
+      x[p][1] = h && jA <= pos1 ? (sc[1] + sd[1]) * a.qk_scale : -INFINITY;
+      x[p][2] = h && jB <= pos0 ? (sc[2] + sd[2]) * a.qk_scale : -INFINITY;
+      x[p][3] = h && jB <= pos1 ? (sc[3] + sd[3]) * a.qk_scale : -INFINITY;
     }
+    float mx0 = fmaxf(x[0][0], x[0][2]), mx1 = fmaxf(x[0][1], x[0][3]);
+#pragma unroll
+    for (int p = 1; p < KP; ++p) {
+      mx0 = fmaxf(mx0, fmaxf(x[p][0], x[p][2]));
+      mx1 = fmaxf(mx1, fmaxf(x[p][1], x[p][3]));
+    }
+#pragma unroll
+    for (int msk = 4; msk <= 16; msk <<= 1) {
+      mx0 = fmaxf(mx0, __shfl_xor_sync(kFull, mx0, msk));
+      mx1 = fmaxf(mx1, __shfl_xor_sync(kFull, mx1, msk));
+    }
+    const float n0 = fmaxf(m0, mx0), n1 = fmaxf(m1, mx1);
+    const float u0 = n0 == -INFINITY ? 0.f : n0, u1 = n1 == -INFINITY ? 0.f : n1;
+    const float al0 = exp2_sfu(m0 - u0), al1 = exp2_sfu(m1 - u1);
+    m0 = n0;
+    m1 = n1;
+    uint32_t pb0[KP], pb1[KP], pl0[KP], pl1[KP];
+    float sum0 = 0.f, sum1 = 0.f;
+#pragma unroll
+    for (int p = 0; p < KP; ++p) {
+      const float e0 = exp2_sfu(x[p][0] - u0), e1 = exp2_sfu(x[p][1] - u1);
+      const float e2 = exp2_sfu(x[p][2] - u0), e3 = exp2_sfu(x[p][3] - u1);
+      sum0 += e0 + e2;
+      sum1 += e1 + e3;
+      const uint32_t top_hi = M::pack(e0, e1), bot_hi = M::pack(e2, e3);
+      const float2 th = M::unpack(top_hi), bh = M::unpack(bot_hi);
+      pb0[p] = movm_t(top_hi);
+      pb1[p] = movm_t(bot_hi);
+      pl0[p] = movm_t(M::pack(e0 - th.x, e1 - th.y));
+      pl1[p] = movm_t(M::pack(e2 - bh.x, e3 - bh.y));
+    }
+    l0 = fmaf(l0, al0, sum0);
+    l1 = fmaf(l1, al1, sum1);
+    if (__any_sync(kFull, al0 != 1.f || al1 != 1.f)) {
+#pragma unroll
+      for (int mt = 0; mt < S::kKSteps; ++mt) {
+        o[mt][0] *= al0;
+        o[mt][1] *= al1;
+        o[mt][2] *= al0;
+        o[mt][3] *= al1;
+      }
+    }
+    // O^T += V^T . P^T per page; slots past a page's tokens may hold
+    // anything (NaN included), so their V is zeroed
+    auto pv = [&](auto masked) {
+      uint32_t keep_lo[KP], keep_hi[KP];
+      if constexpr (decltype(masked)::value) {
+#pragma unroll
+        for (int p = 0; p < KP; ++p) {
+          const int n = nvalid[p];
+          keep_lo[p] = (2 * t4 < n ? 0x0000ffffu : 0u) | (2 * t4 + 1 < n ? 0xffff0000u : 0u);
+          keep_hi[p] = (2 * t4 + 8 < n ? 0x0000ffffu : 0u) | (2 * t4 + 9 < n ? 0xffff0000u : 0u);
+        }
+      }
+      const int row = lr + ((lm >> 1) << 3);
+#pragma unroll
+      for (int mt = 0; mt < S::kKSteps; ++mt) {
+#pragma unroll
+        for (int p = 0; p < KP; ++p) {
+          if constexpr (decltype(masked)::value)
+            if (!held[p]) continue;
+          uint32_t a0, a1, a2, a3;
+          ldsm_x4_t(st + p * S::kPage + S::kTile + swz(row, 2 * mt + (lm & 1)), a0, a1, a2, a3);
+          if constexpr (decltype(masked)::value) {
+            a0 &= keep_lo[p];
+            a1 &= keep_lo[p];
+            a2 &= keep_hi[p];
+            a3 &= keep_hi[p];
+          }
+          M::run(o[mt], a0, a1, a2, a3, pb0[p], pb1[p]);
+          M::run(o[mt], a0, a1, a2, a3, pl0[p], pl1[p]);
+        }
+      }
+    };
+    if (full)
+      pv(std::false_type{});
+    else
+      pv(std::true_type{});
     // this warp is done with stage s; the last of the NW warps to say so
-    // refills it with the page NSTAGE ahead (the fences order every warp's
-    // reads of the stage before the copy that overwrites it)
+    // refills it with the pages NSTAGE steps ahead (the fences order every
+    // warp's reads of the stage before the copy that overwrites it)
     __syncwarp();
     if (lane == 0) {
       __threadfence_block();
       const unsigned int before = atomicAdd(&released[s], 1u);
       if (before % NW == NW - 1) {
         __threadfence_block();
-        issue(i + NSTAGE);
+        issue(c + NSTAGE);
       }
     }
   }
   // every copy this CTA issued lands before the CTA exits: after a give-up,
-  // thread 0 waits (bounded) for the last page issued into each stage
+  // thread 0 waits (bounded) for the last step issued into each stage
   if (__syncthreads_or(bad)) {
     if (threadIdx.x == 0) {
-      unsigned int issued = 0;  // pages issued: NSTAGE + the refills (one per NW releases)
+      unsigned int issued = 0;  // steps issued: NSTAGE + the refills (one per NW releases)
       for (int st = 0; st < NSTAGE; ++st) issued += released[st] / NW;
-      issued = min(static_cast<unsigned int>(nblk), issued + NSTAGE);
-      for (int i = max(0, static_cast<int>(issued) - NSTAGE); i < static_cast<int>(issued); ++i)
-        mbar_wait_bounded(bar0 + 8 * (i % NSTAGE), (i / NSTAGE) & 1u);
+      issued = min(static_cast<unsigned int>(nstep), issued + NSTAGE);
+      for (int c = max(0, static_cast<int>(issued) - NSTAGE); c < static_cast<int>(issued); ++c)
+        mbar_wait_bounded(bar0 + 8 * (c % NSTAGE), (c / NSTAGE) & 1u);
     }
     return;
   }

@@ -61,19 +61,26 @@ pkv_status launch_multi(const pkv::MultiArgs& a, const void* k_cache, const void
 // 8 rows, the warps sharing the pages (paged_multi_rows_kernel).
 int multi_ntiles(long long rows) { return rows <= 8 ? 1 : 2; }
 int multi_rows_warps(long long rows) { return rows <= 16 ? 0 : rows <= 24 ? 3 : 4; }
-constexpr int kRowsStages = 3;
+#ifndef PKV_ROWS_STAGES
+#define PKV_ROWS_STAGES 2
+#endif
+#ifndef PKV_ROWS_PAGES
+#define PKV_ROWS_PAGES 2
+#endif
+constexpr int kRowsStages = PKV_ROWS_STAGES;  // stages in the ring
+constexpr int kRowsPages = PKV_ROWS_PAGES;    // pages per stage (taken in one step)
 
 template <typename T, int D, int G, int NW>
 pkv_status launch_multi_rows(const pkv::MultiArgs& a, const void* k_cache, const void* v_cache, int num_blocks,
                              cudaStream_t st) {
-  using S = pkv::RowsShape<D, NW, kRowsStages>;
+  using S = pkv::RowsShape<D, NW, kRowsStages, kRowsPages>;
   static_assert(kMaxPartition / PKV_BLOCK_SIZE <= S::kMaxPages, "the page table of a partition fits shared memory");
   CUtensorMap mk, mv;
   const long long rows = static_cast<long long>(num_blocks) * a.num_kv_heads * PKV_BLOCK_SIZE;
   if (!encode_cache_map(&mk, k_cache, pkv::Mma<T>::kTmaType, D, rows) ||
       !encode_cache_map(&mv, v_cache, pkv::Mma<T>::kTmaType, D, rows))
     return PKV_ECUDA;
-  auto kfn = pkv::paged_multi_rows_kernel<T, D, G, NW, kRowsStages>;
+  auto kfn = pkv::paged_multi_rows_kernel<T, D, G, NW, kRowsStages, kRowsPages>;
   if (cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(S::kSmem)) !=
       cudaSuccess)
     return PKV_ECUDA;

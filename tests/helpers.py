@@ -85,9 +85,10 @@ def privatise(cache_k, cache_v, tables, context_lens, block_size=16):
     return k2, v2, t2
 
 
-def make_multi_case(ctx, nq, Hq, Hkv, D, dtype, seed):
+def make_multi_case(ctx, nq, Hq, Hkv, D, dtype, seed, v_scale=1.0):
     """Pool, tables and values for sequences of lengths ``ctx`` (the last
-    ``nq[b]`` tokens being the new ones); blocks placed by a permutation."""
+    ``nq[b]`` tokens being the new ones); blocks placed by a permutation.
+    V is drawn N(0, v_scale^2)."""
     rng = np.random.default_rng(seed)
     pages = [-(-c // 16) for c in ctx]
     nb = sum(pages) + 5
@@ -103,7 +104,7 @@ def make_multi_case(ctx, nq, Hq, Hkv, D, dtype, seed):
         tables[b, :pages[b]] = perm[used:used + pages[b]]
         used += pages[b]
         kk = rng.standard_normal((c, Hkv, D)).astype(store)
-        vv = rng.standard_normal((c, Hkv, D)).astype(store)
+        vv = (rng.standard_normal((c, Hkv, D)) * v_scale).astype(store)
         if dtype == "bf16":  # keep the upper half: exact bf16 values
             kk = (kk.view(np.uint32) >> 16).astype(np.uint16)
             vv = (vv.view(np.uint32) >> 16).astype(np.uint16)
