@@ -235,7 +235,8 @@ def run_cuda(args, rank, world, local_rank):
     n_pairs = int(st["cow_pairs"].shape[0])
     ws = cache.workspace(pkv.decode_workspace_bytes(B, Hq, D, max_ctx, args.partition))
     out = torch.empty_like(st["q"])
-    P = max(1, math.ceil(max_ctx / (args.partition or pkv.api.auto_partition(max_ctx))))
+    auto = pkv.api.auto_partition_fp8 if args.kv_fp8 else pkv.api.auto_partition
+    P = max(1, math.ceil(max_ctx / (args.partition or auto(max_ctx))))
     scale = 1.0 / math.sqrt(D)
     # a batch that shares leading blocks is decoded with the cascade (the
     # shared prefix is read once per kv-head)
@@ -568,7 +569,7 @@ def multi_line(args, r, world):
                    "num_kv_heads": wl.Hkv, "head_dim": wl.D, "block_size": 16,
                    "context_lens": {"min": int(np.min(r["lens"])), "max": int(np.max(r["lens"])),
                                     "sum": int(np.sum(r["lens"]))},
-                   "partition_tokens": args.partition or ("auto (%d)" % (1024 if int(np.max(r["lens"])) > 4096 else 512)),
+                   "partition_tokens": args.partition or ("auto (%d)" % auto_partition(int(np.max(r["lens"])), False)),
                    "partitions_max": r["P"], "seed": args.seed,
                    "parallelism": f"replicas{args.gpus}" if args.gpus > 1 else "single-gpu",
                    "l2": "inputs larger than L2 (no flush)" if r["kv"] > 126e6 else "inputs fit in L2"},
@@ -817,12 +818,21 @@ def cpu_baseline(wl, budget_s=12.0, seed=0):
                       f"{nbytes / 1e6:.1f} MB of K/V, fp64 numpy, BLAS limited to 1 thread, {secs:.1f} s"}
 
 
+def auto_partition(max_ctx: int, fp8: bool) -> int:
+    """The library's partition for partition=0 (pkv.h): 512 tokens, 1024 past
+    4096; for the FP8 decode 1024, 2048 past 16384."""
+    if fp8:
+        return 2048 if max_ctx > 16384 else 1024
+    return 1024 if max_ctx > 4096 else 512
+
+
 def config_of(wl, args, P):
     return {"workload": wl.name, "global_batch": wl.B, "num_q_heads": wl.Hq, "num_kv_heads": wl.Hkv,
             "head_dim": wl.D, "block_size": 16, "num_blocks": wl.num_blocks,
             "context_lens": {"min": int(wl.context_lens.min()), "max": int(wl.context_lens.max()),
                              "sum": int(wl.context_lens.astype(np.int64).sum())},
-            "partition_tokens": args.partition or ("auto (%d)" % (1024 if int(wl.context_lens.max()) > 4096 else 512)),
+            "partition_tokens": args.partition or ("auto (%d)" % auto_partition(int(wl.context_lens.max()),
+                                                                                getattr(args, "kv_fp8", False))),
             "partitions_max": P, "seed": args.seed,
             "cuda_graph": bool(getattr(args, "graph", False)),
             "cascade": None if not getattr(args, "_cascade", False) else

@@ -346,7 +346,11 @@ pkv_status pkv_get_error(uint32_t* flags, void* stream);
  * cache; q and out in q_dtype (fp16 or bf16);
  *   s_j = scale * k_scale * q . code(K_j),  out = v_scale * sum_j softmax(s)_j code(V_j)
  * Same arguments, layouts, workspace (pkv_decode_workspace_bytes) and errors
- * as pkv_paged_attention_decode.
+ * as pkv_paged_attention_decode, except the auto partition (partition_tokens
+ * 0): 1024 tokens, or 2048 when max_context_len > 16384 (an FP8 page is half
+ * the bytes, so a work unit covers twice the tokens for the same fixed
+ * cost).  A workspace sized by pkv_decode_workspace_bytes with partition 0
+ * is large enough for it.
  * -------------------------------------------------------------------- */
 pkv_status pkv_kv_append_fp8(const void* k_new, const void* v_new, void* k_cache, void* v_cache,
                              const int64_t* slot_mapping, int num_tokens, int num_kv_heads, int head_dim,

@@ -24,6 +24,12 @@ DEFAULT_PARTITION = 512
 def auto_partition(max_context_len: int) -> int:
     """The library's partition for partition=0: 512 tokens, 1024 past 4096."""
     return 2 * DEFAULT_PARTITION if max_context_len > 4096 else DEFAULT_PARTITION
+
+
+def auto_partition_fp8(max_context_len: int) -> int:
+    """The FP8 decode's partition for partition=0: 1024 tokens, 2048 past
+    16384 (its pages are half the bytes)."""
+    return 4 * DEFAULT_PARTITION if max_context_len > 16384 else 2 * DEFAULT_PARTITION
 # a batch whose sequences share at least this many leading pages (and has at
 # least this many sequences) is decoded with the cascade (prefix read once)
 CASCADE_MIN_PAGES = 8

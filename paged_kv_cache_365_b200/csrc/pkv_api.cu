@@ -647,6 +647,8 @@ pkv_status pkv_paged_attention_decode_fp8(void* out, const void* q, const void* 
     return PKV_EINVAL;
   pkv::DecodeArgs a{};
   long long P = 0;
+  // auto partition: twice the 16-bit one's tokens (half the bytes a page)
+  if (partition_tokens == 0) partition_tokens = max_context_len > 16384 ? 2048 : 1024;
   const pkv_status st0 = prepare_decode(out, q, k_cache, v_cache, block_tables, max_blocks_per_seq, context_lens,
                                         max_context_len, num_seqs, num_q_heads, num_kv_heads, head_dim, num_blocks,
                                         scale, partition_tokens, q_dtype, &a, &P);

@@ -36,3 +36,18 @@ def test_warmup_floor():
     out = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--warmup", "2"], capture_output=True,
                          text=True, timeout=120, cwd=ROOT)
     assert out.returncode != 0 and "warmup" in out.stderr
+
+
+def test_bench_reports_the_library_auto_partitions():
+    """bench.py names the partition the library picks for partition=0 (its
+    own copy of the rule, so the reference arm needs no CUDA library)."""
+    import bench
+    import paged_kv_cache_365_b200 as pkv
+    for n in (1, 512, 4096, 4097, 16384, 16385, 131072):
+        assert bench.auto_partition(n, False) == pkv.api.auto_partition(n)
+        assert bench.auto_partition(n, True) == pkv.api.auto_partition_fp8(n)
+    # the 16-bit rule is also the one the workspace size follows
+    B, Hq, D = 3, 8, 128
+    for n in (700, 5000):
+        P = -(-n // pkv.api.auto_partition(n))
+        assert pkv.decode_workspace_bytes(B, Hq, D, n, 0) == B * Hq * P * (D + 2) * 4

@@ -96,6 +96,7 @@ CASES = [
     ([33, 700, 1100], 8, 2, 128, "bf16"),
     ([5, 48, 300, 2049], 8, 1, 64, "f16"),
     ([64, 129, 513], 16, 4, 64, "bf16"),
+    ([17000, 300, 2100], 8, 1, 128, "bf16"),  # auto partition: 2048 tokens past 16384
 ]
 
 
