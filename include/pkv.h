@@ -323,6 +323,16 @@ pkv_status pkv_paged_attention_decode_static_ws(void* out, const void* q, const 
  * work queued on `stream` so far has finished.  Blocks the host. */
 pkv_status pkv_get_error(uint32_t* flags, void* stream);
 
+/* Test hook for the kernels' failure path.  Every wait of a kernel on its
+ * staged copies (an mbarrier the TMA completes) is bounded: after 2^32 SM
+ * clock cycles (about 2 s) the kernel sets PKV_ERR_TIMEOUT, drains what it
+ * issued with bounded waits and returns, leaving the context usable.  This
+ * call runs that same wait, with limit_cycles in [1, 2^32] as its bound, on
+ * a barrier that nothing completes (one warp, one CTA, async on `stream`):
+ * pkv_get_error then reports PKV_ERR_TIMEOUT.  PKV_EINVAL for a limit out of
+ * range. */
+pkv_status pkv_selftest_bounded_wait(long long limit_cycles, void* stream);
+
 /* ------------------------------------------------------------------------
  * FP8 KV cache: half the bytes of a 16-bit cache per token.
  *

@@ -53,6 +53,7 @@ PROTOTYPES = {
     "pkv_paged_attention_decode_static_ws": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_int,
                                                      c_void_p, c_int, c_int, c_int, c_int, c_int, c_int,
                                                      c_float, c_int, c_int, c_void_p]),
+    "pkv_selftest_bounded_wait": (c_int, [ctypes.c_longlong, c_void_p]),
     "pkv_kv_append_fp8": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_int, c_int, c_int, c_int,
                                   c_int, c_float, c_float, c_void_p]),
     "pkv_paged_attention_decode_fp8": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_int, c_void_p,

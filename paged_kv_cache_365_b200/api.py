@@ -7,12 +7,35 @@ provides device memory and streams.
 """
 from __future__ import annotations
 
+import contextlib
 import ctypes
+import functools
 import math
 from typing import Iterable, List, Optional, Sequence, Tuple
 
 import numpy as np
 import torch
+
+
+@contextlib.contextmanager
+def nvtx_range(name: str):
+    """An NVTX range around host code (shows in Nsight timelines; a no-op
+    without a profiler attached)."""
+    torch.cuda.nvtx.range_push(name)
+    try:
+        yield
+    finally:
+        torch.cuda.nvtx.range_pop()
+
+
+def _traced(name: str):
+    def wrap(fn):
+        @functools.wraps(fn)
+        def inner(*a, **kw):
+            with nvtx_range(name):
+                return fn(*a, **kw)
+        return inner
+    return wrap
 
 from . import _lib
 from ._lib import check, lib
@@ -386,6 +409,13 @@ def get_error(stream=None, device=None) -> int:
     return int(v.value)
 
 
+def selftest_bounded_wait(limit_cycles: int, stream=None, device=None) -> None:
+    """Run the kernels' bounded staged-copy wait on a barrier nothing
+    completes (pkv_selftest_bounded_wait); get_error() then shows
+    ERR_TIMEOUT."""
+    check(lib.pkv_selftest_bounded_wait(int(limit_cycles), _stream(stream, device)), "pkv_selftest_bounded_wait")
+
+
 # ---------------------------------------------------------------------------
 # host allocator
 # ---------------------------------------------------------------------------
@@ -681,6 +711,7 @@ class PagedKVCache:
         self.host_v = torch.empty(shape, dtype=self.k.dtype, pin_memory=True)
         self.alloc.set_host_pool(num_host_blocks)
 
+    @_traced("pkv.swap_out")
     def swap_out(self, seq_ids: Sequence[int], stream=None) -> np.ndarray:
         """Preempt sequences: their blocks go to the host pool (copied on the
         stream before anything later on it can reuse the released blocks)."""
@@ -690,6 +721,7 @@ class PagedKVCache:
                         torch.from_numpy(np.ascontiguousarray(pairs)).to(self.device), stream, self.device)
         return pairs
 
+    @_traced("pkv.swap_in")
     def swap_in(self, seq_ids: Sequence[int], stream=None) -> np.ndarray:
         """Bring preempted sequences back into the device pool."""
         pairs = self.alloc.swap_in(seq_ids)
@@ -706,6 +738,7 @@ class PagedKVCache:
         self._append(k.to(self.device), v.to(self.device), torch.from_numpy(slots).to(self.device), stream)
         return slots
 
+    @_traced("pkv.plan_step")
     def plan_step(self, seq_ids: Sequence[int], width: Optional[int] = None):
         """Host part of a decode step: slots, CoW pairs, tables, lengths."""
         slots, pairs = self.alloc.step(seq_ids)
@@ -715,6 +748,7 @@ class PagedKVCache:
         tables, lens = self.alloc.block_tables(seq_ids, width, self.num_blocks)
         return slots, pairs, tables, lens
 
+    @_traced("pkv.run_step")
     def run_step(self, slot_mapping: torch.Tensor, cow_pairs: torch.Tensor, block_tables: torch.Tensor,
                  context_lens: torch.Tensor, max_context_len: int, q: torch.Tensor, k_new: torch.Tensor,
                  v_new: torch.Tensor, out: Optional[torch.Tensor] = None, scale: Optional[float] = None,
@@ -785,6 +819,7 @@ class PagedKVCache:
             st = torch.cuda.current_stream(self.device) if stream is None else stream
             st.wait_stream(stg.d2h)
 
+    @_traced("pkv.plan_multi_step")
     def plan_multi_step(self, seq_ids: Sequence[int], n_new: Sequence[int], width: Optional[int] = None):
         """Host part of a multi-token step: append n_new[i] tokens to each
         sequence (in order); returns slots [sum n], CoW pairs [k, 2],
@@ -805,6 +840,7 @@ class PagedKVCache:
         tables, lens = self.alloc.block_tables(seq_ids, width, self.num_blocks)
         return slots, pairs, qs, tables, lens
 
+    @_traced("pkv.run_multi_step")
     def run_multi_step(self, slot_mapping: torch.Tensor, cow_pairs: torch.Tensor, block_tables: torch.Tensor,
                        context_lens: torch.Tensor, max_context_len: int, query_start: torch.Tensor,
                        max_query_len: int, q: torch.Tensor, k_new: torch.Tensor, v_new: torch.Tensor,
@@ -832,6 +868,7 @@ class PagedKVCache:
         stg.finish(st, res, out)
         return res
 
+    @_traced("pkv.step")
     def step(self, seq_ids: Sequence[int], q: torch.Tensor, k_new: torch.Tensor, v_new: torch.Tensor,
              scale: Optional[float] = None, partition: int = 0, stream=None) -> torch.Tensor:
         """Host plan (allocator) + device step; returns the output on q's device."""

@@ -18,6 +18,20 @@ namespace pkv {
 __device__ unsigned int g_error_snapshot = 0u;
 
 __global__ void take_error_snapshot_kernel() { g_error_snapshot = atomicExch(&g_error_word, 0u); }
+
+// The staged-copy wait of every kernel, on a barrier that nothing completes:
+// it must give up after `limit` cycles and flag PKV_ERR_TIMEOUT.
+__global__ void bounded_wait_selftest_kernel(long long limit) {
+  __shared__ alignas(8) unsigned long long bar;
+  const uint32_t b = smem_addr(&bar);
+  if (threadIdx.x == 0) {
+    mbar_init(b, 1);
+    fence_barrier_init();
+  }
+  __syncwarp();
+  const bool done = __all_sync(kFull, mbar_wait_bounded(b, 0u, limit));
+  if (!done && threadIdx.x == 0) raise_error(PKV_ERR_TIMEOUT);
+}
 }  // namespace pkv
 
 namespace {
@@ -521,6 +535,12 @@ pkv_status pkv_paged_attention_decode_static_ws(void* out, const void* q, const 
   return pkv_paged_attention_decode(out, q, k_cache, v_cache, block_tables, max_blocks_per_seq, context_lens,
                                     max_context_len, num_seqs, num_q_heads, num_kv_heads, head_dim, num_blocks,
                                     scale, partition_tokens, dtype, ws, PKV_STATIC_WORKSPACE_BYTES, stream);
+}
+
+pkv_status pkv_selftest_bounded_wait(long long limit_cycles, void* stream) {
+  if (limit_cycles <= 0 || limit_cycles > (1ll << 32)) return PKV_EINVAL;
+  pkv::bounded_wait_selftest_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(limit_cycles);
+  return cudaGetLastError() == cudaSuccess ? PKV_OK : PKV_ECUDA;
 }
 
 pkv_status pkv_get_error(uint32_t* flags, void* stream) {

@@ -210,3 +210,8 @@ def test_cow_copy_rows():
     from paged_kv_cache_365_b200 import cow_copy_rows
     rows = cow_copy_rows(np.array([[3, 7], [4, 9], [5, 11]]), np.array([7 * 16 + 5, 9 * 16 + 15, -1, 9 * 16 + 3]))
     assert rows.tolist() == [[3, 7, 5], [4, 9, 3], [5, 11, 16]]
+
+
+def test_selftest_bounded_wait_rejects_limits(lib):
+    for bad in (0, -5, (1 << 32) + 1):
+        assert lib.pkv_selftest_bounded_wait(bad, None) == 1, bad
