@@ -448,7 +448,7 @@ def run_multi(args, rank, world, local_rank):
     out = torch.empty_like(st["q"])
     scale = 1.0 / math.sqrt(wl.D)
     n_pairs = int(st["cow_pairs"].shape[0])
-    P = max(1, math.ceil(max_ctx / (args.partition or pkv.api.auto_partition(max_ctx))))
+    P = max(1, math.ceil(max_ctx / (args.partition or pkv.api.auto_partition_multi(max_ctx))))
 
     def pre():
         if n_pairs:
@@ -569,7 +569,7 @@ def multi_line(args, r, world):
                    "num_kv_heads": wl.Hkv, "head_dim": wl.D, "block_size": 16,
                    "context_lens": {"min": int(np.min(r["lens"])), "max": int(np.max(r["lens"])),
                                     "sum": int(np.sum(r["lens"]))},
-                   "partition_tokens": args.partition or ("auto (%d)" % auto_partition(int(np.max(r["lens"])), False)),
+                   "partition_tokens": args.partition or ("auto (%d)" % auto_partition(int(np.max(r["lens"])), False, True)),
                    "partitions_max": r["P"], "seed": args.seed,
                    "parallelism": f"replicas{args.gpus}" if args.gpus > 1 else "single-gpu",
                    "l2": "inputs larger than L2 (no flush)" if r["kv"] > 126e6 else "inputs fit in L2"},
@@ -818,11 +818,14 @@ def cpu_baseline(wl, budget_s=12.0, seed=0):
                       f"{nbytes / 1e6:.1f} MB of K/V, fp64 numpy, BLAS limited to 1 thread, {secs:.1f} s"}
 
 
-def auto_partition(max_ctx: int, fp8: bool) -> int:
+def auto_partition(max_ctx: int, fp8: bool, multi: bool = False) -> int:
     """The library's partition for partition=0 (pkv.h): 512 tokens, 1024 past
-    4096; for the FP8 decode 1024, 2048 past 16384."""
+    4096; for the FP8 decode 1024, 2048 past 16384; for the multi-token path
+    2048, 1024 past 4096."""
     if fp8:
         return 2048 if max_ctx > 16384 else 1024
+    if multi:
+        return 1024 if max_ctx > 4096 else 2048
     return 1024 if max_ctx > 4096 else 512
 
 

@@ -397,7 +397,11 @@ pkv_status pkv_paged_attention_decode_fp8(void* out, const void* q, const void* 
  * this is skipped, its rows left unwritten, and PKV_ERR_CONTEXT_RANGE set).
  * fp16 / bf16 only (tensor cores).  num_seqs * ceil(max_query_len * G / 16)
  * <= 65535.  workspace: pkv_multi_workspace_bytes(...) bytes (0 when
- * max_context_len <= partition), 16-byte aligned.
+ * max_context_len <= partition), 16-byte aligned.  partition_tokens as in
+ * pkv_paged_attention_decode, except the auto partition (0): 2048 tokens,
+ * or 1024 when max_context_len > 4096 (several rows a sequence make every
+ * partial n_b times the merge work, so short contexts stay unsplit; long
+ * ones are split for balance across the SMs).
  * -------------------------------------------------------------------- */
 size_t pkv_multi_workspace_bytes(int total_query_tokens, int num_q_heads, int head_dim, int max_context_len,
                                  int partition_tokens);

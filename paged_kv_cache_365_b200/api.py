@@ -49,6 +49,12 @@ def auto_partition(max_context_len: int) -> int:
     return 2 * DEFAULT_PARTITION if max_context_len > 4096 else DEFAULT_PARTITION
 
 
+def auto_partition_multi(max_context_len: int) -> int:
+    """The multi-token path's partition for partition=0: 2048 tokens, 1024
+    past 4096."""
+    return 2 * DEFAULT_PARTITION if max_context_len > 4096 else 4 * DEFAULT_PARTITION
+
+
 def auto_partition_fp8(max_context_len: int) -> int:
     """The FP8 decode's partition for partition=0: 1024 tokens, 2048 past
     16384 (its pages are half the bytes)."""

@@ -73,6 +73,10 @@ pkv_status launch_multi(const pkv::MultiArgs& a, const void* k_cache, const void
 // Up to 16 rows per sequence (max_query_len * G): one tile of 8 NT rows,
 // the warps splitting the pages.  More: tiles of 8 NW rows, one warp per
 // 8 rows, the warps sharing the pages (paged_multi_rows_kernel).
+// Auto partition of the multi-token path: 2048 tokens, 1024 past 4096.
+int resolve_multi_partition(int p, long long max_ctx) {
+  return resolve_partition(p != 0 ? p : (max_ctx > 4096 ? 1024 : 2048), max_ctx);
+}
 int multi_ntiles(long long rows) { return rows <= 8 ? 1 : 2; }
 int multi_rows_warps(long long rows) { return rows <= 16 ? 0 : rows <= 24 ? 3 : 4; }
 #ifndef PKV_ROWS_STAGES
@@ -559,7 +563,7 @@ pkv_status pkv_get_error(uint32_t* flags, void* stream) {
 
 size_t pkv_multi_workspace_bytes(int total_query_tokens, int num_q_heads, int head_dim, int max_context_len,
                                  int partition_tokens) {
-  const int part = resolve_partition(partition_tokens, max_context_len);
+  const int part = resolve_multi_partition(partition_tokens, max_context_len);
   if (part < 0 || total_query_tokens < 0 || num_q_heads <= 0 || !head_dim_ok(head_dim) || max_context_len < 0)
     return 0;
   const long long P = (static_cast<long long>(max_context_len) + part - 1) / part;
@@ -574,7 +578,7 @@ pkv_status pkv_paged_attention_multi(void* out, const void* q, const void* k_cac
                                      float scale, int partition_tokens, pkv_dtype dtype, void* workspace,
                                      size_t workspace_bytes_given, void* stream) {
   if (dtype != PKV_F16 && dtype != PKV_BF16) return PKV_EINVAL;  // tensor-core path only
-  const int part = resolve_partition(partition_tokens, max_context_len);
+  const int part = resolve_multi_partition(partition_tokens, max_context_len);
   if (part < 0 || num_seqs < 0 || num_kv_heads <= 0 || num_kv_heads > 65535 || num_q_heads <= 0 ||
       num_q_heads % num_kv_heads != 0 || !group_ok(num_q_heads / num_kv_heads) || !head_dim_ok(head_dim) ||
       num_blocks <= 0 || max_context_len < 0 || max_blocks_per_seq <= 0 || max_query_len < 0 ||

@@ -155,11 +155,16 @@ def test_prefix_workspace_and_rejections(lib):
 
 def test_multi_workspace_and_rejections(lib):
     # one partition: nothing; else T*Hq*P*D*4 (rounded to 16) + T*Hq*P*8
-    assert lib.pkv_multi_workspace_bytes(10, 8, 128, 512, 0) == 0
+    assert lib.pkv_multi_workspace_bytes(10, 8, 128, 512, 512) == 0
     o = 10 * 8 * 3 * 128 * 4
-    assert lib.pkv_multi_workspace_bytes(10, 8, 128, 1100, 0) == (o + 15) // 16 * 16 + 10 * 8 * 3 * 8
-    assert lib.pkv_multi_workspace_bytes(10, 8, 96, 1100, 0) == 0
-    args = [FAKE, FAKE, FAKE, FAKE, FAKE, 100, FAKE, 1100, FAKE, 8, 40, 4, 8, 2, 128, 64, ctypes.c_float(0.1), 0,
+    assert lib.pkv_multi_workspace_bytes(10, 8, 128, 1100, 512) == (o + 15) // 16 * 16 + 10 * 8 * 3 * 8
+    assert lib.pkv_multi_workspace_bytes(10, 8, 96, 1100, 512) == 0
+    # auto partition: 2048 tokens (one partition here), 1024 past 4096 tokens
+    assert lib.pkv_multi_workspace_bytes(10, 8, 128, 2048, 0) == 0
+    o = 10 * 8 * 5 * 128 * 4
+    assert lib.pkv_multi_workspace_bytes(10, 8, 128, 5000, 0) == (o + 15) // 16 * 16 + 10 * 8 * 5 * 8
+    # 512-token partitions: 1100 tokens split, so the workspace is checked
+    args = [FAKE, FAKE, FAKE, FAKE, FAKE, 100, FAKE, 1100, FAKE, 8, 40, 4, 8, 2, 128, 64, ctypes.c_float(0.1), 512,
             1, FAKE, 1 << 30, None]
     for idx, bad in ((18, 0), (18, 3), (14, 96), (12, 6), (9, -1), (10, -1), (8, None), (19, None), (20, 16),
                      (7, 100 * 16 + 1), (16, ctypes.c_float(float("inf")))):

@@ -46,8 +46,14 @@ def test_bench_reports_the_library_auto_partitions():
     for n in (1, 512, 4096, 4097, 16384, 16385, 131072):
         assert bench.auto_partition(n, False) == pkv.api.auto_partition(n)
         assert bench.auto_partition(n, True) == pkv.api.auto_partition_fp8(n)
+        assert bench.auto_partition(n, False, True) == pkv.api.auto_partition_multi(n)
     # the 16-bit rule is also the one the workspace size follows
     B, Hq, D = 3, 8, 128
-    for n in (700, 5000):
+    for n in (700, 3000, 5000, 9000):
         P = -(-n // pkv.api.auto_partition(n))
         assert pkv.decode_workspace_bytes(B, Hq, D, n, 0) == B * Hq * P * (D + 2) * 4
+        # the multi-token path's workspace follows its own rule (T query rows)
+        T = 7
+        Pm = -(-n // pkv.api.auto_partition_multi(n))
+        want = 0 if Pm <= 1 else -(-(T * Hq * Pm * D * 4) // 16) * 16 + T * Hq * Pm * 8
+        assert pkv.multi_workspace_bytes(T, Hq, D, n, 0) == want
