@@ -743,6 +743,354 @@ __global__ void __launch_bounds__(NW * 32, PKV_ROWS_WARPS_PER_SM / NW)
   }
 }
 
+// Many rows per sequence (prefill chunks, long verification runs): the
+// rows are the MMA's M dimension, as in FlashAttention-2.  One CTA of NWF
+// warps per (kv-head, sequence, tile of 16 NWF rows, key partition); warp w
+// owns rows r0 + 16 w .. r0 + 16 w + 15 and keeps their queries in
+// registers as A fragments.  Pages come through the same CTA-wide ring as
+// in paged_multi_rows_kernel (KP pages per stage, release counters).  Per
+// page and warp:
+//   S[16 rows x 16 tokens] = Q . K^T   (B = K rows via ldmatrix)
+//   causal mask per row, online softmax per row (a quad of lanes holds a
+//   row's 16 scores)
+//   O[16 x D] += P . V                 (A = P from S's own registers, in
+//                                       hi + lo 16-bit parts; B = V via
+//                                       ldmatrix.trans)
+// A warp skips the arithmetic of pages past its rows' last position.
+// Against the row-split kernel a page's fragments serve 16 rows of a warp
+// instead of 8 and need no transposes, so the work per row is about a
+// quarter.
+#ifndef PKV_FA_MIN_CTAS
+#define PKV_FA_MIN_CTAS 3
+#endif
+template <typename T, int D, int G, int NWF, int NSTAGE, int KP>
+__global__ void __launch_bounds__(NWF * 32, PKV_FA_MIN_CTAS)
+    paged_multi_fa_kernel(const MultiArgs a, const __grid_constant__ CUtensorMap tmap_k,
+                          const __grid_constant__ CUtensorMap tmap_v) {
+  pdl_enter();
+  using S = RowsShape<D, NWF, NSTAGE, KP>;
+  using M = Mma<T>;
+  constexpr int kRows = 16 * NWF;
+  constexpr int kNT = D / 8;  // n-tiles of O
+  const int kvh = blockIdx.x;
+  const int b = blockIdx.y / a.tiles;
+  const int tile = blockIdx.y % a.tiles;
+  const int z = blockIdx.z;
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int g8 = lane >> 2, t4 = lane & 3, lm = lane >> 3, lr = lane & 7;
+
+  int ctx, q0, nq;
+  if (!multi_seq(a, b, ctx, q0, nq, threadIdx.x == 0 && kvh == 0 && tile == 0 && z == 0)) return;
+  const int R = nq * G;
+  const int r0 = tile * kRows;
+  if (r0 >= R) return;
+  const int base = ctx - nq;
+  const int p_hi = base + (min(R, r0 + kRows) - 1) / G;
+  const bool direct = ctx <= a.partition;
+  const int tok0 = z * a.partition;
+  const int tok1 = min(min(ctx, tok0 + a.partition), p_hi + 1);
+  auto out_row = [&](int tr) -> size_t {
+    return static_cast<size_t>(q0 + tr / G) * a.num_q_heads + kvh * G + tr % G;
+  };
+  if (tok1 <= tok0) {
+    if (direct && z == 0)
+      for (int idx = threadIdx.x; idx < kRows * D; idx += NWF * 32) {
+        const int tr = r0 + idx / D;
+        if (tr < R) reinterpret_cast<T*>(a.out)[out_row(tr) * D + idx % D] = Fmt<T>::from_f32(0.f);
+      }
+    return;
+  }
+
+  extern __shared__ unsigned char smem_raw[];
+  const uint32_t raw_addr = smem_addr(smem_raw);
+  const uint32_t pad = ((raw_addr + 1023u) & ~1023u) - raw_addr;
+  unsigned char* smem = smem_raw + pad;
+  const uint32_t stage0 = smem_addr(smem);
+  const uint32_t bar0 = smem_addr(smem + S::kBarOff);
+  unsigned int* released = reinterpret_cast<unsigned int*>(smem + S::kCntOff);  // warps done, per stage
+  int* table = reinterpret_cast<int*>(smem + S::kTabOff);                       // physical page i, or -1
+
+  const int pg0 = tok0 / kBlockSize;
+  const int nblk = (tok1 - tok0 + kBlockSize - 1) / kBlockSize;  // <= S::kMaxPages
+  const int nstep = (nblk + KP - 1) / KP;
+  for (int j = threadIdx.x; j < nblk; j += NWF * 32) {
+    const int e = a.block_tables[static_cast<long long>(b) * a.bt_stride + pg0 + j];
+    const bool in = e >= 0 && e < a.num_blocks;
+    if (!in) raise_error(PKV_ERR_BLOCK_RANGE);
+    table[j] = in ? e : -1;
+  }
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < NSTAGE; ++s) {
+      mbar_init(bar0 + 8 * s, 1);
+      released[s] = 0u;
+    }
+    fence_barrier_init();
+  }
+  __syncthreads();
+
+  auto issue = [&](int c) {  // pages KP c .. KP c + KP - 1 into stage c % NSTAGE (one lane)
+    if (c >= nstep) return;
+    const uint32_t bar = bar0 + 8 * (c % NSTAGE);
+    uint32_t bytes = 0;
+#pragma unroll
+    for (int p = 0; p < KP; ++p) {
+      const int i = c * KP + p;
+      if (i < nblk && table[i] >= 0) bytes += S::kPage;
+    }
+    if (bytes == 0) {
+      mbar_arrive(bar);
+      return;
+    }
+    fence_proxy_async_smem();
+    mbar_arrive_expect_tx(bar, bytes);
+#pragma unroll
+    for (int p = 0; p < KP; ++p) {
+      const int i = c * KP + p;
+      if (i < nblk && table[i] >= 0) {
+        const uint32_t dst = stage0 + (c % NSTAGE) * S::kStage + p * S::kPage;
+        const int y = (table[i] * a.num_kv_heads + kvh) * kBlockSize;
+#pragma unroll
+        for (int bx = 0; bx < S::kBoxes; ++bx) {
+          tma_load_2d(dst + bx * 2048, &tmap_k, bx * 64, y, bar);
+          tma_load_2d(dst + S::kTile + bx * 2048, &tmap_v, bx * 64, y, bar);
+        }
+      }
+    }
+  };
+  if (threadIdx.x == 0)
+    for (int c = 0; c < NSTAGE; ++c) issue(c);
+
+  // this warp's rows: fragment rows g8 (row A) and g8 + 8 (row B)
+  const int wr0 = r0 + 16 * warp;
+  const int trA = wr0 + g8, trB = wr0 + g8 + 8;
+  const bool okA = trA < R, okB = trB < R;
+  const int posA = okA ? base + trA / G : -1, posB = okB ? base + trB / G : -1;
+  const int wpos = wr0 < R ? base + (min(R, wr0 + 16) - 1) / G : -1;  // the warp's last position
+  uint32_t qa[S::kKSteps][4];
+  {
+    const T* qA = reinterpret_cast<const T*>(a.q) + (okA ? out_row(trA) : 0) * D;
+    const T* qB = reinterpret_cast<const T*>(a.q) + (okB ? out_row(trB) : 0) * D;
+#pragma unroll
+    for (int ks = 0; ks < S::kKSteps; ++ks) {
+      qa[ks][0] = okA ? *reinterpret_cast<const uint32_t*>(qA + ks * 16 + 2 * t4) : 0u;
+      qa[ks][1] = okB ? *reinterpret_cast<const uint32_t*>(qB + ks * 16 + 2 * t4) : 0u;
+      qa[ks][2] = okA ? *reinterpret_cast<const uint32_t*>(qA + ks * 16 + 8 + 2 * t4) : 0u;
+      qa[ks][3] = okB ? *reinterpret_cast<const uint32_t*>(qB + ks * 16 + 8 + 2 * t4) : 0u;
+    }
+  }
+  float o[kNT][4];
+#pragma unroll
+  for (int j = 0; j < kNT; ++j) o[j][0] = o[j][1] = o[j][2] = o[j][3] = 0.f;
+  float mA = -INFINITY, mB = -INFINITY, lA = 0.f, lB = 0.f;  // lA, lB: this lane's part of the row sums
+  uint32_t phase_bits = 0;
+  bool bad = false;
+
+  for (int c = 0; c < nstep; ++c) {
+    const int s = c % NSTAGE;
+    const bool ok = __all_sync(kFull, mbar_wait_bounded(bar0 + 8 * s, (phase_bits >> s) & 1u));
+    phase_bits ^= 1u << s;
+    if (!ok) {  // this warp gives up; the others time out on the stages it never releases
+      if (lane == 0) raise_error(PKV_ERR_TIMEOUT);
+      bad = true;
+      break;
+    }
+    bool run[KP];
+    int nvalid[KP], page_tok[KP];
+    bool any = false, full = true;
+#pragma unroll
+    for (int p = 0; p < KP; ++p) {
+      const int i = c * KP + p;
+      page_tok[p] = tok0 + i * kBlockSize;
+      run[p] = i < nblk && table[i] >= 0 && page_tok[p] <= wpos;
+      nvalid[p] = run[p] ? min(kBlockSize, tok1 - page_tok[p]) : 0;
+      any = any || run[p];
+      full = full && nvalid[p] == kBlockSize;
+    }
+    if (any) {
+      const uint32_t st = stage0 + s * S::kStage;
+      // S per page: n-tile 0 = tokens 0-7, n-tile 1 = tokens 8-15; two
+      // accumulation chains (even and odd k-steps) each
+      float x[KP][2][4];
+#pragma unroll
+      for (int p = 0; p < KP; ++p) {
+        float sa[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+        float sb[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+        if (run[p]) {
+          const uint32_t kt = st + p * S::kPage;
+          const int row = lr + ((lm >> 1) << 3);
+#pragma unroll
+          for (int ks = 0; ks < S::kKSteps; ks += 2) {
+            uint32_t k0, k1, k2, k3, u0, u1, u2, u3;
+            ldsm_x4(kt + swz(row, 2 * ks + (lm & 1)), k0, k1, k2, k3);
+            ldsm_x4(kt + swz(row, 2 * ks + 2 + (lm & 1)), u0, u1, u2, u3);
+            M::run(sa[0], qa[ks][0], qa[ks][1], qa[ks][2], qa[ks][3], k0, k1);
+            M::run(sa[1], qa[ks][0], qa[ks][1], qa[ks][2], qa[ks][3], k2, k3);
+            M::run(sb[0], qa[ks + 1][0], qa[ks + 1][1], qa[ks + 1][2], qa[ks + 1][3], u0, u1);
+            M::run(sb[1], qa[ks + 1][0], qa[ks + 1][1], qa[ks + 1][2], qa[ks + 1][3], u2, u3);
+          }
+        }
+        // causal mask (it also cuts the partition's end and a skipped page:
+        // every row's position is below tok1)
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt) {
+          const int j = page_tok[p] + nt * 8 + 2 * t4;
+          const bool h = run[p];
+          x[p][nt][0] = h && j <= posA ? (sa[nt][0] + sb[nt][0]) * a.qk_scale : -INFINITY;
+          x[p][nt][1] = h && j + 1 <= posA ? (sa[nt][1] + sb[nt][1]) * a.qk_scale : -INFINITY;
+          x[p][nt][2] = h && j <= posB ? (sa[nt][2] + sb[nt][2]) * a.qk_scale : -INFINITY;
+          x[p][nt][3] = h && j + 1 <= posB ? (sa[nt][3] + sb[nt][3]) * a.qk_scale : -INFINITY;
+        }
+      }
+      float mxA = -INFINITY, mxB = -INFINITY;
+#pragma unroll
+      for (int p = 0; p < KP; ++p)
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt) {
+          mxA = fmaxf(mxA, fmaxf(x[p][nt][0], x[p][nt][1]));
+          mxB = fmaxf(mxB, fmaxf(x[p][nt][2], x[p][nt][3]));
+        }
+#pragma unroll
+      for (int msk = 1; msk <= 2; msk <<= 1) {
+        mxA = fmaxf(mxA, __shfl_xor_sync(kFull, mxA, msk));
+        mxB = fmaxf(mxB, __shfl_xor_sync(kFull, mxB, msk));
+      }
+      const float nA = fmaxf(mA, mxA), nB = fmaxf(mB, mxB);
+      const float uA = nA == -INFINITY ? 0.f : nA, uB = nB == -INFINITY ? 0.f : nB;
+      const float alA = exp2_sfu(mA - uA), alB = exp2_sfu(mB - uB);
+      mA = nA;
+      mB = nB;
+      // P as A fragments (rows A / B, tokens 2 t4.. of each n-tile), hi + lo
+      uint32_t ph[KP][4], pl[KP][4];
+      float sumA = 0.f, sumB = 0.f;
+#pragma unroll
+      for (int p = 0; p < KP; ++p) {
+        float e[2][4];
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt) {
+          e[nt][0] = exp2_sfu(x[p][nt][0] - uA);
+          e[nt][1] = exp2_sfu(x[p][nt][1] - uA);
+          e[nt][2] = exp2_sfu(x[p][nt][2] - uB);
+          e[nt][3] = exp2_sfu(x[p][nt][3] - uB);
+          sumA += e[nt][0] + e[nt][1];
+          sumB += e[nt][2] + e[nt][3];
+        }
+        // a0 = (row A, tokens 2t, 2t+1), a1 = (row B, same), a2 / a3 = tokens + 8
+        const float v[4][2] = {{e[0][0], e[0][1]}, {e[0][2], e[0][3]}, {e[1][0], e[1][1]}, {e[1][2], e[1][3]}};
+#pragma unroll
+        for (int r = 0; r < 4; ++r) {
+          ph[p][r] = M::pack(v[r][0], v[r][1]);
+          const float2 hv = M::unpack(ph[p][r]);
+          pl[p][r] = M::pack(v[r][0] - hv.x, v[r][1] - hv.y);
+        }
+      }
+      lA = fmaf(lA, alA, sumA);
+      lB = fmaf(lB, alB, sumB);
+      if (__any_sync(kFull, alA != 1.f || alB != 1.f)) {
+#pragma unroll
+        for (int j = 0; j < kNT; ++j) {
+          o[j][0] *= alA;
+          o[j][1] *= alA;
+          o[j][2] *= alB;
+          o[j][3] *= alB;
+        }
+      }
+      // O += P . V per page; slots past a page's tokens may hold anything
+      // (NaN included), so their V is zeroed on a partial page
+      auto pv = [&](auto masked) {
+        const int row = lr + ((lm & 1) << 3);
+#pragma unroll
+        for (int p = 0; p < KP; ++p) {
+          if constexpr (decltype(masked)::value)
+            if (!run[p]) continue;
+          uint32_t klo = 0xffffffffu, khi = 0xffffffffu;
+          if constexpr (decltype(masked)::value) {
+            const int n = nvalid[p];
+            klo = (2 * t4 < n ? 0x0000ffffu : 0u) | (2 * t4 + 1 < n ? 0xffff0000u : 0u);
+            khi = (2 * t4 + 8 < n ? 0x0000ffffu : 0u) | (2 * t4 + 9 < n ? 0xffff0000u : 0u);
+          }
+          const uint32_t vt = st + p * S::kPage + S::kTile;
+#pragma unroll
+          for (int c2 = 0; c2 < kNT / 2; ++c2) {
+            uint32_t v0, v1, v2, v3;
+            ldsm_x4_t(vt + swz(row, 2 * c2 + (lm >> 1)), v0, v1, v2, v3);
+            if constexpr (decltype(masked)::value) {
+              v0 &= klo;
+              v1 &= khi;
+              v2 &= klo;
+              v3 &= khi;
+            }
+            M::run(o[2 * c2], ph[p][0], ph[p][1], ph[p][2], ph[p][3], v0, v1);
+            M::run(o[2 * c2 + 1], ph[p][0], ph[p][1], ph[p][2], ph[p][3], v2, v3);
+            M::run(o[2 * c2], pl[p][0], pl[p][1], pl[p][2], pl[p][3], v0, v1);
+            M::run(o[2 * c2 + 1], pl[p][0], pl[p][1], pl[p][2], pl[p][3], v2, v3);
+          }
+        }
+      };
+      if (full)
+        pv(std::false_type{});
+      else
+        pv(std::true_type{});
+    }
+    // this warp is done with stage s; the last of the NWF warps to say so
+    // refills it (the fences order every warp's reads of the stage before
+    // the copy that overwrites it)
+    __syncwarp();
+    if (lane == 0) {
+      __threadfence_block();
+      const unsigned int before = atomicAdd(&released[s], 1u);
+      if (before % NWF == NWF - 1) {
+        __threadfence_block();
+        issue(c + NSTAGE);
+      }
+    }
+  }
+  if (__syncthreads_or(bad)) {  // after a give-up: the last step issued into each stage lands first
+    if (threadIdx.x == 0) {
+      unsigned int issued = 0;
+      for (int st = 0; st < NSTAGE; ++st) issued += released[st] / NWF;
+      issued = min(static_cast<unsigned int>(nstep), issued + NSTAGE);
+      for (int c = max(0, static_cast<int>(issued) - NSTAGE); c < static_cast<int>(issued); ++c)
+        mbar_wait_bounded(bar0 + 8 * (c % NSTAGE), (c / NSTAGE) & 1u);
+    }
+    return;
+  }
+#pragma unroll
+  for (int msk = 1; msk <= 2; msk <<= 1) {
+    lA += __shfl_xor_sync(kFull, lA, msk);
+    lB += __shfl_xor_sync(kFull, lB, msk);
+  }
+  // rows A and B: d = 8 j + 2 t4, + 1 of every n-tile j
+#pragma unroll
+  for (int e = 0; e < 2; ++e) {
+    const int tr = e ? trB : trA;
+    if (tr >= R) continue;
+    const int pos = e ? posB : posA;
+    const size_t row = out_row(tr);
+    const float mm = e ? mB : mA, ll = e ? lB : lA;
+    if (pos < tok0) {  // no key of this partition (or before position 0)
+      if (direct)
+#pragma unroll
+        for (int j = 0; j < kNT; ++j)
+          *reinterpret_cast<uint32_t*>(reinterpret_cast<T*>(a.out) + row * D + 8 * j + 2 * t4) = M::pack(0.f, 0.f);
+      continue;
+    }
+    if (direct) {
+      const float inv = 1.f / ll;
+#pragma unroll
+      for (int j = 0; j < kNT; ++j)
+        *reinterpret_cast<uint32_t*>(reinterpret_cast<T*>(a.out) + row * D + 8 * j + 2 * t4) =
+            M::pack(o[j][2 * e] * inv, o[j][2 * e + 1] * inv);
+    } else {
+      const size_t wrow = row * a.num_parts + z;
+#pragma unroll
+      for (int j = 0; j < kNT; ++j)
+        *reinterpret_cast<float2*>(a.ws_o + wrow * D + 8 * j + 2 * t4) = make_float2(o[j][2 * e], o[j][2 * e + 1]);
+      if (t4 == 0) a.ws_ml[wrow] = make_float2(mm, ll);
+    }
+  }
+}
+
 // Merge of the key partitions of each query row (token t = blockIdx.x, HPC
 // heads per CTA from head blockIdx.y * HPC): the row at position pos uses
 // partitions 0 .. pos / partition.

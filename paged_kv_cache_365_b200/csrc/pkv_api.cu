@@ -71,14 +71,26 @@ pkv_status launch_multi(const pkv::MultiArgs& a, const void* k_cache, const void
 }
 
 // Up to 16 rows per sequence (max_query_len * G): one tile of 8 NT rows,
-// the warps splitting the pages.  More: tiles of 8 NW rows, one warp per
-// 8 rows, the warps sharing the pages (paged_multi_rows_kernel).
+// the warps splitting the pages.  Up to 32: one tile of 8 NW rows, one warp
+// per 8 rows, the warps sharing the pages (paged_multi_rows_kernel).  More:
+// tiles of 64 rows as the MMA's M dimension, 16 per warp
+// (paged_multi_fa_kernel).
 // Auto partition of the multi-token path: 2048 tokens, 1024 past 4096.
 int resolve_multi_partition(int p, long long max_ctx) {
   return resolve_partition(p != 0 ? p : (max_ctx > 4096 ? 1024 : 2048), max_ctx);
 }
 int multi_ntiles(long long rows) { return rows <= 8 ? 1 : 2; }
 int multi_rows_warps(long long rows) { return rows <= 16 ? 0 : rows <= 24 ? 3 : 4; }
+#ifndef PKV_FA_ABOVE_ROWS
+#define PKV_FA_ABOVE_ROWS 32
+#endif
+constexpr int kFaAboveRows = PKV_FA_ABOVE_ROWS;  // rows per kv-head past which the M-dimension kernel runs
+constexpr int kFaWarps = 4;  // 16 rows each
+#ifndef PKV_FA_PAGES
+#define PKV_FA_PAGES 2
+#endif
+constexpr int kFaPages = PKV_FA_PAGES;  // pages a warp takes in one step
+constexpr int kFaCode = 100;  // dispatch code of paged_multi_fa_kernel
 #ifndef PKV_ROWS_STAGES
 #define PKV_ROWS_STAGES 2
 #endif
@@ -116,15 +128,43 @@ pkv_status launch_multi_rows(const pkv::MultiArgs& a, const void* k_cache, const
 }
 
 template <typename T, int D, int G>
+pkv_status launch_multi_fa(const pkv::MultiArgs& a, const void* k_cache, const void* v_cache, int num_blocks,
+                           cudaStream_t st) {
+  using S = pkv::RowsShape<D, kFaWarps, kRowsStages, kFaPages>;
+  static_assert(kMaxPartition / PKV_BLOCK_SIZE <= S::kMaxPages, "the page table of a partition fits shared memory");
+  CUtensorMap mk, mv;
+  const long long rows = static_cast<long long>(num_blocks) * a.num_kv_heads * PKV_BLOCK_SIZE;
+  if (!encode_cache_map(&mk, k_cache, pkv::Mma<T>::kTmaType, D, rows) ||
+      !encode_cache_map(&mv, v_cache, pkv::Mma<T>::kTmaType, D, rows))
+    return PKV_ECUDA;
+  auto kfn = pkv::paged_multi_fa_kernel<T, D, G, kFaWarps, kRowsStages, kFaPages>;
+  if (cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(S::kSmem)) !=
+      cudaSuccess)
+    return PKV_ECUDA;
+  const dim3 grid(a.num_kv_heads, a.num_seqs * a.tiles, a.num_parts);
+  if (launch(kfn, grid, dim3(kFaWarps * 32), S::kSmem, st, a, mk, mv) != PKV_OK) return PKV_ECUDA;
+  if (a.num_parts > 1) {
+    const dim3 block(pkv::kMergeWarps * 32);
+    if (a.num_parts >= 32)
+      return launch(MultiMergeK<T, D, 1>::fn, dim3(a.total_q, a.num_q_heads), block, 0, st, a);
+    if (a.num_parts >= 16)
+      return launch(MultiMergeK<T, D, 4>::fn, dim3(a.total_q, (a.num_q_heads + 3) / 4), block, 0, st, a);
+    return launch(MultiMergeK<T, D, 8>::fn, dim3(a.total_q, (a.num_q_heads + 7) / 8), block, 0, st, a);
+  }
+  return PKV_OK;
+}
+
+template <typename T, int D, int G>
 pkv_status dispatch_nt_multi(const pkv::MultiArgs& a, int NT, const void* k, const void* v, int nb,
                              cudaStream_t st) {
-  // NT > 0: n-tiles per CTA (pages split over the warps); NT < 0: -NT warps
-  // splitting the rows
+  // NT 1, 2: n-tiles per CTA (pages split over the warps); -3, -4: warps
+  // splitting the rows; kFaCode: rows as the MMA's M dimension
   switch (NT) {
     case 1: return launch_multi<T, D, G, 1>(a, k, v, nb, st);
     case 2: return launch_multi<T, D, G, 2>(a, k, v, nb, st);
     case -3: return launch_multi_rows<T, D, G, 3>(a, k, v, nb, st);
     case -4: return launch_multi_rows<T, D, G, 4>(a, k, v, nb, st);
+    case kFaCode: return launch_multi_fa<T, D, G>(a, k, v, nb, st);
   }
   return PKV_EINVAL;
 }
@@ -592,9 +632,10 @@ pkv_status pkv_paged_attention_multi(void* out, const void* q, const void* k_cac
   if (static_cast<long long>(num_blocks) * num_kv_heads * PKV_BLOCK_SIZE > 0x7fffffffLL) return PKV_EINVAL;
   const int G = num_q_heads / num_kv_heads;
   const long long rows_max = static_cast<long long>(max_query_len) * G;
-  const int NW = multi_rows_warps(rows_max);
-  const int NT = NW ? -NW : multi_ntiles(rows_max);
-  const int tile_rows = 8 * (NW ? NW : NT);
+  const bool fa = rows_max > kFaAboveRows;
+  const int NW = fa ? 0 : multi_rows_warps(rows_max);
+  const int NT = fa ? kFaCode : NW ? -NW : multi_ntiles(rows_max);
+  const int tile_rows = fa ? 16 * kFaWarps : 8 * (NW ? NW : NT);
   const long long tiles = (rows_max + tile_rows - 1) / tile_rows;
   const long long P = (static_cast<long long>(max_context_len) + part - 1) / part;
   if (tiles * num_seqs > 65535 || P > 65535) return PKV_EINVAL;

@@ -143,6 +143,38 @@ def test_edge_rows_and_flags():
     assert np.abs(got[:3] - want[:3]).max() <= TOL["f16"]
 
 
+@pytest.mark.parametrize("case", [
+    ([70, 600, 37], [37, 20, 37], 4, 4, 128, "f16"),    # 37 rows: one 64-row tile, 27 padded
+    ([900, 300], [20, 11], 16, 2, 64, "bf16"),          # 160 rows: three tiles, the last partial
+    ([2500, 130, 16], [100, 64, 16], 8, 8, 128, "bf16"),  # long chunks, whole contexts of new tokens
+], ids=lambda c: f"{c[5]}_G{c[2] // c[3]}_D{c[4]}_rows{max(c[1]) * c[2] // c[3]}")
+@pytest.mark.parametrize("partition", [0, 64, 2048])
+def test_rows_as_m_kernel(case, partition):
+    """More than 32 rows per kv-head go to the kernel with the rows as the
+    MMA's M dimension (16 per warp, 64 per tile): tiles that start mid-
+    sequence, padded rows, chunks whose causal diagonal crosses pages and
+    partitions, sequences made only of new tokens."""
+    ctx, nq, Hq, Hkv, D, dt = case
+    c = make_multi_case(ctx, nq, Hq, Hkv, D, dt, seed=sum(ctx) + partition)
+    scale = D ** -0.5
+    want = oracle.paged_multi(c["q"], c["k"], c["v"], c["tables"], c["ctx"], c["qs"], scale, dt)
+    got, err = run_gpu(c, scale, partition)
+    assert err == 0
+    assert np.isfinite(got).all()
+    assert np.abs(got - want).max() <= TOL[dt]
+
+
+def test_rows_as_m_kernel_flags_rows_before_the_context():
+    m = pkv()
+    # 40 new tokens against a 30-token context: the first 10 rows of each
+    # head are zeros and flagged
+    c = make_multi_case([30, 200], [40, 40], 4, 4, 64, "f16", seed=9)
+    want = oracle.paged_multi(c["q"], c["k"], c["v"], c["tables"], c["ctx"], c["qs"], 0.125, "f16")
+    got, err = run_gpu(c, 0.125)
+    assert err == m.ERR_CONTEXT_RANGE
+    assert np.abs(got - want).max() <= TOL["f16"]
+
+
 def test_multi_step_through_the_cache_api():
     """PagedKVCache.plan_multi_step + run_multi_step (host inputs, one of
     them forcing a copy-on-write) against the oracle allocator, cache and
