@@ -424,6 +424,124 @@ struct RowsShape {
   static_assert(kPage % 1024 == 0, "swizzled boxes need 1024-byte alignment");
 };
 
+// The CTA-wide page ring of the kernels whose warps all read every page of
+// a partition: the partition's page table in shared memory, NSTAGE stages
+// of KP pages filled by TMA, a full barrier per stage, and a release
+// counter per stage.  Every warp waits for step c's stage; after its last
+// read of the stage a warp counts itself out, and the warp that completes
+// the count refills the stage with step c + NSTAGE, so the warps drift up
+// to NSTAGE steps apart instead of meeting at a CTA barrier.
+template <int D, int NW, int NSTAGE, int KP>
+struct PageRing {
+  using S = RowsShape<D, NW, NSTAGE, KP>;
+  uint32_t stage0, bar0;
+  unsigned int* released;  // warps done with the stage, per stage
+  int* table;              // physical block of page i of the partition, or -1
+  int nblk, nstep;
+  uint32_t phase_bits;
+
+  // Lays the ring out in `smem` (1024-byte aligned), reads the partition's
+  // table entries (flagging any outside the pool), initialises the
+  // barriers and issues the first NSTAGE steps.  Every thread of the CTA
+  // calls it; it ends with a CTA barrier.
+  __device__ void init(unsigned char* smem, const MultiArgs& a, int b, int kvh, int tok0, int tok1,
+                       const CUtensorMap* mk, const CUtensorMap* mv) {
+    stage0 = smem_addr(smem);
+    bar0 = smem_addr(smem + S::kBarOff);
+    released = reinterpret_cast<unsigned int*>(smem + S::kCntOff);
+    table = reinterpret_cast<int*>(smem + S::kTabOff);
+    phase_bits = 0;
+    const int pg0 = tok0 / kBlockSize;
+    nblk = (tok1 - tok0 + kBlockSize - 1) / kBlockSize;  // <= S::kMaxPages
+    nstep = (nblk + KP - 1) / KP;
+    for (int j = threadIdx.x; j < nblk; j += NW * 32) {
+      const int e = a.block_tables[static_cast<long long>(b) * a.bt_stride + pg0 + j];
+      const bool in = e >= 0 && e < a.num_blocks;
+      if (!in) raise_error(PKV_ERR_BLOCK_RANGE);
+      table[j] = in ? e : -1;
+    }
+    if (threadIdx.x == 0) {
+      for (int s = 0; s < NSTAGE; ++s) {
+        mbar_init(bar0 + 8 * s, 1);
+        released[s] = 0u;
+      }
+      fence_barrier_init();
+    }
+    __syncthreads();
+    if (threadIdx.x == 0)
+      for (int c = 0; c < NSTAGE; ++c) issue(c, a.num_kv_heads, kvh, mk, mv);
+  }
+
+  // pages KP c .. KP c + KP - 1 into stage c % NSTAGE (one lane); pages past
+  // the partition or outside the pool are not copied
+  __device__ void issue(int c, int num_kv_heads, int kvh, const CUtensorMap* mk, const CUtensorMap* mv) {
+    if (c >= nstep) return;
+    const uint32_t bar = bar0 + 8 * (c % NSTAGE);
+    uint32_t bytes = 0;
+#pragma unroll
+    for (int p = 0; p < KP; ++p) {
+      const int i = c * KP + p;
+      if (i < nblk && table[i] >= 0) bytes += S::kPage;
+    }
+    if (bytes == 0) {
+      mbar_arrive(bar);
+      return;
+    }
+    fence_proxy_async_smem();
+    mbar_arrive_expect_tx(bar, bytes);
+#pragma unroll
+    for (int p = 0; p < KP; ++p) {
+      const int i = c * KP + p;
+      if (i < nblk && table[i] >= 0) {
+        const uint32_t dst = stage0 + (c % NSTAGE) * S::kStage + p * S::kPage;
+        const int y = (table[i] * num_kv_heads + kvh) * kBlockSize;
+#pragma unroll
+        for (int bx = 0; bx < S::kBoxes; ++bx) {
+          tma_load_2d(dst + bx * 2048, mk, bx * 64, y, bar);
+          tma_load_2d(dst + S::kTile + bx * 2048, mv, bx * 64, y, bar);
+        }
+      }
+    }
+  }
+
+  // Waits (bounded, the whole warp) for step c's stage; false = gave up.
+  __device__ bool wait(int c) {
+    const int s = c % NSTAGE;
+    const bool ok = __all_sync(kFull, mbar_wait_bounded(bar0 + 8 * s, (phase_bits >> s) & 1u));
+    phase_bits ^= 1u << s;
+    return ok;
+  }
+
+  __device__ uint32_t stage(int c) const { return stage0 + (c % NSTAGE) * S::kStage; }
+
+  // This warp is done with step c's stage; the last of the NW warps to say
+  // so refills it (the fences order every warp's reads of the stage before
+  // the copy that overwrites it).
+  __device__ void release(int c, int num_kv_heads, int kvh, const CUtensorMap* mk, const CUtensorMap* mv) {
+    __syncwarp();
+    if ((threadIdx.x & 31) == 0) {
+      __threadfence_block();
+      const unsigned int before = atomicAdd(&released[c % NSTAGE], 1u);
+      if (before % NW == NW - 1) {
+        __threadfence_block();
+        issue(c + NSTAGE, num_kv_heads, kvh, mk, mv);
+      }
+    }
+  }
+
+  // After a give-up, past a CTA barrier: thread 0 waits, bounded, for the
+  // last step issued into each stage, so no copy lands after the CTA exits.
+  __device__ void drain() {
+    if (threadIdx.x == 0) {
+      unsigned int issued = 0;  // NSTAGE + the refills (one per NW releases)
+      for (int st = 0; st < NSTAGE; ++st) issued += released[st] / NW;
+      issued = min(static_cast<unsigned int>(nstep), issued + NSTAGE);
+      for (int c = max(0, static_cast<int>(issued) - NSTAGE); c < static_cast<int>(issued); ++c)
+        mbar_wait_bounded(bar0 + 8 * (c % NSTAGE), (c / NSTAGE) & 1u);
+    }
+  }
+};
+
 // Resident warps per SM the register budget is sized for: 5 CTAs of 3
 // warps (up to 128 registers a thread, no spills) measured faster than 6
 // CTAs (96 registers) or 8 (80).
@@ -471,63 +589,9 @@ __global__ void __launch_bounds__(NW * 32, PKV_ROWS_WARPS_PER_SM / NW)
   extern __shared__ unsigned char smem_raw[];
   const uint32_t raw_addr = smem_addr(smem_raw);
   const uint32_t pad = ((raw_addr + 1023u) & ~1023u) - raw_addr;
-  unsigned char* smem = smem_raw + pad;
-  const uint32_t stage0 = smem_addr(smem);
-  const uint32_t bar0 = smem_addr(smem + S::kBarOff);
-  unsigned int* released = reinterpret_cast<unsigned int*>(smem + S::kCntOff);  // warps done, per stage
-  int* table = reinterpret_cast<int*>(smem + S::kTabOff);                       // physical page i, or -1
-
-  const int pg0 = tok0 / kBlockSize;
-  const int nblk = (tok1 - tok0 + kBlockSize - 1) / kBlockSize;  // <= S::kMaxPages
-  const int nstep = (nblk + KP - 1) / KP;
-  for (int j = threadIdx.x; j < nblk; j += NW * 32) {
-    const int e = a.block_tables[static_cast<long long>(b) * a.bt_stride + pg0 + j];
-    const bool in = e >= 0 && e < a.num_blocks;
-    if (!in) raise_error(PKV_ERR_BLOCK_RANGE);
-    table[j] = in ? e : -1;
-  }
-  if (threadIdx.x == 0) {
-    for (int s = 0; s < NSTAGE; ++s) {
-      mbar_init(bar0 + 8 * s, 1);
-      released[s] = 0u;
-    }
-    fence_barrier_init();
-  }
-  __syncthreads();
-
-  // pages KP c .. KP c + KP - 1 into stage c % NSTAGE (one lane); pages past
-  // the partition or outside the pool are not copied
-  auto issue = [&](int c) {
-    if (c >= nstep) return;
-    const uint32_t bar = bar0 + 8 * (c % NSTAGE);
-    uint32_t bytes = 0;
-#pragma unroll
-    for (int p = 0; p < KP; ++p) {
-      const int i = c * KP + p;
-      if (i < nblk && table[i] >= 0) bytes += S::kPage;
-    }
-    if (bytes == 0) {
-      mbar_arrive(bar);
-      return;
-    }
-    fence_proxy_async_smem();
-    mbar_arrive_expect_tx(bar, bytes);
-#pragma unroll
-    for (int p = 0; p < KP; ++p) {
-      const int i = c * KP + p;
-      if (i < nblk && table[i] >= 0) {
-        const uint32_t dst = stage0 + (c % NSTAGE) * S::kStage + p * S::kPage;
-        const int y = (table[i] * a.num_kv_heads + kvh) * kBlockSize;
-#pragma unroll
-        for (int bx = 0; bx < S::kBoxes; ++bx) {
-          tma_load_2d(dst + bx * 2048, &tmap_k, bx * 64, y, bar);
-          tma_load_2d(dst + S::kTile + bx * 2048, &tmap_v, bx * 64, y, bar);
-        }
-      }
-    }
-  };
-  if (threadIdx.x == 0)
-    for (int c = 0; c < NSTAGE; ++c) issue(c);
+  PageRing<D, NW, NSTAGE, KP> ring;
+  ring.init(smem_raw + pad, a, b, kvh, tok0, tok1, &tmap_k, &tmap_v);
+  const int nstep = ring.nstep;
 
   // this warp's column g8 (row r0 + 8 warp + g8) and its lane's columns 2 t4, 2 t4 + 1
   uint32_t qb[S::kKSteps][2];
@@ -549,14 +613,10 @@ __global__ void __launch_bounds__(NW * 32, PKV_ROWS_WARPS_PER_SM / NW)
 #pragma unroll
   for (int mt = 0; mt < S::kKSteps; ++mt) o[mt][0] = o[mt][1] = o[mt][2] = o[mt][3] = 0.f;
   float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
-  uint32_t phase_bits = 0;
   bool bad = false;
 
   for (int c = 0; c < nstep; ++c) {
-    const int s = c % NSTAGE;
-    const bool ok = __all_sync(kFull, mbar_wait_bounded(bar0 + 8 * s, (phase_bits >> s) & 1u));
-    phase_bits ^= 1u << s;
-    if (!ok) {  // this warp gives up; the others time out on the stages it never releases
+    if (!ring.wait(c)) {  // this warp gives up; the others time out on the stages it never releases
       if (lane == 0) raise_error(PKV_ERR_TIMEOUT);
       bad = true;
       break;
@@ -568,11 +628,11 @@ __global__ void __launch_bounds__(NW * 32, PKV_ROWS_WARPS_PER_SM / NW)
 #pragma unroll
     for (int p = 0; p < KP; ++p) {
       const int i = c * KP + p;
-      held[p] = i < nblk && table[i] >= 0;
+      held[p] = i < ring.nblk && ring.table[i] >= 0;
       nvalid[p] = held[p] ? min(kBlockSize, tok1 - tok0 - i * kBlockSize) : 0;
       full = full && nvalid[p] == kBlockSize;
     }
-    const uint32_t st = stage0 + s * S::kStage;
+    const uint32_t st = ring.stage(c);
     // S^T per page in two independent accumulation chains
     float x[KP][4];
 #pragma unroll
@@ -677,29 +737,11 @@ __global__ void __launch_bounds__(NW * 32, PKV_ROWS_WARPS_PER_SM / NW)
       pv(std::false_type{});
     else
       pv(std::true_type{});
-    // this warp is done with stage s; the last of the NW warps to say so
-    // refills it with the pages NSTAGE steps ahead (the fences order every
-    // warp's reads of the stage before the copy that overwrites it)
-    __syncwarp();
-    if (lane == 0) {
-      __threadfence_block();
-      const unsigned int before = atomicAdd(&released[s], 1u);
-      if (before % NW == NW - 1) {
-        __threadfence_block();
-        issue(c + NSTAGE);
-      }
-    }
+    ring.release(c, a.num_kv_heads, kvh, &tmap_k, &tmap_v);
   }
-  // every copy this CTA issued lands before the CTA exits: after a give-up,
-  // thread 0 waits (bounded) for the last step issued into each stage
+  // every copy this CTA issued lands before the CTA exits
   if (__syncthreads_or(bad)) {
-    if (threadIdx.x == 0) {
-      unsigned int issued = 0;  // steps issued: NSTAGE + the refills (one per NW releases)
-      for (int st = 0; st < NSTAGE; ++st) issued += released[st] / NW;
-      issued = min(static_cast<unsigned int>(nstep), issued + NSTAGE);
-      for (int c = max(0, static_cast<int>(issued) - NSTAGE); c < static_cast<int>(issued); ++c)
-        mbar_wait_bounded(bar0 + 8 * (c % NSTAGE), (c / NSTAGE) & 1u);
-    }
+    ring.drain();
     return;
   }
 #pragma unroll
@@ -805,61 +847,9 @@ __global__ void __launch_bounds__(NWF * 32, PKV_FA_MIN_CTAS)
   extern __shared__ unsigned char smem_raw[];
   const uint32_t raw_addr = smem_addr(smem_raw);
   const uint32_t pad = ((raw_addr + 1023u) & ~1023u) - raw_addr;
-  unsigned char* smem = smem_raw + pad;
-  const uint32_t stage0 = smem_addr(smem);
-  const uint32_t bar0 = smem_addr(smem + S::kBarOff);
-  unsigned int* released = reinterpret_cast<unsigned int*>(smem + S::kCntOff);  // warps done, per stage
-  int* table = reinterpret_cast<int*>(smem + S::kTabOff);                       // physical page i, or -1
-
-  const int pg0 = tok0 / kBlockSize;
-  const int nblk = (tok1 - tok0 + kBlockSize - 1) / kBlockSize;  // <= S::kMaxPages
-  const int nstep = (nblk + KP - 1) / KP;
-  for (int j = threadIdx.x; j < nblk; j += NWF * 32) {
-    const int e = a.block_tables[static_cast<long long>(b) * a.bt_stride + pg0 + j];
-    const bool in = e >= 0 && e < a.num_blocks;
-    if (!in) raise_error(PKV_ERR_BLOCK_RANGE);
-    table[j] = in ? e : -1;
-  }
-  if (threadIdx.x == 0) {
-    for (int s = 0; s < NSTAGE; ++s) {
-      mbar_init(bar0 + 8 * s, 1);
-      released[s] = 0u;
-    }
-    fence_barrier_init();
-  }
-  __syncthreads();
-
-  auto issue = [&](int c) {  // pages KP c .. KP c + KP - 1 into stage c % NSTAGE (one lane)
-    if (c >= nstep) return;
-    const uint32_t bar = bar0 + 8 * (c % NSTAGE);
-    uint32_t bytes = 0;
-#pragma unroll
-    for (int p = 0; p < KP; ++p) {
-      const int i = c * KP + p;
-      if (i < nblk && table[i] >= 0) bytes += S::kPage;
-    }
-    if (bytes == 0) {
-      mbar_arrive(bar);
-      return;
-    }
-    fence_proxy_async_smem();
-    mbar_arrive_expect_tx(bar, bytes);
-#pragma unroll
-    for (int p = 0; p < KP; ++p) {
-      const int i = c * KP + p;
-      if (i < nblk && table[i] >= 0) {
-        const uint32_t dst = stage0 + (c % NSTAGE) * S::kStage + p * S::kPage;
-        const int y = (table[i] * a.num_kv_heads + kvh) * kBlockSize;
-#pragma unroll
-        for (int bx = 0; bx < S::kBoxes; ++bx) {
-          tma_load_2d(dst + bx * 2048, &tmap_k, bx * 64, y, bar);
-          tma_load_2d(dst + S::kTile + bx * 2048, &tmap_v, bx * 64, y, bar);
-        }
-      }
-    }
-  };
-  if (threadIdx.x == 0)
-    for (int c = 0; c < NSTAGE; ++c) issue(c);
+  PageRing<D, NWF, NSTAGE, KP> ring;
+  ring.init(smem_raw + pad, a, b, kvh, tok0, tok1, &tmap_k, &tmap_v);
+  const int nstep = ring.nstep;
 
   // this warp's rows: fragment rows g8 (row A) and g8 + 8 (row B)
   const int wr0 = r0 + 16 * warp;
@@ -883,14 +873,10 @@ __global__ void __launch_bounds__(NWF * 32, PKV_FA_MIN_CTAS)
 #pragma unroll
   for (int j = 0; j < kNT; ++j) o[j][0] = o[j][1] = o[j][2] = o[j][3] = 0.f;
   float mA = -INFINITY, mB = -INFINITY, lA = 0.f, lB = 0.f;  // lA, lB: this lane's part of the row sums
-  uint32_t phase_bits = 0;
   bool bad = false;
 
   for (int c = 0; c < nstep; ++c) {
-    const int s = c % NSTAGE;
-    const bool ok = __all_sync(kFull, mbar_wait_bounded(bar0 + 8 * s, (phase_bits >> s) & 1u));
-    phase_bits ^= 1u << s;
-    if (!ok) {  // this warp gives up; the others time out on the stages it never releases
+    if (!ring.wait(c)) {  // this warp gives up; the others time out on the stages it never releases
       if (lane == 0) raise_error(PKV_ERR_TIMEOUT);
       bad = true;
       break;
@@ -902,13 +888,13 @@ __global__ void __launch_bounds__(NWF * 32, PKV_FA_MIN_CTAS)
     for (int p = 0; p < KP; ++p) {
       const int i = c * KP + p;
       page_tok[p] = tok0 + i * kBlockSize;
-      run[p] = i < nblk && table[i] >= 0 && page_tok[p] <= wpos;
+      run[p] = i < ring.nblk && ring.table[i] >= 0 && page_tok[p] <= wpos;
       nvalid[p] = run[p] ? min(kBlockSize, tok1 - page_tok[p]) : 0;
       any = any || run[p];
       full = full && nvalid[p] == kBlockSize;
     }
     if (any) {
-      const uint32_t st = stage0 + s * S::kStage;
+      const uint32_t st = ring.stage(c);
       // S per page: n-tile 0 = tokens 0-7, n-tile 1 = tokens 8-15; two
       // accumulation chains (even and odd k-steps) each
       float x[KP][2][4];
@@ -1032,27 +1018,11 @@ __global__ void __launch_bounds__(NWF * 32, PKV_FA_MIN_CTAS)
       else
         pv(std::true_type{});
     }
-    // this warp is done with stage s; the last of the NWF warps to say so
-    // refills it (the fences order every warp's reads of the stage before
-    // the copy that overwrites it)
-    __syncwarp();
-    if (lane == 0) {
-      __threadfence_block();
-      const unsigned int before = atomicAdd(&released[s], 1u);
-      if (before % NWF == NWF - 1) {
-        __threadfence_block();
-        issue(c + NSTAGE);
-      }
-    }
+    ring.release(c, a.num_kv_heads, kvh, &tmap_k, &tmap_v);
   }
-  if (__syncthreads_or(bad)) {  // after a give-up: the last step issued into each stage lands first
-    if (threadIdx.x == 0) {
-      unsigned int issued = 0;
-      for (int st = 0; st < NSTAGE; ++st) issued += released[st] / NWF;
-      issued = min(static_cast<unsigned int>(nstep), issued + NSTAGE);
-      for (int c = max(0, static_cast<int>(issued) - NSTAGE); c < static_cast<int>(issued); ++c)
-        mbar_wait_bounded(bar0 + 8 * (c % NSTAGE), (c / NSTAGE) & 1u);
-    }
+  // every copy this CTA issued lands before the CTA exits
+  if (__syncthreads_or(bad)) {
+    ring.drain();
     return;
   }
 #pragma unroll
