@@ -49,6 +49,7 @@ MULTI_METRIC = ("paged multi-token attention (several new tokens per sequence, c
                 "(% of peak), query-tokens/s")
 UNIT = "GB/s"
 FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1400.0
 STORAGE = {"f32": 4, "f16": 2, "bf16": 2}
 DTYPE_NAME = {"f32": "fp32", "f16": "fp16", "bf16": "bf16"}
 # the decode kernels and their launch configuration: a committed ncu traffic
@@ -99,6 +100,40 @@ def measured_peak():
         return float(d["hbm_gbs"]), "measured"
     except Exception:
         return FALLBACK_HBM_GBS, "fallback"
+
+
+def measured_tensor_peak():
+    """Dense bf16 tensor-core TFLOP/s: the sustained figure (the kernels are
+    timed inside a long step loop)."""
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["bf16_tflops_sustained"]), "measured (MEASURED_PEAKS bf16_tflops_sustained)"
+    except Exception:
+        return FALLBACK_BF16_TFLOPS, "fallback"
+
+
+def multi_useful_flops(lens, n_new: int, Hq: int, D: int) -> int:
+    """Flops of one multi-token attention call: new token i of a sequence of
+    (post-append) length L sits at L - n + i and meets L - n + i + 1 keys; per
+    key and head, q.k and p.v cost 2 D flops each."""
+    keys = 0
+    for L in np.asarray(lens, dtype=np.int64):
+        n = min(int(n_new), int(L))
+        keys += n * (int(L) - n) + n * (n + 1) // 2
+    return keys * Hq * D * 4
+
+
+def roofline_of(nbytes: float, flops: float, secs: float, hbm_gbs: float, tensor_tflops: float):
+    """The binding roofline of a call: whichever of its bytes at the copy
+    bandwidth and its flops at the tensor peak takes longer."""
+    t_mem = nbytes / (hbm_gbs * 1e9)
+    t_math = flops / (tensor_tflops * 1e12)
+    if t_math > t_mem:
+        return {"bound": "tensor", "achieved": flops / secs / 1e12, "peak": tensor_tflops, "unit": "TFLOP/s",
+                "frac": t_math / secs}
+    return {"bound": "hbm", "achieved": nbytes / secs / 1e9, "peak": hbm_gbs, "unit": "GB/s", "frac": t_mem / secs}
 
 
 def recorded_traffic(workload: str):
@@ -557,8 +592,10 @@ def multi_line(args, r, world):
     wl = r["wl"]
     K = r["K"]
     peak, peak_kind = measured_peak()
+    tpeak, tpeak_kind = measured_tensor_peak()
     step_s = r["total_ms"] / 1e3 / K
-    achieved = r["att_bytes"] / (r["att_ms"] / 1e3) / 1e9
+    flops = multi_useful_flops(r["lens"], args.new_tokens, wl.Hq, wl.D)
+    roof = roofline_of(r["att_bytes"], flops, r["att_ms"] / 1e3, peak, tpeak)
     line = {
         "metric": MULTI_METRIC, "value": job_throughput(r["kv"], world, K, r["total_ms"] / 1e3), "unit": UNIT,
         "n_gpus": world, "steps": K, "warmup": args.warmup, "ms_per_step": r["total_ms"] / K,
@@ -581,10 +618,11 @@ def multi_line(args, r, world):
                 "h2d_bytes_per_step": r["h2d"], "d2h_bytes_per_step": r["d2h"],
                 "us_per_step": 1e3 * r["e2e_ms"] / K},
         "gpu_launches": r["launches"],
-        "roofline": {"kernel": "paged_multi (partition + merge kernels)", "bound": "hbm", "achieved": achieved,
-                     "peak": peak, "peak_kind": f"{peak_kind} (MEASURED_PEAKS hbm_gbs)" if peak_kind == "measured"
-                     else "fallback", "unit": "GB/s", "frac": achieved / peak, "traffic": None,
-                     "algorithmic_bytes_per_launch": r["att_bytes"], "avg_launch_us": 1e3 * r["att_ms"]},
+        "roofline": {"kernel": "paged_multi (partition + merge kernels)", **roof,
+                     "peak_kind": (tpeak_kind if roof["bound"] == "tensor" else
+                                   f"{peak_kind} (MEASURED_PEAKS hbm_gbs)" if peak_kind == "measured" else "fallback"),
+                     "traffic": None, "algorithmic_bytes_per_launch": r["att_bytes"],
+                     "useful_flops_per_launch": flops, "avg_launch_us": 1e3 * r["att_ms"]},
     }
     if world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = multi_cpu_baseline(wl, args.new_tokens, seed=args.seed)

@@ -57,3 +57,45 @@ def test_bench_reports_the_library_auto_partitions():
         Pm = -(-n // pkv.api.auto_partition_multi(n))
         want = 0 if Pm <= 1 else -(-(T * Hq * Pm * D * 4) // 16) * 16 + T * Hq * Pm * 8
         assert pkv.multi_workspace_bytes(T, Hq, D, n, 0) == want
+
+
+def test_multi_flops_and_roofline_choice():
+    """The multi-token row's flop count against a brute-force count of
+    (query, key) pairs, and the binding roofline picked by the longer of the
+    memory and math times."""
+    import bench
+    lens, n_new, Hq, D = [5, 40, 3], 4, 2, 8
+    pairs = 0
+    for L in lens:
+        n = min(n_new, L)
+        for i in range(n):
+            pos = L - n + i
+            pairs += sum(1 for j in range(L) if j <= pos)
+    assert bench.multi_useful_flops(lens, n_new, Hq, D) == pairs * Hq * D * 4
+    r = bench.roofline_of(1e9, 1e12, 1e-3, 5000.0, 1000.0)   # 0.2 ms of bytes, 1 ms of math
+    assert r["bound"] == "tensor" and abs(r["frac"] - 1.0) < 1e-12 and r["unit"] == "TFLOP/s"
+    r = bench.roofline_of(1e9, 1e9, 4e-4, 5000.0, 1000.0)    # 0.2 ms of bytes, 1 us of math
+    assert r["bound"] == "hbm" and abs(r["frac"] - 0.5) < 1e-12 and abs(r["achieved"] - 2500.0) < 1e-9
+
+
+def test_multi_line_builds_the_contract_json():
+    """multi_line (the multi-token row's JSON) from a timing record, without
+    a GPU: the contract's keys and the roofline's fields."""
+    import argparse
+    import numpy as np
+    import bench
+    import workloads
+    wl = workloads.named("tiny", 0)
+    lens = wl.context_lens.astype(np.int64) + 4
+    r = dict(wl=wl, K=10, T=5 * wl.B, kv=int(lens.sum()) * wl.kv_bytes_per_token, att_bytes=10 ** 6,
+             total_ms=1.0, att_ms=0.8, e2e_ms=1.5, h2d=1000, d2h=2000, clocks={"sm_mhz": 1800.0}, P=1,
+             launches=30, lens=lens)
+    args = argparse.Namespace(warmup=3, partition=0, seed=0, gpus=1, new_tokens=5, no_cpu_baseline=True)
+    d = bench.multi_line(args, r, 1)
+    for key in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better",
+                "scaling", "vs_baseline", "dtype", "data", "config", "clocks", "e2e", "gpu_launches", "roofline"):
+        assert key in d, key
+    roof = d["roofline"]
+    assert roof["bound"] in ("hbm", "tensor") and roof["frac"] > 0
+    assert roof["useful_flops_per_launch"] == bench.multi_useful_flops(lens, 5, wl.Hq, wl.D)
+    json.dumps(d)
