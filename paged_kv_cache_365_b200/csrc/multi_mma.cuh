@@ -394,20 +394,10 @@ __global__ void __launch_bounds__(NWARPS * 32)
   }
 }
 
-// Many rows per sequence (more than two n-tiles' worth): the warps of a CTA
-// split the rows instead of the pages.  Warp w owns the 8 rows r0 + 8 w ..
-// r0 + 8 w + 7 (one n-tile, so registers stay as in decode) and every warp
-// consumes every page of the partition from one CTA-wide ring of NSTAGE
-// stages of KP pages each.  A warp takes a stage's KP pages in one step: their
-// score MMAs form independent chains, one max / rescale serves all of them,
-// and their P.V products interleave, so a step has KP times the independent
-// work of a page at the same per-step softmax cost.  All warps wait on a
-// stage's mbarrier; after its last read of a stage a warp counts itself out
-// on that stage's counter, and the warp that completes the count refills the
-// stage with the pages NSTAGE steps ahead, so the warps drift up to NSTAGE
-// steps apart instead of meeting at a CTA barrier.  The partition's page
-// table sits in shared memory.  A page is read once per CTA for all its
-// 8 NW rows; the warps' rows are disjoint, so each writes its own outputs.
+// Shared-memory layout of the kernels whose warps all read every page of a
+// partition (paged_multi_rows_kernel, paged_multi_fa_kernel): NSTAGE stages
+// of KP pages (K tile then V tile each), a full barrier and a release
+// counter per stage, the partition's page table.
 template <int D, int NW, int NSTAGE, int KP>
 struct RowsShape {
   static constexpr int kTile = kBlockSize * D * 2;
@@ -542,6 +532,17 @@ struct PageRing {
   }
 };
 
+// 17-32 rows per sequence and kv-head (speculative verification with GQA):
+// the warps of a CTA split the rows instead of the pages.  Warp w owns the
+// 8 rows r0 + 8 w .. r0 + 8 w + 7 (one n-tile, so registers stay as in
+// decode) and every warp consumes every page of the partition from the
+// CTA's PageRing.  A warp takes a stage's KP pages in one step: their score
+// MMAs form independent chains, one max / rescale serves all of them, and
+// their P.V products interleave, so a step has KP times the independent
+// work of a page at the same per-step softmax cost.  A page is read once
+// per CTA for all its 8 NW rows; the warps' rows are disjoint, so each
+// writes its own outputs.
+//
 // Resident warps per SM the register budget is sized for: 5 CTAs of 3
 // warps (up to 128 registers a thread, no spills) measured faster than 6
 // CTAs (96 registers) or 8 (80).
