@@ -255,12 +255,12 @@ __global__ void __launch_bounds__(NWARPS * 32)
   for (int i = 0; i < my_n; ++i) {
     const int s = i % NSTAGE;
     bool ok = mbar_wait_bounded(bar0 + 8 * s, (phase_bits >> s) & 1u);
-    phase_bits ^= 1u << s;
     ok = __all_sync(kFull, ok);
     if (!ok) {
       if (lane == 0) raise_error(PKV_ERR_TIMEOUT);
       break;
     }
+    phase_bits ^= 1u << s;  // (a stage that timed out keeps its parity: the drain waits on it again)
     consumed = i + 1;
     const int phys = __shfl_sync(kFull, my_phys, i);
     if (phys >= 0) {
@@ -356,7 +356,7 @@ __global__ void __launch_bounds__(NWARPS * 32)
   // flight before its shared memory is reused
   if (consumed < my_n) {
     const int last = min(my_n, consumed + NSTAGE);
-    for (int i = consumed + 1; i < last; ++i) {
+    for (int i = consumed; i < last; ++i) {
       const int s = i % NSTAGE;
       mbar_wait_bounded(bar0 + 8 * s, (phase_bits >> s) & 1u);
       phase_bits ^= 1u << s;

@@ -235,13 +235,13 @@ __global__ void __launch_bounds__(NWARPS * 32, PKV_FP8_MIN_CTAS)
   for (int i = 0; i < my_n; ++i) {
     const int s = i % NSTAGE;
     bool ok = mbar_wait_bounded(bar0 + 8 * s, (phase_bits >> s) & 1u);
-    phase_bits ^= 1u << s;
     ok = __all_sync(kFull, ok);
     if (!ok) {
       if (lane == 0) raise_error(PKV_ERR_TIMEOUT);
       timed_out = true;
       break;
     }
+    phase_bits ^= 1u << s;  // (a stage that timed out keeps its parity: the drain waits on it again)
     consumed = i + 1;
     if (phys_of(i) >= 0) {
       const int page_tok = tok0 + (warp + i * NWARPS) * kBlockSize;
@@ -353,7 +353,7 @@ __global__ void __launch_bounds__(NWARPS * 32, PKV_FP8_MIN_CTAS)
   }
   if (consumed < my_n) {
     const int last = min(my_n, consumed + NSTAGE);
-    for (int i = consumed + 1; i < last; ++i) {
+    for (int i = consumed; i < last; ++i) {
       const int s = i % NSTAGE;
       mbar_wait_bounded(bar0 + 8 * s, (phase_bits >> s) & 1u);
       phase_bits ^= 1u << s;

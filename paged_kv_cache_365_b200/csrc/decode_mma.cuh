@@ -223,12 +223,12 @@ __device__ __forceinline__ bool prefix_warp(const DecodeArgs& a, const CUtensorM
   for (int i = 0; i < nblk; ++i) {
     const int s = i % NSTAGE;
     ok = mbar_wait_bounded(bar0 + 8 * s, (phase_bits >> s) & 1u);
-    phase_bits ^= 1u << s;
     ok = __all_sync(kFull, ok);
     if (!ok) {
       if (lane == 0) raise_error(PKV_ERR_TIMEOUT);
       break;
     }
+    phase_bits ^= 1u << s;  // (a stage that timed out keeps its parity: the drain waits on it again)
     consumed = i + 1;
     if (__shfl_sync(kFull, my_phys, i) >= 0) {
       const uint32_t kt = stage0 + s * kStage;
@@ -307,7 +307,7 @@ __device__ __forceinline__ bool prefix_warp(const DecodeArgs& a, const CUtensorM
   }
   if (consumed < nblk) {  // after a give-up: wait (bounded) for copies in flight
     const int last = min(nblk, consumed + NSTAGE);
-    for (int i = consumed + 1; i < last; ++i) {
+    for (int i = consumed; i < last; ++i) {
       const int s = i % NSTAGE;
       mbar_wait_bounded(bar0 + 8 * s, (phase_bits >> s) & 1u);
       phase_bits ^= 1u << s;
@@ -527,13 +527,13 @@ __global__ void __launch_bounds__(NWARPS * 32)
     for (int i = 0; i < my_n; ++i) {
       const int s = i % NSTAGE;
       bool ok = mbar_wait_bounded(bar0 + 8 * s, (phase_bits >> s) & 1u);
-      phase_bits ^= 1u << s;
       ok = __all_sync(kFull, ok);
       if (!ok) {
         if (lane == 0) raise_error(PKV_ERR_TIMEOUT);
         timed_out = true;
         break;
       }
+      phase_bits ^= 1u << s;  // (a stage that timed out keeps its parity: the drain waits on it again)
       consumed = i + 1;
       const int phys = phys_of(i);
       if (phys >= 0) {
@@ -622,7 +622,7 @@ __global__ void __launch_bounds__(NWARPS * 32)
     // after a give-up, wait (bounded) for the copies still in flight
     if (consumed < my_n) {
       const int last = min(my_n, consumed + NSTAGE);
-      for (int i = consumed + 1; i < last; ++i) {
+      for (int i = consumed; i < last; ++i) {
         const int s = i % NSTAGE;
         mbar_wait_bounded(bar0 + 8 * s, (phase_bits >> s) & 1u);
         phase_bits ^= 1u << s;
