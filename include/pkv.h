@@ -302,7 +302,11 @@ pkv_status pkv_paged_attention_decode_prefix_phase(void* out, const void* q, con
  *     (use pkv_paged_attention_decode with a caller-owned workspace then).
  *   - The first call on a device looks up that device's address of the
  *     scratch area (a runtime query, no allocation), with the caller's
- *     current device; make that first call before any stream capture.
+ *     current device; make that first call before any stream capture.  The
+ *     address is kept per device and per context (by the context's unique
+ *     id): after the caller destroys and re-creates the device's context
+ *     (cudaDeviceReset, or a primary-context reset), the next call looks it
+ *     up again, so that call too belongs before any capture.
  *   - All calls on a device share the one scratch area, and it keeps what
  *     the previous call left in it.  The decode writes every scratch value
  *     before it reads it, so nothing needs clearing between calls, but two
@@ -414,6 +418,70 @@ pkv_status pkv_paged_attention_multi(void* out, const void* q, const void* k_cac
                                      void* workspace, size_t workspace_bytes, void* stream);
 
 /* ------------------------------------------------------------------------
+ * Step planning on the host (no CUDA call; host arrays).
+ *
+ * pkv_partition_tokens -- the tokens per split-K partition that a call of
+ * `op` makes with this partition_tokens argument (0 = its auto rule) and
+ * max_context_len; prefix_pages is read by PKV_OP_DECODE_PREFIX only.
+ * Auto rules:
+ *   PKV_OP_DECODE         512, or 1024 when max_context_len > 4096;
+ *   PKV_OP_DECODE_FP8     1024, or 2048 when max_context_len > 16384;
+ *   PKV_OP_MULTI          2048, or 1024 when max_context_len > 4096;
+ *   PKV_OP_DECODE_PREFIX  the longest suffix (max_context_len - 16 *
+ *                         prefix_pages) rounded up to a page, kept in
+ *                         [512, 2048] (the cascade's suffix pass).
+ * An explicit partition_tokens must be a multiple of 16 in [16, 2048].
+ * Returns -1 for an invalid op or partition_tokens.
+ * -------------------------------------------------------------------- */
+typedef enum {
+  PKV_OP_DECODE = 0,        /* pkv_paged_attention_decode (and _static_ws) */
+  PKV_OP_DECODE_FP8 = 1,    /* pkv_paged_attention_decode_fp8 */
+  PKV_OP_MULTI = 2,         /* pkv_paged_attention_multi */
+  PKV_OP_DECODE_PREFIX = 3  /* pkv_paged_attention_decode_prefix (suffix pass) */
+} pkv_op;
+int pkv_partition_tokens(pkv_op op, int partition_tokens, int max_context_len, int prefix_pages);
+
+/* pkv_cow_copy_rows -- the rows each copy-on-write copy of a step must move.
+ *
+ * "PagedAttention 与 vLLM 推理加速" §3.2(3): a shared block is copied before
+ * a sharer appends into it.  Such a block is partial (a full shared block
+ * is never copied), so only its first rows hold tokens.  For each pair
+ * (src, dst) of pairs[num_pairs][2]:
+ *   copies[i] = (src, dst, rows),  rows = min over the slots s >= 0 of
+ *   slots[num_slots] with s / 16 == dst of s % 16  (16 when none),
+ * the first row this step writes into dst: rows 0 .. rows-1 hold the
+ * sequence's earlier tokens and are what pkv_kv_append_copy copies.
+ * copies: int32 [num_pairs][3], host memory the caller owns.  PKV_EINVAL
+ * for a negative count or block id, or a NULL array that must be read. */
+pkv_status pkv_cow_copy_rows(const int32_t* pairs, int num_pairs, const int64_t* slots, int num_slots,
+                             int32_t* copies);
+
+/* pkv_common_prefix_pages -- leading pages that every sequence of a batch
+ * shares and fills completely.
+ *
+ * "PagedAttention 与 vLLM 推理加速" §3.2(3): requests with one system prompt
+ * map the same physical blocks, which sit at the start of their block
+ * tables (§2.3).  *prefix_pages = the largest p such that, for every page
+ * j < p, all num_seqs tables hold one block id at column j and every
+ * context_lens[b] >= 16 (j + 1); 0 when num_seqs < 2.  block_tables: int32
+ * [num_seqs][width], context_lens: int32 [num_seqs], host memory.
+ * PKV_EINVAL for negative sizes or lengths, or NULL arrays. */
+pkv_status pkv_common_prefix_pages(const int32_t* block_tables, int num_seqs, int width,
+                                   const int32_t* context_lens, int* prefix_pages);
+
+/* pkv_cascade_prefix_pages -- the prefix pages to give
+ * pkv_paged_attention_decode_prefix for this batch, or 0 when the plain
+ * decode is the better call: the common prefix of pkv_common_prefix_pages
+ * when dtype is PKV_F16 / PKV_BF16 (the cascade's tensor-core path), at
+ * least PKV_CASCADE_MIN_SEQS sequences share it and it spans at least
+ * PKV_CASCADE_MIN_PAGES pages (below that the prefix pass and the merge
+ * cost more than reading the few shared pages once per sequence). */
+#define PKV_CASCADE_MIN_PAGES 8
+#define PKV_CASCADE_MIN_SEQS 4
+pkv_status pkv_cascade_prefix_pages(const int32_t* block_tables, int num_seqs, int width,
+                                    const int32_t* context_lens, pkv_dtype dtype, int* prefix_pages);
+
+/* ------------------------------------------------------------------------
  * Host block allocator.
  *
  * "vLLM + PagedAttention：打造高并发LLM推理引擎", "它是怎么工作的": blocks are
@@ -465,6 +533,11 @@ pkv_status pkv_alloc_append_tokens(pkv_alloc* a, int64_t seq_id, int n, int64_t*
  * All or nothing (PKV_ENOMEM if the pool cannot serve the whole step). */
 pkv_status pkv_alloc_step(pkv_alloc* a, const int64_t* seq_ids, int n, int64_t* slots,
                           int32_t* cow_pairs, int* n_cow);
+/* pkv_alloc_step, its copy pairs cut to rows by pkv_cow_copy_rows:
+ * copies[3 * n] receives *n_copies (src, dst, rows) triples in order, ready
+ * for pkv_kv_append_copy with this step's slots.  All or nothing. */
+pkv_status pkv_alloc_step_copies(pkv_alloc* a, const int64_t* seq_ids, int n, int64_t* slots,
+                                 int32_t* copies, int* n_copies);
 
 /* One sequence's table (up to cap entries), its block count and length. */
 pkv_status pkv_alloc_block_table(const pkv_alloc* a, int64_t seq_id, int32_t* out, int cap,

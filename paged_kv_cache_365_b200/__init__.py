@@ -13,4 +13,5 @@ from .api import (BLOCK_SIZE, DEFAULT_PARTITION, BlockAllocator, PagedKVCache, c
                   paged_attention_decode, paged_attention_decode_static_ws, paged_attention_decode_prefix,
                   decode_prefix_workspace_bytes, common_prefix_pages, swap_blocks, swap_blocks_check,
                   paged_attention_multi, multi_workspace_bytes, kv_append_fp8, paged_attention_decode_fp8,
-                  kv_append_copy, cow_copy_rows, selftest_bounded_wait)
+                  kv_append_copy, cow_copy_rows, selftest_bounded_wait, cascade_prefix_pages,
+                  partition_tokens)

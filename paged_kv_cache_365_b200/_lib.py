@@ -24,6 +24,9 @@ ERR_TIMEOUT = 0x10
 
 STATIC_WORKSPACE_BYTES = 16 << 20  # PKV_STATIC_WORKSPACE_BYTES
 
+# pkv_op: which call's partition rule pkv_partition_tokens applies
+OP_DECODE, OP_DECODE_FP8, OP_MULTI, OP_DECODE_PREFIX = 0, 1, 2, 3
+
 # name -> (restype, argtypes); the same list as include/pkv.h
 PROTOTYPES = {
     "pkv_status_string": (ctypes.c_char_p, [c_int]),
@@ -64,6 +67,11 @@ PROTOTYPES = {
                                           c_void_p, c_int, c_int, c_int, c_int, c_int, c_int, c_int, c_float, c_int,
                                           c_int, c_void_p, c_size_t, c_void_p]),
     "pkv_get_error": (c_int, [P(c_uint32), c_void_p]),
+    "pkv_partition_tokens": (c_int, [c_int, c_int, c_int, c_int]),
+    "pkv_cow_copy_rows": (c_int, [P(c_int32), c_int, P(c_int64), c_int, P(c_int32)]),
+    "pkv_common_prefix_pages": (c_int, [P(c_int32), c_int, c_int, P(c_int32), P(c_int)]),
+    "pkv_cascade_prefix_pages": (c_int, [P(c_int32), c_int, c_int, P(c_int32), c_int, P(c_int)]),
+    "pkv_alloc_step_copies": (c_int, [c_void_p, P(c_int64), c_int, P(c_int64), P(c_int32), P(c_int)]),
     "pkv_alloc_create": (c_int, [c_int, P(c_int32), P(c_void_p)]),
     "pkv_alloc_destroy": (None, [c_void_p]),
     "pkv_alloc_add_seq": (c_int, [c_void_p, c_int64]),

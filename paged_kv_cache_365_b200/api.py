@@ -44,28 +44,42 @@ BLOCK_SIZE = 16
 DEFAULT_PARTITION = 512
 
 
+def partition_tokens(op: int, max_context_len: int, partition: int = 0, prefix_pages: int = 0) -> int:
+    """Tokens per split-K partition that call ``op`` (``_lib.OP_*``) makes
+    with this ``partition`` argument (0 = its auto rule): the library's own
+    rule (pkv_partition_tokens)."""
+    p = int(lib.pkv_partition_tokens(int(op), int(partition), int(max_context_len), int(prefix_pages)))
+    if p < 0:
+        raise ValueError(f"invalid partition {partition} for op {op}")
+    return p
+
+
 def auto_partition(max_context_len: int) -> int:
-    """The library's partition for partition=0: 512 tokens, 1024 past 4096."""
-    return 2 * DEFAULT_PARTITION if max_context_len > 4096 else DEFAULT_PARTITION
+    """The decode's partition for partition=0 (pkv_partition_tokens)."""
+    return partition_tokens(_lib.OP_DECODE, max_context_len)
 
 
 def auto_partition_multi(max_context_len: int) -> int:
-    """The multi-token path's partition for partition=0: 2048 tokens, 1024
-    past 4096."""
-    return 2 * DEFAULT_PARTITION if max_context_len > 4096 else 4 * DEFAULT_PARTITION
+    """The multi-token path's partition for partition=0."""
+    return partition_tokens(_lib.OP_MULTI, max_context_len)
 
 
 def auto_partition_fp8(max_context_len: int) -> int:
-    """The FP8 decode's partition for partition=0: 1024 tokens, 2048 past
-    16384 (its pages are half the bytes)."""
-    return 4 * DEFAULT_PARTITION if max_context_len > 16384 else 2 * DEFAULT_PARTITION
-# a batch whose sequences share at least this many leading pages (and has at
-# least this many sequences) is decoded with the cascade (prefix read once)
-CASCADE_MIN_PAGES = 8
-CASCADE_MIN_SEQS = 4
+    """The FP8 decode's partition for partition=0."""
+    return partition_tokens(_lib.OP_DECODE_FP8, max_context_len)
+
+
 # an FP8 cache holds E4M3 codes: torch.float8_e4m3fn, or uint8 bytes
 _DT = {torch.float32: 0, torch.float16: 1, torch.bfloat16: 2, torch.float8_e4m3fn: 3, torch.uint8: 3}
 _FP8 = (torch.float8_e4m3fn, torch.uint8)
+
+
+def _i32p(a: np.ndarray):
+    return a.ctypes.data_as(ctypes.POINTER(ctypes.c_int32))
+
+
+def _i64p(a: np.ndarray):
+    return a.ctypes.data_as(ctypes.POINTER(ctypes.c_int64))
 
 
 def kv_cache_bytes(num_layers: int, num_heads: int, head_dim: int, seq_len: int, dtype_bytes: int) -> int:
@@ -233,17 +247,14 @@ def paged_attention_decode_fp8(q: torch.Tensor, k_cache: torch.Tensor, v_cache: 
 
 
 def cow_copy_rows(pairs: np.ndarray, slots: np.ndarray) -> np.ndarray:
-    """(src, dst, rows) for each copy-on-write pair of a step: rows = the
-    first row a slot of the step writes into dst (16 when none does), the
-    rows of dst that hold tokens and must be copied."""
-    p = np.asarray(pairs, dtype=np.int64).reshape(-1, 2)
-    s = np.asarray(slots, dtype=np.int64)
-    s = s[s >= 0]
-    out = np.empty((p.shape[0], 3), dtype=np.int32)
-    for i, (src, dst) in enumerate(p):
-        hit = s[s // BLOCK_SIZE == dst] % BLOCK_SIZE
-        out[i] = (src, dst, int(hit.min()) if hit.size else BLOCK_SIZE)
-    return out
+    """(src, dst, rows) for each copy-on-write pair of a step
+    (pkv_cow_copy_rows): rows = the first row a slot of the step writes into
+    dst (16 when none does), the rows of dst that hold tokens."""
+    p = np.ascontiguousarray(np.asarray(pairs, dtype=np.int32).reshape(-1, 2))
+    s = np.ascontiguousarray(np.asarray(slots, dtype=np.int64).reshape(-1))
+    out = np.empty((max(p.shape[0], 1), 3), dtype=np.int32)
+    check(lib.pkv_cow_copy_rows(_i32p(p), p.shape[0], _i64p(s), s.shape[0], _i32p(out)), "pkv_cow_copy_rows")
+    return out[:p.shape[0]]
 
 
 def kv_append_copy(k_new: torch.Tensor, v_new: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
@@ -310,20 +321,35 @@ def decode_prefix_workspace_bytes(num_seqs: int, num_q_heads: int, head_dim: int
                                                      prefix_pages, partition))
 
 
+def _tables_lens(block_tables, context_lens):
+    bt = np.ascontiguousarray(np.asarray(block_tables, dtype=np.int32))
+    if bt.ndim != 2:
+        raise ValueError("block_tables must be [B, W]")
+    lens = np.ascontiguousarray(np.asarray(context_lens, dtype=np.int32).reshape(-1))
+    if lens.shape[0] != bt.shape[0]:
+        raise ValueError("context_lens must be [B]")
+    return bt, lens
+
+
 def common_prefix_pages(block_tables: np.ndarray, context_lens: np.ndarray) -> int:
-    """Number of leading pages that every sequence of the batch shares (same
-    physical blocks) and fills completely: the prefix the cascade decode
-    can read once.  Host arrays: tables [B, W], lengths [B]."""
-    bt = np.asarray(block_tables)
-    lens = np.asarray(context_lens)
-    if bt.shape[0] < 2:
-        return 0
-    full = int(lens.min()) // BLOCK_SIZE
-    full = min(full, bt.shape[1])
-    if full == 0:
-        return 0
-    same = np.all(bt[:, :full] == bt[0:1, :full], axis=0)
-    return int(full if same.all() else np.argmin(same))
+    """Leading pages that every sequence of the batch shares (same physical
+    blocks) and fills completely (pkv_common_prefix_pages).  Host arrays:
+    tables [B, W], lengths [B]."""
+    bt, lens = _tables_lens(block_tables, context_lens)
+    n = ctypes.c_int(0)
+    check(lib.pkv_common_prefix_pages(_i32p(bt), bt.shape[0], bt.shape[1], _i32p(lens), ctypes.byref(n)),
+          "pkv_common_prefix_pages")
+    return int(n.value)
+
+
+def cascade_prefix_pages(block_tables: np.ndarray, context_lens: np.ndarray, dtype: torch.dtype) -> int:
+    """The shared prefix pages the cascade decode should read once, or 0 when
+    the plain decode is the better call (pkv_cascade_prefix_pages)."""
+    bt, lens = _tables_lens(block_tables, context_lens)
+    n = ctypes.c_int(0)
+    check(lib.pkv_cascade_prefix_pages(_i32p(bt), bt.shape[0], bt.shape[1], _i32p(lens), _DT[dtype],
+                                       ctypes.byref(n)), "pkv_cascade_prefix_pages")
+    return int(n.value)
 
 
 def paged_attention_decode_prefix(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
@@ -425,14 +451,6 @@ def selftest_bounded_wait(limit_cycles: int, stream=None, device=None) -> None:
 # ---------------------------------------------------------------------------
 # host allocator
 # ---------------------------------------------------------------------------
-def _i32p(a: np.ndarray):
-    return a.ctypes.data_as(ctypes.POINTER(ctypes.c_int32))
-
-
-def _i64p(a: np.ndarray):
-    return a.ctypes.data_as(ctypes.POINTER(ctypes.c_int64))
-
-
 class BlockAllocator:
     """The library's host block allocator (FIFO free list, refcounts, CoW)."""
 
@@ -487,6 +505,18 @@ class BlockAllocator:
         check(lib.pkv_alloc_step(self._h, _i64p(ids), n, _i64p(slots), _i32p(pairs), ctypes.byref(nc)),
               "pkv_alloc_step")
         return slots[:n], pairs[:2 * nc.value].reshape(-1, 2)
+
+    def step_copies(self, sids: Iterable[int]) -> Tuple[np.ndarray, np.ndarray]:
+        """``step`` with the copy pairs cut to rows (pkv_alloc_step_copies):
+        slots [n] and (src, dst, rows) copies [k, 3] for kv_append_copy."""
+        ids = np.ascontiguousarray(list(sids), dtype=np.int64)
+        n = ids.shape[0]
+        slots = np.empty(max(n, 1), dtype=np.int64)
+        copies = np.empty((max(n, 1), 3), dtype=np.int32)
+        nc = ctypes.c_int()
+        check(lib.pkv_alloc_step_copies(self._h, _i64p(ids), n, _i64p(slots), _i32p(copies), ctypes.byref(nc)),
+              "pkv_alloc_step_copies")
+        return slots[:n], copies[:nc.value]
 
     def block_table(self, sid: int) -> Tuple[List[int], int]:
         nb, ln = ctypes.c_int(), ctypes.c_int64()
@@ -880,9 +910,8 @@ class PagedKVCache:
         """Host plan (allocator) + device step; returns the output on q's device."""
         slots, pairs, tables, lens = self.plan_step(seq_ids)
         max_ctx = int(lens.max()) if len(lens) else 0
-        pp = common_prefix_pages(tables, lens) if (self.dtype != torch.float32 and self.fp8 is None) else 0
-        prefix = (torch.from_numpy(np.ascontiguousarray(tables[0, :pp]))
-                  if pp >= CASCADE_MIN_PAGES and len(lens) >= CASCADE_MIN_SEQS else None)
+        pp = cascade_prefix_pages(tables, lens, self.dtype) if self.fp8 is None else 0
+        prefix = torch.from_numpy(np.ascontiguousarray(tables[0, :pp])) if pp else None
         copies = cow_copy_rows(pairs, slots)  # copy only the rows that hold tokens
         out = self.run_step(torch.from_numpy(slots), torch.from_numpy(copies),
                             torch.from_numpy(np.ascontiguousarray(tables)), torch.from_numpy(lens), max_ctx,

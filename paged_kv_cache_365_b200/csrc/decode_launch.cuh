@@ -115,16 +115,19 @@ pkv_status launch_decode(const pkv::DecodeArgs& a, cudaStream_t st) {
   return PKV_OK;
 }
 
+// A driver API function, reached through the runtime (nullptr when absent).
+void* driver_entry_point(const char* name) {
+  void* p = nullptr;
+  cudaDriverEntryPointQueryResult q;
+  if (cudaGetDriverEntryPoint(name, &p, cudaEnableDefault, &q) != cudaSuccess || q != cudaDriverEntryPointSuccess)
+    return nullptr;
+  return p;
+}
+
 // ---- tensor-core path (fp16 / bf16): tensor-map TMA + mma.sync ----------
 PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = []() -> PFN_cuTensorMapEncodeTiled_v12000 {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) != cudaSuccess ||
-        q != cudaDriverEntryPointSuccess)
-      return nullptr;
-    return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
-  }();
+  static PFN_cuTensorMapEncodeTiled_v12000 fn =
+      reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(driver_entry_point("cuTensorMapEncodeTiled"));
   return fn;
 }
 

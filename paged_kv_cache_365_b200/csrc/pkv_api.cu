@@ -79,6 +79,11 @@ pkv_status launch_multi(const pkv::MultiArgs& a, const void* k_cache, const void
 int resolve_multi_partition(int p, long long max_ctx) {
   return resolve_partition(p != 0 ? p : (max_ctx > 4096 ? 1024 : 2048), max_ctx);
 }
+// Auto partition of the FP8 decode: twice the 16-bit one's tokens (half the
+// bytes a page): 1024, or 2048 past 16384 tokens.
+int resolve_fp8_partition(int p, long long max_ctx) {
+  return resolve_partition(p != 0 ? p : (max_ctx > 16384 ? 2048 : 1024), max_ctx);
+}
 int multi_ntiles(long long rows) { return rows <= 8 ? 1 : 2; }
 int multi_rows_warps(long long rows) { return rows <= 16 ? 0 : rows <= 24 ? 3 : 4; }
 #ifndef PKV_FA_ABOVE_ROWS
@@ -440,6 +445,19 @@ pkv_status pkv_paged_attention_decode(void* out, const void* q, const void* k_ca
   return PKV_EINVAL;
 }
 
+int pkv_partition_tokens(pkv_op op, int partition_tokens, int max_context_len, int prefix_pages) {
+  if (max_context_len < 0) return -1;
+  switch (op) {
+    case PKV_OP_DECODE: return resolve_partition(partition_tokens, max_context_len);
+    case PKV_OP_DECODE_FP8: return resolve_fp8_partition(partition_tokens, max_context_len);
+    case PKV_OP_MULTI: return resolve_multi_partition(partition_tokens, max_context_len);
+    case PKV_OP_DECODE_PREFIX:
+      if (prefix_pages <= 0) return -1;
+      return resolve_prefix_partition(partition_tokens, max_context_len, prefix_pages);
+  }
+  return -1;
+}
+
 size_t pkv_decode_prefix_workspace_bytes(int num_seqs, int num_q_heads, int head_dim, int max_context_len,
                                          int prefix_pages, int partition_tokens) {
   const int part = resolve_prefix_partition(partition_tokens, max_context_len, prefix_pages);
@@ -541,21 +559,54 @@ static __device__ __align__(256) unsigned char g_static_workspace[PKV_STATIC_WOR
 
 constexpr int kMaxDevices = 64;
 std::mutex g_static_ws_mutex;
-void* g_static_ws_addr[kMaxDevices] = {};
+// per device: the id of the context the address was looked up in, and the
+// address
+struct StaticWsEntry {
+  unsigned long long ctx_id;
+  void* addr;
+};
+StaticWsEntry g_static_ws[kMaxDevices] = {};
+
+// Unique id of the calling thread's current context (0 when none is bound).
+// Ids are never reused within a process, unlike context handles.  Driver
+// API calls reached through the runtime's entry-point query, so the library
+// links only the runtime.
+unsigned long long current_context_id() {
+  using GetCurrent = CUresult (*)(CUcontext*);
+  using GetId = CUresult (*)(CUcontext, unsigned long long*);
+  static GetCurrent get_current = reinterpret_cast<GetCurrent>(driver_entry_point("cuCtxGetCurrent"));
+  static GetId get_id = reinterpret_cast<GetId>(driver_entry_point("cuCtxGetId"));
+  CUcontext c = nullptr;
+  unsigned long long id = 0;
+  if (get_current == nullptr || get_id == nullptr || get_current(&c) != CUDA_SUCCESS || c == nullptr ||
+      get_id(c, &id) != CUDA_SUCCESS)
+    return 0;
+  return id;
+}
 
 // Device address of g_static_workspace on the current device.  In host code
-// the array's name only stands in for it, so the address is looked up once
-// per device (with that device current) and kept.
+// the array's name only stands in for it, so the address is looked up with
+// the device current and kept, keyed by the device and the id of its current
+// context: when the caller has destroyed and re-created the device's context
+// (for example after cudaDeviceReset), the module is loaded anew and the
+// address is looked up again.
 pkv_status static_workspace_address(void** addr) {
   int dev = -1;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return PKV_ECUDA;
   std::lock_guard<std::mutex> lock(g_static_ws_mutex);
-  if (g_static_ws_addr[dev] == nullptr) {
+  StaticWsEntry& e = g_static_ws[dev];
+  unsigned long long id = current_context_id();
+  if (e.addr == nullptr || id == 0 || e.ctx_id != id) {
+    // (a thread with no context bound yet gets the device's primary context
+    // from this runtime call; its id is read after it)
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, g_static_workspace) != cudaSuccess || p == nullptr) return PKV_ECUDA;
-    g_static_ws_addr[dev] = p;
+    id = current_context_id();
+    if (id == 0) return PKV_ECUDA;
+    e.ctx_id = id;
+    e.addr = p;
   }
-  *addr = g_static_ws_addr[dev];
+  *addr = e.addr;
   return PKV_OK;
 }
 
@@ -712,8 +763,8 @@ pkv_status pkv_paged_attention_decode_fp8(void* out, const void* q, const void* 
     return PKV_EINVAL;
   pkv::DecodeArgs a{};
   long long P = 0;
-  // auto partition: twice the 16-bit one's tokens (half the bytes a page)
-  if (partition_tokens == 0) partition_tokens = max_context_len > 16384 ? 2048 : 1024;
+  partition_tokens = resolve_fp8_partition(partition_tokens, max_context_len);
+  if (partition_tokens < 0) return PKV_EINVAL;
   const pkv_status st0 = prepare_decode(out, q, k_cache, v_cache, block_tables, max_blocks_per_seq, context_lens,
                                         max_context_len, num_seqs, num_q_heads, num_kv_heads, head_dim, num_blocks,
                                         scale, partition_tokens, q_dtype, &a, &P);
