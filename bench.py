@@ -10,6 +10,10 @@ same planned step is replayed every iteration (its copies and appends are
 idempotent).
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+      (default: the JSON line is quoted on the long-context workload -- the
+      largest single-GPU configuration -- and carries a ``per_config``
+      object with the same figures for tiny, llama7b, gqa8b and prefix13b,
+      each timed with the same --steps / --warmup)
   python bench.py --impl reference ...   (the fp64 CPU oracle, bounded sample)
   python bench.py --row swap ...         (preemption by swapping: one step =
       swap a quarter of the batch out to pinned host memory and back in;
@@ -25,6 +29,7 @@ KV bytes / the slowest rank's time.  Prints one JSON line on rank 0.
 from __future__ import annotations
 
 import argparse
+import gc
 import hashlib
 import json
 import math
@@ -48,6 +53,11 @@ SWAP_METRIC = "block swap device<->pinned host (preempt + resume): GB/s over the
 MULTI_METRIC = ("paged multi-token attention (several new tokens per sequence, causal): KV-cache HBM GB/s "
                 "(% of peak), query-tokens/s")
 UNIT = "GB/s"
+# the headline workload of the default run (the largest single-GPU
+# configuration: 8 sequences of 32k-131k tokens, 2.2 GB of K/V a step) and
+# the workloads reported beside it in ``per_config``
+DEFAULT_WORKLOAD = "long"
+PER_CONFIG = ["tiny", "llama7b", "gqa8b", "prefix13b"]
 FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_TFLOPS = 1400.0
 STORAGE = {"f32": 4, "f16": 2, "bf16": 2}
@@ -252,14 +262,22 @@ def device_values(wl, seed, device):
     return out
 
 
-def run_cuda(args, rank, world, local_rank):
+ROOFLINE_LEG_S = 0.5  # least device time of the decode-call leg (several clock samples)
+
+
+def run_cuda(args, rank, world, local_rank, workload=None, graph=None):
+    """One workload's decode step: the timed K-step region, the decode call
+    alone (event-bracketed, at least ROOFLINE_LEG_S of calls) and the same
+    step end to end through PagedKVCache.run_step.  ``workload`` / ``graph``
+    override args.workload / args.graph."""
     import torch
     from paged_kv_cache_365_b200.replay import build_step
     import paged_kv_cache_365_b200 as pkv
 
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
-    wl = workloads.named(args.workload, replica_seed(args.seed, rank))
+    use_graph = bool(args.graph if graph is None else graph)
+    wl = workloads.named(workload or args.workload, replica_seed(args.seed, rank))
     vals = device_values(wl, replica_seed(args.seed, rank), dev)
     st = build_step(wl, {}, dev, device_values=vals)
     del vals
@@ -270,15 +288,16 @@ def run_cuda(args, rank, world, local_rank):
     n_pairs = int(st["cow_pairs"].shape[0])
     ws = cache.workspace(pkv.decode_workspace_bytes(B, Hq, D, max_ctx, args.partition))
     out = torch.empty_like(st["q"])
-    auto = pkv.api.auto_partition_fp8 if args.kv_fp8 else pkv.api.auto_partition
-    P = max(1, math.ceil(max_ctx / (args.partition or auto(max_ctx))))
+    part_tokens = pkv.partition_tokens(pkv._lib.OP_DECODE_FP8 if args.kv_fp8 else pkv._lib.OP_DECODE, max_ctx,
+                                       args.partition)
+    P = max(1, math.ceil(max_ctx / part_tokens))
     scale = 1.0 / math.sqrt(D)
     # a batch that shares leading blocks is decoded with the cascade (the
-    # shared prefix is read once per kv-head)
-    pp = pkv.common_prefix_pages(st["host"]["block_tables"], st["host"]["context_lens"])
-    use_cascade = (wl.dtype != "f32" and pp >= pkv.api.CASCADE_MIN_PAGES and B >= pkv.api.CASCADE_MIN_SEQS
-                   and not args.no_cascade and not args.kv_fp8)
-    args._cascade = use_cascade
+    # shared prefix is read once per kv-head) when the library says so
+    pp = pkv.cascade_prefix_pages(st["host"]["block_tables"], st["host"]["context_lens"], cache.dtype)
+    use_cascade = pp > 0 and not args.no_cascade and not args.kv_fp8
+    if use_cascade:
+        part_tokens = pkv.partition_tokens(pkv._lib.OP_DECODE_PREFIX, max_ctx, args.partition, pp)
     fp8 = bool(args.kv_fp8)
     if fp8:
         if wl.dtype == "f32":
@@ -369,7 +388,7 @@ def run_cuda(args, rank, world, local_rank):
         decode()
 
     run_step = eager_step
-    if args.graph:
+    if use_graph:
         # one whole step captured once, replayed every iteration
         for _ in range(3):
             eager_step()
@@ -393,27 +412,31 @@ def run_cuda(args, rank, world, local_rank):
     torch.cuda.synchronize()
 
     K = args.steps
-    # (1) the step, K times back to back: events only around the whole run
-    #     (an event between two kernels would break their overlap)
-    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with ClockSampler(local_rank) as clocks:
+        # (1) the step, K times back to back: events only around the whole
+        #     run (an event between two kernels would break their overlap)
+        t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         t0.record(stream)
         for i in range(K):
             run_step()
         t1.record(stream)
         torch.cuda.synchronize()
-    barrier()
-    torch.cuda.synchronize()
-    total_ms = t0.elapsed_time(t1)
-    # (2) the decode call alone, each launch bracketed by events (roofline)
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(K)]
-    for i in range(K):
-        ev[i][0].record(stream)
-        decode()
-        ev[i][1].record(stream)
-    torch.cuda.synchronize()
-    dec_ms = [ev[i][0].elapsed_time(ev[i][1]) for i in range(K)]
-    dec_avg_ms = sum(dec_ms) / K
+        barrier()
+        torch.cuda.synchronize()
+        total_ms = t0.elapsed_time(t1)
+        # (2) the decode call alone, each launch bracketed by events
+        #     (roofline), for at least ROOFLINE_LEG_S of device time; every
+        #     rank makes the same number of calls
+        n_roof = max(K, int(math.ceil(ROOFLINE_LEG_S * 1e3 / max(total_ms / K, 1e-3))))
+        n_roof = int(max_over_ranks([n_roof], world, dev)[0])
+        ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(n_roof)]
+        for i in range(n_roof):
+            ev[i][0].record(stream)
+            decode()
+            ev[i][1].record(stream)
+        torch.cuda.synchronize()
+    dec_ms = [ev[i][0].elapsed_time(ev[i][1]) for i in range(n_roof)]
+    dec_avg_ms = sum(dec_ms) / n_roof
     barrier()
 
     # e2e: the same step with its inputs in pinned host memory, copied in
@@ -452,9 +475,10 @@ def run_cuda(args, rank, world, local_rank):
 
     total_ms, e2e_ms, dec_avg_ms = max_over_ranks([total_ms, e2e_ms, dec_avg_ms], world, dev)
 
-    res = dict(wl=wl, K=K, total_ms=total_ms, e2e_ms=e2e_ms, dec_avg_ms=dec_avg_ms,
+    res = dict(wl=wl, K=K, total_ms=total_ms, e2e_ms=e2e_ms, dec_avg_ms=dec_avg_ms, roof_calls=n_roof,
                launches=launches_per_step * K, h2d=h2d, d2h=d2h, clocks=clocks.summary(), P=P,
-               n_pairs=n_pairs, cache=cache, st=st, cascade_pages=pp if use_cascade else 0)
+               partition_tokens=part_tokens, n_pairs=n_pairs, cascade_pages=pp if use_cascade else 0,
+               graph=use_graph, cascade_overlap=bool(use_cascade and args.cascade_overlap))
     return res
 
 
@@ -483,7 +507,8 @@ def run_multi(args, rank, world, local_rank):
     out = torch.empty_like(st["q"])
     scale = 1.0 / math.sqrt(wl.D)
     n_pairs = int(st["cow_pairs"].shape[0])
-    P = max(1, math.ceil(max_ctx / (args.partition or pkv.api.auto_partition_multi(max_ctx))))
+    part_tokens = pkv.partition_tokens(pkv._lib.OP_MULTI, max_ctx, args.partition)
+    P = max(1, math.ceil(max_ctx / part_tokens))
 
     def pre():
         if n_pairs:
@@ -552,7 +577,8 @@ def run_multi(args, rank, world, local_rank):
     att_bytes = kv + 2 * T * wl.Hq * wl.D * es + int(sum(-(-int(n) // 16) for n in lens)) * 4 + 8 * wl.B + 4
     launches = (1 + (1 if n_pairs else 0) + 1 + (1 if P > 1 else 0)) * K
     return dict(wl=wl, K=K, T=T, kv=kv, att_bytes=att_bytes, total_ms=total_ms, att_ms=att_ms, e2e_ms=e2e_ms,
-                h2d=h2d, d2h=d2h, clocks=clocks.summary(), P=P, launches=launches, lens=lens)
+                h2d=h2d, d2h=d2h, clocks=clocks.summary(), P=P, launches=launches, lens=lens,
+                partition_tokens=part_tokens)
 
 
 def multi_cpu_baseline(wl, n_new, budget_s=10.0, seed=0):
@@ -606,8 +632,7 @@ def multi_line(args, r, world):
                    "num_kv_heads": wl.Hkv, "head_dim": wl.D, "block_size": 16,
                    "context_lens": {"min": int(np.min(r["lens"])), "max": int(np.max(r["lens"])),
                                     "sum": int(np.sum(r["lens"]))},
-                   "partition_tokens": args.partition or ("auto (%d)" % auto_partition(int(np.max(r["lens"])), False, True)),
-                   "partitions_max": r["P"], "seed": args.seed,
+                   "seed": args.seed,
                    "parallelism": f"replicas{args.gpus}" if args.gpus > 1 else "single-gpu",
                    "l2": "inputs larger than L2 (no flush)" if r["kv"] > 126e6 else "inputs fit in L2"},
         "us_per_step": 1e3 * r["total_ms"] / K,
@@ -618,6 +643,8 @@ def multi_line(args, r, world):
                 "h2d_bytes_per_step": r["h2d"], "d2h_bytes_per_step": r["d2h"],
                 "us_per_step": 1e3 * r["e2e_ms"] / K},
         "gpu_launches": r["launches"],
+        "launch": {"partition_tokens": r.get("partition_tokens"), "partition_auto": not args.partition,
+                   "partitions_max": r["P"]},
         "roofline": {"kernel": "paged_multi (partition + merge kernels)", **roof,
                      "peak_kind": (tpeak_kind if roof["bound"] == "tensor" else
                                    f"{peak_kind} (MEASURED_PEAKS hbm_gbs)" if peak_kind == "measured" else "fallback"),
@@ -856,37 +883,30 @@ def cpu_baseline(wl, budget_s=12.0, seed=0):
                       f"{nbytes / 1e6:.1f} MB of K/V, fp64 numpy, BLAS limited to 1 thread, {secs:.1f} s"}
 
 
-def auto_partition(max_ctx: int, fp8: bool, multi: bool = False) -> int:
-    """The library's partition for partition=0 (pkv.h): 512 tokens, 1024 past
-    4096; for the FP8 decode 1024, 2048 past 16384; for the multi-token path
-    2048, 1024 past 4096."""
-    if fp8:
-        return 2048 if max_ctx > 16384 else 1024
-    if multi:
-        return 1024 if max_ctx > 4096 else 2048
-    return 1024 if max_ctx > 4096 else 512
-
-
-def config_of(wl, args, P):
+def config_of(wl, args):
+    """The workload the line is quoted on (the same object on both arms)."""
     return {"workload": wl.name, "global_batch": wl.B, "num_q_heads": wl.Hq, "num_kv_heads": wl.Hkv,
             "head_dim": wl.D, "block_size": 16, "num_blocks": wl.num_blocks,
             "context_lens": {"min": int(wl.context_lens.min()), "max": int(wl.context_lens.max()),
                              "sum": int(wl.context_lens.astype(np.int64).sum())},
-            "partition_tokens": args.partition or ("auto (%d)" % auto_partition(int(wl.context_lens.max()),
-                                                                                getattr(args, "kv_fp8", False))),
-            "partitions_max": P, "seed": args.seed,
-            "cuda_graph": bool(getattr(args, "graph", False)),
-            "cascade": None if not getattr(args, "_cascade", False) else
-            ("prefix pass on a second stream beside copies + append" if args.cascade_overlap else "one launch"),
+            "seed": args.seed,
             "parallelism": f"replicas{args.gpus}" if args.gpus > 1 else "single-gpu",
             "l2": "inputs larger than L2 (no flush)" if kv_bytes(wl, True) > 126e6 else "inputs fit in L2"}
+
+
+def launch_of(args, r):
+    """How the CUDA path ran the workload (partition, graph, cascade)."""
+    return {"partition_tokens": r["partition_tokens"], "partition_auto": not args.partition,
+            "partitions_max": r["P"], "cuda_graph": r["graph"],
+            "cascade": None if not r["cascade_pages"] else
+            ("prefix pass on a second stream beside copies + append" if r["cascade_overlap"] else "one launch")}
 
 
 def run_reference(args, rank, world):
     """The oracle timed on the host cores, every step a bounded sample."""
     if rank != 0:
         return
-    wl = workloads.named(args.workload, args.seed)
+    wl = workloads.named(args.workload or DEFAULT_WORKLOAD, args.seed)
     if getattr(args, "row", "step") == "multi":
         b = multi_cpu_baseline(wl, args.new_tokens, budget_s=min(60.0, 0.5 * (args.steps + args.warmup)),
                                seed=args.seed)
@@ -936,7 +956,7 @@ def run_reference(args, rank, world):
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * tot_s / max(1, args.steps),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-            "data": "synthetic", "config": config_of(wl, args, 0),
+            "data": "synthetic", "config": config_of(wl, args),
             "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle", "sample": sample},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
@@ -948,7 +968,11 @@ def main(argv=None):
     ap.add_argument("--steps", type=int, default=None, help="timed steps (default 2000; 20 with --row swap)")
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", default="llama7b", choices=sorted(workloads.NAMED))
+    ap.add_argument("--workload", default=None, choices=sorted(workloads.NAMED),
+                    help=f"one workload alone (default: {DEFAULT_WORKLOAD} headline + per_config entries for "
+                         f"{', '.join(PER_CONFIG)}; --row swap / multi default to llama7b)")
+    ap.add_argument("--no-per-config", action="store_true",
+                    help="the headline workload alone (no per_config entries)")
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--partition", type=int, default=0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -969,6 +993,8 @@ def main(argv=None):
     args = ap.parse_args(argv)
     if args.steps is None:
         args.steps = 20 if args.row == "swap" else 2000
+    if args.workload is None and args.row != "step":
+        args.workload = "llama7b"
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
 
@@ -999,12 +1025,35 @@ def main(argv=None):
         if rank == 0:
             print(json.dumps(swap_line(args, r, world)), flush=True)
         return 0
-    r = run_cuda(args, rank, world, local_rank)
+    headline = args.workload or DEFAULT_WORKLOAD
+    others = [] if (args.workload or args.no_per_config) else [w for w in PER_CONFIG if w != headline]
+    if args.kv_fp8:  # an FP8 cache holds 16-bit workloads' values only
+        others = [w for w in others if workloads.named(w, args.seed).dtype != "f32"]
+    r = run_cuda(args, rank, world, local_rank, workload=headline)
+    per = {}
+    for name in others:
+        gc.collect()
+        torch.cuda.empty_cache()
+        # the tiny batch (319 KB of K/V) is launch-bound: its step runs as one
+        # captured CUDA graph
+        rr = run_cuda(args, rank, world, local_rank, workload=name, graph=True if name == "tiny" else None)
+        per[name] = config_entry(args, rr, world)
     if world > 1:
         torch.distributed.destroy_process_group()
     if rank != 0:
         return 0
+    line = step_line(args, r, world)
+    if per:
+        line["per_config"] = per
+    if world == 1 and not args.no_cpu_baseline and not args.kv_fp8:
+        line["cpu_baseline"] = cpu_baseline(r["wl"], seed=args.seed)
+    print(json.dumps(line), flush=True)
+    return 0
 
+
+def step_figures(args, r, world):
+    """The decode step's figures from one run_cuda record: throughput, % of
+    the measured HBM peak on unique bytes, the decode call's roofline, e2e."""
     wl = r["wl"]
     peak, peak_kind = measured_peak()
     K = r["K"]
@@ -1012,15 +1061,15 @@ def main(argv=None):
     fp8 = bool(args.kv_fp8)
     kv_unique = kv_bytes(wl, True, fp8)
     kv_logical = kv_bytes(wl, False, fp8)
-    value = job_throughput(kv_logical, world, K, r["total_ms"] / 1e3)
     dec_bytes = decode_algorithmic_bytes(wl, unique=True, fp8=fp8)
     achieved = dec_bytes / (r["dec_avg_ms"] / 1e3) / 1e9
     e2e_step_s = r["e2e_ms"] / 1e3 / K
-    line = {
-        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": args.warmup,
-        "ms_per_step": r["total_ms"] / K, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": wl.dtype, "data": "synthetic (seeded N(0,1) q/K/V on the device, seeded lengths and placement)",
-        "config": config_of(wl, args, r["P"]),
+    kernel = ("paged_decode cascade (prefix/suffix kernel + merge kernel)" if r["cascade_pages"]
+              else "paged_decode_fp8 (partition + merge kernels)" if fp8
+              else "paged_decode (partition + merge kernels)")
+    return {
+        "value": job_throughput(kv_logical, world, K, r["total_ms"] / 1e3),
+        "ms_per_step": r["total_ms"] / K,
         "us_per_step": 1e3 * r["total_ms"] / K,
         "seq_steps_per_s": world * wl.B / step_s,
         "pct_hbm_peak": 100.0 * (world * kv_unique / step_s / 1e9) / (peak * world),
@@ -1030,20 +1079,38 @@ def main(argv=None):
                 "h2d_bytes_per_step": r["h2d"], "d2h_bytes_per_step": r["d2h"],
                 "us_per_step": 1e6 * e2e_step_s},
         "gpu_launches": r["launches"],
+        "launch": launch_of(args, r),
         "cascade_prefix_pages": r["cascade_pages"],
-        "kv_cache": "e4m3 (FP8) codes, scale %.6g for K and V" % FP8_SCALE if fp8 else wl.dtype,
-        "roofline": {"kernel": ("paged_decode cascade (prefix/suffix kernel + merge kernel)" if r["cascade_pages"]
-                                else "paged_decode_fp8 (partition + merge kernels)" if fp8
-                                else "paged_decode (partition + merge kernels)"), "bound": "hbm",
-                     "achieved": achieved, "peak": peak, "peak_kind": f"{peak_kind} (MEASURED_PEAKS hbm_gbs)"
-                     if peak_kind == "measured" else "fallback", "unit": "GB/s", "frac": achieved / peak,
-                     "traffic": None if fp8 else recorded_traffic(wl.name), "algorithmic_bytes_per_launch": dec_bytes,
-                     "avg_launch_us": 1e3 * r["dec_avg_ms"]},
+        "roofline": {"kernel": kernel, "bound": "hbm", "achieved": achieved, "peak": peak,
+                     "peak_kind": f"{peak_kind} (MEASURED_PEAKS hbm_gbs)" if peak_kind == "measured" else "fallback",
+                     "unit": "GB/s", "frac": achieved / peak,
+                     "traffic": None if fp8 else recorded_traffic(wl.name),
+                     "algorithmic_bytes_per_launch": dec_bytes, "avg_launch_us": 1e3 * r["dec_avg_ms"],
+                     "calls_timed": r["roof_calls"]},
     }
-    if world == 1 and not args.no_cpu_baseline and not fp8:
-        line["cpu_baseline"] = cpu_baseline(wl, seed=args.seed)
-    print(json.dumps(line), flush=True)
-    return 0
+
+
+def config_entry(args, r, world):
+    """One workload's entry of ``per_config``."""
+    wl = r["wl"]
+    f = step_figures(args, r, world)
+    return {"config": config_of(wl, args), "dtype": wl.dtype, "unit": UNIT, "steps": r["K"], **f}
+
+
+def step_line(args, r, world):
+    """The contract's JSON line for the decode step on one workload."""
+    wl = r["wl"]
+    f = step_figures(args, r, world)
+    line = {
+        "metric": METRIC, "value": f.pop("value"), "unit": UNIT, "n_gpus": world, "steps": r["K"],
+        "warmup": args.warmup, "ms_per_step": f.pop("ms_per_step"), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": wl.dtype,
+        "data": "synthetic (seeded N(0,1) q/K/V on the device, seeded lengths and placement)",
+        "config": config_of(wl, args),
+        "kv_cache": "e4m3 (FP8) codes, scale %.6g for K and V" % FP8_SCALE if args.kv_fp8 else wl.dtype,
+    }
+    line.update(f)
+    return line
 
 
 if __name__ == "__main__":

@@ -38,25 +38,81 @@ def test_warmup_floor():
     assert out.returncode != 0 and "warmup" in out.stderr
 
 
-def test_bench_reports_the_library_auto_partitions():
-    """bench.py names the partition the library picks for partition=0 (its
-    own copy of the rule, so the reference arm needs no CUDA library)."""
-    import bench
+def test_library_partition_rule_and_workspace_sizes():
+    """pkv_partition_tokens (the one copy of the auto rules, read by the
+    binding and the bench) against the rules pkv.h states, and the workspace
+    sizes that follow from it."""
     import paged_kv_cache_365_b200 as pkv
-    for n in (1, 512, 4096, 4097, 16384, 16385, 131072):
-        assert bench.auto_partition(n, False) == pkv.api.auto_partition(n)
-        assert bench.auto_partition(n, True) == pkv.api.auto_partition_fp8(n)
-        assert bench.auto_partition(n, False, True) == pkv.api.auto_partition_multi(n)
-    # the 16-bit rule is also the one the workspace size follows
+    from paged_kv_cache_365_b200 import _lib
+    pt = pkv.partition_tokens
+    for n in (1, 512, 4096):
+        assert pt(_lib.OP_DECODE, n) == 512
+        assert pt(_lib.OP_MULTI, n) == 2048
+    for n in (4097, 16384, 131072):
+        assert pt(_lib.OP_DECODE, n) == 1024
+        assert pt(_lib.OP_MULTI, n) == 1024
+    for n in (1, 16384):
+        assert pt(_lib.OP_DECODE_FP8, n) == 1024
+    assert pt(_lib.OP_DECODE_FP8, 16385) == 2048
+    # cascade suffix pass: longest suffix rounded up to a page, in [512, 2048]
+    assert pt(_lib.OP_DECODE_PREFIX, 1024 + 100, 0, 64) == 512
+    assert pt(_lib.OP_DECODE_PREFIX, 1024 + 600, 0, 64) == 608
+    assert pt(_lib.OP_DECODE_PREFIX, 1024 + 5000, 0, 64) == 2048
+    for op in (_lib.OP_DECODE, _lib.OP_DECODE_FP8, _lib.OP_MULTI):
+        assert pt(op, 9000, 48) == 48          # an explicit partition is kept
+        for bad in (8, 17, 4096):
+            with pytest.raises(ValueError):
+                pt(op, 9000, bad)
+    with pytest.raises(ValueError):
+        pt(_lib.OP_DECODE_PREFIX, 2000, 0, 0)   # the cascade needs a prefix
+    with pytest.raises(ValueError):
+        pt(7, 2000)
+    # the workspaces follow the rule
     B, Hq, D = 3, 8, 128
     for n in (700, 3000, 5000, 9000):
-        P = -(-n // pkv.api.auto_partition(n))
-        assert pkv.decode_workspace_bytes(B, Hq, D, n, 0) == B * Hq * P * (D + 2) * 4
-        # the multi-token path's workspace follows its own rule (T query rows)
+        P = -(-n // pt(_lib.OP_DECODE, n))
+        assert pkv.decode_workspace_bytes(B, Hq, D, n, 0) == (0 if P <= 1 else B * Hq * P * (D + 2) * 4)
         T = 7
-        Pm = -(-n // pkv.api.auto_partition_multi(n))
+        Pm = -(-n // pt(_lib.OP_MULTI, n))
         want = 0 if Pm <= 1 else -(-(T * Hq * Pm * D * 4) // 16) * 16 + T * Hq * Pm * 8
         assert pkv.multi_workspace_bytes(T, Hq, D, n, 0) == want
+
+
+def test_step_line_builds_the_contract_json():
+    """step_line and the per_config entries from a timing record, without a
+    GPU: the contract's keys, the roofline arithmetic, the e2e bytes."""
+    import argparse
+    import bench
+    import workloads
+    wl = workloads.named("llama7b", 0)
+    r = dict(wl=wl, K=20, total_ms=20 * 0.18, e2e_ms=20 * 0.19, dec_avg_ms=0.175, roof_calls=2800,
+             launches=60, h2d=1606400, d2h=524288, clocks={"sm_mhz": 1965, "sm_max_mhz": 1965, "reasons": []},
+             P=4, partition_tokens=512, n_pairs=0, cascade_pages=0, graph=False, cascade_overlap=False)
+    args = argparse.Namespace(warmup=5, partition=0, seed=0, gpus=1, kv_fp8=False)
+    line = bench.step_line(args, r, 1)
+    for key in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better",
+                "scaling", "vs_baseline", "dtype", "data", "config", "clocks", "e2e", "gpu_launches", "roofline"):
+        assert key in line, key
+    assert line["config"]["workload"] == "llama7b" and "partition_tokens" not in line["config"]
+    peak = bench.measured_peak()[0]
+    dec = bench.decode_algorithmic_bytes(wl)
+    assert abs(line["roofline"]["frac"] - dec / 0.175e-3 / 1e9 / peak) < 1e-12
+    assert abs(line["value"] - bench.kv_bytes(wl, False) / 0.18e-3 / 1e9) < 1e-6
+    e = bench.config_entry(args, r, 1)
+    for key in ("us_per_step", "pct_hbm_peak", "roofline", "e2e", "clocks", "config"):
+        assert key in e, key
+    json.dumps(line)
+
+
+def test_both_arms_quote_the_same_config():
+    """The reference arm's config object is the one the CUDA arm prints."""
+    import argparse
+    import bench
+    import workloads
+    args = argparse.Namespace(seed=0, gpus=1)
+    wl = workloads.named("tiny", 0)
+    d = run("--impl", "reference", "--workload", "tiny", "--steps", "2", "--warmup", "3")
+    assert d["config"] == json.loads(json.dumps(bench.config_of(wl, args)))
 
 
 def test_multi_flops_and_roofline_choice():
