@@ -4,7 +4,9 @@ sequence-steps/s and us per step.
 One step = the whole device path for one batch: the copy-on-write block
 copies (when the step has any), the slot-mapped append of the new tokens'
 K/V, and paged decode attention (partition kernel, plus the merge kernel
-when a sequence spans several partitions).  The host allocator's step is
+when a sequence spans several partitions).  With a 16-bit cache the step is
+one fused launch (pkv_decode_step) plus the merge; --unfused runs the
+copies + append as their own launch.  The host allocator's step is
 planned before the timed region (host microseconds, not device work); the
 same planned step is replayed every iteration (its copies and appends are
 idempotent).
@@ -316,12 +318,13 @@ def run_cuda(args, rank, world, local_rank, workload=None, graph=None):
         cache.fp8 = (FP8_SCALE, FP8_SCALE)
         torch.cuda.synchronize()
     prefix = torch.from_numpy(np.ascontiguousarray(st["host"]["block_tables"][0, :pp])).to(dev) if use_cascade else None
+    fused_step = not fp8 and not (use_cascade and args.cascade_overlap) and wl.dtype != "f32" and not args.unfused
     if use_cascade:
         ws = cache.workspace(pkv.decode_prefix_workspace_bytes(B, Hq, D, max_ctx, pp, args.partition))
-        # copies + append (one launch), cascade (one launch, or prefix + suffix passes), merge
-        launches_per_step = 1 + (1 if (n_pairs and fp8) else 0) + (3 if args.cascade_overlap else 2)
+        # [copies + append (one launch)], cascade (one launch, or prefix + suffix passes), merge
+        launches_per_step = (0 if fused_step else 1) + (3 if args.cascade_overlap else 2)
     else:
-        launches_per_step = 1 + 1 + (1 if (n_pairs and fp8) else 0) + (1 if P > 1 else 0)
+        launches_per_step = (0 if fused_step else 1) + 1 + (1 if (n_pairs and fp8) else 0) + (1 if P > 1 else 0)
 
     # every call goes to the current stream at call time (so that a CUDA
     # graph capture records it)
@@ -380,9 +383,19 @@ def run_cuda(args, rank, world, local_rank, workload=None, graph=None):
             pkv.paged_attention_decode(st["q"], cache.k, cache.v, st["block_tables"], st["context_lens"], max_ctx,
                                        scale, out=out, workspace=ws, partition=args.partition)
 
+    # a 16-bit step is one launch (+ merge): each sequence's copy-on-write
+    # copy and append are made by the decode CTA that reads its last page
+    fused = fused_step
+
     def eager_step():
         if overlap:
             overlapped(True)
+            return
+        if fused:
+            pkv.decode_step(st["q"], cache.k, cache.v, st["k_new"], st["v_new"], st["slot_mapping"],
+                            copies if n_pairs else None, st["block_tables"], st["context_lens"], max_ctx, scale,
+                            prefix_blocks=prefix if use_cascade else None, out=out, workspace=ws,
+                            partition=args.partition)
             return
         pre_decode()
         decode()
@@ -478,7 +491,7 @@ def run_cuda(args, rank, world, local_rank, workload=None, graph=None):
     res = dict(wl=wl, K=K, total_ms=total_ms, e2e_ms=e2e_ms, dec_avg_ms=dec_avg_ms, roof_calls=n_roof,
                launches=launches_per_step * K, h2d=h2d, d2h=d2h, clocks=clocks.summary(), P=P,
                partition_tokens=part_tokens, n_pairs=n_pairs, cascade_pages=pp if use_cascade else 0,
-               graph=use_graph, cascade_overlap=bool(use_cascade and args.cascade_overlap))
+               graph=use_graph, cascade_overlap=bool(use_cascade and args.cascade_overlap), fused=fused)
     return res
 
 
@@ -897,7 +910,7 @@ def config_of(wl, args):
 def launch_of(args, r):
     """How the CUDA path ran the workload (partition, graph, cascade)."""
     return {"partition_tokens": r["partition_tokens"], "partition_auto": not args.partition,
-            "partitions_max": r["P"], "cuda_graph": r["graph"],
+            "partitions_max": r["P"], "cuda_graph": r["graph"], "fused_step": r.get("fused", False),
             "cascade": None if not r["cascade_pages"] else
             ("prefix pass on a second stream beside copies + append" if r["cascade_overlap"] else "one launch")}
 
@@ -983,6 +996,8 @@ def main(argv=None):
     ap.add_argument("--cascade-overlap", action="store_true",
                     help="run the cascade's prefix pass on a second stream beside the copies and append "
                          "(three launches instead of one; no faster on B200 so far)")
+    ap.add_argument("--unfused", action="store_true",
+                    help="run a 16-bit step as separate copy/append and decode launches")
     ap.add_argument("--kv-fp8", action="store_true",
                     help="the step over an FP8 (E4M3) cache: quantising append + FP8 decode")
     ap.add_argument("--row", choices=["step", "swap", "multi"], default="step",

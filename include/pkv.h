@@ -282,6 +282,44 @@ pkv_status pkv_paged_attention_decode_prefix_phase(void* out, const void* q, con
                                                    size_t workspace_bytes, int phase, void* stream);
 
 /* ------------------------------------------------------------------------
+ * pkv_decode_step -- one whole decode step in one launch (plus the merge):
+ * the step's copy-on-write copies and append, then the decode.
+ *
+ * "PagedAttention 与 vLLM 推理加速" §3.2(3) (a shared partial block is copied
+ * before a sharer appends into it), "vLLM + PagedAttention：打造高并发LLM
+ * 推理引擎", "它是怎么工作的" (the new token goes into its slot; the kernel
+ * then reads every block through the table) and §2.3 of the former.  The
+ * result -- the pool and out -- is that of
+ *   pkv_kv_append_copy(k_new, v_new, ..., slot_mapping, num_seqs, copies, ...)
+ * followed by pkv_paged_attention_decode (prefix_pages == 0) or
+ * pkv_paged_attention_decode_prefix (prefix_pages > 0, the cascade).  The
+ * writes are made inside the decode launch: for each sequence b and kv-head,
+ * the CTA that reads the sequence's last page first copies rows 0 .. rows-1
+ * of the copy (src, dst, rows) whose dst is slot_mapping[b]'s block, then
+ * writes k_new[b] / v_new[b] into the slot, then stages the page -- so the
+ * step needs no separate copy / append launch and the copies overlap the
+ * streaming of other sequences.
+ *
+ * One new token per sequence: k_new, v_new [num_seqs, num_kv_heads,
+ * head_dim] in dtype; slot_mapping int64 [num_seqs] (< 0: no token);
+ * context_lens count the new token.  copies int32 [num_copies][3] (device,
+ * num_copies <= num_seqs), as pkv_cow_copy_rows makes them from the
+ * allocator's step: every dst is the block of one slot of this call, and
+ * rows does not pass that slot's row.  The slots must not write into the
+ * shared prefix blocks (an allocator's step never does: a shared block is
+ * copied first).  dtype PKV_F16 or PKV_BF16; the other arguments, the
+ * workspace (pkv_decode_workspace_bytes, or pkv_decode_prefix_workspace_bytes
+ * when prefix_pages > 0) and the errors are those of the two calls.
+ * -------------------------------------------------------------------- */
+pkv_status pkv_decode_step(void* out, const void* q, void* k_cache, void* v_cache, const void* k_new,
+                           const void* v_new, const int64_t* slot_mapping, const int32_t* copies, int num_copies,
+                           const int32_t* block_tables, int max_blocks_per_seq, const int32_t* context_lens,
+                           int max_context_len, const int32_t* prefix_blocks, int prefix_pages, int num_seqs,
+                           int num_q_heads, int num_kv_heads, int head_dim, int num_blocks, float scale,
+                           int partition_tokens, pkv_dtype dtype, void* workspace, size_t workspace_bytes,
+                           void* stream);
+
+/* ------------------------------------------------------------------------
  * pkv_paged_attention_decode_static_ws -- pkv_paged_attention_decode for
  * callers that cannot allocate device memory.
  *
@@ -378,6 +416,37 @@ pkv_status pkv_paged_attention_decode_fp8(void* out, const void* q, const void* 
                                           void* stream);
 
 /* ------------------------------------------------------------------------
+ * pkv_paged_attention_decode_prefix_fp8 -- the shared-prefix (cascade)
+ * decode of pkv_paged_attention_decode_prefix over an FP8 cache.
+ *
+ * "PagedAttention 与 vLLM 推理加速" §3.2(3): sequences with one system prompt
+ * share its blocks; here an FP8 pool's shared prefix is read once per
+ * kv-head too.  Same result as pkv_paged_attention_decode_fp8 (up to fp32
+ * rounding order):
+ *   s_j = scale * k_scale * q . code(K_j),  out = v_scale * sum_j softmax(s)_j code(V_j).
+ * The call converts the prefix tiles to their exact 16-bit code values in
+ * the workspace (every E4M3 value is an fp16 and a bf16 value), runs the
+ * cascade's prefix pass over them on the 16-bit tensor-core path, the
+ * suffix pass over the FP8 cache, and the cascade's merge.  Sequences that
+ * do not start with the prefix, or whose context does not cover it, are
+ * decoded over their whole context (checked on the device).  Arguments as
+ * pkv_paged_attention_decode_prefix, with the scales of
+ * pkv_paged_attention_decode_fp8; q and out in q_dtype (fp16 or bf16).
+ * workspace: pkv_decode_prefix_fp8_workspace_bytes(...) bytes, 16-byte
+ * aligned, always required; no initialisation needed.
+ * -------------------------------------------------------------------- */
+size_t pkv_decode_prefix_fp8_workspace_bytes(int num_seqs, int num_q_heads, int num_kv_heads, int head_dim,
+                                             int max_context_len, int prefix_pages, int partition_tokens);
+pkv_status pkv_paged_attention_decode_prefix_fp8(void* out, const void* q, const void* k_cache,
+                                                 const void* v_cache, const int32_t* block_tables,
+                                                 int max_blocks_per_seq, const int32_t* context_lens,
+                                                 int max_context_len, const int32_t* prefix_blocks,
+                                                 int prefix_pages, int num_seqs, int num_q_heads, int num_kv_heads,
+                                                 int head_dim, int num_blocks, float scale, float k_scale,
+                                                 float v_scale, int partition_tokens, pkv_dtype q_dtype,
+                                                 void* workspace, size_t workspace_bytes, void* stream);
+
+/* ------------------------------------------------------------------------
  * pkv_paged_attention_multi -- paged attention for several query tokens
  * per sequence (speculative-decoding verification, prefill chunks).
  *
@@ -399,8 +468,9 @@ pkv_status pkv_paged_attention_decode_fp8(void* out, const void* q, const void* 
  * [num_seqs + 1] (device), non-decreasing, query_start[num_seqs] <=
  * total_query_tokens, every n_b <= max_query_len (a sequence that breaks
  * this is skipped, its rows left unwritten, and PKV_ERR_CONTEXT_RANGE set).
- * fp16 / bf16 only (tensor cores).  num_seqs * ceil(max_query_len * G / 16)
- * <= 65535.  workspace: pkv_multi_workspace_bytes(...) bytes (0 when
+ * fp16 / bf16 only (tensor cores).  num_seqs * tiles <= 65535, tiles = 1
+ * while max_query_len * G <= 32 rows per kv-head, else ceil(max_query_len *
+ * G / 128) (tiles of 128 rows on the tcgen05 tensor cores).  workspace: pkv_multi_workspace_bytes(...) bytes (0 when
  * max_context_len <= partition), 16-byte aligned.  partition_tokens as in
  * pkv_paged_attention_decode, except the auto partition (0): 2048 tokens,
  * or 1024 when max_context_len > 4096 (several rows a sequence make every

@@ -14,7 +14,7 @@ INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libpkv.so")
 
 SOURCES = ["pkv_api.cu", "allocator.cpp", "plan.cpp"]
-HEADERS = ["common.cuh", "decode.cuh", "decode_mma.cuh", "decode_prefix.cuh", "decode_launch.cuh", "decode_fp8.cuh", "multi_mma.cuh", "cache_ops.cuh"]
+HEADERS = ["common.cuh", "decode.cuh", "decode_mma.cuh", "decode_prefix.cuh", "decode_launch.cuh", "decode_fp8.cuh", "multi_mma.cuh", "multi_tc.cuh", "cache_ops.cuh"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 

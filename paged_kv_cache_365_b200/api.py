@@ -315,6 +315,48 @@ def paged_attention_decode(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torc
     return out
 
 
+def decode_step(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor, k_new: torch.Tensor,
+                v_new: torch.Tensor, slot_mapping: torch.Tensor, copies: Optional[torch.Tensor],
+                block_tables: torch.Tensor, context_lens: torch.Tensor, max_context_len: int, scale: float,
+                prefix_blocks: Optional[torch.Tensor] = None, out: Optional[torch.Tensor] = None,
+                workspace: Optional[torch.Tensor] = None, partition: int = 0, stream=None) -> torch.Tensor:
+    """One decode step in one launch (pkv_decode_step): the step's
+    copy-on-write copies (int32 ``copies`` [n, 3] = (src, dst, rows), from
+    ``cow_copy_rows``) and append of one new token per sequence (k_new /
+    v_new [B, Hkv, D], slot_mapping int64 [B]), then the decode -- the
+    cascade when ``prefix_blocks`` (int32, the shared leading blocks) is
+    given.  16-bit pools."""
+    nb, hkv, d = _cache_dims(k_cache, v_cache)
+    if q.dim() != 3 or q.shape[2] != d or q.dtype != k_cache.dtype:
+        raise ValueError("q must be [B, Hq, D] in the cache dtype")
+    B, hq, _ = q.shape
+    if k_new.shape != (B, hkv, d) or v_new.shape != k_new.shape or slot_mapping.shape != (B,):
+        raise ValueError("k_new/v_new must be [B, Hkv, D] and slot_mapping [B]")
+    if block_tables.dim() != 2 or block_tables.shape[0] != B or context_lens.shape != (B,):
+        raise ValueError("block_tables must be [B, max_blocks] and context_lens [B]")
+    n_copies = 0 if copies is None else int(copies.shape[0])
+    if n_copies and (copies.dim() != 2 or copies.shape[1] != 3):
+        raise ValueError("copies must be [n, 3]")
+    pp = 0 if prefix_blocks is None else int(prefix_blocks.numel())
+    if out is None:
+        out = torch.empty_like(q)
+    need = (decode_prefix_workspace_bytes(B, hq, d, max_context_len, pp, partition) if pp else
+            decode_workspace_bytes(B, hq, d, max_context_len, partition))
+    if need and (workspace is None or workspace.numel() * workspace.element_size() < need):
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    check(lib.pkv_decode_step(
+        _dev(out, "out", q.dtype), _dev(q, "q"), _dev(k_cache, "k_cache"), _dev(v_cache, "v_cache"),
+        _dev(k_new, "k_new", k_cache.dtype), _dev(v_new, "v_new", k_cache.dtype),
+        _dev(slot_mapping, "slot_mapping", torch.int64), _dev(copies, "copies", torch.int32) if n_copies else None,
+        n_copies, _dev(block_tables, "block_tables", torch.int32), block_tables.shape[1],
+        _dev(context_lens, "context_lens", torch.int32), int(max_context_len),
+        _dev(prefix_blocks, "prefix_blocks", torch.int32) if pp else None, pp, B, hq, hkv, d, nb, float(scale),
+        int(partition), _DT[k_cache.dtype], _dev(workspace, "workspace") if need else None,
+        workspace.numel() * workspace.element_size() if need else 0, _stream(stream, q.device)),
+        "pkv_decode_step")
+    return out
+
+
 def decode_prefix_workspace_bytes(num_seqs: int, num_q_heads: int, head_dim: int, max_context_len: int,
                                   prefix_pages: int, partition: int = 0) -> int:
     return int(lib.pkv_decode_prefix_workspace_bytes(num_seqs, num_q_heads, head_dim, max_context_len,
@@ -389,6 +431,46 @@ def paged_attention_decode_prefix(q: torch.Tensor, k_cache: torch.Tensor, v_cach
     else:
         check(lib.pkv_paged_attention_decode_prefix_phase(*args, int(phase), _stream(stream, q.device)),
               "pkv_paged_attention_decode_prefix_phase")
+    return out
+
+
+def decode_prefix_fp8_workspace_bytes(num_seqs: int, num_q_heads: int, num_kv_heads: int, head_dim: int,
+                                      max_context_len: int, prefix_pages: int, partition: int = 0) -> int:
+    return int(lib.pkv_decode_prefix_fp8_workspace_bytes(num_seqs, num_q_heads, num_kv_heads, head_dim,
+                                                         max_context_len, prefix_pages, partition))
+
+
+def paged_attention_decode_prefix_fp8(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
+                                      block_tables: torch.Tensor, context_lens: torch.Tensor, max_context_len: int,
+                                      prefix_blocks: torch.Tensor, scale: float, k_scale: float, v_scale: float,
+                                      out: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
+                                      partition: int = 0, stream=None) -> torch.Tensor:
+    """The shared-prefix decode over an FP8 cache (E4M3 codes, one scale for
+    K and one for V): the prefix blocks ``prefix_blocks`` (int32, device)
+    every table starts with are read once per kv-head.  q / out fp16 or
+    bf16."""
+    nb, hkv, d = _cache_dims(k_cache, v_cache)
+    if k_cache.dtype not in _FP8:
+        raise ValueError("an FP8 cache (float8_e4m3fn or uint8) is required")
+    if q.dim() != 3 or q.shape[2] != d or q.dtype not in (torch.float16, torch.bfloat16):
+        raise ValueError("q must be [B, Hq, D] in fp16 or bf16")
+    B, hq, _ = q.shape
+    if block_tables.dim() != 2 or block_tables.shape[0] != B or context_lens.shape != (B,):
+        raise ValueError("block_tables must be [B, max_blocks] and context_lens [B]")
+    pp = int(prefix_blocks.numel())
+    if out is None:
+        out = torch.empty_like(q)
+    need = decode_prefix_fp8_workspace_bytes(B, hq, hkv, d, max_context_len, pp, partition)
+    if workspace is None or workspace.numel() * workspace.element_size() < need:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
+    check(lib.pkv_paged_attention_decode_prefix_fp8(
+        _dev(out, "out", q.dtype), _dev(q, "q"), _dev(k_cache, "k_cache"), _dev(v_cache, "v_cache"),
+        _dev(block_tables, "block_tables", torch.int32), block_tables.shape[1],
+        _dev(context_lens, "context_lens", torch.int32), int(max_context_len),
+        _dev(prefix_blocks, "prefix_blocks", torch.int32), pp, B, hq, hkv, d, nb, float(scale), float(k_scale),
+        float(v_scale), int(partition), _DT[q.dtype], _dev(workspace, "workspace"),
+        workspace.numel() * workspace.element_size(), _stream(stream, q.device)),
+        "pkv_paged_attention_decode_prefix_fp8")
     return out
 
 
@@ -793,7 +875,9 @@ class PagedKVCache:
 
         ``cow_pairs``: int32 [n, 2] (src, dst) whole-block copies, or [n, 3]
         (src, dst, rows) from ``cow_copy_rows``: the copies cut to the rows
-        that hold tokens, in one launch with the append.
+        that hold tokens.  With [n, 3] copies (or none) and a 16-bit pool the
+        whole step is one decode launch (pkv_decode_step): each sequence's
+        copy and append are made by the CTA that then reads its last page.
         Inputs may be host tensors (pinned for asynchronous copies) or
         device tensors.  Host inputs are uploaded, and a host ``out`` is
         filled, on two side streams with double-buffered device copies, so a
@@ -813,8 +897,26 @@ class PagedKVCache:
             B, hq = q.shape[0], q.shape[1]
             res = out if (out is not None and out.device == dev) else stg.output(st, q.shape, self.dtype)
             sc = (1.0 / math.sqrt(self.D)) if scale is None else scale
+            fused = (self.fp8 is None and self.dtype != torch.float32 and
+                     (cow_pairs.shape[0] == 0 or cow_pairs.shape[1] == 3))
+            if fused:  # copies, append and decode in one launch (+ merge)
+                pp = 0 if prefix_blocks is None else prefix_blocks.numel()
+                ws = self.workspace(decode_prefix_workspace_bytes(B, hq, self.D, max_context_len, pp, partition)
+                                    if pp else decode_workspace_bytes(B, hq, self.D, max_context_len, partition))
+                decode_step(x["q"], self.k, self.v, x["k"], x["v"], x["slots"],
+                            x["pairs"] if cow_pairs.shape[0] else None, x["tables"], x["lens"], max_context_len, sc,
+                            prefix_blocks=x["prefix"] if pp else None, out=res, workspace=ws, partition=partition,
+                            stream=st)
+                stg.finish(st, res, out)
+                return res
             self._copy_append(cow_pairs.shape, x, st)
-            if self.fp8 is not None:  # (the cascade reads 16-bit pools only)
+            if self.fp8 is not None and prefix_blocks is not None and prefix_blocks.numel() > 0:
+                ws = self.workspace(decode_prefix_fp8_workspace_bytes(B, hq, self.Hkv, self.D, max_context_len,
+                                                                      prefix_blocks.numel(), partition))
+                paged_attention_decode_prefix_fp8(x["q"], self.k, self.v, x["tables"], x["lens"], max_context_len,
+                                                  x["prefix"], sc, self.fp8[0], self.fp8[1], out=res, workspace=ws,
+                                                  partition=partition, stream=st)
+            elif self.fp8 is not None:
                 ws = self.workspace(decode_workspace_bytes(B, hq, self.D, max_context_len, partition))
                 paged_attention_decode_fp8(x["q"], self.k, self.v, x["tables"], x["lens"], max_context_len, sc,
                                            self.fp8[0], self.fp8[1], out=res, workspace=ws, partition=partition,
@@ -910,7 +1012,7 @@ class PagedKVCache:
         """Host plan (allocator) + device step; returns the output on q's device."""
         slots, pairs, tables, lens = self.plan_step(seq_ids)
         max_ctx = int(lens.max()) if len(lens) else 0
-        pp = cascade_prefix_pages(tables, lens, self.dtype) if self.fp8 is None else 0
+        pp = cascade_prefix_pages(tables, lens, self.dtype)
         prefix = torch.from_numpy(np.ascontiguousarray(tables[0, :pp])) if pp else None
         copies = cow_copy_rows(pairs, slots)  # copy only the rows that hold tokens
         out = self.run_step(torch.from_numpy(slots), torch.from_numpy(copies),

@@ -68,6 +68,18 @@ struct DecodeArgs {
   float2* wp_ml;       // [B][Hq][num_chunks] (max, sum)
   int* conform;        // [B]: 1 when sequence b starts with the prefix
   int y_offset;        // cascade launched in parts: blockIdx.y + y_offset is the role index
+  int prefix_ident;    // prefix page i is block i of the pool given (a dequantised copy of the prefix)
+  float prefix_out_scale;  // factor on the prefix partial outputs (the V scale of an FP8 cache; else 1)
+  // a decode step fused with its append (pkv_decode_step); slots == nullptr
+  // otherwise.  One new token per sequence: the CTA that reads sequence b's
+  // last page writes k_new[b] / v_new[b] into slot slots[b] (after the
+  // copy-on-write copy whose destination is that slot's block) before it
+  // stages anything.
+  const unsigned char* k_new;  // [B][Hkv][D]
+  const unsigned char* v_new;
+  const int64_t* slots;        // [B]
+  const int32_t* copies;       // [n_copies][3] = (src, dst, rows)
+  int n_copies;
 };
 
 constexpr unsigned kFull = 0xffffffffu;

@@ -15,13 +15,16 @@
 //    2t+8, 2t+9 then stands for d = 16c + 4t .. + 3, and the queries (the
 //    B operand, in registers) are loaded in that same order of d, so the
 //    dot product runs over the same pairs.
-//  * P.V with P as the A operand (queries as M) and V as the B operand,
-//    O[8 queries x D]: lane (g, t) needs V[token][d] for tokens 2t, 2t+1,
-//    2t+8, 2t+9 and column g of every n-tile; with d = (D/8) n + j for
-//    n-tile j and column n, those are D/8 consecutive bytes of four rows:
-//    four shared loads, byte permutes and exact E4M3 -> 16-bit conversions.
-//    Rows 0-7 of A carry the high 16-bit part of P, rows 8-15 the low part,
-//    so one MMA per n-tile accumulates both (their sum is the result).
+//  * P.V as O^T[D x 8 queries] += V^T[D x 16 tokens] . P^T[16 x 8], V^T the
+//    A operand: lane (g, t) needs V[token][d] for tokens 2t, 2t+1, 2t+8,
+//    2t+9 and rows g, g + 8 of every m-tile; with d = (D/8) g + 2i (row g
+//    of m-tile i) and d + 1 (row g + 8), those are D/8 consecutive bytes of
+//    four token rows: four shared loads, byte permutes and exact E4M3 ->
+//    16-bit conversions.  P^T is the B operand, taken from the score
+//    fragment by movmatrix, in hi + lo 16-bit parts that accumulate into
+//    the same registers (two MMAs per m-tile); O^T needs D/16 x 4
+//    accumulator registers a lane, half of what O with the queries as M
+//    would (whose rows past G are padding).
 //  * The K scale is folded into the logit scale, the V scale into the
 //    output.
 //  * The MMAs run in fp16 whatever the query dtype: E4M3 -> fp16 is one
@@ -86,10 +89,17 @@ struct Fp8Shape {
 
 // CTAs per SM the FP8 kernel's register budget is sized for
 #ifndef PKV_FP8_MIN_CTAS
-#define PKV_FP8_MIN_CTAS 1
+#define PKV_FP8_MIN_CTAS 8
 #endif
 
-template <typename T, int D, int G, int NWARPS, int NSTAGE>
+// kCascade: the suffix pass of a shared-prefix decode over an FP8 cache
+// (pkv_paged_attention_decode_prefix_fp8).  A sequence whose table starts
+// with the prefix blocks (and whose context covers them) attends only its
+// suffix, partition `part` counted from the prefix's end; any other
+// sequence attends its whole context.  Every CTA writes partials (the
+// merge kernel combines them with the prefix pass's) and the CTA (kv-head
+// 0, part 0) writes the sequence's conformity flag.
+template <typename T, int D, int G, int NWARPS, int NSTAGE, bool kCascade = false>
 __global__ void __launch_bounds__(NWARPS * 32, PKV_FP8_MIN_CTAS)
     paged_decode_fp8_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tmap_k,
                             const __grid_constant__ CUtensorMap tmap_v, float v_scale) {
@@ -104,16 +114,29 @@ __global__ void __launch_bounds__(NWARPS * 32, PKV_FP8_MIN_CTAS)
   const int lane = threadIdx.x & 31;
   const int g8 = lane >> 2, t4 = lane & 3, lm = lane >> 3, lr = lane & 7;
 
+  int same = 1;
+  if constexpr (kCascade)
+    for (int j = threadIdx.x; j < a.prefix_pages; j += NWARPS * 32)
+      if (a.block_tables[static_cast<long long>(b) * a.bt_stride + j] != a.prefix_blocks[j]) same = 0;
   int ctx = a.context_lens[b];
   if (ctx < 0 || ctx > a.max_ctx) {
     if (threadIdx.x == 0 && kvh == 0 && part == 0) raise_error(PKV_ERR_CONTEXT_RANGE);
     ctx = ctx < 0 ? 0 : a.max_ctx;
   }
-  const int nparts = (ctx + a.partition - 1) / a.partition;
+  int tok_begin = 0;
+  if constexpr (kCascade) {
+    const bool conforming = __syncthreads_and(same) && ctx >= a.prefix_pages * kBlockSize;
+    if (conforming) tok_begin = a.prefix_pages * kBlockSize;
+    if (threadIdx.x == 0 && kvh == 0 && part == 0) a.conform[b] = conforming ? 1 : 0;
+  }
+  const int span = ctx - tok_begin;
+  const int nparts = (span + a.partition - 1) / a.partition;
   if (part >= (nparts > 0 ? nparts : 1)) return;
-  if (ctx == 0) {
-    T* out = reinterpret_cast<T*>(a.out) + (static_cast<size_t>(b) * a.num_q_heads + kvh * G) * D;
-    for (int i = threadIdx.x; i < G * D; i += NWARPS * 32) out[i] = Fmt<T>::from_f32(0.f);
+  if (span == 0) {
+    if (!kCascade) {  // (the cascade's merge writes the zeros of an empty context)
+      T* out = reinterpret_cast<T*>(a.out) + (static_cast<size_t>(b) * a.num_q_heads + kvh * G) * D;
+      for (int i = threadIdx.x; i < G * D; i += NWARPS * 32) out[i] = Fmt<T>::from_f32(0.f);
+    }
     return;
   }
   auto col_row = [&](int n) -> size_t { return static_cast<size_t>(b) * a.num_q_heads + kvh * G + n; };
@@ -176,7 +199,7 @@ __global__ void __launch_bounds__(NWARPS * 32, PKV_FP8_MIN_CTAS)
   const float xs0 = a.qk_scale * __uint_as_float(static_cast<uint32_t>(127 - kq0) << 23);
   const float xs1 = a.qk_scale * __uint_as_float(static_cast<uint32_t>(127 - kq1) << 23);
 
-  const int tok0 = part * a.partition;
+  const int tok0 = tok_begin + part * a.partition;
   const int tok1 = min(ctx, tok0 + a.partition);
   const int pg0 = tok0 / kBlockSize;
   const int nblk = (tok1 - tok0 + kBlockSize - 1) / kBlockSize;
@@ -223,11 +246,12 @@ __global__ void __launch_bounds__(NWARPS * 32, PKV_FP8_MIN_CTAS)
 #pragma unroll
   for (int i = 0; i < NSTAGE; ++i) issue(i);
 
-  // O[query g8][d]: n-tile j, columns 2 t4, 2 t4 + 1 -> d = kNT (2 t4) + j,
-  // kNT (2 t4 + 1) + j; [0..1] from P's high part, [2..3] from its low part
-  float o[kNT][4];
+  // O^T accumulators: m-tile i, rows g8 / g8 + 8 -> d = kNT g8 + 2i / + 1,
+  // columns 2 t4, 2 t4 + 1 (queries)
+  constexpr int kMT = D / 16;
+  float o[kMT][4];
 #pragma unroll
-  for (int j = 0; j < kNT; ++j) o[j][0] = o[j][1] = o[j][2] = o[j][3] = 0.f;
+  for (int i = 0; i < kMT; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
   float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;  // query columns 2 t4, 2 t4 + 1
   int consumed = 0;
   bool timed_out = false;
@@ -285,24 +309,21 @@ __global__ void __launch_bounds__(NWARPS * 32, PKV_FP8_MIN_CTAS)
       const float p0 = exp2_sfu(x0 - n0), p1 = exp2_sfu(x1 - n1), p2 = exp2_sfu(x2 - n0), p3 = exp2_sfu(x3 - n1);
       l0 = fmaf(l0, al0, p0 + p2);
       l1 = fmaf(l1, al1, p1 + p3);
-      // this lane's O rows belong to query g8: its factor comes from the
-      // lane holding query column g8 (t4 = g8 / 2)
-      const float ae = __shfl_sync(kFull, al0, g8 >> 1), ao = __shfl_sync(kFull, al1, g8 >> 1);
-      const float alpha = (g8 & 1) ? ao : ae;
-      if (__any_sync(kFull, alpha != 1.f)) {
+      // this lane's O^T columns are its own query columns 2 t4, 2 t4 + 1
+      if (__any_sync(kFull, al0 != 1.f || al1 != 1.f)) {
 #pragma unroll
-        for (int j = 0; j < kNT; ++j) {
-          o[j][0] *= alpha;
-          o[j][1] *= alpha;
-          o[j][2] *= alpha;
-          o[j][3] *= alpha;
+        for (int i = 0; i < kMT; ++i) {
+          o[i][0] *= al0;
+          o[i][1] *= al1;
+          o[i][2] *= al0;
+          o[i][3] *= al1;
         }
       }
-      // (3) P as A fragments: rows g8 = P high part, rows g8 + 8 = low part
+      // (3) P^T as B fragments, split into hi + lo 16-bit parts
       const uint32_t top_hi = M::pack(p0, p1), bot_hi = M::pack(p2, p3);
       const float2 th = M::unpack(top_hi), bh = M::unpack(bot_hi);
       const uint32_t top_lo = M::pack(p0 - th.x, p1 - th.y), bot_lo = M::pack(p2 - bh.x, p3 - bh.y);
-      const uint32_t pa0 = movm_t(top_hi), pa1 = movm_t(top_lo), pa2 = movm_t(bot_hi), pa3 = movm_t(bot_lo);
+      const uint32_t pb0 = movm_t(top_hi), pb1 = movm_t(bot_hi), pl0 = movm_t(top_lo), pl1 = movm_t(bot_lo);
       // (4) bytes d = kNT g8 .. kNT g8 + kNT - 1 (in 16-byte chunk vch, from
       // byte vb0) of rows 2 t4, 2 t4 + 1, 2 t4 + 8, 2 t4 + 9; rows past the
       // context are zeroed (an unused slot may hold a NaN code)
@@ -333,19 +354,20 @@ __global__ void __launch_bounds__(NWARPS * 32, PKV_FP8_MIN_CTAS)
         load(2 * t4 + 8, w8);
         load(2 * t4 + 9, w9);
       }
-      // n-tile j uses byte j of each row segment; two n-tiles per permute
+      // m-tile i uses bytes 2i (its row g8) and 2i + 1 (row g8 + 8) of each
+      // row segment: one permute per pair of token rows
 #pragma unroll
-      for (int j = 0; j < kNT; j += 2) {
-        const int w = j >> 2, bsel = j & 3;
-        // (row a byte j, row b byte j, row a byte j+1, row b byte j+1)
+      for (int i = 0; i < kMT; ++i) {
+        const int w = i >> 1, bsel = 2 * (i & 1);
+        // (row a byte 2i, row b byte 2i, row a byte 2i+1, row b byte 2i+1)
         const uint32_t sel = bsel | ((4 + bsel) << 4) | ((bsel + 1) << 8) | ((5 + bsel) << 12);
         const uint32_t lo01 = __byte_perm(w0[w], w1[w], sel);
         const uint32_t lo89 = __byte_perm(w8[w], w9[w], sel);
-        uint32_t b0j, b0k, b1j, b1k;
-        e4m3x4_to_f16(lo01, b0j, b0k);
-        e4m3x4_to_f16(lo89, b1j, b1k);
-        M::run(o[j], pa0, pa1, pa2, pa3, b0j, b1j);
-        M::run(o[j + 1], pa0, pa1, pa2, pa3, b0k, b1k);
+        uint32_t a0, a1, a2, a3;
+        e4m3x4_to_f16(lo01, a0, a1);  // tokens 2 t4, 2 t4 + 1 at rows g8, g8 + 8
+        e4m3x4_to_f16(lo89, a2, a3);  // tokens 2 t4 + 8, 2 t4 + 9
+        M::run(o[i], a0, a1, a2, a3, pb0, pb1);
+        M::run(o[i], a0, a1, a2, a3, pl0, pl1);
       }
     }
     __syncwarp();
@@ -367,11 +389,16 @@ __global__ void __launch_bounds__(NWARPS * 32, PKV_FP8_MIN_CTAS)
 
   // warp record [o: 8 x D][m: 8][l: 8]
   float* rec = reinterpret_cast<float*>(my_stages);
-  if (g8 < G) {
 #pragma unroll
-    for (int j = 0; j < kNT; ++j) {
-      rec[g8 * D + kNT * (2 * t4) + j] = o[j][0] + o[j][2];
-      rec[g8 * D + kNT * (2 * t4 + 1) + j] = o[j][1] + o[j][3];
+  for (int i = 0; i < kMT; ++i) {
+    const int d = kNT * g8 + 2 * i;
+    if (2 * t4 < G) {
+      rec[(2 * t4) * D + d] = o[i][0];
+      rec[(2 * t4) * D + d + 1] = o[i][2];
+    }
+    if (2 * t4 + 1 < G) {
+      rec[(2 * t4 + 1) * D + d] = o[i][1];
+      rec[(2 * t4 + 1) * D + d + 1] = o[i][3];
     }
   }
   if (g8 == 0) {
@@ -402,13 +429,57 @@ __global__ void __launch_bounds__(NWARPS * 32, PKV_FP8_MIN_CTAS)
     }
     num *= v_scale;
     const size_t row = col_row(g);
-    if (nparts == 1) {
+    if (nparts == 1 && !kCascade) {
       reinterpret_cast<T*>(a.out)[row * D + d] = Fmt<T>::from_f32(num / den);
     } else {
       const size_t wrow = row * a.num_parts + part;
       a.ws_o[wrow * D + d] = num;
       if (d == 0) a.ws_ml[wrow] = make_float2(Mx, den);
     }
+  }
+}
+
+// The shared prefix of an FP8 cache as exact 16-bit code values, for the
+// cascade's prefix pass (which runs on the 16-bit tensor-core path): tile
+// (page p, kv-head h) of prefix block prefix_blocks[p] goes to block p of a
+// small pool [prefix_pages][Hkv][16][D] of T (every E4M3 value is an fp16
+// and a bf16 value, so nothing is rounded; the scales are applied by the
+// pass).  One thread converts 8 codes; chunks [0, total) are K, [total,
+// 2 total) V.  A prefix entry outside the pool is flagged and its tile
+// zeroed.
+template <typename T>
+__global__ void __launch_bounds__(256)
+    dequant_prefix_kernel(const uint2* __restrict__ k_cache, const uint2* __restrict__ v_cache,
+                          uint4* __restrict__ k_out, uint4* __restrict__ v_out, const int32_t* __restrict__ prefix_blocks,
+                          long long total, int Hkv, int row_chunks, int num_blocks) {
+  pdl_enter();
+  const long long tile_chunks = static_cast<long long>(kBlockSize) * row_chunks;
+  const long long stride = static_cast<long long>(gridDim.x) * blockDim.x;
+  for (long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; i < 2 * total; i += stride) {
+    const bool is_v = i >= total;
+    const long long j = is_v ? i - total : i;
+    const long long tile = j / tile_chunks;  // p * Hkv + h
+    const long long c = j - tile * tile_chunks;
+    const int p = static_cast<int>(tile / Hkv), h = static_cast<int>(tile % Hkv);
+    const int blk = prefix_blocks[p];
+    uint4 o = make_uint4(0u, 0u, 0u, 0u);
+    if (blk >= 0 && blk < num_blocks) {
+      const uint2 w = (is_v ? v_cache : k_cache)[(static_cast<long long>(blk) * Hkv + h) * tile_chunks + c];
+      uint32_t h2[4];
+      e4m3x4_to_f16(w.x, h2[0], h2[1]);
+      e4m3x4_to_f16(w.y, h2[2], h2[3]);
+      if constexpr (!std::is_same<T, __half>::value) {
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&h2[e]));
+          h2[e] = Mma<T>::pack(f.x, f.y);  // exact: an E4M3 value is a bf16 value
+        }
+      }
+      o = make_uint4(h2[0], h2[1], h2[2], h2[3]);
+    } else if (h == 0 && c == 0 && !is_v) {
+      raise_error(PKV_ERR_BLOCK_RANGE);
+    }
+    (is_v ? v_out : k_out)[j] = o;
   }
 }
 

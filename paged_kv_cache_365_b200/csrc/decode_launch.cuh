@@ -311,6 +311,7 @@ pkv_status prepare_decode(void* out, const void* q, const void* k_cache, const v
   a->partition = part;
   a->num_parts = P > 1 ? static_cast<int>(P) : 1;
   a->qk_scale = scale * kLog2e;
+  a->prefix_out_scale = 1.f;
   *P_out = P;
   return PKV_OK;
 }

@@ -165,7 +165,7 @@ __device__ __forceinline__ bool prefix_warp(const DecodeArgs& a, const CUtensorM
   // lane j: block of page pg0 + j (nblk <= 32)
   int my_phys = -1;
   if (lane < nblk) {
-    const int e = a.prefix_blocks[pg0 + lane];
+    const int e = a.prefix_ident ? pg0 + lane : a.prefix_blocks[pg0 + lane];
     if (e >= 0 && e < a.num_blocks)
       my_phys = e;
     else
@@ -329,10 +329,69 @@ __device__ __forceinline__ bool prefix_warp(const DecodeArgs& a, const CUtensorM
     float* dst = a.wp_o + slot * D;
 #pragma unroll
     for (int j = 0; j < kNTiles; ++j)
-      *reinterpret_cast<float2*>(dst + 8 * j + 2 * t4) = make_float2(o[j][2 * r], o[j][2 * r + 1]);
+      *reinterpret_cast<float2*>(dst + 8 * j + 2 * t4) =
+          make_float2(o[j][2 * r] * a.prefix_out_scale, o[j][2 * r + 1] * a.prefix_out_scale);
     if (t4 == 0) a.wp_ml[slot] = make_float2(ms[r], ls[r]);
   }
   return true;
+}
+
+// The step's writes for sequence b and kv-head kvh ("PagedAttention 与 vLLM
+// 推理加速" §3.2(3): the shared partial block is copied before the writer
+// appends; "vLLM + PagedAttention：打造高并发LLM推理引擎", "它是怎么工作的": the
+// new token goes into its slot), made by the one warp that later stages the
+// sequence's last page: rows 0 .. rows-1 of the copy whose destination is
+// the slot's block, then the token.  The stores are issued here and fenced
+// for the async proxy just before that warp's TMA load of the page (see
+// the issue step of the kernel), so their latency hides behind the pages
+// streamed before it.
+template <typename T, int D>
+__device__ __forceinline__ void fused_step_append(const DecodeArgs& a, int b, int kvh, int lane) {
+  constexpr int kRowChunks = D * static_cast<int>(sizeof(T)) / 16;  // 16-byte chunks of a row
+  const int64_t s = a.slots[b];
+  const int64_t blk = s >= 0 ? s / kBlockSize : -1;
+  const bool ok = s >= 0 && blk < a.num_blocks;
+  if (s >= 0 && !ok && lane == 0) raise_error(PKV_ERR_SLOT_RANGE);
+  if (!ok) return;
+  // the copy into this block, if any
+  int src = -1, rows = 0;
+  for (int i0 = 0; i0 < a.n_copies; i0 += 32) {
+    const int i = i0 + lane;
+    const bool hit = i < a.n_copies && a.copies[3 * i + 1] == static_cast<int>(blk);
+    const unsigned m = __ballot_sync(kFull, hit);
+    if (m) {
+      const int w = i0 + __ffs(m) - 1;
+      src = a.copies[3 * w];
+      rows = a.copies[3 * w + 2];
+      break;
+    }
+  }
+  if (src >= 0 && (src >= a.num_blocks || rows < 0 || rows > kBlockSize)) {
+    if (lane == 0) raise_error(PKV_ERR_COPY_RANGE);
+    src = -1;
+  }
+  const size_t head = static_cast<size_t>(kBlockSize) * kRowChunks;  // chunks of one (block, kv-head) tile
+  uint4* kc = reinterpret_cast<uint4*>(const_cast<unsigned char*>(a.k_cache));
+  uint4* vc = reinterpret_cast<uint4*>(const_cast<unsigned char*>(a.v_cache));
+  if (src >= 0) {
+    const size_t from = (static_cast<size_t>(src) * a.num_kv_heads + kvh) * head;
+    const size_t to = (static_cast<size_t>(blk) * a.num_kv_heads + kvh) * head;
+    for (int e = lane; e < 2 * rows * kRowChunks; e += 32) {
+      uint4* c = e < rows * kRowChunks ? kc : vc;
+      const int k = e < rows * kRowChunks ? e : e - rows * kRowChunks;
+      c[to + k] = c[from + k];
+    }
+  }
+  __syncwarp();  // (the token's row may lie inside the copied rows)
+  const size_t dst = (static_cast<size_t>(blk) * a.num_kv_heads + kvh) * head +
+                     static_cast<size_t>(s % kBlockSize) * kRowChunks;
+  const size_t in = (static_cast<size_t>(b) * a.num_kv_heads + kvh) * kRowChunks;
+  for (int e = lane; e < 2 * kRowChunks; e += 32) {
+    if (e < kRowChunks)
+      kc[dst + e] = reinterpret_cast<const uint4*>(a.k_new)[in + e];
+    else
+      vc[dst + e - kRowChunks] = reinterpret_cast<const uint4*>(a.v_new)[in + e - kRowChunks];
+  }
 }
 
 // One CTA of 4 warps does one of two jobs:
@@ -467,6 +526,15 @@ __global__ void __launch_bounds__(NWARPS * 32)
     const int pg0 = tok0 / kBlockSize;
     const int nblk = (tok1 - tok0 + kBlockSize - 1) / kBlockSize;
     const int my_n = warp < nblk ? (nblk - warp + NWARPS - 1) / NWARPS : 0;  // <= 32 * S::kTab
+    // a fused step: the warp that stages the sequence's last page (page
+    // nblk - 1 of the last partition, its page `last_i`) writes the new
+    // token and its copy-on-write copy first, and fences them before that
+    // page's TMA load
+    int last_i = -1;
+    if (!prefix_role && a.slots != nullptr && pidx == nparts - 1 && warp == (nblk - 1) % NWARPS) {
+      last_i = (nblk - 1) / NWARPS;
+      fused_step_append<T, D>(a, b, kvh, lane);
+    }
 
     // lane j: physical blocks of this warp's pages j, j + 32, ... (page
     // warp + j*NWARPS of the partition, and so on)
@@ -496,6 +564,10 @@ __global__ void __launch_bounds__(NWARPS * 32)
 
     auto issue = [&](int i) {
       const int phys = phys_of(i);
+      if (i == last_i) {  // the step's writes into this page, visible to the TMA read
+        asm volatile("fence.proxy.async.global;" ::: "memory");
+        __syncwarp();
+      }
       if (lane == 0 && i < my_n) {
         const uint32_t bar = bar0 + 8 * (i % NSTAGE);
         if (phys >= 0) {

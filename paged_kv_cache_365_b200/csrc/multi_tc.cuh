@@ -1,0 +1,536 @@
+// Multi-token paged attention on the 5th-generation tensor cores (tcgen05),
+// for prefill chunks and long verification runs: many query rows per
+// (sequence, kv-head).
+//
+// "LLM Systems 24: Efficient LLM Inference with PagedAttention and vLLM"
+// §2.2.1.3 (batches that mix prefill chunks with decode steps) and
+// "PagedAttention 与 vLLM 推理加速" §6 (the large model checks a run of
+// guessed tokens in one pass): each new token attends causally over its
+// sequence's paged K/V, read through the block table (§2.3).  The result is
+// the one paged_multi_fa_kernel computes (multi_mma.cuh); what changes is
+// where the contraction runs and where its accumulators live.
+//
+// One CTA per (kv-head, sequence, tile of 128 rows, key partition); a row
+// is a (token, head) pair of the kv-head, as in the other multi-token
+// kernels.  Six warps with fixed jobs:
+//   warp 0      TMA producer: the partition's pages, four per key block (64
+//               keys), into a ring of NS stages (K panels, then V panels);
+//   warp 1      owns the tensor memory and issues the MMAs from one thread:
+//                 S_j  = Q . K_j^T      (M 128, N 64, A and B from shared
+//                                        memory, K-major, 128-byte swizzle)
+//                 O   += P_j . V_j      (A = P from tensor memory, B = V
+//                                        from shared memory, MN-major)
+//               S is double-buffered, so the scores of block j+1 are formed
+//               while block j's softmax runs;
+//   warps 2-5   softmax and epilogue, one thread per row (its tensor-memory
+//               lane): the row's 64 scores of a block come in with
+//               tcgen05.ld, the causal mask and the running max need no
+//               shuffles, and P goes back into the S buffer as hi + lo
+//               16-bit parts (two MMAs, ~2^-16 relative error, as in the
+//               other kernels).  The running max is moved only when a block
+//               raises it by more than 2^8 (then O is rescaled in tensor
+//               memory), so most blocks need no O traffic at all.
+// Tensor memory: O in columns [0, D), S/P buffers at columns 128 and 192
+// (256 columns a CTA, two CTAs an SM).  Invalid V rows of a block (past the
+// context, or pages the table does not name) are zeroed in shared memory
+// before the block's P.V, so a NaN in an unused slot never meets a zero
+// weight; their keys are masked in the softmax.
+//
+// Every wait is bounded (PKV_ERR_TIMEOUT, then a bounded drain of the
+// copies and the MMAs in flight); the tensor memory is released on every
+// path.
+#pragma once
+
+#include "multi_mma.cuh"
+
+namespace pkv {
+
+// ----------------------------------------------------------------------------
+// tcgen05 primitives (inline PTX, cta_group::1)
+// ----------------------------------------------------------------------------
+__device__ __forceinline__ void tmem_alloc(uint32_t dst_smem, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(dst_smem), "r"(ncols)
+               : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish() {
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+// Arrive on `bar` once every tcgen05 operation this thread issued so far
+// has completed.
+__device__ __forceinline__ void tc_commit(uint32_t bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar) : "memory");
+}
+
+// D (tensor memory) = A . B (+ D when acc != 0); A and B in shared memory.
+__device__ __forceinline__ void tc_mma_ss(uint32_t d, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                          uint32_t acc) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t"
+      "}" ::"r"(d),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(acc)
+      : "memory");
+}
+
+// D = A . B (+ D); A in tensor memory, B in shared memory.
+__device__ __forceinline__ void tc_mma_ts(uint32_t d, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                          uint32_t acc) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t"
+      "}" ::"r"(d),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(acc)
+      : "memory");
+}
+
+// 32 consecutive 32-bit columns of this thread's lane (warp-collective; the
+// warp's lane quadrant is in taddr), waited for inside the same statement so
+// that no use of the registers can be scheduled ahead of the wait.
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
+      "%15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];\n\t"
+      "tcgen05.wait::ld.sync.aligned;"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]),
+        "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]),
+        "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
+        "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr)
+      : "memory");
+}
+
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
+      "%15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]),
+      "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]), "r"(r[16]), "r"(r[17]), "r"(r[18]),
+      "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]),
+      "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
+      : "memory");
+}
+__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
+// Shared-memory matrix descriptor (Blackwell form): 128-byte swizzle, start
+// address, leading / stride byte offsets (all in 16-byte units).
+//   K-major operand: rows 128 bytes apart, 8-row groups `sbo` apart; the
+//     leading offset is unused by the swizzled form (1).
+//   MN-major operand: 64 MN-elements of a K-row contiguous, K-rows 128
+//     bytes apart, 8-row K groups `sbo` apart, the next 64 MN-elements
+//     `lbo` further on.
+__device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr, uint32_t lbo_bytes, uint32_t sbo_bytes) {
+  return static_cast<uint64_t>((saddr & 0x3FFFFu) >> 4) | (static_cast<uint64_t>((lbo_bytes >> 4) & 0x3FFFu) << 16) |
+         (static_cast<uint64_t>((sbo_bytes >> 4) & 0x3FFFu) << 32) | (1ull << 46) /* descriptor version */ |
+         (2ull << 61) /* 128-byte swizzle */;
+}
+
+template <typename T>
+struct TcFmt;
+template <>
+struct TcFmt<__half> {
+  static constexpr uint32_t kCode = 0;
+};
+template <>
+struct TcFmt<__nv_bfloat16> {
+  static constexpr uint32_t kCode = 1;
+};
+
+// Instruction descriptor of kind::f16 with fp32 accumulation: A and B of
+// type T, A K-major, B K-major or MN-major, M x N.
+template <typename T>
+__host__ __device__ constexpr uint32_t tc_idesc(int M, int N, bool b_mn_major) {
+  return (1u << 4) /* D fp32 */ | (TcFmt<T>::kCode << 7) | (TcFmt<T>::kCode << 10) |
+         ((b_mn_major ? 1u : 0u) << 16) | (static_cast<uint32_t>(N >> 3) << 17) |
+         (static_cast<uint32_t>(M >> 4) << 24);
+}
+
+// ----------------------------------------------------------------------------
+// the kernel
+// ----------------------------------------------------------------------------
+template <int D, int NS>
+struct TcShape {
+  static constexpr int kRows = 128;                 // query rows of a tile (the MMA's M, one per TMEM lane)
+  static constexpr int kPages = 4;                  // pages per key block
+  static constexpr int kKeys = kPages * kBlockSize;  // keys per block (the S MMA's N)
+  static constexpr int kPanels = D / 64;            // 128-byte column panels of a row
+  static constexpr int kQPanel = kRows * 128;       // bytes of one Q panel
+  static constexpr int kKVPanel = kKeys * 128;      // bytes of one K (or V) panel of a block
+  static constexpr int kKV = kPanels * kKVPanel;    // K (or V) of one block
+  static constexpr int kStage = 2 * kKV;            // K panels, then V panels
+  static constexpr size_t kOffStages = size_t(kPanels) * kQPanel;
+  static constexpr size_t kOffBars = kOffStages + size_t(NS) * kStage;
+  // barriers: full[NS], empty[NS], sfull[2], pfull[2], pvdone, final
+  static constexpr int kBars = 2 * NS + 6;
+  static constexpr size_t kOffTab = kOffBars + size_t(kBars) * 8;
+  static constexpr int kMaxPages = 128;  // pages of the longest partition (2048 tokens)
+  static constexpr size_t kOffSlot = kOffTab + size_t(kMaxPages) * 4;
+  static constexpr size_t kSmem = 1024 /* alignment slack */ + kOffSlot + 16;
+  static constexpr uint32_t kTmemCols = 256;
+  static constexpr uint32_t kColO = 0;
+  static constexpr uint32_t kColS = 128;  // S/P buffer b at kColS + 64 b
+  static constexpr int kThreads = 192;
+  static_assert(D == 64 || D == 128, "head_dim 64 or 128");
+  static_assert(kStage % 1024 == 0 && kQPanel % 1024 == 0, "swizzled panels need 1024-byte alignment");
+};
+
+#ifndef PKV_TC_STAGES
+#define PKV_TC_STAGES 2
+#endif
+#ifndef PKV_TC_MIN_CTAS
+#define PKV_TC_MIN_CTAS 2
+#endif
+
+template <typename T, int D, int G, int NS>
+__global__ void __launch_bounds__(TcShape<D, NS>::kThreads, PKV_TC_MIN_CTAS)
+    paged_multi_tc_kernel(const MultiArgs a, const __grid_constant__ CUtensorMap tmap_k,
+                          const __grid_constant__ CUtensorMap tmap_v) {
+  pdl_enter();
+  using S = TcShape<D, NS>;
+  using M = Mma<T>;
+  const int kvh = blockIdx.x;
+  const int b = blockIdx.y / a.tiles;
+  const int tile = blockIdx.y % a.tiles;
+  const int z = blockIdx.z;
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  int ctx, q0, nq;
+  if (!multi_seq(a, b, ctx, q0, nq, threadIdx.x == 0 && kvh == 0 && tile == 0 && z == 0)) return;
+  const int R = nq * G;
+  const int r0 = tile * S::kRows;
+  if (r0 >= R) return;
+  const int base = ctx - nq;
+  const int p_hi = base + (min(R, r0 + S::kRows) - 1) / G;
+  const bool direct = ctx <= a.partition;
+  const int tok0 = z * a.partition;
+  const int tok1 = min(min(ctx, tok0 + a.partition), p_hi + 1);
+  auto out_row = [&](int tr) -> size_t {
+    return static_cast<size_t>(q0 + tr / G) * a.num_q_heads + kvh * G + tr % G;
+  };
+  if (tok1 <= tok0) {
+    if (direct && z == 0)
+      for (int idx = threadIdx.x; idx < S::kRows * D; idx += S::kThreads) {
+        const int tr = r0 + idx / D;
+        if (tr < R) reinterpret_cast<T*>(a.out)[out_row(tr) * D + idx % D] = Fmt<T>::from_f32(0.f);
+      }
+    return;
+  }
+
+  extern __shared__ unsigned char smem_raw[];
+  const uint32_t raw_addr = smem_addr(smem_raw);
+  unsigned char* smem = smem_raw + (((raw_addr + 1023u) & ~1023u) - raw_addr);
+  const uint32_t sq = smem_addr(smem);
+  const uint32_t sstage = sq + static_cast<uint32_t>(S::kOffStages);
+  const uint32_t bars = sq + static_cast<uint32_t>(S::kOffBars);
+  const uint32_t bar_full = bars, bar_empty = bars + 8 * NS, bar_sfull = bars + 16 * NS;
+  const uint32_t bar_pfull = bar_sfull + 16, bar_pvdone = bar_pfull + 16, bar_final = bar_pvdone + 8;
+  int* table = reinterpret_cast<int*>(smem + S::kOffTab);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + S::kOffSlot);
+
+  const int pg0 = tok0 / kBlockSize;
+  const int nblk = (tok1 - tok0 + kBlockSize - 1) / kBlockSize;  // pages, <= kMaxPages
+  const int nb = (nblk + S::kPages - 1) / S::kPages;              // key blocks
+  for (int j = threadIdx.x; j < nblk; j += S::kThreads) {
+    const int e = a.block_tables[static_cast<long long>(b) * a.bt_stride + pg0 + j];
+    const bool in = e >= 0 && e < a.num_blocks;
+    if (!in) raise_error(PKV_ERR_BLOCK_RANGE);
+    table[j] = in ? e : -1;
+  }
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < NS; ++s) {
+      mbar_init(bar_full + 8 * s, 1);
+      mbar_init(bar_empty + 8 * s, 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(bar_sfull + 8 * i, 1);
+      mbar_init(bar_pfull + 8 * i, 4);  // one arrival per softmax warp
+    }
+    mbar_init(bar_pvdone, 1);
+    mbar_init(bar_final, 1);
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_addr(tmem_slot), S::kTmemCols);
+    tmem_relinquish();
+  }
+  if (warp >= 2) {
+    // this thread's row of Q into the 128-byte-swizzled K-major tile
+    // (rows past the batch are zeros)
+    const int r = 32 * (warp & 3) + lane;
+    const int tr = r0 + r;
+    const uint4* src = tr < R ? reinterpret_cast<const uint4*>(reinterpret_cast<const T*>(a.q) + out_row(tr) * D)
+                              : nullptr;
+#pragma unroll
+    for (int c = 0; c < D / 8; ++c) {
+      const uint4 v = src ? src[c] : make_uint4(0u, 0u, 0u, 0u);
+      *reinterpret_cast<uint4*>(smem + (c >> 3) * S::kQPanel + r * 128 + (((c & 7) ^ (r & 7)) << 4)) = v;
+    }
+    fence_proxy_async_smem();  // the tensor core reads the tile through the async proxy
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  // loaded(i): page i of the partition is staged (in range, named by the table)
+  auto loaded = [&](int i) { return i < nblk && table[i] >= 0; };
+  bool bad = false;
+  int issued = 0;  // producer: key blocks whose copies were issued
+
+  if (warp == 0) {
+    // ---- TMA producer ------------------------------------------------------
+    if (lane == 0) {
+      for (int c = 0; c < nb; ++c) {
+        const int s = c % NS;
+        if (c >= NS && !mbar_wait_bounded(bar_empty + 8 * s, ((c / NS) - 1) & 1)) {
+          raise_error(PKV_ERR_TIMEOUT);
+          bad = true;
+          break;
+        }
+        uint32_t bytes = 0;
+#pragma unroll
+        for (int p = 0; p < S::kPages; ++p)
+          if (loaded(c * S::kPages + p)) bytes += 2 * S::kPanels * 2048;
+        const uint32_t bar = bar_full + 8 * s;
+        if (bytes == 0) {
+          mbar_arrive(bar);
+        } else {
+          fence_proxy_async_smem();
+          mbar_arrive_expect_tx(bar, bytes);
+          const uint32_t kst = sstage + s * S::kStage, vst = kst + S::kKV;
+#pragma unroll
+          for (int p = 0; p < S::kPages; ++p) {
+            const int i = c * S::kPages + p;
+            if (!loaded(i)) continue;
+            const int y = (table[i] * a.num_kv_heads + kvh) * kBlockSize;
+#pragma unroll
+            for (int bx = 0; bx < S::kPanels; ++bx) {
+              tma_load_2d(kst + bx * S::kKVPanel + p * 2048, &tmap_k, bx * 64, y, bar);
+              tma_load_2d(vst + bx * S::kKVPanel + p * 2048, &tmap_v, bx * 64, y, bar);
+            }
+          }
+        }
+        issued = c + 1;
+      }
+    }
+  } else if (warp == 1) {
+    // ---- MMA issuer (lane 0) and V-row zeroing (the whole warp) -------------
+    constexpr uint32_t kIdQK = tc_idesc<T>(128, S::kKeys, false);
+    constexpr uint32_t kIdPV = tc_idesc<T>(128, D, true);
+    auto wait_all = [&](uint32_t bar, uint32_t parity) { return __all_sync(kFull, mbar_wait_bounded(bar, parity)); };
+    auto pv = [&](int j) -> bool {
+      if (!wait_all(bar_pfull + 8 * (j & 1), (j >> 1) & 1)) return false;
+      tc_fence_after();
+      if (lane == 0) {
+        const uint32_t vst = sstage + (j % NS) * S::kStage + S::kKV;
+        const uint32_t pcol = tmem + S::kColS + 64 * (j & 1);
+#pragma unroll
+        for (int kk = 0; kk < S::kKeys / 16; ++kk) {
+          const uint64_t vd = sw128_desc(vst + kk * 2048, S::kKVPanel, 1024);
+          tc_mma_ts(tmem + S::kColO, pcol + 8 * kk, vd, kIdPV, (j > 0 || kk > 0) ? 1u : 0u);  // P hi
+          tc_mma_ts(tmem + S::kColO, pcol + 32 + 8 * kk, vd, kIdPV, 1u);                       // P lo
+        }
+        tc_commit(bar_empty + 8 * (j % NS));  // the block's K and V may be overwritten
+        tc_commit(bar_pvdone);
+      }
+      __syncwarp();
+      return true;
+    };
+    for (int c = 0; c < nb && !bad; ++c) {
+      const int s = c % NS;
+      if (!wait_all(bar_full + 8 * s, (c / NS) & 1)) {
+        bad = true;
+        break;
+      }
+      // zero the V rows of keys that are not there (past the context or
+      // on pages the table does not name)
+      {
+        const uint32_t vst_off = static_cast<uint32_t>(S::kOffStages) + s * S::kStage + S::kKV;
+        bool zeroed = false;
+#pragma unroll
+        for (int p = 0; p < S::kPages; ++p) {
+          const int i = c * S::kPages + p;
+          const int page_tok = tok0 + i * kBlockSize;
+          const int first = loaded(i) ? max(0, min(kBlockSize, tok1 - page_tok)) : 0;
+          if (first >= kBlockSize) continue;
+          zeroed = true;
+          const int n = (kBlockSize - first) * S::kPanels * 8;  // 16-byte chunks
+          for (int e = lane; e < n; e += 32) {
+            const int row = first + e / (S::kPanels * 8);
+            const int pn = (e / 8) % S::kPanels;
+            *reinterpret_cast<uint4*>(smem + vst_off + pn * S::kKVPanel + (p * kBlockSize + row) * 128 +
+                                      (e & 7) * 16) = make_uint4(0u, 0u, 0u, 0u);
+          }
+        }
+        if (zeroed) fence_proxy_async_smem();
+        __syncwarp();
+      }
+      // S buffer c & 1 was last read (as P) by the P.V of block c - 2
+      if (c >= 2 && !wait_all(bar_pvdone, (c - 2) & 1)) {
+        bad = true;
+        break;
+      }
+      tc_fence_after();
+      if (lane == 0) {
+        const uint32_t kst = sstage + s * S::kStage;
+#pragma unroll
+        for (int ks = 0; ks < D / 16; ++ks) {
+          const uint64_t qd = sw128_desc(sq + (ks >> 2) * S::kQPanel + (ks & 3) * 32, 16, 1024);
+          const uint64_t kd = sw128_desc(kst + (ks >> 2) * S::kKVPanel + (ks & 3) * 32, 16, 1024);
+          tc_mma_ss(tmem + S::kColS + 64 * (c & 1), qd, kd, kIdQK, ks > 0 ? 1u : 0u);
+        }
+        tc_commit(bar_sfull + 8 * (c & 1));
+      }
+      __syncwarp();
+      if (c >= 1 && !pv(c - 1)) {
+        bad = true;
+        break;
+      }
+    }
+    if (!bad && !pv(nb - 1)) bad = true;
+    if (bad && lane == 0) raise_error(PKV_ERR_TIMEOUT);
+    // every MMA this thread issued completes before the tensor memory goes
+    if (lane == 0) tc_commit(bar_final);
+    __syncwarp();
+    mbar_wait_bounded(bar_final, 0);
+  } else {
+    // ---- softmax (one thread per row) and epilogue ----------------------------
+    const int r = 32 * (warp & 3) + lane;
+    const uint32_t lane_off = static_cast<uint32_t>(32 * (warp & 3)) << 16;
+    const int tr = r0 + r;
+    const bool valid = tr < R;
+    const int pos = valid ? base + tr / G : -1;
+    float m_ref = -INFINITY, l = 0.f;
+    auto wait_all = [&](uint32_t bar, uint32_t parity) { return __all_sync(kFull, mbar_wait_bounded(bar, parity)); };
+    for (int j = 0; j < nb; ++j) {
+      if (!wait_all(bar_sfull + 8 * (j & 1), (j >> 1) & 1)) {
+        bad = true;
+        break;
+      }
+      tc_fence_after();
+      const uint32_t scol = tmem + lane_off + S::kColS + 64 * (j & 1);
+      const int kb0 = tok0 + j * S::kKeys;
+      uint32_t pages_ok = 0;
+#pragma unroll
+      for (int p = 0; p < S::kPages; ++p) pages_ok |= loaded(j * S::kPages + p) ? (1u << p) : 0u;
+      const bool all_in = pos >= kb0 + S::kKeys - 1 && kb0 + S::kKeys <= tok1 && pages_ok == 0xFu;
+      float x[S::kKeys];
+#pragma unroll
+      for (int h = 0; h < S::kKeys / 32; ++h) {
+        uint32_t v[32];
+        tmem_ld32(scol + 32 * h, v);
+#pragma unroll
+        for (int e = 0; e < 32; ++e) {
+          const int k = kb0 + 32 * h + e;
+          const bool ok = all_in || (k <= pos && k < tok1 && ((pages_ok >> ((32 * h + e) >> 4)) & 1u));
+          x[32 * h + e] = ok ? __uint_as_float(v[e]) * a.qk_scale : -INFINITY;
+        }
+      }
+      float bm = -INFINITY;
+#pragma unroll
+      for (int k = 0; k < S::kKeys; ++k) bm = fmaxf(bm, x[k]);
+      // move the reference max only when this block exceeds it by 2^8
+      float alpha = 1.f;
+      bool rescale = false;
+      if (bm > m_ref + 8.f) {
+        alpha = exp2_sfu(m_ref - bm);  // 0 while no key was seen
+        rescale = m_ref != -INFINITY && j > 0;
+        l *= alpha;
+        m_ref = bm;
+      }
+      const float mr = m_ref == -INFINITY ? 0.f : m_ref;
+      uint32_t ph[S::kKeys / 2], pl[S::kKeys / 2];
+      float sum = 0.f;
+#pragma unroll
+      for (int k = 0; k < S::kKeys; k += 2) {
+        const float p0 = exp2_sfu(x[k] - mr), p1 = exp2_sfu(x[k + 1] - mr);
+        sum += p0 + p1;
+        ph[k / 2] = M::pack(p0, p1);
+        const float2 hv = M::unpack(ph[k / 2]);
+        pl[k / 2] = M::pack(p0 - hv.x, p1 - hv.y);
+      }
+      l += sum;
+      if (__any_sync(kFull, rescale)) {
+        // O holds the P.V of blocks < j: wait for the last of them, then
+        // rescale this thread's row in tensor memory
+        if (!wait_all(bar_pvdone, (j - 1) & 1)) {
+          bad = true;
+          break;
+        }
+        tc_fence_after();
+        const float f = rescale ? alpha : 1.f;
+#pragma unroll
+        for (int h = 0; h < D / 32; ++h) {
+          uint32_t v[32];
+          tmem_ld32(tmem + lane_off + S::kColO + 32 * h, v);
+#pragma unroll
+          for (int e = 0; e < 32; ++e) v[e] = __float_as_uint(__uint_as_float(v[e]) * f);
+          tmem_st32(tmem + lane_off + S::kColO + 32 * h, v);
+        }
+      }
+      tmem_st32(scol, ph);
+      tmem_st32(scol + 32, pl);
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar_pfull + 8 * (j & 1));
+    }
+    // epilogue: every MMA done (the issuer's final commit follows the last
+    // P.V; one phase, so no parity ambiguity), then each row out of tensor
+    // memory
+    if (!bad && !wait_all(bar_final, 0)) bad = true;
+    if (bad) {
+      if (lane == 0) raise_error(PKV_ERR_TIMEOUT);
+    } else {
+      tc_fence_after();
+      const bool has = valid && pos >= tok0;
+      const size_t row = valid ? out_row(tr) : 0;
+      const float inv = has ? 1.f / l : 0.f;
+#pragma unroll
+      for (int h = 0; h < D / 32; ++h) {
+        uint32_t v[32];
+        tmem_ld32(tmem + lane_off + S::kColO + 32 * h, v);
+        if (!valid) continue;
+        if (direct) {
+          uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<T*>(a.out) + row * D + 32 * h);
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            uint32_t w[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+              w[e] = has ? M::pack(__uint_as_float(v[8 * q + 2 * e]) * inv, __uint_as_float(v[8 * q + 2 * e + 1]) * inv)
+                         : 0u;
+            dst[q] = make_uint4(w[0], w[1], w[2], w[3]);
+          }
+        } else if (has) {
+          float4* dst = reinterpret_cast<float4*>(a.ws_o + (row * a.num_parts + z) * D + 32 * h);
+#pragma unroll
+          for (int q = 0; q < 8; ++q)
+            dst[q] = make_float4(__uint_as_float(v[4 * q]), __uint_as_float(v[4 * q + 1]),
+                                 __uint_as_float(v[4 * q + 2]), __uint_as_float(v[4 * q + 3]));
+        }
+      }
+      if (valid && pos >= tok0 && !direct) a.ws_ml[row * a.num_parts + z] = make_float2(m_ref, l);
+    }
+  }
+
+  // ---- teardown ---------------------------------------------------------------
+  tc_fence_before();
+  const bool any_bad = __syncthreads_or(bad);
+  tc_fence_after();
+  if (any_bad && warp == 0 && lane == 0) {
+    // the last block issued into each stage lands before the CTA exits
+    for (int c = max(0, issued - NS); c < issued; ++c) mbar_wait_bounded(bar_full + 8 * (c % NS), (c / NS) & 1);
+  }
+  if (warp == 1) tmem_dealloc(tmem, S::kTmemCols);
+}
+
+}  // namespace pkv

@@ -12,6 +12,7 @@
 #include "decode_fp8.cuh"
 #include "decode_launch.cuh"
 #include "multi_mma.cuh"
+#include "multi_tc.cuh"
 #include "pkv.h"
 
 namespace pkv {
@@ -159,6 +160,42 @@ pkv_status launch_multi_fa(const pkv::MultiArgs& a, const void* k_cache, const v
   return PKV_OK;
 }
 
+// More than kTcAboveRows rows per kv-head: tiles of 128 rows on the tcgen05
+// tensor cores (paged_multi_tc_kernel), accumulators in tensor memory.
+#ifndef PKV_TC_ABOVE_ROWS
+#define PKV_TC_ABOVE_ROWS 32
+#endif
+constexpr int kTcAboveRows = PKV_TC_ABOVE_ROWS;
+constexpr int kTcCode = 200;  // dispatch code of paged_multi_tc_kernel
+constexpr int kTcStages = PKV_TC_STAGES;
+
+template <typename T, int D, int G>
+pkv_status launch_multi_tc(const pkv::MultiArgs& a, const void* k_cache, const void* v_cache, int num_blocks,
+                           cudaStream_t st) {
+  using S = pkv::TcShape<D, kTcStages>;
+  static_assert(kMaxPartition / PKV_BLOCK_SIZE <= S::kMaxPages, "the page table of a partition fits shared memory");
+  CUtensorMap mk, mv;
+  const long long rows = static_cast<long long>(num_blocks) * a.num_kv_heads * PKV_BLOCK_SIZE;
+  if (!encode_cache_map(&mk, k_cache, pkv::Mma<T>::kTmaType, D, rows) ||
+      !encode_cache_map(&mv, v_cache, pkv::Mma<T>::kTmaType, D, rows))
+    return PKV_ECUDA;
+  auto kfn = pkv::paged_multi_tc_kernel<T, D, G, kTcStages>;
+  if (cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(S::kSmem)) !=
+      cudaSuccess)
+    return PKV_ECUDA;
+  const dim3 grid(a.num_kv_heads, a.num_seqs * a.tiles, a.num_parts);
+  if (launch(kfn, grid, dim3(S::kThreads), S::kSmem, st, a, mk, mv) != PKV_OK) return PKV_ECUDA;
+  if (a.num_parts > 1) {
+    const dim3 block(pkv::kMergeWarps * 32);
+    if (a.num_parts >= 32)
+      return launch(MultiMergeK<T, D, 1>::fn, dim3(a.total_q, a.num_q_heads), block, 0, st, a);
+    if (a.num_parts >= 16)
+      return launch(MultiMergeK<T, D, 4>::fn, dim3(a.total_q, (a.num_q_heads + 3) / 4), block, 0, st, a);
+    return launch(MultiMergeK<T, D, 8>::fn, dim3(a.total_q, (a.num_q_heads + 7) / 8), block, 0, st, a);
+  }
+  return PKV_OK;
+}
+
 template <typename T, int D, int G>
 pkv_status dispatch_nt_multi(const pkv::MultiArgs& a, int NT, const void* k, const void* v, int nb,
                              cudaStream_t st) {
@@ -170,6 +207,7 @@ pkv_status dispatch_nt_multi(const pkv::MultiArgs& a, int NT, const void* k, con
     case -3: return launch_multi_rows<T, D, G, 3>(a, k, v, nb, st);
     case -4: return launch_multi_rows<T, D, G, 4>(a, k, v, nb, st);
     case kFaCode: return launch_multi_fa<T, D, G>(a, k, v, nb, st);
+    case kTcCode: return launch_multi_tc<T, D, G>(a, k, v, nb, st);
   }
   return PKV_EINVAL;
 }
@@ -202,7 +240,7 @@ bool encode_fp8_map(CUtensorMap* map, const void* base, int D, long long rows) {
 }
 
 #ifndef PKV_FP8_STAGES
-#define PKV_FP8_STAGES 4
+#define PKV_FP8_STAGES 3
 #endif
 constexpr int kFp8Stages = PKV_FP8_STAGES;  // pages in flight per warp (4 KB each at D = 128)
 
@@ -222,6 +260,90 @@ pkv_status launch_decode_fp8(const pkv::DecodeArgs& a, float v_scale, cudaStream
     if (launch_merge<T, D, ReduceK>(a, a.num_parts, st) != PKV_OK) return PKV_ECUDA;
   }
   return PKV_OK;
+}
+
+// Shared-prefix decode over an FP8 cache: (1) the prefix tiles as exact
+// 16-bit code values in the workspace, (2) the cascade's prefix pass over
+// them on the 16-bit tensor-core path (logits scaled by k_scale, partials by
+// v_scale), (3) the suffix pass over the FP8 cache, (4) the cascade's merge.
+template <typename T, int D, int G>
+pkv_status launch_decode_prefix_fp8(const pkv::DecodeArgs& a0, void* mini_k, void* mini_v, float v_scale,
+                                    cudaStream_t st) {
+  const int row_chunks = D / 8;
+  const long long total = static_cast<long long>(a0.prefix_pages) * a0.num_kv_heads * PKV_BLOCK_SIZE * row_chunks;
+  long long nblk = (2 * total + 255) / 256;
+  if (nblk > 148LL * 16) nblk = 148LL * 16;
+  if (launch(pkv::dequant_prefix_kernel<T>, dim3(static_cast<unsigned>(nblk)), dim3(256), 0, st,
+             reinterpret_cast<const uint2*>(a0.k_cache), reinterpret_cast<const uint2*>(a0.v_cache),
+             static_cast<uint4*>(mini_k), static_cast<uint4*>(mini_v), a0.prefix_blocks, total, a0.num_kv_heads,
+             row_chunks, a0.num_blocks) != PKV_OK)
+    return PKV_ECUDA;
+  {  // prefix pass
+    using S = pkv::MmaShape<T, D, G, kMmaWarps, kMmaStages>;
+    pkv::DecodeArgs ap = a0;
+    ap.k_cache = static_cast<const unsigned char*>(mini_k);
+    ap.v_cache = static_cast<const unsigned char*>(mini_v);
+    ap.num_blocks = a0.prefix_pages;
+    ap.prefix_ident = 1;
+    ap.prefix_out_scale = v_scale;
+    ap.y_offset = 0;
+    CUtensorMap mk, mv;
+    const long long rows = static_cast<long long>(a0.prefix_pages) * a0.num_kv_heads * PKV_BLOCK_SIZE;
+    if (!encode_cache_map(&mk, mini_k, pkv::Mma<T>::kTmaType, D, rows) ||
+        !encode_cache_map(&mv, mini_v, pkv::Mma<T>::kTmaType, D, rows))
+      return PKV_ECUDA;
+    auto kfn = pkv::paged_decode_mma_kernel<T, D, G, kMmaWarps, kMmaStages, true>;
+    if (cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(S::kSmem)) !=
+        cudaSuccess)
+      return PKV_ECUDA;
+    const long long npre = static_cast<long long>(ap.num_qgroups) * ap.num_chunks;
+    if (launch(kfn, dim3(ap.num_kv_heads, static_cast<unsigned>(npre), 1), dim3(kMmaWarps * 32), S::kSmem, st, ap,
+               mk, mv) != PKV_OK)
+      return PKV_ECUDA;
+  }
+  {  // suffix pass
+    using S = pkv::Fp8Shape<D, kMmaWarps, kFp8Stages>;
+    CUtensorMap mk, mv;
+    const long long rows = static_cast<long long>(a0.num_blocks) * a0.num_kv_heads * PKV_BLOCK_SIZE;
+    if (!encode_fp8_map(&mk, a0.k_cache, D, rows) || !encode_fp8_map(&mv, a0.v_cache, D, rows)) return PKV_ECUDA;
+    auto kfn = pkv::paged_decode_fp8_kernel<T, D, G, kMmaWarps, kFp8Stages, true>;
+    if (cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(S::kSmem)) !=
+        cudaSuccess)
+      return PKV_ECUDA;
+    if (launch(kfn, dim3(a0.num_kv_heads, a0.num_seqs, a0.num_parts), dim3(kMmaWarps * 32), S::kSmem, st, a0, mk,
+               mv, v_scale) != PKV_OK)
+      return PKV_ECUDA;
+  }
+  return launch_merge<T, D, PrefixMergeK>(a0, a0.num_chunks + a0.num_parts, st);
+}
+
+template <typename T, int D>
+pkv_status dispatch_group_prefix_fp8(const pkv::DecodeArgs& a, int G, void* mk, void* mv, float v_scale,
+                                     cudaStream_t st) {
+  switch (G) {
+    case 1: return launch_decode_prefix_fp8<T, D, 1>(a, mk, mv, v_scale, st);
+    case 2: return launch_decode_prefix_fp8<T, D, 2>(a, mk, mv, v_scale, st);
+    case 4: return launch_decode_prefix_fp8<T, D, 4>(a, mk, mv, v_scale, st);
+    case 8: return launch_decode_prefix_fp8<T, D, 8>(a, mk, mv, v_scale, st);
+  }
+  return PKV_EINVAL;
+}
+
+// The FP8 cascade's workspace: the 16-bit cascade's, then (1024-aligned) the
+// dequantised prefix tiles of K and of V, [prefix_pages][Hkv][16][D] each.
+struct PrefixFp8Layout {
+  PrefixLayout base;
+  size_t off_k, off_v, total;
+};
+PrefixFp8Layout prefix_fp8_layout(long long B, long long Hq, long long Hkv, long long D, long long max_ctx,
+                                  long long prefix_pages, long long part) {
+  PrefixFp8Layout L;
+  L.base = prefix_layout(B, Hq, D, max_ctx, prefix_pages, part);
+  const size_t tiles = static_cast<size_t>(prefix_pages * Hkv * PKV_BLOCK_SIZE * D * 2);
+  L.off_k = (L.base.total + 1023) / 1024 * 1024;
+  L.off_v = L.off_k + (tiles + 1023) / 1024 * 1024;
+  L.total = L.off_v + tiles;
+  return L;
 }
 
 template <typename T, int D>
@@ -470,13 +592,32 @@ size_t pkv_decode_prefix_workspace_bytes(int num_seqs, int num_q_heads, int head
 }  // extern "C"
 
 namespace {
+// The step's writes a fused decode makes (pkv_decode_step); all null when
+// the decode stands alone.
+struct StepWrites {
+  const void* k_new = nullptr;
+  const void* v_new = nullptr;
+  const int64_t* slots = nullptr;
+  const int32_t* copies = nullptr;
+  int n_copies = 0;
+};
+
+void attach_step(pkv::DecodeArgs* a, const StepWrites& w) {
+  a->k_new = static_cast<const unsigned char*>(w.k_new);
+  a->v_new = static_cast<const unsigned char*>(w.v_new);
+  a->slots = w.slots;
+  a->copies = w.copies;
+  a->n_copies = w.n_copies;
+}
+
 pkv_status decode_prefix_impl(void* out, const void* q, const void* k_cache, const void* v_cache,
                                              const int32_t* block_tables, int max_blocks_per_seq,
                                              const int32_t* context_lens, int max_context_len,
                                              const int32_t* prefix_blocks, int prefix_pages, int num_seqs,
                                              int num_q_heads, int num_kv_heads, int head_dim, int num_blocks,
                                              float scale, int partition_tokens, pkv_dtype dtype, void* workspace,
-                                             size_t workspace_bytes_given, int phase, void* stream) {
+                                             size_t workspace_bytes_given, int phase, void* stream,
+                                             const StepWrites& step = StepWrites{}) {
   if (dtype != PKV_F16 && dtype != PKV_BF16) return PKV_EINVAL;  // tensor-core path only
   if (prefix_pages <= 0 || prefix_pages > max_blocks_per_seq) return PKV_EINVAL;
   pkv::DecodeArgs a{};
@@ -498,6 +639,7 @@ pkv_status decode_prefix_impl(void* out, const void* q, const void* k_cache, con
   a.wp_ml = reinterpret_cast<float2*>(ws + L.off_pml);
   a.conform = reinterpret_cast<int*>(ws + L.off_conform);
   a.prefix_blocks = prefix_blocks;
+  attach_step(&a, step);
   a.prefix_pages = prefix_pages;
   a.chunk_pages = kPrefixChunkPages;
   a.num_chunks = static_cast<int>(L.chunks);
@@ -545,6 +687,50 @@ pkv_status pkv_paged_attention_decode_prefix_phase(void* out, const void* q, con
                             max_context_len, prefix_blocks, prefix_pages, num_seqs, num_q_heads, num_kv_heads,
                             head_dim, num_blocks, scale, partition_tokens, dtype, workspace, workspace_bytes_given,
                             phase, stream);
+}
+
+
+pkv_status pkv_decode_step(void* out, const void* q, void* k_cache, void* v_cache, const void* k_new,
+                           const void* v_new, const int64_t* slot_mapping, const int32_t* copies, int num_copies,
+                           const int32_t* block_tables, int max_blocks_per_seq, const int32_t* context_lens,
+                           int max_context_len, const int32_t* prefix_blocks, int prefix_pages, int num_seqs,
+                           int num_q_heads, int num_kv_heads, int head_dim, int num_blocks, float scale,
+                           int partition_tokens, pkv_dtype dtype, void* workspace, size_t workspace_bytes_given,
+                           void* stream) {
+  if (dtype != PKV_F16 && dtype != PKV_BF16) return PKV_EINVAL;  // tensor-core path only
+  if (num_copies < 0 || num_copies > num_seqs || prefix_pages < 0) return PKV_EINVAL;
+  if (num_seqs > 0 && (!k_new || !v_new || !slot_mapping || !aligned16(k_new) || !aligned16(v_new)))
+    return PKV_EINVAL;
+  if (num_copies > 0 && copies == nullptr) return PKV_EINVAL;
+  StepWrites w;
+  w.k_new = k_new;
+  w.v_new = v_new;
+  w.slots = slot_mapping;
+  w.copies = copies;
+  w.n_copies = num_copies;
+  if (prefix_pages > 0)
+    return decode_prefix_impl(out, q, k_cache, v_cache, block_tables, max_blocks_per_seq, context_lens,
+                              max_context_len, prefix_blocks, prefix_pages, num_seqs, num_q_heads, num_kv_heads,
+                              head_dim, num_blocks, scale, partition_tokens, dtype, workspace, workspace_bytes_given,
+                              -1, stream, w);
+  pkv::DecodeArgs a{};
+  long long P = 0;
+  const pkv_status st0 = prepare_decode(out, q, k_cache, v_cache, block_tables, max_blocks_per_seq, context_lens,
+                                        max_context_len, num_seqs, num_q_heads, num_kv_heads, head_dim, num_blocks,
+                                        scale, partition_tokens, dtype, &a, &P);
+  if (st0 != PKV_OK || num_seqs == 0) return st0;
+  const size_t need = workspace_bytes(num_seqs, num_q_heads, head_dim, P);
+  if (need > 0 && (workspace == nullptr || workspace_bytes_given < need || !aligned16(workspace)))
+    return PKV_EINVAL;
+  a.ws_o = static_cast<float*>(need ? workspace : nullptr);
+  a.ws_ml = need ? reinterpret_cast<float2*>(static_cast<float*>(workspace) +
+                                              static_cast<size_t>(num_seqs) * num_q_heads * P * head_dim)
+                 : nullptr;
+  attach_step(&a, w);
+  const int G = num_q_heads / num_kv_heads;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (dtype == PKV_F16) return dispatch_dim_mma<__half>(a, head_dim, G, st);
+  return dispatch_dim_mma<__nv_bfloat16>(a, head_dim, G, st);
 }
 
 }  // extern "C"
@@ -683,10 +869,11 @@ pkv_status pkv_paged_attention_multi(void* out, const void* q, const void* k_cac
   if (static_cast<long long>(num_blocks) * num_kv_heads * PKV_BLOCK_SIZE > 0x7fffffffLL) return PKV_EINVAL;
   const int G = num_q_heads / num_kv_heads;
   const long long rows_max = static_cast<long long>(max_query_len) * G;
-  const bool fa = rows_max > kFaAboveRows;
-  const int NW = fa ? 0 : multi_rows_warps(rows_max);
-  const int NT = fa ? kFaCode : NW ? -NW : multi_ntiles(rows_max);
-  const int tile_rows = fa ? 16 * kFaWarps : 8 * (NW ? NW : NT);
+  const bool tc = rows_max > kTcAboveRows;
+  const bool fa = !tc && rows_max > kFaAboveRows;
+  const int NW = (fa || tc) ? 0 : multi_rows_warps(rows_max);
+  const int NT = tc ? kTcCode : fa ? kFaCode : NW ? -NW : multi_ntiles(rows_max);
+  const int tile_rows = tc ? 128 : fa ? 16 * kFaWarps : 8 * (NW ? NW : NT);
   const long long tiles = (rows_max + tile_rows - 1) / tile_rows;
   const long long P = (static_cast<long long>(max_context_len) + part - 1) / part;
   if (tiles * num_seqs > 65535 || P > 65535) return PKV_EINVAL;
@@ -723,6 +910,67 @@ pkv_status pkv_paged_attention_multi(void* out, const void* q, const void* k_cac
     return dispatch_group_multi<T, 128>(a, G, NT, k_cache, v_cache, num_blocks, st);
   };
   if (dtype == PKV_F16) return run(__half{});
+  return run(__nv_bfloat16{});
+}
+
+size_t pkv_decode_prefix_fp8_workspace_bytes(int num_seqs, int num_q_heads, int num_kv_heads, int head_dim,
+                                             int max_context_len, int prefix_pages, int partition_tokens) {
+  const int part = resolve_prefix_partition(partition_tokens, max_context_len, prefix_pages);
+  if (part < 0 || num_seqs < 0 || num_q_heads <= 0 || num_kv_heads <= 0 || !head_dim_ok(head_dim) ||
+      max_context_len < 0 || prefix_pages <= 0)
+    return 0;
+  return prefix_fp8_layout(num_seqs, num_q_heads, num_kv_heads, head_dim, max_context_len, prefix_pages, part).total;
+}
+
+pkv_status pkv_paged_attention_decode_prefix_fp8(void* out, const void* q, const void* k_cache,
+                                                 const void* v_cache, const int32_t* block_tables,
+                                                 int max_blocks_per_seq, const int32_t* context_lens,
+                                                 int max_context_len, const int32_t* prefix_blocks,
+                                                 int prefix_pages, int num_seqs, int num_q_heads, int num_kv_heads,
+                                                 int head_dim, int num_blocks, float scale, float k_scale,
+                                                 float v_scale, int partition_tokens, pkv_dtype q_dtype,
+                                                 void* workspace, size_t workspace_bytes_given, void* stream) {
+  if (q_dtype != PKV_F16 && q_dtype != PKV_BF16) return PKV_EINVAL;
+  if (!std::isfinite(k_scale) || !std::isfinite(v_scale) || !(k_scale > 0.f) || !(v_scale > 0.f))
+    return PKV_EINVAL;
+  if (prefix_pages <= 0 || prefix_pages > max_blocks_per_seq) return PKV_EINVAL;
+  const int part = resolve_prefix_partition(partition_tokens, max_context_len, prefix_pages);
+  if (part < 0) return PKV_EINVAL;
+  pkv::DecodeArgs a{};
+  long long P = 0;
+  const pkv_status st0 = prepare_decode(out, q, k_cache, v_cache, block_tables, max_blocks_per_seq, context_lens,
+                                        max_context_len, num_seqs, num_q_heads, num_kv_heads, head_dim, num_blocks,
+                                        scale, part, q_dtype, &a, &P);
+  if (st0 != PKV_OK || num_seqs == 0) return st0;
+  if (prefix_blocks == nullptr) return PKV_EINVAL;
+  if (static_cast<long long>(prefix_pages) * num_kv_heads * PKV_BLOCK_SIZE > 0x7fffffffLL) return PKV_EINVAL;
+  const PrefixFp8Layout L =
+      prefix_fp8_layout(num_seqs, num_q_heads, num_kv_heads, head_dim, max_context_len, prefix_pages, a.partition);
+  if (workspace == nullptr || workspace_bytes_given < L.total || !aligned16(workspace)) return PKV_EINVAL;
+  unsigned char* ws = static_cast<unsigned char*>(workspace);
+  a.num_parts = static_cast<int>(L.base.parts);
+  a.ws_o = reinterpret_cast<float*>(ws + L.base.off_so);
+  a.ws_ml = reinterpret_cast<float2*>(ws + L.base.off_sml);
+  a.wp_o = reinterpret_cast<float*>(ws + L.base.off_po);
+  a.wp_ml = reinterpret_cast<float2*>(ws + L.base.off_pml);
+  a.conform = reinterpret_cast<int*>(ws + L.base.off_conform);
+  a.prefix_blocks = prefix_blocks;
+  a.prefix_pages = prefix_pages;
+  a.chunk_pages = kPrefixChunkPages;
+  a.num_chunks = static_cast<int>(L.base.chunks);
+  a.num_qgroups = (num_seqs * (num_q_heads / num_kv_heads) + kMmaWarps * 16 - 1) / (kMmaWarps * 16);
+  if (static_cast<long long>(a.num_qgroups) * a.num_chunks > 65535 || a.num_parts > 65535) return PKV_EINVAL;
+  a.qk_scale *= k_scale;
+  const int G = num_q_heads / num_kv_heads;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  void* mk = ws + L.off_k;
+  void* mv = ws + L.off_v;
+  auto run = [&](auto tag) -> pkv_status {
+    using T = decltype(tag);
+    if (head_dim == 64) return dispatch_group_prefix_fp8<T, 64>(a, G, mk, mv, v_scale, st);
+    return dispatch_group_prefix_fp8<T, 128>(a, G, mk, mv, v_scale, st);
+  };
+  if (q_dtype == PKV_F16) return run(__half{});
   return run(__nv_bfloat16{});
 }
 

@@ -119,3 +119,28 @@ def make_multi_case(ctx, nq, Hq, Hkv, D, dtype, seed, v_scale=1.0):
         q = (q.view(np.uint32) >> 16).astype(np.uint16)
     return dict(q=q, k=k, v=v, tables=tables, ctx=np.array(ctx, dtype=np.int32), qs=qs, rows_k=rows_k,
                 rows_v=rows_v, dtype=dtype, G=Hq // Hkv)
+
+
+# Mantissa bits of the 16-bit output formats and their smallest normal
+# exponent (below it the spacing stays that of the smallest binade).
+_FMT = {"f16": (10, -14), "bf16": (7, -126)}
+
+
+def half_ulp(x, dtype):
+    """Half the spacing of the output format ``dtype`` at |x| (elementwise):
+    the error of rounding the exact value to that format once."""
+    bits, emin = _FMT[dtype]
+    a = np.abs(np.asarray(x, dtype=np.float64))
+    e = np.where(a > 0, np.floor(np.log2(np.where(a > 0, a, 1.0))), emin)
+    e = np.maximum(e, emin)
+    return np.ldexp(1.0, (e - bits - 1).astype(np.int64))
+
+
+def ulp_aware_bound(ref, dtype, tol):
+    """Elementwise bound for a 16-bit output of a kernel that computes in
+    fp32 and rounds once: the stated max-abs tolerance, or -- where the
+    output's magnitude makes the format's own rounding larger -- half an ulp
+    of the fp64 reference in the output format plus a fp32-level slack of
+    2^-14 |ref| (far below the 16-bit formats' precision)."""
+    ref = np.asarray(ref, dtype=np.float64)
+    return np.maximum(tol, half_ulp(ref, dtype) + np.ldexp(np.abs(ref), -14))

@@ -171,9 +171,10 @@ def test_multi_workspace_and_rejections(lib):
         a = list(args)
         a[idx] = bad
         assert lib.pkv_paged_attention_multi(*a) == 1, (idx, bad)
-    # grid limit: num_seqs * ceil(max_query_len * G / 16) > 65535
+    # grid limit: num_seqs * (row tiles per sequence) > 65535 (4096 tokens x
+    # G 4 = 16384 rows: 128 tiles of 128 rows)
     a = list(args)
-    a[9], a[11] = 4096, 300
+    a[9], a[11] = 4096, 600
     assert lib.pkv_paged_attention_multi(*a) == 1
     # nothing to do
     a = list(args)
@@ -220,3 +221,20 @@ def test_cow_copy_rows():
 def test_selftest_bounded_wait_rejects_limits(lib):
     for bad in (0, -5, (1 << 32) + 1):
         assert lib.pkv_selftest_bounded_wait(bad, None) == 1, bad
+
+
+def test_decode_step_rejections(lib):
+    """pkv_decode_step checks its own arguments (the step's writes) before
+    anything is launched, then those of the decode it fuses."""
+    f = ctypes.c_float
+    ok = [FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 2, FAKE, 8, FAKE, 100, None, 0, 4, 8, 2, 128, 64, f(0.1),
+          0, 1, None, 0, None]
+    for idx, bad in ((22, 0), (22, 3), (8, -1), (8, 5), (7, None), (4, None), (5, ODD), (6, None), (14, -1),
+                     (18, 96), (17, 3), (12, 8 * 16 + 1)):
+        a = list(ok)
+        a[idx] = bad
+        assert lib.pkv_decode_step(*a) == 1, (idx, bad)
+    # the cascade form needs its prefix blocks and workspace
+    a = list(ok)
+    a[14] = 4
+    assert lib.pkv_decode_step(*a) == 1

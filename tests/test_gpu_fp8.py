@@ -8,6 +8,7 @@ import pytest
 import torch
 
 import oracle
+from helpers import ulp_aware_bound
 from oracle import fp8
 
 pytestmark = pytest.mark.gpu
@@ -36,9 +37,9 @@ def to_dev(a, dt):
     return t.cuda()
 
 
-def build(ctx, Hkv, D, dt, ks, vs, seed):
+def build(ctx, Hkv, D, dt, ks, vs, seed, sigma=1.0):
     """An FP8 pool written through the GPU append and the oracle append from
-    the same 16-bit values; returns both plus tables."""
+    the same 16-bit values (N(0, sigma^2)); returns both plus tables."""
     m = pkv()
     rng = np.random.default_rng(seed)
     pages = [-(-c // 16) for c in ctx]
@@ -54,8 +55,8 @@ def build(ctx, Hkv, D, dt, ks, vs, seed):
         slots += [int(tables[b, j // 16]) * 16 + j % 16 for j in range(c)]
     slots = np.array(slots, dtype=np.int64)
     n = len(slots)
-    kx = storage(rng.standard_normal((n, Hkv, D)).astype(np.float32), dt)
-    vx = storage(rng.standard_normal((n, Hkv, D)).astype(np.float32), dt)
+    kx = storage(rng.standard_normal((n, Hkv, D)).astype(np.float32) * sigma, dt)
+    vx = storage(rng.standard_normal((n, Hkv, D)).astype(np.float32) * sigma, dt)
     ref = oracle.RefCache(nb, Hkv, D, "e4m3")
     ref.append_fp8(kx, vx, slots, dt, ks, vs)
     kc = torch.full((nb, Hkv, 16, D), 0x7F, dtype=torch.uint8, device="cuda")
@@ -182,3 +183,90 @@ def test_cache_with_fp8_pool_steps_like_the_oracle():
     held = sorted({b for t in ref.tables.values() for b in t})
     assert np.array_equal(cache.k.cpu().numpy()[held], dev.k[held])
     assert np.array_equal(cache.v.cpu().numpy()[held], dev.v[held])
+
+
+@pytest.mark.parametrize("case", CASES[:4], ids=lambda c: f"{c[4]}_G{c[1] // c[2]}_D{c[3]}")
+@pytest.mark.parametrize("scale", [None, 0.5])
+def test_decode_fp8_wide_values(case, scale):
+    """K, V and q drawn N(0, 4) (scales covering 6 standard deviations),
+    with the default logit scale and a sharper one (peaked attention, whose
+    outputs approach single V values of magnitude up to ~8).  Where the
+    output's magnitude makes the 16-bit format's own half-ulp larger than
+    the stated tolerance (bf16 past 4, fp16 past 8), the bound is that
+    half-ulp of the oracle's value plus a 2^-14 relative slack; elsewhere
+    the stated tolerance."""
+    m = pkv()
+    ctx, Hq, Hkv, D, dt = case
+    ks = vs = 2.0 * 6.0 / 448.0
+    ref, kc, vc, tables, lens = build(ctx, Hkv, D, dt, ks, vs, seed=7 * len(ctx) + D, sigma=2.0)
+    rng = np.random.default_rng(D + len(ctx))
+    q = storage(rng.standard_normal((len(ctx), Hq, D)).astype(np.float32) * 2.0, dt)
+    sc = D ** -0.5 if scale is None else scale
+    want = oracle.paged_decode(q, ref.k, ref.v, tables, lens, sc, dt, kv_dtype="e4m3", k_scale=ks, v_scale=vs)
+    out = m.paged_attention_decode_fp8(to_dev(q, dt), kc, vc, torch.from_numpy(tables).cuda(),
+                                       torch.from_numpy(lens).cuda(), int(lens.max()), sc, ks, vs)
+    torch.cuda.synchronize()
+    assert m.get_error() == 0
+    got = out.float().cpu().numpy()
+    assert np.isfinite(got).all()
+    assert (np.abs(got - want) <= ulp_aware_bound(want, dt, TOL[dt])).all()
+    if scale is not None:
+        assert np.abs(want).max() > 4.0  # the wide range is really exercised
+
+
+@pytest.mark.parametrize("case", [
+    ("f16", 12, 256, (1, 100), 8, 8, 128, 0),
+    ("bf16", 20, 512, (0, 700), 16, 2, 128, 0),
+    ("bf16", 9, 160, (3, 40), 8, 2, 64, 0),
+    ("f16", 12, 256, (1, 300), 8, 4, 128, 64),
+], ids=lambda c: f"{c[0]}_B{c[1]}_G{c[4] // c[5]}_D{c[6]}_p{c[7]}")
+def test_cascade_over_fp8_cache_matches_oracle(case):
+    """The shared-prefix decode over an FP8 pool (prefix pass on the exact
+    16-bit code values, suffix pass over the codes, merge) against the
+    oracle on the stored values, and against the plain FP8 decode; a
+    relabelled table (a sequence that does not start with the prefix) is
+    decoded over its whole context."""
+    import workloads
+    from paged_kv_cache_365_b200.replay import build_step
+    m = pkv()
+    dt, B, pre, suf, Hq, Hkv, D, partition = case
+    wl = workloads.prefix13b(seed=B + pre, B=B, prefix_tokens=pre, suffix_range=suf, Hq=Hq, Hkv=Hkv, D=D, dtype=dt,
+                             name="fp8_cascade")
+    vals = workloads.draw_values(wl)
+    st = build_step(wl, vals, "cuda")
+    c = st["cache"]
+    m.copy_blocks(c.k, c.v, st["cow_pairs"])
+    m.kv_append(st["k_new"], st["v_new"], c.k, c.v, st["slot_mapping"])
+    ks, vs = 6.0 / 448.0, 5.0 / 448.0
+    NB = c.k.shape[0]
+    k8 = torch.empty(c.k.shape, dtype=torch.uint8, device="cuda")
+    v8 = torch.empty(c.v.shape, dtype=torch.uint8, device="cuda")
+    all_slots = torch.arange(NB * 16, dtype=torch.int64, device="cuda")
+    rows_k = c.k.permute(0, 2, 1, 3).reshape(NB * 16, Hkv, D).contiguous()
+    rows_v = c.v.permute(0, 2, 1, 3).reshape(NB * 16, Hkv, D).contiguous()
+    m.kv_append_fp8(rows_k, rows_v, k8, v8, all_slots, ks, vs)
+    tables, lens = st["host"]["block_tables"], st["host"]["context_lens"]
+    tables = tables.copy()
+    pp = m.common_prefix_pages(tables, lens)
+    assert pp >= 8
+    # sequence 1 keeps its blocks but its table names a different block for
+    # page 0: give it a private copy of that block (codes copied bit for bit)
+    spare = int(min(set(range(NB)) - set(tables.ravel().tolist())))  # a block no table of the batch names
+    k8[spare] = k8[int(tables[1, 0])]
+    v8[spare] = v8[int(tables[1, 0])]
+    tables[1, 0] = spare
+    prefix = torch.from_numpy(np.ascontiguousarray(tables[0, :pp])).cuda()
+    dt_t = torch.from_numpy(np.ascontiguousarray(tables)).cuda()
+    out = m.paged_attention_decode_prefix_fp8(st["q"], k8, v8, dt_t, st["context_lens"], st["max_context_len"], prefix,
+                                              wl.scale, ks, vs, partition=partition)
+    plain = m.paged_attention_decode_fp8(st["q"], k8, v8, dt_t, st["context_lens"], st["max_context_len"], wl.scale,
+                                         ks, vs)
+    torch.cuda.synchronize()
+    assert m.get_error() == 0
+    codes_k, codes_v = k8.cpu().numpy(), v8.cpu().numpy()
+    want = oracle.paged_decode(vals["q"], codes_k, codes_v, tables, lens, wl.scale, dt, kv_dtype="e4m3",
+                               k_scale=ks, v_scale=vs)
+    got = out.float().cpu().numpy()
+    assert np.isfinite(got).all()
+    assert np.abs(got - want).max() <= TOL[dt]
+    assert np.abs(got - plain.float().cpu().numpy()).max() <= TOL[dt]

@@ -8,7 +8,7 @@ import pytest
 import torch
 
 import oracle
-from helpers import make_multi_case
+from helpers import make_multi_case, ulp_aware_bound
 
 pytestmark = pytest.mark.gpu
 
@@ -227,3 +227,28 @@ def test_multi_step_through_the_cache_api():
     assert np.array_equal(cache.v.cpu().view(torch.int16).numpy()[held], dev.v.view(np.int16)[held])
     want = oracle.paged_multi(q, dev.k, dev.v, tables, lens, qs, D ** -0.5, "f16")
     assert np.abs(out.float().numpy() - want).max() <= TOL["f16"]
+
+
+@pytest.mark.parametrize("case", [
+    ([700, 1500, 90], [5, 5, 3], 32, 8, 128, "bf16"),     # 20 rows: row-split kernel
+    ([1300, 260], [4, 6], 32, 4, 128, "f16"),             # 24 rows
+    ([900, 300], [20, 11], 16, 2, 64, "bf16"),            # 160 rows: 128-row tiles
+    ([2500, 130], [100, 64], 8, 8, 128, "f16"),           # 100 rows
+], ids=lambda c: f"{c[5]}_G{c[2] // c[3]}_D{c[4]}_rows{max(c[1]) * c[2] // c[3]}")
+@pytest.mark.parametrize("scale", [None, 3.0])
+def test_multi_wide_values(case, scale):
+    """V drawn N(0, 4): peaked attention returns values up to ~8, where the
+    16-bit formats' own half-ulp passes the stated tolerance.  The bound is
+    the stated tolerance, or that half-ulp of the oracle's value plus a
+    2^-14 relative slack where it is larger."""
+    ctx, nq, Hq, Hkv, D, dt = case
+    c = make_multi_case(ctx, nq, Hq, Hkv, D, dt, seed=sum(ctx) + 13, v_scale=2.0)
+    sc = D ** -0.5 if scale is None else scale
+    want = oracle.paged_multi(c["q"], c["k"], c["v"], c["tables"], c["ctx"], c["qs"], sc, dt)
+    for partition in (0, 64):
+        got, err = run_gpu(c, sc, partition)
+        assert err == 0
+        assert np.isfinite(got).all()
+        assert (np.abs(got - want) <= ulp_aware_bound(want, dt, TOL[dt])).all()
+    if scale is not None:
+        assert np.abs(want).max() > 4.0

@@ -214,3 +214,72 @@ def test_partial_copy_append_matches_oracle_on_every_token():
     got, _ = cascade(st, wl)
     want = oracle.paged_decode(vals["q"], ref["cache"].k, ref["cache"].v, tables, lens, wl.scale, wl.dtype)
     assert np.abs(got - want).max() <= TOL["f16"]
+
+
+FUSED_CASES = [
+    (workloads.prefix13b(seed=61, B=24, prefix_tokens=128, suffix_range=(1, 90), Hq=8, Hkv=8, D=128,
+                         dtype="f16", name="fused_f16"), True, 0),
+    (workloads.prefix13b(seed=62, B=20, prefix_tokens=512, suffix_range=(0, 700), Hq=16, Hkv=2, D=128,
+                         dtype="bf16", name="fused_bf16_gqa"), True, 0),
+    (workloads.prefix13b(seed=63, B=20, prefix_tokens=512, suffix_range=(0, 700), Hq=16, Hkv=2, D=128,
+                         dtype="bf16", name="fused_bf16_plain"), False, 0),
+    (workloads.prefix13b(seed=64, B=12, prefix_tokens=256, suffix_range=(1, 300), Hq=8, Hkv=4, D=64,
+                         dtype="f16", name="fused_f16_split"), False, 64),
+    (workloads.prefix13b(seed=65, B=12, prefix_tokens=256, suffix_range=(1, 300), Hq=8, Hkv=4, D=128,
+                         dtype="bf16", name="fused_bf16_cascade_split"), True, 64),
+]
+
+
+@pytest.mark.parametrize("case", FUSED_CASES, ids=lambda c: c[0].name)
+def test_fused_step_matches_separate_calls(case):
+    """pkv_decode_step (the copy-on-write copies, the append and the decode
+    in one launch: the CTA that reads a sequence's last page writes its
+    token first) against kv_append_copy followed by the decode on the same
+    state: every token row of the pool and the output bit-identical, and
+    the output within tolerance of the oracle.  Cascade and plain decode,
+    with and without several partitions per sequence."""
+    import paged_kv_cache_365_b200 as pkv
+    from paged_kv_cache_365_b200.replay import build_step
+    wl, use_cascade, partition = case
+    vals = workloads.draw_values(wl)
+    st = build_step(wl, vals, "cuda")
+    c = st["cache"]
+    copies = pkv.cow_copy_rows(st["host"]["cow_pairs"], st["host"]["step_slots"])
+    assert len(copies) > 0
+    dcopies = torch.from_numpy(copies).cuda()
+    tables, lens = st["host"]["block_tables"], st["host"]["context_lens"]
+    prefix = None
+    if use_cascade:
+        pp = pkv.cascade_prefix_pages(tables, lens, c.k.dtype)
+        assert pp > 0
+        prefix = torch.from_numpy(np.ascontiguousarray(tables[0, :pp])).cuda()
+    k2, v2 = c.k.clone(), c.v.clone()
+    # separate launches on the copy of the pool
+    pkv.kv_append_copy(st["k_new"], st["v_new"], k2, v2, st["slot_mapping"], dcopies)
+    if use_cascade:
+        sep = pkv.paged_attention_decode_prefix(st["q"], k2, v2, st["block_tables"], st["context_lens"],
+                                                st["max_context_len"], prefix, wl.scale, partition=partition)
+    else:
+        sep = pkv.paged_attention_decode(st["q"], k2, v2, st["block_tables"], st["context_lens"],
+                                         st["max_context_len"], wl.scale, partition=partition)
+    fused = pkv.decode_step(st["q"], c.k, c.v, st["k_new"], st["v_new"], st["slot_mapping"], dcopies,
+                            st["block_tables"], st["context_lens"], st["max_context_len"], wl.scale,
+                            prefix_blocks=prefix, partition=partition)
+    torch.cuda.synchronize()
+    assert pkv.get_error() == 0
+    assert torch.equal(fused.view(torch.int16), sep.view(torch.int16))
+    gk, gv = c.k.cpu().view(torch.int16).numpy(), c.v.cpu().view(torch.int16).numpy()
+    sk, sv = k2.cpu().view(torch.int16).numpy(), v2.cpu().view(torch.int16).numpy()
+    for b in range(wl.B):
+        tok = np.arange(int(lens[b]))
+        blk, off = tables[b, tok // 16], tok % 16
+        assert np.array_equal(gk[blk, :, off], sk[blk, :, off])
+        assert np.array_equal(gv[blk, :, off], sv[blk, :, off])
+    ref = oracle.replay(wl, vals)
+    for b in range(wl.B):
+        tok = np.arange(int(lens[b]))
+        blk, off = tables[b, tok // 16], tok % 16
+        assert np.array_equal(gk[blk, :, off], ref["cache"].k[blk, :, off].view(np.int16))
+    want = oracle.paged_decode(vals["q"], ref["cache"].k, ref["cache"].v, ref["block_tables"], ref["context_lens"],
+                               wl.scale, wl.dtype)
+    assert np.abs(fused.float().cpu().numpy() - want).max() <= TOL[wl.dtype]
