@@ -4,9 +4,9 @@ sequence-steps/s and us per step.
 One step = the whole device path for one batch: the copy-on-write block
 copies (when the step has any), the slot-mapped append of the new tokens'
 K/V, and paged decode attention (partition kernel, plus the merge kernel
-when a sequence spans several partitions).  With a 16-bit cache the step is
-one fused launch (pkv_decode_step) plus the merge; --unfused runs the
-copies + append as their own launch.  The host allocator's step is
+when a sequence spans several partitions).  A plain 16-bit step is one
+fused launch (pkv_decode_step) plus the merge; --unfused runs the append as
+its own launch (the cascade always does).  The host allocator's step is
 planned before the timed region (host microseconds, not device work); the
 same planned step is replayed every iteration (its copies and appends are
 idempotent).
@@ -318,7 +318,10 @@ def run_cuda(args, rank, world, local_rank, workload=None, graph=None):
         cache.fp8 = (FP8_SCALE, FP8_SCALE)
         torch.cuda.synchronize()
     prefix = torch.from_numpy(np.ascontiguousarray(st["host"]["block_tables"][0, :pp])).to(dev) if use_cascade else None
-    fused_step = not fp8 and not (use_cascade and args.cascade_overlap) and wl.dtype != "f32" and not args.unfused
+    # a plain 16-bit step is one launch (+ merge); the cascade keeps its copies
+    # and append in their own launch (measured faster: their loads stay off
+    # the short suffix CTAs' critical path)
+    fused_step = not fp8 and not use_cascade and wl.dtype != "f32" and not args.unfused
     if use_cascade:
         ws = cache.workspace(pkv.decode_prefix_workspace_bytes(B, Hq, D, max_ctx, pp, args.partition))
         # [copies + append (one launch)], cascade (one launch, or prefix + suffix passes), merge
@@ -383,8 +386,6 @@ def run_cuda(args, rank, world, local_rank, workload=None, graph=None):
             pkv.paged_attention_decode(st["q"], cache.k, cache.v, st["block_tables"], st["context_lens"], max_ctx,
                                        scale, out=out, workspace=ws, partition=args.partition)
 
-    # a 16-bit step is one launch (+ merge): each sequence's copy-on-write
-    # copy and append are made by the decode CTA that reads its last page
     fused = fused_step
 
     def eager_step():

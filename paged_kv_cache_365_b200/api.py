@@ -875,9 +875,10 @@ class PagedKVCache:
 
         ``cow_pairs``: int32 [n, 2] (src, dst) whole-block copies, or [n, 3]
         (src, dst, rows) from ``cow_copy_rows``: the copies cut to the rows
-        that hold tokens.  With [n, 3] copies (or none) and a 16-bit pool the
-        whole step is one decode launch (pkv_decode_step): each sequence's
-        copy and append are made by the CTA that then reads its last page.
+        that hold tokens.  With [n, 3] copies (or none), a 16-bit pool and
+        no shared prefix the whole step is one decode launch
+        (pkv_decode_step): each sequence's copy and append are made by the
+        warp that then stages its last page.
         Inputs may be host tensors (pinned for asynchronous copies) or
         device tensors.  Host inputs are uploaded, and a host ``out`` is
         filled, on two side streams with double-buffered device copies, so a
@@ -897,16 +898,15 @@ class PagedKVCache:
             B, hq = q.shape[0], q.shape[1]
             res = out if (out is not None and out.device == dev) else stg.output(st, q.shape, self.dtype)
             sc = (1.0 / math.sqrt(self.D)) if scale is None else scale
-            fused = (self.fp8 is None and self.dtype != torch.float32 and
+            # a plain decode takes its copies and append into its own launch;
+            # the cascade's short suffix CTAs keep them in a launch of their own
+            fused = (self.fp8 is None and self.dtype != torch.float32 and prefix_blocks is None and
                      (cow_pairs.shape[0] == 0 or cow_pairs.shape[1] == 3))
             if fused:  # copies, append and decode in one launch (+ merge)
-                pp = 0 if prefix_blocks is None else prefix_blocks.numel()
-                ws = self.workspace(decode_prefix_workspace_bytes(B, hq, self.D, max_context_len, pp, partition)
-                                    if pp else decode_workspace_bytes(B, hq, self.D, max_context_len, partition))
+                ws = self.workspace(decode_workspace_bytes(B, hq, self.D, max_context_len, partition))
                 decode_step(x["q"], self.k, self.v, x["k"], x["v"], x["slots"],
                             x["pairs"] if cow_pairs.shape[0] else None, x["tables"], x["lens"], max_context_len, sc,
-                            prefix_blocks=x["prefix"] if pp else None, out=res, workspace=ws, partition=partition,
-                            stream=st)
+                            out=res, workspace=ws, partition=partition, stream=st)
                 stg.finish(st, res, out)
                 return res
             self._copy_append(cow_pairs.shape, x, st)

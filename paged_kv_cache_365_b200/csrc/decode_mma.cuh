@@ -353,18 +353,17 @@ __device__ __forceinline__ void fused_step_append(const DecodeArgs& a, int b, in
   const bool ok = s >= 0 && blk < a.num_blocks;
   if (s >= 0 && !ok && lane == 0) raise_error(PKV_ERR_SLOT_RANGE);
   if (!ok) return;
-  // the copy into this block, if any
+  // the copy into this block, if any: every lane scans its share of the
+  // list with independent loads (one round trip), the first match wins
+  int first = 0x7fffffff;
+  for (int i = lane; i < a.n_copies; i += 32)
+    if (a.copies[3 * i + 1] == static_cast<int>(blk)) first = min(first, i);
+#pragma unroll
+  for (int m = 16; m >= 1; m >>= 1) first = min(first, __shfl_xor_sync(kFull, first, m));
   int src = -1, rows = 0;
-  for (int i0 = 0; i0 < a.n_copies; i0 += 32) {
-    const int i = i0 + lane;
-    const bool hit = i < a.n_copies && a.copies[3 * i + 1] == static_cast<int>(blk);
-    const unsigned m = __ballot_sync(kFull, hit);
-    if (m) {
-      const int w = i0 + __ffs(m) - 1;
-      src = a.copies[3 * w];
-      rows = a.copies[3 * w + 2];
-      break;
-    }
+  if (first != 0x7fffffff) {
+    src = a.copies[3 * first];
+    rows = a.copies[3 * first + 2];
   }
   if (src >= 0 && (src >= a.num_blocks || rows < 0 || rows > kBlockSize)) {
     if (lane == 0) raise_error(PKV_ERR_COPY_RANGE);
@@ -531,10 +530,8 @@ __global__ void __launch_bounds__(NWARPS * 32)
     // token and its copy-on-write copy first, and fences them before that
     // page's TMA load
     int last_i = -1;
-    if (!prefix_role && a.slots != nullptr && pidx == nparts - 1 && warp == (nblk - 1) % NWARPS) {
+    if (!prefix_role && a.slots != nullptr && pidx == nparts - 1 && warp == (nblk - 1) % NWARPS)
       last_i = (nblk - 1) / NWARPS;
-      fused_step_append<T, D>(a, b, kvh, lane);
-    }
 
     // lane j: physical blocks of this warp's pages j, j + 32, ... (page
     // warp + j*NWARPS of the partition, and so on)
@@ -564,7 +561,7 @@ __global__ void __launch_bounds__(NWARPS * 32)
 
     auto issue = [&](int i) {
       const int phys = phys_of(i);
-      if (i == last_i) {  // the step's writes into this page, visible to the TMA read
+      if (i == last_i) {  // the step's writes into this page (made below), visible to the TMA read
         asm volatile("fence.proxy.async.global;" ::: "memory");
         __syncwarp();
       }
@@ -585,8 +582,18 @@ __global__ void __launch_bounds__(NWARPS * 32)
         }
       }
     };
+    if (last_i >= 0) {
+      // the warp's first pages go out before the step's writes, so that
+      // the writes' latency overlaps them; the last page waits for them
 #pragma unroll
-    for (int i = 0; i < NSTAGE; ++i) issue(i);
+      for (int i = 0; i < NSTAGE; ++i)
+        if (i != last_i) issue(i);
+      fused_step_append<T, D>(a, b, kvh, lane);
+      if (last_i < NSTAGE) issue(last_i);
+    } else {
+#pragma unroll
+      for (int i = 0; i < NSTAGE; ++i) issue(i);
+    }
 
     // O^T accumulator fragments: o[i] = rows d = 16 i + g8 (+8), columns 2 t4 (+1)
     float o[S::kKSteps][4];

@@ -13,8 +13,11 @@
 // One CTA per (kv-head, sequence, tile of 128 rows, key partition); a row
 // is a (token, head) pair of the kv-head, as in the other multi-token
 // kernels.  Six warps with fixed jobs:
-//   warp 0      TMA producer: the partition's pages, four per key block (64
-//               keys), into a ring of NS stages (K panels, then V panels);
+//   warp 0      TMA producers (lane 0 for K, lane 1 for V): the partition's
+//               pages, four per key block (64 keys), into a K ring and a V
+//               ring; a K stage is free again once its block's scores are
+//               formed, a V stage once its P.V is done, so the K loads run
+//               ahead of the S-buffer turnaround;
 //   warp 1      owns the tensor memory and issues the MMAs from one thread:
 //                 S_j  = Q . K_j^T      (M 128, N 64, A and B from shared
 //                                        memory, K-major, 128-byte swizzle)
@@ -152,10 +155,25 @@ __host__ __device__ constexpr uint32_t tc_idesc(int M, int N, bool b_mn_major) {
          (static_cast<uint32_t>(M >> 4) << 24);
 }
 
+// Timeline probe (debug builds with PKV_TC_TRACE only): SM clock at fixed
+// points of the pipeline for the first 64 CTAs and their first 32 blocks.
+#ifdef PKV_TC_TRACE
+__device__ long long g_tc_trace[64][32][10];
+#define TC_TRACE(j, slot)                                                                   \
+  do {                                                                                      \
+    const int cta_ = blockIdx.x + gridDim.x * (blockIdx.y + gridDim.y * blockIdx.z);       \
+    if (cta_ < 64 && (j) < 32) g_tc_trace[cta_][(j)][(slot)] = clock64();                  \
+  } while (0)
+#else
+#define TC_TRACE(j, slot) \
+  do {                    \
+  } while (0)
+#endif
+
 // ----------------------------------------------------------------------------
 // the kernel
 // ----------------------------------------------------------------------------
-template <int D, int NS>
+template <int D, int NSK, int NSV>
 struct TcShape {
   static constexpr int kRows = 128;                 // query rows of a tile (the MMA's M, one per TMEM lane)
   static constexpr int kPages = 4;                  // pages per key block
@@ -163,12 +181,13 @@ struct TcShape {
   static constexpr int kPanels = D / 64;            // 128-byte column panels of a row
   static constexpr int kQPanel = kRows * 128;       // bytes of one Q panel
   static constexpr int kKVPanel = kKeys * 128;      // bytes of one K (or V) panel of a block
-  static constexpr int kKV = kPanels * kKVPanel;    // K (or V) of one block
-  static constexpr int kStage = 2 * kKV;            // K panels, then V panels
-  static constexpr size_t kOffStages = size_t(kPanels) * kQPanel;
-  static constexpr size_t kOffBars = kOffStages + size_t(NS) * kStage;
-  // barriers: full[NS], empty[NS], sfull[2], pfull[2], pvdone, final
-  static constexpr int kBars = 2 * NS + 6;
+  static constexpr int kKV = kPanels * kKVPanel;    // K (or V) of one block: one stage of a ring
+  static constexpr size_t kOffK = size_t(kPanels) * kQPanel;         // K ring: NSK stages
+  static constexpr size_t kOffV = kOffK + size_t(NSK) * kKV;        // V ring: NSV stages
+  static constexpr size_t kOffBars = kOffV + size_t(NSV) * kKV;
+  // barriers: kfull[NSK], kempty[NSK], vfull[NSV], vempty[NSV], sfull[2],
+  // pfull[2], pvdone, final
+  static constexpr int kBars = 2 * NSK + 2 * NSV + 6;
   static constexpr size_t kOffTab = kOffBars + size_t(kBars) * 8;
   static constexpr int kMaxPages = 128;  // pages of the longest partition (2048 tokens)
   static constexpr size_t kOffSlot = kOffTab + size_t(kMaxPages) * 4;
@@ -178,22 +197,26 @@ struct TcShape {
   static constexpr uint32_t kColS = 128;  // S/P buffer b at kColS + 64 b
   static constexpr int kThreads = 192;
   static_assert(D == 64 || D == 128, "head_dim 64 or 128");
-  static_assert(kStage % 1024 == 0 && kQPanel % 1024 == 0, "swizzled panels need 1024-byte alignment");
+  static_assert(kKV % 1024 == 0 && kQPanel % 1024 == 0, "swizzled panels need 1024-byte alignment");
 };
 
-#ifndef PKV_TC_STAGES
-#define PKV_TC_STAGES 2
+#ifndef PKV_TC_K_STAGES
+#define PKV_TC_K_STAGES 2
+#endif
+#ifndef PKV_TC_V_STAGES
+#define PKV_TC_V_STAGES 2
 #endif
 #ifndef PKV_TC_MIN_CTAS
 #define PKV_TC_MIN_CTAS 2
 #endif
 
-template <typename T, int D, int G, int NS>
-__global__ void __launch_bounds__(TcShape<D, NS>::kThreads, PKV_TC_MIN_CTAS)
+template <typename T, int D, int G, int NSK, int NSV>
+__global__ void __launch_bounds__(TcShape<D, NSK, NSV>::kThreads, PKV_TC_MIN_CTAS)
     paged_multi_tc_kernel(const MultiArgs a, const __grid_constant__ CUtensorMap tmap_k,
                           const __grid_constant__ CUtensorMap tmap_v) {
   pdl_enter();
-  using S = TcShape<D, NS>;
+  if (threadIdx.x == 0) TC_TRACE(0, 9);
+  using S = TcShape<D, NSK, NSV>;
   using M = Mma<T>;
   const int kvh = blockIdx.x;
   const int b = blockIdx.y / a.tiles;
@@ -228,9 +251,12 @@ __global__ void __launch_bounds__(TcShape<D, NS>::kThreads, PKV_TC_MIN_CTAS)
   const uint32_t raw_addr = smem_addr(smem_raw);
   unsigned char* smem = smem_raw + (((raw_addr + 1023u) & ~1023u) - raw_addr);
   const uint32_t sq = smem_addr(smem);
-  const uint32_t sstage = sq + static_cast<uint32_t>(S::kOffStages);
+  const uint32_t sk = sq + static_cast<uint32_t>(S::kOffK);
+  const uint32_t sv = sq + static_cast<uint32_t>(S::kOffV);
   const uint32_t bars = sq + static_cast<uint32_t>(S::kOffBars);
-  const uint32_t bar_full = bars, bar_empty = bars + 8 * NS, bar_sfull = bars + 16 * NS;
+  const uint32_t bar_kfull = bars, bar_kempty = bar_kfull + 8 * NSK;
+  const uint32_t bar_vfull = bar_kempty + 8 * NSK, bar_vempty = bar_vfull + 8 * NSV;
+  const uint32_t bar_sfull = bar_vempty + 8 * NSV;
   const uint32_t bar_pfull = bar_sfull + 16, bar_pvdone = bar_pfull + 16, bar_final = bar_pvdone + 8;
   int* table = reinterpret_cast<int*>(smem + S::kOffTab);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + S::kOffSlot);
@@ -245,9 +271,13 @@ __global__ void __launch_bounds__(TcShape<D, NS>::kThreads, PKV_TC_MIN_CTAS)
     table[j] = in ? e : -1;
   }
   if (threadIdx.x == 0) {
-    for (int s = 0; s < NS; ++s) {
-      mbar_init(bar_full + 8 * s, 1);
-      mbar_init(bar_empty + 8 * s, 1);
+    for (int s = 0; s < NSK; ++s) {
+      mbar_init(bar_kfull + 8 * s, 1);
+      mbar_init(bar_kempty + 8 * s, 1);
+    }
+    for (int s = 0; s < NSV; ++s) {
+      mbar_init(bar_vfull + 8 * s, 1);
+      mbar_init(bar_vempty + 8 * s, 1);
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(bar_sfull + 8 * i, 1);
@@ -283,14 +313,22 @@ __global__ void __launch_bounds__(TcShape<D, NS>::kThreads, PKV_TC_MIN_CTAS)
   // loaded(i): page i of the partition is staged (in range, named by the table)
   auto loaded = [&](int i) { return i < nblk && table[i] >= 0; };
   bool bad = false;
-  int issued = 0;  // producer: key blocks whose copies were issued
+  int issued = 0;  // producer lane: key blocks whose copies it issued
 
   if (warp == 0) {
-    // ---- TMA producer ------------------------------------------------------
-    if (lane == 0) {
+    // ---- TMA producers: lane 0 fills the K ring, lane 1 the V ring -----------
+    // A K stage is released as soon as the block's S = Q.K^T MMAs are done,
+    // a V stage once its P.V MMAs are done, so K runs up to NSK blocks
+    // ahead of the scores and V up to NSV blocks ahead of the P.V products.
+    if (lane < 2) {
+      const bool is_v = lane == 1;
+      const int ns = is_v ? NSV : NSK;
+      const uint32_t full0 = is_v ? bar_vfull : bar_kfull, empty0 = is_v ? bar_vempty : bar_kempty;
+      const uint32_t ring = is_v ? sv : sk;
+      const CUtensorMap* map = is_v ? &tmap_v : &tmap_k;
       for (int c = 0; c < nb; ++c) {
-        const int s = c % NS;
-        if (c >= NS && !mbar_wait_bounded(bar_empty + 8 * s, ((c / NS) - 1) & 1)) {
+        const int s = c % ns;
+        if (c >= ns && !mbar_wait_bounded(empty0 + 8 * s, ((c / ns) - 1) & 1)) {
           raise_error(PKV_ERR_TIMEOUT);
           bad = true;
           break;
@@ -298,27 +336,25 @@ __global__ void __launch_bounds__(TcShape<D, NS>::kThreads, PKV_TC_MIN_CTAS)
         uint32_t bytes = 0;
 #pragma unroll
         for (int p = 0; p < S::kPages; ++p)
-          if (loaded(c * S::kPages + p)) bytes += 2 * S::kPanels * 2048;
-        const uint32_t bar = bar_full + 8 * s;
+          if (loaded(c * S::kPages + p)) bytes += S::kPanels * 2048;
+        const uint32_t bar = full0 + 8 * s;
         if (bytes == 0) {
           mbar_arrive(bar);
         } else {
           fence_proxy_async_smem();
           mbar_arrive_expect_tx(bar, bytes);
-          const uint32_t kst = sstage + s * S::kStage, vst = kst + S::kKV;
+          const uint32_t st = ring + s * S::kKV;
 #pragma unroll
           for (int p = 0; p < S::kPages; ++p) {
             const int i = c * S::kPages + p;
             if (!loaded(i)) continue;
             const int y = (table[i] * a.num_kv_heads + kvh) * kBlockSize;
 #pragma unroll
-            for (int bx = 0; bx < S::kPanels; ++bx) {
-              tma_load_2d(kst + bx * S::kKVPanel + p * 2048, &tmap_k, bx * 64, y, bar);
-              tma_load_2d(vst + bx * S::kKVPanel + p * 2048, &tmap_v, bx * 64, y, bar);
-            }
+            for (int bx = 0; bx < S::kPanels; ++bx) tma_load_2d(st + bx * S::kKVPanel + p * 2048, map, bx * 64, y, bar);
           }
         }
         issued = c + 1;
+        TC_TRACE(c, is_v ? 1 : 0);
       }
     }
   } else if (warp == 1) {
@@ -328,9 +364,33 @@ __global__ void __launch_bounds__(TcShape<D, NS>::kThreads, PKV_TC_MIN_CTAS)
     auto wait_all = [&](uint32_t bar, uint32_t parity) { return __all_sync(kFull, mbar_wait_bounded(bar, parity)); };
     auto pv = [&](int j) -> bool {
       if (!wait_all(bar_pfull + 8 * (j & 1), (j >> 1) & 1)) return false;
+      if (lane == 0) TC_TRACE(j, 4);
+      const int s = j % NSV;
+      if (!wait_all(bar_vfull + 8 * s, (j / NSV) & 1)) return false;
+      // zero the V rows of keys that are not there (past the context or on
+      // pages the table does not name): a zero weight must not meet a NaN
+      const uint32_t vst_off = static_cast<uint32_t>(S::kOffV) + s * S::kKV;
+      bool zeroed = false;
+#pragma unroll
+      for (int p = 0; p < S::kPages; ++p) {
+        const int i = j * S::kPages + p;
+        const int page_tok = tok0 + i * kBlockSize;
+        const int first = loaded(i) ? max(0, min(kBlockSize, tok1 - page_tok)) : 0;
+        if (first >= kBlockSize) continue;
+        zeroed = true;
+        const int n = (kBlockSize - first) * S::kPanels * 8;  // 16-byte chunks
+        for (int e = lane; e < n; e += 32) {
+          const int row = first + e / (S::kPanels * 8);
+          const int pn = (e / 8) % S::kPanels;
+          *reinterpret_cast<uint4*>(smem + vst_off + pn * S::kKVPanel + (p * kBlockSize + row) * 128 + (e & 7) * 16) =
+              make_uint4(0u, 0u, 0u, 0u);
+        }
+      }
+      if (zeroed) fence_proxy_async_smem();
+      __syncwarp();
       tc_fence_after();
       if (lane == 0) {
-        const uint32_t vst = sstage + (j % NS) * S::kStage + S::kKV;
+        const uint32_t vst = sv + s * S::kKV;
         const uint32_t pcol = tmem + S::kColS + 64 * (j & 1);
 #pragma unroll
         for (int kk = 0; kk < S::kKeys / 16; ++kk) {
@@ -338,41 +398,20 @@ __global__ void __launch_bounds__(TcShape<D, NS>::kThreads, PKV_TC_MIN_CTAS)
           tc_mma_ts(tmem + S::kColO, pcol + 8 * kk, vd, kIdPV, (j > 0 || kk > 0) ? 1u : 0u);  // P hi
           tc_mma_ts(tmem + S::kColO, pcol + 32 + 8 * kk, vd, kIdPV, 1u);                       // P lo
         }
-        tc_commit(bar_empty + 8 * (j % NS));  // the block's K and V may be overwritten
+        tc_commit(bar_vempty + 8 * s);  // the block's V may be overwritten
         tc_commit(bar_pvdone);
+        TC_TRACE(j, 5);
       }
       __syncwarp();
       return true;
     };
     for (int c = 0; c < nb && !bad; ++c) {
-      const int s = c % NS;
-      if (!wait_all(bar_full + 8 * s, (c / NS) & 1)) {
+      const int s = c % NSK;
+      if (!wait_all(bar_kfull + 8 * s, (c / NSK) & 1)) {
         bad = true;
         break;
       }
-      // zero the V rows of keys that are not there (past the context or
-      // on pages the table does not name)
-      {
-        const uint32_t vst_off = static_cast<uint32_t>(S::kOffStages) + s * S::kStage + S::kKV;
-        bool zeroed = false;
-#pragma unroll
-        for (int p = 0; p < S::kPages; ++p) {
-          const int i = c * S::kPages + p;
-          const int page_tok = tok0 + i * kBlockSize;
-          const int first = loaded(i) ? max(0, min(kBlockSize, tok1 - page_tok)) : 0;
-          if (first >= kBlockSize) continue;
-          zeroed = true;
-          const int n = (kBlockSize - first) * S::kPanels * 8;  // 16-byte chunks
-          for (int e = lane; e < n; e += 32) {
-            const int row = first + e / (S::kPanels * 8);
-            const int pn = (e / 8) % S::kPanels;
-            *reinterpret_cast<uint4*>(smem + vst_off + pn * S::kKVPanel + (p * kBlockSize + row) * 128 +
-                                      (e & 7) * 16) = make_uint4(0u, 0u, 0u, 0u);
-          }
-        }
-        if (zeroed) fence_proxy_async_smem();
-        __syncwarp();
-      }
+      if (lane == 0) TC_TRACE(c, 2);
       // S buffer c & 1 was last read (as P) by the P.V of block c - 2
       if (c >= 2 && !wait_all(bar_pvdone, (c - 2) & 1)) {
         bad = true;
@@ -380,14 +419,16 @@ __global__ void __launch_bounds__(TcShape<D, NS>::kThreads, PKV_TC_MIN_CTAS)
       }
       tc_fence_after();
       if (lane == 0) {
-        const uint32_t kst = sstage + s * S::kStage;
+        const uint32_t kst = sk + s * S::kKV;
 #pragma unroll
         for (int ks = 0; ks < D / 16; ++ks) {
           const uint64_t qd = sw128_desc(sq + (ks >> 2) * S::kQPanel + (ks & 3) * 32, 16, 1024);
           const uint64_t kd = sw128_desc(kst + (ks >> 2) * S::kKVPanel + (ks & 3) * 32, 16, 1024);
           tc_mma_ss(tmem + S::kColS + 64 * (c & 1), qd, kd, kIdQK, ks > 0 ? 1u : 0u);
         }
+        tc_commit(bar_kempty + 8 * s);  // the block's K may be overwritten
         tc_commit(bar_sfull + 8 * (c & 1));
+        TC_TRACE(c, 3);
       }
       __syncwarp();
       if (c >= 1 && !pv(c - 1)) {
@@ -409,13 +450,24 @@ __global__ void __launch_bounds__(TcShape<D, NS>::kThreads, PKV_TC_MIN_CTAS)
     const bool valid = tr < R;
     const int pos = valid ? base + tr / G : -1;
     float m_ref = -INFINITY, l = 0.f;
+    // a warp whose 32 rows are all padding (a tile of <= 96 rows) keeps
+    // step with the others but computes nothing: its rows of P and O are
+    // never read back
+    const bool warp_pad = r0 + 32 * (warp & 3) >= R;
     auto wait_all = [&](uint32_t bar, uint32_t parity) { return __all_sync(kFull, mbar_wait_bounded(bar, parity)); };
     for (int j = 0; j < nb; ++j) {
       if (!wait_all(bar_sfull + 8 * (j & 1), (j >> 1) & 1)) {
         bad = true;
         break;
       }
+      if (warp == 4 && lane == 0) TC_TRACE(j, 6);
       tc_fence_after();
+      if (warp_pad) {
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar_pfull + 8 * (j & 1));
+        continue;
+      }
       const uint32_t scol = tmem + lane_off + S::kColS + 64 * (j & 1);
       const int kb0 = tok0 + j * S::kKeys;
       uint32_t pages_ok = 0;
@@ -434,6 +486,7 @@ __global__ void __launch_bounds__(TcShape<D, NS>::kThreads, PKV_TC_MIN_CTAS)
           x[32 * h + e] = ok ? __uint_as_float(v[e]) * a.qk_scale : -INFINITY;
         }
       }
+      if (warp == 4 && lane == 0) TC_TRACE(j, 7);
       float bm = -INFINITY;
 #pragma unroll
       for (int k = 0; k < S::kKeys; ++k) bm = fmaxf(bm, x[k]);
@@ -481,6 +534,7 @@ __global__ void __launch_bounds__(TcShape<D, NS>::kThreads, PKV_TC_MIN_CTAS)
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
+      if (warp == 4 && lane == 0) TC_TRACE(j, 8);
       if (lane == 0) mbar_arrive(bar_pfull + 8 * (j & 1));
     }
     // epilogue: every MMA done (the issuer's final commit follows the last
@@ -489,7 +543,7 @@ __global__ void __launch_bounds__(TcShape<D, NS>::kThreads, PKV_TC_MIN_CTAS)
     if (!bad && !wait_all(bar_final, 0)) bad = true;
     if (bad) {
       if (lane == 0) raise_error(PKV_ERR_TIMEOUT);
-    } else {
+    } else if (!warp_pad) {
       tc_fence_after();
       const bool has = valid && pos >= tok0;
       const size_t row = valid ? out_row(tr) : 0;
@@ -526,9 +580,12 @@ __global__ void __launch_bounds__(TcShape<D, NS>::kThreads, PKV_TC_MIN_CTAS)
   tc_fence_before();
   const bool any_bad = __syncthreads_or(bad);
   tc_fence_after();
-  if (any_bad && warp == 0 && lane == 0) {
-    // the last block issued into each stage lands before the CTA exits
-    for (int c = max(0, issued - NS); c < issued; ++c) mbar_wait_bounded(bar_full + 8 * (c % NS), (c / NS) & 1);
+  if (any_bad && warp == 0 && lane < 2) {
+    // the last block each producer issued into each stage lands before the
+    // CTA exits
+    const int ns = lane ? NSV : NSK;
+    const uint32_t full0 = lane ? bar_vfull : bar_kfull;
+    for (int c = max(0, issued - ns); c < issued; ++c) mbar_wait_bounded(full0 + 8 * (c % ns), (c / ns) & 1);
   }
   if (warp == 1) tmem_dealloc(tmem, S::kTmemCols);
 }

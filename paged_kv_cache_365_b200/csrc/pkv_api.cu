@@ -167,19 +167,20 @@ pkv_status launch_multi_fa(const pkv::MultiArgs& a, const void* k_cache, const v
 #endif
 constexpr int kTcAboveRows = PKV_TC_ABOVE_ROWS;
 constexpr int kTcCode = 200;  // dispatch code of paged_multi_tc_kernel
-constexpr int kTcStages = PKV_TC_STAGES;
+constexpr int kTcKStages = PKV_TC_K_STAGES;
+constexpr int kTcVStages = PKV_TC_V_STAGES;
 
 template <typename T, int D, int G>
 pkv_status launch_multi_tc(const pkv::MultiArgs& a, const void* k_cache, const void* v_cache, int num_blocks,
                            cudaStream_t st) {
-  using S = pkv::TcShape<D, kTcStages>;
+  using S = pkv::TcShape<D, kTcKStages, kTcVStages>;
   static_assert(kMaxPartition / PKV_BLOCK_SIZE <= S::kMaxPages, "the page table of a partition fits shared memory");
   CUtensorMap mk, mv;
   const long long rows = static_cast<long long>(num_blocks) * a.num_kv_heads * PKV_BLOCK_SIZE;
   if (!encode_cache_map(&mk, k_cache, pkv::Mma<T>::kTmaType, D, rows) ||
       !encode_cache_map(&mv, v_cache, pkv::Mma<T>::kTmaType, D, rows))
     return PKV_ECUDA;
-  auto kfn = pkv::paged_multi_tc_kernel<T, D, G, kTcStages>;
+  auto kfn = pkv::paged_multi_tc_kernel<T, D, G, kTcKStages, kTcVStages>;
   if (cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(S::kSmem)) !=
       cudaSuccess)
     return PKV_ECUDA;
@@ -817,6 +818,13 @@ pkv_status pkv_paged_attention_decode_static_ws(void* out, const void* q, const 
                                     max_context_len, num_seqs, num_q_heads, num_kv_heads, head_dim, num_blocks,
                                     scale, partition_tokens, dtype, ws, PKV_STATIC_WORKSPACE_BYTES, stream);
 }
+
+#ifdef PKV_TC_TRACE
+// debug builds only: the tcgen05 kernel's timeline probe (64 x 32 x 10 clocks)
+int pkv_debug_tc_trace(long long* out) {
+  return cudaMemcpyFromSymbol(out, pkv::g_tc_trace, sizeof(pkv::g_tc_trace)) == cudaSuccess ? 0 : 1;
+}
+#endif
 
 pkv_status pkv_selftest_bounded_wait(long long limit_cycles, void* stream) {
   if (limit_cycles <= 0 || limit_cycles > (1ll << 32)) return PKV_EINVAL;
