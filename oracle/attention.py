@@ -75,7 +75,7 @@ def paged_decode(q, k_cache, v_cache, block_tables, context_lens, scale, dtype,
 
 
 def paged_multi(q, k_cache, v_cache, block_tables, context_lens, query_start, scale, dtype,
-                block_size=16, seqs=None):
+                block_size=16, seqs=None, kv_dtype=None, k_scale=1.0, v_scale=1.0):
     """float64 output [T, Hq, D] for T = query_start[-1] query tokens.
 
     Rows query_start[b] .. query_start[b+1]-1 of q [T, Hq, D] are sequence
@@ -83,7 +83,11 @@ def paged_multi(q, k_cache, v_cache, block_tables, context_lens, query_start, sc
     query_start[b] + i attends over the sequence's tokens 0 .. ctx - n_b + i.
     A row whose position would be negative (n_b > ctx) yields zeros.
     ``seqs`` restricts the work to those sequences (other rows stay NaN).
+    An FP8 cache as in ``paged_decode``: ``kv_dtype='e4m3'`` (q stays in
+    ``dtype``), a stored K value is its code's value times ``k_scale`` (V
+    alike).
     """
+    kvd = dtype if kv_dtype is None else kv_dtype
     T, Hq, D = q.shape
     Hkv = k_cache.shape[1]
     G = Hq // Hkv
@@ -96,8 +100,8 @@ def paged_multi(q, k_cache, v_cache, block_tables, context_lens, query_start, sc
         n_pages = -(-n // block_size)
         pages = np.asarray(block_tables[b][:n_pages], dtype=np.int64)
         for g in range(Hkv):
-            keys = widen(_gather(k_cache, pages, g, n, block_size), dtype)
-            values = widen(_gather(v_cache, pages, g, n, block_size), dtype)
+            keys = widen(_gather(k_cache, pages, g, n, block_size), kvd) * k_scale
+            values = widen(_gather(v_cache, pages, g, n, block_size), kvd) * v_scale
             for i in range(nq):
                 pos = n - nq + i
                 qi = widen(q[r0 + i], dtype)

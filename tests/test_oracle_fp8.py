@@ -105,3 +105,63 @@ def test_quantisation_error_within_half_an_fp8_step():
     assert np.all(np.abs(dq - x)[normal & inside] <= 2.0 ** -4 * np.abs(x)[normal & inside] * (1 + 1e-6))
     assert np.all(np.abs(dq - x)[~normal] <= 2.0 ** -10 * scale * (1 + 1e-6))
     assert np.all(np.abs(dq[~inside]) == 448 * scale)
+
+
+def _fp8_multi_case(rng, ctx, nq, Hkv, Hq, D, ks, vs):
+    """Sequences' K/V drawn in logical order, quantised into a permuted FP8
+    pool by append_fp8; their new tokens' queries in fp16."""
+    import oracle
+    pages = [-(-n // 16) for n in ctx]
+    nb = sum(pages) + 3
+    perm = rng.permutation(nb)
+    cache = oracle.RefCache(nb, Hkv, D, "e4m3")
+    tables = np.full((len(ctx), max(pages) + 1), nb + 5, dtype=np.int32)
+    codes, at = [], 0
+    for b, n in enumerate(ctx):
+        kx = rng.standard_normal((n, Hkv, D)).astype(np.float16)
+        vx = rng.standard_normal((n, Hkv, D)).astype(np.float16)
+        blocks = perm[at:at + pages[b]]
+        at += pages[b]
+        tables[b, :pages[b]] = blocks
+        slots = np.array([blocks[j // 16] * 16 + j % 16 for j in range(n)], dtype=np.int64)
+        cache.append_fp8(kx, vx, slots, "f16", ks, vs)
+        codes.append((fp8.quantize(kx.astype(np.float32), ks), fp8.quantize(vx.astype(np.float32), vs)))
+    qs = np.concatenate([[0], np.cumsum(nq)]).astype(np.int32)
+    q = rng.standard_normal((int(qs[-1]), Hq, D)).astype(np.float16)
+    return cache, tables, qs, q, codes
+
+
+def test_fp8_multi_matches_causal_brute_force():
+    """Several new tokens per sequence over an FP8 cache: the paged oracle
+    against pure Python causal attention over the codes in logical order
+    (no table, no slots), each code's value times its scale."""
+    import oracle
+    rng = np.random.default_rng(5)
+    Hkv, Hq, D, ks, vs = 2, 4, 16, 0.03, 0.07
+    ctx, nq = [37, 16, 9], [5, 16, 2]
+    cache, tables, qs, q, codes = _fp8_multi_case(rng, ctx, nq, Hkv, Hq, D, ks, vs)
+    out = oracle.paged_multi(q, cache.k, cache.v, tables, np.array(ctx), qs, 0.25, "f16", kv_dtype="e4m3",
+                             k_scale=ks, v_scale=vs)
+    G = Hq // Hkv
+    for b, n in enumerate(ctx):
+        kc, vc = codes[b]
+        for i in range(nq[b]):
+            pos = n - nq[b] + i
+            for h in range(Hq):
+                keys = [[fp8.e4m3_value(int(c)) * ks for c in kc[j, h // G]] for j in range(pos + 1)]
+                vals = [[fp8.e4m3_value(int(c)) * vs for c in vc[j, h // G]] for j in range(pos + 1)]
+                want = oracle.contiguous_decode([float(x) for x in q[qs[b] + i, h]], keys, vals, 0.25)
+                np.testing.assert_allclose(out[qs[b] + i, h], want, rtol=0, atol=1e-12)
+
+
+def test_fp8_multi_brute_force_catches_a_swapped_scale():
+    """A planted slip -- V's scale applied to K -- is caught."""
+    import oracle
+    rng = np.random.default_rng(6)
+    Hkv, Hq, D = 1, 2, 16
+    cache, tables, qs, q, _ = _fp8_multi_case(rng, [20], [4], Hkv, Hq, D, 0.03, 0.07)
+    good = oracle.paged_multi(q, cache.k, cache.v, tables, np.array([20]), qs, 0.25, "f16", kv_dtype="e4m3",
+                              k_scale=0.03, v_scale=0.07)
+    bad = oracle.paged_multi(q, cache.k, cache.v, tables, np.array([20]), qs, 0.25, "f16", kv_dtype="e4m3",
+                             k_scale=0.07, v_scale=0.07)
+    assert np.abs(good - bad).max() > 1e-4
