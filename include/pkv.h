@@ -468,10 +468,11 @@ pkv_status pkv_paged_attention_decode_prefix_fp8(void* out, const void* q, const
  * [num_seqs + 1] (device), non-decreasing, query_start[num_seqs] <=
  * total_query_tokens, every n_b <= max_query_len (a sequence that breaks
  * this is skipped, its rows left unwritten, and PKV_ERR_CONTEXT_RANGE set).
- * fp16 / bf16 only (tensor cores).  num_seqs * tiles <= 65535, tiles = 1
- * while max_query_len * G <= 32 rows per kv-head, else ceil(max_query_len *
- * G / 128) (tiles of 128 rows on the tcgen05 tensor cores).  workspace: pkv_multi_workspace_bytes(...) bytes (0 when
- * max_context_len <= partition), 16-byte aligned.  partition_tokens as in
+ * fp16 / bf16 only (tensor cores).  num_seqs * tiles <= 65535, with R =
+ * max_query_len * G rows per kv-head: tiles = 1 while R <= 32, else
+ * ceil(R / 128) (tiles of 128 rows on the tcgen05 tensor cores).
+ * workspace: pkv_multi_workspace_bytes(...) bytes (0 when max_context_len <=
+ * partition), 16-byte aligned.  partition_tokens as in
  * pkv_paged_attention_decode, except the auto partition (0): 2048 tokens,
  * or 1024 when max_context_len > 4096 (several rows a sequence make every
  * partial n_b times the merge work, so short contexts stay unsplit; long

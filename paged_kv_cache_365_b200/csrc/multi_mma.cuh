@@ -1062,41 +1062,59 @@ __global__ void __launch_bounds__(NWF * 32, PKV_FA_MIN_CTAS)
   }
 }
 
-// Merge of the key partitions of each query row (token t = blockIdx.x, HPC
-// heads per CTA from head blockIdx.y * HPC): the row at position pos uses
-// partitions 0 .. pos / partition.
-// Sequences held by one partition were written by the partition kernel.
-template <typename T, int D, int HPC>
+// Merge of the key partitions of the query rows of one (sequence b =
+// blockIdx.x, kv-head blockIdx.y): the row at position pos uses partitions
+// 0 .. pos / partition.  A sequence held by one partition was written by
+// the partition kernel, so its CTA stops after reading the sequence's
+// length.  Otherwise each warp merges whole rows (token, head) on its own:
+// the partitions' common max, then their rescaled sums in partition order.
+template <typename T, int D, int G>
 __global__ void __launch_bounds__(kMergeWarps * 32) paged_multi_merge_kernel(const MultiArgs a) {
   pdl_enter();
-  const int hs = (threadIdx.x >> 5) / (kMergeWarps / HPC);
-  const int h = blockIdx.y * HPC + hs;
-  const int t = blockIdx.x;
-  // the sequence of row t: last b with query_start[b] <= t
-  int lo = 0, hi = a.num_seqs - 1;
-  while (lo < hi) {
-    const int mid = (lo + hi + 1) >> 1;
-    if (a.query_start[mid] <= t)
-      lo = mid;
-    else
-      hi = mid - 1;
-  }
-  const int b = lo;
+  const int b = blockIdx.x, kvh = blockIdx.y;
   int ctx, q0, nq;
-  const bool ok = multi_seq(a, b, ctx, q0, nq, false) && t >= q0 && t < q0 + nq;
-  const bool direct = ctx <= a.partition;
-  const bool skip = !ok || direct;
-  if (__syncthreads_and(skip)) return;  // uniform: same row t for the whole CTA
-  const int pos = ctx - nq + (t - q0);
-  const bool head_ok = h < a.num_q_heads;
-  const int hh = head_ok ? h : 0;
-  const size_t row = static_cast<size_t>(t) * a.num_q_heads + hh;
-  __shared__ T sink[D];
-  T* out = head_ok ? reinterpret_cast<T*>(a.out) + row * D : sink;
-  const int n = (head_ok && pos >= 0) ? pos / a.partition + 1 : 0;  // n = 0 writes zeros
-  const size_t w0 = row * a.num_parts;
-  merge_partials<T, D, HPC>(
-      n, [&](int p) { return a.ws_ml[w0 + p]; }, [&](int p) { return a.ws_o + (w0 + p) * D; }, out, hs);
+  if (!multi_seq(a, b, ctx, q0, nq, false) || ctx <= a.partition) return;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  constexpr int kEpl = D / 32;
+  for (int r = warp; r < nq * G; r += kMergeWarps) {
+    const int i = r / G;
+    const size_t row = static_cast<size_t>(q0 + i) * a.num_q_heads + kvh * G + r % G;
+    const int pos = ctx - nq + i;
+    const int n = pos >= 0 ? pos / a.partition + 1 : 0;  // n = 0 writes zeros
+    const size_t w0 = row * a.num_parts;
+    float M = -INFINITY;
+    for (int p = lane; p < n; p += 32) M = fmaxf(M, a.ws_ml[w0 + p].x);
+    M = warp_max(M);
+    float acc[kEpl];
+#pragma unroll
+    for (int e = 0; e < kEpl; ++e) acc[e] = 0.f;
+    float den = 0.f;
+    for (int p = 0; p < n; ++p) {
+      const float2 v = a.ws_ml[w0 + p];
+      const float w = exp2f(v.x - M);
+      den = fmaf(w, v.y, den);
+      // this lane's kEpl (2 or 4) consecutive elements in one load
+      const float2* o = reinterpret_cast<const float2*>(a.ws_o + (w0 + p) * D + lane * kEpl);
+      float2 f[kEpl / 2];
+      if constexpr (kEpl == 4) {
+        const float4 g = *reinterpret_cast<const float4*>(o);
+        f[0] = make_float2(g.x, g.y);
+        f[1] = make_float2(g.z, g.w);
+      } else {
+#pragma unroll
+        for (int e = 0; e < kEpl / 2; ++e) f[e] = o[e];
+      }
+#pragma unroll
+      for (int e = 0; e < kEpl / 2; ++e) {
+        acc[2 * e] = fmaf(w, f[e].x, acc[2 * e]);
+        acc[2 * e + 1] = fmaf(w, f[e].y, acc[2 * e + 1]);
+      }
+    }
+    T* out = reinterpret_cast<T*>(a.out) + row * D + lane * kEpl;
+    const float inv = n > 0 ? 1.f / den : 0.f;
+#pragma unroll
+    for (int e = 0; e < kEpl; ++e) out[e] = Fmt<T>::from_f32(acc[e] * inv);
+  }
 }
 
 }  // namespace pkv

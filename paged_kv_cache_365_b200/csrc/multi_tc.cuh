@@ -110,6 +110,34 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
       : "memory");
 }
 
+// 64 consecutive 32-bit columns of this thread's lane in one load, waited
+// for inside the same statement.
+__device__ __forceinline__ void tmem_ld64(uint32_t taddr, uint32_t (&r)[64]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x64.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
+      "%15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32, %33, %34, %35, "
+      "%36, %37, %38, %39, %40, %41, %42, %43, %44, %45, %46, %47, %48, %49, %50, %51, %52, %53, %54, %55, %56, "
+      "%57, %58, %59, %60, %61, %62, %63}, [%64];\n\t"
+      "tcgen05.wait::ld.sync.aligned;"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]),
+        "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]),
+        "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
+        "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31]), "=r"(r[32]),
+        "=r"(r[33]), "=r"(r[34]), "=r"(r[35]), "=r"(r[36]), "=r"(r[37]), "=r"(r[38]), "=r"(r[39]), "=r"(r[40]),
+        "=r"(r[41]), "=r"(r[42]), "=r"(r[43]), "=r"(r[44]), "=r"(r[45]), "=r"(r[46]), "=r"(r[47]), "=r"(r[48]),
+        "=r"(r[49]), "=r"(r[50]), "=r"(r[51]), "=r"(r[52]), "=r"(r[53]), "=r"(r[54]), "=r"(r[55]), "=r"(r[56]),
+        "=r"(r[57]), "=r"(r[58]), "=r"(r[59]), "=r"(r[60]), "=r"(r[61]), "=r"(r[62]), "=r"(r[63])
+      : "r"(taddr)
+      : "memory");
+}
+
+// max of three (one instruction)
+__device__ __forceinline__ float fmax3(float x, float y, float z) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(x), "f"(y), "f"(z));
+  return d;
+}
+
 __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
   asm volatile(
       "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
@@ -158,15 +186,31 @@ __host__ __device__ constexpr uint32_t tc_idesc(int M, int N, bool b_mn_major) {
 // Timeline probe (debug builds with PKV_TC_TRACE only): SM clock at fixed
 // points of the pipeline for the first 64 CTAs and their first 32 blocks.
 #ifdef PKV_TC_TRACE
-__device__ long long g_tc_trace[64][32][10];
+__device__ long long g_tc_trace[64][32][12];
 #define TC_TRACE(j, slot)                                                                   \
   do {                                                                                      \
     const int cta_ = blockIdx.x + gridDim.x * (blockIdx.y + gridDim.y * blockIdx.z);       \
     if (cta_ < 64 && (j) < 32) g_tc_trace[cta_][(j)][(slot)] = clock64();                  \
   } while (0)
+// per CTA (first 16384): global timer at entry, at the first K copy and at
+// exit, and (SM id, key blocks)
+__device__ long long g_tc_cta[16384][4];
+__device__ __forceinline__ long long tc_gtime() {
+  long long t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+#define TC_CTA(slot, v)                                                                    \
+  do {                                                                                      \
+    const int cta_ = blockIdx.x + gridDim.x * (blockIdx.y + gridDim.y * blockIdx.z);       \
+    if (cta_ < 16384) g_tc_cta[cta_][(slot)] = (v);                                         \
+  } while (0)
 #else
 #define TC_TRACE(j, slot) \
   do {                    \
+  } while (0)
+#define TC_CTA(slot, v) \
+  do {                  \
   } while (0)
 #endif
 
@@ -186,8 +230,8 @@ struct TcShape {
   static constexpr size_t kOffV = kOffK + size_t(NSK) * kKV;        // V ring: NSV stages
   static constexpr size_t kOffBars = kOffV + size_t(NSV) * kKV;
   // barriers: kfull[NSK], kempty[NSK], vfull[NSV], vempty[NSV], sfull[2],
-  // pfull[2], pvdone, final
-  static constexpr int kBars = 2 * NSK + 2 * NSV + 6;
+  // pfull[2], pvdone, final, qfull
+  static constexpr int kBars = 2 * NSK + 2 * NSV + 7;
   static constexpr size_t kOffTab = kOffBars + size_t(kBars) * 8;
   static constexpr int kMaxPages = 128;  // pages of the longest partition (2048 tokens)
   static constexpr size_t kOffSlot = kOffTab + size_t(kMaxPages) * 4;
@@ -214,8 +258,15 @@ template <typename T, int D, int G, int NSK, int NSV>
 __global__ void __launch_bounds__(TcShape<D, NSK, NSV>::kThreads, PKV_TC_MIN_CTAS)
     paged_multi_tc_kernel(const MultiArgs a, const __grid_constant__ CUtensorMap tmap_k,
                           const __grid_constant__ CUtensorMap tmap_v) {
+  if (threadIdx.x == 0) {
+    // the descriptors are kernel parameters: fetch them while the previous
+    // kernel drains
+    asm volatile("prefetch.tensormap [%0];" ::"l"(&tmap_k) : "memory");
+    asm volatile("prefetch.tensormap [%0];" ::"l"(&tmap_v) : "memory");
+  }
   pdl_enter();
   if (threadIdx.x == 0) TC_TRACE(0, 9);
+  if (threadIdx.x == 0) TC_CTA(0, tc_gtime());
   using S = TcShape<D, NSK, NSV>;
   using M = Mma<T>;
   const int kvh = blockIdx.x;
@@ -258,6 +309,7 @@ __global__ void __launch_bounds__(TcShape<D, NSK, NSV>::kThreads, PKV_TC_MIN_CTA
   const uint32_t bar_vfull = bar_kempty + 8 * NSK, bar_vempty = bar_vfull + 8 * NSV;
   const uint32_t bar_sfull = bar_vempty + 8 * NSV;
   const uint32_t bar_pfull = bar_sfull + 16, bar_pvdone = bar_pfull + 16, bar_final = bar_pvdone + 8;
+  const uint32_t bar_qfull = bar_final + 8;
   int* table = reinterpret_cast<int*>(smem + S::kOffTab);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + S::kOffSlot);
 
@@ -285,25 +337,12 @@ __global__ void __launch_bounds__(TcShape<D, NSK, NSV>::kThreads, PKV_TC_MIN_CTA
     }
     mbar_init(bar_pvdone, 1);
     mbar_init(bar_final, 1);
+    mbar_init(bar_qfull, 4);  // one arrival per softmax warp
     fence_barrier_init();
   }
   if (warp == 1) {
     tmem_alloc(smem_addr(tmem_slot), S::kTmemCols);
     tmem_relinquish();
-  }
-  if (warp >= 2) {
-    // this thread's row of Q into the 128-byte-swizzled K-major tile
-    // (rows past the batch are zeros)
-    const int r = 32 * (warp & 3) + lane;
-    const int tr = r0 + r;
-    const uint4* src = tr < R ? reinterpret_cast<const uint4*>(reinterpret_cast<const T*>(a.q) + out_row(tr) * D)
-                              : nullptr;
-#pragma unroll
-    for (int c = 0; c < D / 8; ++c) {
-      const uint4 v = src ? src[c] : make_uint4(0u, 0u, 0u, 0u);
-      *reinterpret_cast<uint4*>(smem + (c >> 3) * S::kQPanel + r * 128 + (((c & 7) ^ (r & 7)) << 4)) = v;
-    }
-    fence_proxy_async_smem();  // the tensor core reads the tile through the async proxy
   }
   tc_fence_before();
   __syncthreads();
@@ -313,48 +352,66 @@ __global__ void __launch_bounds__(TcShape<D, NSK, NSV>::kThreads, PKV_TC_MIN_CTA
   // loaded(i): page i of the partition is staged (in range, named by the table)
   auto loaded = [&](int i) { return i < nblk && table[i] >= 0; };
   bool bad = false;
-  int issued = 0;  // producer lane: key blocks whose copies it issued
+  int issued = 0, issued_v = 0;  // producer: key blocks whose K (V) copies it issued
 
   if (warp == 0) {
-    // ---- TMA producers: lane 0 fills the K ring, lane 1 the V ring -----------
+    // ---- TMA producer (lane 0): the K ring and the V ring ------------------
     // A K stage is released as soon as the block's S = Q.K^T MMAs are done,
     // a V stage once its P.V MMAs are done, so K runs up to NSK blocks
     // ahead of the scores and V up to NSV blocks ahead of the P.V products.
-    if (lane < 2) {
-      const bool is_v = lane == 1;
-      const int ns = is_v ? NSV : NSK;
-      const uint32_t full0 = is_v ? bar_vfull : bar_kfull, empty0 = is_v ? bar_vempty : bar_kempty;
-      const uint32_t ring = is_v ? sv : sk;
-      const CUtensorMap* map = is_v ? &tmap_v : &tmap_k;
-      for (int c = 0; c < nb; ++c) {
-        const int s = c % ns;
-        if (c >= ns && !mbar_wait_bounded(empty0 + 8 * s, ((c / ns) - 1) & 1)) {
-          raise_error(PKV_ERR_TIMEOUT);
-          bad = true;
-          break;
-        }
+    // One thread polls both rings, so a V stage that frees late never holds
+    // back the next K copy.
+    if (lane == 0) {
+      auto issue = [&](bool is_v, int c) {
+        const int s = c % (is_v ? NSV : NSK);
         uint32_t bytes = 0;
 #pragma unroll
         for (int p = 0; p < S::kPages; ++p)
           if (loaded(c * S::kPages + p)) bytes += S::kPanels * 2048;
-        const uint32_t bar = full0 + 8 * s;
+        const uint32_t bar = (is_v ? bar_vfull : bar_kfull) + 8 * s;
         if (bytes == 0) {
           mbar_arrive(bar);
-        } else {
-          fence_proxy_async_smem();
-          mbar_arrive_expect_tx(bar, bytes);
-          const uint32_t st = ring + s * S::kKV;
-#pragma unroll
-          for (int p = 0; p < S::kPages; ++p) {
-            const int i = c * S::kPages + p;
-            if (!loaded(i)) continue;
-            const int y = (table[i] * a.num_kv_heads + kvh) * kBlockSize;
-#pragma unroll
-            for (int bx = 0; bx < S::kPanels; ++bx) tma_load_2d(st + bx * S::kKVPanel + p * 2048, map, bx * 64, y, bar);
-          }
+          return;
         }
-        issued = c + 1;
-        TC_TRACE(c, is_v ? 1 : 0);
+        mbar_arrive_expect_tx(bar, bytes);
+        const uint32_t st = (is_v ? sv : sk) + s * S::kKV;
+        const CUtensorMap* map = is_v ? &tmap_v : &tmap_k;
+#pragma unroll
+        for (int p = 0; p < S::kPages; ++p) {
+          const int i = c * S::kPages + p;
+          if (!loaded(i)) continue;
+          const int y = (table[i] * a.num_kv_heads + kvh) * kBlockSize;
+#pragma unroll
+          for (int bx = 0; bx < S::kPanels; ++bx) tma_load_2d(st + bx * S::kKVPanel + p * 2048, map, bx * 64, y, bar);
+        }
+      };
+      long long t0 = clock64();
+      while (issued < nb || issued_v < nb) {
+        bool moved = false;
+        if (issued < nb &&
+            (issued < NSK || mbar_test(bar_kempty + 8 * (issued % NSK), ((issued / NSK) - 1) & 1))) {
+          issue(false, issued);
+          TC_TRACE(issued, 0);
+          if (issued == 0) TC_CTA(1, tc_gtime());
+          ++issued;
+          moved = true;
+        }
+        if (issued_v < nb &&
+            (issued_v < NSV || mbar_test(bar_vempty + 8 * (issued_v % NSV), ((issued_v / NSV) - 1) & 1))) {
+          issue(true, issued_v);
+          TC_TRACE(issued_v, 1);
+          ++issued_v;
+          moved = true;
+        }
+        if (moved) {
+          t0 = clock64();
+        } else if (clock64() - t0 > (1ll << 32)) {
+          raise_error(PKV_ERR_TIMEOUT);
+          bad = true;
+          break;
+        } else {
+          __nanosleep(32);
+        }
       }
     }
   } else if (warp == 1) {
@@ -396,7 +453,9 @@ __global__ void __launch_bounds__(TcShape<D, NSK, NSV>::kThreads, PKV_TC_MIN_CTA
         for (int kk = 0; kk < S::kKeys / 16; ++kk) {
           const uint64_t vd = sw128_desc(vst + kk * 2048, S::kKVPanel, 1024);
           tc_mma_ts(tmem + S::kColO, pcol + 8 * kk, vd, kIdPV, (j > 0 || kk > 0) ? 1u : 0u);  // P hi
+#ifndef PKV_TC_NO_LO
           tc_mma_ts(tmem + S::kColO, pcol + 32 + 8 * kk, vd, kIdPV, 1u);                       // P lo
+#endif
         }
         tc_commit(bar_vempty + 8 * s);  // the block's V may be overwritten
         tc_commit(bar_pvdone);
@@ -405,6 +464,7 @@ __global__ void __launch_bounds__(TcShape<D, NSK, NSV>::kThreads, PKV_TC_MIN_CTA
       __syncwarp();
       return true;
     };
+    if (!wait_all(bar_qfull, 0)) bad = true;
     for (int c = 0; c < nb && !bad; ++c) {
       const int s = c % NSK;
       if (!wait_all(bar_kfull + 8 * s, (c / NSK) & 1)) {
@@ -443,6 +503,22 @@ __global__ void __launch_bounds__(TcShape<D, NSK, NSV>::kThreads, PKV_TC_MIN_CTA
     __syncwarp();
     mbar_wait_bounded(bar_final, 0);
   } else {
+    {
+      // this thread's row of Q into the 128-byte-swizzled K-major tile
+      // (rows past the batch are zeros), while the first copies fly
+      const int r = 32 * (warp & 3) + lane;
+      const int tr = r0 + r;
+      const uint4* src = tr < R ? reinterpret_cast<const uint4*>(reinterpret_cast<const T*>(a.q) + out_row(tr) * D)
+                                : nullptr;
+#pragma unroll
+      for (int c = 0; c < D / 8; ++c) {
+        const uint4 v = src ? src[c] : make_uint4(0u, 0u, 0u, 0u);
+        *reinterpret_cast<uint4*>(smem + (c >> 3) * S::kQPanel + r * 128 + (((c & 7) ^ (r & 7)) << 4)) = v;
+      }
+      fence_proxy_async_smem();  // the tensor core reads the tile through the async proxy
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar_qfull);
+    }
     // ---- softmax (one thread per row) and epilogue ----------------------------
     const int r = 32 * (warp & 3) + lane;
     const uint32_t lane_off = static_cast<uint32_t>(32 * (warp & 3)) << 16;
@@ -456,6 +532,16 @@ __global__ void __launch_bounds__(TcShape<D, NSK, NSV>::kThreads, PKV_TC_MIN_CTA
     const bool warp_pad = r0 + 32 * (warp & 3) >= R;
     auto wait_all = [&](uint32_t bar, uint32_t parity) { return __all_sync(kFull, mbar_wait_bounded(bar, parity)); };
     for (int j = 0; j < nb; ++j) {
+      // the block's key limits need no scores: keys kb0 + e with e <= lim
+      // are causal for this row and inside the partition and the context
+      const int kb0 = tok0 + j * S::kKeys;
+      uint32_t pages_ok = 0;
+#pragma unroll
+      for (int p = 0; p < S::kPages; ++p) pages_ok |= loaded(j * S::kPages + p) ? (1u << p) : 0u;
+      const int lim = min(pos, tok1 - 1) - kb0;
+      // plain block: every key in, and a positive scale, so the max can be
+      // taken on the raw scores and the scale folded into the exponent
+      const bool plain = __all_sync(kFull, lim >= S::kKeys - 1 && pages_ok == 0xFu && a.qk_scale > 0.f);
       if (!wait_all(bar_sfull + 8 * (j & 1), (j >> 1) & 1)) {
         bad = true;
         break;
@@ -469,27 +555,34 @@ __global__ void __launch_bounds__(TcShape<D, NSK, NSV>::kThreads, PKV_TC_MIN_CTA
         continue;
       }
       const uint32_t scol = tmem + lane_off + S::kColS + 64 * (j & 1);
-      const int kb0 = tok0 + j * S::kKeys;
-      uint32_t pages_ok = 0;
-#pragma unroll
-      for (int p = 0; p < S::kPages; ++p) pages_ok |= loaded(j * S::kPages + p) ? (1u << p) : 0u;
-      const bool all_in = pos >= kb0 + S::kKeys - 1 && kb0 + S::kKeys <= tok1 && pages_ok == 0xFu;
+      uint32_t v[S::kKeys];
+      if (warp == 4 && lane == 0) TC_TRACE(j, 10);
+      tmem_ld64(scol, v);
+      if (warp == 4 && lane == 0) TC_TRACE(j, 11);
       float x[S::kKeys];
+      float mul = a.qk_scale;  // x * mul is the score in log2 units
+      if (plain) {
 #pragma unroll
-      for (int h = 0; h < S::kKeys / 32; ++h) {
-        uint32_t v[32];
-        tmem_ld32(scol + 32 * h, v);
+        for (int k = 0; k < S::kKeys; ++k) x[k] = __uint_as_float(v[k]);
+      } else {
+        // masked keys to -inf, the scale applied here
 #pragma unroll
-        for (int e = 0; e < 32; ++e) {
-          const int k = kb0 + 32 * h + e;
-          const bool ok = all_in || (k <= pos && k < tok1 && ((pages_ok >> ((32 * h + e) >> 4)) & 1u));
-          x[32 * h + e] = ok ? __uint_as_float(v[e]) * a.qk_scale : -INFINITY;
+        for (int k = 0; k < S::kKeys; ++k) {
+          const bool ok = k <= lim && ((pages_ok >> (k >> 4)) & 1u);
+          x[k] = ok ? __uint_as_float(v[k]) * a.qk_scale : -INFINITY;
         }
+        mul = 1.f;
       }
       if (warp == 4 && lane == 0) TC_TRACE(j, 7);
-      float bm = -INFINITY;
+      // block max: a tree of three-input maxima
+      float t[S::kKeys / 4];
 #pragma unroll
-      for (int k = 0; k < S::kKeys; ++k) bm = fmaxf(bm, x[k]);
+      for (int k = 0; k < S::kKeys / 4; ++k) t[k] = fmax3(x[4 * k], x[4 * k + 1], fmaxf(x[4 * k + 2], x[4 * k + 3]));
+#pragma unroll
+      for (int w = S::kKeys / 4; w > 1; w /= 2)
+#pragma unroll
+        for (int k = 0; k < w / 2; ++k) t[k] = fmaxf(t[k], t[k + w / 2]);
+      const float bm = t[0] * mul;
       // move the reference max only when this block exceeds it by 2^8
       float alpha = 1.f;
       bool rescale = false;
@@ -499,17 +592,20 @@ __global__ void __launch_bounds__(TcShape<D, NSK, NSV>::kThreads, PKV_TC_MIN_CTA
         l *= alpha;
         m_ref = bm;
       }
-      const float mr = m_ref == -INFINITY ? 0.f : m_ref;
+      const float nmr = m_ref == -INFINITY ? 0.f : -m_ref;
       uint32_t ph[S::kKeys / 2], pl[S::kKeys / 2];
-      float sum = 0.f;
+      float acc[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) acc[i] = 0.f;
 #pragma unroll
       for (int k = 0; k < S::kKeys; k += 2) {
-        const float p0 = exp2_sfu(x[k] - mr), p1 = exp2_sfu(x[k + 1] - mr);
-        sum += p0 + p1;
+        const float p0 = exp2_sfu(fmaf(x[k], mul, nmr)), p1 = exp2_sfu(fmaf(x[k + 1], mul, nmr));
+        acc[(k / 2) & 7] += p0 + p1;
         ph[k / 2] = M::pack(p0, p1);
         const float2 hv = M::unpack(ph[k / 2]);
         pl[k / 2] = M::pack(p0 - hv.x, p1 - hv.y);
       }
+      const float sum = ((acc[0] + acc[1]) + (acc[2] + acc[3])) + ((acc[4] + acc[5]) + (acc[6] + acc[7]));
       l += sum;
       if (__any_sync(kFull, rescale)) {
         // O holds the P.V of blocks < j: wait for the last of them, then
@@ -580,14 +676,20 @@ __global__ void __launch_bounds__(TcShape<D, NSK, NSV>::kThreads, PKV_TC_MIN_CTA
   tc_fence_before();
   const bool any_bad = __syncthreads_or(bad);
   tc_fence_after();
-  if (any_bad && warp == 0 && lane < 2) {
-    // the last block each producer issued into each stage lands before the
+  if (any_bad && warp == 0 && lane == 0) {
+    // the last block the producer issued into each stage lands before the
     // CTA exits
-    const int ns = lane ? NSV : NSK;
-    const uint32_t full0 = lane ? bar_vfull : bar_kfull;
-    for (int c = max(0, issued - ns); c < issued; ++c) mbar_wait_bounded(full0 + 8 * (c % ns), (c / ns) & 1);
+    for (int c = max(0, issued - NSK); c < issued; ++c) mbar_wait_bounded(bar_kfull + 8 * (c % NSK), (c / NSK) & 1);
+    for (int c = max(0, issued_v - NSV); c < issued_v; ++c)
+      mbar_wait_bounded(bar_vfull + 8 * (c % NSV), (c / NSV) & 1);
   }
   if (warp == 1) tmem_dealloc(tmem, S::kTmemCols);
+  if (threadIdx.x == 0) {
+    TC_CTA(2, tc_gtime());
+    unsigned smid_;
+    asm volatile("mov.u32 %0, %%smid;" : "=r"(smid_));
+    TC_CTA(3, static_cast<long long>(smid_) | (static_cast<long long>(nb) << 16));
+  }
 }
 
 }  // namespace pkv

@@ -38,10 +38,12 @@ __global__ void bounded_wait_selftest_kernel(long long limit) {
 namespace {
 
 // ---- several query tokens per sequence (tensor cores) -----------------------
-template <typename T, int D, int HPC>
-struct MultiMergeK {
-  static constexpr auto fn = pkv::paged_multi_merge_kernel<T, D, HPC>;
-};
+// The multi-token merge: one CTA per (sequence, kv-head).
+template <typename T, int D, int G>
+pkv_status launch_multi_merge(const pkv::MultiArgs& a, cudaStream_t st) {
+  return launch(pkv::paged_multi_merge_kernel<T, D, G>, dim3(a.num_seqs, a.num_kv_heads), dim3(pkv::kMergeWarps * 32),
+                0, st, a);
+}
 
 template <typename T, int D, int G, int NT>
 pkv_status launch_multi(const pkv::MultiArgs& a, const void* k_cache, const void* v_cache, int num_blocks,
@@ -59,15 +61,7 @@ pkv_status launch_multi(const pkv::MultiArgs& a, const void* k_cache, const void
     return PKV_ECUDA;
   const dim3 grid(a.num_kv_heads, a.num_seqs * a.tiles, a.num_parts);
   if (launch(kfn, grid, dim3(kMmaWarps * 32), S::kSmem, st, a, mk, mv) != PKV_OK) return PKV_ECUDA;
-  if (a.num_parts > 1) {
-    const dim3 block(pkv::kMergeWarps * 32);
-    // one CTA per query token; heads per CTA from the partitions a row may span
-    if (a.num_parts >= 32)
-      return launch(MultiMergeK<T, D, 1>::fn, dim3(a.total_q, a.num_q_heads), block, 0, st, a);
-    if (a.num_parts >= 16)  // (a row's own partitions are usually far fewer than the batch's most)
-      return launch(MultiMergeK<T, D, 4>::fn, dim3(a.total_q, (a.num_q_heads + 3) / 4), block, 0, st, a);
-    return launch(MultiMergeK<T, D, 8>::fn, dim3(a.total_q, (a.num_q_heads + 7) / 8), block, 0, st, a);
-  }
+  if (a.num_parts > 1) return launch_multi_merge<T, D, G>(a, st);
   return PKV_OK;
 }
 
@@ -122,14 +116,7 @@ pkv_status launch_multi_rows(const pkv::MultiArgs& a, const void* k_cache, const
     return PKV_ECUDA;
   const dim3 grid(a.num_kv_heads, a.num_seqs * a.tiles, a.num_parts);
   if (launch(kfn, grid, dim3(NW * 32), S::kSmem, st, a, mk, mv) != PKV_OK) return PKV_ECUDA;
-  if (a.num_parts > 1) {
-    const dim3 block(pkv::kMergeWarps * 32);
-    if (a.num_parts >= 32)
-      return launch(MultiMergeK<T, D, 1>::fn, dim3(a.total_q, a.num_q_heads), block, 0, st, a);
-    if (a.num_parts >= 16)  // (a row's own partitions are usually far fewer than the batch's most)
-      return launch(MultiMergeK<T, D, 4>::fn, dim3(a.total_q, (a.num_q_heads + 3) / 4), block, 0, st, a);
-    return launch(MultiMergeK<T, D, 8>::fn, dim3(a.total_q, (a.num_q_heads + 7) / 8), block, 0, st, a);
-  }
+  if (a.num_parts > 1) return launch_multi_merge<T, D, G>(a, st);
   return PKV_OK;
 }
 
@@ -149,14 +136,7 @@ pkv_status launch_multi_fa(const pkv::MultiArgs& a, const void* k_cache, const v
     return PKV_ECUDA;
   const dim3 grid(a.num_kv_heads, a.num_seqs * a.tiles, a.num_parts);
   if (launch(kfn, grid, dim3(kFaWarps * 32), S::kSmem, st, a, mk, mv) != PKV_OK) return PKV_ECUDA;
-  if (a.num_parts > 1) {
-    const dim3 block(pkv::kMergeWarps * 32);
-    if (a.num_parts >= 32)
-      return launch(MultiMergeK<T, D, 1>::fn, dim3(a.total_q, a.num_q_heads), block, 0, st, a);
-    if (a.num_parts >= 16)
-      return launch(MultiMergeK<T, D, 4>::fn, dim3(a.total_q, (a.num_q_heads + 3) / 4), block, 0, st, a);
-    return launch(MultiMergeK<T, D, 8>::fn, dim3(a.total_q, (a.num_q_heads + 7) / 8), block, 0, st, a);
-  }
+  if (a.num_parts > 1) return launch_multi_merge<T, D, G>(a, st);
   return PKV_OK;
 }
 
@@ -186,14 +166,7 @@ pkv_status launch_multi_tc(const pkv::MultiArgs& a, const void* k_cache, const v
     return PKV_ECUDA;
   const dim3 grid(a.num_kv_heads, a.num_seqs * a.tiles, a.num_parts);
   if (launch(kfn, grid, dim3(S::kThreads), S::kSmem, st, a, mk, mv) != PKV_OK) return PKV_ECUDA;
-  if (a.num_parts > 1) {
-    const dim3 block(pkv::kMergeWarps * 32);
-    if (a.num_parts >= 32)
-      return launch(MultiMergeK<T, D, 1>::fn, dim3(a.total_q, a.num_q_heads), block, 0, st, a);
-    if (a.num_parts >= 16)
-      return launch(MultiMergeK<T, D, 4>::fn, dim3(a.total_q, (a.num_q_heads + 3) / 4), block, 0, st, a);
-    return launch(MultiMergeK<T, D, 8>::fn, dim3(a.total_q, (a.num_q_heads + 7) / 8), block, 0, st, a);
-  }
+  if (a.num_parts > 1) return launch_multi_merge<T, D, G>(a, st);
   return PKV_OK;
 }
 
@@ -820,9 +793,17 @@ pkv_status pkv_paged_attention_decode_static_ws(void* out, const void* q, const 
 }
 
 #ifdef PKV_TC_TRACE
-// debug builds only: the tcgen05 kernel's timeline probe (64 x 32 x 10 clocks)
+// debug builds only: the tcgen05 kernel's timeline probe (64 x 32 x 12 clocks)
 int pkv_debug_tc_trace(long long* out) {
   return cudaMemcpyFromSymbol(out, pkv::g_tc_trace, sizeof(pkv::g_tc_trace)) == cudaSuccess ? 0 : 1;
+}
+// per-CTA entry / first copy / exit times and (SM, blocks): 16384 x 4
+int pkv_debug_tc_cta(long long* out) {
+  return cudaMemcpyFromSymbol(out, pkv::g_tc_cta, sizeof(pkv::g_tc_cta)) == cudaSuccess ? 0 : 1;
+}
+int pkv_debug_tc_cta_clear() {
+  static long long zero[16384][4];
+  return cudaMemcpyToSymbol(pkv::g_tc_cta, zero, sizeof(zero)) == cudaSuccess ? 0 : 1;
 }
 #endif
 
