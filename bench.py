@@ -304,19 +304,7 @@ def run_cuda(args, rank, world, local_rank, workload=None, graph=None):
     if fp8:
         if wl.dtype == "f32":
             raise SystemExit("--kv-fp8 needs an fp16 / bf16 workload")
-        # the same pool quantised once to E4M3 codes (one scale for K, one
-        # for V, covering ~6 standard deviations of the N(0,1) values)
-        NB, Hkv = cache.k.shape[0], cache.k.shape[1]
-        k8 = torch.empty(cache.k.shape, dtype=torch.uint8, device=dev)
-        v8 = torch.empty(cache.v.shape, dtype=torch.uint8, device=dev)
-        all_slots = torch.arange(NB * 16, dtype=torch.int64, device=dev)
-        for src, dst in ((cache.k, k8), (cache.v, v8)):
-            rows = src.permute(0, 2, 1, 3).reshape(NB * 16, Hkv, D).contiguous()
-            pkv.kv_append_fp8(rows, rows, dst, dst, all_slots, FP8_SCALE, FP8_SCALE)
-            del rows
-        cache.k, cache.v = k8, v8  # the 16-bit pool is released
-        cache.fp8 = (FP8_SCALE, FP8_SCALE)
-        torch.cuda.synchronize()
+        to_fp8_pool(cache, dev)
     prefix = torch.from_numpy(np.ascontiguousarray(st["host"]["block_tables"][0, :pp])).to(dev) if use_cascade else None
     # a plain 16-bit step is one launch (+ merge); the cascade keeps its copies
     # and append in their own launch (measured faster: their loads stay off
@@ -499,6 +487,25 @@ def run_cuda(args, rank, world, local_rank, workload=None, graph=None):
 # ---------------------------------------------------------------------------
 # several new tokens per sequence (speculative verification)
 # ---------------------------------------------------------------------------
+def to_fp8_pool(cache, dev):
+    """The cache's pool quantised once to E4M3 codes (one scale for K, one
+    for V, covering ~6 standard deviations of the N(0,1) values); the 16-bit
+    pool is released."""
+    import torch
+    import paged_kv_cache_365_b200 as pkv
+    NB, Hkv, D = cache.k.shape[0], cache.k.shape[1], cache.k.shape[3]
+    k8 = torch.empty(cache.k.shape, dtype=torch.uint8, device=dev)
+    v8 = torch.empty(cache.v.shape, dtype=torch.uint8, device=dev)
+    all_slots = torch.arange(NB * 16, dtype=torch.int64, device=dev)
+    for src, dst in ((cache.k, k8), (cache.v, v8)):
+        rows = src.permute(0, 2, 1, 3).reshape(NB * 16, Hkv, D).contiguous()
+        pkv.kv_append_fp8(rows, rows, dst, dst, all_slots, FP8_SCALE, FP8_SCALE)
+        del rows
+    cache.k, cache.v = k8, v8
+    cache.fp8 = (FP8_SCALE, FP8_SCALE)
+    torch.cuda.synchronize()
+
+
 def run_multi(args, rank, world, local_rank):
     import torch
     from paged_kv_cache_365_b200.replay import build_multi_step
@@ -513,6 +520,9 @@ def run_multi(args, rank, world, local_rank):
     st = build_multi_step(wl, args.new_tokens, dev, device_values=vals, seed=replica_seed(args.seed, rank))
     del vals
     cache = st["cache"]
+    fp8 = bool(args.kv_fp8)
+    if fp8:
+        to_fp8_pool(cache, dev)
     stream = torch.cuda.current_stream(dev)
     lens = st["host"]["context_lens"]
     T = int(st["q"].shape[0])
@@ -527,12 +537,20 @@ def run_multi(args, rank, world, local_rank):
     def pre():
         if n_pairs:
             pkv.copy_blocks(cache.k, cache.v, st["cow_pairs"])
-        pkv.kv_append(st["k_new"], st["v_new"], cache.k, cache.v, st["slot_mapping"])
+        if fp8:
+            pkv.kv_append_fp8(st["k_new"], st["v_new"], cache.k, cache.v, st["slot_mapping"], FP8_SCALE, FP8_SCALE)
+        else:
+            pkv.kv_append(st["k_new"], st["v_new"], cache.k, cache.v, st["slot_mapping"])
 
     def attend():
-        pkv.paged_attention_multi(st["q"], cache.k, cache.v, st["block_tables"], st["context_lens"],
-                                  st["query_start"], max_ctx, max_q, scale, out=out, workspace=ws,
-                                  partition=args.partition)
+        if fp8:
+            pkv.paged_attention_multi_fp8(st["q"], cache.k, cache.v, st["block_tables"], st["context_lens"],
+                                          st["query_start"], max_ctx, max_q, scale, FP8_SCALE, FP8_SCALE, out=out,
+                                          workspace=ws, partition=args.partition)
+        else:
+            pkv.paged_attention_multi(st["q"], cache.k, cache.v, st["block_tables"], st["context_lens"],
+                                      st["query_start"], max_ctx, max_q, scale, out=out, workspace=ws,
+                                      partition=args.partition)
 
     def step():
         pre()
@@ -587,7 +605,7 @@ def run_multi(args, rank, world, local_rank):
         raise RuntimeError("device error flags raised during timing")
     total_ms, att_ms, e2e_ms = max_over_ranks([total_ms, att_ms, e2e_ms], world, dev)
     es = STORAGE[wl.dtype]
-    kv = int(np.asarray(lens, dtype=np.int64).sum()) * wl.Hkv * wl.D * 2 * es
+    kv = int(np.asarray(lens, dtype=np.int64).sum()) * wl.Hkv * wl.D * 2 * (1 if fp8 else es)
     att_bytes = kv + 2 * T * wl.Hq * wl.D * es + int(sum(-(-int(n) // 16) for n in lens)) * 4 + 8 * wl.B + 4
     launches = (1 + (1 if n_pairs else 0) + 1 + (1 if P > 1 else 0)) * K
     return dict(wl=wl, K=K, T=T, kv=kv, att_bytes=att_bytes, total_ms=total_ms, att_ms=att_ms, e2e_ms=e2e_ms,
@@ -665,7 +683,11 @@ def multi_line(args, r, world):
                      "traffic": None, "algorithmic_bytes_per_launch": r["att_bytes"],
                      "useful_flops_per_launch": flops, "avg_launch_us": 1e3 * r["att_ms"]},
     }
-    if world == 1 and not args.no_cpu_baseline:
+    fp8 = bool(getattr(args, "kv_fp8", False))
+    if fp8:
+        line["config"]["kv_cache"] = "e4m3 (FP8) codes, scale %.6g for K and V" % FP8_SCALE
+        line["roofline"]["kernel"] = "paged_multi_fp8 (tcgen05 kernel + merge)"
+    if world == 1 and not args.no_cpu_baseline and not fp8:
         line["cpu_baseline"] = multi_cpu_baseline(wl, args.new_tokens, seed=args.seed)
     return line
 

@@ -488,6 +488,26 @@ pkv_status pkv_paged_attention_multi(void* out, const void* q, const void* k_cac
                                      int num_blocks, float scale, int partition_tokens, pkv_dtype dtype,
                                      void* workspace, size_t workspace_bytes, void* stream);
 
+/* pkv_paged_attention_multi_fp8 -- pkv_paged_attention_multi over an FP8
+ * (E4M3) pool written by pkv_kv_append_fp8: the rows, causal rule, tiles,
+ * partitions, workspace and errors of pkv_paged_attention_multi, and the
+ * cache layout and scales of pkv_paged_attention_decode_fp8 (a stored K
+ * value is code * k_scale, V alike; k_scale, v_scale finite and > 0, else
+ * PKV_EINVAL).  q and out in q_dtype (fp16 or bf16).  Every shape runs on
+ * the tcgen05 kernel: tiles of 128 rows (num_seqs * ceil(max_query_len * G
+ * / 128) <= 65535); each key block's codes are copied (TMA) into shared
+ * memory and widened there to fp16 (exact), bf16 queries are rescaled into
+ * fp16 per row by a power of two, the K scale goes into the logits and the
+ * V scale into the output. */
+pkv_status pkv_paged_attention_multi_fp8(void* out, const void* q, const void* k_cache, const void* v_cache,
+                                         const int32_t* block_tables, int max_blocks_per_seq,
+                                         const int32_t* context_lens, int max_context_len,
+                                         const int32_t* query_start, int max_query_len, int total_query_tokens,
+                                         int num_seqs, int num_q_heads, int num_kv_heads, int head_dim,
+                                         int num_blocks, float scale, float k_scale, float v_scale,
+                                         int partition_tokens, pkv_dtype q_dtype, void* workspace,
+                                         size_t workspace_bytes, void* stream);
+
 /* ------------------------------------------------------------------------
  * Step planning on the host (no CUDA call; host arrays).
  *

@@ -66,6 +66,10 @@ PROTOTYPES = {
     "pkv_paged_attention_multi": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_int, c_void_p, c_int,
                                           c_void_p, c_int, c_int, c_int, c_int, c_int, c_int, c_int, c_float, c_int,
                                           c_int, c_void_p, c_size_t, c_void_p]),
+    "pkv_paged_attention_multi_fp8": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_int, c_void_p,
+                                              c_int, c_void_p, c_int, c_int, c_int, c_int, c_int, c_int, c_int,
+                                              c_float, c_float, c_float, c_int, c_int, c_void_p, c_size_t,
+                                              c_void_p]),
     "pkv_get_error": (c_int, [P(c_uint32), c_void_p]),
     "pkv_partition_tokens": (c_int, [c_int, c_int, c_int, c_int]),
     "pkv_decode_prefix_fp8_workspace_bytes": (c_size_t, [c_int, c_int, c_int, c_int, c_int, c_int, c_int]),

@@ -516,6 +516,40 @@ def paged_attention_multi(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch
     return out
 
 
+def paged_attention_multi_fp8(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
+                              block_tables: torch.Tensor, context_lens: torch.Tensor, query_start: torch.Tensor,
+                              max_context_len: int, max_query_len: int, scale: float, k_scale: float,
+                              v_scale: float, out: Optional[torch.Tensor] = None,
+                              workspace: Optional[torch.Tensor] = None, partition: int = 0,
+                              stream=None) -> torch.Tensor:
+    """paged_attention_multi over an FP8 cache (E4M3 codes, one scale for K
+    and one for V); q and the output in fp16 or bf16."""
+    nb, hkv, d = _cache_dims(k_cache, v_cache)
+    if k_cache.dtype not in _FP8:
+        raise ValueError("an FP8 cache (float8_e4m3fn or uint8) is required")
+    if q.dim() != 3 or q.shape[2] != d or q.dtype not in (torch.float16, torch.bfloat16):
+        raise ValueError("q must be [T, Hq, D] in fp16 or bf16")
+    T, hq, _ = q.shape
+    B = block_tables.shape[0]
+    if block_tables.dim() != 2 or context_lens.shape != (B,) or query_start.shape != (B + 1,):
+        raise ValueError("block_tables [B, W], context_lens [B] and query_start [B + 1] required")
+    if out is None:
+        out = torch.empty_like(q)
+    need = multi_workspace_bytes(T, hq, d, max_context_len, partition)
+    if need and (workspace is None or workspace.numel() * workspace.element_size() < need):
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    ws_ptr = _dev(workspace, "workspace") if need else None
+    ws_len = workspace.numel() * workspace.element_size() if need else 0
+    check(lib.pkv_paged_attention_multi_fp8(
+        _dev(out, "out", q.dtype), _dev(q, "q"), _dev(k_cache, "k_cache"), _dev(v_cache, "v_cache"),
+        _dev(block_tables, "block_tables", torch.int32), block_tables.shape[1],
+        _dev(context_lens, "context_lens", torch.int32), int(max_context_len),
+        _dev(query_start, "query_start", torch.int32), int(max_query_len), T, B, hq, hkv, d, nb, float(scale),
+        float(k_scale), float(v_scale), int(partition), _DT[q.dtype], ws_ptr, ws_len, _stream(stream, q.device)),
+        "pkv_paged_attention_multi_fp8")
+    return out
+
+
 def get_error(stream=None, device=None) -> int:
     """Read and clear the device error word (PKV_ERR_* bits); synchronises."""
     v = ctypes.c_uint32(0)
@@ -989,8 +1023,6 @@ class PagedKVCache:
         causal attention of each new token over its sequence.  Host inputs
         are copied in (pinned: asynchronously); a host ``out`` receives the
         result asynchronously.  Returns the device output [T, Hq, D]."""
-        if self.fp8 is not None:
-            raise ValueError("multi-token attention reads 16-bit pools only")
         dev = self.device
         st = torch.cuda.current_stream(dev) if stream is None else stream
         stg = self._staging()
@@ -1001,8 +1033,13 @@ class PagedKVCache:
             res = out if (out is not None and out.device == dev) else stg.output(st, q.shape, self.dtype)
             sc = (1.0 / math.sqrt(self.D)) if scale is None else scale
             ws = self.workspace(multi_workspace_bytes(q.shape[0], q.shape[1], self.D, max_context_len, partition))
-            paged_attention_multi(x["q"], self.k, self.v, x["tables"], x["lens"], x["qs"], max_context_len,
-                                  max_query_len, sc, out=res, workspace=ws, partition=partition, stream=st)
+            if self.fp8 is not None:
+                paged_attention_multi_fp8(x["q"], self.k, self.v, x["tables"], x["lens"], x["qs"], max_context_len,
+                                          max_query_len, sc, self.fp8[0], self.fp8[1], out=res, workspace=ws,
+                                          partition=partition, stream=st)
+            else:
+                paged_attention_multi(x["q"], self.k, self.v, x["tables"], x["lens"], x["qs"], max_context_len,
+                                      max_query_len, sc, out=res, workspace=ws, partition=partition, stream=st)
         stg.finish(st, res, out)
         return res
 

@@ -50,7 +50,8 @@ struct MultiArgs {
   int tiles;      // row tiles per sequence in the grid: ceil(max_query_len * G / 16)
   int max_q;      // max_query_len
   int total_q;    // T
-  float qk_scale; // scale * log2(e)
+  float qk_scale; // scale * log2(e) (times the K scale over an FP8 pool)
+  float v_scale;  // the V scale over an FP8 pool (tcgen05 kernel only)
 };
 
 // Range-checked view of sequence b: context length, first row, new tokens.

@@ -44,6 +44,7 @@
 // path.
 #pragma once
 
+#include "decode_fp8.cuh"
 #include "multi_mma.cuh"
 
 namespace pkv {
@@ -244,6 +245,64 @@ struct TcShape {
   static_assert(kKV % 1024 == 0 && kQPanel % 1024 == 0, "swizzled panels need 1024-byte alignment");
 };
 
+// FP8 pools: a block's 64 x D E4M3 codes land (TMA, the pool's per-page
+// swizzle of decode_fp8.cuh) in the upper half of a 16-bit stage and are
+// widened in place into the stage's 16-bit layout by one warp; keys not in
+// `valid` (bit r: key r of the block) become zeros.  Outputs below the codes
+// are written while the codes are read; the rest only after the whole warp
+// has read its codes (__syncwarp), since they overwrite them.
+template <int D, int NSK, int NSV>
+__device__ __forceinline__ void tc_widen_fp8(unsigned char* stage, uint64_t valid, int lane) {
+  using S = TcShape<D, NSK, NSV>;
+  constexpr int kH = S::kKV / 2;  // byte offset of the codes
+  constexpr int kPer = D / 8;     // 8-code pieces per lane in each half
+  // piece k of half h of this lane: key r, codes 8 u .. 8 u + 7
+  auto piece = [&](int h, int k, int& r, int& u) {
+    const int i = lane + 32 * k;
+    if constexpr (D == 128) {
+      r = i >> 3;
+      u = (i & 7) + 8 * h;  // half 0: columns 0..63 (panel 0), half 1: panel 1
+    } else {
+      r = (i >> 3) + 32 * h;  // half 0: keys 0..31, half 1: keys 32..63
+      u = i & 7;
+    }
+  };
+  auto src = [&](int r, int u) {
+    return reinterpret_cast<const uint2*>(stage + kH + swz8<D>(r, u >> 1) + 8 * (u & 1));
+  };
+  auto dst = [&](int r, int u) {
+    return reinterpret_cast<uint4*>(stage + (u >> 3) * S::kKVPanel + r * 128 + (((u & 7) ^ (r & 7)) << 4));
+  };
+  auto widen = [&](uint2 w, int r) {
+    uint4 o = make_uint4(0u, 0u, 0u, 0u);
+    if ((valid >> r) & 1ull) {
+      e4m3x4_to_f16(w.x, o.x, o.y);
+      e4m3x4_to_f16(w.y, o.z, o.w);
+    }
+    return o;
+  };
+#pragma unroll
+  for (int k = 0; k < kPer; ++k) {
+    int r, u;
+    piece(0, k, r, u);
+    *dst(r, u) = widen(*src(r, u), r);
+  }
+  uint2 w[kPer];
+#pragma unroll
+  for (int k = 0; k < kPer; ++k) {
+    int r, u;
+    piece(1, k, r, u);
+    w[k] = *src(r, u);
+  }
+  __syncwarp();
+#pragma unroll
+  for (int k = 0; k < kPer; ++k) {
+    int r, u;
+    piece(1, k, r, u);
+    *dst(r, u) = widen(w[k], r);
+  }
+}
+
 #ifndef PKV_TC_K_STAGES
 #define PKV_TC_K_STAGES 2
 #endif
@@ -254,7 +313,7 @@ struct TcShape {
 #define PKV_TC_MIN_CTAS 2
 #endif
 
-template <typename T, int D, int G, int NSK, int NSV>
+template <typename T, int D, int G, int NSK, int NSV, bool F8 = false>
 __global__ void __launch_bounds__(TcShape<D, NSK, NSV>::kThreads, PKV_TC_MIN_CTAS)
     paged_multi_tc_kernel(const MultiArgs a, const __grid_constant__ CUtensorMap tmap_k,
                           const __grid_constant__ CUtensorMap tmap_v) {
@@ -268,7 +327,10 @@ __global__ void __launch_bounds__(TcShape<D, NSK, NSV>::kThreads, PKV_TC_MIN_CTA
   if (threadIdx.x == 0) TC_TRACE(0, 9);
   if (threadIdx.x == 0) TC_CTA(0, tc_gtime());
   using S = TcShape<D, NSK, NSV>;
-  using M = Mma<T>;
+  // the MMAs' element type: T, or fp16 over an FP8 pool (every E4M3 value
+  // is an fp16 value; bf16 queries are rescaled into fp16 per row)
+  using TM = typename std::conditional<F8, __half, T>::type;
+  using M = Mma<TM>;
   const int kvh = blockIdx.x;
   const int b = blockIdx.y / a.tiles;
   const int tile = blockIdx.y % a.tiles;
@@ -364,10 +426,11 @@ __global__ void __launch_bounds__(TcShape<D, NSK, NSV>::kThreads, PKV_TC_MIN_CTA
     if (lane == 0) {
       auto issue = [&](bool is_v, int c) {
         const int s = c % (is_v ? NSV : NSK);
+        constexpr uint32_t kPageBytes = F8 ? kBlockSize * D : kBlockSize * D * 2;
         uint32_t bytes = 0;
 #pragma unroll
         for (int p = 0; p < S::kPages; ++p)
-          if (loaded(c * S::kPages + p)) bytes += S::kPanels * 2048;
+          if (loaded(c * S::kPages + p)) bytes += kPageBytes;
         const uint32_t bar = (is_v ? bar_vfull : bar_kfull) + 8 * s;
         if (bytes == 0) {
           mbar_arrive(bar);
@@ -381,8 +444,13 @@ __global__ void __launch_bounds__(TcShape<D, NSK, NSV>::kThreads, PKV_TC_MIN_CTA
           const int i = c * S::kPages + p;
           if (!loaded(i)) continue;
           const int y = (table[i] * a.num_kv_heads + kvh) * kBlockSize;
+          if constexpr (F8) {
+            tma_load_2d(st + S::kKV / 2 + p * kPageBytes, map, 0, y, bar);  // one box of 16 rows x D codes
+          } else {
 #pragma unroll
-          for (int bx = 0; bx < S::kPanels; ++bx) tma_load_2d(st + bx * S::kKVPanel + p * 2048, map, bx * 64, y, bar);
+            for (int bx = 0; bx < S::kPanels; ++bx)
+              tma_load_2d(st + bx * S::kKVPanel + p * 2048, map, bx * 64, y, bar);
+          }
         }
       };
       long long t0 = clock64();
@@ -415,35 +483,55 @@ __global__ void __launch_bounds__(TcShape<D, NSK, NSV>::kThreads, PKV_TC_MIN_CTA
       }
     }
   } else if (warp == 1) {
-    // ---- MMA issuer (lane 0) and V-row zeroing (the whole warp) -------------
-    constexpr uint32_t kIdQK = tc_idesc<T>(128, S::kKeys, false);
-    constexpr uint32_t kIdPV = tc_idesc<T>(128, D, true);
+    // ---- MMA issuer (lane 0); V-row zeroing, or the widening of FP8 codes,
+    // by the whole warp ---------------------------------------------------
+    constexpr uint32_t kIdQK = tc_idesc<TM>(128, S::kKeys, false);
+    constexpr uint32_t kIdPV = tc_idesc<TM>(128, D, true);
     auto wait_all = [&](uint32_t bar, uint32_t parity) { return __all_sync(kFull, mbar_wait_bounded(bar, parity)); };
-    auto pv = [&](int j) -> bool {
-      if (!wait_all(bar_pfull + 8 * (j & 1), (j >> 1) & 1)) return false;
-      if (lane == 0) TC_TRACE(j, 4);
-      const int s = j % NSV;
-      if (!wait_all(bar_vfull + 8 * s, (j / NSV) & 1)) return false;
-      // zero the V rows of keys that are not there (past the context or on
-      // pages the table does not name): a zero weight must not meet a NaN
-      const uint32_t vst_off = static_cast<uint32_t>(S::kOffV) + s * S::kKV;
-      bool zeroed = false;
+    // keys of block c that are there (inside the partition and the context,
+    // on pages the table names): bit r for key r
+    auto valid_keys = [&](int c) -> uint64_t {
+      const int lim = tok1 - (tok0 + c * S::kKeys);
+      uint64_t m = lim >= S::kKeys ? ~0ull : (lim > 0 ? (1ull << lim) - 1ull : 0ull);
 #pragma unroll
-      for (int p = 0; p < S::kPages; ++p) {
-        const int i = j * S::kPages + p;
-        const int page_tok = tok0 + i * kBlockSize;
-        const int first = loaded(i) ? max(0, min(kBlockSize, tok1 - page_tok)) : 0;
-        if (first >= kBlockSize) continue;
-        zeroed = true;
-        const int n = (kBlockSize - first) * S::kPanels * 8;  // 16-byte chunks
-        for (int e = lane; e < n; e += 32) {
-          const int row = first + e / (S::kPanels * 8);
-          const int pn = (e / 8) % S::kPanels;
-          *reinterpret_cast<uint4*>(smem + vst_off + pn * S::kKVPanel + (p * kBlockSize + row) * 128 + (e & 7) * 16) =
-              make_uint4(0u, 0u, 0u, 0u);
+      for (int p = 0; p < S::kPages; ++p)
+        if (!loaded(c * S::kPages + p)) m &= ~(0xFFFFull << (16 * p));
+      return m;
+    };
+    auto pv = [&](int j) -> bool {
+      const int s = j % NSV;
+      if constexpr (F8) {
+        // the block's V codes widened while its softmax runs
+        if (!wait_all(bar_vfull + 8 * s, (j / NSV) & 1)) return false;
+        tc_widen_fp8<D, NSK, NSV>(smem + S::kOffV + s * S::kKV, valid_keys(j), lane);
+        fence_proxy_async_smem();
+        if (!wait_all(bar_pfull + 8 * (j & 1), (j >> 1) & 1)) return false;
+        if (lane == 0) TC_TRACE(j, 4);
+      } else {
+        if (!wait_all(bar_pfull + 8 * (j & 1), (j >> 1) & 1)) return false;
+        if (lane == 0) TC_TRACE(j, 4);
+        if (!wait_all(bar_vfull + 8 * s, (j / NSV) & 1)) return false;
+        // zero the V rows of keys that are not there (past the context or on
+        // pages the table does not name): a zero weight must not meet a NaN
+        const uint32_t vst_off = static_cast<uint32_t>(S::kOffV) + s * S::kKV;
+        bool zeroed = false;
+#pragma unroll
+        for (int p = 0; p < S::kPages; ++p) {
+          const int i = j * S::kPages + p;
+          const int page_tok = tok0 + i * kBlockSize;
+          const int first = loaded(i) ? max(0, min(kBlockSize, tok1 - page_tok)) : 0;
+          if (first >= kBlockSize) continue;
+          zeroed = true;
+          const int n = (kBlockSize - first) * S::kPanels * 8;  // 16-byte chunks
+          for (int e = lane; e < n; e += 32) {
+            const int row = first + e / (S::kPanels * 8);
+            const int pn = (e / 8) % S::kPanels;
+            *reinterpret_cast<uint4*>(smem + vst_off + pn * S::kKVPanel + (p * kBlockSize + row) * 128 + (e & 7) * 16) =
+                make_uint4(0u, 0u, 0u, 0u);
+          }
         }
+        if (zeroed) fence_proxy_async_smem();
       }
-      if (zeroed) fence_proxy_async_smem();
       __syncwarp();
       tc_fence_after();
       if (lane == 0) {
@@ -472,6 +560,11 @@ __global__ void __launch_bounds__(TcShape<D, NSK, NSV>::kThreads, PKV_TC_MIN_CTA
         break;
       }
       if (lane == 0) TC_TRACE(c, 2);
+      if constexpr (F8) {
+        tc_widen_fp8<D, NSK, NSV>(smem + S::kOffK + s * S::kKV, valid_keys(c), lane);
+        fence_proxy_async_smem();
+        __syncwarp();
+      }
       // S buffer c & 1 was last read (as P) by the P.V of block c - 2
       if (c >= 2 && !wait_all(bar_pvdone, (c - 2) & 1)) {
         bad = true;
@@ -503,6 +596,9 @@ __global__ void __launch_bounds__(TcShape<D, NSK, NSV>::kThreads, PKV_TC_MIN_CTA
     __syncwarp();
     mbar_wait_bounded(bar_final, 0);
   } else {
+    // the row's logit multiplier (log2 units; over an FP8 pool it carries
+    // the K scale and, for bf16 queries, the row's power-of-two rescale)
+    float qmul = a.qk_scale;
     {
       // this thread's row of Q into the 128-byte-swizzled K-major tile
       // (rows past the batch are zeros), while the first copies fly
@@ -510,11 +606,41 @@ __global__ void __launch_bounds__(TcShape<D, NSK, NSV>::kThreads, PKV_TC_MIN_CTA
       const int tr = r0 + r;
       const uint4* src = tr < R ? reinterpret_cast<const uint4*>(reinterpret_cast<const T*>(a.q) + out_row(tr) * D)
                                 : nullptr;
+      uint4 qv[D / 8];
 #pragma unroll
-      for (int c = 0; c < D / 8; ++c) {
-        const uint4 v = src ? src[c] : make_uint4(0u, 0u, 0u, 0u);
-        *reinterpret_cast<uint4*>(smem + (c >> 3) * S::kQPanel + r * 128 + (((c & 7) ^ (r & 7)) << 4)) = v;
+      for (int c = 0; c < D / 8; ++c) qv[c] = src ? src[c] : make_uint4(0u, 0u, 0u, 0u);
+      if constexpr (F8 && !std::is_same<T, __half>::value) {
+        // bf16 row -> fp16 times 2^kq, kq putting the row's largest
+        // magnitude just under 2^15 (exact unless an element falls below
+        // fp16's normal range); the logits take 2^-kq back
+        float mx = 0.f;
+#pragma unroll
+        for (int c = 0; c < D / 8; ++c) {
+          const uint32_t w[4] = {qv[c].x, qv[c].y, qv[c].z, qv[c].w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float2 f = Mma<T>::unpack(w[e]);
+            mx = fmax3(mx, fabsf(f.x), fabsf(f.y));
+          }
+        }
+        const int ex = static_cast<int>((__float_as_uint(mx) >> 23) & 0xffu) - 127;
+        const int kq = mx > 0.f ? min(max(14 - ex, -126), 126) : 0;
+        const float sc = __uint_as_float(static_cast<uint32_t>(kq + 127) << 23);
+        qmul *= __uint_as_float(static_cast<uint32_t>(127 - kq) << 23);
+#pragma unroll
+        for (int c = 0; c < D / 8; ++c) {
+          uint32_t w[4] = {qv[c].x, qv[c].y, qv[c].z, qv[c].w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float2 f = Mma<T>::unpack(w[e]);
+            w[e] = Mma<__half>::pack(f.x * sc, f.y * sc);
+          }
+          qv[c] = make_uint4(w[0], w[1], w[2], w[3]);
+        }
       }
+#pragma unroll
+      for (int c = 0; c < D / 8; ++c)
+        *reinterpret_cast<uint4*>(smem + (c >> 3) * S::kQPanel + r * 128 + (((c & 7) ^ (r & 7)) << 4)) = qv[c];
       fence_proxy_async_smem();  // the tensor core reads the tile through the async proxy
       __syncwarp();
       if (lane == 0) mbar_arrive(bar_qfull);
@@ -541,7 +667,7 @@ __global__ void __launch_bounds__(TcShape<D, NSK, NSV>::kThreads, PKV_TC_MIN_CTA
       const int lim = min(pos, tok1 - 1) - kb0;
       // plain block: every key in, and a positive scale, so the max can be
       // taken on the raw scores and the scale folded into the exponent
-      const bool plain = __all_sync(kFull, lim >= S::kKeys - 1 && pages_ok == 0xFu && a.qk_scale > 0.f);
+      const bool plain = __all_sync(kFull, lim >= S::kKeys - 1 && pages_ok == 0xFu && qmul > 0.f);
       if (!wait_all(bar_sfull + 8 * (j & 1), (j >> 1) & 1)) {
         bad = true;
         break;
@@ -560,7 +686,7 @@ __global__ void __launch_bounds__(TcShape<D, NSK, NSV>::kThreads, PKV_TC_MIN_CTA
       tmem_ld64(scol, v);
       if (warp == 4 && lane == 0) TC_TRACE(j, 11);
       float x[S::kKeys];
-      float mul = a.qk_scale;  // x * mul is the score in log2 units
+      float mul = qmul;  // x * mul is the score in log2 units
       if (plain) {
 #pragma unroll
         for (int k = 0; k < S::kKeys; ++k) x[k] = __uint_as_float(v[k]);
@@ -569,7 +695,7 @@ __global__ void __launch_bounds__(TcShape<D, NSK, NSV>::kThreads, PKV_TC_MIN_CTA
 #pragma unroll
         for (int k = 0; k < S::kKeys; ++k) {
           const bool ok = k <= lim && ((pages_ok >> (k >> 4)) & 1u);
-          x[k] = ok ? __uint_as_float(v[k]) * a.qk_scale : -INFINITY;
+          x[k] = ok ? __uint_as_float(v[k]) * qmul : -INFINITY;
         }
         mul = 1.f;
       }
@@ -591,6 +717,15 @@ __global__ void __launch_bounds__(TcShape<D, NSK, NSV>::kThreads, PKV_TC_MIN_CTA
         rescale = m_ref != -INFINITY && j > 0;
         l *= alpha;
         m_ref = bm;
+      }
+      // 2^(x mul - m) as one FFMA leaves the residual of the rounded max
+      // product, up to half an ulp of m: harmless while |m| < 2^20 (under
+      // 2^-4); past that the scores are rounded to their products first,
+      // so the maximal one gives exactly 2^0
+      if (__any_sync(kFull, fabsf(m_ref) >= 1048576.f && mul != 1.f)) {
+#pragma unroll
+        for (int k = 0; k < S::kKeys; ++k) x[k] *= mul;
+        mul = 1.f;
       }
       const float nmr = m_ref == -INFINITY ? 0.f : -m_ref;
       uint32_t ph[S::kKeys / 2], pl[S::kKeys / 2];
@@ -643,7 +778,10 @@ __global__ void __launch_bounds__(TcShape<D, NSK, NSV>::kThreads, PKV_TC_MIN_CTA
       tc_fence_after();
       const bool has = valid && pos >= tok0;
       const size_t row = valid ? out_row(tr) : 0;
-      const float inv = has ? 1.f / l : 0.f;
+      // over an FP8 pool the V scale multiplies the output (or the partial:
+      // the merge is linear in it)
+      const float osc = F8 ? a.v_scale : 1.f;
+      const float inv = has ? osc / l : 0.f;
 #pragma unroll
       for (int h = 0; h < D / 32; ++h) {
         uint32_t v[32];
@@ -656,7 +794,8 @@ __global__ void __launch_bounds__(TcShape<D, NSK, NSV>::kThreads, PKV_TC_MIN_CTA
             uint32_t w[4];
 #pragma unroll
             for (int e = 0; e < 4; ++e)
-              w[e] = has ? M::pack(__uint_as_float(v[8 * q + 2 * e]) * inv, __uint_as_float(v[8 * q + 2 * e + 1]) * inv)
+              w[e] = has ? Mma<T>::pack(__uint_as_float(v[8 * q + 2 * e]) * inv,
+                                        __uint_as_float(v[8 * q + 2 * e + 1]) * inv)
                          : 0u;
             dst[q] = make_uint4(w[0], w[1], w[2], w[3]);
           }
@@ -664,8 +803,8 @@ __global__ void __launch_bounds__(TcShape<D, NSK, NSV>::kThreads, PKV_TC_MIN_CTA
           float4* dst = reinterpret_cast<float4*>(a.ws_o + (row * a.num_parts + z) * D + 32 * h);
 #pragma unroll
           for (int q = 0; q < 8; ++q)
-            dst[q] = make_float4(__uint_as_float(v[4 * q]), __uint_as_float(v[4 * q + 1]),
-                                 __uint_as_float(v[4 * q + 2]), __uint_as_float(v[4 * q + 3]));
+            dst[q] = make_float4(__uint_as_float(v[4 * q]) * osc, __uint_as_float(v[4 * q + 1]) * osc,
+                                 __uint_as_float(v[4 * q + 2]) * osc, __uint_as_float(v[4 * q + 3]) * osc);
         }
       }
       if (valid && pos >= tok0 && !direct) a.ws_ml[row * a.num_parts + z] = make_float2(m_ref, l);

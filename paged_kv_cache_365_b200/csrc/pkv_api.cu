@@ -146,21 +146,25 @@ pkv_status launch_multi_fa(const pkv::MultiArgs& a, const void* k_cache, const v
 #define PKV_TC_ABOVE_ROWS 32
 #endif
 constexpr int kTcAboveRows = PKV_TC_ABOVE_ROWS;
-constexpr int kTcCode = 200;  // dispatch code of paged_multi_tc_kernel
+constexpr int kTcCode = 200;     // dispatch code of paged_multi_tc_kernel
+constexpr int kTcFp8Code = 201;  // the same over an FP8 pool
 constexpr int kTcKStages = PKV_TC_K_STAGES;
 constexpr int kTcVStages = PKV_TC_V_STAGES;
 
-template <typename T, int D, int G>
+bool encode_fp8_map(CUtensorMap* map, const void* base, int D, long long rows);
+
+template <typename T, int D, int G, bool F8 = false>
 pkv_status launch_multi_tc(const pkv::MultiArgs& a, const void* k_cache, const void* v_cache, int num_blocks,
                            cudaStream_t st) {
   using S = pkv::TcShape<D, kTcKStages, kTcVStages>;
   static_assert(kMaxPartition / PKV_BLOCK_SIZE <= S::kMaxPages, "the page table of a partition fits shared memory");
   CUtensorMap mk, mv;
   const long long rows = static_cast<long long>(num_blocks) * a.num_kv_heads * PKV_BLOCK_SIZE;
-  if (!encode_cache_map(&mk, k_cache, pkv::Mma<T>::kTmaType, D, rows) ||
-      !encode_cache_map(&mv, v_cache, pkv::Mma<T>::kTmaType, D, rows))
+  if (F8 ? !encode_fp8_map(&mk, k_cache, D, rows) || !encode_fp8_map(&mv, v_cache, D, rows)
+         : !encode_cache_map(&mk, k_cache, pkv::Mma<T>::kTmaType, D, rows) ||
+               !encode_cache_map(&mv, v_cache, pkv::Mma<T>::kTmaType, D, rows))
     return PKV_ECUDA;
-  auto kfn = pkv::paged_multi_tc_kernel<T, D, G, kTcKStages, kTcVStages>;
+  auto kfn = pkv::paged_multi_tc_kernel<T, D, G, kTcKStages, kTcVStages, F8>;
   if (cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(S::kSmem)) !=
       cudaSuccess)
     return PKV_ECUDA;
@@ -182,6 +186,7 @@ pkv_status dispatch_nt_multi(const pkv::MultiArgs& a, int NT, const void* k, con
     case -4: return launch_multi_rows<T, D, G, 4>(a, k, v, nb, st);
     case kFaCode: return launch_multi_fa<T, D, G>(a, k, v, nb, st);
     case kTcCode: return launch_multi_tc<T, D, G>(a, k, v, nb, st);
+    case kTcFp8Code: return launch_multi_tc<T, D, G, true>(a, k, v, nb, st);
   }
   return PKV_EINVAL;
 }
@@ -836,14 +841,20 @@ size_t pkv_multi_workspace_bytes(int total_query_tokens, int num_q_heads, int he
   return multi_workspace_bytes(total_query_tokens, num_q_heads, head_dim, P);
 }
 
-pkv_status pkv_paged_attention_multi(void* out, const void* q, const void* k_cache, const void* v_cache,
-                                     const int32_t* block_tables, int max_blocks_per_seq,
-                                     const int32_t* context_lens, int max_context_len,
-                                     const int32_t* query_start, int max_query_len, int total_query_tokens,
-                                     int num_seqs, int num_q_heads, int num_kv_heads, int head_dim, int num_blocks,
-                                     float scale, int partition_tokens, pkv_dtype dtype, void* workspace,
-                                     size_t workspace_bytes_given, void* stream) {
+}  // extern "C"
+
+namespace {
+// Both multi-token entry points: a 16-bit pool (fp8 false; every kernel by
+// rows per kv-head) or an FP8 pool (the tcgen05 kernel for every shape).
+pkv_status multi_impl(void* out, const void* q, const void* k_cache, const void* v_cache,
+                      const int32_t* block_tables, int max_blocks_per_seq, const int32_t* context_lens,
+                      int max_context_len, const int32_t* query_start, int max_query_len, int total_query_tokens,
+                      int num_seqs, int num_q_heads, int num_kv_heads, int head_dim, int num_blocks, float scale,
+                      int partition_tokens, pkv_dtype dtype, void* workspace, size_t workspace_bytes_given,
+                      void* stream, bool fp8, float k_scale, float v_scale) {
   if (dtype != PKV_F16 && dtype != PKV_BF16) return PKV_EINVAL;  // tensor-core path only
+  if (fp8 && (!std::isfinite(k_scale) || !std::isfinite(v_scale) || !(k_scale > 0.f) || !(v_scale > 0.f)))
+    return PKV_EINVAL;
   const int part = resolve_multi_partition(partition_tokens, max_context_len);
   if (part < 0 || num_seqs < 0 || num_kv_heads <= 0 || num_kv_heads > 65535 || num_q_heads <= 0 ||
       num_q_heads % num_kv_heads != 0 || !group_ok(num_q_heads / num_kv_heads) || !head_dim_ok(head_dim) ||
@@ -858,10 +869,10 @@ pkv_status pkv_paged_attention_multi(void* out, const void* q, const void* k_cac
   if (static_cast<long long>(num_blocks) * num_kv_heads * PKV_BLOCK_SIZE > 0x7fffffffLL) return PKV_EINVAL;
   const int G = num_q_heads / num_kv_heads;
   const long long rows_max = static_cast<long long>(max_query_len) * G;
-  const bool tc = rows_max > kTcAboveRows;
+  const bool tc = fp8 || rows_max > kTcAboveRows;
   const bool fa = !tc && rows_max > kFaAboveRows;
   const int NW = (fa || tc) ? 0 : multi_rows_warps(rows_max);
-  const int NT = tc ? kTcCode : fa ? kFaCode : NW ? -NW : multi_ntiles(rows_max);
+  const int NT = tc ? (fp8 ? kTcFp8Code : kTcCode) : fa ? kFaCode : NW ? -NW : multi_ntiles(rows_max);
   const int tile_rows = tc ? 128 : fa ? 16 * kFaWarps : 8 * (NW ? NW : NT);
   const long long tiles = (rows_max + tile_rows - 1) / tile_rows;
   const long long P = (static_cast<long long>(max_context_len) + part - 1) / part;
@@ -891,7 +902,8 @@ pkv_status pkv_paged_attention_multi(void* out, const void* q, const void* k_cac
   a.tiles = static_cast<int>(tiles);
   a.max_q = max_query_len;
   a.total_q = total_query_tokens;
-  a.qk_scale = scale * kLog2e;
+  a.qk_scale = scale * kLog2e * (fp8 ? k_scale : 1.f);
+  a.v_scale = fp8 ? v_scale : 1.f;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   auto run = [&](auto tag) -> pkv_status {
     using T = decltype(tag);
@@ -900,6 +912,36 @@ pkv_status pkv_paged_attention_multi(void* out, const void* q, const void* k_cac
   };
   if (dtype == PKV_F16) return run(__half{});
   return run(__nv_bfloat16{});
+}
+}  // namespace
+
+extern "C" {
+
+pkv_status pkv_paged_attention_multi(void* out, const void* q, const void* k_cache, const void* v_cache,
+                                     const int32_t* block_tables, int max_blocks_per_seq,
+                                     const int32_t* context_lens, int max_context_len,
+                                     const int32_t* query_start, int max_query_len, int total_query_tokens,
+                                     int num_seqs, int num_q_heads, int num_kv_heads, int head_dim, int num_blocks,
+                                     float scale, int partition_tokens, pkv_dtype dtype, void* workspace,
+                                     size_t workspace_bytes_given, void* stream) {
+  return multi_impl(out, q, k_cache, v_cache, block_tables, max_blocks_per_seq, context_lens, max_context_len,
+                    query_start, max_query_len, total_query_tokens, num_seqs, num_q_heads, num_kv_heads, head_dim,
+                    num_blocks, scale, partition_tokens, dtype, workspace, workspace_bytes_given, stream, false, 1.f,
+                    1.f);
+}
+
+pkv_status pkv_paged_attention_multi_fp8(void* out, const void* q, const void* k_cache, const void* v_cache,
+                                         const int32_t* block_tables, int max_blocks_per_seq,
+                                         const int32_t* context_lens, int max_context_len,
+                                         const int32_t* query_start, int max_query_len, int total_query_tokens,
+                                         int num_seqs, int num_q_heads, int num_kv_heads, int head_dim,
+                                         int num_blocks, float scale, float k_scale, float v_scale,
+                                         int partition_tokens, pkv_dtype q_dtype, void* workspace,
+                                         size_t workspace_bytes_given, void* stream) {
+  return multi_impl(out, q, k_cache, v_cache, block_tables, max_blocks_per_seq, context_lens, max_context_len,
+                    query_start, max_query_len, total_query_tokens, num_seqs, num_q_heads, num_kv_heads, head_dim,
+                    num_blocks, scale, partition_tokens, q_dtype, workspace, workspace_bytes_given, stream, true,
+                    k_scale, v_scale);
 }
 
 size_t pkv_decode_prefix_fp8_workspace_bytes(int num_seqs, int num_q_heads, int num_kv_heads, int head_dim,

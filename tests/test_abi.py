@@ -238,3 +238,25 @@ def test_decode_step_rejections(lib):
     a = list(ok)
     a[14] = 4
     assert lib.pkv_decode_step(*a) == 1
+
+
+def test_multi_fp8_rejections(lib):
+    """pkv_paged_attention_multi_fp8: the multi-token argument checks plus
+    the two scales (finite, > 0), all before any CUDA call."""
+    f = ctypes.c_float
+    args = [FAKE, FAKE, FAKE, FAKE, FAKE, 100, FAKE, 1100, FAKE, 8, 40, 4, 8, 2, 128, 64, f(0.1), f(0.05), f(0.05),
+            512, 1, FAKE, 1 << 30, None]
+    for idx, bad in ((20, 0), (20, 3), (14, 96), (12, 6), (9, -1), (8, None), (21, None), (22, 16),
+                     (7, 100 * 16 + 1), (16, f(float("inf"))), (17, f(0.0)), (18, f(-1.0)), (17, f(float("nan"))),
+                     (18, f(float("inf")))):
+        a = list(args)
+        a[idx] = bad
+        assert lib.pkv_paged_attention_multi_fp8(*a) == 1, (idx, bad)
+    # every shape takes 128-row tiles: 600 sequences x ceil(9 x 4 / 128) = 600
+    # tiles fit, 4096 tokens x G 4 = 128 tiles a sequence do not
+    a = list(args)
+    a[9], a[11] = 4096, 600
+    assert lib.pkv_paged_attention_multi_fp8(*a) == 1
+    a = list(args)
+    a[10] = 0
+    assert lib.pkv_paged_attention_multi_fp8(*a) == 0

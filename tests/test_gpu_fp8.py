@@ -270,3 +270,158 @@ def test_cascade_over_fp8_cache_matches_oracle(case):
     assert np.isfinite(got).all()
     assert np.abs(got - want).max() <= TOL[dt]
     assert np.abs(got - plain.float().cpu().numpy()).max() <= TOL[dt]
+
+
+# ---- several query tokens per sequence over an FP8 cache ---------------------
+
+MULTI_CASES = [
+    # ctx, new tokens, Hq, Hkv, D, q dtype
+    ([5, 16, 17, 40, 1], [1, 4, 17, 8, 1], 4, 4, 128, "f16"),   # a few rows (one padded tile)
+    ([33, 20, 3, 64], [5, 20, 3, 16], 8, 2, 64, "bf16"),        # 64 rows per kv-head
+    ([300, 140, 2100], [150, 40, 33], 2, 1, 128, "bf16"),       # 300 rows: three tiles; two partitions
+    ([1030, 600], [40, 33], 2, 2, 64, "f16"),
+    ([700, 1500, 90], [5, 5, 3], 32, 8, 128, "bf16"),           # G = 4, 20 rows
+]
+
+
+def run_multi_fp8(q, kc, vc, tables, lens, qs, scale, ks, vs, dt, partition=0):
+    m = pkv()
+    out = m.paged_attention_multi_fp8(to_dev(q, dt), kc, vc, torch.from_numpy(tables).cuda(),
+                                      torch.from_numpy(lens).cuda(), torch.from_numpy(qs).cuda(), int(lens.max()),
+                                      int(np.diff(qs).max()), scale, ks, vs, partition=partition)
+    torch.cuda.synchronize()
+    return out.float().cpu().numpy(), m.get_error()
+
+
+@pytest.mark.parametrize("case", MULTI_CASES, ids=lambda c: f"{c[5]}_G{c[2] // c[3]}_D{c[4]}_rows{max(c[1]) * c[2] // c[3]}")
+@pytest.mark.parametrize("partition", [0, 16, 96])
+def test_multi_fp8_matches_oracle(case, partition):
+    """The tcgen05 kernel over E4M3 codes (widened in shared memory) against
+    the oracle's multi-token attention on the stored values; unwritten slots
+    hold the NaN code, tables are padded with out-of-range ids."""
+    ctx, nq, Hq, Hkv, D, dt = case
+    ks, vs = 0.011, 0.017
+    ref, kc, vc, tables, lens = build(ctx, Hkv, D, dt, ks, vs, seed=sum(ctx) + D)
+    qs = np.concatenate([[0], np.cumsum(nq)]).astype(np.int32)
+    rng = np.random.default_rng(partition + D + len(ctx))
+    q = storage(rng.standard_normal((int(qs[-1]), Hq, D)).astype(np.float32), dt)
+    scale = D ** -0.5
+    want = oracle.paged_multi(q, ref.k, ref.v, tables, lens, qs, scale, dt, kv_dtype="e4m3", k_scale=ks, v_scale=vs)
+    got, err = run_multi_fp8(q, kc, vc, tables, lens, qs, scale, ks, vs, dt, partition)
+    assert err == 0
+    assert np.isfinite(got).all()
+    assert np.abs(got - want).max() <= TOL[dt]
+
+
+@pytest.mark.parametrize("case", [MULTI_CASES[1], MULTI_CASES[2]],
+                         ids=lambda c: f"{c[5]}_G{c[2] // c[3]}_D{c[4]}")
+@pytest.mark.parametrize("scale", [None, 0.5])
+def test_multi_fp8_wide_values(case, scale):
+    """K, V and q drawn N(0, 4), bf16 queries with magnitudes that the
+    per-row power-of-two rescale must carry into fp16; bound as in
+    test_decode_fp8_wide_values (ulp-aware where the output is large)."""
+    ctx, nq, Hq, Hkv, D, dt = case
+    ks = vs = 2.0 * 6.0 / 448.0
+    ref, kc, vc, tables, lens = build(ctx, Hkv, D, dt, ks, vs, seed=3 * sum(ctx) + D, sigma=2.0)
+    qs = np.concatenate([[0], np.cumsum(nq)]).astype(np.int32)
+    rng = np.random.default_rng(D + 5)
+    q = storage(rng.standard_normal((int(qs[-1]), Hq, D)).astype(np.float32) * 2.0, dt)
+    sc = D ** -0.5 if scale is None else scale
+    want = oracle.paged_multi(q, ref.k, ref.v, tables, lens, qs, sc, dt, kv_dtype="e4m3", k_scale=ks, v_scale=vs)
+    got, err = run_multi_fp8(q, kc, vc, tables, lens, qs, sc, ks, vs, dt)
+    assert err == 0
+    assert np.isfinite(got).all()
+    assert (np.abs(got - want) <= ulp_aware_bound(want, dt, TOL[dt])).all()
+    if scale is not None:
+        assert np.abs(want).max() > 4.0
+
+
+def test_multi_fp8_large_and_small_query_rows():
+    """bf16 query rows far outside fp16's range (1e6) and far below its
+    normal range (1e-6): the per-row rescale keeps both; the logit scale is
+    chosen so the attention stays well-conditioned."""
+    ctx, nq, Hq, Hkv, D, dt = [90, 40], [20, 9], 4, 2, 128, "bf16"
+    ks, vs = 0.011, 0.017
+    ref, kc, vc, tables, lens = build(ctx, Hkv, D, dt, ks, vs, seed=77)
+    qs = np.concatenate([[0], np.cumsum(nq)]).astype(np.int32)
+    rng = np.random.default_rng(8)
+    q32 = rng.standard_normal((int(qs[-1]), Hq, D)).astype(np.float32)
+    q32[::2] *= 1e6
+    q32[1::2] *= 1e-6
+    q = storage(q32, dt)
+    for scale in (1e-7, 1e5):
+        want = oracle.paged_multi(q, ref.k, ref.v, tables, lens, qs, scale, dt, kv_dtype="e4m3", k_scale=ks,
+                                  v_scale=vs)
+        got, err = run_multi_fp8(q, kc, vc, tables, lens, qs, scale, ks, vs, dt)
+        assert err == 0 and np.isfinite(got).all()
+        rows = slice(0, None, 2) if scale < 1 else slice(1, None, 2)
+        assert np.abs(got[rows] - want[rows]).max() <= TOL[dt]
+
+
+def test_multi_fp8_rejects_bad_scales_and_16_bit_pools():
+    m = pkv()
+    ref, kc, vc, tables, lens = build([20], 1, 64, "f16", 0.05, 0.05, seed=1)
+    qs = np.array([0, 4], dtype=np.int32)
+    q = torch.zeros((4, 1, 64), dtype=torch.float16, device="cuda")
+    args = (q, kc, vc, torch.from_numpy(tables).cuda(), torch.from_numpy(lens).cuda(), torch.from_numpy(qs).cuda(),
+            20, 4, 0.125)
+    for ks, vs in ((0.0, 0.05), (0.05, -1.0), (float("inf"), 0.05)):
+        with pytest.raises(m.PkvError):
+            m.paged_attention_multi_fp8(*args, ks, vs)
+    with pytest.raises(ValueError):
+        m.paged_attention_multi_fp8(q, kc.half(), vc.half(), *args[3:], 0.05, 0.05)
+
+
+def test_multi_step_over_an_fp8_pool_through_the_cache_api():
+    """PagedKVCache with an FP8 pool: prefill, a fork that forces a
+    copy-on-write, then plan_multi_step + run_multi_step (host inputs); the
+    pool's codes bit-exact and the output against the oracle."""
+    m = pkv()
+    rng = np.random.default_rng(43)
+    Hq, Hkv, D, nb, ks, vs = 8, 2, 128, 48, 0.013, 0.019
+    order = rng.permutation(nb).astype(np.int32)
+    cache = m.PagedKVCache(nb, Hkv, D, torch.bfloat16, free_order=order, fp8_scales=(ks, vs))
+    ref = oracle.RefAllocator(nb, order)
+    dev = oracle.RefCache(nb, Hkv, D, "e4m3")
+
+    def vals(n):
+        return (storage(rng.standard_normal((n, Hkv, D)).astype(np.float32), "bf16"),
+                storage(rng.standard_normal((n, Hkv, D)).astype(np.float32), "bf16"))
+
+    for sid, n in ((0, 70), (1, 16), (2, 200)):
+        ref.add_seq(sid)
+        cache.add_seq(sid)
+        k, v = vals(n)
+        slots, cows = ref.append_tokens(sid, n)
+        dev.copy_blocks(cows)
+        dev.append_fp8(k, v, np.array(slots), "bf16", ks, vs)
+        cache.prefill(sid, to_dev(k, "bf16"), to_dev(v, "bf16"))
+    ref.fork(0, 3)
+    cache.fork(0, 3)
+    ids, n_new = [0, 1, 2, 3], [5, 3, 40, 4]
+    slots, pairs, qs, tables, lens = cache.plan_multi_step(ids, n_new)
+    r_slots, r_pairs = [], []
+    for sid, n in zip(ids, n_new):
+        s_, p_ = ref.append_tokens(sid, n)
+        r_slots += s_
+        r_pairs += p_
+    assert list(slots) == r_slots and [tuple(p) for p in pairs] == r_pairs
+    T = int(qs[-1])
+    q = storage(rng.standard_normal((T, Hq, D)).astype(np.float32), "bf16")
+    kn, vn = vals(T)
+    dev.copy_blocks(r_pairs)
+    dev.append_fp8(kn, vn, np.array(r_slots), "bf16", ks, vs)
+    out = torch.empty((T, Hq, D), dtype=torch.bfloat16, pin_memory=True)
+    cache.run_multi_step(torch.from_numpy(slots).pin_memory(), torch.from_numpy(pairs).pin_memory(),
+                         torch.from_numpy(tables).pin_memory(), torch.from_numpy(lens).pin_memory(),
+                         int(lens.max()), torch.from_numpy(qs).pin_memory(), max(n_new),
+                         to_dev(q, "bf16").cpu().pin_memory(), to_dev(kn, "bf16").cpu().pin_memory(),
+                         to_dev(vn, "bf16").cpu().pin_memory(), out=out)
+    torch.cuda.synchronize()
+    assert m.get_error() == 0
+    held = sorted({b for t in ref.tables.values() for b in t})
+    assert np.array_equal(cache.k.cpu().numpy()[held], dev.k[held])
+    assert np.array_equal(cache.v.cpu().numpy()[held], dev.v[held])
+    want = oracle.paged_multi(q, dev.k, dev.v, tables, lens, qs, D ** -0.5, "bf16", kv_dtype="e4m3", k_scale=ks,
+                              v_scale=vs)
+    assert np.abs(out.float().numpy() - want).max() <= TOL["bf16"]

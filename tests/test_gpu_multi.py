@@ -252,3 +252,20 @@ def test_multi_wide_values(case, scale):
         assert (np.abs(got - want) <= ulp_aware_bound(want, dt, TOL[dt])).all()
     if scale is not None:
         assert np.abs(want).max() > 4.0
+
+
+def test_tcgen05_kernel_huge_logits():
+    """Scores far past 2^20 in log2 units (q scaled by 1e4, logit scale
+    1e3) on the tcgen05 kernel (160 rows per kv-head): the attention is
+    one-hot on each row's best key, and the output must be that V row,
+    finite, within the stated tolerance."""
+    ctx, nq, Hq, Hkv, D, dt = [900, 300], [40, 11], 8, 2, 128, "bf16"
+    c = make_multi_case(ctx, nq, Hq, Hkv, D, dt, seed=12)
+    import workloads
+    q = oracle.widen(c["q"], dt) * 1e4
+    c["q"] = workloads._to_storage(q.astype(np.float32), dt)
+    want = oracle.paged_multi(c["q"], c["k"], c["v"], c["tables"], c["ctx"], c["qs"], 1e3, dt)
+    got, err = run_gpu(c, 1e3)
+    assert err == 0
+    assert np.isfinite(got).all()
+    assert np.abs(got - want).max() <= TOL[dt]
