@@ -52,6 +52,8 @@ struct MultiArgs {
   int total_q;    // T
   float qk_scale; // scale * log2(e) (times the K scale over an FP8 pool)
   float v_scale;  // the V scale over an FP8 pool (tcgen05 kernel only)
+  int* tc_ctr;           // tcgen05 kernel: [0] claim counter, [1] work-list length
+  int2* tc_items;        // tcgen05 kernel: the work list
 };
 
 // Range-checked view of sequence b: context length, first row, new tokens.

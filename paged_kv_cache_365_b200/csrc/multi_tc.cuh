@@ -184,37 +184,6 @@ __host__ __device__ constexpr uint32_t tc_idesc(int M, int N, bool b_mn_major) {
          (static_cast<uint32_t>(M >> 4) << 24);
 }
 
-// Timeline probe (debug builds with PKV_TC_TRACE only): SM clock at fixed
-// points of the pipeline for the first 64 CTAs and their first 32 blocks.
-#ifdef PKV_TC_TRACE
-__device__ long long g_tc_trace[64][32][12];
-#define TC_TRACE(j, slot)                                                                   \
-  do {                                                                                      \
-    const int cta_ = blockIdx.x + gridDim.x * (blockIdx.y + gridDim.y * blockIdx.z);       \
-    if (cta_ < 64 && (j) < 32) g_tc_trace[cta_][(j)][(slot)] = clock64();                  \
-  } while (0)
-// per CTA (first 16384): global timer at entry, at the first K copy and at
-// exit, and (SM id, key blocks)
-__device__ long long g_tc_cta[16384][4];
-__device__ __forceinline__ long long tc_gtime() {
-  long long t;
-  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-  return t;
-}
-#define TC_CTA(slot, v)                                                                    \
-  do {                                                                                      \
-    const int cta_ = blockIdx.x + gridDim.x * (blockIdx.y + gridDim.y * blockIdx.z);       \
-    if (cta_ < 16384) g_tc_cta[cta_][(slot)] = (v);                                         \
-  } while (0)
-#else
-#define TC_TRACE(j, slot) \
-  do {                    \
-  } while (0)
-#define TC_CTA(slot, v) \
-  do {                  \
-  } while (0)
-#endif
-
 // ----------------------------------------------------------------------------
 // the kernel
 // ----------------------------------------------------------------------------
@@ -231,11 +200,14 @@ struct TcShape {
   static constexpr size_t kOffV = kOffK + size_t(NSK) * kKV;        // V ring: NSV stages
   static constexpr size_t kOffBars = kOffV + size_t(NSV) * kKV;
   // barriers: kfull[NSK], kempty[NSK], vfull[NSV], vempty[NSV], sfull[2],
-  // pfull[2], pvdone, final, qfull
-  static constexpr int kBars = 2 * NSK + 2 * NSV + 7;
+  // pfull[2], pvdone, final, qfull, qempty, oempty, itemfull[2],
+  // itemempty[2], drain
+  static constexpr int kBars = 2 * NSK + 2 * NSV + 14;
   static constexpr size_t kOffTab = kOffBars + size_t(kBars) * 8;
   static constexpr int kMaxPages = 128;  // pages of the longest partition (2048 tokens)
-  static constexpr size_t kOffSlot = kOffTab + size_t(kMaxPages) * 4;
+  // two work-item slots: their page tables, then their descriptions
+  static constexpr size_t kOffItem = kOffTab + 2 * size_t(kMaxPages) * 4;
+  static constexpr size_t kOffSlot = kOffItem + 2 * 64;
   static constexpr size_t kSmem = 1024 /* alignment slack */ + kOffSlot + 16;
   static constexpr uint32_t kTmemCols = 256;
   static constexpr uint32_t kColO = 0;
@@ -255,39 +227,41 @@ template <int D, int NSK, int NSV>
 __device__ __forceinline__ void tc_widen_fp8(unsigned char* stage, uint64_t valid, int lane) {
   using S = TcShape<D, NSK, NSV>;
   constexpr int kH = S::kKV / 2;  // byte offset of the codes
-  constexpr int kPer = D / 8;     // 8-code pieces per lane in each half
-  // piece k of half h of this lane: key r, codes 8 u .. 8 u + 7
+  constexpr int kPer = D / 16;    // 16-code pieces per lane in each half
+  // piece k of half h of this lane: key r, codes 16 u .. 16 u + 15 (16-byte
+  // chunk u of the key's row of codes)
   auto piece = [&](int h, int k, int& r, int& u) {
     const int i = lane + 32 * k;
     if constexpr (D == 128) {
-      r = i >> 3;
-      u = (i & 7) + 8 * h;  // half 0: columns 0..63 (panel 0), half 1: panel 1
+      r = i >> 2;
+      u = (i & 3) + 4 * h;  // half 0: columns 0..63 (panel 0), half 1: panel 1
     } else {
-      r = (i >> 3) + 32 * h;  // half 0: keys 0..31, half 1: keys 32..63
-      u = i & 7;
+      r = (i >> 2) + 32 * h;  // half 0: keys 0..31, half 1: keys 32..63
+      u = i & 3;
     }
   };
-  auto src = [&](int r, int u) {
-    return reinterpret_cast<const uint2*>(stage + kH + swz8<D>(r, u >> 1) + 8 * (u & 1));
-  };
-  auto dst = [&](int r, int u) {
-    return reinterpret_cast<uint4*>(stage + (u >> 3) * S::kKVPanel + r * 128 + (((u & 7) ^ (r & 7)) << 4));
-  };
-  auto widen = [&](uint2 w, int r) {
-    uint4 o = make_uint4(0u, 0u, 0u, 0u);
+  auto src = [&](int r, int u) { return reinterpret_cast<const uint4*>(stage + kH + swz8<D>(r, u)); };
+  // the two 16-bit chunks (8 elements each) of codes 16 u .. 16 u + 15
+  auto put = [&](int r, int u, uint4 w) {
+    uint4 lo = make_uint4(0u, 0u, 0u, 0u), hi = lo;
     if ((valid >> r) & 1ull) {
-      e4m3x4_to_f16(w.x, o.x, o.y);
-      e4m3x4_to_f16(w.y, o.z, o.w);
+      e4m3x4_to_f16(w.x, lo.x, lo.y);
+      e4m3x4_to_f16(w.y, lo.z, lo.w);
+      e4m3x4_to_f16(w.z, hi.x, hi.y);
+      e4m3x4_to_f16(w.w, hi.z, hi.w);
     }
-    return o;
+    unsigned char* row = stage + (u >> 2) * S::kKVPanel + r * 128;
+    const int c = (2 * u) & 7;
+    *reinterpret_cast<uint4*>(row + ((c ^ (r & 7)) << 4)) = lo;
+    *reinterpret_cast<uint4*>(row + (((c + 1) ^ (r & 7)) << 4)) = hi;
   };
 #pragma unroll
   for (int k = 0; k < kPer; ++k) {
     int r, u;
     piece(0, k, r, u);
-    *dst(r, u) = widen(*src(r, u), r);
+    put(r, u, *src(r, u));
   }
-  uint2 w[kPer];
+  uint4 w[kPer];
 #pragma unroll
   for (int k = 0; k < kPer; ++k) {
     int r, u;
@@ -299,7 +273,79 @@ __device__ __forceinline__ void tc_widen_fp8(unsigned char* stage, uint64_t vali
   for (int k = 0; k < kPer; ++k) {
     int r, u;
     piece(1, k, r, u);
-    *dst(r, u) = widen(w[k], r);
+    put(r, u, w[k]);
+  }
+}
+
+// One work item of the persistent kernel: a (sequence, kv-head, row tile,
+// key partition), described by the producer warp for the other warps.
+struct TcItem {
+  int nb;  // key blocks of 64; < 0: no more work
+  int b, kvh, z, r0, R, q0, base, tok0, tok1, nblk, direct;
+};
+static_assert(sizeof(TcItem) <= 64, "an item slot is 64 bytes");
+
+// Key partitions of row tile t of a sequence that the kernel visits: the
+// partitions up to the tile's last position (a sequence held by one
+// partition: that one, also when it has nothing to attend, so its rows are
+// written as zeros).
+__host__ __device__ inline int tc_tile_parts(int ctx, int nq, int G, int t, int partition) {
+  if (ctx <= partition) return 1;
+  const int R = nq * G;
+  const int p_hi = ctx - nq + (min(R, t * 128 + 128) - 1) / G;
+  const int lim = min(ctx, p_hi + 1);
+  return lim > 0 ? (lim + partition - 1) / partition : 0;
+}
+
+// Key blocks (64 keys) of partition z of row tile t.
+__device__ __forceinline__ int tc_item_blocks(int ctx, int nq, int G, int t, int z, int partition) {
+  const int R = nq * G;
+  const int p_hi = ctx - nq + (min(R, t * 128 + 128) - 1) / G;
+  const int tok0 = z * partition;
+  const int tok1 = min(min(ctx, tok0 + partition), p_hi + 1);
+  return tok1 > tok0 ? (tok1 - tok0 + 63) / 64 : 0;
+}
+
+// The work list: one entry (b, tile << 16 | partition) per visited
+// (sequence, row tile, partition), longest first (a counting sort on the
+// number of key blocks, at most 32 for a 2048-token partition), so the
+// items left at the end of the kernel are the short ones; its length; the
+// claim counter zeroed.  One CTA of 1024 threads.
+template <int G>
+__global__ void __launch_bounds__(1024) paged_multi_tc_plan_kernel(const MultiArgs a) {
+  pdl_enter();
+  constexpr int kMaxNb = 32;
+  __shared__ int cnt[kMaxNb + 1], at[kMaxNb + 1];
+  const int tid = threadIdx.x;
+  if (tid <= kMaxNb) cnt[tid] = 0;
+  __syncthreads();
+  for (int pass = 0; pass < 2; ++pass) {
+    for (int b = tid; b < a.num_seqs; b += 1024) {
+      int ctx, q0, nq;
+      if (!multi_seq(a, b, ctx, q0, nq, pass == 0)) continue;
+      const int nt = (nq * G + 127) / 128;
+      for (int t = 0; t < nt; ++t) {
+        const int nz = tc_tile_parts(ctx, nq, G, t, a.partition);
+        for (int z = 0; z < nz; ++z) {
+          const int nb = min(tc_item_blocks(ctx, nq, G, t, z, a.partition), kMaxNb);
+          if (pass == 0)
+            atomicAdd(&cnt[nb], 1);
+          else
+            a.tc_items[atomicAdd(&at[nb], 1)] = make_int2(b, (t << 16) | z);
+        }
+      }
+    }
+    __syncthreads();
+    if (pass == 0 && tid == 0) {
+      int o = 0;
+      for (int nb = kMaxNb; nb >= 0; --nb) {
+        at[nb] = o;
+        o += cnt[nb];
+      }
+      a.tc_ctr[0] = 0;
+      a.tc_ctr[1] = o;
+    }
+    __syncthreads();
   }
 }
 
@@ -324,41 +370,13 @@ __global__ void __launch_bounds__(TcShape<D, NSK, NSV>::kThreads, PKV_TC_MIN_CTA
     asm volatile("prefetch.tensormap [%0];" ::"l"(&tmap_v) : "memory");
   }
   pdl_enter();
-  if (threadIdx.x == 0) TC_TRACE(0, 9);
-  if (threadIdx.x == 0) TC_CTA(0, tc_gtime());
   using S = TcShape<D, NSK, NSV>;
   // the MMAs' element type: T, or fp16 over an FP8 pool (every E4M3 value
   // is an fp16 value; bf16 queries are rescaled into fp16 per row)
   using TM = typename std::conditional<F8, __half, T>::type;
   using M = Mma<TM>;
-  const int kvh = blockIdx.x;
-  const int b = blockIdx.y / a.tiles;
-  const int tile = blockIdx.y % a.tiles;
-  const int z = blockIdx.z;
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-
-  int ctx, q0, nq;
-  if (!multi_seq(a, b, ctx, q0, nq, threadIdx.x == 0 && kvh == 0 && tile == 0 && z == 0)) return;
-  const int R = nq * G;
-  const int r0 = tile * S::kRows;
-  if (r0 >= R) return;
-  const int base = ctx - nq;
-  const int p_hi = base + (min(R, r0 + S::kRows) - 1) / G;
-  const bool direct = ctx <= a.partition;
-  const int tok0 = z * a.partition;
-  const int tok1 = min(min(ctx, tok0 + a.partition), p_hi + 1);
-  auto out_row = [&](int tr) -> size_t {
-    return static_cast<size_t>(q0 + tr / G) * a.num_q_heads + kvh * G + tr % G;
-  };
-  if (tok1 <= tok0) {
-    if (direct && z == 0)
-      for (int idx = threadIdx.x; idx < S::kRows * D; idx += S::kThreads) {
-        const int tr = r0 + idx / D;
-        if (tr < R) reinterpret_cast<T*>(a.out)[out_row(tr) * D + idx % D] = Fmt<T>::from_f32(0.f);
-      }
-    return;
-  }
 
   extern __shared__ unsigned char smem_raw[];
   const uint32_t raw_addr = smem_addr(smem_raw);
@@ -371,19 +389,12 @@ __global__ void __launch_bounds__(TcShape<D, NSK, NSV>::kThreads, PKV_TC_MIN_CTA
   const uint32_t bar_vfull = bar_kempty + 8 * NSK, bar_vempty = bar_vfull + 8 * NSV;
   const uint32_t bar_sfull = bar_vempty + 8 * NSV;
   const uint32_t bar_pfull = bar_sfull + 16, bar_pvdone = bar_pfull + 16, bar_final = bar_pvdone + 8;
-  const uint32_t bar_qfull = bar_final + 8;
-  int* table = reinterpret_cast<int*>(smem + S::kOffTab);
+  const uint32_t bar_qfull = bar_final + 8, bar_qempty = bar_qfull + 8, bar_oempty = bar_qempty + 8;
+  const uint32_t bar_itemfull = bar_oempty + 8, bar_itemempty = bar_itemfull + 16, bar_drain = bar_itemempty + 16;
+  int* tables = reinterpret_cast<int*>(smem + S::kOffTab);
+  TcItem* items = reinterpret_cast<TcItem*>(smem + S::kOffItem);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + S::kOffSlot);
 
-  const int pg0 = tok0 / kBlockSize;
-  const int nblk = (tok1 - tok0 + kBlockSize - 1) / kBlockSize;  // pages, <= kMaxPages
-  const int nb = (nblk + S::kPages - 1) / S::kPages;              // key blocks
-  for (int j = threadIdx.x; j < nblk; j += S::kThreads) {
-    const int e = a.block_tables[static_cast<long long>(b) * a.bt_stride + pg0 + j];
-    const bool in = e >= 0 && e < a.num_blocks;
-    if (!in) raise_error(PKV_ERR_BLOCK_RANGE);
-    table[j] = in ? e : -1;
-  }
   if (threadIdx.x == 0) {
     for (int s = 0; s < NSK; ++s) {
       mbar_init(bar_kfull + 8 * s, 1);
@@ -395,11 +406,16 @@ __global__ void __launch_bounds__(TcShape<D, NSK, NSV>::kThreads, PKV_TC_MIN_CTA
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(bar_sfull + 8 * i, 1);
-      mbar_init(bar_pfull + 8 * i, 4);  // one arrival per softmax warp
+      mbar_init(bar_pfull + 8 * i, 4);      // one arrival per softmax warp
+      mbar_init(bar_itemfull + 8 * i, 1);   // the producer
+      mbar_init(bar_itemempty + 8 * i, 5);  // the MMA warp and the softmax warps
     }
     mbar_init(bar_pvdone, 1);
     mbar_init(bar_final, 1);
-    mbar_init(bar_qfull, 4);  // one arrival per softmax warp
+    mbar_init(bar_qfull, 4);
+    mbar_init(bar_qempty, 1);
+    mbar_init(bar_oempty, 4);
+    mbar_init(bar_drain, 1);
     fence_barrier_init();
   }
   if (warp == 1) {
@@ -410,405 +426,553 @@ __global__ void __launch_bounds__(TcShape<D, NSK, NSV>::kThreads, PKV_TC_MIN_CTA
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  const int n_items = a.tc_ctr[1] * a.num_kv_heads;  // written by the plan kernel
 
-  // loaded(i): page i of the partition is staged (in range, named by the table)
-  auto loaded = [&](int i) { return i < nblk && table[i] >= 0; };
   bool bad = false;
-  int issued = 0, issued_v = 0;  // producer: key blocks whose K (V) copies it issued
+  int issued_k = 0, issued_v = 0;  // producer: key blocks whose K (V) copies it issued, over all items
+  auto wait_all = [&](uint32_t bar, uint32_t parity) { return __all_sync(kFull, mbar_wait_bounded(bar, parity)); };
+  // every warp walks the same items in the same order; item `it` sits in
+  // slot it & 1, its key blocks are numbered on from those of the items
+  // before it (g0 + j), which fixes their ring stages and barrier phases
+  auto loaded_in = [&](const TcItem& item, const int* tab, int i) { return i < item.nblk && tab[i] >= 0; };
 
   if (warp == 0) {
-    // ---- TMA producer (lane 0): the K ring and the V ring ------------------
+    // ---- producer (the whole warp): claims items, describes them, and
+    // (lane 0) issues their K and V copies ------------------------------------
     // A K stage is released as soon as the block's S = Q.K^T MMAs are done,
     // a V stage once its P.V MMAs are done, so K runs up to NSK blocks
-    // ahead of the scores and V up to NSV blocks ahead of the P.V products.
-    // One thread polls both rings, so a V stage that frees late never holds
-    // back the next K copy.
-    if (lane == 0) {
-      auto issue = [&](bool is_v, int c) {
-        const int s = c % (is_v ? NSV : NSK);
-        constexpr uint32_t kPageBytes = F8 ? kBlockSize * D : kBlockSize * D * 2;
-        uint32_t bytes = 0;
-#pragma unroll
-        for (int p = 0; p < S::kPages; ++p)
-          if (loaded(c * S::kPages + p)) bytes += kPageBytes;
-        const uint32_t bar = (is_v ? bar_vfull : bar_kfull) + 8 * s;
-        if (bytes == 0) {
-          mbar_arrive(bar);
-          return;
+    // ahead of the scores and V up to NSV blocks ahead of the P.V products;
+    // one thread polls both rings, so a V stage that frees late never holds
+    // back the next K copy, and the next item's copies start as soon as the
+    // rings have room.
+    for (int it = 0; !bad; ++it) {
+      const int slot = it & 1;
+      if (it >= 2 && !wait_all(bar_itemempty + 8 * slot, ((it >> 1) - 1) & 1)) {
+        bad = true;
+        break;
+      }
+      int w = 0;
+      if (lane == 0) w = atomicAdd(a.tc_ctr, 1);
+      w = __shfl_sync(kFull, w, 0);
+      TcItem& item = items[slot];
+      int* tab = tables + slot * S::kMaxPages;
+      if (w >= n_items) {
+        if (lane == 0) {
+          item.nb = -1;
+          mbar_arrive(bar_itemfull + 8 * slot);
         }
-        mbar_arrive_expect_tx(bar, bytes);
-        const uint32_t st = (is_v ? sv : sk) + s * S::kKV;
-        const CUtensorMap* map = is_v ? &tmap_v : &tmap_k;
+        break;
+      }
+      const int2 e = a.tc_items[w / a.num_kv_heads];
+      TcItem d;
+      d.kvh = w % a.num_kv_heads;
+      d.b = e.x;
+      d.z = e.y & 0xffff;
+      const int tile = e.y >> 16;
+      int ctx, q0, nq;
+      multi_seq(a, d.b, ctx, q0, nq, false);  // the plan kernel listed valid sequences only
+      d.q0 = q0;
+      d.R = nq * G;
+      d.r0 = tile * S::kRows;
+      d.base = ctx - nq;
+      const int p_hi = d.base + (min(d.R, d.r0 + S::kRows) - 1) / G;
+      d.direct = ctx <= a.partition;
+      d.tok0 = d.z * a.partition;
+      d.tok1 = min(min(ctx, d.tok0 + a.partition), p_hi + 1);
+      d.nblk = d.tok1 > d.tok0 ? (d.tok1 - d.tok0 + kBlockSize - 1) / kBlockSize : 0;  // <= kMaxPages
+      d.nb = (d.nblk + S::kPages - 1) / S::kPages;
+      const int pg0 = d.tok0 / kBlockSize;
+      for (int j = lane; j < d.nblk; j += 32) {
+        const int t = a.block_tables[static_cast<long long>(d.b) * a.bt_stride + pg0 + j];
+        const bool in = t >= 0 && t < a.num_blocks;
+        if (!in) raise_error(PKV_ERR_BLOCK_RANGE);
+        tab[j] = in ? t : -1;
+      }
+      __threadfence_block();
+      __syncwarp();
+      if (lane == 0) {
+        item = d;
+        mbar_arrive(bar_itemfull + 8 * slot);  // release: the table and the description
+        auto issue = [&](bool is_v, int c) {
+          const int g = (is_v ? issued_v : issued_k);
+          const int s = g % (is_v ? NSV : NSK);
+          constexpr uint32_t kPageBytes = F8 ? kBlockSize * D : kBlockSize * D * 2;
+          uint32_t bytes = 0;
 #pragma unroll
-        for (int p = 0; p < S::kPages; ++p) {
-          const int i = c * S::kPages + p;
-          if (!loaded(i)) continue;
-          const int y = (table[i] * a.num_kv_heads + kvh) * kBlockSize;
-          if constexpr (F8) {
-            tma_load_2d(st + S::kKV / 2 + p * kPageBytes, map, 0, y, bar);  // one box of 16 rows x D codes
+          for (int p = 0; p < S::kPages; ++p)
+            if (loaded_in(d, tab, c * S::kPages + p)) bytes += kPageBytes;
+          const uint32_t bar = (is_v ? bar_vfull : bar_kfull) + 8 * s;
+          if (bytes == 0) {
+            mbar_arrive(bar);
+            return;
+          }
+          mbar_arrive_expect_tx(bar, bytes);
+          const uint32_t st = (is_v ? sv : sk) + s * S::kKV;
+          const CUtensorMap* map = is_v ? &tmap_v : &tmap_k;
+#pragma unroll
+          for (int p = 0; p < S::kPages; ++p) {
+            const int i = c * S::kPages + p;
+            if (!loaded_in(d, tab, i)) continue;
+            const int y = (tab[i] * a.num_kv_heads + d.kvh) * kBlockSize;
+            if constexpr (F8) {
+              tma_load_2d(st + S::kKV / 2 + p * kPageBytes, map, 0, y, bar);  // one box of 16 rows x D codes
+            } else {
+#pragma unroll
+              for (int bx = 0; bx < S::kPanels; ++bx)
+                tma_load_2d(st + bx * S::kKVPanel + p * 2048, map, bx * 64, y, bar);
+            }
+          }
+        };
+        int ck = 0, cv = 0;  // this item's blocks issued
+        long long t0 = clock64();
+        while (ck < d.nb || cv < d.nb) {
+          bool moved = false;
+          if (ck < d.nb && (issued_k < NSK || mbar_test(bar_kempty + 8 * (issued_k % NSK),
+                                                        ((issued_k / NSK) - 1) & 1))) {
+            issue(false, ck++);
+            ++issued_k;
+            moved = true;
+          }
+          if (cv < d.nb && (issued_v < NSV || mbar_test(bar_vempty + 8 * (issued_v % NSV),
+                                                        ((issued_v / NSV) - 1) & 1))) {
+            issue(true, cv++);
+            ++issued_v;
+            moved = true;
+          }
+          if (moved) {
+            t0 = clock64();
+          } else if (clock64() - t0 > (1ll << 32)) {
+            raise_error(PKV_ERR_TIMEOUT);
+            bad = true;
+            break;
           } else {
-#pragma unroll
-            for (int bx = 0; bx < S::kPanels; ++bx)
-              tma_load_2d(st + bx * S::kKVPanel + p * 2048, map, bx * 64, y, bar);
+            __nanosleep(32);
           }
         }
-      };
-      long long t0 = clock64();
-      while (issued < nb || issued_v < nb) {
-        bool moved = false;
-        if (issued < nb &&
-            (issued < NSK || mbar_test(bar_kempty + 8 * (issued % NSK), ((issued / NSK) - 1) & 1))) {
-          issue(false, issued);
-          TC_TRACE(issued, 0);
-          if (issued == 0) TC_CTA(1, tc_gtime());
-          ++issued;
-          moved = true;
-        }
-        if (issued_v < nb &&
-            (issued_v < NSV || mbar_test(bar_vempty + 8 * (issued_v % NSV), ((issued_v / NSV) - 1) & 1))) {
-          issue(true, issued_v);
-          TC_TRACE(issued_v, 1);
-          ++issued_v;
-          moved = true;
-        }
-        if (moved) {
-          t0 = clock64();
-        } else if (clock64() - t0 > (1ll << 32)) {
-          raise_error(PKV_ERR_TIMEOUT);
-          bad = true;
-          break;
-        } else {
-          __nanosleep(32);
-        }
       }
+      bad = __shfl_sync(kFull, bad, 0);
     }
   } else if (warp == 1) {
     // ---- MMA issuer (lane 0); V-row zeroing, or the widening of FP8 codes,
     // by the whole warp ---------------------------------------------------
     constexpr uint32_t kIdQK = tc_idesc<TM>(128, S::kKeys, false);
     constexpr uint32_t kIdPV = tc_idesc<TM>(128, D, true);
-    auto wait_all = [&](uint32_t bar, uint32_t parity) { return __all_sync(kFull, mbar_wait_bounded(bar, parity)); };
-    // keys of block c that are there (inside the partition and the context,
-    // on pages the table names): bit r for key r
-    auto valid_keys = [&](int c) -> uint64_t {
-      const int lim = tok1 - (tok0 + c * S::kKeys);
-      uint64_t m = lim >= S::kKeys ? ~0ull : (lim > 0 ? (1ull << lim) - 1ull : 0ull);
+    int g0 = 0;  // key blocks of the items before this one
+    for (int it = 0; !bad; ++it) {
+      const int slot = it & 1;
+      if (!wait_all(bar_itemfull + 8 * slot, (it >> 1) & 1)) {
+        bad = true;
+        break;
+      }
+      const TcItem& d = items[slot];
+      if (d.nb < 0) break;
+      const int* tab = tables + slot * S::kMaxPages;
+      // keys of block c that are there (inside the partition and the
+      // context, on pages the table names): bit r for key r
+      auto valid_keys = [&](int c) -> uint64_t {
+        const int lim = d.tok1 - (d.tok0 + c * S::kKeys);
+        uint64_t m = lim >= S::kKeys ? ~0ull : (lim > 0 ? (1ull << lim) - 1ull : 0ull);
 #pragma unroll
-      for (int p = 0; p < S::kPages; ++p)
-        if (!loaded(c * S::kPages + p)) m &= ~(0xFFFFull << (16 * p));
-      return m;
-    };
-    auto pv = [&](int j) -> bool {
-      const int s = j % NSV;
-      if constexpr (F8) {
-        // the block's V codes widened while its softmax runs
-        if (!wait_all(bar_vfull + 8 * s, (j / NSV) & 1)) return false;
-        tc_widen_fp8<D, NSK, NSV>(smem + S::kOffV + s * S::kKV, valid_keys(j), lane);
-        fence_proxy_async_smem();
-        if (!wait_all(bar_pfull + 8 * (j & 1), (j >> 1) & 1)) return false;
-        if (lane == 0) TC_TRACE(j, 4);
-      } else {
-        if (!wait_all(bar_pfull + 8 * (j & 1), (j >> 1) & 1)) return false;
-        if (lane == 0) TC_TRACE(j, 4);
-        if (!wait_all(bar_vfull + 8 * s, (j / NSV) & 1)) return false;
-        // zero the V rows of keys that are not there (past the context or on
-        // pages the table does not name): a zero weight must not meet a NaN
-        const uint32_t vst_off = static_cast<uint32_t>(S::kOffV) + s * S::kKV;
-        bool zeroed = false;
+        for (int p = 0; p < S::kPages; ++p)
+          if (!loaded_in(d, tab, c * S::kPages + p)) m &= ~(0xFFFFull << (16 * p));
+        return m;
+      };
+      // O still holds the previous item's result until its epilogue has read
+      // it: the first P.V of this item (or the end of an item without keys)
+      // waits for that
+      bool o_free = it == 0;
+      auto free_o = [&]() -> bool {
+        if (o_free) return true;
+        o_free = true;
+        return wait_all(bar_oempty, (it - 1) & 1);
+      };
+      auto pv = [&](int j) -> bool {
+        const int g = g0 + j;
+        const int s = g % NSV;
+        if constexpr (F8) {
+          // the block's V codes widened while its softmax runs
+          if (!wait_all(bar_vfull + 8 * s, (g / NSV) & 1)) return false;
+          tc_widen_fp8<D, NSK, NSV>(smem + S::kOffV + s * S::kKV, valid_keys(j), lane);
+          fence_proxy_async_smem();
+          if (!wait_all(bar_pfull + 8 * (g & 1), (g >> 1) & 1)) return false;
+        } else {
+          if (!wait_all(bar_pfull + 8 * (g & 1), (g >> 1) & 1)) return false;
+          if (!wait_all(bar_vfull + 8 * s, (g / NSV) & 1)) return false;
+          // zero the V rows of keys that are not there (past the context or
+          // on pages the table does not name): a zero weight must not meet
+          // a NaN
+          const uint32_t vst_off = static_cast<uint32_t>(S::kOffV) + s * S::kKV;
+          bool zeroed = false;
 #pragma unroll
-        for (int p = 0; p < S::kPages; ++p) {
-          const int i = j * S::kPages + p;
-          const int page_tok = tok0 + i * kBlockSize;
-          const int first = loaded(i) ? max(0, min(kBlockSize, tok1 - page_tok)) : 0;
-          if (first >= kBlockSize) continue;
-          zeroed = true;
-          const int n = (kBlockSize - first) * S::kPanels * 8;  // 16-byte chunks
-          for (int e = lane; e < n; e += 32) {
-            const int row = first + e / (S::kPanels * 8);
-            const int pn = (e / 8) % S::kPanels;
-            *reinterpret_cast<uint4*>(smem + vst_off + pn * S::kKVPanel + (p * kBlockSize + row) * 128 + (e & 7) * 16) =
-                make_uint4(0u, 0u, 0u, 0u);
+          for (int p = 0; p < S::kPages; ++p) {
+            const int i = j * S::kPages + p;
+            const int page_tok = d.tok0 + i * kBlockSize;
+            const int first = loaded_in(d, tab, i) ? max(0, min(kBlockSize, d.tok1 - page_tok)) : 0;
+            if (first >= kBlockSize) continue;
+            zeroed = true;
+            const int n = (kBlockSize - first) * S::kPanels * 8;  // 16-byte chunks
+            for (int e = lane; e < n; e += 32) {
+              const int row = first + e / (S::kPanels * 8);
+              const int pn = (e / 8) % S::kPanels;
+              *reinterpret_cast<uint4*>(smem + vst_off + pn * S::kKVPanel + (p * kBlockSize + row) * 128 +
+                                        (e & 7) * 16) = make_uint4(0u, 0u, 0u, 0u);
+            }
           }
+          if (zeroed) fence_proxy_async_smem();
         }
-        if (zeroed) fence_proxy_async_smem();
-      }
-      __syncwarp();
-      tc_fence_after();
-      if (lane == 0) {
-        const uint32_t vst = sv + s * S::kKV;
-        const uint32_t pcol = tmem + S::kColS + 64 * (j & 1);
-#pragma unroll
-        for (int kk = 0; kk < S::kKeys / 16; ++kk) {
-          const uint64_t vd = sw128_desc(vst + kk * 2048, S::kKVPanel, 1024);
-          tc_mma_ts(tmem + S::kColO, pcol + 8 * kk, vd, kIdPV, (j > 0 || kk > 0) ? 1u : 0u);  // P hi
-#ifndef PKV_TC_NO_LO
-          tc_mma_ts(tmem + S::kColO, pcol + 32 + 8 * kk, vd, kIdPV, 1u);                       // P lo
-#endif
-        }
-        tc_commit(bar_vempty + 8 * s);  // the block's V may be overwritten
-        tc_commit(bar_pvdone);
-        TC_TRACE(j, 5);
-      }
-      __syncwarp();
-      return true;
-    };
-    if (!wait_all(bar_qfull, 0)) bad = true;
-    for (int c = 0; c < nb && !bad; ++c) {
-      const int s = c % NSK;
-      if (!wait_all(bar_kfull + 8 * s, (c / NSK) & 1)) {
-        bad = true;
-        break;
-      }
-      if (lane == 0) TC_TRACE(c, 2);
-      if constexpr (F8) {
-        tc_widen_fp8<D, NSK, NSV>(smem + S::kOffK + s * S::kKV, valid_keys(c), lane);
-        fence_proxy_async_smem();
+        if (j == 0 && !free_o()) return false;
         __syncwarp();
-      }
-      // S buffer c & 1 was last read (as P) by the P.V of block c - 2
-      if (c >= 2 && !wait_all(bar_pvdone, (c - 2) & 1)) {
+        tc_fence_after();
+        if (lane == 0) {
+          const uint32_t vst = sv + s * S::kKV;
+          const uint32_t pcol = tmem + S::kColS + 64 * (g & 1);
+#pragma unroll
+          for (int kk = 0; kk < S::kKeys / 16; ++kk) {
+            const uint64_t vd = sw128_desc(vst + kk * 2048, S::kKVPanel, 1024);
+            tc_mma_ts(tmem + S::kColO, pcol + 8 * kk, vd, kIdPV, (j > 0 || kk > 0) ? 1u : 0u);  // P hi
+#ifndef PKV_TC_NO_LO
+            tc_mma_ts(tmem + S::kColO, pcol + 32 + 8 * kk, vd, kIdPV, 1u);                       // P lo
+#endif
+          }
+          tc_commit(bar_vempty + 8 * s);  // the block's V may be overwritten
+          tc_commit(bar_pvdone);
+        }
+        __syncwarp();
+        return true;
+      };
+      if (!wait_all(bar_qfull, it & 1)) {
         bad = true;
         break;
       }
-      tc_fence_after();
-      if (lane == 0) {
-        const uint32_t kst = sk + s * S::kKV;
-#pragma unroll
-        for (int ks = 0; ks < D / 16; ++ks) {
-          const uint64_t qd = sw128_desc(sq + (ks >> 2) * S::kQPanel + (ks & 3) * 32, 16, 1024);
-          const uint64_t kd = sw128_desc(kst + (ks >> 2) * S::kKVPanel + (ks & 3) * 32, 16, 1024);
-          tc_mma_ss(tmem + S::kColS + 64 * (c & 1), qd, kd, kIdQK, ks > 0 ? 1u : 0u);
+      for (int c = 0; c < d.nb && !bad; ++c) {
+        const int g = g0 + c;
+        const int s = g % NSK;
+        if (!wait_all(bar_kfull + 8 * s, (g / NSK) & 1)) {
+          bad = true;
+          break;
         }
-        tc_commit(bar_kempty + 8 * s);  // the block's K may be overwritten
-        tc_commit(bar_sfull + 8 * (c & 1));
-        TC_TRACE(c, 3);
+        if constexpr (F8) {
+          tc_widen_fp8<D, NSK, NSV>(smem + S::kOffK + s * S::kKV, valid_keys(c), lane);
+          fence_proxy_async_smem();
+          __syncwarp();
+        }
+        // S buffer g & 1 was last read (as P) by the P.V of block g - 2.
+        // Inside an item that is the latest P.V issued; at an item's first
+        // block the previous item's last P.V (g - 1) is issued too, so that
+        // one is waited for (a phase wait must name the newest phase that
+        // can have completed)
+        const int last_pv = c == 0 ? g - 1 : g - 2;
+        if (last_pv >= 0 && !wait_all(bar_pvdone, last_pv & 1)) {
+          bad = true;
+          break;
+        }
+        tc_fence_after();
+        if (lane == 0) {
+          const uint32_t kst = sk + s * S::kKV;
+#pragma unroll
+          for (int ks = 0; ks < D / 16; ++ks) {
+            const uint64_t qd = sw128_desc(sq + (ks >> 2) * S::kQPanel + (ks & 3) * 32, 16, 1024);
+            const uint64_t kd = sw128_desc(kst + (ks >> 2) * S::kKVPanel + (ks & 3) * 32, 16, 1024);
+            tc_mma_ss(tmem + S::kColS + 64 * (g & 1), qd, kd, kIdQK, ks > 0 ? 1u : 0u);
+          }
+          tc_commit(bar_kempty + 8 * s);  // the block's K may be overwritten
+          tc_commit(bar_sfull + 8 * (g & 1));
+          if (c == d.nb - 1) tc_commit(bar_qempty);  // the item's Q tile is no longer read
+        }
+        __syncwarp();
+        if (c >= 1 && !pv(c - 1)) {
+          bad = true;
+          break;
+        }
+      }
+      if (bad) break;
+      if (d.nb > 0) {
+        if (!pv(d.nb - 1)) {
+          bad = true;
+          break;
+        }
+      } else {
+        if (lane == 0) tc_commit(bar_qempty);
+        if (!free_o()) {
+          bad = true;
+          break;
+        }
+      }
+      // the item's result is complete once its last P.V is (one phase per
+      // item, so no parity ambiguity)
+      g0 += d.nb;  // (read before the slot is released)
+      __syncwarp();
+      if (lane == 0) {
+        tc_commit(bar_final);
+        mbar_arrive(bar_itemempty + 8 * slot);
       }
       __syncwarp();
-      if (c >= 1 && !pv(c - 1)) {
-        bad = true;
-        break;
-      }
     }
-    if (!bad && !pv(nb - 1)) bad = true;
     if (bad && lane == 0) raise_error(PKV_ERR_TIMEOUT);
     // every MMA this thread issued completes before the tensor memory goes
-    if (lane == 0) tc_commit(bar_final);
+    if (lane == 0) tc_commit(bar_drain);
     __syncwarp();
-    mbar_wait_bounded(bar_final, 0);
+    mbar_wait_bounded(bar_drain, 0);
   } else {
-    // the row's logit multiplier (log2 units; over an FP8 pool it carries
-    // the K scale and, for bf16 queries, the row's power-of-two rescale)
-    float qmul = a.qk_scale;
-    {
-      // this thread's row of Q into the 128-byte-swizzled K-major tile
-      // (rows past the batch are zeros), while the first copies fly
-      const int r = 32 * (warp & 3) + lane;
-      const int tr = r0 + r;
-      const uint4* src = tr < R ? reinterpret_cast<const uint4*>(reinterpret_cast<const T*>(a.q) + out_row(tr) * D)
-                                : nullptr;
-      uint4 qv[D / 8];
-#pragma unroll
-      for (int c = 0; c < D / 8; ++c) qv[c] = src ? src[c] : make_uint4(0u, 0u, 0u, 0u);
+    // ---- softmax (one thread per row) and epilogue ----------------------------
+    const int r = 32 * (warp & 3) + lane;
+    const uint32_t lane_off = static_cast<uint32_t>(32 * (warp & 3)) << 16;
+    // this thread's row of the item's Q into the 128-byte-swizzled K-major
+    // tile (rows past the item's are zeros); returns the row's logit
+    // multiplier (log2 units; over an FP8 pool it carries the K scale and,
+    // for bf16 queries, the row's power-of-two rescale)
+    auto load_q = [&](const TcItem& d) -> float {
+      float qmul = a.qk_scale;
+      const int tr = d.r0 + r;
+      const uint4* src =
+          tr < d.R ? reinterpret_cast<const uint4*>(reinterpret_cast<const T*>(a.q) +
+                                                    (static_cast<size_t>(d.q0 + tr / G) * a.num_q_heads +
+                                                     d.kvh * G + tr % G) * D)
+                   : nullptr;
+      // (8 chunks of 16 bytes at a time: the row is live next to the
+      // current item's softmax state)
+      float sc = 1.f;
       if constexpr (F8 && !std::is_same<T, __half>::value) {
         // bf16 row -> fp16 times 2^kq, kq putting the row's largest
         // magnitude just under 2^15 (exact unless an element falls below
         // fp16's normal range); the logits take 2^-kq back
         float mx = 0.f;
+        if (src) {
+#pragma unroll 4
+          for (int c = 0; c < D / 8; ++c) {
+            const uint4 u = src[c];
+            const uint32_t w[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
-        for (int c = 0; c < D / 8; ++c) {
-          const uint32_t w[4] = {qv[c].x, qv[c].y, qv[c].z, qv[c].w};
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const float2 f = Mma<T>::unpack(w[e]);
-            mx = fmax3(mx, fabsf(f.x), fabsf(f.y));
+            for (int e = 0; e < 4; ++e) {
+              const float2 f = Mma<T>::unpack(w[e]);
+              mx = fmax3(mx, fabsf(f.x), fabsf(f.y));
+            }
           }
         }
         const int ex = static_cast<int>((__float_as_uint(mx) >> 23) & 0xffu) - 127;
         const int kq = mx > 0.f ? min(max(14 - ex, -126), 126) : 0;
-        const float sc = __uint_as_float(static_cast<uint32_t>(kq + 127) << 23);
+        sc = __uint_as_float(static_cast<uint32_t>(kq + 127) << 23);
         qmul *= __uint_as_float(static_cast<uint32_t>(127 - kq) << 23);
-#pragma unroll
-        for (int c = 0; c < D / 8; ++c) {
-          uint32_t w[4] = {qv[c].x, qv[c].y, qv[c].z, qv[c].w};
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const float2 f = Mma<T>::unpack(w[e]);
-            w[e] = Mma<__half>::pack(f.x * sc, f.y * sc);
-          }
-          qv[c] = make_uint4(w[0], w[1], w[2], w[3]);
-        }
       }
 #pragma unroll
-      for (int c = 0; c < D / 8; ++c)
-        *reinterpret_cast<uint4*>(smem + (c >> 3) * S::kQPanel + r * 128 + (((c & 7) ^ (r & 7)) << 4)) = qv[c];
+      for (int h = 0; h < D / 64; ++h) {
+        uint4 qv[8];
+#pragma unroll
+        for (int c = 0; c < 8; ++c) qv[c] = src ? src[8 * h + c] : make_uint4(0u, 0u, 0u, 0u);
+        if constexpr (F8 && !std::is_same<T, __half>::value) {
+#pragma unroll
+          for (int c = 0; c < 8; ++c) {
+            uint32_t w[4] = {qv[c].x, qv[c].y, qv[c].z, qv[c].w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const float2 f = Mma<T>::unpack(w[e]);
+              w[e] = Mma<__half>::pack(f.x * sc, f.y * sc);
+            }
+            qv[c] = make_uint4(w[0], w[1], w[2], w[3]);
+          }
+        }
+#pragma unroll
+        for (int c = 0; c < 8; ++c)
+          *reinterpret_cast<uint4*>(smem + h * S::kQPanel + r * 128 + ((c ^ (r & 7)) << 4)) = qv[c];
+      }
       fence_proxy_async_smem();  // the tensor core reads the tile through the async proxy
       __syncwarp();
       if (lane == 0) mbar_arrive(bar_qfull);
-    }
-    // ---- softmax (one thread per row) and epilogue ----------------------------
-    const int r = 32 * (warp & 3) + lane;
-    const uint32_t lane_off = static_cast<uint32_t>(32 * (warp & 3)) << 16;
-    const int tr = r0 + r;
-    const bool valid = tr < R;
-    const int pos = valid ? base + tr / G : -1;
-    float m_ref = -INFINITY, l = 0.f;
-    // a warp whose 32 rows are all padding (a tile of <= 96 rows) keeps
-    // step with the others but computes nothing: its rows of P and O are
-    // never read back
-    const bool warp_pad = r0 + 32 * (warp & 3) >= R;
-    auto wait_all = [&](uint32_t bar, uint32_t parity) { return __all_sync(kFull, mbar_wait_bounded(bar, parity)); };
-    for (int j = 0; j < nb; ++j) {
-      // the block's key limits need no scores: keys kb0 + e with e <= lim
-      // are causal for this row and inside the partition and the context
-      const int kb0 = tok0 + j * S::kKeys;
-      uint32_t pages_ok = 0;
+      return qmul;
+    };
+
+    int g0 = 0;  // key blocks of the items before this one
+    if (!wait_all(bar_itemfull, 0)) bad = true;  // item 0 sits in slot 0
+    float qmul = 0.f;
+    if (!bad && items[0].nb >= 0) qmul = load_q(items[0]);
+    // the item descriptions are read in shared memory, where they stay
+    // until this warp releases the slot
+    for (int it = 0; !bad && items[it & 1].nb >= 0; ++it) {
+      const int slot = it & 1;
+      const TcItem& d = items[slot];
+      const int* tab = tables + slot * S::kMaxPages;
+      const int tr = d.r0 + r;
+      const bool valid = tr < d.R;
+      const int pos = valid ? d.base + tr / G : -1;
+      float m_ref = -INFINITY, l = 0.f;
+      // a warp whose 32 rows are all padding (a tile of <= 96 rows) keeps
+      // step with the others but computes nothing: its rows of P and O are
+      // never read back
+      const bool warp_pad = d.r0 + 32 * (warp & 3) >= d.R;
+      for (int j = 0; j < d.nb; ++j) {
+        const int g = g0 + j;
+        // the block's key limits need no scores: keys kb0 + e with e <= lim
+        // are causal for this row and inside the partition and the context
+        const int kb0 = d.tok0 + j * S::kKeys;
+        uint32_t pages_ok = 0;
 #pragma unroll
-      for (int p = 0; p < S::kPages; ++p) pages_ok |= loaded(j * S::kPages + p) ? (1u << p) : 0u;
-      const int lim = min(pos, tok1 - 1) - kb0;
-      // plain block: every key in, and a positive scale, so the max can be
-      // taken on the raw scores and the scale folded into the exponent
-      const bool plain = __all_sync(kFull, lim >= S::kKeys - 1 && pages_ok == 0xFu && qmul > 0.f);
-      if (!wait_all(bar_sfull + 8 * (j & 1), (j >> 1) & 1)) {
-        bad = true;
-        break;
-      }
-      if (warp == 4 && lane == 0) TC_TRACE(j, 6);
-      tc_fence_after();
-      if (warp_pad) {
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(bar_pfull + 8 * (j & 1));
-        continue;
-      }
-      const uint32_t scol = tmem + lane_off + S::kColS + 64 * (j & 1);
-      uint32_t v[S::kKeys];
-      if (warp == 4 && lane == 0) TC_TRACE(j, 10);
-      tmem_ld64(scol, v);
-      if (warp == 4 && lane == 0) TC_TRACE(j, 11);
-      float x[S::kKeys];
-      float mul = qmul;  // x * mul is the score in log2 units
-      if (plain) {
-#pragma unroll
-        for (int k = 0; k < S::kKeys; ++k) x[k] = __uint_as_float(v[k]);
-      } else {
-        // masked keys to -inf, the scale applied here
-#pragma unroll
-        for (int k = 0; k < S::kKeys; ++k) {
-          const bool ok = k <= lim && ((pages_ok >> (k >> 4)) & 1u);
-          x[k] = ok ? __uint_as_float(v[k]) * qmul : -INFINITY;
-        }
-        mul = 1.f;
-      }
-      if (warp == 4 && lane == 0) TC_TRACE(j, 7);
-      // block max: a tree of three-input maxima
-      float t[S::kKeys / 4];
-#pragma unroll
-      for (int k = 0; k < S::kKeys / 4; ++k) t[k] = fmax3(x[4 * k], x[4 * k + 1], fmaxf(x[4 * k + 2], x[4 * k + 3]));
-#pragma unroll
-      for (int w = S::kKeys / 4; w > 1; w /= 2)
-#pragma unroll
-        for (int k = 0; k < w / 2; ++k) t[k] = fmaxf(t[k], t[k + w / 2]);
-      const float bm = t[0] * mul;
-      // move the reference max only when this block exceeds it by 2^8
-      float alpha = 1.f;
-      bool rescale = false;
-      if (bm > m_ref + 8.f) {
-        alpha = exp2_sfu(m_ref - bm);  // 0 while no key was seen
-        rescale = m_ref != -INFINITY && j > 0;
-        l *= alpha;
-        m_ref = bm;
-      }
-      // 2^(x mul - m) as one FFMA leaves the residual of the rounded max
-      // product, up to half an ulp of m: harmless while |m| < 2^20 (under
-      // 2^-4); past that the scores are rounded to their products first,
-      // so the maximal one gives exactly 2^0
-      if (__any_sync(kFull, fabsf(m_ref) >= 1048576.f && mul != 1.f)) {
-#pragma unroll
-        for (int k = 0; k < S::kKeys; ++k) x[k] *= mul;
-        mul = 1.f;
-      }
-      const float nmr = m_ref == -INFINITY ? 0.f : -m_ref;
-      uint32_t ph[S::kKeys / 2], pl[S::kKeys / 2];
-      float acc[8];
-#pragma unroll
-      for (int i = 0; i < 8; ++i) acc[i] = 0.f;
-#pragma unroll
-      for (int k = 0; k < S::kKeys; k += 2) {
-        const float p0 = exp2_sfu(fmaf(x[k], mul, nmr)), p1 = exp2_sfu(fmaf(x[k + 1], mul, nmr));
-        acc[(k / 2) & 7] += p0 + p1;
-        ph[k / 2] = M::pack(p0, p1);
-        const float2 hv = M::unpack(ph[k / 2]);
-        pl[k / 2] = M::pack(p0 - hv.x, p1 - hv.y);
-      }
-      const float sum = ((acc[0] + acc[1]) + (acc[2] + acc[3])) + ((acc[4] + acc[5]) + (acc[6] + acc[7]));
-      l += sum;
-      if (__any_sync(kFull, rescale)) {
-        // O holds the P.V of blocks < j: wait for the last of them, then
-        // rescale this thread's row in tensor memory
-        if (!wait_all(bar_pvdone, (j - 1) & 1)) {
+        for (int p = 0; p < S::kPages; ++p) pages_ok |= loaded_in(d, tab, j * S::kPages + p) ? (1u << p) : 0u;
+        const int lim = min(pos, d.tok1 - 1) - kb0;
+        // plain block: every key in, and a positive scale, so the max can be
+        // taken on the raw scores and the scale folded into the exponent
+        const bool plain = __all_sync(kFull, lim >= S::kKeys - 1 && pages_ok == 0xFu && qmul > 0.f);
+        if (!wait_all(bar_sfull + 8 * (g & 1), (g >> 1) & 1)) {
           bad = true;
           break;
         }
         tc_fence_after();
-        const float f = rescale ? alpha : 1.f;
+        if (warp_pad) {
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(bar_pfull + 8 * (g & 1));
+          continue;
+        }
+        const uint32_t scol = tmem + lane_off + S::kColS + 64 * (g & 1);
+        uint32_t v[S::kKeys];
+        tmem_ld64(scol, v);
+        float x[S::kKeys];
+        float mul = qmul;  // x * mul is the score in log2 units
+        if (plain) {
+#pragma unroll
+          for (int k = 0; k < S::kKeys; ++k) x[k] = __uint_as_float(v[k]);
+        } else {
+          // masked keys to -inf, the scale applied here
+#pragma unroll
+          for (int k = 0; k < S::kKeys; ++k) {
+            const bool ok = k <= lim && ((pages_ok >> (k >> 4)) & 1u);
+            x[k] = ok ? __uint_as_float(v[k]) * qmul : -INFINITY;
+          }
+          mul = 1.f;
+        }
+        // block max: a tree of three-input maxima
+        float t[S::kKeys / 4];
+#pragma unroll
+        for (int k = 0; k < S::kKeys / 4; ++k) t[k] = fmax3(x[4 * k], x[4 * k + 1], fmaxf(x[4 * k + 2], x[4 * k + 3]));
+#pragma unroll
+        for (int w = S::kKeys / 4; w > 1; w /= 2)
+#pragma unroll
+          for (int k = 0; k < w / 2; ++k) t[k] = fmaxf(t[k], t[k + w / 2]);
+        const float bm = t[0] * mul;
+        // move the reference max only when this block exceeds it by 2^8
+        float alpha = 1.f;
+        bool rescale = false;
+        if (bm > m_ref + 8.f) {
+          alpha = exp2_sfu(m_ref - bm);  // 0 while no key was seen
+          rescale = m_ref != -INFINITY && j > 0;
+          l *= alpha;
+          m_ref = bm;
+        }
+        // 2^(x mul - m) as one FFMA leaves the residual of the rounded max
+        // product, up to half an ulp of m: harmless while |m| < 2^20 (under
+        // 2^-4); past that the scores are rounded to their products first,
+        // so the maximal one gives exactly 2^0
+        if (__any_sync(kFull, fabsf(m_ref) >= 1048576.f && mul != 1.f)) {
+#pragma unroll
+          for (int k = 0; k < S::kKeys; ++k) x[k] *= mul;
+          mul = 1.f;
+        }
+        const float nmr = m_ref == -INFINITY ? 0.f : -m_ref;
+        uint32_t ph[S::kKeys / 2], pl[S::kKeys / 2];
+        float acc[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) acc[i] = 0.f;
+#pragma unroll
+        for (int k = 0; k < S::kKeys; k += 2) {
+          const float p0 = exp2_sfu(fmaf(x[k], mul, nmr)), p1 = exp2_sfu(fmaf(x[k + 1], mul, nmr));
+          acc[(k / 2) & 7] += p0 + p1;
+          ph[k / 2] = M::pack(p0, p1);
+          const float2 hv = M::unpack(ph[k / 2]);
+          pl[k / 2] = M::pack(p0 - hv.x, p1 - hv.y);
+        }
+        const float sum = ((acc[0] + acc[1]) + (acc[2] + acc[3])) + ((acc[4] + acc[5]) + (acc[6] + acc[7]));
+        l += sum;
+        if (__any_sync(kFull, rescale)) {
+          // O holds the P.V of blocks < j: wait for the last of them, then
+          // rescale this thread's row in tensor memory
+          if (!wait_all(bar_pvdone, (g - 1) & 1)) {
+            bad = true;
+            break;
+          }
+          tc_fence_after();
+          const float f = rescale ? alpha : 1.f;
+#pragma unroll
+          for (int h = 0; h < D / 32; ++h) {
+            uint32_t o[32];
+            tmem_ld32(tmem + lane_off + S::kColO + 32 * h, o);
+#pragma unroll
+            for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * f);
+            tmem_st32(tmem + lane_off + S::kColO + 32 * h, o);
+          }
+        }
+        tmem_st32(scol, ph);
+        tmem_st32(scol + 32, pl);
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar_pfull + 8 * (g & 1));
+      }
+      if (bad) break;
+      // the next item's Q goes in while this item's last P.V runs
+      const int nslot = (it + 1) & 1;
+      if (!wait_all(bar_itemfull + 8 * nslot, ((it + 1) >> 1) & 1)) {
+        bad = true;
+        break;
+      }
+      const TcItem& nd = items[nslot];
+      float nqmul = 0.f;
+      if (nd.nb >= 0) {
+        if (!wait_all(bar_qempty, it & 1)) {
+          bad = true;
+          break;
+        }
+        nqmul = load_q(nd);
+      }
+      // epilogue: the item's MMAs done (its final commit follows its last
+      // P.V), then each row out of tensor memory
+      if (!wait_all(bar_final, it & 1)) {
+        bad = true;
+        break;
+      }
+      if (!warp_pad) {
+        tc_fence_after();
+        const bool has = valid && pos >= d.tok0;
+        const size_t row = valid ? static_cast<size_t>(d.q0 + tr / G) * a.num_q_heads + d.kvh * G + tr % G : 0;
+        // over an FP8 pool the V scale multiplies the output (or the
+        // partial: the merge is linear in it)
+        const float osc = F8 ? a.v_scale : 1.f;
+        const float inv = has ? osc / l : 0.f;
 #pragma unroll
         for (int h = 0; h < D / 32; ++h) {
-          uint32_t v[32];
-          tmem_ld32(tmem + lane_off + S::kColO + 32 * h, v);
+          uint32_t o[32];
+          tmem_ld32(tmem + lane_off + S::kColO + 32 * h, o);
+          if (!valid) continue;
+          if (d.direct) {
+            uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<T*>(a.out) + row * D + 32 * h);
 #pragma unroll
-          for (int e = 0; e < 32; ++e) v[e] = __float_as_uint(__uint_as_float(v[e]) * f);
-          tmem_st32(tmem + lane_off + S::kColO + 32 * h, v);
+            for (int q = 0; q < 4; ++q) {
+              uint32_t w[4];
+#pragma unroll
+              for (int e = 0; e < 4; ++e)
+                w[e] = has ? Mma<T>::pack(__uint_as_float(o[8 * q + 2 * e]) * inv,
+                                          __uint_as_float(o[8 * q + 2 * e + 1]) * inv)
+                           : 0u;
+              dst[q] = make_uint4(w[0], w[1], w[2], w[3]);
+            }
+          } else if (has) {
+            float4* dst = reinterpret_cast<float4*>(a.ws_o + (row * a.num_parts + d.z) * D + 32 * h);
+#pragma unroll
+            for (int q = 0; q < 8; ++q)
+              dst[q] = make_float4(__uint_as_float(o[4 * q]) * osc, __uint_as_float(o[4 * q + 1]) * osc,
+                                   __uint_as_float(o[4 * q + 2]) * osc, __uint_as_float(o[4 * q + 3]) * osc);
+          }
         }
+        if (has && !d.direct) a.ws_ml[row * a.num_parts + d.z] = make_float2(m_ref, l);
       }
-      tmem_st32(scol, ph);
-      tmem_st32(scol + 32, pl);
-      tmem_wait_st();
+      g0 += d.nb;
       tc_fence_before();
       __syncwarp();
-      if (warp == 4 && lane == 0) TC_TRACE(j, 8);
-      if (lane == 0) mbar_arrive(bar_pfull + 8 * (j & 1));
-    }
-    // epilogue: every MMA done (the issuer's final commit follows the last
-    // P.V; one phase, so no parity ambiguity), then each row out of tensor
-    // memory
-    if (!bad && !wait_all(bar_final, 0)) bad = true;
-    if (bad) {
-      if (lane == 0) raise_error(PKV_ERR_TIMEOUT);
-    } else if (!warp_pad) {
-      tc_fence_after();
-      const bool has = valid && pos >= tok0;
-      const size_t row = valid ? out_row(tr) : 0;
-      // over an FP8 pool the V scale multiplies the output (or the partial:
-      // the merge is linear in it)
-      const float osc = F8 ? a.v_scale : 1.f;
-      const float inv = has ? osc / l : 0.f;
-#pragma unroll
-      for (int h = 0; h < D / 32; ++h) {
-        uint32_t v[32];
-        tmem_ld32(tmem + lane_off + S::kColO + 32 * h, v);
-        if (!valid) continue;
-        if (direct) {
-          uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<T*>(a.out) + row * D + 32 * h);
-#pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            uint32_t w[4];
-#pragma unroll
-            for (int e = 0; e < 4; ++e)
-              w[e] = has ? Mma<T>::pack(__uint_as_float(v[8 * q + 2 * e]) * inv,
-                                        __uint_as_float(v[8 * q + 2 * e + 1]) * inv)
-                         : 0u;
-            dst[q] = make_uint4(w[0], w[1], w[2], w[3]);
-          }
-        } else if (has) {
-          float4* dst = reinterpret_cast<float4*>(a.ws_o + (row * a.num_parts + z) * D + 32 * h);
-#pragma unroll
-          for (int q = 0; q < 8; ++q)
-            dst[q] = make_float4(__uint_as_float(v[4 * q]) * osc, __uint_as_float(v[4 * q + 1]) * osc,
-                                 __uint_as_float(v[4 * q + 2]) * osc, __uint_as_float(v[4 * q + 3]) * osc);
-        }
+      if (lane == 0) {
+        mbar_arrive(bar_oempty);                 // O may be overwritten
+        mbar_arrive(bar_itemempty + 8 * slot);  // the slot may be refilled
       }
-      if (valid && pos >= tok0 && !direct) a.ws_ml[row * a.num_parts + z] = make_float2(m_ref, l);
+      qmul = nqmul;
     }
+    if (bad && lane == 0) raise_error(PKV_ERR_TIMEOUT);
   }
 
   // ---- teardown ---------------------------------------------------------------
@@ -818,17 +982,12 @@ __global__ void __launch_bounds__(TcShape<D, NSK, NSV>::kThreads, PKV_TC_MIN_CTA
   if (any_bad && warp == 0 && lane == 0) {
     // the last block the producer issued into each stage lands before the
     // CTA exits
-    for (int c = max(0, issued - NSK); c < issued; ++c) mbar_wait_bounded(bar_kfull + 8 * (c % NSK), (c / NSK) & 1);
+    for (int c = max(0, issued_k - NSK); c < issued_k; ++c)
+      mbar_wait_bounded(bar_kfull + 8 * (c % NSK), (c / NSK) & 1);
     for (int c = max(0, issued_v - NSV); c < issued_v; ++c)
       mbar_wait_bounded(bar_vfull + 8 * (c % NSV), (c / NSV) & 1);
   }
   if (warp == 1) tmem_dealloc(tmem, S::kTmemCols);
-  if (threadIdx.x == 0) {
-    TC_CTA(2, tc_gtime());
-    unsigned smid_;
-    asm volatile("mov.u32 %0, %%smid;" : "=r"(smid_));
-    TC_CTA(3, static_cast<long long>(smid_) | (static_cast<long long>(nb) << 16));
-  }
 }
 
 }  // namespace pkv

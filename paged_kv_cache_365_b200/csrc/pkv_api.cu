@@ -1,6 +1,7 @@
 // C ABI of libpkv: argument checks, dispatch to the kernel instantiations,
 // launches.  Every host-checkable argument is checked before any CUDA call,
 // so a rejected call has no side effect (and works without a GPU).
+#include <algorithm>
 #include <cmath>
 #include <cstdint>
 #include <mutex>
@@ -168,8 +169,15 @@ pkv_status launch_multi_tc(const pkv::MultiArgs& a, const void* k_cache, const v
   if (cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(S::kSmem)) !=
       cudaSuccess)
     return PKV_ECUDA;
-  const dim3 grid(a.num_kv_heads, a.num_seqs * a.tiles, a.num_parts);
-  if (launch(kfn, grid, dim3(S::kThreads), S::kSmem, st, a, mk, mv) != PKV_OK) return PKV_ECUDA;
+  // the work list (one CTA), then a persistent grid of PKV_TC_MIN_CTAS CTAs
+  // per SM claiming (list entry, kv-head) items until the list runs out
+  if (launch(pkv::paged_multi_tc_plan_kernel<G>, dim3(1), dim3(1024), 0, st, a) != PKV_OK) return PKV_ECUDA;
+  int sms = 148, dev = 0;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const long long upper = static_cast<long long>(a.num_kv_heads) * a.num_seqs * a.tiles * a.num_parts;
+  const long long ctas = std::min<long long>(static_cast<long long>(sms) * PKV_TC_MIN_CTAS, upper);
+  if (launch(kfn, dim3(static_cast<unsigned>(ctas)), dim3(S::kThreads), S::kSmem, st, a, mk, mv) != PKV_OK)
+    return PKV_ECUDA;
   if (a.num_parts > 1) return launch_multi_merge<T, D, G>(a, st);
   return PKV_OK;
 }
@@ -338,10 +346,19 @@ pkv_status dispatch_group_fp8(const pkv::DecodeArgs& a, int G, float v_scale, cu
 
 // Workspace of the multi-token path: partials [T][Hq][P][D] then (max, sum)
 // [T][Hq][P]; nothing when every key fits one partition.
-size_t multi_workspace_bytes(long long total_q, long long Hq, long long D, long long P) {
+// Multi-token workspace: the partitions' partials (P > 1), then for the
+// tcgen05 kernel its claim counter and work list (at most 2 T P entries:
+// fewer than 2 T row tiles, each with at most P partitions).
+size_t multi_partials_bytes(long long total_q, long long Hq, long long D, long long P) {
   if (P <= 1) return 0;
   const size_t o = static_cast<size_t>(total_q * Hq * P * D * 4);
   return (o + 15) / 16 * 16 + static_cast<size_t>(total_q * Hq * P * 8);
+}
+size_t multi_tc_list_offset(long long total_q, long long Hq, long long D, long long P) {
+  return (multi_partials_bytes(total_q, Hq, D, P) + 15) / 16 * 16;
+}
+size_t multi_workspace_bytes(long long total_q, long long Hq, long long D, long long P) {
+  return multi_tc_list_offset(total_q, Hq, D, P) + 16 + static_cast<size_t>(2 * total_q * (P > 1 ? P : 1)) * 8;
 }
 
 // Device address of caller memory the kernels may touch: device memory of
@@ -797,20 +814,6 @@ pkv_status pkv_paged_attention_decode_static_ws(void* out, const void* q, const 
                                     scale, partition_tokens, dtype, ws, PKV_STATIC_WORKSPACE_BYTES, stream);
 }
 
-#ifdef PKV_TC_TRACE
-// debug builds only: the tcgen05 kernel's timeline probe (64 x 32 x 12 clocks)
-int pkv_debug_tc_trace(long long* out) {
-  return cudaMemcpyFromSymbol(out, pkv::g_tc_trace, sizeof(pkv::g_tc_trace)) == cudaSuccess ? 0 : 1;
-}
-// per-CTA entry / first copy / exit times and (SM, blocks): 16384 x 4
-int pkv_debug_tc_cta(long long* out) {
-  return cudaMemcpyFromSymbol(out, pkv::g_tc_cta, sizeof(pkv::g_tc_cta)) == cudaSuccess ? 0 : 1;
-}
-int pkv_debug_tc_cta_clear() {
-  static long long zero[16384][4];
-  return cudaMemcpyToSymbol(pkv::g_tc_cta, zero, sizeof(zero)) == cudaSuccess ? 0 : 1;
-}
-#endif
 
 pkv_status pkv_selftest_bounded_wait(long long limit_cycles, void* stream) {
   if (limit_cycles <= 0 || limit_cycles > (1ll << 32)) return PKV_EINVAL;
@@ -876,8 +879,16 @@ pkv_status multi_impl(void* out, const void* q, const void* k_cache, const void*
   const int tile_rows = tc ? 128 : fa ? 16 * kFaWarps : 8 * (NW ? NW : NT);
   const long long tiles = (rows_max + tile_rows - 1) / tile_rows;
   const long long P = (static_cast<long long>(max_context_len) + part - 1) / part;
-  if (tiles * num_seqs > 65535 || P > 65535) return PKV_EINVAL;
-  const size_t need = multi_workspace_bytes(total_query_tokens, num_q_heads, head_dim, P);
+  if (P > 65535) return PKV_EINVAL;
+  if (tc) {
+    // the persistent kernel's work list: a tile index fits 15 bits, the
+    // (entry, kv-head) items an int
+    if (tiles > 32767 || 2LL * total_query_tokens * P * num_kv_heads >= (1LL << 31)) return PKV_EINVAL;
+  } else if (tiles * num_seqs > 65535) {
+    return PKV_EINVAL;
+  }
+  const size_t need = tc ? multi_workspace_bytes(total_query_tokens, num_q_heads, head_dim, P)
+                        : multi_partials_bytes(total_query_tokens, num_q_heads, head_dim, P);
   if (need > 0 && (workspace == nullptr || workspace_bytes_given < need || !aligned16(workspace)))
     return PKV_EINVAL;
   pkv::MultiArgs a{};
@@ -886,10 +897,16 @@ pkv_status multi_impl(void* out, const void* q, const void* k_cache, const void*
   a.block_tables = block_tables;
   a.context_lens = context_lens;
   a.query_start = query_start;
-  if (need) {
+  if (P > 1) {
     a.ws_o = static_cast<float*>(workspace);
     const size_t o = static_cast<size_t>(total_query_tokens) * num_q_heads * P * head_dim * 4;
     a.ws_ml = reinterpret_cast<float2*>(static_cast<unsigned char*>(workspace) + (o + 15) / 16 * 16);
+  }
+  if (tc) {
+    unsigned char* l = static_cast<unsigned char*>(workspace) +
+                       multi_tc_list_offset(total_query_tokens, num_q_heads, head_dim, P);
+    a.tc_ctr = reinterpret_cast<int*>(l);
+    a.tc_items = reinterpret_cast<int2*>(l + 16);
   }
   a.bt_stride = max_blocks_per_seq;
   a.max_ctx = max_context_len;

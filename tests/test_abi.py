@@ -153,16 +153,23 @@ def test_prefix_workspace_and_rejections(lib):
         assert lib.pkv_paged_attention_decode_prefix_phase(*args[:-1], phase, None) == 1
 
 
+def multi_ws(T, Hq, D, P):
+    """Partials T*Hq*P*D*4 (rounded to 16) + T*Hq*P*8 when P > 1, then the
+    tcgen05 kernel's counter (16) and work list (2*T*P entries of 8)."""
+    part = 0
+    if P > 1:
+        o = T * Hq * P * D * 4
+        part = (o + 15) // 16 * 16 + T * Hq * P * 8
+    return (part + 15) // 16 * 16 + 16 + 2 * T * P * 8
+
+
 def test_multi_workspace_and_rejections(lib):
-    # one partition: nothing; else T*Hq*P*D*4 (rounded to 16) + T*Hq*P*8
-    assert lib.pkv_multi_workspace_bytes(10, 8, 128, 512, 512) == 0
-    o = 10 * 8 * 3 * 128 * 4
-    assert lib.pkv_multi_workspace_bytes(10, 8, 128, 1100, 512) == (o + 15) // 16 * 16 + 10 * 8 * 3 * 8
+    assert lib.pkv_multi_workspace_bytes(10, 8, 128, 512, 512) == multi_ws(10, 8, 128, 1)
+    assert lib.pkv_multi_workspace_bytes(10, 8, 128, 1100, 512) == multi_ws(10, 8, 128, 3)
     assert lib.pkv_multi_workspace_bytes(10, 8, 96, 1100, 512) == 0
     # auto partition: 2048 tokens (one partition here), 1024 past 4096 tokens
-    assert lib.pkv_multi_workspace_bytes(10, 8, 128, 2048, 0) == 0
-    o = 10 * 8 * 5 * 128 * 4
-    assert lib.pkv_multi_workspace_bytes(10, 8, 128, 5000, 0) == (o + 15) // 16 * 16 + 10 * 8 * 5 * 8
+    assert lib.pkv_multi_workspace_bytes(10, 8, 128, 2048, 0) == multi_ws(10, 8, 128, 1)
+    assert lib.pkv_multi_workspace_bytes(10, 8, 128, 5000, 0) == multi_ws(10, 8, 128, 5)
     # 512-token partitions: 1100 tokens split, so the workspace is checked
     args = [FAKE, FAKE, FAKE, FAKE, FAKE, 100, FAKE, 1100, FAKE, 8, 40, 4, 8, 2, 128, 64, ctypes.c_float(0.1), 512,
             1, FAKE, 1 << 30, None]
@@ -171,10 +178,15 @@ def test_multi_workspace_and_rejections(lib):
         a = list(args)
         a[idx] = bad
         assert lib.pkv_paged_attention_multi(*a) == 1, (idx, bad)
-    # grid limit: num_seqs * (row tiles per sequence) > 65535 (4096 tokens x
-    # G 4 = 16384 rows: 128 tiles of 128 rows)
+    # grid limit of the kernels below the tcgen05 one: num_seqs * (row tiles
+    # per sequence) <= 65535 (8 tokens x G 4 = 32 rows: one tile)
     a = list(args)
-    a[9], a[11] = 4096, 600
+    a[11] = 65536
+    assert lib.pkv_paged_attention_multi(*a) == 1
+    # the tcgen05 kernel's work list: at most 32767 tiles of 128 rows per
+    # sequence (2^20 tokens x G 4 = 32768 tiles)
+    a = list(args)
+    a[9], a[10] = 1 << 20, 1 << 20
     assert lib.pkv_paged_attention_multi(*a) == 1
     # nothing to do
     a = list(args)
@@ -252,10 +264,9 @@ def test_multi_fp8_rejections(lib):
         a = list(args)
         a[idx] = bad
         assert lib.pkv_paged_attention_multi_fp8(*a) == 1, (idx, bad)
-    # every shape takes 128-row tiles: 600 sequences x ceil(9 x 4 / 128) = 600
-    # tiles fit, 4096 tokens x G 4 = 128 tiles a sequence do not
+    # every shape takes 128-row tiles, at most 32767 a sequence
     a = list(args)
-    a[9], a[11] = 4096, 600
+    a[9], a[10] = 1 << 20, 1 << 20
     assert lib.pkv_paged_attention_multi_fp8(*a) == 1
     a = list(args)
     a[10] = 0

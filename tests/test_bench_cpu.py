@@ -74,7 +74,9 @@ def test_library_partition_rule_and_workspace_sizes():
         assert pkv.decode_workspace_bytes(B, Hq, D, n, 0) == (0 if P <= 1 else B * Hq * P * (D + 2) * 4)
         T = 7
         Pm = -(-n // pt(_lib.OP_MULTI, n))
-        want = 0 if Pm <= 1 else -(-(T * Hq * Pm * D * 4) // 16) * 16 + T * Hq * Pm * 8
+        part = 0 if Pm <= 1 else -(-(T * Hq * Pm * D * 4) // 16) * 16 + T * Hq * Pm * 8
+        # then the tcgen05 kernel's claim counter and work list
+        want = -(-part // 16) * 16 + 16 + 2 * T * Pm * 8
         assert pkv.multi_workspace_bytes(T, Hq, D, n, 0) == want
 
 
