@@ -1079,44 +1079,68 @@ __global__ void __launch_bounds__(kMergeWarps * 32) paged_multi_merge_kernel(con
   if (!multi_seq(a, b, ctx, q0, nq, false) || ctx <= a.partition) return;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   constexpr int kEpl = D / 32;
-  for (int r = warp; r < nq * G; r += kMergeWarps) {
-    const int i = r / G;
-    const size_t row = static_cast<size_t>(q0 + i) * a.num_q_heads + kvh * G + r % G;
-    const int pos = ctx - nq + i;
-    const int n = pos >= 0 ? pos / a.partition + 1 : 0;  // n = 0 writes zeros
-    const size_t w0 = row * a.num_parts;
-    float M = -INFINITY;
-    for (int p = lane; p < n; p += 32) M = fmaxf(M, a.ws_ml[w0 + p].x);
-    M = warp_max(M);
-    float acc[kEpl];
+  constexpr int kRows = 4;  // rows a warp merges at once (their loads in flight together)
+  const int rows = nq * G;
+  for (int r0 = warp; r0 < rows; r0 += kMergeWarps * kRows) {
+    size_t w0[kRows];
+    int n[kRows];
+    int nmax = 0;
 #pragma unroll
-    for (int e = 0; e < kEpl; ++e) acc[e] = 0.f;
-    float den = 0.f;
-    for (int p = 0; p < n; ++p) {
-      const float2 v = a.ws_ml[w0 + p];
-      const float w = exp2f(v.x - M);
-      den = fmaf(w, v.y, den);
-      // this lane's kEpl (2 or 4) consecutive elements in one load
-      const float2* o = reinterpret_cast<const float2*>(a.ws_o + (w0 + p) * D + lane * kEpl);
-      float2 f[kEpl / 2];
-      if constexpr (kEpl == 4) {
-        const float4 g = *reinterpret_cast<const float4*>(o);
-        f[0] = make_float2(g.x, g.y);
-        f[1] = make_float2(g.z, g.w);
-      } else {
+    for (int k = 0; k < kRows; ++k) {
+      const int r = r0 + k * kMergeWarps;
+      const int i = r / G;
+      const int pos = ctx - nq + i;
+      n[k] = r < rows && pos >= 0 ? pos / a.partition + 1 : 0;  // n = 0 writes zeros
+      w0[k] = (static_cast<size_t>(q0 + i) * a.num_q_heads + kvh * G + r % G) * a.num_parts;
+      nmax = max(nmax, n[k]);
+    }
+    float M[kRows];
 #pragma unroll
-        for (int e = 0; e < kEpl / 2; ++e) f[e] = o[e];
-      }
+    for (int k = 0; k < kRows; ++k) M[k] = -INFINITY;
+    for (int p = lane; p < nmax; p += 32)
 #pragma unroll
-      for (int e = 0; e < kEpl / 2; ++e) {
-        acc[2 * e] = fmaf(w, f[e].x, acc[2 * e]);
-        acc[2 * e + 1] = fmaf(w, f[e].y, acc[2 * e + 1]);
+      for (int k = 0; k < kRows; ++k)
+        if (p < n[k]) M[k] = fmaxf(M[k], a.ws_ml[w0[k] + p].x);
+#pragma unroll
+    for (int k = 0; k < kRows; ++k) M[k] = warp_max(M[k]);
+    float acc[kRows][kEpl], den[kRows];
+#pragma unroll
+    for (int k = 0; k < kRows; ++k) {
+      den[k] = 0.f;
+#pragma unroll
+      for (int e = 0; e < kEpl; ++e) acc[k][e] = 0.f;
+    }
+    for (int p = 0; p < nmax; ++p) {
+#pragma unroll
+      for (int k = 0; k < kRows; ++k) {
+        if (p >= n[k]) continue;
+        const float2 v = a.ws_ml[w0[k] + p];
+        const float w = exp2f(v.x - M[k]);
+        den[k] = fmaf(w, v.y, den[k]);
+        // this lane's kEpl (2 or 4) consecutive elements in one load
+        const float* o = a.ws_o + (w0[k] + p) * D + lane * kEpl;
+        if constexpr (kEpl == 4) {
+          const float4 g = *reinterpret_cast<const float4*>(o);
+          acc[k][0] = fmaf(w, g.x, acc[k][0]);
+          acc[k][1] = fmaf(w, g.y, acc[k][1]);
+          acc[k][2] = fmaf(w, g.z, acc[k][2]);
+          acc[k][3] = fmaf(w, g.w, acc[k][3]);
+        } else {
+          const float2 g = *reinterpret_cast<const float2*>(o);
+          acc[k][0] = fmaf(w, g.x, acc[k][0]);
+          acc[k][1] = fmaf(w, g.y, acc[k][1]);
+        }
       }
     }
-    T* out = reinterpret_cast<T*>(a.out) + row * D + lane * kEpl;
-    const float inv = n > 0 ? 1.f / den : 0.f;
 #pragma unroll
-    for (int e = 0; e < kEpl; ++e) out[e] = Fmt<T>::from_f32(acc[e] * inv);
+    for (int k = 0; k < kRows; ++k) {
+      const int r = r0 + k * kMergeWarps;
+      if (r >= rows) continue;
+      T* out = reinterpret_cast<T*>(a.out) + w0[k] / a.num_parts * D + lane * kEpl;
+      const float inv = n[k] > 0 ? 1.f / den[k] : 0.f;
+#pragma unroll
+      for (int e = 0; e < kEpl; ++e) out[e] = Fmt<T>::from_f32(acc[k][e] * inv);
+    }
   }
 }
 
