@@ -201,8 +201,8 @@ struct TcShape {
   static constexpr size_t kOffBars = kOffV + size_t(NSV) * kKV;
   // barriers: kfull[NSK], kempty[NSK], vfull[NSV], vempty[NSV], sfull[2],
   // pfull[2], pvdone, final, qfull, qempty, oempty, itemfull[2],
-  // itemempty[2], drain
-  static constexpr int kBars = 2 * NSK + 2 * NSV + 14;
+  // itemempty[2], drain, kready[NSK] (FP8: the K block widened)
+  static constexpr int kBars = 3 * NSK + 2 * NSV + 14;
   static constexpr size_t kOffTab = kOffBars + size_t(kBars) * 8;
   static constexpr int kMaxPages = 128;  // pages of the longest partition (2048 tokens)
   // two work-item slots: their page tables, then their descriptions
@@ -391,6 +391,7 @@ __global__ void __launch_bounds__(TcShape<D, NSK, NSV>::kThreads, PKV_TC_MIN_CTA
   const uint32_t bar_pfull = bar_sfull + 16, bar_pvdone = bar_pfull + 16, bar_final = bar_pvdone + 8;
   const uint32_t bar_qfull = bar_final + 8, bar_qempty = bar_qfull + 8, bar_oempty = bar_qempty + 8;
   const uint32_t bar_itemfull = bar_oempty + 8, bar_itemempty = bar_itemfull + 16, bar_drain = bar_itemempty + 16;
+  const uint32_t bar_kready = bar_drain + 8;
   int* tables = reinterpret_cast<int*>(smem + S::kOffTab);
   TcItem* items = reinterpret_cast<TcItem*>(smem + S::kOffItem);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + S::kOffSlot);
@@ -416,6 +417,7 @@ __global__ void __launch_bounds__(TcShape<D, NSK, NSV>::kThreads, PKV_TC_MIN_CTA
     mbar_init(bar_qempty, 1);
     mbar_init(bar_oempty, 4);
     mbar_init(bar_drain, 1);
+    for (int s = 0; s < NSK; ++s) mbar_init(bar_kready + 8 * s, 1);
     fence_barrier_init();
   }
   if (warp == 1) {
@@ -493,64 +495,89 @@ __global__ void __launch_bounds__(TcShape<D, NSK, NSV>::kThreads, PKV_TC_MIN_CTA
       if (lane == 0) {
         item = d;
         mbar_arrive(bar_itemfull + 8 * slot);  // release: the table and the description
-        auto issue = [&](bool is_v, int c) {
-          const int g = (is_v ? issued_v : issued_k);
-          const int s = g % (is_v ? NSV : NSK);
-          constexpr uint32_t kPageBytes = F8 ? kBlockSize * D : kBlockSize * D * 2;
-          uint32_t bytes = 0;
+      }
+      // lane 0 issues a block's copies
+      auto issue = [&](bool is_v, int c) {
+        const int g = (is_v ? issued_v : issued_k);
+        const int s = g % (is_v ? NSV : NSK);
+        constexpr uint32_t kPageBytes = F8 ? kBlockSize * D : kBlockSize * D * 2;
+        uint32_t bytes = 0;
 #pragma unroll
-          for (int p = 0; p < S::kPages; ++p)
-            if (loaded_in(d, tab, c * S::kPages + p)) bytes += kPageBytes;
-          const uint32_t bar = (is_v ? bar_vfull : bar_kfull) + 8 * s;
-          if (bytes == 0) {
-            mbar_arrive(bar);
-            return;
-          }
-          mbar_arrive_expect_tx(bar, bytes);
-          const uint32_t st = (is_v ? sv : sk) + s * S::kKV;
-          const CUtensorMap* map = is_v ? &tmap_v : &tmap_k;
+        for (int p = 0; p < S::kPages; ++p)
+          if (loaded_in(d, tab, c * S::kPages + p)) bytes += kPageBytes;
+        const uint32_t bar = (is_v ? bar_vfull : bar_kfull) + 8 * s;
+        if (bytes == 0) {
+          mbar_arrive(bar);
+          return;
+        }
+        mbar_arrive_expect_tx(bar, bytes);
+        const uint32_t st = (is_v ? sv : sk) + s * S::kKV;
+        const CUtensorMap* map = is_v ? &tmap_v : &tmap_k;
 #pragma unroll
-          for (int p = 0; p < S::kPages; ++p) {
-            const int i = c * S::kPages + p;
-            if (!loaded_in(d, tab, i)) continue;
-            const int y = (tab[i] * a.num_kv_heads + d.kvh) * kBlockSize;
-            if constexpr (F8) {
-              tma_load_2d(st + S::kKV / 2 + p * kPageBytes, map, 0, y, bar);  // one box of 16 rows x D codes
-            } else {
-#pragma unroll
-              for (int bx = 0; bx < S::kPanels; ++bx)
-                tma_load_2d(st + bx * S::kKVPanel + p * 2048, map, bx * 64, y, bar);
-            }
-          }
-        };
-        int ck = 0, cv = 0;  // this item's blocks issued
-        long long t0 = clock64();
-        while (ck < d.nb || cv < d.nb) {
-          bool moved = false;
-          if (ck < d.nb && (issued_k < NSK || mbar_test(bar_kempty + 8 * (issued_k % NSK),
-                                                        ((issued_k / NSK) - 1) & 1))) {
-            issue(false, ck++);
-            ++issued_k;
-            moved = true;
-          }
-          if (cv < d.nb && (issued_v < NSV || mbar_test(bar_vempty + 8 * (issued_v % NSV),
-                                                        ((issued_v / NSV) - 1) & 1))) {
-            issue(true, cv++);
-            ++issued_v;
-            moved = true;
-          }
-          if (moved) {
-            t0 = clock64();
-          } else if (clock64() - t0 > (1ll << 32)) {
-            raise_error(PKV_ERR_TIMEOUT);
-            bad = true;
-            break;
+        for (int p = 0; p < S::kPages; ++p) {
+          const int i = c * S::kPages + p;
+          if (!loaded_in(d, tab, i)) continue;
+          const int y = (tab[i] * a.num_kv_heads + d.kvh) * kBlockSize;
+          if constexpr (F8) {
+            tma_load_2d(st + S::kKV / 2 + p * kPageBytes, map, 0, y, bar);  // one box of 16 rows x D codes
           } else {
-            __nanosleep(32);
+#pragma unroll
+            for (int bx = 0; bx < S::kPanels; ++bx)
+              tma_load_2d(st + bx * S::kKVPanel + p * 2048, map, bx * 64, y, bar);
           }
         }
+      };
+      // the whole warp runs the loop (each decision taken by lane 0 and
+      // shared); over an FP8 pool it also widens each K block once its codes
+      // have landed, so the MMA warp widens only V
+      int ck = 0, cv = 0, cw = 0;  // this item's blocks issued (K, V), K blocks widened
+      long long t0 = clock64();
+      while (ck < d.nb || cv < d.nb || (F8 && cw < d.nb)) {
+        bool moved = false;
+        const bool k_go = __shfl_sync(kFull, ck < d.nb && (issued_k < NSK || mbar_test(bar_kempty + 8 * (issued_k % NSK),
+                                                                                         ((issued_k / NSK) - 1) & 1)), 0);
+        if (k_go) {
+          if (lane == 0) issue(false, ck);
+          ++ck;
+          ++issued_k;
+          moved = true;
+        }
+        const bool v_go = __shfl_sync(kFull, cv < d.nb && (issued_v < NSV || mbar_test(bar_vempty + 8 * (issued_v % NSV),
+                                                                                         ((issued_v / NSV) - 1) & 1)), 0);
+        if (v_go) {
+          if (lane == 0) issue(true, cv);
+          ++cv;
+          ++issued_v;
+          moved = true;
+        }
+        if constexpr (F8) {
+          const int gw = issued_k - ck + cw;  // the K block to widen next
+          const bool w_go = __shfl_sync(kFull, cw < ck && mbar_test(bar_kfull + 8 * (gw % NSK), (gw / NSK) & 1), 0);
+          if (w_go) {
+            // the keys of block cw that are there
+            const int lim = d.tok1 - (d.tok0 + cw * S::kKeys);
+            uint64_t m = lim >= S::kKeys ? ~0ull : (lim > 0 ? (1ull << lim) - 1ull : 0ull);
+#pragma unroll
+            for (int p = 0; p < S::kPages; ++p)
+              if (!loaded_in(d, tab, cw * S::kPages + p)) m &= ~(0xFFFFull << (16 * p));
+            tc_widen_fp8<D, NSK, NSV>(smem + S::kOffK + (gw % NSK) * S::kKV, m, lane);
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar_kready + 8 * (gw % NSK));
+            ++cw;
+            moved = true;
+          }
+        }
+        if (moved) {
+          t0 = clock64();
+        } else if (__shfl_sync(kFull, clock64() - t0 > (1ll << 32), 0)) {
+          if (lane == 0) raise_error(PKV_ERR_TIMEOUT);
+          bad = true;
+          break;
+        } else {
+          __nanosleep(32);
+        }
       }
-      bad = __shfl_sync(kFull, bad, 0);
     }
   } else if (warp == 1) {
     // ---- MMA issuer (lane 0); V-row zeroing, or the widening of FP8 codes,
@@ -647,14 +674,11 @@ __global__ void __launch_bounds__(TcShape<D, NSK, NSV>::kThreads, PKV_TC_MIN_CTA
       for (int c = 0; c < d.nb && !bad; ++c) {
         const int g = g0 + c;
         const int s = g % NSK;
-        if (!wait_all(bar_kfull + 8 * s, (g / NSK) & 1)) {
+        // (over an FP8 pool: the block's K codes landed and widened by the
+        // producer warp)
+        if (!wait_all((F8 ? bar_kready : bar_kfull) + 8 * s, (g / NSK) & 1)) {
           bad = true;
           break;
-        }
-        if constexpr (F8) {
-          tc_widen_fp8<D, NSK, NSV>(smem + S::kOffK + s * S::kKV, valid_keys(c), lane);
-          fence_proxy_async_smem();
-          __syncwarp();
         }
         // S buffer g & 1 was last read (as P) by the P.V of block g - 2.
         // Inside an item that is the latest P.V issued; at an item's first
