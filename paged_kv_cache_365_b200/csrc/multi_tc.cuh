@@ -10,21 +10,28 @@
 // the one paged_multi_fa_kernel computes (multi_mma.cuh); what changes is
 // where the contraction runs and where its accumulators live.
 //
-// One CTA per (kv-head, sequence, tile of 128 rows, key partition); a row
-// is a (token, head) pair of the kv-head, as in the other multi-token
-// kernels.  Six warps with fixed jobs:
-//   warp 0      TMA producers (lane 0 for K, lane 1 for V): the partition's
-//               pages, four per key block (64 keys), into a K ring and a V
-//               ring; a K stage is free again once its block's scores are
-//               formed, a V stage once its P.V is done, so the K loads run
-//               ahead of the S-buffer turnaround;
+// Work items are (sequence, row tile of 128, key partition, kv-head); a
+// row is a (token, head) pair of the kv-head, as in the other multi-token
+// kernels.  A plan kernel (one CTA) lists the (sequence, tile, partition)
+// entries that have keys to attend, longest first; a persistent grid of two
+// CTAs per SM claims items from an atomic counter until the list runs out.
+// Six warps with fixed jobs, walking the same items in the same order:
+//   warp 0      claims the next item, writes its page table and bounds into
+//               a two-slot ring in shared memory, and (lane 0) issues the
+//               TMA copies of its pages, four per key block (64 keys), into
+//               a K ring and a V ring; a K stage is free again once its
+//               block's scores are formed, a V stage once its P.V is done,
+//               so the K loads run ahead of the S-buffer turnaround; over an
+//               FP8 pool it also widens each K block's codes to fp16 in
+//               place once they have landed;
 //   warp 1      owns the tensor memory and issues the MMAs from one thread:
 //                 S_j  = Q . K_j^T      (M 128, N 64, A and B from shared
 //                                        memory, K-major, 128-byte swizzle)
 //                 O   += P_j . V_j      (A = P from tensor memory, B = V
 //                                        from shared memory, MN-major)
 //               S is double-buffered, so the scores of block j+1 are formed
-//               while block j's softmax runs;
+//               while block j's softmax runs; over an FP8 pool the whole
+//               warp widens each V block while the block's softmax runs;
 //   warps 2-5   softmax and epilogue, one thread per row (its tensor-memory
 //               lane): the row's 64 scores of a block come in with
 //               tcgen05.ld, the causal mask and the running max need no
@@ -32,7 +39,9 @@
 //               16-bit parts (two MMAs, ~2^-16 relative error, as in the
 //               other kernels).  The running max is moved only when a block
 //               raises it by more than 2^8 (then O is rescaled in tensor
-//               memory), so most blocks need no O traffic at all.
+//               memory), so most blocks need no O traffic at all.  At an
+//               item's end they load the next item's Q while its last P.V
+//               runs, then read O out and release it.
 // Tensor memory: O in columns [0, D), S/P buffers at columns 128 and 192
 // (256 columns a CTA, two CTAs an SM).  Invalid V rows of a block (past the
 // context, or pages the table does not name) are zeroed in shared memory
@@ -219,7 +228,8 @@ struct TcShape {
 
 // FP8 pools: a block's 64 x D E4M3 codes land (TMA, the pool's per-page
 // swizzle of decode_fp8.cuh) in the upper half of a 16-bit stage and are
-// widened in place into the stage's 16-bit layout by one warp; keys not in
+// widened in place into the stage's 16-bit layout by one warp (K by the
+// producer, V by the MMA warp); keys not in
 // `valid` (bit r: key r of the block) become zeros.  Outputs below the codes
 // are written while the codes are read; the rest only after the whole warp
 // has read its codes (__syncwarp), since they overwrite them.
@@ -580,7 +590,7 @@ __global__ void __launch_bounds__(TcShape<D, NSK, NSV>::kThreads, PKV_TC_MIN_CTA
       }
     }
   } else if (warp == 1) {
-    // ---- MMA issuer (lane 0); V-row zeroing, or the widening of FP8 codes,
+    // ---- MMA issuer (lane 0); V-row zeroing, or the widening of FP8 V codes,
     // by the whole warp ---------------------------------------------------
     constexpr uint32_t kIdQK = tc_idesc<TM>(128, S::kKeys, false);
     constexpr uint32_t kIdPV = tc_idesc<TM>(128, D, true);
