@@ -506,36 +506,36 @@ __global__ void __launch_bounds__(TcShape<D, NSK, NSV>::kThreads, PKV_TC_MIN_CTA
         item = d;
         mbar_arrive(bar_itemfull + 8 * slot);  // release: the table and the description
       }
-      // lane 0 issues a block's copies
+      // a block's copies, one TMA box per lane (page p, 64-column panel):
+      // lane 0 first arms the stage's barrier with the block's bytes
       auto issue = [&](bool is_v, int c) {
         const int g = (is_v ? issued_v : issued_k);
         const int s = g % (is_v ? NSV : NSK);
         constexpr uint32_t kPageBytes = F8 ? kBlockSize * D : kBlockSize * D * 2;
+        constexpr int kBoxes = F8 ? 1 : S::kPanels;  // boxes a page
         uint32_t bytes = 0;
 #pragma unroll
         for (int p = 0; p < S::kPages; ++p)
           if (loaded_in(d, tab, c * S::kPages + p)) bytes += kPageBytes;
         const uint32_t bar = (is_v ? bar_vfull : bar_kfull) + 8 * s;
-        if (bytes == 0) {
-          mbar_arrive(bar);
-          return;
+        if (lane == 0) {
+          if (bytes == 0)
+            mbar_arrive(bar);
+          else
+            mbar_arrive_expect_tx(bar, bytes);
         }
-        mbar_arrive_expect_tx(bar, bytes);
+        __syncwarp();
+        if (bytes == 0 || lane >= S::kPages * kBoxes) return;
+        const int p = lane / kBoxes, bx = lane % kBoxes;
+        const int i = c * S::kPages + p;
+        if (!loaded_in(d, tab, i)) return;
         const uint32_t st = (is_v ? sv : sk) + s * S::kKV;
         const CUtensorMap* map = is_v ? &tmap_v : &tmap_k;
-#pragma unroll
-        for (int p = 0; p < S::kPages; ++p) {
-          const int i = c * S::kPages + p;
-          if (!loaded_in(d, tab, i)) continue;
-          const int y = (tab[i] * a.num_kv_heads + d.kvh) * kBlockSize;
-          if constexpr (F8) {
-            tma_load_2d(st + S::kKV / 2 + p * kPageBytes, map, 0, y, bar);  // one box of 16 rows x D codes
-          } else {
-#pragma unroll
-            for (int bx = 0; bx < S::kPanels; ++bx)
-              tma_load_2d(st + bx * S::kKVPanel + p * 2048, map, bx * 64, y, bar);
-          }
-        }
+        const int y = (tab[i] * a.num_kv_heads + d.kvh) * kBlockSize;
+        if constexpr (F8)
+          tma_load_2d(st + S::kKV / 2 + p * kPageBytes, map, 0, y, bar);  // one box of 16 rows x D codes
+        else
+          tma_load_2d(st + bx * S::kKVPanel + p * 2048, map, bx * 64, y, bar);
       };
       // the whole warp runs the loop (each decision taken by lane 0 and
       // shared); over an FP8 pool it also widens each K block once its codes
@@ -547,7 +547,7 @@ __global__ void __launch_bounds__(TcShape<D, NSK, NSV>::kThreads, PKV_TC_MIN_CTA
         const bool k_go = __shfl_sync(kFull, ck < d.nb && (issued_k < NSK || mbar_test(bar_kempty + 8 * (issued_k % NSK),
                                                                                          ((issued_k / NSK) - 1) & 1)), 0);
         if (k_go) {
-          if (lane == 0) issue(false, ck);
+          issue(false, ck);
           ++ck;
           ++issued_k;
           moved = true;
@@ -555,7 +555,7 @@ __global__ void __launch_bounds__(TcShape<D, NSK, NSV>::kThreads, PKV_TC_MIN_CTA
         const bool v_go = __shfl_sync(kFull, cv < d.nb && (issued_v < NSV || mbar_test(bar_vempty + 8 * (issued_v % NSV),
                                                                                          ((issued_v / NSV) - 1) & 1)), 0);
         if (v_go) {
-          if (lane == 0) issue(true, cv);
+          issue(true, cv);
           ++cv;
           ++issued_v;
           moved = true;
