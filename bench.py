@@ -531,7 +531,8 @@ def run_multi(args, rank, world, local_rank):
     out = torch.empty_like(st["q"])
     scale = 1.0 / math.sqrt(wl.D)
     n_pairs = int(st["cow_pairs"].shape[0])
-    part_tokens = pkv.partition_tokens(pkv._lib.OP_MULTI, max_ctx, args.partition)
+    part_tokens = pkv.partition_tokens(pkv._lib.OP_MULTI_FP8 if fp8 else pkv._lib.OP_MULTI, max_ctx, args.partition,
+                                       rows=max_q * wl.Hq // wl.Hkv)
     P = max(1, math.ceil(max_ctx / part_tokens))
 
     def pre():

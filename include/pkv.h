@@ -468,15 +468,18 @@ pkv_status pkv_paged_attention_decode_prefix_fp8(void* out, const void* q, const
  * [num_seqs + 1] (device), non-decreasing, query_start[num_seqs] <=
  * total_query_tokens, every n_b <= max_query_len (a sequence that breaks
  * this is skipped, its rows left unwritten, and PKV_ERR_CONTEXT_RANGE set).
- * fp16 / bf16 only (tensor cores).  num_seqs * tiles <= 65535, with R =
- * max_query_len * G rows per kv-head: tiles = 1 while R <= 32, else
- * ceil(R / 128) (tiles of 128 rows on the tcgen05 tensor cores).
- * workspace: pkv_multi_workspace_bytes(...) bytes (0 when max_context_len <=
- * partition), 16-byte aligned.  partition_tokens as in
- * pkv_paged_attention_decode, except the auto partition (0): 2048 tokens,
- * or 1024 when max_context_len > 4096 (several rows a sequence make every
- * partial n_b times the merge work, so short contexts stay unsplit; long
- * ones are split for balance across the SMs).
+ * fp16 / bf16 only (tensor cores).  With R = max_query_len * G rows per
+ * kv-head: R <= 32 takes one tile per sequence (num_seqs <= 65535), else
+ * tiles of 128 rows on the tcgen05 tensor cores (ceil(R / 128) <= 32767),
+ * in a persistent kernel fed by a work list it writes into the workspace.
+ * workspace: pkv_multi_workspace_bytes(...) bytes, 16-byte aligned (it
+ * may be NULL when R <= 32 and max_context_len <= the partition).
+ * partition_tokens as in pkv_paged_attention_decode, except the auto
+ * partition (0): 2048 tokens, or 1024 when max_context_len > 4096 (several
+ * rows a sequence make every partial n_b times the merge work, so short
+ * contexts stay unsplit; long ones are split for balance across the SMs);
+ * 8192 for the tcgen05 kernel (its items are claimed dynamically, longest
+ * first, so long partitions leave no tail, while every split adds a merge).
  * -------------------------------------------------------------------- */
 size_t pkv_multi_workspace_bytes(int total_query_tokens, int num_q_heads, int head_dim, int max_context_len,
                                  int partition_tokens);
@@ -513,11 +516,16 @@ pkv_status pkv_paged_attention_multi_fp8(void* out, const void* q, const void* k
  *
  * pkv_partition_tokens -- the tokens per split-K partition that a call of
  * `op` makes with this partition_tokens argument (0 = its auto rule) and
- * max_context_len; prefix_pages is read by PKV_OP_DECODE_PREFIX only.
+ * max_context_len.  `extra` is PKV_OP_DECODE_PREFIX's prefix_pages and
+ * PKV_OP_MULTI's rows per kv-head (max_query_len * num_q_heads /
+ * num_kv_heads; 0 if unknown), and is read by those two ops only.
  * Auto rules:
  *   PKV_OP_DECODE         512, or 1024 when max_context_len > 4096;
  *   PKV_OP_DECODE_FP8     1024, or 2048 when max_context_len > 16384;
- *   PKV_OP_MULTI          2048, or 1024 when max_context_len > 4096;
+ *   PKV_OP_MULTI          2048, or 1024 when max_context_len > 4096; with
+ *                         more than 32 rows per kv-head (the tcgen05
+ *                         kernel) 8192;
+ *   PKV_OP_MULTI_FP8      8192 (the tcgen05 kernel);
  *   PKV_OP_DECODE_PREFIX  the longest suffix (max_context_len - 16 *
  *                         prefix_pages) rounded up to a page, kept in
  *                         [512, 2048] (the cascade's suffix pass).
@@ -528,9 +536,10 @@ typedef enum {
   PKV_OP_DECODE = 0,        /* pkv_paged_attention_decode (and _static_ws) */
   PKV_OP_DECODE_FP8 = 1,    /* pkv_paged_attention_decode_fp8 */
   PKV_OP_MULTI = 2,         /* pkv_paged_attention_multi */
-  PKV_OP_DECODE_PREFIX = 3  /* pkv_paged_attention_decode_prefix (suffix pass) */
+  PKV_OP_DECODE_PREFIX = 3, /* pkv_paged_attention_decode_prefix (suffix pass) */
+  PKV_OP_MULTI_FP8 = 4      /* pkv_paged_attention_multi_fp8 */
 } pkv_op;
-int pkv_partition_tokens(pkv_op op, int partition_tokens, int max_context_len, int prefix_pages);
+int pkv_partition_tokens(pkv_op op, int partition_tokens, int max_context_len, int extra);
 
 /* pkv_cow_copy_rows -- the rows each copy-on-write copy of a step must move.
  *

@@ -25,7 +25,7 @@ ERR_TIMEOUT = 0x10
 STATIC_WORKSPACE_BYTES = 16 << 20  # PKV_STATIC_WORKSPACE_BYTES
 
 # pkv_op: which call's partition rule pkv_partition_tokens applies
-OP_DECODE, OP_DECODE_FP8, OP_MULTI, OP_DECODE_PREFIX = 0, 1, 2, 3
+OP_DECODE, OP_DECODE_FP8, OP_MULTI, OP_DECODE_PREFIX, OP_MULTI_FP8 = 0, 1, 2, 3, 4
 
 # name -> (restype, argtypes); the same list as include/pkv.h
 PROTOTYPES = {

@@ -44,11 +44,15 @@ BLOCK_SIZE = 16
 DEFAULT_PARTITION = 512
 
 
-def partition_tokens(op: int, max_context_len: int, partition: int = 0, prefix_pages: int = 0) -> int:
+def partition_tokens(op: int, max_context_len: int, partition: int = 0, prefix_pages: int = 0,
+                     rows: int = 0) -> int:
     """Tokens per split-K partition that call ``op`` (``_lib.OP_*``) makes
     with this ``partition`` argument (0 = its auto rule): the library's own
-    rule (pkv_partition_tokens)."""
-    p = int(lib.pkv_partition_tokens(int(op), int(partition), int(max_context_len), int(prefix_pages)))
+    rule (pkv_partition_tokens).  ``prefix_pages``: the cascade's shared
+    pages (OP_DECODE_PREFIX); ``rows``: rows per kv-head of a multi-token
+    call, max_query_len * Hq / Hkv (OP_MULTI)."""
+    extra = prefix_pages if int(op) == _lib.OP_DECODE_PREFIX else rows
+    p = int(lib.pkv_partition_tokens(int(op), int(partition), int(max_context_len), int(extra)))
     if p < 0:
         raise ValueError(f"invalid partition {partition} for op {op}")
     return p

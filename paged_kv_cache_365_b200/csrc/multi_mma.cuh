@@ -1079,7 +1079,7 @@ __global__ void __launch_bounds__(kMergeWarps * 32) paged_multi_merge_kernel(con
   if (!multi_seq(a, b, ctx, q0, nq, false) || ctx <= a.partition) return;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   constexpr int kEpl = D / 32;
-  constexpr int kRows = 4;  // rows a warp merges at once (their loads in flight together)
+  constexpr int kRows = 8;  // rows a warp merges at once (their loads in flight together)
   const int rows = nq * G;
   for (int r0 = warp; r0 < rows; r0 += kMergeWarps * kRows) {
     size_t w0[kRows];

@@ -196,6 +196,12 @@ __host__ __device__ constexpr uint32_t tc_idesc(int M, int N, bool b_mn_major) {
 // ----------------------------------------------------------------------------
 // the kernel
 // ----------------------------------------------------------------------------
+// Tokens of the kernel's auto key partition (its page table in shared
+// memory holds that many pages).
+#ifndef PKV_TC_AUTO_PARTITION
+#define PKV_TC_AUTO_PARTITION 8192
+#endif
+
 template <int D, int NSK, int NSV>
 struct TcShape {
   static constexpr int kRows = 128;                 // query rows of a tile (the MMA's M, one per TMEM lane)
@@ -213,7 +219,8 @@ struct TcShape {
   // itemempty[2], drain, kready[NSK] (FP8: the K block widened)
   static constexpr int kBars = 3 * NSK + 2 * NSV + 14;
   static constexpr size_t kOffTab = kOffBars + size_t(kBars) * 8;
-  static constexpr int kMaxPages = 128;  // pages of the longest partition (2048 tokens)
+  // pages of the longest partition (the auto one, or 2048 tokens)
+  static constexpr int kMaxPages = PKV_TC_AUTO_PARTITION / kBlockSize > 128 ? PKV_TC_AUTO_PARTITION / kBlockSize : 128;
   // two work-item slots: their page tables, then their descriptions
   static constexpr size_t kOffItem = kOffTab + 2 * size_t(kMaxPages) * 4;
   static constexpr size_t kOffSlot = kOffItem + 2 * 64;
@@ -318,13 +325,13 @@ __device__ __forceinline__ int tc_item_blocks(int ctx, int nq, int G, int t, int
 
 // The work list: one entry (b, tile << 16 | partition) per visited
 // (sequence, row tile, partition), longest first (a counting sort on the
-// number of key blocks, at most 32 for a 2048-token partition), so the
+// number of key blocks, at most a partition's pages / 4), so the
 // items left at the end of the kernel are the short ones; its length; the
 // claim counter zeroed.  One CTA of 1024 threads.
 template <int G>
 __global__ void __launch_bounds__(1024) paged_multi_tc_plan_kernel(const MultiArgs a) {
   pdl_enter();
-  constexpr int kMaxNb = 32;
+  constexpr int kMaxNb = TcShape<128, 2, 2>::kMaxPages / 4;  // key blocks of the longest partition
   __shared__ int cnt[kMaxNb + 1], at[kMaxNb + 1];
   const int tid = threadIdx.x;
   if (tid <= kMaxNb) cnt[tid] = 0;

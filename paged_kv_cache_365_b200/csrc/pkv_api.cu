@@ -75,6 +75,14 @@ pkv_status launch_multi(const pkv::MultiArgs& a, const void* k_cache, const void
 int resolve_multi_partition(int p, long long max_ctx) {
   return resolve_partition(p != 0 ? p : (max_ctx > 4096 ? 1024 : 2048), max_ctx);
 }
+// Auto partition of the tcgen05 multi-token kernel (more than 32 rows per
+// kv-head, or an FP8 pool): PKV_TC_AUTO_PARTITION tokens.  Its items are
+// claimed dynamically and listed longest first, so long partitions cost no
+// tail, while each split adds partials and a merge.  Never more partitions
+// than the multi-token rule above, so a workspace sized by it suffices.
+int resolve_multi_tc_partition(int p, long long max_ctx) {
+  return p != 0 ? resolve_partition(p, max_ctx) : PKV_TC_AUTO_PARTITION;
+}
 // Auto partition of the FP8 decode: twice the 16-bit one's tokens (half the
 // bytes a page): 1024, or 2048 past 16384 tokens.
 int resolve_fp8_partition(int p, long long max_ctx) {
@@ -158,7 +166,8 @@ template <typename T, int D, int G, bool F8 = false>
 pkv_status launch_multi_tc(const pkv::MultiArgs& a, const void* k_cache, const void* v_cache, int num_blocks,
                            cudaStream_t st) {
   using S = pkv::TcShape<D, kTcKStages, kTcVStages>;
-  static_assert(kMaxPartition / PKV_BLOCK_SIZE <= S::kMaxPages, "the page table of a partition fits shared memory");
+  static_assert(kMaxPartition / PKV_BLOCK_SIZE <= S::kMaxPages && PKV_TC_AUTO_PARTITION / PKV_BLOCK_SIZE <= S::kMaxPages,
+                "the page table of a partition fits shared memory");
   CUtensorMap mk, mv;
   const long long rows = static_cast<long long>(num_blocks) * a.num_kv_heads * PKV_BLOCK_SIZE;
   if (F8 ? !encode_fp8_map(&mk, k_cache, D, rows) || !encode_fp8_map(&mv, v_cache, D, rows)
@@ -563,15 +572,18 @@ pkv_status pkv_paged_attention_decode(void* out, const void* q, const void* k_ca
   return PKV_EINVAL;
 }
 
-int pkv_partition_tokens(pkv_op op, int partition_tokens, int max_context_len, int prefix_pages) {
+int pkv_partition_tokens(pkv_op op, int partition_tokens, int max_context_len, int extra) {
   if (max_context_len < 0) return -1;
   switch (op) {
     case PKV_OP_DECODE: return resolve_partition(partition_tokens, max_context_len);
     case PKV_OP_DECODE_FP8: return resolve_fp8_partition(partition_tokens, max_context_len);
-    case PKV_OP_MULTI: return resolve_multi_partition(partition_tokens, max_context_len);
+    case PKV_OP_MULTI:
+      if (extra > kTcAboveRows) return resolve_multi_tc_partition(partition_tokens, max_context_len);
+      return resolve_multi_partition(partition_tokens, max_context_len);
+    case PKV_OP_MULTI_FP8: return resolve_multi_tc_partition(partition_tokens, max_context_len);
     case PKV_OP_DECODE_PREFIX:
-      if (prefix_pages <= 0) return -1;
-      return resolve_prefix_partition(partition_tokens, max_context_len, prefix_pages);
+      if (extra <= 0) return -1;
+      return resolve_prefix_partition(partition_tokens, max_context_len, extra);
   }
   return -1;
 }
@@ -858,7 +870,7 @@ pkv_status multi_impl(void* out, const void* q, const void* k_cache, const void*
   if (dtype != PKV_F16 && dtype != PKV_BF16) return PKV_EINVAL;  // tensor-core path only
   if (fp8 && (!std::isfinite(k_scale) || !std::isfinite(v_scale) || !(k_scale > 0.f) || !(v_scale > 0.f)))
     return PKV_EINVAL;
-  const int part = resolve_multi_partition(partition_tokens, max_context_len);
+  int part = resolve_multi_partition(partition_tokens, max_context_len);
   if (part < 0 || num_seqs < 0 || num_kv_heads <= 0 || num_kv_heads > 65535 || num_q_heads <= 0 ||
       num_q_heads % num_kv_heads != 0 || !group_ok(num_q_heads / num_kv_heads) || !head_dim_ok(head_dim) ||
       num_blocks <= 0 || max_context_len < 0 || max_blocks_per_seq <= 0 || max_query_len < 0 ||
@@ -876,6 +888,7 @@ pkv_status multi_impl(void* out, const void* q, const void* k_cache, const void*
   const bool fa = !tc && rows_max > kFaAboveRows;
   const int NW = (fa || tc) ? 0 : multi_rows_warps(rows_max);
   const int NT = tc ? (fp8 ? kTcFp8Code : kTcCode) : fa ? kFaCode : NW ? -NW : multi_ntiles(rows_max);
+  if (tc) part = resolve_multi_tc_partition(partition_tokens, max_context_len);
   const int tile_rows = tc ? 128 : fa ? 16 * kFaWarps : 8 * (NW ? NW : NT);
   const long long tiles = (rows_max + tile_rows - 1) / tile_rows;
   const long long P = (static_cast<long long>(max_context_len) + part - 1) / part;

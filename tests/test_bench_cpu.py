@@ -54,6 +54,13 @@ def test_library_partition_rule_and_workspace_sizes():
     for n in (1, 16384):
         assert pt(_lib.OP_DECODE_FP8, n) == 1024
     assert pt(_lib.OP_DECODE_FP8, 16385) == 2048
+    # the tcgen05 multi-token kernel (more than 32 rows per kv-head, or an
+    # FP8 pool): 8192 tokens at any length; up to 32 rows the rules above
+    for n in (1, 4097, 131072):
+        assert pt(_lib.OP_MULTI, n, rows=33) == 8192
+        assert pt(_lib.OP_MULTI_FP8, n) == 8192
+        assert pt(_lib.OP_MULTI, n, rows=32) == (2048 if n <= 4096 else 1024)
+    assert pt(_lib.OP_MULTI, 9000, 48, rows=128) == 48
     # cascade suffix pass: longest suffix rounded up to a page, in [512, 2048]
     assert pt(_lib.OP_DECODE_PREFIX, 1024 + 100, 0, 64) == 512
     assert pt(_lib.OP_DECODE_PREFIX, 1024 + 600, 0, 64) == 608
