@@ -269,3 +269,27 @@ def test_tcgen05_kernel_huge_logits():
     assert err == 0
     assert np.isfinite(got).all()
     assert np.abs(got - want).max() <= TOL[dt]
+
+
+@pytest.mark.parametrize("partition", [0, 32])
+def test_tcgen05_scheduler_many_items(partition):
+    """Far more work items than CTAs for the persistent tcgen05 kernel: 200
+    sequences with random lengths (some empty, some shorter than their new
+    tokens, whose first rows are zeros and flagged) and 0..70 new tokens each
+    (G = 2: up to 140 rows, two 128-row tiles), with the auto partition and
+    with 32-token partitions (thousands of items, most sequences split and
+    merged). Every row against the oracle."""
+    m = pkv()
+    rng = np.random.default_rng(31 + partition)
+    B = 200
+    nq = rng.integers(0, 71, size=B)
+    nq[:3] = 70  # at least one sequence with more than 32 rows per kv-head
+    ctx = np.maximum(nq + rng.integers(-5, 180, size=B), 0)
+    ctx[5] = 0
+    c = make_multi_case(list(ctx), list(nq), 4, 2, 64, "bf16", seed=77 + partition)
+    want = oracle.paged_multi(c["q"], c["k"], c["v"], c["tables"], c["ctx"], c["qs"], 0.125, "bf16")
+    got, err = run_gpu(c, 0.125, partition)
+    assert err in (0, m.ERR_CONTEXT_RANGE)
+    assert (err != 0) == bool(np.any(nq > ctx))
+    assert np.isfinite(got).all()
+    assert np.abs(got - want).max() <= TOL["bf16"]
