@@ -608,8 +608,11 @@ def run_multi(args, rank, world, local_rank):
     es = STORAGE[wl.dtype]
     kv = int(np.asarray(lens, dtype=np.int64).sum()) * wl.Hkv * wl.D * 2 * (1 if fp8 else es)
     att_bytes = kv + 2 * T * wl.Hq * wl.D * es + int(sum(-(-int(n) // 16) for n in lens)) * 4 + 8 * wl.B + 4
-    launches = (1 + (1 if n_pairs else 0) + 1 + (1 if P > 1 else 0)) * K
-    return dict(wl=wl, K=K, T=T, kv=kv, att_bytes=att_bytes, total_ms=total_ms, att_ms=att_ms, e2e_ms=e2e_ms,
+    # the tcgen05 kernel (more than 32 rows per kv-head, or an FP8 pool) adds
+    # its one-CTA plan kernel
+    tc = fp8 or max_q * wl.Hq // wl.Hkv > 32
+    launches = (1 + (1 if n_pairs else 0) + (2 if tc else 1) + (1 if P > 1 else 0)) * K
+    return dict(wl=wl, K=K, T=T, kv=kv, att_bytes=att_bytes, total_ms=total_ms, att_ms=att_ms, e2e_ms=e2e_ms, tc=tc,
                 h2d=h2d, d2h=d2h, clocks=clocks.summary(), P=P, launches=launches, lens=lens,
                 partition_tokens=part_tokens)
 
@@ -678,7 +681,8 @@ def multi_line(args, r, world):
         "gpu_launches": r["launches"],
         "launch": {"partition_tokens": r.get("partition_tokens"), "partition_auto": not args.partition,
                    "partitions_max": r["P"]},
-        "roofline": {"kernel": "paged_multi (partition + merge kernels)", **roof,
+        "roofline": {"kernel": ("paged_multi_tc (plan + persistent tcgen05 kernel" if r.get("tc") else
+                                "paged_multi (partition kernel") + (" + merge)" if r["P"] > 1 else ")"), **roof,
                      "peak_kind": (tpeak_kind if roof["bound"] == "tensor" else
                                    f"{peak_kind} (MEASURED_PEAKS hbm_gbs)" if peak_kind == "measured" else "fallback"),
                      "traffic": None, "algorithmic_bytes_per_launch": r["att_bytes"],
@@ -687,7 +691,7 @@ def multi_line(args, r, world):
     fp8 = bool(getattr(args, "kv_fp8", False))
     if fp8:
         line["config"]["kv_cache"] = "e4m3 (FP8) codes, scale %.6g for K and V" % FP8_SCALE
-        line["roofline"]["kernel"] = "paged_multi_fp8 (tcgen05 kernel + merge)"
+        line["roofline"]["kernel"] = line["roofline"]["kernel"].replace("paged_multi_tc", "paged_multi_fp8", 1)
     if world == 1 and not args.no_cpu_baseline and not fp8:
         line["cpu_baseline"] = multi_cpu_baseline(wl, args.new_tokens, seed=args.seed)
     return line
