@@ -306,14 +306,14 @@ def run_cuda(args, rank, world, local_rank, workload=None, graph=None):
             raise SystemExit("--kv-fp8 needs an fp16 / bf16 workload")
         to_fp8_pool(cache, dev)
     prefix = torch.from_numpy(np.ascontiguousarray(st["host"]["block_tables"][0, :pp])).to(dev) if use_cascade else None
-    # a plain 16-bit step is one launch (+ merge); the cascade keeps its copies
-    # and append in their own launch (measured faster: their loads stay off
-    # the short suffix CTAs' critical path)
-    fused_step = not fp8 and not use_cascade and wl.dtype != "f32" and not args.unfused
+    # the step through pkv_decode_step: a plain 16-bit step is one launch
+    # (+ merge); the cascade keeps its copies and append in a launch of their
+    # own, which it overlaps (it waits for it only at each sequence's last page)
+    fused_step = not fp8 and wl.dtype != "f32" and not args.unfused and not args.cascade_overlap
     if use_cascade:
         ws = cache.workspace(pkv.decode_prefix_workspace_bytes(B, Hq, D, max_ctx, pp, args.partition))
-        # [copies + append (one launch)], cascade (one launch, or prefix + suffix passes), merge
-        launches_per_step = (0 if fused_step else 1) + (3 if args.cascade_overlap else 2)
+        # copies + append (one launch), cascade (one launch, or prefix + suffix passes), merge
+        launches_per_step = 1 + (3 if args.cascade_overlap else 2)
     else:
         launches_per_step = (0 if fused_step else 1) + 1 + (1 if (n_pairs and fp8) else 0) + (1 if P > 1 else 0)
 

@@ -292,13 +292,18 @@ pkv_status pkv_paged_attention_decode_prefix_phase(void* out, const void* q, con
  * result -- the pool and out -- is that of
  *   pkv_kv_append_copy(k_new, v_new, ..., slot_mapping, num_seqs, copies, ...)
  * followed by pkv_paged_attention_decode (prefix_pages == 0) or
- * pkv_paged_attention_decode_prefix (prefix_pages > 0, the cascade).  The
- * writes are made inside the decode launch: for each sequence b and kv-head,
- * the CTA that reads the sequence's last page first copies rows 0 .. rows-1
- * of the copy (src, dst, rows) whose dst is slot_mapping[b]'s block, then
- * writes k_new[b] / v_new[b] into the slot, then stages the page -- so the
- * step needs no separate copy / append launch and the copies overlap the
- * streaming of other sequences.
+ * pkv_paged_attention_decode_prefix (prefix_pages > 0, the cascade).
+ * Without a prefix the writes are made inside the decode launch: for each
+ * sequence b and kv-head, the CTA that reads the sequence's last page first
+ * copies rows 0 .. rows-1 of the copy (src, dst, rows) whose dst is
+ * slot_mapping[b]'s block, then writes k_new[b] / v_new[b] into the slot,
+ * then stages the page -- so the step needs no separate copy / append
+ * launch and the copies overlap the streaming of other sequences.  With a
+ * prefix the copies and the append are one launch of their own
+ * (pkv_kv_append_copy), which the cascade launch does not wait for except
+ * where it reads what they write: the warp that stages a sequence's last
+ * page waits for it (programmatic dependent launch) just before that page,
+ * while the prefix pass and the other pages stream.
  *
  * One new token per sequence: k_new, v_new [num_seqs, num_kv_heads,
  * head_dim] in dtype; slot_mapping int64 [num_seqs] (< 0: no token);

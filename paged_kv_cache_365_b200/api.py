@@ -936,15 +936,19 @@ class PagedKVCache:
             B, hq = q.shape[0], q.shape[1]
             res = out if (out is not None and out.device == dev) else stg.output(st, q.shape, self.dtype)
             sc = (1.0 / math.sqrt(self.D)) if scale is None else scale
-            # a plain decode takes its copies and append into its own launch;
-            # the cascade's short suffix CTAs keep them in a launch of their own
-            fused = (self.fp8 is None and self.dtype != torch.float32 and prefix_blocks is None and
+            # the step through pkv_decode_step: a plain decode takes its copies
+            # and append into its own launch; the cascade overlaps their
+            # launch, waiting for it only at each sequence's last page
+            fused = (self.fp8 is None and self.dtype != torch.float32 and
                      (cow_pairs.shape[0] == 0 or cow_pairs.shape[1] == 3))
-            if fused:  # copies, append and decode in one launch (+ merge)
-                ws = self.workspace(decode_workspace_bytes(B, hq, self.D, max_context_len, partition))
+            if fused:
+                pp = 0 if prefix_blocks is None else int(prefix_blocks.numel())
+                ws = self.workspace(decode_prefix_workspace_bytes(B, hq, self.D, max_context_len, pp, partition) if pp
+                                    else decode_workspace_bytes(B, hq, self.D, max_context_len, partition))
                 decode_step(x["q"], self.k, self.v, x["k"], x["v"], x["slots"],
                             x["pairs"] if cow_pairs.shape[0] else None, x["tables"], x["lens"], max_context_len, sc,
-                            out=res, workspace=ws, partition=partition, stream=st)
+                            prefix_blocks=x["prefix"] if pp else None, out=res, workspace=ws, partition=partition,
+                            stream=st)
                 stg.finish(st, res, out)
                 return res
             self._copy_append(cow_pairs.shape, x, st)

@@ -80,6 +80,11 @@ struct DecodeArgs {
   const int64_t* slots;        // [B]
   const int32_t* copies;       // [n_copies][3] = (src, dst, rows)
   int n_copies;
+  // the preceding launch is this step's copy-on-write copies and append
+  // (they write only the sequences' last pages): the decode starts without
+  // waiting for it, and only the warp that stages a sequence's last page
+  // waits (griddepcontrol.wait) before that page's copy
+  int defer_wait;
 };
 
 constexpr unsigned kFull = 0xffffffffu;

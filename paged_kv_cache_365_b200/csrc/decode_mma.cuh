@@ -408,7 +408,13 @@ template <typename T, int D, int G, int NWARPS, int NSTAGE, bool kCascade>
 __global__ void __launch_bounds__(NWARPS * 32)
     paged_decode_mma_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tmap_k,
                             const __grid_constant__ CUtensorMap tmap_v) {
-  pdl_enter();
+  // a deferred wait lets the dependents launch at once, but the
+  // prerequisite launch is still waited for: by the warps that stage the
+  // pages it writes, and by every CTA before it exits (below)
+  if (a.defer_wait)
+    pdl_trigger();
+  else
+    pdl_enter();
   using S = MmaShape<T, D, G, NWARPS, NSTAGE>;
   using M = Mma<T>;
   const int kvh = blockIdx.x;
@@ -460,12 +466,16 @@ __global__ void __launch_bounds__(NWARPS * 32)
     }
     span = ctx - tok_begin;
     nparts = (span + a.partition - 1) / a.partition;
-    if (part >= (nparts > 0 ? nparts : 1)) return;
+    if (part >= (nparts > 0 ? nparts : 1)) {
+      if (a.defer_wait && threadIdx.x == 0) pdl_wait();
+      return;
+    }
     if (span == 0) {
       if (tok_begin == 0) {  // nothing to attend to at all
         T* out = reinterpret_cast<T*>(a.out) + (static_cast<size_t>(b) * a.num_q_heads + kvh * G) * D;
         for (int i = threadIdx.x; i < G * D; i += NWARPS * 32) out[i] = Fmt<T>::from_f32(0.f);
       }
+      if (a.defer_wait && threadIdx.x == 0) pdl_wait();
       return;
     }
   } else {
@@ -499,6 +509,7 @@ __global__ void __launch_bounds__(NWARPS * 32)
     const int nblk = min(a.prefix_pages - pg0, a.chunk_pages);
     prefix_warp<T, D, G, NSTAGE>(a, &tmap_k, &tmap_v, kvh, (qg * NWARPS + warp) * 16, chunk, pg0, nblk, stage0,
                                  bar0, phase_bits, lane);
+    if (a.defer_wait && threadIdx.x == 0) pdl_wait();
     return;
   }
 
@@ -530,7 +541,7 @@ __global__ void __launch_bounds__(NWARPS * 32)
     // token and its copy-on-write copy first, and fences them before that
     // page's TMA load
     int last_i = -1;
-    if (!prefix_role && a.slots != nullptr && pidx == nparts - 1 && warp == (nblk - 1) % NWARPS)
+    if (!prefix_role && (a.slots != nullptr || a.defer_wait) && pidx == nparts - 1 && warp == (nblk - 1) % NWARPS)
       last_i = (nblk - 1) / NWARPS;
 
     // lane j: physical blocks of this warp's pages j, j + 32, ... (page
@@ -561,7 +572,9 @@ __global__ void __launch_bounds__(NWARPS * 32)
 
     auto issue = [&](int i) {
       const int phys = phys_of(i);
-      if (i == last_i) {  // the step's writes into this page (made below), visible to the TMA read
+      if (i == last_i) {  // the step's writes into this page (made below, or by the
+                          // preceding launch), visible to the TMA read
+        if (a.defer_wait) pdl_wait();
         asm volatile("fence.proxy.async.global;" ::: "memory");
         __syncwarp();
       }
@@ -588,7 +601,7 @@ __global__ void __launch_bounds__(NWARPS * 32)
 #pragma unroll
       for (int i = 0; i < NSTAGE; ++i)
         if (i != last_i) issue(i);
-      fused_step_append<T, D>(a, b, kvh, lane);
+      if (a.slots != nullptr) fused_step_append<T, D>(a, b, kvh, lane);
       if (last_i < NSTAGE) issue(last_i);
     } else {
 #pragma unroll
@@ -773,6 +786,8 @@ __global__ void __launch_bounds__(NWARPS * 32)
     __syncthreads();
     if (__syncthreads_or(timed_out)) break;
   }
+  // with a deferred wait the launch still ends after the one it follows
+  if (a.defer_wait && threadIdx.x == 0) pdl_wait();
 }
 
 }  // namespace pkv

@@ -608,6 +608,7 @@ struct StepWrites {
   const int64_t* slots = nullptr;
   const int32_t* copies = nullptr;
   int n_copies = 0;
+  bool defer = false;  // the writes were launched just before the decode (see DecodeArgs::defer_wait)
 };
 
 void attach_step(pkv::DecodeArgs* a, const StepWrites& w) {
@@ -616,7 +617,10 @@ void attach_step(pkv::DecodeArgs* a, const StepWrites& w) {
   a->slots = w.slots;
   a->copies = w.copies;
   a->n_copies = w.n_copies;
+  a->defer_wait = w.defer ? 1 : 0;
 }
+
+constexpr int kValidateOnly = -2;  // decode_prefix_impl's phase: check the arguments, launch nothing
 
 pkv_status decode_prefix_impl(void* out, const void* q, const void* k_cache, const void* v_cache,
                                              const int32_t* block_tables, int max_blocks_per_seq,
@@ -660,6 +664,7 @@ pkv_status decode_prefix_impl(void* out, const void* q, const void* k_cache, con
   if (static_cast<long long>(a.num_qgroups) * a.num_chunks + static_cast<long long>(num_seqs) * a.suffix_z > 65535)
     return PKV_EINVAL;
 
+  if (phase == kValidateOnly) return PKV_OK;
   const int G = num_q_heads / num_kv_heads;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (dtype == PKV_F16) return dispatch_dim_prefix<__half>(a, head_dim, G, phase, st);
@@ -716,11 +721,27 @@ pkv_status pkv_decode_step(void* out, const void* q, void* k_cache, void* v_cach
   w.slots = slot_mapping;
   w.copies = copies;
   w.n_copies = num_copies;
-  if (prefix_pages > 0)
+  if (prefix_pages > 0) {
+    // the cascade: the copies and the append in their own launch, which
+    // the cascade does not wait for except where it reads what they write
+    // (each sequence's last page): its CTAs stream the prefix and the other
+    // pages meanwhile
+    const pkv_status sv = decode_prefix_impl(out, q, k_cache, v_cache, block_tables, max_blocks_per_seq,
+                                             context_lens, max_context_len, prefix_blocks, prefix_pages, num_seqs,
+                                             num_q_heads, num_kv_heads, head_dim, num_blocks, scale,
+                                             partition_tokens, dtype, workspace, workspace_bytes_given,
+                                             kValidateOnly, stream);
+    if (sv != PKV_OK || num_seqs == 0) return sv;
+    const pkv_status sc = pkv_kv_append_copy(k_new, v_new, k_cache, v_cache, slot_mapping, num_seqs, copies,
+                                             num_copies, num_kv_heads, head_dim, num_blocks, dtype, stream);
+    if (sc != PKV_OK) return sc;
+    StepWrites after;
+    after.defer = true;
     return decode_prefix_impl(out, q, k_cache, v_cache, block_tables, max_blocks_per_seq, context_lens,
                               max_context_len, prefix_blocks, prefix_pages, num_seqs, num_q_heads, num_kv_heads,
                               head_dim, num_blocks, scale, partition_tokens, dtype, workspace, workspace_bytes_given,
-                              -1, stream, w);
+                              -1, stream, after);
+  }
   pkv::DecodeArgs a{};
   long long P = 0;
   const pkv_status st0 = prepare_decode(out, q, k_cache, v_cache, block_tables, max_blocks_per_seq, context_lens,
