@@ -17,8 +17,8 @@
 // CTAs per SM claims items from an atomic counter until the list runs out.
 // Six warps with fixed jobs, walking the same items in the same order:
 //   warp 0      claims the next item, writes its page table and bounds into
-//               a two-slot ring in shared memory, and (lane 0) issues the
-//               TMA copies of its pages, four per key block (64 keys), into
+//               a two-slot ring in shared memory, and issues the TMA copies
+//               of its pages (a box per lane), four per key block (64 keys), into
 //               a K ring and a V ring; a K stage is free again once its
 //               block's scores are formed, a V stage once its P.V is done,
 //               so the K loads run ahead of the S-buffer turnaround; over an
@@ -457,11 +457,11 @@ __global__ void __launch_bounds__(TcShape<D, NSK, NSV>::kThreads, PKV_TC_MIN_CTA
 
   if (warp == 0) {
     // ---- producer (the whole warp): claims items, describes them, and
-    // (lane 0) issues their K and V copies ------------------------------------
+    // issues their K and V copies (one TMA box per lane) -----------------------
     // A K stage is released as soon as the block's S = Q.K^T MMAs are done,
     // a V stage once its P.V MMAs are done, so K runs up to NSK blocks
     // ahead of the scores and V up to NSV blocks ahead of the P.V products;
-    // one thread polls both rings, so a V stage that frees late never holds
+    // one loop polls both rings, so a V stage that frees late never holds
     // back the next K copy, and the next item's copies start as soon as the
     // rings have room.
     for (int it = 0; !bad; ++it) {
