@@ -87,6 +87,10 @@ struct Fp8Shape {
   static_assert(kTile % 512 == 0, "swizzled tiles want 512/1024-byte alignment");
 };
 
+#ifndef PKV_FP8_PACK
+#define PKV_FP8_PACK 1
+#endif
+
 // CTAs per SM the FP8 kernel's register budget is sized for
 #ifndef PKV_FP8_MIN_CTAS
 #define PKV_FP8_MIN_CTAS 8
@@ -107,6 +111,15 @@ __global__ void __launch_bounds__(NWARPS * 32, PKV_FP8_MIN_CTAS)
   using S = Fp8Shape<D, NWARPS, NSTAGE>;
   using M = Mma<__half>;      // the MMAs run in fp16 (see above)
   constexpr int kNT = D / 8;  // PV n-tiles; also the d values a column spans
+  // kPack (G <= 4): the spare query columns [G, 2G) repeat queries [0, G)
+  // (identical scores, max and sum), carry P's lo part where columns
+  // [0, G) carry its hi part, and the two columns' O^T are added at the
+  // end: one P.V MMA per m-tile instead of two.
+#if PKV_FP8_PACK
+  constexpr bool kPack = G <= 4;
+#else
+  constexpr bool kPack = false;
+#endif
   const int kvh = blockIdx.x;
   const int b = blockIdx.y;
   const int part = blockIdx.z;
@@ -157,11 +170,12 @@ __global__ void __launch_bounds__(NWARPS * 32, PKV_FP8_MIN_CTAS)
   // Q^T as fp16 B fragments in the d order the converted K fragments use:
   // chunk c: b0 = q[16c + 4t .. +1], b1 = q[16c + 4t + 2 .. +3].  A bf16
   // row is first scaled by 2^kq (exact) so that it fits fp16.
+  // With kPack the query columns [G, 2G) repeat queries [0, G).
   uint32_t qb[S::kChunks][2];
   int kq = 0;  // this lane's row (query g8): q was multiplied by 2^kq
   {
-    const bool ok = g8 < G;
-    const T* qp = reinterpret_cast<const T*>(a.q) + (ok ? col_row(g8) : 0) * D;
+    const bool ok = g8 < (kPack ? 2 * G : G);
+    const T* qp = reinterpret_cast<const T*>(a.q) + (ok ? col_row(g8 & (G - 1)) : 0) * D;
     float qf[S::kChunks][4];
 #pragma unroll
     for (int c = 0; c < S::kChunks; ++c) {
@@ -319,11 +333,21 @@ __global__ void __launch_bounds__(NWARPS * 32, PKV_FP8_MIN_CTAS)
           o[i][3] *= al1;
         }
       }
-      // (3) P^T as B fragments, split into hi + lo 16-bit parts
+      // (3) P^T as B fragments, split into hi + lo 16-bit parts (kPack:
+      // one fragment, hi in columns [0, G), lo in [G, 2G))
       const uint32_t top_hi = M::pack(p0, p1), bot_hi = M::pack(p2, p3);
       const float2 th = M::unpack(top_hi), bh = M::unpack(bot_hi);
-      const uint32_t top_lo = M::pack(p0 - th.x, p1 - th.y), bot_lo = M::pack(p2 - bh.x, p3 - bh.y);
-      const uint32_t pb0 = movm_t(top_hi), pb1 = movm_t(bot_hi), pl0 = movm_t(top_lo), pl1 = movm_t(bot_lo);
+      uint32_t top_lo, bot_lo;
+      if constexpr (kPack) {
+        const bool h0 = 2 * t4 < G, h1 = 2 * t4 + 1 < G;
+        top_lo = M::pack(h0 ? th.x : p0 - th.x, h1 ? th.y : p1 - th.y);
+        bot_lo = M::pack(h0 ? bh.x : p2 - bh.x, h1 ? bh.y : p3 - bh.y);
+      } else {
+        top_lo = M::pack(p0 - th.x, p1 - th.y);
+        bot_lo = M::pack(p2 - bh.x, p3 - bh.y);
+      }
+      const uint32_t pl0 = movm_t(top_lo), pl1 = movm_t(bot_lo);
+      const uint32_t pb0 = kPack ? 0u : movm_t(top_hi), pb1 = kPack ? 0u : movm_t(bot_hi);
       // (4) bytes d = kNT g8 .. kNT g8 + kNT - 1 (in 16-byte chunk vch, from
       // byte vb0) of rows 2 t4, 2 t4 + 1, 2 t4 + 8, 2 t4 + 9; rows past the
       // context are zeroed (an unused slot may hold a NaN code)
@@ -366,7 +390,7 @@ __global__ void __launch_bounds__(NWARPS * 32, PKV_FP8_MIN_CTAS)
         uint32_t a0, a1, a2, a3;
         e4m3x4_to_f16(lo01, a0, a1);  // tokens 2 t4, 2 t4 + 1 at rows g8, g8 + 8
         e4m3x4_to_f16(lo89, a2, a3);  // tokens 2 t4 + 8, 2 t4 + 9
-        M::run(o[i], a0, a1, a2, a3, pb0, pb1);
+        if constexpr (!kPack) M::run(o[i], a0, a1, a2, a3, pb0, pb1);
         M::run(o[i], a0, a1, a2, a3, pl0, pl1);
       }
     }
@@ -387,6 +411,18 @@ __global__ void __launch_bounds__(NWARPS * 32, PKV_FP8_MIN_CTAS)
     l1 += __shfl_xor_sync(kFull, l1, msk);
   }
 
+  if constexpr (kPack) {  // query n: column n (hi) + column n + G (lo)
+#pragma unroll
+    for (int i = 0; i < kMT; ++i) {
+      if constexpr (G == 1) {
+        o[i][0] += o[i][1];
+        o[i][2] += o[i][3];
+      } else {
+#pragma unroll
+        for (int e = 0; e < 4; ++e) o[i][e] += __shfl_xor_sync(kFull, o[i][e], G / 2);
+      }
+    }
+  }
   // warp record [o: 8 x D][m: 8][l: 8]
   float* rec = reinterpret_cast<float*>(my_stages);
 #pragma unroll
