@@ -404,10 +404,10 @@ pkv_status pkv_selftest_bounded_wait(long long limit_cycles, void* stream);
  *   s_j = scale * k_scale * q . code(K_j),  out = v_scale * sum_j softmax(s)_j code(V_j)
  * Same arguments, layouts, workspace (pkv_decode_workspace_bytes) and errors
  * as pkv_paged_attention_decode, except the auto partition (partition_tokens
- * 0): 1024 tokens, or 2048 when max_context_len > 16384 (an FP8 page is half
- * the bytes, so a work unit covers twice the tokens for the same fixed
- * cost).  A workspace sized by pkv_decode_workspace_bytes with partition 0
- * is large enough for it.
+ * 0): 768 tokens, 1024 when max_context_len > 4096, 2048 when it is
+ * > 16384 (an FP8 page is half the bytes, so a work unit covers more tokens
+ * for the same fixed cost).  A workspace sized by pkv_decode_workspace_bytes
+ * with partition 0 is large enough for it.
  * -------------------------------------------------------------------- */
 pkv_status pkv_kv_append_fp8(const void* k_new, const void* v_new, void* k_cache, void* v_cache,
                              const int64_t* slot_mapping, int num_tokens, int num_kv_heads, int head_dim,
@@ -526,7 +526,8 @@ pkv_status pkv_paged_attention_multi_fp8(void* out, const void* q, const void* k
  * num_kv_heads; 0 if unknown), and is read by those two ops only.
  * Auto rules:
  *   PKV_OP_DECODE         512, or 1024 when max_context_len > 4096;
- *   PKV_OP_DECODE_FP8     1024, or 2048 when max_context_len > 16384;
+ *   PKV_OP_DECODE_FP8     768, 1024 when max_context_len > 4096, 2048 when
+ *                         it is > 16384;
  *   PKV_OP_MULTI          2048, or 1024 when max_context_len > 4096; with
  *                         more than 32 rows per kv-head (the tcgen05
  *                         kernel) 8192;

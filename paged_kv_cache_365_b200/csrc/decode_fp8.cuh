@@ -87,10 +87,6 @@ struct Fp8Shape {
   static_assert(kTile % 512 == 0, "swizzled tiles want 512/1024-byte alignment");
 };
 
-#ifndef PKV_FP8_PACK
-#define PKV_FP8_PACK 1
-#endif
-
 // CTAs per SM the FP8 kernel's register budget is sized for
 #ifndef PKV_FP8_MIN_CTAS
 #define PKV_FP8_MIN_CTAS 8
@@ -115,11 +111,9 @@ __global__ void __launch_bounds__(NWARPS * 32, PKV_FP8_MIN_CTAS)
   // (identical scores, max and sum), carry P's lo part where columns
   // [0, G) carry its hi part, and the two columns' O^T are added at the
   // end: one P.V MMA per m-tile instead of two.
-#if PKV_FP8_PACK
   constexpr bool kPack = G <= 4;
-#else
-  constexpr bool kPack = false;
-#endif
+  // the reference max moves only past 2^kLazyMax (see the softmax below)
+  constexpr float kLazyMax = 8.f;
   const int kvh = blockIdx.x;
   const int b = blockIdx.y;
   const int part = blockIdx.z;
@@ -311,20 +305,23 @@ __global__ void __launch_bounds__(NWARPS * 32, PKV_FP8_MIN_CTAS)
       const float x2 = v_hi ? (sc[2] + sd[2]) * xs0 : -INFINITY;
       const float x3 = v_hi ? (sc[3] + sd[3]) * xs1 : -INFINITY;
       float mx0 = fmaxf(x0, x2), mx1 = fmaxf(x1, x3);
+      // The reference max m of a column moves only when one of the page's
+      // scores passes it by more than kLazyMax (so p <= 2^kLazyMax): most
+      // pages then need one vote, no reduction and no rescale.  Any
+      // reference is exact once the same m scales l and O.
+      if (__any_sync(kFull, mx0 > m0 + kLazyMax || mx1 > m1 + kLazyMax)) {
 #pragma unroll
-      for (int msk = 4; msk <= 16; msk <<= 1) {
-        mx0 = fmaxf(mx0, __shfl_xor_sync(kFull, mx0, msk));
-        mx1 = fmaxf(mx1, __shfl_xor_sync(kFull, mx1, msk));
-      }
-      const float n0 = fmaxf(m0, mx0), n1 = fmaxf(m1, mx1);
-      const float al0 = exp2_sfu(m0 - n0), al1 = exp2_sfu(m1 - n1);
-      m0 = n0;
-      m1 = n1;
-      const float p0 = exp2_sfu(x0 - n0), p1 = exp2_sfu(x1 - n1), p2 = exp2_sfu(x2 - n0), p3 = exp2_sfu(x3 - n1);
-      l0 = fmaf(l0, al0, p0 + p2);
-      l1 = fmaf(l1, al1, p1 + p3);
-      // this lane's O^T columns are its own query columns 2 t4, 2 t4 + 1
-      if (__any_sync(kFull, al0 != 1.f || al1 != 1.f)) {
+        for (int msk = 4; msk <= 16; msk <<= 1) {
+          mx0 = fmaxf(mx0, __shfl_xor_sync(kFull, mx0, msk));
+          mx1 = fmaxf(mx1, __shfl_xor_sync(kFull, mx1, msk));
+        }
+        const float n0 = fmaxf(m0, mx0), n1 = fmaxf(m1, mx1);
+        const float al0 = exp2_sfu(m0 - n0), al1 = exp2_sfu(m1 - n1);
+        m0 = n0;
+        m1 = n1;
+        l0 *= al0;
+        l1 *= al1;
+        // this lane's O^T columns are its own query columns 2 t4, 2 t4 + 1
 #pragma unroll
         for (int i = 0; i < kMT; ++i) {
           o[i][0] *= al0;
@@ -333,6 +330,9 @@ __global__ void __launch_bounds__(NWARPS * 32, PKV_FP8_MIN_CTAS)
           o[i][3] *= al1;
         }
       }
+      const float p0 = exp2_sfu(x0 - m0), p1 = exp2_sfu(x1 - m1), p2 = exp2_sfu(x2 - m0), p3 = exp2_sfu(x3 - m1);
+      l0 += p0 + p2;
+      l1 += p1 + p3;
       // (3) P^T as B fragments, split into hi + lo 16-bit parts (kPack:
       // one fragment, hi in columns [0, G), lo in [G, 2G))
       const uint32_t top_hi = M::pack(p0, p1), bot_hi = M::pack(p2, p3);

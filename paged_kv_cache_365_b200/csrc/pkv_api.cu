@@ -83,10 +83,13 @@ int resolve_multi_partition(int p, long long max_ctx) {
 int resolve_multi_tc_partition(int p, long long max_ctx) {
   return p != 0 ? resolve_partition(p, max_ctx) : PKV_TC_AUTO_PARTITION;
 }
-// Auto partition of the FP8 decode: twice the 16-bit one's tokens (half the
-// bytes a page): 1024, or 2048 past 16384 tokens.
+// Auto partition of the FP8 decode (a page is half the bytes of a 16-bit
+// one): 768 tokens up to 4096 (1.5x the 16-bit rule: short batches keep
+// enough, evenly sized CTAs for the last wave), 1024 up to 16384, 2048
+// past it.  Never more partitions than the 16-bit rule, so its workspace
+// suffices.
 int resolve_fp8_partition(int p, long long max_ctx) {
-  return resolve_partition(p != 0 ? p : (max_ctx > 16384 ? 2048 : 1024), max_ctx);
+  return resolve_partition(p != 0 ? p : (max_ctx > 16384 ? 2048 : max_ctx > 4096 ? 1024 : 768), max_ctx);
 }
 int multi_ntiles(long long rows) { return rows <= 8 ? 1 : 2; }
 int multi_rows_warps(long long rows) { return rows <= 16 ? 0 : rows <= 24 ? 3 : 4; }

@@ -51,9 +51,14 @@ def test_library_partition_rule_and_workspace_sizes():
     for n in (4097, 16384, 131072):
         assert pt(_lib.OP_DECODE, n) == 1024
         assert pt(_lib.OP_MULTI, n) == 1024
-    for n in (1, 16384):
+    for n in (1, 4096):
+        assert pt(_lib.OP_DECODE_FP8, n) == 768
+    for n in (4097, 16384):
         assert pt(_lib.OP_DECODE_FP8, n) == 1024
     assert pt(_lib.OP_DECODE_FP8, 16385) == 2048
+    # never more FP8 partitions than 16-bit ones (one workspace serves both)
+    for n in (1, 700, 769, 1537, 4096, 4097, 9000, 16385, 131072):
+        assert -(-n // pt(_lib.OP_DECODE_FP8, n)) <= -(-n // pt(_lib.OP_DECODE, n))
     # the tcgen05 multi-token kernel (more than 32 rows per kv-head, or an
     # FP8 pool): 8192 tokens at any length; up to 32 rows the rules above
     for n in (1, 4097, 131072):
