@@ -306,16 +306,18 @@ def run_cuda(args, rank, world, local_rank, workload=None, graph=None):
             raise SystemExit("--kv-fp8 needs an fp16 / bf16 workload")
         to_fp8_pool(cache, dev)
     prefix = torch.from_numpy(np.ascontiguousarray(st["host"]["block_tables"][0, :pp])).to(dev) if use_cascade else None
-    # the step through pkv_decode_step: a plain 16-bit step is one launch
-    # (+ merge); the cascade keeps its copies and append in a launch of their
-    # own, which it overlaps (it waits for it only at each sequence's last page)
-    fused_step = not fp8 and wl.dtype != "f32" and not args.unfused and not args.cascade_overlap
+    # the step through pkv_decode_step (pkv_decode_step_fp8 over an FP8
+    # pool): a plain step is one launch (+ merge); the cascade keeps its
+    # copies and append in a launch of their own, which it overlaps (it waits
+    # for it only at each sequence's last page)
+    fused_step = wl.dtype != "f32" and not args.unfused and not args.cascade_overlap
     if use_cascade:
         ws = cache.workspace(pkv.decode_prefix_workspace_bytes(B, Hq, D, max_ctx, pp, args.partition))
         # copies + append (one launch), cascade (one launch, or prefix + suffix passes), merge
         launches_per_step = 1 + (3 if args.cascade_overlap else 2)
     else:
-        launches_per_step = (0 if fused_step else 1) + 1 + (1 if (n_pairs and fp8) else 0) + (1 if P > 1 else 0)
+        launches_per_step = ((0 if fused_step else 1) + 1 + (1 if (n_pairs and fp8 and not fused_step) else 0) +
+                             (1 if P > 1 else 0))
 
     # every call goes to the current stream at call time (so that a CUDA
     # graph capture records it)
@@ -379,6 +381,11 @@ def run_cuda(args, rank, world, local_rank, workload=None, graph=None):
     def eager_step():
         if overlap:
             overlapped(True)
+            return
+        if fused and fp8:
+            pkv.decode_step_fp8(st["q"], cache.k, cache.v, st["k_new"], st["v_new"], st["slot_mapping"],
+                                copies if n_pairs else None, st["block_tables"], st["context_lens"], max_ctx, scale,
+                                FP8_SCALE, FP8_SCALE, out=out, workspace=ws, partition=args.partition)
             return
         if fused:
             pkv.decode_step(st["q"], cache.k, cache.v, st["k_new"], st["v_new"], st["slot_mapping"],
@@ -445,7 +452,7 @@ def run_cuda(args, rank, world, local_rank, workload=None, graph=None):
     # every step, and the output read back every step
     host = {k: st[k].cpu().pin_memory() for k in ("q", "k_new", "v_new", "slot_mapping", "cow_pairs",
                                                     "block_tables", "context_lens")}
-    if n_pairs and not fp8:
+    if n_pairs and (fused_step or not fp8):
         host["cow_pairs"] = torch.from_numpy(copies_host).pin_memory()
     if use_cascade:
         host["prefix_blocks"] = prefix.cpu().pin_memory()

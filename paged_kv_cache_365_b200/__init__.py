@@ -15,4 +15,4 @@ from .api import (BLOCK_SIZE, DEFAULT_PARTITION, BlockAllocator, PagedKVCache, c
                   paged_attention_multi, multi_workspace_bytes, kv_append_fp8, paged_attention_decode_fp8,
                   kv_append_copy, cow_copy_rows, selftest_bounded_wait, cascade_prefix_pages,
                   partition_tokens, decode_step, paged_attention_decode_prefix_fp8,
-                  decode_prefix_fp8_workspace_bytes, paged_attention_multi_fp8)
+                  decode_prefix_fp8_workspace_bytes, paged_attention_multi_fp8, decode_step_fp8)

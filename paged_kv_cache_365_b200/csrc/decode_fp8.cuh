@@ -71,6 +71,81 @@ __device__ __forceinline__ uint32_t swz8(int row, int chunk) {
     return static_cast<uint32_t>(row * 64 + ((chunk ^ ((row >> 1) & 3)) << 4));
 }
 
+// Eight 16-bit values (T) to eight E4M3 codes: code = E4M3(x / scale), the
+// division in float32, nearest value, ties to even, saturating at +-448.
+template <typename T>
+__device__ __forceinline__ uint2 quant8_e4m3(uint4 in, float scale) {
+  const uint32_t w[4] = {in.x, in.y, in.z, in.w};
+  uint32_t packed[2];
+#pragma unroll
+  for (int p = 0; p < 2; ++p) {
+    unsigned short q2[2];
+#pragma unroll
+    for (int hh = 0; hh < 2; ++hh) {
+      const float2 f = Mma<T>::unpack(w[2 * p + hh]);
+      const float x0 = __fdiv_rn(f.x, scale), x1 = __fdiv_rn(f.y, scale);
+      // first operand -> upper byte, second -> lower byte
+      asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(q2[hh]) : "f"(x1), "f"(x0));
+    }
+    packed[p] = static_cast<uint32_t>(q2[0]) | (static_cast<uint32_t>(q2[1]) << 16);
+  }
+  return make_uint2(packed[0], packed[1]);
+}
+
+// The step's writes over an FP8 pool (pkv_decode_step_fp8), made by the one
+// warp that later stages sequence b's last page, as fused_step_append does
+// for a 16-bit pool: rows 0 .. rows-1 of the copy whose destination is the
+// slot's block (codes, copied as bytes), then the new token quantised as
+// quant8_e4m3 does.  The caller fences them for the async proxy before
+// that page's TMA load.
+template <typename T, int D>
+__device__ __forceinline__ void fused_step_append_fp8(const DecodeArgs& a, int b, int kvh, int lane, float k_scale,
+                                                      float v_scale) {
+  constexpr int kRowChunks = D / 16;  // 16-byte chunks of a row of codes
+  const int64_t s = a.slots[b];
+  const int64_t blk = s >= 0 ? s / kBlockSize : -1;
+  const bool ok = s >= 0 && blk < a.num_blocks;
+  if (s >= 0 && !ok && lane == 0) raise_error(PKV_ERR_SLOT_RANGE);
+  if (!ok) return;
+  int first = 0x7fffffff;
+  for (int i = lane; i < a.n_copies; i += 32)
+    if (a.copies[3 * i + 1] == static_cast<int>(blk)) first = min(first, i);
+#pragma unroll
+  for (int m = 16; m >= 1; m >>= 1) first = min(first, __shfl_xor_sync(kFull, first, m));
+  int src = -1, rows = 0;
+  if (first != 0x7fffffff) {
+    src = a.copies[3 * first];
+    rows = a.copies[3 * first + 2];
+  }
+  if (src >= 0 && (src >= a.num_blocks || rows < 0 || rows > kBlockSize)) {
+    if (lane == 0) raise_error(PKV_ERR_COPY_RANGE);
+    src = -1;
+  }
+  const size_t head = static_cast<size_t>(kBlockSize) * kRowChunks;  // chunks of one (block, kv-head) tile
+  uint4* kc = reinterpret_cast<uint4*>(const_cast<unsigned char*>(a.k_cache));
+  uint4* vc = reinterpret_cast<uint4*>(const_cast<unsigned char*>(a.v_cache));
+  if (src >= 0) {
+    const size_t from = (static_cast<size_t>(src) * a.num_kv_heads + kvh) * head;
+    const size_t to = (static_cast<size_t>(blk) * a.num_kv_heads + kvh) * head;
+    for (int e = lane; e < 2 * rows * kRowChunks; e += 32) {
+      uint4* c = e < rows * kRowChunks ? kc : vc;
+      const int k = e < rows * kRowChunks ? e : e - rows * kRowChunks;
+      c[to + k] = c[from + k];
+    }
+  }
+  __syncwarp();  // (the token's row may lie inside the copied rows)
+  // the token: 8 elements (16 bytes in, 8 codes out) a lane and tensor
+  constexpr int kIn = D / 8;
+  const size_t row = ((static_cast<size_t>(blk) * a.num_kv_heads + kvh) * kBlockSize + s % kBlockSize) * kIn;
+  const size_t in = (static_cast<size_t>(b) * a.num_kv_heads + kvh) * kIn;
+  for (int e = lane; e < 2 * kIn; e += 32) {
+    const bool is_v = e >= kIn;
+    const int c = is_v ? e - kIn : e;
+    const uint4 x = reinterpret_cast<const uint4*>(is_v ? a.v_new : a.k_new)[in + c];
+    reinterpret_cast<uint2*>(is_v ? vc : kc)[row + c] = quant8_e4m3<T>(x, is_v ? v_scale : k_scale);
+  }
+}
+
 template <int D, int NWARPS, int NSTAGE>
 struct Fp8Shape {
   static constexpr int kTile = kBlockSize * D;  // bytes of a (block, kv-head) tile
@@ -102,7 +177,7 @@ struct Fp8Shape {
 template <typename T, int D, int G, int NWARPS, int NSTAGE, bool kCascade = false>
 __global__ void __launch_bounds__(NWARPS * 32, PKV_FP8_MIN_CTAS)
     paged_decode_fp8_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tmap_k,
-                            const __grid_constant__ CUtensorMap tmap_v, float v_scale) {
+                            const __grid_constant__ CUtensorMap tmap_v, float v_scale, float k_scale) {
   pdl_enter();
   using S = Fp8Shape<D, NWARPS, NSTAGE>;
   using M = Mma<__half>;      // the MMAs run in fp16 (see above)
@@ -234,9 +309,19 @@ __global__ void __launch_bounds__(NWARPS * 32, PKV_FP8_MIN_CTAS)
     }
     return r;
   };
+  // a fused step (pkv_decode_step_fp8): the warp that stages the sequence's
+  // last page (page nblk - 1 of the last partition, its page last_i) makes
+  // the step's writes first and fences them before that page's TMA load
+  int last_i = -1;
+  if constexpr (!kCascade)
+    if (a.slots != nullptr && part == nparts - 1 && warp == (nblk - 1) % NWARPS) last_i = (nblk - 1) / NWARPS;
   uint32_t phase_bits = 0;
   auto issue = [&](int i) {
     const int phys = phys_of(i);
+    if (i == last_i) {
+      asm volatile("fence.proxy.async.global;" ::: "memory");
+      __syncwarp();
+    }
     if (lane == 0 && i < my_n) {
       const uint32_t bar = bar0 + 8 * (i % NSTAGE);
       if (phys >= 0) {
@@ -251,8 +336,18 @@ __global__ void __launch_bounds__(NWARPS * 32, PKV_FP8_MIN_CTAS)
       }
     }
   };
+  if (last_i >= 0) {
+    // the warp's first pages go out before the writes, whose latency
+    // overlaps them; the last page waits for them
 #pragma unroll
-  for (int i = 0; i < NSTAGE; ++i) issue(i);
+    for (int i = 0; i < NSTAGE; ++i)
+      if (i != last_i) issue(i);
+    fused_step_append_fp8<T, D>(a, b, kvh, lane, k_scale, v_scale);
+    if (last_i < NSTAGE) issue(last_i);
+  } else {
+#pragma unroll
+    for (int i = 0; i < NSTAGE; ++i) issue(i);
+  }
 
   // O^T accumulators: m-tile i, rows g8 / g8 + 8 -> d = kNT g8 + 2i / + 1,
   // columns 2 t4, 2 t4 + 1 (queries)
@@ -546,23 +641,8 @@ __global__ void __launch_bounds__(256)
       continue;
     }
     const uint4 in = (is_v ? v_new : k_new)[j];
-    const float sc = is_v ? v_scale : k_scale;
-    const uint32_t w[4] = {in.x, in.y, in.z, in.w};
-    uint32_t packed[2];
-#pragma unroll
-    for (int p = 0; p < 2; ++p) {
-      unsigned short q2[2];
-#pragma unroll
-      for (int hh = 0; hh < 2; ++hh) {
-        const float2 f = Mma<T>::unpack(w[2 * p + hh]);
-        const float x0 = __fdiv_rn(f.x, sc), x1 = __fdiv_rn(f.y, sc);
-        // first operand -> upper byte, second -> lower byte
-        asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(q2[hh]) : "f"(x1), "f"(x0));
-      }
-      packed[p] = static_cast<uint32_t>(q2[0]) | (static_cast<uint32_t>(q2[1]) << 16);
-    }
     const long long dst = ((blk * Hkv + h) * kBlockSize + off) * row_chunks + c;
-    (is_v ? v_cache : k_cache)[dst] = make_uint2(packed[0], packed[1]);
+    (is_v ? v_cache : k_cache)[dst] = quant8_e4m3<T>(in, is_v ? v_scale : k_scale);
   }
 }
 

@@ -244,7 +244,7 @@ bool encode_fp8_map(CUtensorMap* map, const void* base, int D, long long rows) {
 constexpr int kFp8Stages = PKV_FP8_STAGES;  // pages in flight per warp (4 KB each at D = 128)
 
 template <typename T, int D, int G>
-pkv_status launch_decode_fp8(const pkv::DecodeArgs& a, float v_scale, cudaStream_t st) {
+pkv_status launch_decode_fp8(const pkv::DecodeArgs& a, float k_scale, float v_scale, cudaStream_t st) {
   using S = pkv::Fp8Shape<D, kMmaWarps, kFp8Stages>;
   CUtensorMap mk, mv;
   const long long rows = static_cast<long long>(a.num_blocks) * a.num_kv_heads * PKV_BLOCK_SIZE;
@@ -254,7 +254,8 @@ pkv_status launch_decode_fp8(const pkv::DecodeArgs& a, float v_scale, cudaStream
       cudaSuccess)
     return PKV_ECUDA;
   const dim3 grid(a.num_kv_heads, a.num_seqs, a.num_parts);
-  if (launch(kfn, grid, dim3(kMmaWarps * 32), S::kSmem, st, a, mk, mv, v_scale) != PKV_OK) return PKV_ECUDA;
+  if (launch(kfn, grid, dim3(kMmaWarps * 32), S::kSmem, st, a, mk, mv, v_scale, k_scale) != PKV_OK)
+    return PKV_ECUDA;
   if (a.num_parts > 1) {
     if (launch_merge<T, D, ReduceK>(a, a.num_parts, st) != PKV_OK) return PKV_ECUDA;
   }
@@ -310,7 +311,7 @@ pkv_status launch_decode_prefix_fp8(const pkv::DecodeArgs& a0, void* mini_k, voi
         cudaSuccess)
       return PKV_ECUDA;
     if (launch(kfn, dim3(a0.num_kv_heads, a0.num_seqs, a0.num_parts), dim3(kMmaWarps * 32), S::kSmem, st, a0, mk,
-               mv, v_scale) != PKV_OK)
+               mv, v_scale, 1.f) != PKV_OK)
       return PKV_ECUDA;
   }
   return launch_merge<T, D, PrefixMergeK>(a0, a0.num_chunks + a0.num_parts, st);
@@ -346,12 +347,12 @@ PrefixFp8Layout prefix_fp8_layout(long long B, long long Hq, long long Hkv, long
 }
 
 template <typename T, int D>
-pkv_status dispatch_group_fp8(const pkv::DecodeArgs& a, int G, float v_scale, cudaStream_t st) {
+pkv_status dispatch_group_fp8(const pkv::DecodeArgs& a, int G, float k_scale, float v_scale, cudaStream_t st) {
   switch (G) {
-    case 1: return launch_decode_fp8<T, D, 1>(a, v_scale, st);
-    case 2: return launch_decode_fp8<T, D, 2>(a, v_scale, st);
-    case 4: return launch_decode_fp8<T, D, 4>(a, v_scale, st);
-    case 8: return launch_decode_fp8<T, D, 8>(a, v_scale, st);
+    case 1: return launch_decode_fp8<T, D, 1>(a, k_scale, v_scale, st);
+    case 2: return launch_decode_fp8<T, D, 2>(a, k_scale, v_scale, st);
+    case 4: return launch_decode_fp8<T, D, 4>(a, k_scale, v_scale, st);
+    case 8: return launch_decode_fp8<T, D, 8>(a, k_scale, v_scale, st);
   }
   return PKV_EINVAL;
 }
@@ -1084,13 +1085,15 @@ pkv_status pkv_kv_append_fp8(const void* k_new, const void* v_new, void* k_cache
   return run(pkv::kv_append_fp8_kernel<__nv_bfloat16>);
 }
 
-pkv_status pkv_paged_attention_decode_fp8(void* out, const void* q, const void* k_cache, const void* v_cache,
-                                          const int32_t* block_tables, int max_blocks_per_seq,
-                                          const int32_t* context_lens, int max_context_len, int num_seqs,
-                                          int num_q_heads, int num_kv_heads, int head_dim, int num_blocks,
-                                          float scale, float k_scale, float v_scale, int partition_tokens,
-                                          pkv_dtype q_dtype, void* workspace, size_t workspace_bytes_given,
-                                          void* stream) {
+}  // extern "C"
+
+namespace {
+pkv_status decode_fp8_impl(void* out, const void* q, const void* k_cache, const void* v_cache,
+                           const int32_t* block_tables, int max_blocks_per_seq, const int32_t* context_lens,
+                           int max_context_len, int num_seqs, int num_q_heads, int num_kv_heads, int head_dim,
+                           int num_blocks, float scale, float k_scale, float v_scale, int partition_tokens,
+                           pkv_dtype q_dtype, void* workspace, size_t workspace_bytes_given, void* stream,
+                           const StepWrites& w = StepWrites{}) {
   if (q_dtype != PKV_F16 && q_dtype != PKV_BF16) return PKV_EINVAL;
   if (!std::isfinite(k_scale) || !std::isfinite(v_scale) || !(k_scale > 0.f) || !(v_scale > 0.f))
     return PKV_EINVAL;
@@ -1110,15 +1113,52 @@ pkv_status pkv_paged_attention_decode_fp8(void* out, const void* q, const void* 
                                               static_cast<size_t>(num_seqs) * num_q_heads * P * head_dim)
                  : nullptr;
   a.qk_scale *= k_scale;
+  attach_step(&a, w);
   const int G = num_q_heads / num_kv_heads;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   auto run = [&](auto tag) -> pkv_status {
     using T = decltype(tag);
-    if (head_dim == 64) return dispatch_group_fp8<T, 64>(a, G, v_scale, st);
-    return dispatch_group_fp8<T, 128>(a, G, v_scale, st);
+    if (head_dim == 64) return dispatch_group_fp8<T, 64>(a, G, k_scale, v_scale, st);
+    return dispatch_group_fp8<T, 128>(a, G, k_scale, v_scale, st);
   };
   if (q_dtype == PKV_F16) return run(__half{});
   return run(__nv_bfloat16{});
+}
+}  // namespace
+
+extern "C" {
+
+pkv_status pkv_paged_attention_decode_fp8(void* out, const void* q, const void* k_cache, const void* v_cache,
+                                          const int32_t* block_tables, int max_blocks_per_seq,
+                                          const int32_t* context_lens, int max_context_len, int num_seqs,
+                                          int num_q_heads, int num_kv_heads, int head_dim, int num_blocks,
+                                          float scale, float k_scale, float v_scale, int partition_tokens,
+                                          pkv_dtype q_dtype, void* workspace, size_t workspace_bytes_given,
+                                          void* stream) {
+  return decode_fp8_impl(out, q, k_cache, v_cache, block_tables, max_blocks_per_seq, context_lens, max_context_len,
+                         num_seqs, num_q_heads, num_kv_heads, head_dim, num_blocks, scale, k_scale, v_scale,
+                         partition_tokens, q_dtype, workspace, workspace_bytes_given, stream);
+}
+
+pkv_status pkv_decode_step_fp8(void* out, const void* q, void* k_cache, void* v_cache, const void* k_new,
+                               const void* v_new, const int64_t* slot_mapping, const int32_t* copies, int num_copies,
+                               const int32_t* block_tables, int max_blocks_per_seq, const int32_t* context_lens,
+                               int max_context_len, int num_seqs, int num_q_heads, int num_kv_heads, int head_dim,
+                               int num_blocks, float scale, float k_scale, float v_scale, int partition_tokens,
+                               pkv_dtype q_dtype, void* workspace, size_t workspace_bytes_given, void* stream) {
+  if (num_copies < 0 || num_copies > num_seqs) return PKV_EINVAL;
+  if (num_seqs > 0 && (!k_new || !v_new || !slot_mapping || !aligned16(k_new) || !aligned16(v_new)))
+    return PKV_EINVAL;
+  if (num_copies > 0 && copies == nullptr) return PKV_EINVAL;
+  StepWrites w;
+  w.k_new = k_new;
+  w.v_new = v_new;
+  w.slots = slot_mapping;
+  w.copies = copies;
+  w.n_copies = num_copies;
+  return decode_fp8_impl(out, q, k_cache, v_cache, block_tables, max_blocks_per_seq, context_lens, max_context_len,
+                         num_seqs, num_q_heads, num_kv_heads, head_dim, num_blocks, scale, k_scale, v_scale,
+                         partition_tokens, q_dtype, workspace, workspace_bytes_given, stream, w);
 }
 
 }  // extern "C"

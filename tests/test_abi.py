@@ -252,6 +252,24 @@ def test_decode_step_rejections(lib):
     assert lib.pkv_decode_step(*a) == 1
 
 
+def test_decode_step_fp8_rejections(lib):
+    """pkv_decode_step_fp8 checks the step's writes, the two scales and the
+    FP8 decode's arguments before anything is launched."""
+    f = ctypes.c_float
+    ok = [FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 2, FAKE, 8, FAKE, 100, 4, 8, 2, 128, 64, f(0.1), f(0.05),
+          f(0.05), 0, 1, None, 0, None]
+    for idx, bad in ((22, 0), (22, 3), (8, -1), (8, 5), (7, None), (4, None), (5, ODD), (6, None), (16, 96),
+                     (15, 3), (12, 8 * 16 + 1), (19, f(0.0)), (20, f(float("inf"))), (20, f(float("nan"))),
+                     (19, f(-1.0))):
+        a = list(ok)
+        a[idx] = bad
+        assert lib.pkv_decode_step_fp8(*a) == 1, (idx, bad)
+    # a context past one partition needs the workspace
+    a = list(ok)
+    a[10], a[12] = 128, 2000
+    assert lib.pkv_decode_step_fp8(*a) == 1
+
+
 def test_multi_fp8_rejections(lib):
     """pkv_paged_attention_multi_fp8: the multi-token argument checks plus
     the two scales (finite, > 0), all before any CUDA call."""

@@ -425,3 +425,72 @@ def test_multi_step_over_an_fp8_pool_through_the_cache_api():
     want = oracle.paged_multi(q, dev.k, dev.v, tables, lens, qs, D ** -0.5, "bf16", kv_dtype="e4m3", k_scale=ks,
                               v_scale=vs)
     assert np.abs(out.float().numpy() - want).max() <= TOL["bf16"]
+
+
+STEP_CASES = [  # (name, dtype, Hq, Hkv, D, partition)
+    ("fp8_step_f16_G4", "f16", 8, 2, 128, 0),
+    ("fp8_step_bf16_G2_split", "bf16", 8, 4, 64, 64),
+    ("fp8_step_bf16_G8", "bf16", 8, 1, 128, 0),
+    ("fp8_step_f16_G1_split", "f16", 4, 4, 128, 32),
+]
+
+
+@pytest.mark.parametrize("case", STEP_CASES, ids=lambda c: c[0])
+def test_fused_fp8_step_matches_separate_calls(case):
+    """pkv_decode_step_fp8 (the copy-on-write copies, the quantising append
+    and the FP8 decode in one launch) against copy_blocks, kv_append_fp8
+    and paged_attention_decode_fp8 on the same FP8 pool: every token row of
+    the pool and the output bit-identical; the output within tolerance of
+    the oracle, whose FP8 pool is its own replay of the workload with every
+    token row quantised by oracle.fp8.quantize."""
+    import workloads
+    from paged_kv_cache_365_b200.replay import build_step
+    m = pkv()
+    name, dt, Hq, Hkv, D, partition = case
+    wl = workloads.prefix13b(seed=71, B=10, prefix_tokens=256, suffix_range=(1, 300), Hq=Hq, Hkv=Hkv, D=D,
+                             dtype=dt, name=name)
+    ks, vs = 0.011, 0.017
+    vals = workloads.draw_values(wl)
+    st = build_step(wl, vals, "cuda")
+    c = st["cache"]
+    copies = m.cow_copy_rows(st["host"]["cow_pairs"], st["host"]["step_slots"])
+    assert len(copies) > 0
+    dcopies = torch.from_numpy(copies).cuda()
+    tables, lens = st["host"]["block_tables"], st["host"]["context_lens"]
+    nb = c.k.shape[0]
+    # the 16-bit pool before the step, quantised row by row
+    rows_k = c.k.permute(0, 2, 1, 3).reshape(nb * 16, wl.Hkv, D).contiguous()
+    rows_v = c.v.permute(0, 2, 1, 3).reshape(nb * 16, wl.Hkv, D).contiguous()
+    slots_all = torch.arange(nb * 16, dtype=torch.int64, device="cuda")
+    kf = torch.full((nb, wl.Hkv, 16, D), 0x7F, dtype=torch.uint8, device="cuda")
+    vf = torch.full_like(kf, 0x7F)
+    m.kv_append_fp8(rows_k, rows_v, kf, vf, slots_all, ks, vs)
+    kf2, vf2 = kf.clone(), vf.clone()
+    m.copy_blocks(kf2, vf2, st["cow_pairs"])
+    m.kv_append_fp8(st["k_new"], st["v_new"], kf2, vf2, st["slot_mapping"], ks, vs)
+    sep = m.paged_attention_decode_fp8(st["q"], kf2, vf2, st["block_tables"], st["context_lens"],
+                                       st["max_context_len"], wl.scale, ks, vs, partition=partition)
+    fused = m.decode_step_fp8(st["q"], kf, vf, st["k_new"], st["v_new"], st["slot_mapping"], dcopies,
+                              st["block_tables"], st["context_lens"], st["max_context_len"], wl.scale, ks, vs,
+                              partition=partition)
+    torch.cuda.synchronize()
+    assert m.get_error() == 0
+    assert torch.equal(fused.view(torch.int16), sep.view(torch.int16))
+    gk, gv, sk, sv = (t.cpu().numpy() for t in (kf, vf, kf2, vf2))
+    ref = oracle.replay(wl, vals)
+    rk = oracle.RefCache(nb, wl.Hkv, D, "e4m3")
+    for b in range(wl.B):
+        tok = np.arange(int(lens[b]))
+        blk, off = tables[b, tok // 16], tok % 16
+        assert np.array_equal(gk[blk, :, off], sk[blk, :, off])
+        assert np.array_equal(gv[blk, :, off], sv[blk, :, off])
+        rk.append_fp8(ref["cache"].k[blk, :, off], ref["cache"].v[blk, :, off],
+                      blk.astype(np.int64) * 16 + off, wl.dtype, ks, vs)
+    for b in range(wl.B):
+        tok = np.arange(int(lens[b]))
+        blk, off = tables[b, tok // 16], tok % 16
+        assert np.array_equal(gk[blk, :, off], rk.k[blk, :, off])
+        assert np.array_equal(gv[blk, :, off], rk.v[blk, :, off])
+    want = oracle.paged_decode(vals["q"], rk.k, rk.v, ref["block_tables"], ref["context_lens"], wl.scale, wl.dtype,
+                               kv_dtype="e4m3", k_scale=ks, v_scale=vs)
+    assert np.abs(fused.float().cpu().numpy() - want).max() <= TOL[dt]
