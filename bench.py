@@ -297,7 +297,7 @@ def run_cuda(args, rank, world, local_rank, workload=None, graph=None):
     # a batch that shares leading blocks is decoded with the cascade (the
     # shared prefix is read once per kv-head) when the library says so
     pp = pkv.cascade_prefix_pages(st["host"]["block_tables"], st["host"]["context_lens"], cache.dtype)
-    use_cascade = pp > 0 and not args.no_cascade and not args.kv_fp8
+    use_cascade = pp > 0 and not args.no_cascade
     if use_cascade:
         part_tokens = pkv.partition_tokens(pkv._lib.OP_DECODE_PREFIX, max_ctx, args.partition, pp)
     fp8 = bool(args.kv_fp8)
@@ -311,7 +311,15 @@ def run_cuda(args, rank, world, local_rank, workload=None, graph=None):
     # copies and append in a launch of their own, which it overlaps (it waits
     # for it only at each sequence's last page)
     fused_step = wl.dtype != "f32" and not args.unfused and not args.cascade_overlap
-    if use_cascade:
+    if use_cascade and fp8:
+        # the FP8 cascade: the prefix widened to 16 bits, the prefix pass,
+        # the suffix pass beside it (making the step's copies and append when
+        # fused), the merge
+        if args.cascade_overlap:
+            raise SystemExit("--cascade-overlap takes a 16-bit pool")
+        ws = cache.workspace(pkv.decode_prefix_fp8_workspace_bytes(B, Hq, wl.Hkv, D, max_ctx, pp, args.partition))
+        launches_per_step = (0 if fused_step else (1 if n_pairs else 0) + 1) + 4
+    elif use_cascade:
         ws = cache.workspace(pkv.decode_prefix_workspace_bytes(B, Hq, D, max_ctx, pp, args.partition))
         # copies + append (one launch), cascade (one launch, or prefix + suffix passes), merge
         launches_per_step = 1 + (3 if args.cascade_overlap else 2)
@@ -364,7 +372,11 @@ def run_cuda(args, rank, world, local_rank, workload=None, graph=None):
         if overlap:
             overlapped(False)
             return
-        if fp8:
+        if fp8 and use_cascade:
+            pkv.paged_attention_decode_prefix_fp8(st["q"], cache.k, cache.v, st["block_tables"], st["context_lens"],
+                                                  max_ctx, prefix, scale, FP8_SCALE, FP8_SCALE, out=out, workspace=ws,
+                                                  partition=args.partition)
+        elif fp8:
             pkv.paged_attention_decode_fp8(st["q"], cache.k, cache.v, st["block_tables"], st["context_lens"],
                                            max_ctx, scale, FP8_SCALE, FP8_SCALE, out=out, workspace=ws,
                                            partition=args.partition)
@@ -385,7 +397,8 @@ def run_cuda(args, rank, world, local_rank, workload=None, graph=None):
         if fused and fp8:
             pkv.decode_step_fp8(st["q"], cache.k, cache.v, st["k_new"], st["v_new"], st["slot_mapping"],
                                 copies if n_pairs else None, st["block_tables"], st["context_lens"], max_ctx, scale,
-                                FP8_SCALE, FP8_SCALE, out=out, workspace=ws, partition=args.partition)
+                                FP8_SCALE, FP8_SCALE, prefix_blocks=prefix if use_cascade else None, out=out,
+                                workspace=ws, partition=args.partition)
             return
         if fused:
             pkv.decode_step(st["q"], cache.k, cache.v, st["k_new"], st["v_new"], st["slot_mapping"],
@@ -1114,7 +1127,9 @@ def step_figures(args, r, world):
     dec_bytes = decode_algorithmic_bytes(wl, unique=True, fp8=fp8)
     achieved = dec_bytes / (r["dec_avg_ms"] / 1e3) / 1e9
     e2e_step_s = r["e2e_ms"] / 1e3 / K
-    kernel = ("paged_decode cascade (prefix/suffix kernel + merge kernel)" if r["cascade_pages"]
+    kernel = ("paged_decode_fp8 cascade (prefix widening, prefix pass, suffix pass, merge kernels)"
+              if r["cascade_pages"] and fp8
+              else "paged_decode cascade (prefix/suffix kernel + merge kernel)" if r["cascade_pages"]
               else "paged_decode_fp8 (partition + merge kernels)" if fp8
               else "paged_decode (partition + merge kernels)")
     return {

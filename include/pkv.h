@@ -420,29 +420,34 @@ pkv_status pkv_paged_attention_decode_fp8(void* out, const void* q, const void* 
                                           pkv_dtype q_dtype, void* workspace, size_t workspace_bytes,
                                           void* stream);
 
-/* pkv_decode_step_fp8 -- pkv_decode_step over an FP8 cache, without a
- * shared prefix: one launch (plus the merge) makes the step's copy-on-write
- * copies, quantises and appends the new token and decodes.
+/* pkv_decode_step_fp8 -- pkv_decode_step over an FP8 cache: the step's
+ * copy-on-write copies, the quantised append of the new token and the
+ * decode, with no launch of their own for the copies and the append.
  *
  * Same passages as pkv_decode_step.  The result -- the pool and out -- is
  * that of pkv_kv_append_copy's copies (whole rows of codes), then
  * pkv_kv_append_fp8(k_new, v_new, ..., k_scale, v_scale), then
- * pkv_paged_attention_decode_fp8: the CTA that reads a sequence's last page
- * first copies rows 0 .. rows-1 of the copy whose dst is slot_mapping[b]'s
- * block, then writes the token's codes (E4M3(x / scale), as
- * pkv_kv_append_fp8 rounds them), then stages the page.
+ * pkv_paged_attention_decode_fp8 (prefix_pages == 0) or
+ * pkv_paged_attention_decode_prefix_fp8 (prefix_pages > 0): the CTA that
+ * reads a sequence's last page (in the cascade: of its suffix pass) first
+ * copies rows 0 .. rows-1 of the copy whose dst is slot_mapping[b]'s block,
+ * then writes the token's codes (E4M3(x / scale), as pkv_kv_append_fp8
+ * rounds them), then stages the page.  The slots must not write into the
+ * shared prefix blocks (an allocator's step never does).
  * k_new, v_new [num_seqs, num_kv_heads, head_dim] in q_dtype (fp16 or
  * bf16); slot_mapping int64 [num_seqs] (< 0: no token); copies int32
  * [num_copies][3] (device, num_copies <= num_seqs) as for pkv_decode_step.
- * The other arguments, the workspace (pkv_decode_workspace_bytes) and the
- * errors are those of pkv_paged_attention_decode_fp8 and pkv_decode_step.
+ * The other arguments, the workspace (pkv_decode_workspace_bytes, or
+ * pkv_decode_prefix_fp8_workspace_bytes when prefix_pages > 0) and the
+ * errors are those of the FP8 decode called and of pkv_decode_step.
  * -------------------------------------------------------------------- */
 pkv_status pkv_decode_step_fp8(void* out, const void* q, void* k_cache, void* v_cache, const void* k_new,
                                const void* v_new, const int64_t* slot_mapping, const int32_t* copies, int num_copies,
                                const int32_t* block_tables, int max_blocks_per_seq, const int32_t* context_lens,
-                               int max_context_len, int num_seqs, int num_q_heads, int num_kv_heads, int head_dim,
-                               int num_blocks, float scale, float k_scale, float v_scale, int partition_tokens,
-                               pkv_dtype q_dtype, void* workspace, size_t workspace_bytes, void* stream);
+                               int max_context_len, const int32_t* prefix_blocks, int prefix_pages, int num_seqs,
+                               int num_q_heads, int num_kv_heads, int head_dim, int num_blocks, float scale,
+                               float k_scale, float v_scale, int partition_tokens, pkv_dtype q_dtype, void* workspace,
+                               size_t workspace_bytes, void* stream);
 
 /* ------------------------------------------------------------------------
  * pkv_paged_attention_decode_prefix_fp8 -- the shared-prefix (cascade)
@@ -602,8 +607,9 @@ pkv_status pkv_common_prefix_pages(const int32_t* block_tables, int num_seqs, in
 /* pkv_cascade_prefix_pages -- the prefix pages to give
  * pkv_paged_attention_decode_prefix for this batch, or 0 when the plain
  * decode is the better call: the common prefix of pkv_common_prefix_pages
- * when dtype is PKV_F16 / PKV_BF16 (the cascade's tensor-core path), at
- * least PKV_CASCADE_MIN_SEQS sequences share it and it spans at least
+ * when dtype is PKV_F16 / PKV_BF16 (the cascade's tensor-core path) or
+ * PKV_E4M3 (pkv_paged_attention_decode_prefix_fp8), at least
+ * PKV_CASCADE_MIN_SEQS sequences share it and it spans at least
  * PKV_CASCADE_MIN_PAGES pages (below that the prefix pass and the merge
  * cost more than reading the few shared pages once per sequence). */
 #define PKV_CASCADE_MIN_PAGES 8

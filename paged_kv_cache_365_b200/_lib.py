@@ -81,8 +81,9 @@ PROTOTYPES = {
                                 c_int, c_void_p, c_int, c_void_p, c_int, c_void_p, c_int, c_int, c_int, c_int,
                                 c_int, c_int, c_float, c_int, c_int, c_void_p, c_size_t, c_void_p]),
     "pkv_decode_step_fp8": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
-                                    c_void_p, c_int, c_void_p, c_int, c_void_p, c_int, c_int, c_int, c_int, c_int,
-                                    c_int, c_float, c_float, c_float, c_int, c_int, c_void_p, c_size_t, c_void_p]),
+                                    c_void_p, c_int, c_void_p, c_int, c_void_p, c_int, c_void_p, c_int, c_int, c_int,
+                                    c_int, c_int, c_int, c_float, c_float, c_float, c_int, c_int, c_void_p, c_size_t,
+                                    c_void_p]),
     "pkv_cow_copy_rows": (c_int, [P(c_int32), c_int, P(c_int64), c_int, P(c_int32)]),
     "pkv_common_prefix_pages": (c_int, [P(c_int32), c_int, c_int, P(c_int32), P(c_int)]),
     "pkv_cascade_prefix_pages": (c_int, [P(c_int32), c_int, c_int, P(c_int32), c_int, P(c_int)]),

@@ -364,12 +364,14 @@ def decode_step(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor, k
 def decode_step_fp8(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor, k_new: torch.Tensor,
                     v_new: torch.Tensor, slot_mapping: torch.Tensor, copies: Optional[torch.Tensor],
                     block_tables: torch.Tensor, context_lens: torch.Tensor, max_context_len: int, scale: float,
-                    k_scale: float, v_scale: float, out: Optional[torch.Tensor] = None,
-                    workspace: Optional[torch.Tensor] = None, partition: int = 0, stream=None) -> torch.Tensor:
-    """decode_step over an FP8 cache (pkv_decode_step_fp8), no shared
-    prefix: the copies (int32 [n, 3] from ``cow_copy_rows``), the append of
-    one new token per sequence (k_new / v_new [B, Hkv, D] in q's dtype,
-    quantised with k_scale / v_scale) and the decode in one launch."""
+                    k_scale: float, v_scale: float, prefix_blocks: Optional[torch.Tensor] = None,
+                    out: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None, partition: int = 0,
+                    stream=None) -> torch.Tensor:
+    """decode_step over an FP8 cache (pkv_decode_step_fp8): the copies
+    (int32 [n, 3] from ``cow_copy_rows``) and the append of one new token
+    per sequence (k_new / v_new [B, Hkv, D] in q's dtype, quantised with
+    k_scale / v_scale) made by the decode's CTAs -- the FP8 cascade's when
+    ``prefix_blocks`` (int32, the shared leading blocks) is given."""
     nb, hkv, d = _cache_dims(k_cache, v_cache)
     if k_cache.dtype not in _FP8:
         raise ValueError("an FP8 cache (float8_e4m3fn or uint8) is required")
@@ -383,9 +385,11 @@ def decode_step_fp8(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tenso
     n_copies = 0 if copies is None else int(copies.shape[0])
     if n_copies and (copies.dim() != 2 or copies.shape[1] != 3):
         raise ValueError("copies must be [n, 3]")
+    pp = 0 if prefix_blocks is None else int(prefix_blocks.numel())
     if out is None:
         out = torch.empty_like(q)
-    need = decode_workspace_bytes(B, hq, d, max_context_len, partition)
+    need = (decode_prefix_fp8_workspace_bytes(B, hq, hkv, d, max_context_len, pp, partition) if pp else
+            decode_workspace_bytes(B, hq, d, max_context_len, partition))
     if need and (workspace is None or workspace.numel() * workspace.element_size() < need):
         workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
     check(lib.pkv_decode_step_fp8(
@@ -393,7 +397,8 @@ def decode_step_fp8(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tenso
         _dev(k_new, "k_new", q.dtype), _dev(v_new, "v_new", q.dtype), _dev(slot_mapping, "slot_mapping", torch.int64),
         _dev(copies, "copies", torch.int32) if n_copies else None, n_copies,
         _dev(block_tables, "block_tables", torch.int32), block_tables.shape[1],
-        _dev(context_lens, "context_lens", torch.int32), int(max_context_len), B, hq, hkv, d, nb, float(scale),
+        _dev(context_lens, "context_lens", torch.int32), int(max_context_len),
+        _dev(prefix_blocks, "prefix_blocks", torch.int32) if pp else None, pp, B, hq, hkv, d, nb, float(scale),
         float(k_scale), float(v_scale), int(partition), _DT[q.dtype], _dev(workspace, "workspace") if need else None,
         workspace.numel() * workspace.element_size() if need else 0, _stream(stream, q.device)),
         "pkv_decode_step_fp8")
@@ -952,10 +957,11 @@ class PagedKVCache:
 
         ``cow_pairs``: int32 [n, 2] (src, dst) whole-block copies, or [n, 3]
         (src, dst, rows) from ``cow_copy_rows``: the copies cut to the rows
-        that hold tokens.  With [n, 3] copies (or none), a 16-bit or FP8
-        pool and no shared prefix the whole step is one decode launch
-        (pkv_decode_step, pkv_decode_step_fp8): each sequence's copy and
-        append are made by the warp that then stages its last page.
+        that hold tokens.  With [n, 3] copies (or none) the step goes through
+        pkv_decode_step (16-bit pools) or pkv_decode_step_fp8: without a
+        shared prefix it is one decode launch, each sequence's copy and
+        append made by the warp that then stages its last page (so too in
+        the FP8 cascade's suffix pass).
         Inputs may be host tensors (pinned for asynchronous copies) or
         device tensors.  Host inputs are uploaded, and a host ``out`` is
         filled, on two side streams with double-buffered device copies, so a
@@ -980,16 +986,18 @@ class PagedKVCache:
             # launch, waiting for it only at each sequence's last page
             cut = cow_pairs.shape[0] == 0 or cow_pairs.shape[1] == 3
             fused = self.fp8 is None and self.dtype != torch.float32 and cut
-            no_prefix = prefix_blocks is None or prefix_blocks.numel() == 0
-            if self.fp8 is not None and cut and no_prefix:
-                ws = self.workspace(decode_workspace_bytes(B, hq, self.D, max_context_len, partition))
+            pp = 0 if prefix_blocks is None else int(prefix_blocks.numel())
+            if self.fp8 is not None and cut:
+                ws = self.workspace(decode_prefix_fp8_workspace_bytes(B, hq, self.Hkv, self.D, max_context_len, pp,
+                                                                      partition) if pp
+                                    else decode_workspace_bytes(B, hq, self.D, max_context_len, partition))
                 decode_step_fp8(x["q"], self.k, self.v, x["k"], x["v"], x["slots"],
                                 x["pairs"] if cow_pairs.shape[0] else None, x["tables"], x["lens"], max_context_len,
-                                sc, self.fp8[0], self.fp8[1], out=res, workspace=ws, partition=partition, stream=st)
+                                sc, self.fp8[0], self.fp8[1], prefix_blocks=x["prefix"] if pp else None, out=res,
+                                workspace=ws, partition=partition, stream=st)
                 stg.finish(st, res, out)
                 return res
             if fused:
-                pp = 0 if prefix_blocks is None else int(prefix_blocks.numel())
                 ws = self.workspace(decode_prefix_workspace_bytes(B, hq, self.D, max_context_len, pp, partition) if pp
                                     else decode_workspace_bytes(B, hq, self.D, max_context_len, partition))
                 decode_step(x["q"], self.k, self.v, x["k"], x["v"], x["slots"],

@@ -178,7 +178,21 @@ template <typename T, int D, int G, int NWARPS, int NSTAGE, bool kCascade = fals
 __global__ void __launch_bounds__(NWARPS * 32, PKV_FP8_MIN_CTAS)
     paged_decode_fp8_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tmap_k,
                             const __grid_constant__ CUtensorMap tmap_v, float v_scale, float k_scale) {
-  pdl_enter();
+  // The cascade's suffix pass reads nothing the launch before it (the
+  // prefix pass) writes: with defer_wait it lets its dependents launch and
+  // starts at once, running beside the prefix pass, and waits for that
+  // launch only before each CTA exits, so that it still ends after it (the
+  // merge after it reads both).  The launches before the prefix pass are
+  // complete by then: every prefix CTA waited for them before it let this
+  // launch start.
+  const bool defer = kCascade && a.defer_wait;
+  if (defer)
+    pdl_trigger();
+  else
+    pdl_enter();
+  auto exit_wait = [&]() {
+    if (defer && threadIdx.x == 0) pdl_wait();
+  };
   using S = Fp8Shape<D, NWARPS, NSTAGE>;
   using M = Mma<__half>;      // the MMAs run in fp16 (see above)
   constexpr int kNT = D / 8;  // PV n-tiles; also the d values a column spans
@@ -213,12 +227,16 @@ __global__ void __launch_bounds__(NWARPS * 32, PKV_FP8_MIN_CTAS)
   }
   const int span = ctx - tok_begin;
   const int nparts = (span + a.partition - 1) / a.partition;
-  if (part >= (nparts > 0 ? nparts : 1)) return;
+  if (part >= (nparts > 0 ? nparts : 1)) {
+    exit_wait();
+    return;
+  }
   if (span == 0) {
     if (!kCascade) {  // (the cascade's merge writes the zeros of an empty context)
       T* out = reinterpret_cast<T*>(a.out) + (static_cast<size_t>(b) * a.num_q_heads + kvh * G) * D;
       for (int i = threadIdx.x; i < G * D; i += NWARPS * 32) out[i] = Fmt<T>::from_f32(0.f);
     }
+    exit_wait();
     return;
   }
   auto col_row = [&](int n) -> size_t { return static_cast<size_t>(b) * a.num_q_heads + kvh * G + n; };
@@ -311,10 +329,11 @@ __global__ void __launch_bounds__(NWARPS * 32, PKV_FP8_MIN_CTAS)
   };
   // a fused step (pkv_decode_step_fp8): the warp that stages the sequence's
   // last page (page nblk - 1 of the last partition, its page last_i) makes
-  // the step's writes first and fences them before that page's TMA load
+  // the step's writes first and fences them before that page's TMA load.
+  // In a cascade that is the suffix's last page: the step never writes
+  // into the shared prefix blocks, which the prefix pass reads meanwhile.
   int last_i = -1;
-  if constexpr (!kCascade)
-    if (a.slots != nullptr && part == nparts - 1 && warp == (nblk - 1) % NWARPS) last_i = (nblk - 1) / NWARPS;
+  if (a.slots != nullptr && part == nparts - 1 && warp == (nblk - 1) % NWARPS) last_i = (nblk - 1) / NWARPS;
   uint32_t phase_bits = 0;
   auto issue = [&](int i) {
     const int phys = phys_of(i);
@@ -542,7 +561,10 @@ __global__ void __launch_bounds__(NWARPS * 32, PKV_FP8_MIN_CTAS)
       rec[S::kRecL + 2 * t4 + 1] = l1;
     }
   }
-  if (__syncthreads_or(timed_out)) return;
+  if (__syncthreads_or(timed_out)) {
+    exit_wait();
+    return;
+  }
 
   for (int idx = threadIdx.x; idx < G * D; idx += NWARPS * 32) {
     const int g = idx / D, d = idx % D;
@@ -568,6 +590,7 @@ __global__ void __launch_bounds__(NWARPS * 32, PKV_FP8_MIN_CTAS)
       if (d == 0) a.ws_ml[wrow] = make_float2(Mx, den);
     }
   }
+  exit_wait();
 }
 
 // The shared prefix of an FP8 cache as exact 16-bit code values, for the

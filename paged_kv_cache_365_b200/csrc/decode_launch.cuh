@@ -207,12 +207,12 @@ struct PrefixLayout {
 // Workspace of the cascade: suffix partials [B][Hq][P][D] + (max, sum)
 // [B][Hq][P], prefix partials [B][Hq][C][D] + [B][Hq][C], flags [B].
 PrefixLayout prefix_layout(long long B, long long Hq, long long D, long long max_ctx, long long prefix_pages,
-                           long long part) {
+                           long long part, long long chunk_pages = kPrefixChunkPages) {
   auto up16 = [](size_t x) { return (x + 15) / 16 * 16; };
   PrefixLayout L;
   L.parts = (max_ctx + part - 1) / part;
   if (L.parts < 1) L.parts = 1;
-  L.chunks = (prefix_pages + kPrefixChunkPages - 1) / kPrefixChunkPages;
+  L.chunks = (prefix_pages + chunk_pages - 1) / chunk_pages;
   L.off_so = 0;
   L.off_sml = up16(L.off_so + static_cast<size_t>(B * Hq * L.parts * D * 4));
   L.off_po = up16(L.off_sml + static_cast<size_t>(B * Hq * L.parts * 8));

@@ -265,10 +265,11 @@ pkv_status launch_decode_fp8(const pkv::DecodeArgs& a, float k_scale, float v_sc
 // Shared-prefix decode over an FP8 cache: (1) the prefix tiles as exact
 // 16-bit code values in the workspace, (2) the cascade's prefix pass over
 // them on the 16-bit tensor-core path (logits scaled by k_scale, partials by
-// v_scale), (3) the suffix pass over the FP8 cache, (4) the cascade's merge.
+// v_scale), (3) the suffix pass over the FP8 cache (beside the prefix pass;
+// it makes a fused step's copies and append), (4) the cascade's merge.
 template <typename T, int D, int G>
-pkv_status launch_decode_prefix_fp8(const pkv::DecodeArgs& a0, void* mini_k, void* mini_v, float v_scale,
-                                    cudaStream_t st) {
+pkv_status launch_decode_prefix_fp8(const pkv::DecodeArgs& a0, void* mini_k, void* mini_v, float k_scale,
+                                    float v_scale, cudaStream_t st) {
   const int row_chunks = D / 8;
   const long long total = static_cast<long long>(a0.prefix_pages) * a0.num_kv_heads * PKV_BLOCK_SIZE * row_chunks;
   long long nblk = (2 * total + 255) / 256;
@@ -281,6 +282,8 @@ pkv_status launch_decode_prefix_fp8(const pkv::DecodeArgs& a0, void* mini_k, voi
   {  // prefix pass
     using S = pkv::MmaShape<T, D, G, kMmaWarps, kMmaStages>;
     pkv::DecodeArgs ap = a0;
+    ap.slots = nullptr;  // (the suffix pass makes the step's writes)
+    ap.defer_wait = 0;
     ap.k_cache = static_cast<const unsigned char*>(mini_k);
     ap.v_cache = static_cast<const unsigned char*>(mini_v);
     ap.num_blocks = a0.prefix_pages;
@@ -310,27 +313,40 @@ pkv_status launch_decode_prefix_fp8(const pkv::DecodeArgs& a0, void* mini_k, voi
     if (cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(S::kSmem)) !=
         cudaSuccess)
       return PKV_ECUDA;
-    if (launch(kfn, dim3(a0.num_kv_heads, a0.num_seqs, a0.num_parts), dim3(kMmaWarps * 32), S::kSmem, st, a0, mk,
-               mv, v_scale, 1.f) != PKV_OK)
+    pkv::DecodeArgs as = a0;
+    as.defer_wait = 1;  // beside the prefix pass (see the kernel)
+    if (launch(kfn, dim3(a0.num_kv_heads, a0.num_seqs, a0.num_parts), dim3(kMmaWarps * 32), S::kSmem, st, as, mk,
+               mv, v_scale, k_scale) != PKV_OK)
       return PKV_ECUDA;
   }
   return launch_merge<T, D, PrefixMergeK>(a0, a0.num_chunks + a0.num_parts, st);
 }
 
 template <typename T, int D>
-pkv_status dispatch_group_prefix_fp8(const pkv::DecodeArgs& a, int G, void* mk, void* mv, float v_scale,
+pkv_status dispatch_group_prefix_fp8(const pkv::DecodeArgs& a, int G, void* mk, void* mv, float k_scale, float v_scale,
                                      cudaStream_t st) {
   switch (G) {
-    case 1: return launch_decode_prefix_fp8<T, D, 1>(a, mk, mv, v_scale, st);
-    case 2: return launch_decode_prefix_fp8<T, D, 2>(a, mk, mv, v_scale, st);
-    case 4: return launch_decode_prefix_fp8<T, D, 4>(a, mk, mv, v_scale, st);
-    case 8: return launch_decode_prefix_fp8<T, D, 8>(a, mk, mv, v_scale, st);
+    case 1: return launch_decode_prefix_fp8<T, D, 1>(a, mk, mv, k_scale, v_scale, st);
+    case 2: return launch_decode_prefix_fp8<T, D, 2>(a, mk, mv, k_scale, v_scale, st);
+    case 4: return launch_decode_prefix_fp8<T, D, 4>(a, mk, mv, k_scale, v_scale, st);
+    case 8: return launch_decode_prefix_fp8<T, D, 8>(a, mk, mv, k_scale, v_scale, st);
   }
   return PKV_EINVAL;
 }
 
-// The FP8 cascade's workspace: the 16-bit cascade's, then (1024-aligned) the
-// dequantised prefix tiles of K and of V, [prefix_pages][Hkv][16][D] each.
+// Prefix pages per prefix-role CTA of the FP8 cascade.  Its prefix pass is
+// a launch of its own that the suffix pass runs beside; shorter chunks make
+// more, shorter prefix CTAs, so the pass ends sooner and leaves the SMs to
+// the suffix streaming.
+#ifndef PKV_FP8_PREFIX_CHUNK
+#define PKV_FP8_PREFIX_CHUNK 16
+#endif
+constexpr int kPrefixChunkPagesFp8 = PKV_FP8_PREFIX_CHUNK;
+static_assert(kPrefixChunkPagesFp8 >= 1 && kPrefixChunkPagesFp8 <= 32, "one table entry per lane");
+
+// The FP8 cascade's workspace: the 16-bit cascade's (with the FP8 chunk
+// size), then (1024-aligned) the dequantised prefix tiles of K and of V,
+// [prefix_pages][Hkv][16][D] each.
 struct PrefixFp8Layout {
   PrefixLayout base;
   size_t off_k, off_v, total;
@@ -338,7 +354,7 @@ struct PrefixFp8Layout {
 PrefixFp8Layout prefix_fp8_layout(long long B, long long Hq, long long Hkv, long long D, long long max_ctx,
                                   long long prefix_pages, long long part) {
   PrefixFp8Layout L;
-  L.base = prefix_layout(B, Hq, D, max_ctx, prefix_pages, part);
+  L.base = prefix_layout(B, Hq, D, max_ctx, prefix_pages, part, kPrefixChunkPagesFp8);
   const size_t tiles = static_cast<size_t>(prefix_pages * Hkv * PKV_BLOCK_SIZE * D * 2);
   L.off_k = (L.base.total + 1023) / 1024 * 1024;
   L.off_v = L.off_k + (tiles + 1023) / 1024 * 1024;
@@ -1008,14 +1024,16 @@ size_t pkv_decode_prefix_fp8_workspace_bytes(int num_seqs, int num_q_heads, int 
   return prefix_fp8_layout(num_seqs, num_q_heads, num_kv_heads, head_dim, max_context_len, prefix_pages, part).total;
 }
 
-pkv_status pkv_paged_attention_decode_prefix_fp8(void* out, const void* q, const void* k_cache,
-                                                 const void* v_cache, const int32_t* block_tables,
-                                                 int max_blocks_per_seq, const int32_t* context_lens,
-                                                 int max_context_len, const int32_t* prefix_blocks,
-                                                 int prefix_pages, int num_seqs, int num_q_heads, int num_kv_heads,
-                                                 int head_dim, int num_blocks, float scale, float k_scale,
-                                                 float v_scale, int partition_tokens, pkv_dtype q_dtype,
-                                                 void* workspace, size_t workspace_bytes_given, void* stream) {
+}  // extern "C"
+
+namespace {
+pkv_status decode_prefix_fp8_impl(void* out, const void* q, const void* k_cache, const void* v_cache,
+                                  const int32_t* block_tables, int max_blocks_per_seq, const int32_t* context_lens,
+                                  int max_context_len, const int32_t* prefix_blocks, int prefix_pages, int num_seqs,
+                                  int num_q_heads, int num_kv_heads, int head_dim, int num_blocks, float scale,
+                                  float k_scale, float v_scale, int partition_tokens, pkv_dtype q_dtype,
+                                  void* workspace, size_t workspace_bytes_given, void* stream,
+                                  const StepWrites& w = StepWrites{}) {
   if (q_dtype != PKV_F16 && q_dtype != PKV_BF16) return PKV_EINVAL;
   if (!std::isfinite(k_scale) || !std::isfinite(v_scale) || !(k_scale > 0.f) || !(v_scale > 0.f))
     return PKV_EINVAL;
@@ -1042,22 +1060,40 @@ pkv_status pkv_paged_attention_decode_prefix_fp8(void* out, const void* q, const
   a.conform = reinterpret_cast<int*>(ws + L.base.off_conform);
   a.prefix_blocks = prefix_blocks;
   a.prefix_pages = prefix_pages;
-  a.chunk_pages = kPrefixChunkPages;
+  a.chunk_pages = kPrefixChunkPagesFp8;
   a.num_chunks = static_cast<int>(L.base.chunks);
   a.num_qgroups = (num_seqs * (num_q_heads / num_kv_heads) + kMmaWarps * 16 - 1) / (kMmaWarps * 16);
   if (static_cast<long long>(a.num_qgroups) * a.num_chunks > 65535 || a.num_parts > 65535) return PKV_EINVAL;
   a.qk_scale *= k_scale;
+  attach_step(&a, w);
   const int G = num_q_heads / num_kv_heads;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   void* mk = ws + L.off_k;
   void* mv = ws + L.off_v;
   auto run = [&](auto tag) -> pkv_status {
     using T = decltype(tag);
-    if (head_dim == 64) return dispatch_group_prefix_fp8<T, 64>(a, G, mk, mv, v_scale, st);
-    return dispatch_group_prefix_fp8<T, 128>(a, G, mk, mv, v_scale, st);
+    if (head_dim == 64) return dispatch_group_prefix_fp8<T, 64>(a, G, mk, mv, k_scale, v_scale, st);
+    return dispatch_group_prefix_fp8<T, 128>(a, G, mk, mv, k_scale, v_scale, st);
   };
   if (q_dtype == PKV_F16) return run(__half{});
   return run(__nv_bfloat16{});
+}
+}  // namespace
+
+extern "C" {
+
+pkv_status pkv_paged_attention_decode_prefix_fp8(void* out, const void* q, const void* k_cache,
+                                                 const void* v_cache, const int32_t* block_tables,
+                                                 int max_blocks_per_seq, const int32_t* context_lens,
+                                                 int max_context_len, const int32_t* prefix_blocks,
+                                                 int prefix_pages, int num_seqs, int num_q_heads, int num_kv_heads,
+                                                 int head_dim, int num_blocks, float scale, float k_scale,
+                                                 float v_scale, int partition_tokens, pkv_dtype q_dtype,
+                                                 void* workspace, size_t workspace_bytes_given, void* stream) {
+  return decode_prefix_fp8_impl(out, q, k_cache, v_cache, block_tables, max_blocks_per_seq, context_lens,
+                                max_context_len, prefix_blocks, prefix_pages, num_seqs, num_q_heads, num_kv_heads,
+                                head_dim, num_blocks, scale, k_scale, v_scale, partition_tokens, q_dtype, workspace,
+                                workspace_bytes_given, stream);
 }
 
 pkv_status pkv_kv_append_fp8(const void* k_new, const void* v_new, void* k_cache, void* v_cache,
@@ -1143,10 +1179,11 @@ pkv_status pkv_paged_attention_decode_fp8(void* out, const void* q, const void* 
 pkv_status pkv_decode_step_fp8(void* out, const void* q, void* k_cache, void* v_cache, const void* k_new,
                                const void* v_new, const int64_t* slot_mapping, const int32_t* copies, int num_copies,
                                const int32_t* block_tables, int max_blocks_per_seq, const int32_t* context_lens,
-                               int max_context_len, int num_seqs, int num_q_heads, int num_kv_heads, int head_dim,
-                               int num_blocks, float scale, float k_scale, float v_scale, int partition_tokens,
-                               pkv_dtype q_dtype, void* workspace, size_t workspace_bytes_given, void* stream) {
-  if (num_copies < 0 || num_copies > num_seqs) return PKV_EINVAL;
+                               int max_context_len, const int32_t* prefix_blocks, int prefix_pages, int num_seqs,
+                               int num_q_heads, int num_kv_heads, int head_dim, int num_blocks, float scale,
+                               float k_scale, float v_scale, int partition_tokens, pkv_dtype q_dtype, void* workspace,
+                               size_t workspace_bytes_given, void* stream) {
+  if (num_copies < 0 || num_copies > num_seqs || prefix_pages < 0) return PKV_EINVAL;
   if (num_seqs > 0 && (!k_new || !v_new || !slot_mapping || !aligned16(k_new) || !aligned16(v_new)))
     return PKV_EINVAL;
   if (num_copies > 0 && copies == nullptr) return PKV_EINVAL;
@@ -1156,6 +1193,11 @@ pkv_status pkv_decode_step_fp8(void* out, const void* q, void* k_cache, void* v_
   w.slots = slot_mapping;
   w.copies = copies;
   w.n_copies = num_copies;
+  if (prefix_pages > 0)  // the cascade: its suffix pass makes the writes
+    return decode_prefix_fp8_impl(out, q, k_cache, v_cache, block_tables, max_blocks_per_seq, context_lens,
+                                  max_context_len, prefix_blocks, prefix_pages, num_seqs, num_q_heads, num_kv_heads,
+                                  head_dim, num_blocks, scale, k_scale, v_scale, partition_tokens, q_dtype, workspace,
+                                  workspace_bytes_given, stream, w);
   return decode_fp8_impl(out, q, k_cache, v_cache, block_tables, max_blocks_per_seq, context_lens, max_context_len,
                          num_seqs, num_q_heads, num_kv_heads, head_dim, num_blocks, scale, k_scale, v_scale,
                          partition_tokens, q_dtype, workspace, workspace_bytes_given, stream, w);

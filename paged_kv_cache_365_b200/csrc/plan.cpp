@@ -85,7 +85,7 @@ pkv_status pkv_cascade_prefix_pages(const int32_t* block_tables, int num_seqs, i
   int p = 0;
   const pkv_status st = pkv_common_prefix_pages(block_tables, num_seqs, width, context_lens, &p);
   if (st != PKV_OK) return st;
-  const bool eligible = (dtype == PKV_F16 || dtype == PKV_BF16) && num_seqs >= PKV_CASCADE_MIN_SEQS &&
+  const bool eligible = (dtype == PKV_F16 || dtype == PKV_BF16 || dtype == PKV_E4M3) && num_seqs >= PKV_CASCADE_MIN_SEQS &&
                         p >= PKV_CASCADE_MIN_PAGES;
   *prefix_pages = eligible ? p : 0;
   return PKV_OK;

@@ -256,17 +256,23 @@ def test_decode_step_fp8_rejections(lib):
     """pkv_decode_step_fp8 checks the step's writes, the two scales and the
     FP8 decode's arguments before anything is launched."""
     f = ctypes.c_float
-    ok = [FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 2, FAKE, 8, FAKE, 100, 4, 8, 2, 128, 64, f(0.1), f(0.05),
-          f(0.05), 0, 1, None, 0, None]
-    for idx, bad in ((22, 0), (22, 3), (8, -1), (8, 5), (7, None), (4, None), (5, ODD), (6, None), (16, 96),
-                     (15, 3), (12, 8 * 16 + 1), (19, f(0.0)), (20, f(float("inf"))), (20, f(float("nan"))),
-                     (19, f(-1.0))):
+    ok = [FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 2, FAKE, 8, FAKE, 100, None, 0, 4, 8, 2, 128, 64, f(0.1),
+          f(0.05), f(0.05), 0, 1, None, 0, None]
+    for idx, bad in ((24, 0), (24, 3), (8, -1), (8, 5), (7, None), (4, None), (5, ODD), (6, None), (18, 96),
+                     (17, 3), (12, 8 * 16 + 1), (21, f(0.0)), (22, f(float("inf"))), (22, f(float("nan"))),
+                     (21, f(-1.0)), (14, -1)):
         a = list(ok)
         a[idx] = bad
         assert lib.pkv_decode_step_fp8(*a) == 1, (idx, bad)
-    # a context past one partition needs the workspace
+    # a context past one partition needs the workspace; so does the cascade,
+    # which also needs its prefix blocks
     a = list(ok)
     a[10], a[12] = 128, 2000
+    assert lib.pkv_decode_step_fp8(*a) == 1
+    a = list(ok)
+    a[14] = 4
+    assert lib.pkv_decode_step_fp8(*a) == 1
+    a[13] = FAKE
     assert lib.pkv_decode_step_fp8(*a) == 1
 
 

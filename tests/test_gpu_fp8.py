@@ -427,26 +427,29 @@ def test_multi_step_over_an_fp8_pool_through_the_cache_api():
     assert np.abs(out.float().numpy() - want).max() <= TOL["bf16"]
 
 
-STEP_CASES = [  # (name, dtype, Hq, Hkv, D, partition)
-    ("fp8_step_f16_G4", "f16", 8, 2, 128, 0),
-    ("fp8_step_bf16_G2_split", "bf16", 8, 4, 64, 64),
-    ("fp8_step_bf16_G8", "bf16", 8, 1, 128, 0),
-    ("fp8_step_f16_G1_split", "f16", 4, 4, 128, 32),
+STEP_CASES = [  # (name, dtype, Hq, Hkv, D, partition, cascade)
+    ("fp8_step_f16_G4", "f16", 8, 2, 128, 0, False),
+    ("fp8_step_bf16_G2_split", "bf16", 8, 4, 64, 64, False),
+    ("fp8_step_bf16_G8", "bf16", 8, 1, 128, 0, False),
+    ("fp8_step_f16_G1_split", "f16", 4, 4, 128, 32, False),
+    ("fp8_step_cascade_f16_G4", "f16", 8, 2, 128, 0, True),
+    ("fp8_step_cascade_bf16_G1_split", "bf16", 4, 4, 64, 64, True),
 ]
 
 
 @pytest.mark.parametrize("case", STEP_CASES, ids=lambda c: c[0])
 def test_fused_fp8_step_matches_separate_calls(case):
-    """pkv_decode_step_fp8 (the copy-on-write copies, the quantising append
-    and the FP8 decode in one launch) against copy_blocks, kv_append_fp8
-    and paged_attention_decode_fp8 on the same FP8 pool: every token row of
-    the pool and the output bit-identical; the output within tolerance of
-    the oracle, whose FP8 pool is its own replay of the workload with every
-    token row quantised by oracle.fp8.quantize."""
+    """pkv_decode_step_fp8 (the copy-on-write copies and the quantising
+    append made by the decode's CTAs; in the cascade by its suffix pass,
+    which runs beside the prefix pass) against copy_blocks, kv_append_fp8
+    and paged_attention_decode_fp8 / _prefix_fp8 on the same FP8 pool:
+    every token row of the pool and the output bit-identical; the output
+    within tolerance of the oracle, whose FP8 pool is its own replay of the
+    workload with every token row quantised by oracle.fp8.quantize."""
     import workloads
     from paged_kv_cache_365_b200.replay import build_step
     m = pkv()
-    name, dt, Hq, Hkv, D, partition = case
+    name, dt, Hq, Hkv, D, partition, cascade = case
     wl = workloads.prefix13b(seed=71, B=10, prefix_tokens=256, suffix_range=(1, 300), Hq=Hq, Hkv=Hkv, D=D,
                              dtype=dt, name=name)
     ks, vs = 0.011, 0.017
@@ -466,13 +469,23 @@ def test_fused_fp8_step_matches_separate_calls(case):
     vf = torch.full_like(kf, 0x7F)
     m.kv_append_fp8(rows_k, rows_v, kf, vf, slots_all, ks, vs)
     kf2, vf2 = kf.clone(), vf.clone()
+    prefix = None
+    if cascade:
+        pp = m.cascade_prefix_pages(tables, lens, torch.uint8)
+        assert pp > 0
+        prefix = torch.from_numpy(np.ascontiguousarray(tables[0, :pp])).cuda()
     m.copy_blocks(kf2, vf2, st["cow_pairs"])
     m.kv_append_fp8(st["k_new"], st["v_new"], kf2, vf2, st["slot_mapping"], ks, vs)
-    sep = m.paged_attention_decode_fp8(st["q"], kf2, vf2, st["block_tables"], st["context_lens"],
-                                       st["max_context_len"], wl.scale, ks, vs, partition=partition)
+    if cascade:
+        sep = m.paged_attention_decode_prefix_fp8(st["q"], kf2, vf2, st["block_tables"], st["context_lens"],
+                                                  st["max_context_len"], prefix, wl.scale, ks, vs,
+                                                  partition=partition)
+    else:
+        sep = m.paged_attention_decode_fp8(st["q"], kf2, vf2, st["block_tables"], st["context_lens"],
+                                           st["max_context_len"], wl.scale, ks, vs, partition=partition)
     fused = m.decode_step_fp8(st["q"], kf, vf, st["k_new"], st["v_new"], st["slot_mapping"], dcopies,
                               st["block_tables"], st["context_lens"], st["max_context_len"], wl.scale, ks, vs,
-                              partition=partition)
+                              prefix_blocks=prefix, partition=partition)
     torch.cuda.synchronize()
     assert m.get_error() == 0
     assert torch.equal(fused.view(torch.int16), sep.view(torch.int16))

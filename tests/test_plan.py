@@ -146,7 +146,8 @@ def test_cascade_prefix_pages_thresholds(pkv):
     base = np.arange(w, dtype=np.int32)
     for n, pages, dtype, want in [
             (4, 8, torch.float16, 8), (4, 7, torch.float16, 0), (3, 12, torch.bfloat16, 0),
-            (6, 12, torch.bfloat16, 12), (6, 12, torch.float32, 0), (6, 12, torch.uint8, 0)]:
+            (6, 12, torch.bfloat16, 12), (6, 12, torch.float32, 0), (6, 12, torch.uint8, 12),
+            (3, 12, torch.uint8, 0), (6, 7, torch.uint8, 0)]:
         tables = np.tile(base, (n, 1))
         tables[:, pages:] = 100 + np.arange(n)[:, None] * w + np.arange(w - pages)[None, :]
         lens = np.full(n, 16 * w, dtype=np.int32)
