@@ -16,11 +16,14 @@
 //    B operand, in registers) are loaded in that same order of d, so the
 //    dot product runs over the same pairs.
 //  * P.V as O^T[D x 8 queries] += V^T[D x 16 tokens] . P^T[16 x 8], V^T the
-//    A operand: lane (g, t) needs V[token][d] for tokens 2t, 2t+1, 2t+8,
-//    2t+9 and rows g, g + 8 of every m-tile; with d = (D/8) g + 2i (row g
-//    of m-tile i) and d + 1 (row g + 8), those are D/8 consecutive bytes of
-//    four token rows: four shared loads, byte permutes and exact E4M3 ->
-//    16-bit conversions.  P^T is the B operand, taken from the score
+//    A operand: a transposed byte load (ldmatrix .m16n16 .trans .b8) of two
+//    16-token x 16-byte blocks of the V tile gives lane (g, t) the codes of
+//    tokens 4t .. 4t + 3 at d = 16 i + g and 16 i + g + 8 of m-tiles i and
+//    i + 1, each pair of them one exact E4M3 -> 16-bit conversion away from
+//    an A register.  The MMA's k index then stands for the tokens in the
+//    order 0, 1, 4, 5, 8, 9, 12, 13, 2, 3, 6, 7, ..., so the K tile's rows
+//    are read in that order too (score_row_token) and the score rows, P^T's
+//    k index and V^T's name the same tokens.  P^T is the B operand, taken from the score
 //    fragment by movmatrix, in hi + lo 16-bit parts that accumulate into
 //    the same registers (two MMAs per m-tile); O^T needs D/16 x 4
 //    accumulator registers a lane, half of what O with the queries as M
@@ -59,6 +62,24 @@ __device__ __forceinline__ void e4m3x4_to_f16(uint32_t w, uint32_t& lo, uint32_t
   hi = e4m3x2_to<__half>(w >> 16);
 }
 
+
+// Two 16 x 16 byte matrices, transposed: lanes 0-15 give the row addresses
+// of the first, lanes 16-31 those of the second; lane (g, t) receives, of
+// each matrix, the bytes (rows 4t .. 4t + 3, column g) in r0 / r2 and
+// (rows 4t .. 4t + 3, column g + 8) in r1 / r3.
+__device__ __forceinline__ void ldsm_b8_x2_t(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m16n16.x2.trans.shared.b8 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr));
+}
+
+// The token a score row stands for: rows 2t, 2t + 1 (and 2t + 8, 2t + 9)
+// of S^T hold tokens 4t, 4t + 1 (and 4t + 2, 4t + 3), the order in which
+// the transposed byte loads deliver V's tokens (ldsm_b8_x2_t), so that the
+// k index of P^T and of V^T name the same token.
+__device__ __forceinline__ int score_row_token(int row) {
+  return ((row & 6) << 1) | (row & 1) | ((row >> 3) << 1);
+}
 
 // Byte offset of 16-byte chunk `chunk` of row `row` in an FP8 tile of 16
 // rows x D bytes stored with the TMA swizzle matching its row length
@@ -195,7 +216,6 @@ __global__ void __launch_bounds__(NWARPS * 32, PKV_FP8_MIN_CTAS)
   };
   using S = Fp8Shape<D, NWARPS, NSTAGE>;
   using M = Mma<__half>;      // the MMAs run in fp16 (see above)
-  constexpr int kNT = D / 8;  // PV n-tiles; also the d values a column spans
   // kPack (G <= 4): the spare query columns [G, 2G) repeat queries [0, G)
   // (identical scores, max and sum), carry P's lo part where columns
   // [0, G) carry its hi part, and the two columns' O^T are added at the
@@ -368,7 +388,7 @@ __global__ void __launch_bounds__(NWARPS * 32, PKV_FP8_MIN_CTAS)
     for (int i = 0; i < NSTAGE; ++i) issue(i);
   }
 
-  // O^T accumulators: m-tile i, rows g8 / g8 + 8 -> d = kNT g8 + 2i / + 1,
+  // O^T accumulators: m-tile i, rows g8 / g8 + 8 -> d = 16 i + g8 / + 8,
   // columns 2 t4, 2 t4 + 1 (queries)
   constexpr int kMT = D / 16;
   float o[kMT][4];
@@ -402,7 +422,7 @@ __global__ void __launch_bounds__(NWARPS * 32, PKV_FP8_MIN_CTAS)
 #pragma unroll
         for (int c = 0; c < S::kChunks; c += 2) {
           uint32_t r0, r1, r2, r3;
-          ldsm_x4(kt + swz8<D>(row, c + (lm >> 1)), r0, r1, r2, r3);
+          ldsm_x4(kt + swz8<D>(score_row_token(row), c + (lm >> 1)), r0, r1, r2, r3);
           uint32_t f0, f1, f2, f3, f4, f5, f6, f7;
           e4m3x4_to_f16(r0, f0, f2);
           e4m3x4_to_f16(r1, f1, f3);
@@ -413,7 +433,7 @@ __global__ void __launch_bounds__(NWARPS * 32, PKV_FP8_MIN_CTAS)
         }
       }
       // (2) scale (K scale folded in), mask the tail, online softmax
-      const bool v_lo = g8 < nvalid, v_hi = g8 + 8 < nvalid;
+      const bool v_lo = score_row_token(g8) < nvalid, v_hi = score_row_token(g8 + 8) < nvalid;
       const float x0 = v_lo ? (sc[0] + sd[0]) * xs0 : -INFINITY;
       const float x1 = v_lo ? (sc[1] + sd[1]) * xs1 : -INFINITY;
       const float x2 = v_hi ? (sc[2] + sd[2]) * xs0 : -INFINITY;
@@ -462,50 +482,29 @@ __global__ void __launch_bounds__(NWARPS * 32, PKV_FP8_MIN_CTAS)
       }
       const uint32_t pl0 = movm_t(top_lo), pl1 = movm_t(bot_lo);
       const uint32_t pb0 = kPack ? 0u : movm_t(top_hi), pb1 = kPack ? 0u : movm_t(bot_hi);
-      // (4) bytes d = kNT g8 .. kNT g8 + kNT - 1 (in 16-byte chunk vch, from
-      // byte vb0) of rows 2 t4, 2 t4 + 1, 2 t4 + 8, 2 t4 + 9; rows past the
-      // context are zeroed (an unused slot may hold a NaN code)
-      constexpr int kW = kNT / 4;  // 32-bit words per row segment (4 or 2)
-      const int vch = (kNT * g8) >> 4, vb0 = (kNT * g8) & 15;
-      uint32_t w0[kW], w1[kW], w8[kW], w9[kW];
-      {
-        const unsigned char* vbase = my_stages + s * S::kStage + S::kTile;
-        auto load = [&](int row, uint32_t (&w)[kW]) {
-          const unsigned char* p = vbase + swz8<D>(row, vch) + vb0;
-          if constexpr (kW == 4) {
-            const uint4 v = *reinterpret_cast<const uint4*>(p);
-            w[0] = v.x;
-            w[1] = v.y;
-            w[2] = v.z;
-            w[3] = v.w;
-          } else {
-            const uint2 v = *reinterpret_cast<const uint2*>(p);
-            w[0] = v.x;
-            w[1] = v.y;
-          }
-          if (nvalid < kBlockSize && row >= nvalid)
-#pragma unroll
-            for (int e = 0; e < kW; ++e) w[e] = 0u;
-        };
-        load(2 * t4, w0);
-        load(2 * t4 + 1, w1);
-        load(2 * t4 + 8, w8);
-        load(2 * t4 + 9, w9);
+      // (4) V^T fragments straight from the tile: the transposed byte load
+      // gives lane (g8, t4) the codes of tokens 4 t4 .. 4 t4 + 3 at d =
+      // 16 i + g8 and 16 i + g8 + 8 of m-tiles i and i + 1; each pair of
+      // codes converts exactly into one 16-bit A register.  Tokens past the
+      // context are zeroed (an unused slot may hold a NaN code).
+      uint32_t keep = 0xffffffffu;
+      if (nvalid < kBlockSize) {
+        const int n = nvalid - 4 * t4;
+        keep = n >= 4 ? 0xffffffffu : n <= 0 ? 0u : 0xffffffffu >> (32 - 8 * n);
       }
-      // m-tile i uses bytes 2i (its row g8) and 2i + 1 (row g8 + 8) of each
-      // row segment: one permute per pair of token rows
 #pragma unroll
-      for (int i = 0; i < kMT; ++i) {
-        const int w = i >> 1, bsel = 2 * (i & 1);
-        // (row a byte 2i, row b byte 2i, row a byte 2i+1, row b byte 2i+1)
-        const uint32_t sel = bsel | ((4 + bsel) << 4) | ((bsel + 1) << 8) | ((5 + bsel) << 12);
-        const uint32_t lo01 = __byte_perm(w0[w], w1[w], sel);
-        const uint32_t lo89 = __byte_perm(w8[w], w9[w], sel);
+      for (int i = 0; i < kMT; i += 2) {
+        uint32_t w0, w1, w2, w3;
+        ldsm_b8_x2_t(vt + swz8<D>(lane & 15, i + (lane >> 4)), w0, w1, w2, w3);
         uint32_t a0, a1, a2, a3;
-        e4m3x4_to_f16(lo01, a0, a1);  // tokens 2 t4, 2 t4 + 1 at rows g8, g8 + 8
-        e4m3x4_to_f16(lo89, a2, a3);  // tokens 2 t4 + 8, 2 t4 + 9
+        e4m3x4_to_f16(w0 & keep, a0, a2);  // tokens 4 t4, +1 | 4 t4 + 2, +3 at row g8
+        e4m3x4_to_f16(w1 & keep, a1, a3);  // the same at row g8 + 8
         if constexpr (!kPack) M::run(o[i], a0, a1, a2, a3, pb0, pb1);
         M::run(o[i], a0, a1, a2, a3, pl0, pl1);
+        e4m3x4_to_f16(w2 & keep, a0, a2);
+        e4m3x4_to_f16(w3 & keep, a1, a3);
+        if constexpr (!kPack) M::run(o[i + 1], a0, a1, a2, a3, pb0, pb1);
+        M::run(o[i + 1], a0, a1, a2, a3, pl0, pl1);
       }
     }
     __syncwarp();
@@ -541,14 +540,14 @@ __global__ void __launch_bounds__(NWARPS * 32, PKV_FP8_MIN_CTAS)
   float* rec = reinterpret_cast<float*>(my_stages);
 #pragma unroll
   for (int i = 0; i < kMT; ++i) {
-    const int d = kNT * g8 + 2 * i;
+    const int d = 16 * i + g8;
     if (2 * t4 < G) {
       rec[(2 * t4) * D + d] = o[i][0];
-      rec[(2 * t4) * D + d + 1] = o[i][2];
+      rec[(2 * t4) * D + d + 8] = o[i][2];
     }
     if (2 * t4 + 1 < G) {
       rec[(2 * t4 + 1) * D + d] = o[i][1];
-      rec[(2 * t4 + 1) * D + d + 1] = o[i][3];
+      rec[(2 * t4 + 1) * D + d + 8] = o[i][3];
     }
   }
   if (g8 == 0) {
