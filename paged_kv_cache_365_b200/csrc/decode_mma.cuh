@@ -417,6 +417,7 @@ __global__ void __launch_bounds__(NWARPS * 32)
     pdl_enter();
   using S = MmaShape<T, D, G, NWARPS, NSTAGE>;
   using M = Mma<T>;
+  constexpr float kLazyMax = 8.f;  // the reference max moves only past 2^kLazyMax (see the softmax)
   const int kvh = blockIdx.x;
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -652,19 +653,22 @@ __global__ void __launch_bounds__(NWARPS * 32)
         const float x2 = v_hi ? sc[2] * a.qk_scale : -INFINITY;  // token g8+8, column 2 t4
         const float x3 = v_hi ? sc[3] * a.qk_scale : -INFINITY;  // token g8+8, column 2 t4 + 1
         float mx0 = fmaxf(x0, x2), mx1 = fmaxf(x1, x3);
+        // The reference max of a column moves only when one of the page's
+        // scores passes it by more than 2^8 (so p <= 2^8): most pages then
+        // need one vote, no reduction and no rescale.  Any reference is
+        // exact once the same one scales l and O.
+        if (__any_sync(kFull, mx0 > m0 + kLazyMax || mx1 > m1 + kLazyMax)) {
 #pragma unroll
-        for (int msk = 4; msk <= 16; msk <<= 1) {
-          mx0 = fmaxf(mx0, __shfl_xor_sync(kFull, mx0, msk));
-          mx1 = fmaxf(mx1, __shfl_xor_sync(kFull, mx1, msk));
-        }
-        const float n0 = fmaxf(m0, mx0), n1 = fmaxf(m1, mx1);
-        const float al0 = exp2_sfu(m0 - n0), al1 = exp2_sfu(m1 - n1);
-        m0 = n0;
-        m1 = n1;
-        const float p0 = exp2_sfu(x0 - n0), p1 = exp2_sfu(x1 - n1), p2 = exp2_sfu(x2 - n0), p3 = exp2_sfu(x3 - n1);
-        l0 = fmaf(l0, al0, p0 + p2);
-        l1 = fmaf(l1, al1, p1 + p3);
-        if (__any_sync(kFull, al0 != 1.f || al1 != 1.f)) {  // a running max moved
+          for (int msk = 4; msk <= 16; msk <<= 1) {
+            mx0 = fmaxf(mx0, __shfl_xor_sync(kFull, mx0, msk));
+            mx1 = fmaxf(mx1, __shfl_xor_sync(kFull, mx1, msk));
+          }
+          const float n0 = fmaxf(m0, mx0), n1 = fmaxf(m1, mx1);
+          const float al0 = exp2_sfu(m0 - n0), al1 = exp2_sfu(m1 - n1);
+          m0 = n0;
+          m1 = n1;
+          l0 *= al0;
+          l1 *= al1;
 #pragma unroll
           for (int mt = 0; mt < S::kKSteps; ++mt) {
             o[mt][0] *= al0;
@@ -673,6 +677,9 @@ __global__ void __launch_bounds__(NWARPS * 32)
             o[mt][3] *= al1;
           }
         }
+        const float p0 = exp2_sfu(x0 - m0), p1 = exp2_sfu(x1 - m1), p2 = exp2_sfu(x2 - m0), p3 = exp2_sfu(x3 - m1);
+        l0 += p0 + p2;
+        l1 += p1 + p3;
         // (3) P^T as B fragments, split into hi + lo 16-bit parts
         const uint32_t top_hi = M::pack(p0, p1), bot_hi = M::pack(p2, p3);
         const float2 th = M::unpack(top_hi), bh = M::unpack(bot_hi);
