@@ -251,26 +251,20 @@ __device__ __forceinline__ bool prefix_warp(const DecodeArgs& a, const CUtensorM
         for (int e = 0; e < 4; ++e) x[nt][e] = sc[nt][e] * a.qk_scale;
       float mxA = fmaxf(fmaxf(x[0][0], x[0][1]), fmaxf(x[1][0], x[1][1]));
       float mxB = fmaxf(fmaxf(x[0][2], x[0][3]), fmaxf(x[1][2], x[1][3]));
+      // the reference max moves only when a score passes it by more than
+      // 2^8 (one vote a page otherwise; see the sequence role)
+      if (__any_sync(kFull, mxA > mA + 8.f || mxB > mB + 8.f)) {
 #pragma unroll
-      for (int msk = 1; msk <= 2; msk <<= 1) {
-        mxA = fmaxf(mxA, __shfl_xor_sync(kFull, mxA, msk));
-        mxB = fmaxf(mxB, __shfl_xor_sync(kFull, mxB, msk));
-      }
-      const float nA = fmaxf(mA, mxA), nB = fmaxf(mB, mxB);
-      const float alA = exp2_sfu(mA - nA), alB = exp2_sfu(mB - nB);
-      mA = nA;
-      mB = nB;
-      float p[2][4];
-#pragma unroll
-      for (int nt = 0; nt < 2; ++nt) {
-        p[nt][0] = exp2_sfu(x[nt][0] - nA);
-        p[nt][1] = exp2_sfu(x[nt][1] - nA);
-        p[nt][2] = exp2_sfu(x[nt][2] - nB);
-        p[nt][3] = exp2_sfu(x[nt][3] - nB);
-      }
-      lA = fmaf(lA, alA, p[0][0] + p[0][1] + p[1][0] + p[1][1]);
-      lB = fmaf(lB, alB, p[0][2] + p[0][3] + p[1][2] + p[1][3]);
-      if (__any_sync(kFull, alA != 1.f || alB != 1.f)) {
+        for (int msk = 1; msk <= 2; msk <<= 1) {
+          mxA = fmaxf(mxA, __shfl_xor_sync(kFull, mxA, msk));
+          mxB = fmaxf(mxB, __shfl_xor_sync(kFull, mxB, msk));
+        }
+        const float nA = fmaxf(mA, mxA), nB = fmaxf(mB, mxB);
+        const float alA = exp2_sfu(mA - nA), alB = exp2_sfu(mB - nB);
+        mA = nA;
+        mB = nB;
+        lA *= alA;
+        lB *= alB;
 #pragma unroll
         for (int j = 0; j < kNTiles; ++j) {
           o[j][0] *= alA;
@@ -279,6 +273,16 @@ __device__ __forceinline__ bool prefix_warp(const DecodeArgs& a, const CUtensorM
           o[j][3] *= alB;
         }
       }
+      float p[2][4];
+#pragma unroll
+      for (int nt = 0; nt < 2; ++nt) {
+        p[nt][0] = exp2_sfu(x[nt][0] - mA);
+        p[nt][1] = exp2_sfu(x[nt][1] - mA);
+        p[nt][2] = exp2_sfu(x[nt][2] - mB);
+        p[nt][3] = exp2_sfu(x[nt][3] - mB);
+      }
+      lA += p[0][0] + p[0][1] + p[1][0] + p[1][1];
+      lB += p[0][2] + p[0][3] + p[1][2] + p[1][3];
       uint32_t ph[4], pl[4];
       {
         const float v[4][2] = {{p[0][0], p[0][1]}, {p[0][2], p[0][3]}, {p[1][0], p[1][1]}, {p[1][2], p[1][3]}};

@@ -82,6 +82,7 @@ __global__ void __launch_bounds__(NWARPS * 32)
   pdl_enter();
   using S = MmaShape<T, D, G, NWARPS, NSTAGE>;
   using M = Mma<T>;
+  constexpr float kLazyMax = 8.f;  // the reference max moves only past 2^kLazyMax
   constexpr int kCols = 8 * NT;                 // query rows of a tile (the MMA's N)
   constexpr int kRecM = kCols * D, kRecL = kCols * D + kCols;  // warp record: o[kCols][D], m, l
   static_assert(size_t(kRecL + kCols) * sizeof(float) <= size_t(S::kWarpStageBytes),
@@ -254,22 +255,30 @@ __global__ void __launch_bounds__(NWARPS * 32)
         const float x2 = jB <= pos[nt][0] ? sc[nt][2] * a.qk_scale : -INFINITY;
         const float x3 = jB <= pos[nt][1] ? sc[nt][3] * a.qk_scale : -INFINITY;
         float mx0 = fmaxf(x0, x2), mx1 = fmaxf(x1, x3);
+        // the reference max moves only when a score passes it by more than
+        // 2^kLazyMax (one vote a page otherwise; see the decode kernel)
+        al[nt][0] = al[nt][1] = 1.f;
+        if (__any_sync(kFull, mx0 > mr[nt][0] + kLazyMax || mx1 > mr[nt][1] + kLazyMax)) {
 #pragma unroll
-        for (int msk = 4; msk <= 16; msk <<= 1) {
-          mx0 = fmaxf(mx0, __shfl_xor_sync(kFull, mx0, msk));
-          mx1 = fmaxf(mx1, __shfl_xor_sync(kFull, mx1, msk));
+          for (int msk = 4; msk <= 16; msk <<= 1) {
+            mx0 = fmaxf(mx0, __shfl_xor_sync(kFull, mx0, msk));
+            mx1 = fmaxf(mx1, __shfl_xor_sync(kFull, mx1, msk));
+          }
+          const float n0 = fmaxf(mr[nt][0], mx0), n1 = fmaxf(mr[nt][1], mx1);
+          // a column that has seen no key yet keeps max -inf: subtract 0 instead
+          const float u0 = n0 == -INFINITY ? 0.f : n0, u1 = n1 == -INFINITY ? 0.f : n1;
+          al[nt][0] = exp2_sfu(mr[nt][0] - u0);
+          al[nt][1] = exp2_sfu(mr[nt][1] - u1);
+          mr[nt][0] = n0;
+          mr[nt][1] = n1;
+          lr_[nt][0] *= al[nt][0];
+          lr_[nt][1] *= al[nt][1];
+          moved = true;
         }
-        const float n0 = fmaxf(mr[nt][0], mx0), n1 = fmaxf(mr[nt][1], mx1);
-        // a column that has seen no key yet keeps max -inf: subtract 0 instead
-        const float u0 = n0 == -INFINITY ? 0.f : n0, u1 = n1 == -INFINITY ? 0.f : n1;
-        al[nt][0] = exp2_sfu(mr[nt][0] - u0);
-        al[nt][1] = exp2_sfu(mr[nt][1] - u1);
-        mr[nt][0] = n0;
-        mr[nt][1] = n1;
+        const float u0 = mr[nt][0] == -INFINITY ? 0.f : mr[nt][0], u1 = mr[nt][1] == -INFINITY ? 0.f : mr[nt][1];
         const float p0 = exp2_sfu(x0 - u0), p1 = exp2_sfu(x1 - u1), p2 = exp2_sfu(x2 - u0), p3 = exp2_sfu(x3 - u1);
-        lr_[nt][0] = fmaf(lr_[nt][0], al[nt][0], p0 + p2);
-        lr_[nt][1] = fmaf(lr_[nt][1], al[nt][1], p1 + p3);
-        moved |= al[nt][0] != 1.f || al[nt][1] != 1.f;
+        lr_[nt][0] += p0 + p2;
+        lr_[nt][1] += p1 + p3;
         const uint32_t top_hi = M::pack(p0, p1), bot_hi = M::pack(p2, p3);
         const float2 th = M::unpack(top_hi), bh = M::unpack(bot_hi);
         pb[nt][0] = movm_t(top_hi);
@@ -559,6 +568,7 @@ __global__ void __launch_bounds__(NW * 32, PKV_ROWS_WARPS_PER_SM / NW)
   pdl_enter();
   using S = RowsShape<D, NW, NSTAGE, KP>;
   using M = Mma<T>;
+  constexpr float kLazyMax = 8.f;  // the reference max moves only past 2^kLazyMax
   constexpr int kCols = 8 * NW;
   const int kvh = blockIdx.x;
   const int b = blockIdx.y / a.tiles;
@@ -669,16 +679,23 @@ __global__ void __launch_bounds__(NW * 32, PKV_ROWS_WARPS_PER_SM / NW)
       mx0 = fmaxf(mx0, fmaxf(x[p][0], x[p][2]));
       mx1 = fmaxf(mx1, fmaxf(x[p][1], x[p][3]));
     }
+    // the reference max moves only when a score passes it by more than
+    // 2^kLazyMax (one vote a step otherwise; see the decode kernel)
+    float al0 = 1.f, al1 = 1.f;
+    if (__any_sync(kFull, mx0 > m0 + kLazyMax || mx1 > m1 + kLazyMax)) {
 #pragma unroll
-    for (int msk = 4; msk <= 16; msk <<= 1) {
-      mx0 = fmaxf(mx0, __shfl_xor_sync(kFull, mx0, msk));
-      mx1 = fmaxf(mx1, __shfl_xor_sync(kFull, mx1, msk));
+      for (int msk = 4; msk <= 16; msk <<= 1) {
+        mx0 = fmaxf(mx0, __shfl_xor_sync(kFull, mx0, msk));
+        mx1 = fmaxf(mx1, __shfl_xor_sync(kFull, mx1, msk));
+      }
+      const float n0 = fmaxf(m0, mx0), n1 = fmaxf(m1, mx1);
+      const float v0 = n0 == -INFINITY ? 0.f : n0, v1 = n1 == -INFINITY ? 0.f : n1;
+      al0 = exp2_sfu(m0 - v0);
+      al1 = exp2_sfu(m1 - v1);
+      m0 = n0;
+      m1 = n1;
     }
-    const float n0 = fmaxf(m0, mx0), n1 = fmaxf(m1, mx1);
-    const float u0 = n0 == -INFINITY ? 0.f : n0, u1 = n1 == -INFINITY ? 0.f : n1;
-    const float al0 = exp2_sfu(m0 - u0), al1 = exp2_sfu(m1 - u1);
-    m0 = n0;
-    m1 = n1;
+    const float u0 = m0 == -INFINITY ? 0.f : m0, u1 = m1 == -INFINITY ? 0.f : m1;
     uint32_t pb0[KP], pb1[KP], pl0[KP], pl1[KP];
     float sum0 = 0.f, sum1 = 0.f;
 #pragma unroll
