@@ -123,6 +123,7 @@ __device__ __forceinline__ uint32_t swz(int row, int chunk) {
   return static_cast<uint32_t>((chunk >> 3) * 2048 + row * 128 + (((chunk & 7) ^ (row & 7)) << 4));
 }
 
+
 template <typename T, int D, int G, int NWARPS, int NSTAGE>
 struct MmaShape {
   static constexpr int kTile = kBlockSize * D * 2;   // bytes of a (block, kv-head) tile
@@ -422,6 +423,11 @@ __global__ void __launch_bounds__(NWARPS * 32)
   using S = MmaShape<T, D, G, NWARPS, NSTAGE>;
   using M = Mma<T>;
   constexpr float kLazyMax = 8.f;  // the reference max moves only past 2^kLazyMax (see the softmax)
+  // kPack (G <= 4): the spare query columns [G, 2G) repeat queries [0, G)
+  // (identical scores, max and sum) and carry P's lo part where columns
+  // [0, G) carry its hi part; the two columns of O^T are added at the end,
+  // so P.V takes one MMA per m-tile instead of two
+  constexpr bool kPack = G <= 4;
   const int kvh = blockIdx.x;
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -519,10 +525,11 @@ __global__ void __launch_bounds__(NWARPS * 32)
   }
 
   // B fragments of Q^T (k = d, n = query column g8), zero past the columns
+  // (with kPack the columns [G, 2G) repeat queries [0, G))
   uint32_t qb[S::kKSteps][2];
   {
-    const bool ok = col_valid(g8);
-    const T* qp = reinterpret_cast<const T*>(a.q) + (ok ? col_row(g8) : 0) * D;
+    const bool ok = kPack ? g8 < 2 * ncol : col_valid(g8);
+    const T* qp = reinterpret_cast<const T*>(a.q) + (ok ? col_row(g8 & (G - 1)) : 0) * D;
 #pragma unroll
     for (int ks = 0; ks < S::kKSteps; ++ks) {
       qb[ks][0] = ok ? *reinterpret_cast<const uint32_t*>(qp + ks * 16 + 2 * t4) : 0u;
@@ -684,12 +691,21 @@ __global__ void __launch_bounds__(NWARPS * 32)
         const float p0 = exp2_sfu(x0 - m0), p1 = exp2_sfu(x1 - m1), p2 = exp2_sfu(x2 - m0), p3 = exp2_sfu(x3 - m1);
         l0 += p0 + p2;
         l1 += p1 + p3;
-        // (3) P^T as B fragments, split into hi + lo 16-bit parts
+        // (3) P^T as B fragments, split into hi + lo 16-bit parts (kPack:
+        // one fragment, hi in columns [0, G), lo in [G, 2G))
         const uint32_t top_hi = M::pack(p0, p1), bot_hi = M::pack(p2, p3);
         const float2 th = M::unpack(top_hi), bh = M::unpack(bot_hi);
-        const uint32_t top_lo = M::pack(p0 - th.x, p1 - th.y), bot_lo = M::pack(p2 - bh.x, p3 - bh.y);
-        const uint32_t pb0 = movm_t(top_hi), pb1 = movm_t(bot_hi);
+        uint32_t top_lo, bot_lo;
+        if constexpr (kPack) {
+          const bool h0 = 2 * t4 < G, h1 = 2 * t4 + 1 < G;
+          top_lo = M::pack(h0 ? th.x : p0 - th.x, h1 ? th.y : p1 - th.y);
+          bot_lo = M::pack(h0 ? bh.x : p2 - bh.x, h1 ? bh.y : p3 - bh.y);
+        } else {
+          top_lo = M::pack(p0 - th.x, p1 - th.y);
+          bot_lo = M::pack(p2 - bh.x, p3 - bh.y);
+        }
         const uint32_t pl0 = movm_t(top_lo), pl1 = movm_t(bot_lo);
+        const uint32_t pb0 = kPack ? 0u : movm_t(top_hi), pb1 = kPack ? 0u : movm_t(bot_hi);
         // V^T fragment halves of tokens past the context are zeroed
         uint32_t keep_lo = 0xffffffffu, keep_hi = 0xffffffffu;
         if (nvalid < kBlockSize) {
@@ -709,7 +725,7 @@ __global__ void __launch_bounds__(NWARPS * 32)
               a2 &= keep_hi;
               a3 &= keep_hi;
             }
-            M::run(o[mt], a0, a1, a2, a3, pb0, pb1);
+            if constexpr (!kPack) M::run(o[mt], a0, a1, a2, a3, pb0, pb1);
             M::run(o[mt], a0, a1, a2, a3, pl0, pl1);
           }
         };
@@ -739,6 +755,18 @@ __global__ void __launch_bounds__(NWARPS * 32)
       l1 += __shfl_xor_sync(kFull, l1, msk);
     }
 
+    if constexpr (kPack) {  // query n: column n (hi) + column n + G (lo)
+#pragma unroll
+      for (int mt = 0; mt < S::kKSteps; ++mt) {
+        if constexpr (G == 1) {
+          o[mt][0] += o[mt][1];
+          o[mt][2] += o[mt][3];
+        } else {
+#pragma unroll
+          for (int e = 0; e < 4; ++e) o[mt][e] += __shfl_xor_sync(kFull, o[mt][e], G / 2);
+        }
+      }
+    }
     // warp record [o: 8 x D][m: 8][l: 8] in the warp's own (drained) stages
     float* rec = reinterpret_cast<float*>(my_stages);
     const int ha = 2 * t4, hb = 2 * t4 + 1;
