@@ -777,6 +777,11 @@ class _Staging:
         self.bufs = [{}, {}]
         self.computed = [None, None]    # compute that last read set s is done
         self.downloaded = [None, None]  # download that last read set s's output is done
+        # one event of each kind per buffer set, recorded again each time the
+        # set comes round (every wait on the previous record is queued by then)
+        self.ev_ready = [torch.cuda.Event(), torch.cuda.Event()]
+        self.ev_done = [torch.cuda.Event(), torch.cuda.Event()]
+        self.ev_dl = [torch.cuda.Event(), torch.cuda.Event()]
 
     def _buf(self, key, shape, dtype, st):
         b = self.bufs[self.slot].get(key)
@@ -806,7 +811,7 @@ class _Staging:
             with torch.cuda.stream(self.h2d):
                 for k, t in host.items():
                     out[k].copy_(t, non_blocking=True)
-                ready = torch.cuda.Event()
+                ready = self.ev_ready[s]
                 ready.record(self.h2d)
             st.wait_event(ready)
         return out
@@ -822,14 +827,14 @@ class _Staging:
         """After the step's kernels on ``st``: download into a host ``out`` on
         the download stream; flip to the other buffer set."""
         s = self.slot
-        done = torch.cuda.Event()
+        done = self.ev_done[s]
         done.record(st)
         self.computed[s] = done
         if out is not None and out.device != self.device:
             self.d2h.wait_event(done)
             with torch.cuda.stream(self.d2h):
                 out.copy_(res, non_blocking=True)
-                ev = torch.cuda.Event()
+                ev = self.ev_dl[s]
                 ev.record(self.d2h)
             self.downloaded[s] = ev
         self.slot ^= 1
