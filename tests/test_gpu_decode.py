@@ -318,3 +318,47 @@ def test_workspace_contents_and_graph_replays_do_not_matter():
     want = oracle.paged_decode(vals["q"], ref["cache"].k, ref["cache"].v, ref["block_tables"], ref["context_lens"],
                                wl.scale, wl.dtype)
     assert np.abs(clean.float().cpu().numpy() - want).max() <= TOL["f16"]
+
+
+def _ramp_values(wl, step):
+    """Values whose scores climb along every sequence: q[..., 0] = 4 and
+    k[token t, :, 0] = step * t / 16, the other entries N(0, 1), so that a
+    later page's scores pass the first pages' maximum by many units and the
+    kernels' reference max has to move (and O and l be rescaled) mid-sequence,
+    in every partition."""
+    vals = workloads.draw_values(wl)
+    f = {k: oracle.widen(v, wl.dtype).astype(np.float32) for k, v in vals.items()}
+    f["q"][:, :, 0] = 4.0
+    r = 0
+    for b, c in enumerate(wl.context_lens):
+        n = max(int(c) - 1, 0)
+        f["k_tokens"][r:r + n, :, 0] = (step * np.arange(n) / 16.0)[:, None]
+        f["k_new"][b, :, 0] = step * max(int(c) - 1, 0) / 16.0
+        r += n
+    return {k: workloads._to_storage(v, wl.dtype) for k, v in f.items()}
+
+
+@pytest.mark.parametrize("dtype", ["f16", "bf16"])
+@pytest.mark.parametrize("G", [1, 4, 8])
+@pytest.mark.parametrize("partition", [0, 256])
+def test_reference_max_moves_mid_sequence(dtype, G, partition):
+    """Scores that climb page after page (and one sequence whose scores fall
+    instead): the decode's reference max moves only when a page passes it by
+    more than 2^8, rescaling what was accumulated; the result must still be
+    the oracle's softmax within the stated tolerance."""
+    wl = workloads.custom([700, 1500, 37, 2100], Hq=2 * G, Hkv=2, D=128, dtype=dtype, seed=31 + G,
+                          name=f"ramp_{dtype}_{G}")
+    vals = _ramp_values(wl, 3.0)
+    # sequence 2 falls instead of climbing
+    f = oracle.widen(vals["k_tokens"], dtype).astype(np.float32)
+    r0 = sum(max(int(c) - 1, 0) for c in wl.context_lens[:2])
+    n2 = int(wl.context_lens[2]) - 1
+    f[r0:r0 + n2, :, 0] = f[r0:r0 + n2, :, 0][::-1]
+    vals["k_tokens"] = workloads._to_storage(f, dtype)
+    ref = oracle.replay(wl, vals)
+    out, _ = run_gpu_step(wl, vals, partition=partition)
+    want = oracle.paged_decode(vals["q"], ref["cache"].k, ref["cache"].v, ref["block_tables"],
+                               ref["context_lens"], wl.scale, wl.dtype)
+    got = to_f64(out)
+    assert np.isfinite(got).all()
+    assert np.abs(got - want).max() <= TOL[dtype]

@@ -37,9 +37,11 @@ def to_dev(a, dt):
     return t.cuda()
 
 
-def build(ctx, Hkv, D, dt, ks, vs, seed, sigma=1.0):
+def build(ctx, Hkv, D, dt, ks, vs, seed, sigma=1.0, ramp=0.0):
     """An FP8 pool written through the GPU append and the oracle append from
-    the same 16-bit values (N(0, sigma^2)); returns both plus tables."""
+    the same 16-bit values (N(0, sigma^2); with ``ramp``, K's first entry of
+    token j of every sequence is ramp * j / 16 instead); returns both plus
+    tables."""
     m = pkv()
     rng = np.random.default_rng(seed)
     pages = [-(-c // 16) for c in ctx]
@@ -55,7 +57,10 @@ def build(ctx, Hkv, D, dt, ks, vs, seed, sigma=1.0):
         slots += [int(tables[b, j // 16]) * 16 + j % 16 for j in range(c)]
     slots = np.array(slots, dtype=np.int64)
     n = len(slots)
-    kx = storage(rng.standard_normal((n, Hkv, D)).astype(np.float32) * sigma, dt)
+    k32 = rng.standard_normal((n, Hkv, D)).astype(np.float32) * sigma
+    if ramp:
+        k32[:, :, 0] = (ramp * np.concatenate([np.arange(c) for c in ctx]) / 16.0)[:, None]
+    kx = storage(k32, dt)
     vx = storage(rng.standard_normal((n, Hkv, D)).astype(np.float32) * sigma, dt)
     ref = oracle.RefCache(nb, Hkv, D, "e4m3")
     ref.append_fp8(kx, vx, slots, dt, ks, vs)
@@ -507,3 +512,31 @@ def test_fused_fp8_step_matches_separate_calls(case):
     want = oracle.paged_decode(vals["q"], rk.k, rk.v, ref["block_tables"], ref["context_lens"], wl.scale, wl.dtype,
                                kv_dtype="e4m3", k_scale=ks, v_scale=vs)
     assert np.abs(fused.float().cpu().numpy() - want).max() <= TOL[dt]
+
+
+@pytest.mark.parametrize("G", [1, 4, 8])
+@pytest.mark.parametrize("partition", [0, 256])
+def test_fp8_reference_max_moves_mid_sequence(G, partition):
+    """Scores that climb page after page over an FP8 pool (K's first entry
+    grows along each sequence, the queries' first entry is 4): the FP8
+    decode's reference max moves only past 2^8, rescaling what it has
+    accumulated, and the result must stay the oracle's within tolerance."""
+    m = pkv()
+    dt, Hkv, D = "f16", 2, 128
+    ctx = [700, 1500, 37, 2100]
+    ks, vs = 1.0, 0.017
+    ref, kc, vc, tables, lens = build(ctx, Hkv, D, dt, ks, vs, seed=41 + G, ramp=3.0)
+    rng = np.random.default_rng(7 + G)
+    q32 = rng.standard_normal((len(ctx), Hkv * G, D)).astype(np.float32)
+    q32[:, :, 0] = 4.0
+    q = storage(q32, dt)
+    scale = D ** -0.5
+    want = oracle.paged_decode(q, ref.k, ref.v, tables, lens, scale, dt, kv_dtype="e4m3", k_scale=ks, v_scale=vs)
+    out = m.paged_attention_decode_fp8(to_dev(q, dt), kc, vc, torch.from_numpy(tables).cuda(),
+                                       torch.from_numpy(lens).cuda(), int(lens.max()), scale, ks, vs,
+                                       partition=partition)
+    torch.cuda.synchronize()
+    assert m.get_error() == 0
+    got = out.float().cpu().numpy()
+    assert np.isfinite(got).all()
+    assert np.abs(got - want).max() <= TOL[dt]
